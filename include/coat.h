@@ -1,0 +1,194 @@
+/*
+ * coat.h -- C ABI of the B200 (sm_100a) COAT FP8-optimizer-state library.
+ *
+ * COAT ("Compressing Optimizer states and Activation for memory-efficient
+ * FP8 Training") keeps the AdamW first and second moments in FP8, one scale
+ * and one dynamic-range-expansion exponent k per group of elements.  Sources:
+ *   [P1] web page "FP8训练新范式：减少40%显存占用，训练速度提高1.4倍",
+ *        sections "FP8优化器状态" (per-group FP8 moments; E4M3 spans
+ *        0.00195..448, about 200000; typical group max/min ~1000 for m and
+ *        ~10 for v) and "解决方案：动态范围扩展" (expansion f(.) with one k
+ *        per group, recomputed every step; E4M3+E4M3 or E4M3+E5M2), and
+ *        "解决方案：混合粒度FP8精度流" (mixed-granularity FP8 activations).
+ *   [P4] web page "FP8量化训练实战指南：解决大模型训练效率瓶颈的终极方案",
+ *        sections "格式选择：E4M3与E5M2的智能搭配" (1+4+3 and 1+5+2 bit
+ *        layouts) and "分块级缩放：精度优化的进阶方案" (1x128 tiles for
+ *        activations, 128x128 blocks for weights, one scale per tile).
+ * The expansion formula is missing from the pages' text; this library fixes
+ *   f(x) = sign(x) |x|^k,   k = clamp(ln(448 / 2^-9) / ln(M / mu), 1, 16),
+ * with M = max|x| and mu = min nonzero |x| over the group (M == mu gives 16;
+ * an all-zero group gives k = 1 and scale 1), and the same 448/2^-9 target for
+ * E5M2.  Codes are y = FMT_MAX (|x|/M)^k encoded to the nearest finite FP8
+ * value (ties to the even code, saturating; a zero magnitude is code 0x00).
+ *
+ * SCALE CONVENTION.  The per-group "scale" stored by every call is the root
+ * scale s_r = M * FMT_MAX^(-1/k) (the k-th root of s = M^k / FMT_MAX, which
+ * underflows FP32 for second moments); dequantisation is
+ *   x = sign(q) * s_r * |fp8(q)|^(1/k)       ( = sign(q) |fp8(q) s|^(1/k) ).
+ *
+ * Common rules for every call below:
+ *   - All data pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates on these paths (a multi-tensor plan owns one small
+ *     device table, see coat_multi_plan_create).
+ *   - Work is enqueued on `stream` and runs asynchronously; a return of
+ *     COAT_OK means the arguments were valid and the launch was accepted.
+ *   - Arguments are validated before anything is launched; on any error no
+ *     kernel runs and no output is touched.  coat_last_error() then returns a
+ *     thread-local message.
+ *   - Buffers passed to one call must not overlap, except where stated.
+ *   - bf16 data is passed as its 16-bit patterns (uint16_t).
+ */
+#ifndef COAT_H_
+#define COAT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { COAT_E4M3 = 0, COAT_E5M2 = 1 } coat_fmt;
+typedef enum { COAT_F32 = 0, COAT_BF16 = 1 } coat_dtype;
+
+typedef enum {
+    COAT_OK = 0,
+    COAT_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad enum, bad hyperparameter */
+    COAT_ERR_MISALIGNED = 2,  /* a pointer or leading dimension breaks the 16-byte rule */
+    COAT_ERR_UNSUPPORTED = 3, /* a valid request this library does not implement (e.g. group != 128) */
+    COAT_ERR_CUDA = 4,        /* the CUDA runtime reported an error at launch or copy */
+    COAT_ERR_TIMEOUT = 5,     /* a kernel gave up a bounded wait; results are invalid */
+    COAT_ERR_NOMEM = 6        /* host or device allocation failed (plan creation only) */
+} coat_status;
+
+/* Thread-local description of the last non-OK status returned on this thread. */
+const char *coat_last_error(void);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int coat_version(void);
+
+/* ---------------------------------------------------------------------------
+ * FP8 element codec (the encode/decode steps of [P1]'s per-group quantiser;
+ * formats of [P4] 格式选择).
+ *
+ * coat_fp8_encode: q[i] = nearest finite FP8 value to y[i] (FP32), round to
+ *   nearest, ties to the even code, saturating to +-FMT_MAX (448 for E4M3,
+ *   57344 for E5M2); NaN -> 0x7F | sign; a result of magnitude zero is 0x00.
+ * coat_fp8_decode: out[i] = FP32 value of code q[i] (E5M2 0x7C is +inf;
+ *   NaN codes give NaN).
+ * n >= 0 elements; y / out need 4-byte alignment, q none.
+ * ------------------------------------------------------------------------- */
+coat_status coat_fp8_encode(const float *y, int64_t n, coat_fmt fmt, uint8_t *q,
+                            cudaStream_t stream);
+coat_status coat_fp8_decode(const uint8_t *q, int64_t n, coat_fmt fmt, float *out,
+                            cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Per-group quantise / dequantise with dynamic range expansion ([P1]
+ * 解决方案：动态范围扩展), at mixed granularity ([P1] 混合粒度FP8精度流;
+ * [P4] 分块级缩放: 1x128 per-token groups, 128x128 weight blocks).
+ *
+ * x      : rows x cols matrix of dtype xt (COAT_F32 or COAT_BF16), row-major,
+ *          leading dimension ld_x elements (ld_x >= cols).
+ * groups : group_rows x group_cols blocks; supported: 1x128 and 128x128.
+ *          Edge blocks that are cut by rows/cols hold only the valid elements.
+ * expand : 0 -> k = 1 (plain per-group scaling), 1 -> k from the formula.
+ * q      : rows x cols codes, leading dimension ld_q bytes (ld_q >= cols); only
+ *          the valid elements are written.
+ * scale,k: ceil(rows/group_rows) x ceil(cols/group_cols) floats, row-major.
+ * out    : dequantised rows x cols of dtype ot, leading dimension ld_out.
+ * Alignment: x, q, out 16-byte aligned; ld_x*size(xt), ld_q, ld_out*size(ot)
+ * multiples of 16 bytes; scale, k 4-byte aligned.  rows, cols >= 0 (0 is a
+ * no-op).
+ * ------------------------------------------------------------------------- */
+coat_status coat_group_quantize(const void *x, coat_dtype xt, int64_t rows, int64_t cols,
+                                int64_t ld_x, int group_rows, int group_cols, int expand,
+                                coat_fmt fmt, uint8_t *q, int64_t ld_q, float *scale,
+                                float *k, cudaStream_t stream);
+coat_status coat_group_dequantize(const uint8_t *q, int64_t ld_q, const float *scale,
+                                  const float *k, int64_t rows, int64_t cols,
+                                  int group_rows, int group_cols, coat_fmt fmt, void *out,
+                                  coat_dtype ot, int64_t ld_out, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * The fused AdamW step over FP8 moments ([P1] FP8优化器状态 and
+ * 动态范围扩展: per group, dequantise m and v, update, recompute k each step,
+ * requantise).  For each element i (t = step >= 1):
+ *   m  = dequant(m_q[i]),  v = dequant(v_q[i]),  g = bf16 grad[i]
+ *   m' = b1 m + (1-b1) g;   v' = b2 v + (1-b2) g^2
+ *   p  = master[i] (1 - lr wd) - (lr / (1-b1^t)) m' / (sqrt(v') / sqrt(1-b2^t) + eps)
+ *   master[i] = p (FP32, in place);  weight_bf16_out[i] = RNE_bf16(p)
+ * then m' and v' are requantised per group (expansion on) into m_q/m_scale/m_k
+ * and v_q/v_scale/v_k, in place.  The update uses the unquantised m', v'.
+ * This is torch.optim.AdamW's arithmetic (decoupled weight decay, no amsgrad).
+ *
+ * n        : number of elements (>= 0; 0 is a no-op).
+ * group    : must be 128.
+ * master   : n floats.            grad: n bf16 patterns.
+ * weight_bf16_out: n bf16 patterns, or NULL to skip the bf16 copy.
+ * m_q, v_q : ceil(n/128)*128 bytes; padding codes of a partial last group are
+ *            ignored on input and written 0.
+ * m_scale, m_k, v_scale, v_k: ceil(n/128) floats each.
+ * Alignment: every pointer 16-byte aligned (COAT_ERR_MISALIGNED otherwise).
+ * Hyperparameters: lr >= 0, 0 <= beta1, beta2 < 1, eps > 0, wd >= 0, all finite;
+ * step >= 1.  fmt_m, fmt_v: COAT_E4M3 or COAT_E5M2.
+ * ------------------------------------------------------------------------- */
+coat_status coat_adamw_step(float *master, uint16_t *weight_bf16_out, const uint16_t *grad,
+                            uint8_t *m_q, float *m_scale, float *m_k, uint8_t *v_q,
+                            float *v_scale, float *v_k, int64_t n, int group, float lr,
+                            float beta1, float beta2, float eps, float wd, int64_t step,
+                            coat_fmt fmt_m, coat_fmt fmt_v, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Multi-tensor launcher over a ragged list of parameter tensors: one kernel
+ * launch per step updates every tensor, each exactly as coat_adamw_step would
+ * (groups never span tensors; each tensor's last group may be partial).
+ *
+ * coat_multi_plan_create copies `num` host descriptors (each obeying the
+ * coat_adamw_step rules for its own n) into a device table owned by the plan
+ * (one cudaMalloc; COAT_ERR_NOMEM on failure); the copy is enqueued on
+ * `stream`.  The plan refers to the caller's buffers, which must stay valid
+ * while the plan is used.  Tensors with n == 0 are allowed.  num >= 1.
+ * coat_adamw_step_multi applies one step to all tensors on `stream`.
+ * coat_multi_plan_destroy frees the table (after synchronising the device);
+ * passing NULL is a no-op.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+    float *master;
+    uint16_t *weight_bf16_out; /* may be NULL */
+    const uint16_t *grad;
+    uint8_t *m_q;
+    float *m_scale;
+    float *m_k;
+    uint8_t *v_q;
+    float *v_scale;
+    float *v_k;
+    int64_t n;
+} coat_tensor_desc;
+
+typedef struct coat_multi_plan *coat_multi_plan_t;
+
+coat_status coat_multi_plan_create(const coat_tensor_desc *host_descs, int num, int group,
+                                   coat_fmt fmt_m, coat_fmt fmt_v, cudaStream_t stream,
+                                   coat_multi_plan_t *out_plan);
+coat_status coat_adamw_step_multi(coat_multi_plan_t plan, float lr, float beta1, float beta2,
+                                  float eps, float wd, int64_t step, cudaStream_t stream);
+coat_status coat_multi_plan_destroy(coat_multi_plan_t plan);
+/* Number of elements and tensors covered by a plan. */
+coat_status coat_multi_plan_info(coat_multi_plan_t plan, int64_t *total_elements,
+                                 int *num_tensors);
+
+/* ---------------------------------------------------------------------------
+ * Device error word.  Kernels that wait on a shared-memory barrier give up
+ * after a bounded time (about one second), set a flag and return;
+ * coat_check_device_error synchronises `stream`, reads and clears the flag,
+ * and returns COAT_ERR_TIMEOUT if it was set (COAT_OK otherwise, or
+ * COAT_ERR_CUDA if the synchronisation itself failed).
+ * ------------------------------------------------------------------------- */
+coat_status coat_check_device_error(cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* COAT_H_ */

@@ -1,0 +1,235 @@
+"""CPU oracle for the COAT FP8-optimizer-state AdamW step (test infrastructure).
+
+Plain double-precision C (``coat_oracle.c``) behind a small ctypes loader.
+Only the test-suite, ``__graft_entry__.smoke()`` and the benchmark's CPU
+baseline leg import this package; the product library never does.  The
+arithmetic, its sources and the readings taken where the COAT pages are
+silent are documented at the top of ``coat_oracle.c``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "coat_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+E4M3 = 0
+E5M2 = 1
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c99", "-ffp-contract=off", "-fno-fast-math",
+             "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _P(t):
+    return ctypes.POINTER(t)
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        L.orc_fp8_decode.restype = ctypes.c_double
+        L.orc_fp8_decode.argtypes = [ctypes.c_int, ctypes.c_uint]
+        L.orc_fp8_encode.restype = ctypes.c_uint
+        L.orc_fp8_encode.argtypes = [ctypes.c_int, ctypes.c_float]
+        L.orc_fp8_encode_array.restype = None
+        L.orc_fp8_encode_array.argtypes = [ctypes.c_int, _P(ctypes.c_float), ctypes.c_int64,
+                                           _P(ctypes.c_uint8)]
+        L.orc_fmt_max.restype = ctypes.c_double
+        L.orc_fmt_max.argtypes = [ctypes.c_int]
+        L.orc_target_range.restype = ctypes.c_double
+        L.orc_target_range.argtypes = []
+        L.orc_float_to_bf16.restype = ctypes.c_uint16
+        L.orc_float_to_bf16.argtypes = [ctypes.c_float]
+        L.orc_group_params.restype = ctypes.c_double
+        L.orc_group_params.argtypes = [_P(ctypes.c_double), ctypes.c_int64, ctypes.c_int,
+                                       ctypes.c_int, _P(ctypes.c_float), _P(ctypes.c_float)]
+        L.orc_quantize_group.restype = None
+        L.orc_quantize_group.argtypes = [_P(ctypes.c_double), ctypes.c_int64, ctypes.c_int,
+                                         ctypes.c_int, _P(ctypes.c_uint8), _P(ctypes.c_float),
+                                         _P(ctypes.c_float)]
+        L.orc_dequant_value.restype = ctypes.c_double
+        L.orc_dequant_value.argtypes = [ctypes.c_int, ctypes.c_uint8, ctypes.c_float, ctypes.c_float]
+        L.orc_group_quantize.restype = ctypes.c_int
+        L.orc_group_quantize.argtypes = [_P(ctypes.c_double), ctypes.c_int64, ctypes.c_int64,
+                                         ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int, _P(ctypes.c_uint8), ctypes.c_int64,
+                                         _P(ctypes.c_float), _P(ctypes.c_float)]
+        L.orc_group_dequantize.restype = ctypes.c_int
+        L.orc_group_dequantize.argtypes = [_P(ctypes.c_uint8), ctypes.c_int64, _P(ctypes.c_float),
+                                           _P(ctypes.c_float), ctypes.c_int64, ctypes.c_int64,
+                                           ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           _P(ctypes.c_double), ctypes.c_int64]
+        L.orc_adamw_step.restype = ctypes.c_int
+        L.orc_adamw_step.argtypes = [_P(ctypes.c_float), _P(ctypes.c_uint16), _P(ctypes.c_uint16),
+                                     _P(ctypes.c_uint8), _P(ctypes.c_float), _P(ctypes.c_float),
+                                     _P(ctypes.c_uint8), _P(ctypes.c_float), _P(ctypes.c_float),
+                                     ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_float,
+                                     ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_int64,
+                                     ctypes.c_int, ctypes.c_int, _P(ctypes.c_double)]
+        L.orc_adamw_step_unquantized.restype = ctypes.c_int
+        L.orc_adamw_step_unquantized.argtypes = [_P(ctypes.c_double)] * 4 + [
+            ctypes.c_int64, ctypes.c_double, ctypes.c_double, ctypes.c_double, ctypes.c_double,
+            ctypes.c_double, ctypes.c_int64]
+        _lib = L
+    return _lib
+
+
+def _ptr(a, ctype):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(_P(ctype))
+
+
+# ----------------------------------------------------------------------------
+# FP8 formats
+# ----------------------------------------------------------------------------
+
+def fp8_decode(fmt: int, code: int) -> float:
+    return lib().orc_fp8_decode(fmt, int(code))
+
+
+def fp8_decode_table(fmt: int) -> np.ndarray:
+    """All 256 code values (float64), from the bit definitions."""
+    return np.array([fp8_decode(fmt, c) for c in range(256)], dtype=np.float64)
+
+
+def fp8_encode(fmt: int, y: float) -> int:
+    return int(lib().orc_fp8_encode(fmt, float(y)))
+
+
+def fp8_encode_array(fmt: int, y) -> np.ndarray:
+    y = np.ascontiguousarray(y, dtype=np.float32).ravel()
+    out = np.zeros(y.size, dtype=np.uint8)
+    lib().orc_fp8_encode_array(fmt, _ptr(y, ctypes.c_float), y.size, _ptr(out, ctypes.c_uint8))
+    return out
+
+
+def fmt_max(fmt: int) -> float:
+    return lib().orc_fmt_max(fmt)
+
+
+def target_range() -> float:
+    return lib().orc_target_range()
+
+
+def float_to_bf16_bits(x) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32).ravel()
+    f = lib().orc_float_to_bf16
+    return np.fromiter((f(float(v)) for v in x), dtype=np.uint16, count=x.size)
+
+
+# ----------------------------------------------------------------------------
+# Codec
+# ----------------------------------------------------------------------------
+
+def group_params(x, expand: bool, fmt: int):
+    """(M, k, s_r) for one group of values."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    k = ctypes.c_float()
+    s = ctypes.c_float()
+    M = lib().orc_group_params(_ptr(x, ctypes.c_double), x.size, int(bool(expand)), fmt,
+                               ctypes.byref(k), ctypes.byref(s))
+    return M, k.value, s.value
+
+
+def quantize_group(x, expand: bool, fmt: int):
+    """Codes (uint8), k, s_r for one group."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    codes = np.zeros(x.size, dtype=np.uint8)
+    k = ctypes.c_float()
+    s = ctypes.c_float()
+    lib().orc_quantize_group(_ptr(x, ctypes.c_double), x.size, int(bool(expand)), fmt,
+                             _ptr(codes, ctypes.c_uint8), ctypes.byref(k), ctypes.byref(s))
+    return codes, k.value, s.value
+
+
+def dequant_value(fmt: int, code: int, s_r: float, k: float) -> float:
+    return lib().orc_dequant_value(fmt, int(code), float(s_r), float(k))
+
+
+def group_quantize(x, group_rows: int, group_cols: int, expand: bool, fmt: int):
+    """x: 2-D array (any float dtype, converted exactly to float64).
+    Returns (q uint8 [rows, cols], scale f32 [nbr, nbc], k f32 [nbr, nbc])."""
+    x = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    assert x.ndim == 2
+    rows, cols = x.shape
+    nbr = -(-rows // group_rows)
+    nbc = -(-cols // group_cols)
+    q = np.zeros((rows, cols), dtype=np.uint8)
+    scale = np.zeros((nbr, nbc), dtype=np.float32)
+    k = np.zeros((nbr, nbc), dtype=np.float32)
+    rc = lib().orc_group_quantize(_ptr(x, ctypes.c_double), rows, cols, cols, group_rows,
+                                  group_cols, int(bool(expand)), fmt, _ptr(q, ctypes.c_uint8),
+                                  cols, _ptr(scale, ctypes.c_float), _ptr(k, ctypes.c_float))
+    assert rc == 0
+    return q, scale, k
+
+
+def group_dequantize(q, scale, k, group_rows: int, group_cols: int, fmt: int) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    scale = np.ascontiguousarray(scale, dtype=np.float32)
+    k = np.ascontiguousarray(k, dtype=np.float32)
+    rows, cols = q.shape
+    out = np.zeros((rows, cols), dtype=np.float64)
+    rc = lib().orc_group_dequantize(_ptr(q, ctypes.c_uint8), cols, _ptr(scale, ctypes.c_float),
+                                    _ptr(k, ctypes.c_float), rows, cols, group_rows, group_cols,
+                                    fmt, _ptr(out, ctypes.c_double), cols)
+    assert rc == 0
+    return out
+
+
+# ----------------------------------------------------------------------------
+# AdamW step
+# ----------------------------------------------------------------------------
+
+def adamw_step(master, weight_out, grad_bits, m_q, m_scale, m_k, v_q, v_scale, v_k, *, group=128,
+               lr, beta1, beta2, eps, wd, step, fmt_m, fmt_v, want_update=False):
+    """In-place oracle step on numpy arrays (master f32, weight_out u16 or None,
+    grad_bits u16, codes u8 padded to whole groups, scale/k f32 per group).
+    Returns the per-element |adaptive update| (float64) if want_update."""
+    n = master.size
+    for a, dt in ((master, np.float32), (grad_bits, np.uint16), (m_q, np.uint8),
+                  (v_q, np.uint8), (m_scale, np.float32), (m_k, np.float32),
+                  (v_scale, np.float32), (v_k, np.float32)):
+        assert a.dtype == dt and a.flags["C_CONTIGUOUS"]
+    if weight_out is not None:
+        assert weight_out.dtype == np.uint16 and weight_out.size == n
+    ng = -(-n // group)
+    assert m_q.size >= ng * group and v_q.size >= ng * group and m_k.size >= ng
+    upd = np.zeros(n, dtype=np.float64) if want_update else None
+    rc = lib().orc_adamw_step(_ptr(master, ctypes.c_float), _ptr(weight_out, ctypes.c_uint16),
+                              _ptr(grad_bits, ctypes.c_uint16), _ptr(m_q, ctypes.c_uint8),
+                              _ptr(m_scale, ctypes.c_float), _ptr(m_k, ctypes.c_float),
+                              _ptr(v_q, ctypes.c_uint8), _ptr(v_scale, ctypes.c_float),
+                              _ptr(v_k, ctypes.c_float), n, group, lr, beta1, beta2, eps, wd,
+                              step, fmt_m, fmt_v, _ptr(upd, ctypes.c_double))
+    assert rc == 0
+    return upd
+
+
+def adamw_step_unquantized(p, m, v, g, *, lr, beta1, beta2, eps, wd, step):
+    """In-place plain AdamW on float64 arrays."""
+    for a in (p, m, v, g):
+        assert a.dtype == np.float64 and a.flags["C_CONTIGUOUS"]
+    rc = lib().orc_adamw_step_unquantized(_ptr(p, ctypes.c_double), _ptr(m, ctypes.c_double),
+                                          _ptr(v, ctypes.c_double), _ptr(g, ctypes.c_double),
+                                          p.size, lr, beta1, beta2, eps, wd, step)
+    assert rc == 0
