@@ -1,0 +1,472 @@
+"""Benchmark of the COAT FP8-state AdamW step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one fused AdamW step (dequantise FP8 m/v, AdamW on the FP32 master,
+bf16 copy, recompute k, requantise) over the whole parameter list, launched as a
+single multi-tensor kernel.  Default workload: the Llama-2-7B-shaped parameter
+list (291 tensors, 6,738,415,616 parameters, E4M3 m + E5M2 v, group 128), all
+inputs resident in HBM (68 GB per step, far larger than the 126 MB L2, so no L2
+flush is needed between steps).  Synthetic data from the seeded generator.
+
+Multi-GPU (torchrun): every rank updates its own full parameter list (the
+parameter groups are independent; there is no exchange step), so per-GPU work
+is fixed ("weak" scaling); time = max over ranks of device time.
+
+--impl reference times the CPU oracle (plain double-precision C, one host
+thread) on a bounded sample of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Gparams/s of FP8-state AdamW step; HBM GB/s as % of B200 roofline"
+UNIT = "Gparams/s"
+HBM_FALLBACK_GBS = 6650.0
+KERNEL_SOURCES = ["fp8_optimizer_state_b200/csrc/adamw_fp8.cu",
+                  "fp8_optimizer_state_b200/csrc/coat_device.cuh"]
+# DRAM bytes per launch of the step kernel from an ncu capture (see profiles/),
+# valid only for the kernel sources with this hash.
+TRAFFIC = {"sources_sha256": None, "bytes_per_param": None}
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
+    except Exception:
+        return None
+
+
+def algorithmic_bytes(sizes, with_weight=True):
+    """Per step: master read+write 8 B, grad 2 B, bf16 copy 2 B, m and v codes
+    read+write 4 B per stored code (whole groups), 4 metadata floats read+write
+    per group (32 B)."""
+    tot = 0
+    for n in sizes:
+        ng = -(-n // 128)
+        tot += 8 * n + 2 * n + (2 * n if with_weight else 0) + 4 * ng * 128 + 32 * ng
+    return tot
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id):
+        self.bus_id = (bus_id or "").lower()
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0, t1):
+        rows = []
+        for ts, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            bus = parts[1].lower()
+            if self.bus_id and not (bus.endswith(self.bus_id[-12:]) or self.bus_id.endswith(bus[-12:])):
+                continue
+            rows.append((ts, parts))
+        inside = [p for ts, p in rows if t0 - 0.05 <= ts <= t1 + 0.05] or [p for _, p in rows]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(p[2]) for p in inside if num(p[2]) is not None]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for p in inside:
+            for name, val in zip(names, p[6:10]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": num(inside[0][3]), "reasons": sorted(reasons),
+                "power_w_max": max((num(p[4]) or 0.0) for p in inside), "samples": len(inside)}
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timing (the reference arm and the cpu_baseline key)
+# ----------------------------------------------------------------------------
+def oracle_sample_inputs(cfg, count, use_device):
+    """Inputs of the first `count` elements of the workload's first tensor (bits
+    from the seeded generator; on the device when one is in use, which is
+    bit-identical and much faster than the NumPy generator)."""
+    import synth
+    if use_device:
+        import torch
+        m = torch.empty(count, dtype=torch.float32, device="cuda")
+        g = torch.empty(count, dtype=torch.int16, device="cuda")
+        synth.device_master(m, 0, 0)
+        master = m.cpu().numpy()
+        synth.device_m_warm(m, 0, 0)
+        m0 = m.cpu().numpy()
+        synth.device_v_warm(m, 0, 0)
+        v0 = m.cpu().numpy()
+        synth.device_grad(g, 0, 0, 1)
+        grad = g.cpu().numpy().view(np.uint16)
+        del m, g
+    else:
+        master = synth.master(0, 0, 0, count)
+        m0 = synth.m_warm(0, 0, 0, count)
+        v0 = synth.v_warm(0, 0, 0, count)
+        grad = synth.grad_bits(0, 0, 1, 0, count)
+    return master, m0, v0, grad
+
+
+def time_oracle(cfg, count, steps, use_device):
+    import oracle as orc
+    from synth.params import HYPER as H
+    master, m0, v0, grad = oracle_sample_inputs(cfg, count, use_device)
+    ng = -(-count // 128)
+    mq = np.zeros(ng * 128, np.uint8)
+    vq = np.zeros(ng * 128, np.uint8)
+    q, s, k = orc.group_quantize(m0.reshape(1, count), 1, 128, True, cfg["fmt_m"])
+    mq[:count], ms, mk = q.ravel(), s.ravel().copy(), k.ravel().copy()
+    q, s, k = orc.group_quantize(v0.reshape(1, count), 1, 128, True, cfg["fmt_v"])
+    vq[:count], vs, vk = q.ravel(), s.ravel().copy(), k.ravel().copy()
+    weight = np.zeros(count, np.uint16)
+    times = []
+    for t in range(1, steps + 1):
+        t0 = time.perf_counter()
+        orc.adamw_step(master, weight, grad, mq, ms, mk, vq, vs, vk, lr=H["lr"], beta1=H["beta1"],
+                       beta2=H["beta2"], eps=H["eps"], wd=H["wd"], step=t, fmt_m=cfg["fmt_m"],
+                       fmt_v=cfg["fmt_v"])
+        times.append(time.perf_counter() - t0)
+    return times
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing
+# ----------------------------------------------------------------------------
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def max_over_ranks(x, ws, device):
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws, device):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[device.index] if device is not None and device.type == "cuda" else None)
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+def run_ours(args, cfg, ws, rank, local):
+    import torch
+    import fp8_optimizer_state_b200 as coat
+    from synth.params import HYPER as H
+    from synth.workload import DeviceParamSet
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    coat.lib()
+
+    shapes = cfg["shapes"]()
+    ps = DeviceParamSet(shapes, seed=rank)
+    ps.fill_master()
+    ps.fill_grad(1)
+    tmp = None
+    for i in range(len(ps)):
+        v = ps.views(i)
+        if v["n"] == 0:
+            continue
+        tmp = ps.warm_values(i, "m", tmp)
+        coat.coat_group_quantize(tmp.view(1, -1), 1, 128, True, cfg["fmt_m"], v["mq"].view(1, -1),
+                                 v["ms"].view(1, -1), v["mk"].view(1, -1))
+        tmp = ps.warm_values(i, "v", tmp)
+        coat.coat_group_quantize(tmp.view(1, -1), 1, 128, True, cfg["fmt_v"], v["vq"].view(1, -1),
+                                 v["vs"].view(1, -1), v["vk"].view(1, -1))
+    del tmp
+    descs = []
+    for i in range(len(ps)):
+        v = ps.views(i)
+        descs.append(coat.make_desc(v["master"], v["weight"], v["grad"], v["mq"], v["ms"], v["mk"],
+                                    v["vq"], v["vs"], v["vk"]))
+    plan = coat.coat_multi_plan_create(descs, cfg["fmt_m"], cfg["fmt_v"])
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+    step_no = [0]
+
+    def one_step():
+        step_no[0] += 1
+        coat.coat_adamw_step_multi(plan, lr=H["lr"], beta1=H["beta1"], beta2=H["beta2"],
+                                   eps=H["eps"], wd=H["wd"], step=step_no[0])
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    coat.coat_check_device_error()
+
+    props = torch.cuda.get_device_properties(dev)
+    bus = getattr(props, "pci_bus_id", None)
+    if bus is None:
+        bus = "%08x:%02x:%02x.0" % (getattr(props, "pci_domain_id", 0), getattr(props, "pci_bus_id", 0),
+                                     getattr(props, "pci_device_id", 0))
+    sampler = ClockSampler(str(bus))
+    sampler.start()
+    time.sleep(0.3)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier(ws, dev)
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    t_start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        one_step()
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    barrier(ws, dev)
+    time.sleep(0.2)
+    sampler.stop()
+    coat.coat_check_device_error()
+
+    elapsed_ms = t_start.elapsed_time(t_end)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    elapsed_ms = max_over_ranks(elapsed_ms, ws, dev)
+    kernel_ms = max_over_ranks(statistics.mean(launch_ms), ws, dev)
+    n_params = ps.total_elements
+    value = ws * n_params * args.steps / (elapsed_ms * 1e-3) / 1e9
+
+    # roofline of the step kernel
+    peaks = measured_peaks()
+    peak = peaks["hbm_gbs"] if peaks and peaks.get("hbm_gbs") else HBM_FALLBACK_GBS
+    alg = algorithmic_bytes(ps.sizes, with_weight=True)
+    achieved = alg / (kernel_ms * 1e-3) / 1e9
+    traffic = None
+    if TRAFFIC["sources_sha256"] == kernel_hash() and TRAFFIC["bytes_per_param"]:
+        traffic = TRAFFIC["bytes_per_param"] * n_params
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "peak_source": "measured" if peaks else "fallback",
+                "algorithmic_bytes_per_launch": alg,
+                "bytes_per_param": round(alg / n_params, 4), "kernel_ms": round(kernel_ms, 4),
+                "frac_of_nominal_8TBs": round(achieved / 8000.0, 4)}
+    clocks = sampler.summary(wall0, wall1)
+
+    # end to end through the public API with host buffers: per step, H2D of the
+    # bf16 gradients from pinned memory, the step (per tensor, overlapped with the
+    # copies on separate streams), D2H of the bf16 weight copy
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, cfg, ps, ws, dev, H, coat)
+
+    plan.destroy()
+    result = None
+    if rank == 0:
+        cpu = None
+        if ws == 1 and not args.no_cpu_baseline:
+            count = args.cpu_sample
+            times = time_oracle(cfg, count, 1, use_device=True)
+            cpu = {"value": round(count / times[0] / 1e9, 6), "unit": UNIT, "cores": 1,
+                   "kind": "oracle",
+                   "sample": "first %d elements of tensor 0 of the workload, 1 step, one host "
+                             "thread (%.1f s)" % (count, times[0])}
+        result = {
+            "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(elapsed_ms / args.steps, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": cfg["workload"], "params_per_gpu": n_params,
+                       "tensors": len(ps), "group": 128,
+                       "fmt_m": "E4M3" if cfg["fmt_m"] == 0 else "E5M2",
+                       "fmt_v": "E4M3" if cfg["fmt_v"] == 0 else "E5M2",
+                       "hyper": H, "l2": "no flush: %.1f GB of inputs per step >> 126 MB L2"
+                                         % (alg / 1e9),
+                       "parallelism": "replicas%d (independent parameter groups, no collective)" % ws
+                       if ws > 1 else "single GPU"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": args.steps, "clocks": clocks,
+        }
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return result
+
+
+def run_e2e(args, cfg, ps, ws, dev, H, coat):
+    import torch
+    n_pad = ps.master.numel()
+    host_grad = torch.empty(n_pad, dtype=torch.int16, pin_memory=True)
+    host_w = torch.empty(n_pad, dtype=torch.int16, pin_memory=True)
+    host_grad.copy_(ps.grad)
+    torch.cuda.synchronize()
+    comp = torch.cuda.current_stream()
+    h2d = torch.cuda.Stream()
+    d2h = torch.cuda.Stream()
+    views = [ps.views(i) for i in range(len(ps))]
+    offs = ps.off
+    ev_in = [torch.cuda.Event() for _ in views]
+    ev_done = [torch.cuda.Event() for _ in views]
+    steps = max(1, min(args.steps, args.e2e_steps))
+    base_step = 1000
+
+    def step(t):
+        for i, v in enumerate(views):
+            a, n = int(offs[i]), v["n"]
+            if n == 0:
+                continue
+            with torch.cuda.stream(h2d):
+                v["grad"].copy_(host_grad[a:a + n], non_blocking=True)
+                ev_in[i].record(h2d)
+            comp.wait_event(ev_in[i])
+            coat.coat_adamw_step(v["master"], v["weight"], v["grad"], v["mq"], v["ms"], v["mk"],
+                                 v["vq"], v["vs"], v["vk"], lr=H["lr"], beta1=H["beta1"],
+                                 beta2=H["beta2"], eps=H["eps"], wd=H["wd"], step=t,
+                                 fmt_m=cfg["fmt_m"], fmt_v=cfg["fmt_v"], stream=comp)
+            ev_done[i].record(comp)
+            d2h.wait_event(ev_done[i])
+            with torch.cuda.stream(d2h):
+                host_w[a:a + n].copy_(v["weight"], non_blocking=True)
+        d2h.synchronize()
+        comp.synchronize()
+
+    step(base_step)   # warm-up
+    barrier(ws, dev)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for s in range(steps):
+        step(base_step + 1 + s)
+    torch.cuda.synchronize()
+    el = time.perf_counter() - t0
+    el = max_over_ranks(el, ws, dev)
+    coat.coat_check_device_error()
+    value = ws * ps.total_elements * steps / el / 1e9
+    nbytes = 2 * ps.total_elements
+    return {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": nbytes,
+            "d2h_bytes_per_step": nbytes, "steps": steps,
+            "how": "per step: H2D bf16 grads from pinned host memory, one coat_adamw_step per "
+                   "tensor, D2H bf16 weight copy to pinned host memory; copies on two side "
+                   "streams overlapped with the steps; host wall clock, max over ranks",
+            "gpu_launches_per_step": sum(1 for v in views if v["n"] > 0)}
+
+
+def run_reference(args, cfg, ws, rank):
+    """The CPU oracle on a bounded sample per step (one host thread)."""
+    if rank != 0:
+        return None
+    count = args.ref_sample
+    times = time_oracle(cfg, count, args.warmup + args.steps, use_device=False)
+    timed = times[args.warmup:]
+    total = sum(timed)
+    value = count * len(timed) / total / 1e9
+    sample = ("first %d elements of tensor 0 of the workload per step (bits from the seeded "
+              "generator), oracle adamw_step, one host thread" % count)
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * total / len(timed), 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg["workload"], "sample_elements": count},
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    from synth.params import CONFIGS
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="llama2-7b", choices=sorted(CONFIGS))
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample", type=int, default=16 << 20)
+    ap.add_argument("--ref-sample", type=int, default=2 << 20)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    ws, rank, local = dist_env()
+    cfg = CONFIGS[args.config]
+    if args.impl == "reference":
+        res = run_reference(args, cfg, ws, rank)
+    else:
+        res = run_ours(args, cfg, ws, rank, local)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,197 @@
+"""Python binding of libcoat.so, the B200 COAT FP8-optimizer-state library.
+
+Argument marshalling only: every function here has the name of a C entry point
+in include/coat.h, takes CUDA tensors (or None for optional pointers), passes
+their device pointers and the current CUDA stream, and raises CoatError on a
+non-OK status.  All arithmetic runs in the library's CUDA kernels; there is no
+CPU fallback -- if libcoat.so is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libcoat.so")
+
+COAT_E4M3, COAT_E5M2 = 0, 1
+COAT_F32, COAT_BF16 = 0, 1
+GROUP = 128
+STATUS = {0: "COAT_OK", 1: "COAT_ERR_INVALID_ARG", 2: "COAT_ERR_MISALIGNED",
+          3: "COAT_ERR_UNSUPPORTED", 4: "COAT_ERR_CUDA", 5: "COAT_ERR_TIMEOUT", 6: "COAT_ERR_NOMEM"}
+
+# (name, restype, argtypes) of every exported entry point
+_vp, _i64, _i32, _f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+EXPORTS = [
+    ("coat_last_error", ctypes.c_char_p, []),
+    ("coat_version", _i32, []),
+    ("coat_fp8_encode", _i32, [_vp, _i64, _i32, _vp, _vp]),
+    ("coat_fp8_decode", _i32, [_vp, _i64, _i32, _vp, _vp]),
+    ("coat_group_quantize", _i32, [_vp, _i32, _i64, _i64, _i64, _i32, _i32, _i32, _i32, _vp, _i64,
+                                   _vp, _vp, _vp]),
+    ("coat_group_dequantize", _i32, [_vp, _i64, _vp, _vp, _i64, _i64, _i32, _i32, _i32, _vp, _i32,
+                                     _i64, _vp]),
+    ("coat_adamw_step", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _f32, _f32,
+                               _f32, _f32, _f32, _i64, _i32, _i32, _vp]),
+    ("coat_multi_plan_create", _i32, [_vp, _i32, _i32, _i32, _i32, _vp, ctypes.POINTER(_vp)]),
+    ("coat_adamw_step_multi", _i32, [_vp, _f32, _f32, _f32, _f32, _f32, _i64, _vp]),
+    ("coat_multi_plan_destroy", _i32, [_vp]),
+    ("coat_multi_plan_info", _i32, [_vp, ctypes.POINTER(_i64), ctypes.POINTER(_i32)]),
+    ("coat_check_device_error", _i32, [_vp]),
+]
+
+
+class CoatError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__("%s: %s" % (STATUS.get(status, status), message))
+        self.status = status
+
+
+class TensorDesc(ctypes.Structure):
+    """coat_tensor_desc"""
+    _fields_ = [("master", _vp), ("weight_bf16_out", _vp), ("grad", _vp), ("m_q", _vp),
+                ("m_scale", _vp), ("m_k", _vp), ("v_q", _vp), ("v_scale", _vp), ("v_k", _vp),
+                ("n", _i64)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libcoat.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libcoat.so is not built (%s); run "
+                               "`python -m fp8_optimizer_state_b200.build`" % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        for name, res, args in EXPORTS:
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status):
+    if status != 0:
+        raise CoatError(status, lib().coat_last_error().decode())
+
+
+def _p(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    return t.data_ptr()
+
+
+def _s(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _dt(t):
+    import torch
+    if t.dtype == torch.float32:
+        return COAT_F32
+    if t.dtype in (torch.bfloat16, torch.int16, torch.uint16):
+        return COAT_BF16
+    raise ValueError("expected float32 or bfloat16 data, got %s" % t.dtype)
+
+
+def coat_version():
+    return lib().coat_version()
+
+
+def coat_last_error():
+    return lib().coat_last_error().decode()
+
+
+def coat_fp8_encode(y, fmt, q, stream=None):
+    """q[i] = FP8 code of FP32 y[i] (nearest, ties to even, saturating)."""
+    _check(lib().coat_fp8_encode(_p(y), y.numel(), fmt, _p(q), _s(stream)))
+
+
+def coat_fp8_decode(q, fmt, out, stream=None):
+    _check(lib().coat_fp8_decode(_p(q), q.numel(), fmt, _p(out), _s(stream)))
+
+
+def coat_group_quantize(x, group_rows, group_cols, expand, fmt, q, scale, k, stream=None):
+    """x: 2-D CUDA tensor (f32 or bf16) with unit column stride; q: uint8 [rows, >=cols];
+    scale, k: float32 [ceil(rows/gr), ceil(cols/gc)]."""
+    rows, cols = x.shape
+    _check(lib().coat_group_quantize(_p(x), _dt(x), rows, cols, x.stride(0), group_rows, group_cols,
+                                     int(bool(expand)), fmt, _p(q), q.stride(0), _p(scale), _p(k),
+                                     _s(stream)))
+
+
+def coat_group_dequantize(q, scale, k, group_rows, group_cols, fmt, out, stream=None):
+    rows, cols = out.shape
+    _check(lib().coat_group_dequantize(_p(q), q.stride(0), _p(scale), _p(k), rows, cols, group_rows,
+                                       group_cols, fmt, _p(out), _dt(out), out.stride(0),
+                                       _s(stream)))
+
+
+def coat_adamw_step(master, weight_bf16_out, grad, m_q, m_scale, m_k, v_q, v_scale, v_k, *, lr,
+                    beta1, beta2, eps, wd, step, fmt_m=COAT_E4M3, fmt_v=COAT_E4M3, group=GROUP,
+                    stream=None):
+    """One fused AdamW step over FP8 moments (in place); see include/coat.h."""
+    _check(lib().coat_adamw_step(_p(master), _p(weight_bf16_out), _p(grad), _p(m_q), _p(m_scale),
+                                 _p(m_k), _p(v_q), _p(v_scale), _p(v_k), master.numel(), group, lr,
+                                 beta1, beta2, eps, wd, step, fmt_m, fmt_v, _s(stream)))
+
+
+def make_desc(master, weight_bf16_out, grad, m_q, m_scale, m_k, v_q, v_scale, v_k):
+    return TensorDesc(_p(master), _p(weight_bf16_out), _p(grad), _p(m_q), _p(m_scale), _p(m_k),
+                      _p(v_q), _p(v_scale), _p(v_k), master.numel())
+
+
+class coat_multi_plan:
+    """Owns a coat_multi_plan_t (created by coat_multi_plan_create)."""
+
+    def __init__(self, handle, descs):
+        self.handle = handle
+        self._descs = descs
+
+    def info(self):
+        n = ctypes.c_int64()
+        c = ctypes.c_int()
+        _check(lib().coat_multi_plan_info(self.handle, ctypes.byref(n), ctypes.byref(c)))
+        return n.value, c.value
+
+    def destroy(self):
+        if self.handle:
+            _check(lib().coat_multi_plan_destroy(self.handle))
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+
+def coat_multi_plan_create(descs, fmt_m=COAT_E4M3, fmt_v=COAT_E4M3, group=GROUP, stream=None):
+    """descs: list of TensorDesc (see make_desc)."""
+    arr = (TensorDesc * len(descs))(*descs)
+    h = ctypes.c_void_p()
+    _check(lib().coat_multi_plan_create(ctypes.cast(arr, ctypes.c_void_p), len(descs), group, fmt_m,
+                                        fmt_v, _s(stream), ctypes.byref(h)))
+    return coat_multi_plan(h.value, arr)
+
+
+def coat_adamw_step_multi(plan, *, lr, beta1, beta2, eps, wd, step, stream=None):
+    _check(lib().coat_adamw_step_multi(plan.handle, lr, beta1, beta2, eps, wd, step, _s(stream)))
+
+
+def coat_multi_plan_destroy(plan):
+    plan.destroy()
+
+
+def coat_check_device_error(stream=None):
+    _check(lib().coat_check_device_error(_s(stream)))

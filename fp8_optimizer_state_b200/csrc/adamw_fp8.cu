@@ -1,0 +1,413 @@
+// adamw_fp8.cu -- the fused COAT AdamW step over FP8 moments on sm_100a.
+//
+// What it computes ([P1] "FP8训练新范式：减少40%显存占用，训练速度提高1.4倍",
+// sections "FP8优化器状态" and "解决方案：动态范围扩展"; AdamW as in
+// torch.optim.AdamW): per group of 128 elements, dequantise the FP8 moments
+// (x = sign(q) s_r |q|^(1/k)), update them with the bf16 gradient, apply the
+// decoupled-weight-decay AdamW update to the FP32 master weight, write its
+// bf16 copy, recompute each moment's expansion exponent k and root scale from
+// the new group max/min, and requantise.
+//
+// Design (HBM-bound: 16.25 algorithmic bytes per parameter, no tensor cores):
+//  * persistent CTAs, 2 per SM; tiles of 32 groups (4096 elements);
+//  * one producer thread streams whole tiles (master, grad, both code arrays,
+//    the four metadata arrays: 33,280 B) into a 3-stage shared-memory ring
+//    with 1-D cp.async.bulk copies completing on an mbarrier, so that bytes in
+//    flight do not depend on registers;
+//  * 8 consumer warps; each warp owns 4 groups of a tile, 8 lanes per group,
+//    16 elements per lane in 4 chunks of 4 contiguous elements (chunk order
+//    rotated per group to keep shared-memory reads conflict-free); group
+//    max / min-nonzero by 3 xor-shuffles inside the 8 lanes;
+//  * a consumer copies its slice of the stage into registers and releases the
+//    stage before computing; results go straight to HBM with coalesced
+//    16/8/4-byte stores (every warp store instruction writes whole sectors);
+//  * tiles that are not entirely valid (a tensor's last tile when n is not a
+//    multiple of 4096) take a direct path: the consumers load from global
+//    memory with bounds checks; padding elements count as zero and their
+//    codes are written 0;
+//  * every mbarrier wait is bounded (about a second); on timeout the kernel
+//    sets a device error bit and returns.
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "coat_device.cuh"
+#include "coat_internal.h"
+
+namespace coat {
+namespace {
+
+constexpr int kConsumerWarps = 8;
+constexpr int kGroupsPerWarp = 4;
+constexpr int kTileGroups = kConsumerWarps * kGroupsPerWarp;  // 32
+constexpr int kTileElems = kTileGroups * kGroup;               // 4096
+constexpr int kStages = 3;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;             // 288
+constexpr int kCtasPerSm = 2;
+
+// Stage layout (bytes): every array starts on a 128-byte boundary.
+constexpr uint32_t kOffMaster = 0;
+constexpr uint32_t kOffGrad = kOffMaster + kTileElems * 4;   // 16384
+constexpr uint32_t kOffMq = kOffGrad + kTileElems * 2;       // 24576
+constexpr uint32_t kOffVq = kOffMq + kTileElems;             // 28672
+constexpr uint32_t kOffMs = kOffVq + kTileElems;             // 32768
+constexpr uint32_t kOffMk = kOffMs + kTileGroups * 4;
+constexpr uint32_t kOffVs = kOffMk + kTileGroups * 4;
+constexpr uint32_t kOffVk = kOffVs + kTileGroups * 4;
+constexpr uint32_t kStageBytes = kOffVk + kTileGroups * 4;   // 33280
+
+struct TileHeader {
+  int64_t g0;       // first group of the tile within its tensor
+  int32_t tensor;   // tensor index (multi-tensor launch)
+  int32_t ngroups;  // groups of this tile that exist
+  int32_t full;     // 1: all 4096 elements valid and staged in shared memory
+  int32_t pad;
+};
+
+struct Smem {
+  float tab_m[256];
+  float tab_v[256];
+  uint64_t full_bar[kStages];
+  uint64_t empty_bar[kStages];
+  TileHeader hdr[kStages];
+};
+constexpr size_t kSmemBytes = ((sizeof(Smem) + 127) / 128) * 128 + size_t(kStages) * kStageBytes;
+
+// Tile -> tensor lookup.  Single-tensor launches use one descriptor passed by
+// value; multi-tensor launches use the plan's device tables.
+struct SingleTensor {
+  TensorArgs t;
+  __device__ __forceinline__ int64_t tiles() const { return t.tiles; }
+  __device__ __forceinline__ int32_t tensor_of(int64_t) const { return 0; }
+  __device__ __forceinline__ int64_t first_tile(int32_t) const { return 0; }
+  __device__ __forceinline__ const TensorArgs& get(int32_t) const { return t; }
+};
+struct MultiTensor {
+  const TensorArgs* descs;
+  const int32_t* tile_tensor;
+  int64_t total_tiles;
+  __device__ __forceinline__ int64_t tiles() const { return total_tiles; }
+  __device__ __forceinline__ int32_t tensor_of(int64_t tile) const { return tile_tensor[tile]; }
+  __device__ __forceinline__ int64_t first_tile(int32_t i) const { return descs[i].tile_begin; }
+  __device__ __forceinline__ TensorArgs get(int32_t i) const { return descs[i]; }
+};
+
+// The 16 elements a lane owns, as loaded.
+struct LaneIn {
+  float4 p[4];
+  uint2 g[4];
+  uint32_t mq[4], vq[4];
+  float ms, mk, vs, vk;
+};
+
+__device__ __forceinline__ int chunk_of(int j, int slot) { return (j + slot) & 3; }
+
+__device__ __forceinline__ void load_from_stage(const uint8_t* st, int lg, int slot, int l,
+                                                LaneIn& in) {
+  const float* sm = reinterpret_cast<const float*>(st + kOffMaster) + lg * kGroup;
+  const uint16_t* sg = reinterpret_cast<const uint16_t*>(st + kOffGrad) + lg * kGroup;
+  const uint8_t* smq = st + kOffMq + lg * kGroup;
+  const uint8_t* svq = st + kOffVq + lg * kGroup;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int e = 32 * chunk_of(j, slot) + 4 * l;
+    in.p[j] = *reinterpret_cast<const float4*>(sm + e);
+    in.g[j] = *reinterpret_cast<const uint2*>(sg + e);
+    in.mq[j] = *reinterpret_cast<const uint32_t*>(smq + e);
+    in.vq[j] = *reinterpret_cast<const uint32_t*>(svq + e);
+  }
+  in.ms = reinterpret_cast<const float*>(st + kOffMs)[lg];
+  in.mk = reinterpret_cast<const float*>(st + kOffMk)[lg];
+  in.vs = reinterpret_cast<const float*>(st + kOffVs)[lg];
+  in.vk = reinterpret_cast<const float*>(st + kOffVk)[lg];
+}
+
+// Direct loads for a tile that is not entirely valid.  Elements at or beyond
+// n read as zero; codes of a group that exists are always readable (the code
+// arrays hold whole groups).
+__device__ __forceinline__ void load_direct(const TensorArgs& t, int64_t gi, bool active, int slot,
+                                            int l, LaneIn& in) {
+  const int64_t base = gi * kGroup;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int64_t e = base + 32 * chunk_of(j, slot) + 4 * l;
+    float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
+    uint2 g = make_uint2(0u, 0u);
+    uint32_t mq = 0u, vq = 0u;
+    if (active) {
+      if (e + 4 <= t.n) {
+        p = *reinterpret_cast<const float4*>(t.master + e);
+        g = *reinterpret_cast<const uint2*>(t.grad + e);
+      } else {
+        float pv[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t gv[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (e + i < t.n) {
+            pv[i] = t.master[e + i];
+            gv[i] = t.grad[e + i];
+          }
+        p = make_float4(pv[0], pv[1], pv[2], pv[3]);
+        g = make_uint2(gv[0] | (gv[1] << 16), gv[2] | (gv[3] << 16));
+      }
+      mq = *reinterpret_cast<const uint32_t*>(t.mq + e);
+      vq = *reinterpret_cast<const uint32_t*>(t.vq + e);
+    }
+    in.p[j] = p;
+    in.g[j] = g;
+    in.mq[j] = mq;
+    in.vq[j] = vq;
+  }
+  in.ms = active ? t.ms[gi] : 1.f;
+  in.mk = active ? t.mk[gi] : 1.f;
+  in.vs = active ? t.vs[gi] : 1.f;
+  in.vk = active ? t.vk[gi] : 1.f;
+}
+
+__device__ __forceinline__ float f4get(const float4& v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// The per-lane body: everything after the loads.
+template <int FM, int FV>
+__device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, int64_t gi,
+                                        bool active, int slot, int l, const StepHyper& h,
+                                        const float* tab_m, const float* tab_v) {
+  const int64_t base = gi * kGroup;
+  // dequantisation constants of this group (stored k and root scale)
+  const float invk_m = rcp_approx(in.mk), sb_m = in.ms * h.beta1;
+  const float invk_v = rcp_approx(in.vk), sb_v = in.vs * h.beta2;
+
+  float m1[16], v1[16];
+  float maxm = 0.f, maxv = 0.f;
+  uint32_t minm = 0xFFFFFFFFu, minv = 0xFFFFFFFFu;
+
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int64_t e = base + 32 * chunk_of(j, slot) + 4 * l;
+    float pn[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t gw = (i < 2) ? in.g[j].x : in.g[j].y;
+      const float g = (i & 1) ? bf16hi(gw) : bf16lo(gw);
+      const uint32_t cm = (in.mq[j] >> (8 * i)) & 0xFFu;
+      const uint32_t cv = (in.vq[j] >> (8 * i)) & 0xFFu;
+      // beta1 * m and beta2 * v, dequantised: s_r * beta * 2^(log2|q| / k)
+      float bm = ex2_approx(tab_m[cm] * invk_m) * sb_m;
+      bm = __uint_as_float(__float_as_uint(bm) ^ ((cm & 0x80u) << 24));
+      const float bv = ex2_approx(tab_v[cv] * invk_v) * sb_v;
+      const float mn = __fmaf_rn(h.omb1, g, bm);
+      const float vn = __fmaf_rn(h.omb2 * g, g, bv);
+      const float p = f4get(in.p[j], i);
+      const float denom = __fmaf_rn(sqrt_approx(vn), h.rsbc2, h.eps);
+      const float upd = (h.step_size * mn) * rcp_approx(denom);
+      pn[i] = p + __fmaf_rn(-p, h.lrwd, -upd);
+      const bool valid = active && (e + i < t.n);
+      m1[4 * j + i] = valid ? mn : 0.f;
+      v1[4 * j + i] = valid ? vn : 0.f;
+      maxm = fmaxf(maxm, fabsf(m1[4 * j + i]));
+      maxv = fmaxf(maxv, v1[4 * j + i]);
+      minm = min(minm, (__float_as_uint(m1[4 * j + i]) & 0x7FFFFFFFu) - 1u);
+      minv = min(minv, __float_as_uint(v1[4 * j + i]) - 1u);
+    }
+    if (active) {
+      if (e + 4 <= t.n) {
+        *reinterpret_cast<float4*>(t.master + e) = make_float4(pn[0], pn[1], pn[2], pn[3]);
+        if (t.wout)
+          *reinterpret_cast<uint2*>(t.wout + e) =
+              make_uint2(pack_bf16x2(pn[0], pn[1]), pack_bf16x2(pn[2], pn[3]));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (e + i < t.n) {
+            t.master[e + i] = pn[i];
+            if (t.wout) t.wout[e + i] = static_cast<uint16_t>(pack_bf16x2(pn[i], 0.f));
+          }
+      }
+    }
+  }
+
+  // group statistics over the 8 lanes of this group
+#pragma unroll
+  for (int off = 1; off < 8; off <<= 1) {
+    maxm = fmaxf(maxm, __shfl_xor_sync(0xFFFFFFFFu, maxm, off));
+    maxv = fmaxf(maxv, __shfl_xor_sync(0xFFFFFFFFu, maxv, off));
+    minm = min(minm, __shfl_xor_sync(0xFFFFFFFFu, minm, off));
+    minv = min(minv, __shfl_xor_sync(0xFFFFFFFFu, minv, off));
+  }
+  const float mum = __uint_as_float(minm + 1u), muv = __uint_as_float(minv + 1u);
+  float km, srm, invMm, kv, srv, invMv;
+  group_params<FM>(maxm, mum, true, km, srm, invMm);
+  group_params<FV>(maxv, muv, true, kv, srv, invMv);
+
+  // expand + encode, store codes (whole group, padding included) and metadata
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int64_t e = base + 32 * chunk_of(j, slot) + 4 * l;
+    uint32_t cmw[4], cvw[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float xm = m1[4 * j + i], xv = v1[4 * j + i];
+      cmw[i] = enc_signed<FM>(xm, expand_value<FM>(xm, invMm, km));
+      cvw[i] = enc_signed<FV>(xv, expand_value<FV>(xv, invMv, kv));
+    }
+    if (active) {
+      *reinterpret_cast<uint32_t*>(t.mq + e) =
+          __byte_perm(__byte_perm(cmw[0], cmw[1], 0x0040), __byte_perm(cmw[2], cmw[3], 0x0040), 0x5410);
+      *reinterpret_cast<uint32_t*>(t.vq + e) =
+          __byte_perm(__byte_perm(cvw[0], cvw[1], 0x0040), __byte_perm(cvw[2], cvw[3], 0x0040), 0x5410);
+    }
+  }
+  if (active && l == 0) {
+    t.ms[gi] = srm;
+    t.mk[gi] = km;
+    t.vs[gi] = srv;
+    t.vk[gi] = kv;
+  }
+}
+
+template <int FM, int FV, class Map>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    adamw_fp8_kernel(const Map map, const StepHyper h, unsigned* err) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  Smem& S = *reinterpret_cast<Smem*>(smem_raw);
+  uint8_t* stages = smem_raw + ((sizeof(Smem) + 127) / 128) * 128;
+
+  fill_log2_table<FM>(S.tab_m);
+  fill_log2_table<FV>(S.tab_v);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&S.full_bar[s], 1);
+      mbar_init(&S.empty_bar[s], kConsumerWarps);
+    }
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t ntiles = map.tiles();
+
+  if (warp == kConsumerWarps) {
+    // ---------------- producer ----------------
+    if (lane != 0) return;
+    int64_t it = 0;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+      const int s = static_cast<int>(it % kStages);
+      const uint32_t use = static_cast<uint32_t>(it / kStages);
+      if (use > 0 && !mbar_wait(&S.empty_bar[s], (use - 1) & 1u, kWaitBudgetCycles)) {
+        atomicOr(err, kErrTimeoutProducer);
+        // Drain copies still in flight into stages the consumers never freed.
+        for (int d = 0; d < kStages; ++d) {
+          const int64_t itd = it - 1 - d;
+          if (itd < 0) break;
+          const int sd = static_cast<int>(itd % kStages);
+          if (!mbar_wait(&S.full_bar[sd], static_cast<uint32_t>(itd / kStages) & 1u,
+                         kWaitBudgetCycles))
+            atomicOr(err, kErrCopyDrain);
+        }
+        return;
+      }
+      const int32_t ti = map.tensor_of(tile);
+      const TensorArgs t = map.get(ti);
+      const int64_t local = tile - map.first_tile(ti);
+      const int64_t g0 = local * kTileGroups;
+      const int64_t groups = (t.n + kGroup - 1) / kGroup;
+      const int64_t ng = (groups - g0) < kTileGroups ? (groups - g0) : int64_t(kTileGroups);
+      const int64_t e0 = g0 * kGroup;
+      const bool full = (e0 + kTileElems <= t.n);
+      TileHeader& hd = S.hdr[s];
+      hd.g0 = g0;
+      hd.tensor = ti;
+      hd.ngroups = static_cast<int32_t>(ng);
+      hd.full = full ? 1 : 0;
+      if (full) {
+        uint8_t* st = stages + size_t(s) * kStageBytes;
+        mbar_arrive_expect_tx(&S.full_bar[s], kStageBytes);
+        bulk_g2s(st + kOffMaster, t.master + e0, kTileElems * 4, &S.full_bar[s]);
+        bulk_g2s(st + kOffGrad, t.grad + e0, kTileElems * 2, &S.full_bar[s]);
+        bulk_g2s(st + kOffMq, t.mq + e0, kTileElems, &S.full_bar[s]);
+        bulk_g2s(st + kOffVq, t.vq + e0, kTileElems, &S.full_bar[s]);
+        bulk_g2s(st + kOffMs, t.ms + g0, kTileGroups * 4, &S.full_bar[s]);
+        bulk_g2s(st + kOffMk, t.mk + g0, kTileGroups * 4, &S.full_bar[s]);
+        bulk_g2s(st + kOffVs, t.vs + g0, kTileGroups * 4, &S.full_bar[s]);
+        bulk_g2s(st + kOffVk, t.vk + g0, kTileGroups * 4, &S.full_bar[s]);
+      } else {
+        mbar_arrive(&S.full_bar[s]);
+      }
+    }
+    return;
+  }
+
+  // ---------------- consumers ----------------
+  const int slot = lane >> 3, l = lane & 7;
+  const int lg = warp * kGroupsPerWarp + slot;  // group within the tile
+  int64_t it = 0;
+  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+    const int s = static_cast<int>(it % kStages);
+    const uint32_t use = static_cast<uint32_t>(it / kStages);
+    if (!mbar_wait(&S.full_bar[s], use & 1u, kWaitBudgetCycles)) {
+      atomicOr(err, kErrTimeoutConsumer);
+      return;
+    }
+    const TileHeader hd = S.hdr[s];
+    const TensorArgs t = map.get(hd.tensor);
+    const bool active = lg < hd.ngroups;
+    const int64_t gi = hd.g0 + lg;
+    LaneIn in;
+    if (hd.full)
+      load_from_stage(stages + size_t(s) * kStageBytes, lg, slot, l, in);
+    else
+      load_direct(t, gi, active, slot, l, in);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S.empty_bar[s]);
+    process<FM, FV>(in, t, gi, active, slot, l, h, S.tab_m, S.tab_v);
+  }
+}
+
+template <int FM, int FV, class Map>
+cudaError_t launch_step(const Map& map, int64_t ntiles, const StepHyper& h, unsigned* err,
+                        cudaStream_t stream) {
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  auto kern = adamw_fp8_kernel<FM, FV, Map>;
+  if (dev < 64 && !configured[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes));
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  const int64_t want = int64_t(sm_count(dev)) * kCtasPerSm;
+  const int64_t grid = ntiles < want ? ntiles : want;
+  if (grid <= 0) return cudaSuccess;
+  kern<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(map, h, err);
+  return cudaGetLastError();
+}
+
+template <class Map>
+cudaError_t dispatch(int fm, int fv, const Map& map, int64_t ntiles, const StepHyper& h,
+                     unsigned* err, cudaStream_t stream) {
+  if (fm == kE4M3 && fv == kE4M3) return launch_step<kE4M3, kE4M3>(map, ntiles, h, err, stream);
+  if (fm == kE4M3 && fv == kE5M2) return launch_step<kE4M3, kE5M2>(map, ntiles, h, err, stream);
+  if (fm == kE5M2 && fv == kE4M3) return launch_step<kE5M2, kE4M3>(map, ntiles, h, err, stream);
+  return launch_step<kE5M2, kE5M2>(map, ntiles, h, err, stream);
+}
+
+}  // namespace
+
+int64_t step_tile_groups() { return kTileGroups; }
+
+cudaError_t launch_adamw_single(const TensorArgs& t, int fm, int fv, const StepHyper& h,
+                                unsigned* err, cudaStream_t stream) {
+  SingleTensor map{t};
+  return dispatch(fm, fv, map, t.tiles, h, err, stream);
+}
+
+cudaError_t launch_adamw_multi(const TensorArgs* d_descs, const int32_t* d_tile_tensor,
+                               int64_t total_tiles, int fm, int fv, const StepHyper& h,
+                               unsigned* err, cudaStream_t stream) {
+  MultiTensor map{d_descs, d_tile_tensor, total_tiles};
+  return dispatch(fm, fv, map, total_tiles, h, err, stream);
+}
+
+}  // namespace coat

@@ -1,0 +1,373 @@
+// api.cu -- the C ABI declared in include/coat.h: argument validation (before
+// any CUDA call, so a bad call launches nothing and touches nothing), error
+// reporting, multi-tensor plans, and kernel launches on the caller's stream.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "coat.h"
+#include "coat_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+coat_status fail(coat_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+coat_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(COAT_ERR_CUDA, "%s: %s (%d)", where, cudaGetErrorString(e), static_cast<int>(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool valid_fmt(int f) { return f == COAT_E4M3 || f == COAT_E5M2; }
+bool valid_dtype(int d) { return d == COAT_F32 || d == COAT_BF16; }
+size_t dtype_size(int d) { return d == COAT_F32 ? 4 : 2; }
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// device-side error word and per-device caches
+// ---------------------------------------------------------------------------
+__device__ unsigned g_coat_device_error;
+
+namespace coat {
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int g_sm_count[kMaxDevices];
+unsigned* g_err_ptr[kMaxDevices];
+}  // namespace
+
+int sm_count(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_sm_count[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      v = 148;
+    g_sm_count[dev] = v;
+  }
+  return g_sm_count[dev];
+}
+
+// Device address of the error word on the current device (looked up once per
+// device with that device current).
+static cudaError_t device_error_ptr(unsigned** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_coat_device_error);
+    if (e != cudaSuccess) return e;
+    g_err_ptr[dev] = static_cast<unsigned*>(p);
+  }
+  *out = g_err_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace coat
+
+// ---------------------------------------------------------------------------
+// helpers shared by the step entry points
+// ---------------------------------------------------------------------------
+namespace {
+
+coat_status check_hyper(float lr, float beta1, float beta2, float eps, float wd, int64_t step) {
+  if (!std::isfinite(lr) || lr < 0.f) return fail(COAT_ERR_INVALID_ARG, "lr must be finite and >= 0");
+  if (!(beta1 >= 0.f && beta1 < 1.f)) return fail(COAT_ERR_INVALID_ARG, "beta1 must be in [0, 1)");
+  if (!(beta2 >= 0.f && beta2 < 1.f)) return fail(COAT_ERR_INVALID_ARG, "beta2 must be in [0, 1)");
+  if (!std::isfinite(eps) || !(eps > 0.f)) return fail(COAT_ERR_INVALID_ARG, "eps must be finite and > 0");
+  if (!std::isfinite(wd) || wd < 0.f) return fail(COAT_ERR_INVALID_ARG, "weight decay must be finite and >= 0");
+  if (step < 1) return fail(COAT_ERR_INVALID_ARG, "step must be >= 1");
+  return COAT_OK;
+}
+
+coat::StepHyper make_hyper(float lr, float beta1, float beta2, float eps, float wd, int64_t step) {
+  const double b1 = beta1, b2 = beta2;
+  const double bc1 = 1.0 - std::pow(b1, static_cast<double>(step));
+  const double bc2 = 1.0 - std::pow(b2, static_cast<double>(step));
+  coat::StepHyper h;
+  h.beta1 = beta1;
+  h.beta2 = beta2;
+  h.omb1 = static_cast<float>(1.0 - b1);
+  h.omb2 = static_cast<float>(1.0 - b2);
+  h.step_size = static_cast<float>(static_cast<double>(lr) / bc1);
+  h.rsbc2 = static_cast<float>(1.0 / std::sqrt(bc2));
+  h.eps = eps;
+  h.lrwd = static_cast<float>(static_cast<double>(lr) * static_cast<double>(wd));
+  return h;
+}
+
+coat_status check_tensor(const coat_tensor_desc& d, int index) {
+  if (d.n < 0) return fail(COAT_ERR_INVALID_ARG, "tensor %d: n < 0", index);
+  if (d.n == 0) return COAT_OK;
+  const void* req[] = {d.master, d.grad, d.m_q, d.m_scale, d.m_k, d.v_q, d.v_scale, d.v_k};
+  const char* names[] = {"master", "grad", "m_q", "m_scale", "m_k", "v_q", "v_scale", "v_k"};
+  for (int i = 0; i < 8; ++i) {
+    if (!req[i]) return fail(COAT_ERR_INVALID_ARG, "tensor %d: %s is NULL", index, names[i]);
+    if (!aligned(req[i], 16))
+      return fail(COAT_ERR_MISALIGNED, "tensor %d: %s is not 16-byte aligned", index, names[i]);
+  }
+  if (d.weight_bf16_out && !aligned(d.weight_bf16_out, 16))
+    return fail(COAT_ERR_MISALIGNED, "tensor %d: weight_bf16_out is not 16-byte aligned", index);
+  return COAT_OK;
+}
+
+coat::TensorArgs to_args(const coat_tensor_desc& d, int64_t tile_begin) {
+  coat::TensorArgs t;
+  t.master = d.master;
+  t.wout = d.weight_bf16_out;
+  t.grad = d.grad;
+  t.mq = d.m_q;
+  t.ms = d.m_scale;
+  t.mk = d.m_k;
+  t.vq = d.v_q;
+  t.vs = d.v_scale;
+  t.vk = d.v_k;
+  t.n = d.n;
+  const int64_t groups = (d.n + 127) / 128;
+  const int64_t tg = coat::step_tile_groups();
+  t.tiles = (groups + tg - 1) / tg;
+  t.tile_begin = tile_begin;
+  return t;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// public ABI
+// ---------------------------------------------------------------------------
+extern "C" {
+
+const char* coat_last_error(void) { return g_last_error.c_str(); }
+
+int coat_version(void) { return 10000; }
+
+coat_status coat_fp8_encode(const float* y, int64_t n, coat_fmt fmt, uint8_t* q, cudaStream_t stream) {
+  if (n < 0) return fail(COAT_ERR_INVALID_ARG, "coat_fp8_encode: n < 0");
+  if (!valid_fmt(fmt)) return fail(COAT_ERR_INVALID_ARG, "coat_fp8_encode: bad fmt %d", int(fmt));
+  if (n == 0) return COAT_OK;
+  if (!y || !q) return fail(COAT_ERR_INVALID_ARG, "coat_fp8_encode: NULL pointer");
+  if (!aligned(y, 4)) return fail(COAT_ERR_MISALIGNED, "coat_fp8_encode: y not 4-byte aligned");
+  cudaError_t e = coat::launch_fp8_encode(y, n, fmt, q, stream);
+  return e == cudaSuccess ? COAT_OK : cuda_fail(e, "coat_fp8_encode");
+}
+
+coat_status coat_fp8_decode(const uint8_t* q, int64_t n, coat_fmt fmt, float* out, cudaStream_t stream) {
+  if (n < 0) return fail(COAT_ERR_INVALID_ARG, "coat_fp8_decode: n < 0");
+  if (!valid_fmt(fmt)) return fail(COAT_ERR_INVALID_ARG, "coat_fp8_decode: bad fmt %d", int(fmt));
+  if (n == 0) return COAT_OK;
+  if (!q || !out) return fail(COAT_ERR_INVALID_ARG, "coat_fp8_decode: NULL pointer");
+  if (!aligned(out, 4)) return fail(COAT_ERR_MISALIGNED, "coat_fp8_decode: out not 4-byte aligned");
+  cudaError_t e = coat::launch_fp8_decode(q, n, fmt, out, stream);
+  return e == cudaSuccess ? COAT_OK : cuda_fail(e, "coat_fp8_decode");
+}
+
+static coat_status check_groups(const char* fn, int gr, int gc) {
+  if (gr < 1 || gc < 1) return fail(COAT_ERR_INVALID_ARG, "%s: group shape must be positive", fn);
+  if (!((gr == 1 && gc == 128) || (gr == 128 && gc == 128)))
+    return fail(COAT_ERR_UNSUPPORTED, "%s: group %dx%d not supported (1x128 or 128x128)", fn, gr, gc);
+  return COAT_OK;
+}
+
+coat_status coat_group_quantize(const void* x, coat_dtype xt, int64_t rows, int64_t cols,
+                                int64_t ld_x, int group_rows, int group_cols, int expand,
+                                coat_fmt fmt, uint8_t* q, int64_t ld_q, float* scale, float* k,
+                                cudaStream_t stream) {
+  const char* fn = "coat_group_quantize";
+  if (rows < 0 || cols < 0) return fail(COAT_ERR_INVALID_ARG, "%s: negative shape", fn);
+  if (!valid_dtype(xt)) return fail(COAT_ERR_INVALID_ARG, "%s: bad dtype %d", fn, int(xt));
+  if (!valid_fmt(fmt)) return fail(COAT_ERR_INVALID_ARG, "%s: bad fmt %d", fn, int(fmt));
+  if (expand != 0 && expand != 1) return fail(COAT_ERR_INVALID_ARG, "%s: expand must be 0 or 1", fn);
+  coat_status st = check_groups(fn, group_rows, group_cols);
+  if (st != COAT_OK) return st;
+  if (ld_x < cols || ld_q < cols) return fail(COAT_ERR_INVALID_ARG, "%s: leading dimension < cols", fn);
+  if (rows == 0 || cols == 0) return COAT_OK;
+  if (!x || !q || !scale || !k) return fail(COAT_ERR_INVALID_ARG, "%s: NULL pointer", fn);
+  if (!aligned(x, 16) || !aligned(q, 16)) return fail(COAT_ERR_MISALIGNED, "%s: x and q must be 16-byte aligned", fn);
+  if (rows > 1 && ((ld_x * int64_t(dtype_size(xt))) % 16 != 0 || ld_q % 16 != 0))
+    return fail(COAT_ERR_MISALIGNED, "%s: row strides must be multiples of 16 bytes", fn);
+  if (!aligned(scale, 4) || !aligned(k, 4)) return fail(COAT_ERR_MISALIGNED, "%s: scale/k not 4-byte aligned", fn);
+  cudaError_t e = coat::launch_group_quantize(x, xt, rows, cols, ld_x, group_rows, expand, fmt, q,
+                                              ld_q, scale, k, stream);
+  return e == cudaSuccess ? COAT_OK : cuda_fail(e, fn);
+}
+
+coat_status coat_group_dequantize(const uint8_t* q, int64_t ld_q, const float* scale, const float* k,
+                                  int64_t rows, int64_t cols, int group_rows, int group_cols,
+                                  coat_fmt fmt, void* out, coat_dtype ot, int64_t ld_out,
+                                  cudaStream_t stream) {
+  const char* fn = "coat_group_dequantize";
+  if (rows < 0 || cols < 0) return fail(COAT_ERR_INVALID_ARG, "%s: negative shape", fn);
+  if (!valid_dtype(ot)) return fail(COAT_ERR_INVALID_ARG, "%s: bad dtype %d", fn, int(ot));
+  if (!valid_fmt(fmt)) return fail(COAT_ERR_INVALID_ARG, "%s: bad fmt %d", fn, int(fmt));
+  coat_status st = check_groups(fn, group_rows, group_cols);
+  if (st != COAT_OK) return st;
+  if (ld_out < cols || ld_q < cols) return fail(COAT_ERR_INVALID_ARG, "%s: leading dimension < cols", fn);
+  if (rows == 0 || cols == 0) return COAT_OK;
+  if (!out || !q || !scale || !k) return fail(COAT_ERR_INVALID_ARG, "%s: NULL pointer", fn);
+  if (!aligned(out, 16) || !aligned(q, 16)) return fail(COAT_ERR_MISALIGNED, "%s: q and out must be 16-byte aligned", fn);
+  if (rows > 1 && ((ld_out * int64_t(dtype_size(ot))) % 16 != 0 || ld_q % 16 != 0))
+    return fail(COAT_ERR_MISALIGNED, "%s: row strides must be multiples of 16 bytes", fn);
+  if (!aligned(scale, 4) || !aligned(k, 4)) return fail(COAT_ERR_MISALIGNED, "%s: scale/k not 4-byte aligned", fn);
+  cudaError_t e = coat::launch_group_dequantize(q, ld_q, scale, k, rows, cols, group_rows,
+                                                group_cols, fmt, out, ot, ld_out, stream);
+  return e == cudaSuccess ? COAT_OK : cuda_fail(e, fn);
+}
+
+coat_status coat_adamw_step(float* master, uint16_t* weight_bf16_out, const uint16_t* grad,
+                            uint8_t* m_q, float* m_scale, float* m_k, uint8_t* v_q, float* v_scale,
+                            float* v_k, int64_t n, int group, float lr, float beta1, float beta2,
+                            float eps, float wd, int64_t step, coat_fmt fmt_m, coat_fmt fmt_v,
+                            cudaStream_t stream) {
+  if (n < 0) return fail(COAT_ERR_INVALID_ARG, "coat_adamw_step: n < 0");
+  if (group < 1) return fail(COAT_ERR_INVALID_ARG, "coat_adamw_step: group must be positive");
+  if (group != 128) return fail(COAT_ERR_UNSUPPORTED, "coat_adamw_step: group %d not supported (128)", group);
+  if (!valid_fmt(fmt_m) || !valid_fmt(fmt_v)) return fail(COAT_ERR_INVALID_ARG, "coat_adamw_step: bad fmt");
+  coat_status st = check_hyper(lr, beta1, beta2, eps, wd, step);
+  if (st != COAT_OK) return st;
+  const coat_tensor_desc d = {master, weight_bf16_out, grad, m_q, m_scale, m_k, v_q, v_scale, v_k, n};
+  st = check_tensor(d, 0);
+  if (st != COAT_OK) return st;
+  if (n == 0) return COAT_OK;
+  unsigned* err = nullptr;
+  cudaError_t e = coat::device_error_ptr(&err);
+  if (e != cudaSuccess) return cuda_fail(e, "coat_adamw_step");
+  e = coat::launch_adamw_single(to_args(d, 0), fmt_m, fmt_v,
+                                make_hyper(lr, beta1, beta2, eps, wd, step), err, stream);
+  return e == cudaSuccess ? COAT_OK : cuda_fail(e, "coat_adamw_step");
+}
+
+}  // extern "C"
+
+struct coat_multi_plan {
+  coat::TensorArgs* d_descs = nullptr;  // one allocation: descriptors, then tile->tensor map
+  int32_t* d_tile_tensor = nullptr;
+  int64_t total_tiles = 0;
+  int64_t total_elements = 0;
+  int num = 0;
+  int fmt_m = 0, fmt_v = 0;
+  int device = 0;
+};
+
+extern "C" {
+
+coat_status coat_multi_plan_create(const coat_tensor_desc* host_descs, int num, int group,
+                                   coat_fmt fmt_m, coat_fmt fmt_v, cudaStream_t stream,
+                                   coat_multi_plan_t* out_plan) {
+  const char* fn = "coat_multi_plan_create";
+  if (!out_plan) return fail(COAT_ERR_INVALID_ARG, "%s: out_plan is NULL", fn);
+  *out_plan = nullptr;
+  if (!host_descs || num < 1) return fail(COAT_ERR_INVALID_ARG, "%s: need num >= 1 descriptors", fn);
+  if (group < 1) return fail(COAT_ERR_INVALID_ARG, "%s: group must be positive", fn);
+  if (group != 128) return fail(COAT_ERR_UNSUPPORTED, "%s: group %d not supported (128)", fn, group);
+  if (!valid_fmt(fmt_m) || !valid_fmt(fmt_v)) return fail(COAT_ERR_INVALID_ARG, "%s: bad fmt", fn);
+  std::vector<coat::TensorArgs> descs(static_cast<size_t>(num));
+  int64_t tiles = 0, elems = 0;
+  for (int i = 0; i < num; ++i) {
+    coat_status st = check_tensor(host_descs[i], i);
+    if (st != COAT_OK) return st;
+    descs[i] = to_args(host_descs[i], tiles);
+    tiles += descs[i].tiles;
+    elems += host_descs[i].n;
+  }
+  if (tiles >= (int64_t(1) << 31)) return fail(COAT_ERR_UNSUPPORTED, "%s: too many tiles", fn);
+  std::vector<int32_t> map(static_cast<size_t>(tiles > 0 ? tiles : 1));
+  for (int i = 0; i < num; ++i)
+    for (int64_t t = 0; t < descs[i].tiles; ++t) map[descs[i].tile_begin + t] = i;
+
+  coat_multi_plan* p = new (std::nothrow) coat_multi_plan;
+  if (!p) return fail(COAT_ERR_NOMEM, "%s: host allocation failed", fn);
+  const size_t desc_bytes = ((sizeof(coat::TensorArgs) * num + 255) / 256) * 256;
+  const size_t map_bytes = sizeof(int32_t) * map.size();
+  void* mem = nullptr;
+  cudaError_t e = cudaGetDevice(&p->device);
+  if (e == cudaSuccess) e = cudaMalloc(&mem, desc_bytes + map_bytes);
+  if (e != cudaSuccess) {
+    delete p;
+    cudaGetLastError();
+    return e == cudaErrorMemoryAllocation ? fail(COAT_ERR_NOMEM, "%s: device allocation failed", fn)
+                                          : cuda_fail(e, fn);
+  }
+  p->d_descs = static_cast<coat::TensorArgs*>(mem);
+  p->d_tile_tensor = reinterpret_cast<int32_t*>(static_cast<char*>(mem) + desc_bytes);
+  e = cudaMemcpyAsync(p->d_descs, descs.data(), sizeof(coat::TensorArgs) * num,
+                      cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(p->d_tile_tensor, map.data(), map_bytes, cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);  // host vectors die on return
+  if (e != cudaSuccess) {
+    cudaFree(mem);
+    delete p;
+    return cuda_fail(e, fn);
+  }
+  p->total_tiles = tiles;
+  p->total_elements = elems;
+  p->num = num;
+  p->fmt_m = fmt_m;
+  p->fmt_v = fmt_v;
+  *out_plan = p;
+  return COAT_OK;
+}
+
+coat_status coat_adamw_step_multi(coat_multi_plan_t plan, float lr, float beta1, float beta2,
+                                  float eps, float wd, int64_t step, cudaStream_t stream) {
+  if (!plan) return fail(COAT_ERR_INVALID_ARG, "coat_adamw_step_multi: plan is NULL");
+  coat_status st = check_hyper(lr, beta1, beta2, eps, wd, step);
+  if (st != COAT_OK) return st;
+  if (plan->total_tiles == 0) return COAT_OK;
+  unsigned* err = nullptr;
+  cudaError_t e = coat::device_error_ptr(&err);
+  if (e != cudaSuccess) return cuda_fail(e, "coat_adamw_step_multi");
+  e = coat::launch_adamw_multi(plan->d_descs, plan->d_tile_tensor, plan->total_tiles, plan->fmt_m,
+                               plan->fmt_v, make_hyper(lr, beta1, beta2, eps, wd, step), err, stream);
+  return e == cudaSuccess ? COAT_OK : cuda_fail(e, "coat_adamw_step_multi");
+}
+
+coat_status coat_multi_plan_destroy(coat_multi_plan_t plan) {
+  if (!plan) return COAT_OK;
+  cudaError_t e = cudaFree(plan->d_descs);
+  delete plan;
+  return e == cudaSuccess ? COAT_OK : cuda_fail(e, "coat_multi_plan_destroy");
+}
+
+coat_status coat_multi_plan_info(coat_multi_plan_t plan, int64_t* total_elements, int* num_tensors) {
+  if (!plan) return fail(COAT_ERR_INVALID_ARG, "coat_multi_plan_info: plan is NULL");
+  if (total_elements) *total_elements = plan->total_elements;
+  if (num_tensors) *num_tensors = plan->num;
+  return COAT_OK;
+}
+
+coat_status coat_check_device_error(cudaStream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "coat_check_device_error");
+  unsigned v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_coat_device_error, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e, "coat_check_device_error");
+  if (v != 0) {
+    const unsigned zero = 0;
+    cudaMemcpyToSymbol(g_coat_device_error, &zero, sizeof(zero));
+    return fail(COAT_ERR_TIMEOUT, "a kernel gave up a bounded wait (device error bits 0x%x)", v);
+  }
+  return COAT_OK;
+}
+
+}  // extern "C"

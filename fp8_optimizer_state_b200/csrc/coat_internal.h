@@ -1,0 +1,54 @@
+// coat_internal.h -- host-side launch interface between the C ABI (api.cu) and
+// the kernels (adamw_fp8.cu, codec.cu).  Not part of the public ABI.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace coat {
+
+// One parameter tensor as the step kernel sees it (device pointers).
+struct TensorArgs {
+  float* master;
+  uint16_t* wout;  // may be null
+  const uint16_t* grad;
+  uint8_t* mq;
+  float* ms;
+  float* mk;
+  uint8_t* vq;
+  float* vs;
+  float* vk;
+  int64_t n;
+  int64_t tiles;       // ceil(ceil(n/128) / groups-per-tile)
+  int64_t tile_begin;  // first tile of this tensor in a multi-tensor launch
+};
+
+// Hyperparameters as the kernel uses them (bias corrections folded on the host
+// in double): m' = beta1 m + omb1 g, v' = beta2 v + omb2 g^2,
+// p <- p - p lrwd - step_size m' / (sqrt(v') rsbc2 + eps).
+struct StepHyper {
+  float beta1, beta2, omb1, omb2;
+  float step_size;  // lr / (1 - beta1^t)
+  float rsbc2;      // 1 / sqrt(1 - beta2^t)
+  float eps;
+  float lrwd;       // lr * wd
+};
+
+int sm_count(int dev);
+int64_t step_tile_groups();
+
+cudaError_t launch_adamw_single(const TensorArgs& t, int fm, int fv, const StepHyper& h,
+                                unsigned* err, cudaStream_t stream);
+cudaError_t launch_adamw_multi(const TensorArgs* d_descs, const int32_t* d_tile_tensor,
+                               int64_t total_tiles, int fm, int fv, const StepHyper& h,
+                               unsigned* err, cudaStream_t stream);
+
+cudaError_t launch_fp8_encode(const float* y, int64_t n, int fmt, uint8_t* q, cudaStream_t s);
+cudaError_t launch_fp8_decode(const uint8_t* q, int64_t n, int fmt, float* out, cudaStream_t s);
+cudaError_t launch_group_quantize(const void* x, int xt, int64_t rows, int64_t cols, int64_t ldx,
+                                  int gr, int expand, int fmt, uint8_t* q, int64_t ldq,
+                                  float* scale, float* k, cudaStream_t s);
+cudaError_t launch_group_dequantize(const uint8_t* q, int64_t ldq, const float* scale,
+                                    const float* k, int64_t rows, int64_t cols, int gr, int gc,
+                                    int fmt, void* out, int ot, int64_t ldo, cudaStream_t s);
+
+}  // namespace coat

@@ -98,9 +98,9 @@ coat_status coat_fp8_decode(const uint8_t *q, int64_t n, coat_fmt fmt, float *ou
  *          the valid elements are written.
  * scale,k: ceil(rows/group_rows) x ceil(cols/group_cols) floats, row-major.
  * out    : dequantised rows x cols of dtype ot, leading dimension ld_out.
- * Alignment: x, q, out 16-byte aligned; ld_x*size(xt), ld_q, ld_out*size(ot)
- * multiples of 16 bytes; scale, k 4-byte aligned.  rows, cols >= 0 (0 is a
- * no-op).
+ * Alignment: x, q, out 16-byte aligned; when rows > 1, ld_x*size(xt), ld_q and
+ * ld_out*size(ot) multiples of 16 bytes; scale, k 4-byte aligned.  rows,
+ * cols >= 0 (0 is a no-op).
  * ------------------------------------------------------------------------- */
 coat_status coat_group_quantize(const void *x, coat_dtype xt, int64_t rows, int64_t cols,
                                 int64_t ld_x, int group_rows, int group_cols, int expand,

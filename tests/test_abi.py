@@ -1,0 +1,128 @@
+"""The C ABI library on a host without a GPU: it loads, exports every entry point
+declared in include/coat.h, and rejects bad arguments with the documented status
+codes before making any CUDA call (so these run on CPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import fp8_optimizer_state_b200 as coat
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "coat.h")
+
+OK, INVALID, MISALIGNED, UNSUPPORTED = 0, 1, 2, 3
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(coat_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_and_binding_agree():
+    names = declared_functions()
+    assert len(names) >= 12
+    assert sorted(n for n, _, _ in coat.EXPORTS) == names
+
+
+def test_library_exports_every_declared_symbol():
+    L = coat.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    assert coat.coat_version() == 10000
+
+
+def test_nm_exports_match():
+    import shutil
+    import subprocess
+    nm = shutil.which("nm")
+    if nm is None:
+        pytest.skip("nm not available")
+    out = subprocess.run([nm, "-D", "--defined-only", coat.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    exported = set(re.findall(r" T (coat_[a-z0-9_]+)$", out, flags=re.M))
+    assert set(declared_functions()) <= exported
+
+
+A = 1 << 20   # a fake, 16-byte aligned "device address" (never dereferenced)
+HP = dict(lr=1e-3, b1=0.9, b2=0.95, eps=1e-8, wd=0.1, step=1)
+
+
+def step(ptrs=None, n=1000, group=128, fm=0, fv=0, **kw):
+    p = dict(HP)
+    p.update(kw)
+    ptrs = ptrs or [A] * 9
+    return coat.lib().coat_adamw_step(*ptrs, n, group, p["lr"], p["b1"], p["b2"], p["eps"], p["wd"],
+                                      p["step"], fm, fv, None)
+
+
+def test_step_validation():
+    assert step(n=-1) == INVALID
+    assert step(group=0) == INVALID
+    assert step(group=64) == UNSUPPORTED
+    assert step(fm=2) == INVALID and step(fv=-1) == INVALID
+    assert step(lr=-1.0) == INVALID and step(lr=float("nan")) == INVALID
+    assert step(b1=1.0) == INVALID and step(b2=-0.1) == INVALID
+    assert step(eps=0.0) == INVALID and step(wd=-0.5) == INVALID
+    assert step(step=0) == INVALID
+    for i in range(9):
+        ptrs = [A] * 9
+        ptrs[i] = None
+        expect = OK if i == 1 else INVALID     # weight_bf16_out may be NULL
+        if expect == INVALID:
+            assert step(ptrs) == INVALID, i
+        ptrs[i] = A + 8
+        assert step(ptrs) == MISALIGNED, i
+    # n == 0 is a no-op that needs no pointers and no device
+    assert step([None] * 9, n=0) == OK
+    assert "aligned" in coat.coat_last_error() or coat.coat_last_error() != ""
+
+
+def test_codec_validation():
+    L = coat.lib()
+    q = lambda **k: L.coat_group_quantize(k.get("x", A), k.get("xt", 1), k.get("rows", 8),
+                                          k.get("cols", 256), k.get("ldx", 256), k.get("gr", 1),
+                                          k.get("gc", 128), k.get("expand", 1), k.get("fmt", 0),
+                                          k.get("q", A), k.get("ldq", 256), A, A, None)
+    assert q(gr=2) == UNSUPPORTED and q(gc=64) == UNSUPPORTED and q(gr=0) == INVALID
+    assert q(xt=7) == INVALID and q(fmt=3) == INVALID and q(expand=2) == INVALID
+    assert q(rows=-1) == INVALID and q(ldx=100) == INVALID and q(ldq=255) == INVALID
+    assert q(x=A + 4) == MISALIGNED and q(q=A + 1) == MISALIGNED
+    assert q(ldx=260) == MISALIGNED      # 520-byte bf16 rows
+    assert q(ldq=264) == MISALIGNED
+    assert q(rows=0) == OK and q(cols=0, x=None) == OK
+    d = lambda **k: L.coat_group_dequantize(k.get("q", A), k.get("ldq", 256), A, A, 8, 256,
+                                            k.get("gr", 128), 128, k.get("fmt", 1), k.get("out", A),
+                                            k.get("ot", 0), k.get("ldo", 256), None)
+    assert d(gr=3) == UNSUPPORTED and d(ot=5) == INVALID and d(out=A + 2) == MISALIGNED
+    assert L.coat_fp8_encode(A, -1, 0, A, None) == INVALID
+    assert L.coat_fp8_encode(A + 2, 10, 0, A, None) == MISALIGNED
+    assert L.coat_fp8_encode(A, 10, 9, A, None) == INVALID
+    assert L.coat_fp8_decode(A, 0, 0, None, None) == OK
+
+
+def test_plan_validation():
+    L = coat.lib()
+    h = ctypes.c_void_p()
+    d = coat.TensorDesc(A, None, A, A, A, A, A, A, A, 1000)
+    arr = (coat.TensorDesc * 1)(d)
+    assert L.coat_multi_plan_create(None, 1, 128, 0, 0, None, ctypes.byref(h)) == INVALID
+    assert L.coat_multi_plan_create(ctypes.cast(arr, ctypes.c_void_p), 0, 128, 0, 0, None,
+                                    ctypes.byref(h)) == INVALID
+    assert L.coat_multi_plan_create(ctypes.cast(arr, ctypes.c_void_p), 1, 256, 0, 0, None,
+                                    ctypes.byref(h)) == UNSUPPORTED
+    bad = (coat.TensorDesc * 2)(d, coat.TensorDesc(A, None, A + 4, A, A, A, A, A, A, 10))
+    assert L.coat_multi_plan_create(ctypes.cast(bad, ctypes.c_void_p), 2, 128, 0, 0, None,
+                                    ctypes.byref(h)) == MISALIGNED
+    assert "tensor 1" in coat.coat_last_error()
+    assert L.coat_adamw_step_multi(None, 1e-3, 0.9, 0.95, 1e-8, 0.1, 1, None) == INVALID
+    assert L.coat_multi_plan_destroy(None) == OK
+    assert L.coat_multi_plan_info(None, None, None) == INVALID
+
+
+def test_binding_raises_without_fallback():
+    with pytest.raises(coat.CoatError) as ei:
+        coat._check(step(group=64))
+    assert ei.value.status == UNSUPPORTED

@@ -1,0 +1,125 @@
+"""GPU parity of the FP8 element codec and the per-group quantiser (1x128 and
+128x128, expansion on/off) against the CPU oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import fp8_optimizer_state_b200 as coat
+import synth
+from tests.parity import compare_codes, rel_err, K_RTOL, SCALE_RTOL, FLIP_FRACTION
+
+pytestmark = pytest.mark.gpu
+E4M3, E5M2 = 0, 1
+TORCH_DT = {E4M3: torch.float8_e4m3fn, E5M2: torch.float8_e5m2}
+
+
+def encoder_probe_values():
+    """Every FP32 exponent; for each, all 2^12 combinations of the top 12 mantissa
+    bits with the low 11 bits at 0, 1 and all-ones -- which covers, for both
+    formats, every rounding midpoint and its two FP32 neighbours -- both signs,
+    plus NaN and infinities."""
+    e = np.arange(256, dtype=np.uint32)[:, None, None]
+    top = np.arange(4096, dtype=np.uint32)[None, :, None]
+    low = np.array([0, 1, 0x7FF], dtype=np.uint32)[None, None, :]
+    bits = ((e << np.uint32(23)) | (top << np.uint32(11)) | low).ravel()
+    bits = np.concatenate([bits, bits | np.uint32(0x80000000)])
+    return bits.view(np.float32)
+
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+def test_encoder_bit_identical_to_oracle(orc, fmt):
+    y = encoder_probe_values()
+    q = torch.empty(y.size, dtype=torch.uint8, device="cuda")
+    coat.coat_fp8_encode(torch.from_numpy(y).cuda(), fmt, q)
+    got = q.cpu().numpy()
+    ref = orc.fp8_encode_array(fmt, y)
+    nan = np.isnan(y)
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert np.all(got[nan] & 0x7F == 0x7F)
+
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+def test_encoder_matches_hardware_cast_in_range(fmt):
+    top = 448.0 if fmt == E4M3 else 57344.0
+    g = torch.Generator(device="cuda").manual_seed(5)
+    y = (torch.rand(1 << 22, device="cuda", generator=g) * 2 - 1) * top
+    y[: 1 << 20] *= 1e-3
+    q = torch.empty(y.numel(), dtype=torch.uint8, device="cuda")
+    coat.coat_fp8_encode(y, fmt, q)
+    ref = y.to(TORCH_DT[fmt]).view(torch.uint8).clone()
+    ref[ref == 0x80] = 0
+    assert torch.equal(q, ref)
+
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+def test_decoder_all_codes(orc, fmt):
+    q = torch.arange(256, dtype=torch.int32).to(torch.uint8).cuda()
+    out = torch.empty(256, dtype=torch.float32, device="cuda")
+    coat.coat_fp8_decode(q, fmt, out)
+    got = out.cpu().numpy().astype(np.float64)
+    ref = orc.fp8_decode_table(fmt)
+    assert np.all((got == ref) | (np.isnan(got) & np.isnan(ref)))
+
+
+def _check_quant(gq, gs, gk, oq, os_, ok_):
+    assert rel_err(gk, ok_).max() <= K_RTOL
+    assert rel_err(gs, os_).max() <= SCALE_RTOL
+    diff, maxd = compare_codes(gq, oq)
+    assert maxd <= 1
+    assert diff.sum() <= max(1, FLIP_FRACTION * diff.size), int(diff.sum())
+
+
+CASES = [(1, 128, 200, 1000), (1, 128, 64, 4096), (128, 128, 300, 260), (128, 128, 256, 384)]
+
+
+@pytest.mark.parametrize("gr,gc,rows,cols", CASES)
+@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+@pytest.mark.parametrize("expand", [False, True])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_group_quantize_vs_oracle(orc, gr, gc, rows, cols, fmt, expand, dtype):
+    n = rows * cols
+    if dtype == "bf16":
+        bits = synth.activations_bits(0, rows + cols, 0, n).reshape(rows, cols)
+        xh = synth.bf16_bits_to_f32(bits)
+        xd = torch.from_numpy(bits.view(np.int16)).cuda()
+    else:
+        xh = (synth.master(0, rows + cols, 0, n) * np.float32(50.0)).reshape(rows, cols)
+        xd = torch.from_numpy(xh).cuda()
+    nbr, nbc = -(-rows // gr), -(-cols // gc)
+    ldq = -(-cols // 16) * 16
+    q = torch.zeros((rows, ldq), dtype=torch.uint8, device="cuda")
+    s = torch.zeros((nbr, nbc), dtype=torch.float32, device="cuda")
+    k = torch.zeros((nbr, nbc), dtype=torch.float32, device="cuda")
+    coat.coat_group_quantize(xd, gr, gc, expand, fmt, q, s, k)
+    oq, os_, ok_ = orc.group_quantize(xh.astype(np.float64), gr, gc, expand, fmt)
+    torch.cuda.synchronize()
+    _check_quant(q.cpu().numpy()[:, :cols], s.cpu().numpy(), k.cpu().numpy(), oq, os_, ok_)
+    assert not q.cpu().numpy()[:, cols:].any()     # nothing written past cols
+
+
+@pytest.mark.parametrize("gr", [1, 128])
+@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+def test_group_dequantize_vs_oracle(orc, gr, fmt):
+    rows, cols = 256, 640
+    rng = np.random.default_rng(30 + gr + fmt)
+    top = 0x7E if fmt == E4M3 else 0x7B
+    q = rng.integers(0, top + 1, (rows, cols)).astype(np.uint8) | \
+        rng.choice([0, 0x80], (rows, cols)).astype(np.uint8)
+    nbr, nbc = -(-rows // gr), -(-cols // 128)
+    k = rng.uniform(1.0, 16.0, (nbr, nbc)).astype(np.float32)
+    k[0, 0] = 1.0
+    s = np.exp(rng.uniform(-25, 0, (nbr, nbc))).astype(np.float32)
+    ref = orc.group_dequantize(q, s, k, gr, 128, fmt)
+    out = torch.empty((rows, cols), dtype=torch.float32, device="cuda")
+    coat.coat_group_dequantize(torch.from_numpy(q).cuda(), torch.from_numpy(s).cuda(),
+                               torch.from_numpy(k).cuda(), gr, 128, fmt, out)
+    got = out.cpu().numpy().astype(np.float64)
+    # x = s * 2^(log2|q| / k): FP32 exponent arithmetic and MUFU ex2 give a few
+    # 1e-7 relative (the argument reaches |log2 q| <= 16 at k = 1)
+    assert np.all(np.sign(got) == np.sign(ref))
+    assert rel_err(got[ref != 0], ref[ref != 0]).max() < 2e-6
+    outb = torch.empty((rows, cols), dtype=torch.bfloat16, device="cuda")
+    coat.coat_group_dequantize(torch.from_numpy(q).cuda(), torch.from_numpy(s).cuda(),
+                               torch.from_numpy(k).cuda(), gr, 128, fmt, outb)
+    gb = outb.float().cpu().numpy()
+    assert np.array_equal(gb, torch.from_numpy(got.astype(np.float32)).bfloat16().float().numpy())
