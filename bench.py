@@ -272,11 +272,10 @@ def run_ours(args, cfg, ws, rank, local):
     coat.coat_check_device_error()
 
     props = torch.cuda.get_device_properties(dev)
-    bus = getattr(props, "pci_bus_id", None)
-    if bus is None:
-        bus = "%08x:%02x:%02x.0" % (getattr(props, "pci_domain_id", 0), getattr(props, "pci_bus_id", 0),
-                                     getattr(props, "pci_device_id", 0))
-    sampler = ClockSampler(str(bus))
+    bus = "%08x:%02x:%02x.0" % (int(getattr(props, "pci_domain_id", 0)),
+                                int(getattr(props, "pci_bus_id", 0)),
+                                int(getattr(props, "pci_device_id", 0)))
+    sampler = ClockSampler(bus)
     sampler.start()
     time.sleep(0.3)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))

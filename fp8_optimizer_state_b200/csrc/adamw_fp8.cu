@@ -64,6 +64,7 @@ struct TileHeader {
 };
 
 struct Smem {
+  double tabd_m[256];  // log2|value(code)| of the m format in double (min-element recompute)
   float tab_m[256];
   float tab_v[256];
   uint64_t full_bar[kStages];
@@ -168,10 +169,33 @@ __device__ __forceinline__ float f4get(const float4& v, int i) {
 }
 
 // The per-lane body: everything after the loads.
+// The element of a group with the smallest nonzero |m'| usually comes from
+// cancellation between beta1*m and (1-beta1)*g, so its FP32 value carries the
+// FP32 error of the dequantised m amplified by |beta1 m| / |m'| (often 100x to
+// 1000x) -- and k depends on it through ln(max/min).  The kernel therefore
+// tracks which element is the minimum (its position is packed into the low 4
+// bits of the comparison key, at a cost of 2^-19 relative in the ordering) and
+// recomputes that one element's m' in double precision.
+__device__ __forceinline__ float recompute_m_double(const LaneIn& in, int idx,
+                                                    const StepHyper& h, const double* tabd_m) {
+  const int j = idx >> 2, i = idx & 3;
+  const uint32_t mw = j == 0 ? in.mq[0] : j == 1 ? in.mq[1] : j == 2 ? in.mq[2] : in.mq[3];
+  const uint2 gw2 = j == 0 ? in.g[0] : j == 1 ? in.g[1] : j == 2 ? in.g[2] : in.g[3];
+  const uint32_t c = (mw >> (8 * i)) & 0xFFu;
+  const uint32_t gw = (i < 2) ? gw2.x : gw2.y;
+  const float g = (i & 1) ? bf16hi(gw) : bf16lo(gw);
+  const double b1 = static_cast<double>(h.beta1);
+  double x = exp2(tabd_m[c] / static_cast<double>(in.mk)) * static_cast<double>(in.ms);
+  if (c & 0x80u) x = -x;
+  const double m1 = fma(b1, x, (1.0 - b1) * static_cast<double>(g));
+  return __double2float_rn(fabs(m1));
+}
+
 template <int FM, int FV>
 __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, int64_t gi,
                                         bool active, int slot, int l, const StepHyper& h,
-                                        const float* tab_m, const float* tab_v) {
+                                        const float* tab_m, const float* tab_v,
+                                        const double* tabd_m) {
   const int64_t base = gi * kGroup;
   // dequantisation constants of this group (stored k and root scale)
   const float invk_m = rcp_approx(in.mk), sb_m = in.ms * h.beta1;
@@ -206,7 +230,8 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
       v1[4 * j + i] = valid ? vn : 0.f;
       maxm = fmaxf(maxm, fabsf(m1[4 * j + i]));
       maxv = fmaxf(maxv, v1[4 * j + i]);
-      minm = min(minm, (__float_as_uint(m1[4 * j + i]) & 0x7FFFFFFFu) - 1u);
+      minm = min(minm, (((__float_as_uint(m1[4 * j + i]) & 0x7FFFFFFFu) - 1u) & 0xFFFFFFF0u) |
+                           static_cast<uint32_t>(4 * j + i));
       minv = min(minv, __float_as_uint(v1[4 * j + i]) - 1u);
     }
     if (active) {
@@ -226,7 +251,9 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
     }
   }
 
-  // group statistics over the 8 lanes of this group
+  // group statistics over the 8 lanes of this group; the m key carries the
+  // position (lane l, element idx) of the minimum in its low 7 bits
+  minm = (minm & ~0x70u) | (static_cast<uint32_t>(l) << 4);
 #pragma unroll
   for (int off = 1; off < 8; off <<= 1) {
     maxm = fmaxf(maxm, __shfl_xor_sync(0xFFFFFFFFu, maxm, off));
@@ -234,7 +261,13 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
     minm = min(minm, __shfl_xor_sync(0xFFFFFFFFu, minm, off));
     minv = min(minv, __shfl_xor_sync(0xFFFFFFFFu, minv, off));
   }
-  const float mum = __uint_as_float(minm + 1u), muv = __uint_as_float(minv + 1u);
+  // exact-as-FP32 min of |m'|: the owning lane recomputes it in double
+  float mum = 0.f;
+  const bool any_m = minm < 0xFFFFFF80u;
+  if (any_m && static_cast<int>((minm >> 4) & 7u) == l)
+    mum = recompute_m_double(in, static_cast<int>(minm & 15u), h, tabd_m);
+  mum = __shfl_sync(0xFFFFFFFFu, mum, (slot << 3) | static_cast<int>((minm >> 4) & 7u));
+  const float muv = __uint_as_float(minv + 1u);
   float km, srm, invMm, kv, srv, invMv;
   group_params<FM>(maxm, mum, true, km, srm, invMm);
   group_params<FV>(maxv, muv, true, kv, srv, invMv);
@@ -274,6 +307,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
   fill_log2_table<FM>(S.tab_m);
   fill_log2_table<FV>(S.tab_v);
+  for (int c = threadIdx.x; c < 256; c += blockDim.x)
+    S.tabd_m[c] = log2(static_cast<double>(fabsf(dec_value<FM>(c))));
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&S.full_bar[s], 1);
@@ -359,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       load_direct(t, gi, active, slot, l, in);
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.empty_bar[s]);
-    process<FM, FV>(in, t, gi, active, slot, l, h, S.tab_m, S.tab_v);
+    process<FM, FV>(in, t, gi, active, slot, l, h, S.tab_m, S.tab_v, S.tabd_m);
   }
 }
 

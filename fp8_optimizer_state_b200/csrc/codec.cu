@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
       uint32_t c[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        c[i] = enc_signed<FMT>(v[4 * j + i], expand_value<FMT>(v[4 * j + i], invM, k));
+        c[i] = enc_signed<FMT>(v[4 * j + i], codec_value<FMT>(v[4 * j + i], M, invM, k));
       if (valid > 0) store_codes4(q + r * ldq + c0, c, valid);
     }
     if (active && l == 0) {
@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
       uint32_t c[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        c[i] = enc_signed<FMT>(v[4 * rr + i], expand_value<FMT>(v[4 * rr + i], invM, k));
+        c[i] = enc_signed<FMT>(v[4 * rr + i], codec_value<FMT>(v[4 * rr + i], M, invM, k));
       if (valid > 0) store_codes4(q + r * ldq + c0, c, valid);
     }
     if (threadIdx.x == 0) {

@@ -312,9 +312,12 @@ int orc_group_dequantize(const uint8_t *q, int64_t ldq, const float *scale,
  * partial).  master (float) is updated in place; weight_out (bf16 bits, may
  * be NULL) receives RNE(master); grad holds bf16 bits.  m_q / v_q hold
  * ceil(n/group)*group codes (padding written 0); *_scale / *_k hold one
- * float per group.  If upd_out is not NULL it receives |lr/bc1 * m' /
- * (sqrt(v')/sqrt(bc2) + eps)| per element (the adaptive part of the update),
- * used by tests to size tolerances.  Returns 0, or -1 on bad arguments. */
+ * float per group.  If upd_out is not NULL it receives, per element, the
+ * adaptive update evaluated on the magnitudes of the two summands of m',
+ * lr/bc1 * (|b1 m| + |(1-b1) g|) / (sqrt(v')/sqrt(bc2) + eps): the size of
+ * the update before any cancellation between the old moment and the new
+ * gradient.  Tests use it to size the master-weight tolerance (it is not part
+ * of the method's result).  Returns 0, or -1 on bad arguments. */
 int orc_adamw_step(float *master, uint16_t *weight_out, const uint16_t *grad,
                    uint8_t *m_q, float *m_scale, float *m_k, uint8_t *v_q,
                    float *v_scale, float *v_k, int64_t n, int group, float lr,
@@ -352,7 +355,8 @@ int orc_adamw_step(float *master, uint16_t *weight_out, const uint16_t *grad,
             if (weight_out)
                 weight_out[i] = orc_float_to_bf16(master[i]);
             if (upd_out)
-                upd_out[i] = fabs(adapt);
+                upd_out[i] = (dlr / bc1) * (fabs(b1 * m) + fabs((1.0 - b1) * gi)) /
+                             (sqrt(v1) / sqrt(bc2) + deps);
             mb[j] = m1;
             vb[j] = v1;
         }

@@ -41,7 +41,14 @@ def ragged(num=10000, lo=64, hi=1 << 20, seed=0):
     return [("t%d" % i, int(s)) for i, s in enumerate(sizes)]
 
 
+def flat(n):
+    return lambda: [("flat", n)]
+
+
 CONFIGS = {
+    "flat-256m": dict(shapes=flat(1 << 28), fmt_m=0, fmt_v=1, steps=3,
+                      workload="One flat tensor of 268,435,456 params, E4M3 m + E5M2 v "
+                               "(profiling case: 2.7 GB, larger than L2)"),
     "tiny": dict(shapes=tiny, fmt_m=0, fmt_v=0, steps=10,
                  workload="Tiny: one flat tensor of 1,048,576, E4M3 m + E4M3 v"),
     "llama2-7b": dict(shapes=llama2_7b, fmt_m=0, fmt_v=1, steps=3,

@@ -78,13 +78,17 @@ CASES = [(1, 128, 200, 1000), (1, 128, 64, 4096), (128, 128, 300, 260), (128, 12
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_group_quantize_vs_oracle(orc, gr, gc, rows, cols, fmt, expand, dtype):
     n = rows * cols
+    ldx = -(-cols // 8) * 8          # rows padded to 16 bytes (the ABI's stride rule)
     if dtype == "bf16":
         bits = synth.activations_bits(0, rows + cols, 0, n).reshape(rows, cols)
         xh = synth.bf16_bits_to_f32(bits)
-        xd = torch.from_numpy(bits.view(np.int16)).cuda()
+        xd = torch.zeros((rows, ldx), dtype=torch.int16, device="cuda")
+        xd[:, :cols] = torch.from_numpy(bits.view(np.int16)).cuda()
     else:
         xh = (synth.master(0, rows + cols, 0, n) * np.float32(50.0)).reshape(rows, cols)
-        xd = torch.from_numpy(xh).cuda()
+        xd = torch.zeros((rows, ldx), dtype=torch.float32, device="cuda")
+        xd[:, :cols] = torch.from_numpy(xh).cuda()
+    xd = xd[:, :cols]
     nbr, nbc = -(-rows // gr), -(-cols // gc)
     ldq = -(-cols // 16) * 16
     q = torch.zeros((rows, ldq), dtype=torch.uint8, device="cuda")
