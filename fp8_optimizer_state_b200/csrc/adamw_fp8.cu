@@ -13,7 +13,9 @@
 //  * one producer thread streams whole tiles (master, grad, both code arrays,
 //    the four metadata arrays: 33,280 B) into a 3-stage shared-memory ring
 //    with 1-D cp.async.bulk copies completing on an mbarrier, so that bytes in
-//    flight do not depend on registers;
+//    flight do not depend on registers.  It keeps the current tensor's
+//    descriptor in registers, prefetches the next tile's tensor index, and
+//    writes the descriptor into the stage header for the consumers;
 //  * 8 consumer warps; each warp owns 4 groups of a tile, 8 lanes per group,
 //    16 elements per lane in 4 chunks of 4 contiguous elements (chunk order
 //    rotated per group to keep shared-memory reads conflict-free); group
@@ -21,10 +23,10 @@
 //  * a consumer copies its slice of the stage into registers and releases the
 //    stage before computing; results go straight to HBM with coalesced
 //    16/8/4-byte stores (every warp store instruction writes whole sectors);
-//  * tiles that are not entirely valid (a tensor's last tile when n is not a
-//    multiple of 4096) take a direct path: the consumers load from global
-//    memory with bounds checks; padding elements count as zero and their
-//    codes are written 0;
+//  * fully valid tiles run a specialised body with no bounds logic; a
+//    tensor's last tile, when not fully valid, takes a direct path: the
+//    consumers load from global memory with bounds checks, padding elements
+//    count as zero and their codes are written 0;
 //  * every mbarrier wait is bounded (about a second); on timeout the kernel
 //    sets a device error bit and returns.
 #include <cstdint>
@@ -56,39 +58,40 @@ constexpr uint32_t kOffVk = kOffVs + kTileGroups * 4;
 constexpr uint32_t kStageBytes = kOffVk + kTileGroups * 4;   // 33280
 
 struct TileHeader {
+  TensorArgs t;     // descriptor of the tile's tensor
   int64_t g0;       // first group of the tile within its tensor
-  int32_t tensor;   // tensor index (multi-tensor launch)
   int32_t ngroups;  // groups of this tile that exist
   int32_t full;     // 1: all 4096 elements valid and staged in shared memory
-  int32_t pad;
 };
 
 struct Smem {
-  double tabd_m[256];  // log2|value(code)| of the m format in double (min-element recompute)
-  float tab_m[256];
-  float tab_v[256];
+  double tabd_m[256];  // log2|value(code)| of the m format, double (min recompute)
+  double exp2_16[16];  // 2^(j/16), double
+  float tab_m[256];    // log2|value(code)| of the m format
+  float tab_v[256];    // log2|value(code)| of the v format
   uint64_t full_bar[kStages];
   uint64_t empty_bar[kStages];
   TileHeader hdr[kStages];
 };
-constexpr size_t kSmemBytes = ((sizeof(Smem) + 127) / 128) * 128 + size_t(kStages) * kStageBytes;
+constexpr size_t kSmemHead = ((sizeof(Smem) + 127) / 128) * 128;
+constexpr size_t kSmemBytes = kSmemHead + size_t(kStages) * kStageBytes;
 
 // Tile -> tensor lookup.  Single-tensor launches use one descriptor passed by
 // value; multi-tensor launches use the plan's device tables.
 struct SingleTensor {
+  static constexpr bool kSingle = true;
   TensorArgs t;
   __device__ __forceinline__ int64_t tiles() const { return t.tiles; }
   __device__ __forceinline__ int32_t tensor_of(int64_t) const { return 0; }
-  __device__ __forceinline__ int64_t first_tile(int32_t) const { return 0; }
-  __device__ __forceinline__ const TensorArgs& get(int32_t) const { return t; }
+  __device__ __forceinline__ TensorArgs get(int32_t) const { return t; }
 };
 struct MultiTensor {
+  static constexpr bool kSingle = false;
   const TensorArgs* descs;
   const int32_t* tile_tensor;
   int64_t total_tiles;
   __device__ __forceinline__ int64_t tiles() const { return total_tiles; }
-  __device__ __forceinline__ int32_t tensor_of(int64_t tile) const { return tile_tensor[tile]; }
-  __device__ __forceinline__ int64_t first_tile(int32_t i) const { return descs[i].tile_begin; }
+  __device__ __forceinline__ int32_t tensor_of(int64_t tile) const { return __ldg(tile_tensor + tile); }
   __device__ __forceinline__ TensorArgs get(int32_t i) const { return descs[i]; }
 };
 
@@ -168,34 +171,63 @@ __device__ __forceinline__ float f4get(const float4& v, int i) {
   return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-// The per-lane body: everything after the loads.
+// 2^t in double for |t| < 1000, table-driven (P. T. P. Tang, "Table-driven
+// implementation of the exponential function", ACM TOMS 15(2), 1989):
+// t = (16n' + j)/16 + r with |r| <= 1/32, 2^t = 2^n' * 2^(j/16) * e^(r ln 2),
+// the last factor by its Taylor series to the z^5 term (|z| <= ln2/32, so the
+// truncation is below 2e-13 relative).
+__device__ __forceinline__ double exp2_table(double t, const double* exp2_16) {
+  const double s = t * 16.0;
+  const double n = rint(s);
+  const double z = (s - n) * 0.043321698784996581;  // (s - n)/16 * ln 2
+  const int ni = static_cast<int>(n);
+  double p = fma(z, 1.0 / 120.0, 1.0 / 24.0);
+  p = fma(p, z, 1.0 / 6.0);
+  p = fma(p, z, 0.5);
+  p = fma(p, z, 1.0);
+  p = fma(p, z, 1.0);
+  const double scale = __longlong_as_double(static_cast<long long>((ni >> 4) + 1023) << 52);
+  return exp2_16[ni & 15] * p * scale;
+}
+
 // The element of a group with the smallest nonzero |m'| usually comes from
 // cancellation between beta1*m and (1-beta1)*g, so its FP32 value carries the
-// FP32 error of the dequantised m amplified by |beta1 m| / |m'| (often 100x to
-// 1000x) -- and k depends on it through ln(max/min).  The kernel therefore
-// tracks which element is the minimum (its position is packed into the low 4
-// bits of the comparison key, at a cost of 2^-19 relative in the ordering) and
-// recomputes that one element's m' in double precision.
+// FP32 dequantisation error amplified by |beta1 m| / |m'| (often 100x-1000x),
+// and k depends on it through ln(max/min).  The kernel keeps the two smallest
+// candidates (their positions packed into the low bits of the comparison keys,
+// at a cost of 2^-18 relative in the ordering) and recomputes both in double
+// precision: dequantisation, then m' = beta1 m + (1 - beta1) g.
 __device__ __forceinline__ float recompute_m_double(const LaneIn& in, int idx,
-                                                    const StepHyper& h, const double* tabd_m) {
+                                                    const StepHyper& h, const double* tabd_m,
+                                                    const double* exp2_16) {
   const int j = idx >> 2, i = idx & 3;
   const uint32_t mw = j == 0 ? in.mq[0] : j == 1 ? in.mq[1] : j == 2 ? in.mq[2] : in.mq[3];
   const uint2 gw2 = j == 0 ? in.g[0] : j == 1 ? in.g[1] : j == 2 ? in.g[2] : in.g[3];
   const uint32_t c = (mw >> (8 * i)) & 0xFFu;
   const uint32_t gw = (i < 2) ? gw2.x : gw2.y;
   const float g = (i & 1) ? bf16hi(gw) : bf16lo(gw);
-  const double b1 = static_cast<double>(h.beta1);
-  double x = exp2(tabd_m[c] / static_cast<double>(in.mk)) * static_cast<double>(in.ms);
+  const double k = static_cast<double>(in.mk);
+  const double r0 = static_cast<double>(rcp_approx(in.mk));
+  const double invk = r0 * fma(-k, r0, 2.0);   // one Newton step: ~1e-14 relative
+  double x = exp2_table(tabd_m[c] * invk, exp2_16) * static_cast<double>(in.ms);
   if (c & 0x80u) x = -x;
+  const double b1 = static_cast<double>(h.beta1);
   const double m1 = fma(b1, x, (1.0 - b1) * static_cast<double>(g));
   return __double2float_rn(fabs(m1));
 }
 
-template <int FM, int FV>
+// Comparison key of |x|: FP32 bits without the sign, minus one (so that zero
+// becomes the largest key), low 4 bits replaced by the element index.
+__device__ __forceinline__ uint32_t min_key(float x, int idx) {
+  return (((__float_as_uint(x) & 0x7FFFFFFFu) - 1u) & 0xFFFFFFF0u) | static_cast<uint32_t>(idx);
+}
+
+// The per-lane body: everything after the loads.  FULL: every element of the
+// tile is valid (no bounds logic).
+template <int FM, int FV, bool FULL>
 __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, int64_t gi,
                                         bool active, int slot, int l, const StepHyper& h,
-                                        const float* tab_m, const float* tab_v,
-                                        const double* tabd_m) {
+                                        const Smem& S) {
   const int64_t base = gi * kGroup;
   // dequantisation constants of this group (stored k and root scale)
   const float invk_m = rcp_approx(in.mk), sb_m = in.ms * h.beta1;
@@ -203,7 +235,7 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
 
   float m1[16], v1[16];
   float maxm = 0.f, maxv = 0.f;
-  uint32_t minm = 0xFFFFFFFFu, minv = 0xFFFFFFFFu;
+  uint32_t minm1 = 0xFFFFFFFFu, minm2 = 0xFFFFFFFFu, minv = 0xFFFFFFFFu;
 
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -213,60 +245,72 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
     for (int i = 0; i < 4; ++i) {
       const uint32_t gw = (i < 2) ? in.g[j].x : in.g[j].y;
       const float g = (i & 1) ? bf16hi(gw) : bf16lo(gw);
-      const uint32_t cm = (in.mq[j] >> (8 * i)) & 0xFFu;
-      const uint32_t cv = (in.vq[j] >> (8 * i)) & 0xFFu;
+      const uint32_t cm = __byte_perm(in.mq[j], 0u, 0x4440u + i);
+      const uint32_t cv = __byte_perm(in.vq[j], 0u, 0x4440u + i);
       // beta1 * m and beta2 * v, dequantised: s_r * beta * 2^(log2|q| / k)
-      float bm = ex2_approx(tab_m[cm] * invk_m) * sb_m;
-      bm = __uint_as_float(__float_as_uint(bm) ^ ((cm & 0x80u) << 24));
-      const float bv = ex2_approx(tab_v[cv] * invk_v) * sb_v;
-      const float mn = __fmaf_rn(h.omb1, g, bm);
-      const float vn = __fmaf_rn(h.omb2 * g, g, bv);
+      float bm = ex2_approx(S.tab_m[cm] * invk_m) * sb_m;
+      bm = __uint_as_float(__float_as_uint(bm) ^ ((in.mq[j] << (24 - 8 * i)) & 0x80000000u));
+      const float bv = ex2_approx(S.tab_v[cv] * invk_v) * sb_v;
+      float mn = __fmaf_rn(h.omb1, g, bm);
+      float vn = __fmaf_rn(h.omb2 * g, g, bv);
       const float p = f4get(in.p[j], i);
       const float denom = __fmaf_rn(sqrt_approx(vn), h.rsbc2, h.eps);
       const float upd = (h.step_size * mn) * rcp_approx(denom);
       pn[i] = p + __fmaf_rn(-p, h.lrwd, -upd);
-      const bool valid = active && (e + i < t.n);
-      m1[4 * j + i] = valid ? mn : 0.f;
-      v1[4 * j + i] = valid ? vn : 0.f;
-      maxm = fmaxf(maxm, fabsf(m1[4 * j + i]));
-      maxv = fmaxf(maxv, v1[4 * j + i]);
-      minm = min(minm, (((__float_as_uint(m1[4 * j + i]) & 0x7FFFFFFFu) - 1u) & 0xFFFFFFF0u) |
-                           static_cast<uint32_t>(4 * j + i));
-      minv = min(minv, __float_as_uint(v1[4 * j + i]) - 1u);
-    }
-    if (active) {
-      if (e + 4 <= t.n) {
-        *reinterpret_cast<float4*>(t.master + e) = make_float4(pn[0], pn[1], pn[2], pn[3]);
-        if (t.wout)
-          *reinterpret_cast<uint2*>(t.wout + e) =
-              make_uint2(pack_bf16x2(pn[0], pn[1]), pack_bf16x2(pn[2], pn[3]));
-      } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (e + i < t.n) {
-            t.master[e + i] = pn[i];
-            if (t.wout) t.wout[e + i] = static_cast<uint16_t>(pack_bf16x2(pn[i], 0.f));
-          }
+      if (!FULL) {
+        const bool valid = active && (e + i < t.n);
+        mn = valid ? mn : 0.f;
+        vn = valid ? vn : 0.f;
       }
+      m1[4 * j + i] = mn;
+      v1[4 * j + i] = vn;
+      maxm = fmaxf(maxm, fabsf(mn));
+      maxv = fmaxf(maxv, vn);
+      const uint32_t key = min_key(mn, 4 * j + i);
+      minm2 = min(minm2, max(minm1, key));
+      minm1 = min(minm1, key);
+      minv = min(minv, __float_as_uint(vn) - 1u);
+    }
+    if (FULL || (active && e + 4 <= t.n)) {
+      *reinterpret_cast<float4*>(t.master + e) = make_float4(pn[0], pn[1], pn[2], pn[3]);
+      if (t.wout)
+        *reinterpret_cast<uint2*>(t.wout + e) =
+            make_uint2(pack_bf16x2(pn[0], pn[1]), pack_bf16x2(pn[2], pn[3]));
+    } else if (active) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (e + i < t.n) {
+          t.master[e + i] = pn[i];
+          if (t.wout) t.wout[e + i] = static_cast<uint16_t>(pack_bf16x2(pn[i], 0.f));
+        }
     }
   }
 
-  // group statistics over the 8 lanes of this group; the m key carries the
-  // position (lane l, element idx) of the minimum in its low 7 bits
-  minm = (minm & ~0x70u) | (static_cast<uint32_t>(l) << 4);
+  // group statistics over the 8 lanes of this group.  The m keys carry the
+  // position (lane l, element index) of the two smallest |m'| in their low 7
+  // bits; merging two sorted pairs keeps the two smallest of the union.
+  minm1 = (minm1 & ~0x70u) | (static_cast<uint32_t>(l) << 4);
+  minm2 = (minm2 & ~0x70u) | (static_cast<uint32_t>(l) << 4);
 #pragma unroll
   for (int off = 1; off < 8; off <<= 1) {
     maxm = fmaxf(maxm, __shfl_xor_sync(0xFFFFFFFFu, maxm, off));
     maxv = fmaxf(maxv, __shfl_xor_sync(0xFFFFFFFFu, maxv, off));
-    minm = min(minm, __shfl_xor_sync(0xFFFFFFFFu, minm, off));
     minv = min(minv, __shfl_xor_sync(0xFFFFFFFFu, minv, off));
+    const uint32_t o1 = __shfl_xor_sync(0xFFFFFFFFu, minm1, off);
+    const uint32_t o2 = __shfl_xor_sync(0xFFFFFFFFu, minm2, off);
+    minm2 = min(max(minm1, o1), min(minm2, o2));
+    minm1 = min(minm1, o1);
   }
-  // exact-as-FP32 min of |m'|: the owning lane recomputes it in double
-  float mum = 0.f;
-  const bool any_m = minm < 0xFFFFFF80u;
-  if (any_m && static_cast<int>((minm >> 4) & 7u) == l)
-    mum = recompute_m_double(in, static_cast<int>(minm & 15u), h, tabd_m);
-  mum = __shfl_sync(0xFFFFFFFFu, mum, (slot << 3) | static_cast<int>((minm >> 4) & 7u));
+  // min |m'| exact as FP32: the lanes owning the two candidates recompute them
+  float mum = __int_as_float(0x7F800000);
+  if (minm1 < 0xFFFFFF80u && static_cast<int>((minm1 >> 4) & 7u) == l)
+    mum = recompute_m_double(in, static_cast<int>(minm1 & 15u), h, S.tabd_m, S.exp2_16);
+  if (minm2 < 0xFFFFFF80u && static_cast<int>((minm2 >> 4) & 7u) == l)
+    mum = fminf(mum, recompute_m_double(in, static_cast<int>(minm2 & 15u), h, S.tabd_m,
+                                        S.exp2_16));
+#pragma unroll
+  for (int off = 1; off < 8; off <<= 1) mum = fminf(mum, __shfl_xor_sync(0xFFFFFFFFu, mum, off));
+  if (!(minm1 < 0xFFFFFF80u)) mum = 0.f;   // no nonzero element
   const float muv = __uint_as_float(minv + 1u);
   float km, srm, invMm, kv, srv, invMv;
   group_params<FM>(maxm, mum, true, km, srm, invMm);
@@ -281,16 +325,16 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
     for (int i = 0; i < 4; ++i) {
       const float xm = m1[4 * j + i], xv = v1[4 * j + i];
       cmw[i] = enc_signed<FM>(xm, expand_value<FM>(xm, invMm, km));
-      cvw[i] = enc_signed<FV>(xv, expand_value<FV>(xv, invMv, kv));
+      cvw[i] = enc_mag<FV>(expand_value<FV>(xv, invMv, kv));
     }
-    if (active) {
+    if (FULL || active) {
       *reinterpret_cast<uint32_t*>(t.mq + e) =
           __byte_perm(__byte_perm(cmw[0], cmw[1], 0x0040), __byte_perm(cmw[2], cmw[3], 0x0040), 0x5410);
       *reinterpret_cast<uint32_t*>(t.vq + e) =
           __byte_perm(__byte_perm(cvw[0], cvw[1], 0x0040), __byte_perm(cvw[2], cvw[3], 0x0040), 0x5410);
     }
   }
-  if (active && l == 0) {
+  if ((FULL || active) && l == 0) {
     t.ms[gi] = srm;
     t.mk[gi] = km;
     t.vs[gi] = srv;
@@ -299,16 +343,17 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
 }
 
 template <int FM, int FV, class Map>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+__global__ void __maxnreg__(112)
     adamw_fp8_kernel(const Map map, const StepHyper h, unsigned* err) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>(smem_raw);
-  uint8_t* stages = smem_raw + ((sizeof(Smem) + 127) / 128) * 128;
+  uint8_t* stages = smem_raw + kSmemHead;
 
   fill_log2_table<FM>(S.tab_m);
   fill_log2_table<FV>(S.tab_v);
   for (int c = threadIdx.x; c < 256; c += blockDim.x)
     S.tabd_m[c] = log2(static_cast<double>(fabsf(dec_value<FM>(c))));
+  if (threadIdx.x < 16) S.exp2_16[threadIdx.x] = exp2(static_cast<double>(threadIdx.x) / 16.0);
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&S.full_bar[s], 1);
@@ -324,8 +369,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   if (warp == kConsumerWarps) {
     // ---------------- producer ----------------
     if (lane != 0) return;
+    int32_t cur = -1;
+    TensorArgs ct{};
+    int32_t next_ti = blockIdx.x < ntiles ? map.tensor_of(blockIdx.x) : 0;
     int64_t it = 0;
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+      const int32_t ti = next_ti;
+      if (tile + gridDim.x < ntiles) next_ti = map.tensor_of(tile + gridDim.x);  // prefetch
+      if (ti != cur) {
+        ct = map.get(ti);
+        cur = ti;
+      }
       const int s = static_cast<int>(it % kStages);
       const uint32_t use = static_cast<uint32_t>(it / kStages);
       if (use > 0 && !mbar_wait(&S.empty_bar[s], (use - 1) & 1u, kWaitBudgetCycles)) {
@@ -341,30 +395,27 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         }
         return;
       }
-      const int32_t ti = map.tensor_of(tile);
-      const TensorArgs t = map.get(ti);
-      const int64_t local = tile - map.first_tile(ti);
-      const int64_t g0 = local * kTileGroups;
-      const int64_t groups = (t.n + kGroup - 1) / kGroup;
+      const int64_t g0 = (tile - ct.tile_begin) * kTileGroups;
+      const int64_t groups = (ct.n + kGroup - 1) / kGroup;
       const int64_t ng = (groups - g0) < kTileGroups ? (groups - g0) : int64_t(kTileGroups);
       const int64_t e0 = g0 * kGroup;
-      const bool full = (e0 + kTileElems <= t.n);
+      const bool full = (e0 + kTileElems <= ct.n);
       TileHeader& hd = S.hdr[s];
+      if (!Map::kSingle) hd.t = ct;
       hd.g0 = g0;
-      hd.tensor = ti;
       hd.ngroups = static_cast<int32_t>(ng);
       hd.full = full ? 1 : 0;
       if (full) {
         uint8_t* st = stages + size_t(s) * kStageBytes;
         mbar_arrive_expect_tx(&S.full_bar[s], kStageBytes);
-        bulk_g2s(st + kOffMaster, t.master + e0, kTileElems * 4, &S.full_bar[s]);
-        bulk_g2s(st + kOffGrad, t.grad + e0, kTileElems * 2, &S.full_bar[s]);
-        bulk_g2s(st + kOffMq, t.mq + e0, kTileElems, &S.full_bar[s]);
-        bulk_g2s(st + kOffVq, t.vq + e0, kTileElems, &S.full_bar[s]);
-        bulk_g2s(st + kOffMs, t.ms + g0, kTileGroups * 4, &S.full_bar[s]);
-        bulk_g2s(st + kOffMk, t.mk + g0, kTileGroups * 4, &S.full_bar[s]);
-        bulk_g2s(st + kOffVs, t.vs + g0, kTileGroups * 4, &S.full_bar[s]);
-        bulk_g2s(st + kOffVk, t.vk + g0, kTileGroups * 4, &S.full_bar[s]);
+        bulk_g2s(st + kOffMaster, ct.master + e0, kTileElems * 4, &S.full_bar[s]);
+        bulk_g2s(st + kOffGrad, ct.grad + e0, kTileElems * 2, &S.full_bar[s]);
+        bulk_g2s(st + kOffMq, ct.mq + e0, kTileElems, &S.full_bar[s]);
+        bulk_g2s(st + kOffVq, ct.vq + e0, kTileElems, &S.full_bar[s]);
+        bulk_g2s(st + kOffMs, ct.ms + g0, kTileGroups * 4, &S.full_bar[s]);
+        bulk_g2s(st + kOffMk, ct.mk + g0, kTileGroups * 4, &S.full_bar[s]);
+        bulk_g2s(st + kOffVs, ct.vs + g0, kTileGroups * 4, &S.full_bar[s]);
+        bulk_g2s(st + kOffVk, ct.vk + g0, kTileGroups * 4, &S.full_bar[s]);
       } else {
         mbar_arrive(&S.full_bar[s]);
       }
@@ -383,18 +434,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       atomicOr(err, kErrTimeoutConsumer);
       return;
     }
-    const TileHeader hd = S.hdr[s];
-    const TensorArgs t = map.get(hd.tensor);
-    const bool active = lg < hd.ngroups;
+    const TileHeader& hd = S.hdr[s];
+    const TensorArgs t = Map::kSingle ? map.get(0) : hd.t;
     const int64_t gi = hd.g0 + lg;
+    const bool full = hd.full != 0;
+    const bool active = lg < hd.ngroups;
     LaneIn in;
-    if (hd.full)
+    if (full)
       load_from_stage(stages + size_t(s) * kStageBytes, lg, slot, l, in);
     else
       load_direct(t, gi, active, slot, l, in);
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.empty_bar[s]);
-    process<FM, FV>(in, t, gi, active, slot, l, h, S.tab_m, S.tab_v, S.tabd_m);
+    if (full)
+      process<FM, FV, true>(in, t, gi, true, slot, l, h, S);
+    else
+      process<FM, FV, false>(in, t, gi, active, slot, l, h, S);
   }
 }
 

@@ -35,6 +35,7 @@ import numpy as np
 
 # stream ids (Philox key word 1)
 MASTER, GRAD, MSTATE, VSTATE, GSCALE, ACT, ACT_OUTLIER, WEIGHT = 1, 2, 3, 4, 5, 6, 7, 8
+MCODE, VCODE, GSTATE = 9, 10, 11
 
 _PHILOX_M0 = np.uint64(0xD2511F53)
 _PHILOX_M1 = np.uint64(0xCD9E8D57)
@@ -168,6 +169,46 @@ def weight_bits(seed, tensor, start, count):
 
 
 # ----------------------------------------------------------------------------
+# Stored-state inputs: FP8 codes and per-group (k, scale) drawn directly, so
+# that two implementations can start a step from bit-identical states.  Codes
+# are uniform over the magnitudes an expanded group occupies (E4M3 0x01-0x7E,
+# i.e. 2^-9..448; E5M2 0x34-0x7B, i.e. 0.25..57344), m with a random sign.
+# k_m in [1.5, 2.2) (a group span of ~200..5000), root scale s_m = s_g *
+# [0.02, 0.06) (largest |m| ~ s_g); k_v in [4, 8) (span ~5..22), s_v = s_g^2 *
+# [0.1, 0.3).  `step` selects an independent draw per step.
+# ----------------------------------------------------------------------------
+CODE_RANGE = {0: (0x01, 0x7E), 1: (0x34, 0x7B)}
+
+
+def _unit24(u):
+    """[0, 1) FP32 from the top 24 bits (exact)."""
+    return (u >> np.uint32(8)).astype(np.float32) * np.float32(2.0 ** -24)
+
+
+def state_codes(seed, tensor, step, start, count, fmt, signed):
+    lo, hi = CODE_RANGE[fmt]
+    u = _draw(seed, MCODE if signed else VCODE, _idx(start, count), tensor, step)
+    mag = (np.uint32(lo) + u[0] % np.uint32(hi - lo + 1)).astype(np.uint8)
+    if signed:
+        mag = mag | np.where((u[1] >> np.uint32(31)) != 0, 0x80, 0).astype(np.uint8)
+    return mag
+
+
+def state_groups(seed, tensor, step, gstart, gcount):
+    """(k_m, s_m, k_v, s_v) float32 arrays for groups gstart.. of a tensor."""
+    u = _draw(seed, GSTATE, _idx(gstart, gcount), tensor, step)
+    sg = group_scale(seed, tensor, gstart, gcount)
+    f = np.float32
+    k_m = (f(0.7) * _unit24(u[0])).astype(np.float32) + f(1.5)
+    s_m = sg * ((f(0.04) * _unit24(u[1])).astype(np.float32) + f(0.02))
+    k_v = (f(4.0) * _unit24(u[2])).astype(np.float32) + f(4.0)
+    sg2 = (sg * sg).astype(np.float32)
+    s_v = sg2 * ((f(0.2) * _unit24(u[3])).astype(np.float32) + f(0.1))
+    return (k_m.astype(np.float32), s_m.astype(np.float32), k_v.astype(np.float32),
+            s_v.astype(np.float32))
+
+
+# ----------------------------------------------------------------------------
 # Device generator (CUDA, csrc/synth.cu) -- same numbers, written into
 # caller-owned device buffers.
 # ----------------------------------------------------------------------------
@@ -191,6 +232,10 @@ def device_lib():
             f.argtypes = [vp, i64, u32, u32, i64, vp]
         L.synth_grad.restype = ctypes.c_int
         L.synth_grad.argtypes = [vp, i64, u32, u32, u32, i64, vp]
+        L.synth_state_codes.restype = ctypes.c_int
+        L.synth_state_codes.argtypes = [vp, i64, u32, u32, u32, i64, ctypes.c_int, ctypes.c_int, vp]
+        L.synth_state_groups.restype = ctypes.c_int
+        L.synth_state_groups.argtypes = [vp, vp, vp, vp, i64, u32, u32, u32, i64, vp]
         _dlib = L
     return _dlib
 
@@ -237,3 +282,17 @@ def device_activations(out, seed, tensor, start=0, stream=None):
 def device_weight(out, seed, tensor, start=0, stream=None):
     _check(device_lib().synth_weight(out.data_ptr(), out.numel(), seed, tensor, start,
                                      _stream_ptr(stream)), "synth_weight")
+
+
+def device_state_codes(out, seed, tensor, step, fmt, signed, start=0, stream=None):
+    """Fill a uint8 CUDA tensor with state_codes(...)."""
+    _check(device_lib().synth_state_codes(out.data_ptr(), out.numel(), seed, tensor, step, start,
+                                          fmt, int(bool(signed)), _stream_ptr(stream)),
+           "synth_state_codes")
+
+
+def device_state_groups(k_m, s_m, k_v, s_v, seed, tensor, step, gstart=0, stream=None):
+    """Fill four float32 CUDA tensors (one entry per group) with state_groups(...)."""
+    _check(device_lib().synth_state_groups(k_m.data_ptr(), s_m.data_ptr(), k_v.data_ptr(),
+                                           s_v.data_ptr(), k_m.numel(), seed, tensor, step, gstart,
+                                           _stream_ptr(stream)), "synth_state_groups")

@@ -10,7 +10,7 @@
 namespace {
 
 enum : uint32_t { MASTER = 1, GRAD = 2, MSTATE = 3, VSTATE = 4, GSCALE = 5, ACT = 6,
-                  ACT_OUTLIER = 7, WEIGHT = 8 };
+                  ACT_OUTLIER = 7, WEIGHT = 8, MCODE = 9, VCODE = 10, GSTATE = 11 };
 
 constexpr double kIH4Scale = 1.7320508075688772 / 4294967296.0;  // sqrt(3)/2^32
 constexpr int64_t kIH4Centre = (int64_t(1) << 33) - 2;
@@ -56,9 +56,17 @@ __device__ __forceinline__ uint16_t bf16_rne(float f) {
   return static_cast<uint16_t>((u + 0x7FFFu + ((u >> 16) & 1u)) >> 16);
 }
 
-__device__ __forceinline__ float group_scale(uint32_t seed, uint32_t tensor, int64_t i) {
-  const Words u = draw(seed, GSCALE, i / kGroup, tensor, 0);
+__device__ __forceinline__ float group_scale_of_group(uint32_t seed, uint32_t tensor, int64_t g) {
+  const Words u = draw(seed, GSCALE, g, tensor, 0);
   return loguniform(u.w0, 1e-5f, 1e-2f);
+}
+
+__device__ __forceinline__ float group_scale(uint32_t seed, uint32_t tensor, int64_t i) {
+  return group_scale_of_group(seed, tensor, i / kGroup);
+}
+
+__device__ __forceinline__ float unit24(uint32_t u) {
+  return __fmul_rn(static_cast<float>(u >> 8), 5.9604644775390625e-08f);  // 2^-24
 }
 
 template <class F>
@@ -137,6 +145,30 @@ int synth_weight(uint16_t* out, int64_t count, uint32_t seed, uint32_t tensor, i
   return launch(count, s, [=] __device__(int64_t t) {
     const double z = ih4(draw(seed, WEIGHT, start + t, tensor, 0));
     out[t] = bf16_rne(__double2float_rn(__dmul_rn(0.02, z)));
+  });
+}
+
+int synth_state_codes(uint8_t* out, int64_t count, uint32_t seed, uint32_t tensor, uint32_t step,
+                      int64_t start, int fmt, int is_signed, cudaStream_t s) {
+  const uint32_t lo = fmt == 0 ? 0x01u : 0x34u, hi = fmt == 0 ? 0x7Eu : 0x7Bu;
+  return launch(count, s, [=] __device__(int64_t t) {
+    const Words u = draw(seed, is_signed ? MCODE : VCODE, start + t, tensor, step);
+    uint32_t c = lo + u.w0 % (hi - lo + 1u);
+    if (is_signed && (u.w1 >> 31)) c |= 0x80u;
+    out[t] = static_cast<uint8_t>(c);
+  });
+}
+
+int synth_state_groups(float* k_m, float* s_m, float* k_v, float* s_v, int64_t count, uint32_t seed,
+                       uint32_t tensor, uint32_t step, int64_t gstart, cudaStream_t s) {
+  return launch(count, s, [=] __device__(int64_t t) {
+    const int64_t g = gstart + t;
+    const Words u = draw(seed, GSTATE, g, tensor, step);
+    const float sg = group_scale_of_group(seed, tensor, g);
+    k_m[t] = __fadd_rn(__fmul_rn(0.7f, unit24(u.w0)), 1.5f);
+    s_m[t] = __fmul_rn(sg, __fadd_rn(__fmul_rn(0.04f, unit24(u.w1)), 0.02f));
+    k_v[t] = __fadd_rn(__fmul_rn(4.0f, unit24(u.w2)), 4.0f);
+    s_v[t] = __fmul_rn(__fmul_rn(sg, sg), __fadd_rn(__fmul_rn(0.2f, unit24(u.w3)), 0.1f));
   });
 }
 

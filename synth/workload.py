@@ -58,6 +58,19 @@ class DeviceParamSet:
         for i in range(len(self)):
             synth.device_grad(self.views(i)["grad"], self.seed, i, step)
 
+    def fill_states(self, step, fmt_m, fmt_v):
+        """Stored states (codes, k, root scale) drawn directly by the generator."""
+        for i in range(len(self)):
+            v = self.views(i)
+            n = v["n"]
+            if n == 0:
+                continue
+            synth.device_state_codes(v["mq"][:n], self.seed, i, step, fmt_m, True)
+            synth.device_state_codes(v["vq"][:n], self.seed, i, step, fmt_v, False)
+            v["mq"][n:].zero_()
+            v["vq"][n:].zero_()
+            synth.device_state_groups(v["mk"], v["ms"], v["vk"], v["vs"], self.seed, i, step)
+
     def warm_values(self, i, which, out=None):
         """FP32 warm-start values of moment `which` ('m' or 'v') of tensor i."""
         n = self.sizes[i]

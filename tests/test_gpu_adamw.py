@@ -1,8 +1,11 @@
 """GPU parity of the fused AdamW step (through the C ABI) against the CPU oracle.
 
-Free-running: both sides start from the same seeded inputs (FP32 master, FP32
-warm-start moments, bf16 gradients per step), each quantises the warm start with
-its own codec and runs its own trajectory; see tests/parity.py for the rules."""
+Identical-input steps: both sides start from the same generated state (codes,
+k, root scale drawn by the seeded generator), the same master and gradient;
+every tolerance applies to every element.  Master trajectory: 10 steps with the
+master carried forward on each side and a fresh identical state each step.
+Free-running: each side quantises the FP32 warm start with its own codec and
+runs its own 10-step trajectory (see tests/parity.py for what is compared)."""
 import numpy as np
 import pytest
 import torch
@@ -10,7 +13,7 @@ import torch
 import fp8_optimizer_state_b200 as coat
 import synth
 from synth import params as P
-from tests.parity import FreeRun, bf16_rne_bits
+from tests.parity import FreeRun, bf16_rne_bits, check_master, check_state_all
 
 pytestmark = pytest.mark.gpu
 H = P.HYPER
@@ -24,8 +27,19 @@ def to_dev(a, dtype=None):
     return t.cuda()
 
 
+def gen_state(n, tensor, step, fm, fv, seed=0):
+    """Generated stored state: (m_q, m_scale, m_k, v_q, v_scale, v_k) numpy arrays."""
+    ng = -(-n // 128)
+    mq = np.zeros(ng * 128, np.uint8)
+    vq = np.zeros(ng * 128, np.uint8)
+    mq[:n] = synth.state_codes(seed, tensor, step, 0, n, fm, True)
+    vq[:n] = synth.state_codes(seed, tensor, step, 0, n, fv, False)
+    km, sm, kv, sv = synth.state_groups(seed, tensor, step, 0, ng)
+    return mq, sm, km, vq, sv, kv
+
+
 class GpuSide:
-    def __init__(self, master, m0, v0, fmt_m, fmt_v, with_weight=True):
+    def __init__(self, master, fmt_m, fmt_v, with_weight=True):
         n = master.size
         ng = -(-n // 128)
         self.n, self.ng, self.fm, self.fv = n, ng, fmt_m, fmt_v
@@ -36,8 +50,19 @@ class GpuSide:
         self.vq = torch.zeros((1, ng * 128), dtype=torch.uint8, device="cuda")
         self.ms, self.mk, self.vs, self.vk = (torch.zeros((1, ng), dtype=torch.float32, device="cuda")
                                               for _ in range(4))
-        coat.coat_group_quantize(to_dev(m0).view(1, n), 1, 128, True, fmt_m, self.mq, self.ms, self.mk)
-        coat.coat_group_quantize(to_dev(v0).view(1, n), 1, 128, True, fmt_v, self.vq, self.vs, self.vk)
+
+    def warm_start(self, m0, v0):
+        n = self.n
+        coat.coat_group_quantize(to_dev(m0).view(1, n), 1, 128, True, self.fm, self.mq, self.ms, self.mk)
+        coat.coat_group_quantize(to_dev(v0).view(1, n), 1, 128, True, self.fv, self.vq, self.vs, self.vk)
+        return self
+
+    def set_state(self, st):
+        mq, sm, km, vq, sv, kv = st
+        for dst, src in ((self.mq, mq), (self.ms, sm), (self.mk, km), (self.vq, vq), (self.vs, sv),
+                         (self.vk, kv)):
+            dst.copy_(torch.from_numpy(np.ascontiguousarray(src)).view(dst.shape))
+        return self
 
     def step(self, g_bits, t):
         self.grad.copy_(torch.from_numpy(g_bits.view(np.int16)))
@@ -54,18 +79,29 @@ class GpuSide:
 
 
 class OracleSide:
-    def __init__(self, orc, master, m0, v0, fmt_m, fmt_v):
+    def __init__(self, orc, master, fmt_m, fmt_v):
         n = master.size
         ng = -(-n // 128)
-        self.orc, self.fm, self.fv = orc, fmt_m, fmt_v
+        self.orc, self.n, self.fm, self.fv = orc, n, fmt_m, fmt_v
         self.master = master.copy()
         self.weight = np.zeros(n, dtype=np.uint16)
         self.mq = np.zeros(ng * 128, np.uint8)
         self.vq = np.zeros(ng * 128, np.uint8)
-        q, s, k = orc.group_quantize(m0.reshape(1, n), 1, 128, True, fmt_m)
+        self.ms = self.mk = self.vs = self.vk = None
+
+    def warm_start(self, m0, v0):
+        n = self.n
+        q, s, k = self.orc.group_quantize(m0.reshape(1, n), 1, 128, True, self.fm)
         self.mq[:n], self.ms, self.mk = q.ravel(), s.ravel().copy(), k.ravel().copy()
-        q, s, k = orc.group_quantize(v0.reshape(1, n), 1, 128, True, fmt_v)
+        q, s, k = self.orc.group_quantize(v0.reshape(1, n), 1, 128, True, self.fv)
         self.vq[:n], self.vs, self.vk = q.ravel(), s.ravel().copy(), k.ravel().copy()
+        return self
+
+    def set_state(self, st):
+        mq, sm, km, vq, sv, kv = st
+        self.mq, self.ms, self.mk = mq.copy(), sm.copy(), km.copy()
+        self.vq, self.vs, self.vk = vq.copy(), sv.copy(), kv.copy()
+        return self
 
     def step(self, g_bits, t):
         return self.orc.adamw_step(self.master, self.weight, g_bits, self.mq, self.ms, self.mk,
@@ -74,59 +110,102 @@ class OracleSide:
                                    fmt_m=self.fm, fmt_v=self.fv, want_update=True)
 
 
-def run_free(orc, n, fmt_m, fmt_v, steps, tensor=0, seed=0):
-    master = synth.master(seed, tensor, 0, n)
-    m0 = synth.m_warm(seed, tensor, 0, n)
-    v0 = synth.v_warm(seed, tensor, 0, n)
-    gpu = GpuSide(master, m0, v0, fmt_m, fmt_v)
-    ora = OracleSide(orc, master, m0, v0, fmt_m, fmt_v)
+def compare_step(tag, gpu, ora, upd_sum, n, fm, fv):
+    h = gpu.host()
+    check_master(tag + " master", h["master"], ora.master, upd_sum)
+    assert np.array_equal(h["weight"], bf16_rne_bits(h["master"])), "bf16 copy != RNE(master)"
+    same = h["master"] == ora.master
+    assert np.array_equal(h["weight"][same], ora.weight[same])
+    fm_ = check_state_all(tag + " m", n, fm, h["mq"], h["ms"], h["mk"], ora.mq, ora.ms, ora.mk)[0]
+    fv_ = check_state_all(tag + " v", n, fv, h["vq"], h["vs"], h["vk"], ora.vq, ora.vs, ora.vk)[0]
+    assert not h["mq"][n:].any() and not h["vq"][n:].any()    # padding codes written 0
+    return fm_, fv_
+
+
+def one_step_identical(orc, n, fm, fv, t, tensor=0):
+    master = synth.master(0, tensor, 0, n)
+    st = gen_state(n, tensor, t, fm, fv)
+    gpu = GpuSide(master, fm, fv).set_state(st)
+    ora = OracleSide(orc, master, fm, fv).set_state(st)
+    g = synth.grad_bits(0, tensor, t, 0, n)
+    gpu.step(g, t)
+    upd = ora.step(g, t)
+    return compare_step("n=%d t=%d" % (n, t), gpu, ora, upd, n, fm, fv)
+
+
+@pytest.mark.parametrize("t", [1, 2, 5, 10])
+def test_one_step_identical_inputs_tiny(orc, t):
+    """Tiny workload size (1,048,576 elements, E4M3 + E4M3), steps 1, 2, 5, 10."""
+    flips = one_step_identical(orc, 1 << 20, E4M3, E4M3, t)
+    print("t=%d code flips m %d v %d of %d" % (t, flips[0], flips[1], 1 << 20))
+
+
+@pytest.mark.parametrize("fm,fv", [(E4M3, E5M2), (E5M2, E5M2), (E5M2, E4M3)])
+def test_one_step_identical_inputs_formats(orc, fm, fv):
+    one_step_identical(orc, 300000, fm, fv, 3, tensor=fm * 2 + fv)
+
+
+@pytest.mark.parametrize("n", [1, 5, 127, 128, 129, 4095, 4096, 4097, 3 * 4096 + 77, 70000])
+def test_ragged_sizes_identical_inputs(orc, n):
+    one_step_identical(orc, n, E4M3, E5M2, 1, tensor=n % 97)
+
+
+def test_master_trajectory_10_steps(orc):
+    """The FP32 master over 10 steps (tiny size, E4M3 + E4M3): the master is carried
+    forward on each side, every step gets a fresh identical state and gradient."""
+    n = 1 << 20
+    master = synth.master(0, 3, 0, n)
+    gpu = GpuSide(master, E4M3, E4M3)
+    ora = OracleSide(orc, master, E4M3, E4M3)
+    upd_sum = np.zeros(n)
+    for t in range(1, 11):
+        st = gen_state(n, 3, t, E4M3, E4M3)
+        gpu.set_state(st)
+        ora.set_state(st)
+        g = synth.grad_bits(0, 3, t, 0, n)
+        gpu.step(g, t)
+        upd_sum += ora.step(g, t)
+        h = gpu.host()
+        check_master("step %d" % t, h["master"], ora.master, upd_sum)
+    rel = np.abs(h["master"].astype(np.float64) - ora.master) / (np.abs(ora.master) + upd_sum)
+    print("master after 10 steps: max rel err %.3g, median %.3g" % (rel.max(), np.median(rel)))
+
+
+def test_free_running_10_steps(orc):
+    """Tiny workload, free-running from each side's own warm-start quantisation."""
+    n, fm, fv = 1 << 20, E4M3, E4M3
+    master = synth.master(0, 0, 0, n)
+    m0, v0 = synth.m_warm(0, 0, 0, n), synth.v_warm(0, 0, 0, n)
+    gpu = GpuSide(master, fm, fv).warm_start(m0, v0)
+    ora = OracleSide(orc, master, fm, fv).warm_start(m0, v0)
     fr = FreeRun(n)
     h = gpu.host()
-    fl = fr.check_state("warm m", h["mq"], h["ms"], h["mk"], ora.mq, ora.ms, ora.mk)
-    fl |= fr.check_state("warm v", h["vq"], h["vs"], h["vk"], ora.vq, ora.vs, ora.vk)
-    fr.exclude(fl)
-    for t in range(1, steps + 1):
-        g = synth.grad_bits(seed, tensor, t, 0, n)
+    cd1, sd1 = fr.check_state("warm m", fm, h["mq"], h["ms"], h["mk"], ora.mq, ora.ms, ora.mk)
+    cd2, sd2 = fr.check_state("warm v", fv, h["vq"], h["vs"], h["vk"], ora.vq, ora.vs, ora.vk)
+    fr.after_step(cd1 | cd2, sd1 | sd2)
+    for t in range(1, 11):
+        g = synth.grad_bits(0, 0, t, 0, n)
         gpu.step(g, t)
         upd = ora.step(g, t)
         h = gpu.host()
         fr.check_master("step %d master" % t, h["master"], ora.master, upd)
-        assert np.array_equal(h["weight"], bf16_rne_bits(h["master"])), "bf16 copy != RNE(master)"
-        same = h["master"] == ora.master
-        assert np.array_equal(h["weight"][same & fr.element_mask()],
-                              ora.weight[same & fr.element_mask()])
-        fl = fr.check_state("step %d m" % t, h["mq"], h["ms"], h["mk"], ora.mq, ora.ms, ora.mk)
-        fl |= fr.check_state("step %d v" % t, h["vq"], h["vs"], h["vk"], ora.vq, ora.vs, ora.vk)
-        fr.exclude(fl)
-    return fr, gpu, ora
-
-
-def test_tiny_config_free_running_10_steps(orc):
-    """Tiny workload: one flat tensor of 1,048,576, E4M3 + E4M3, 10 steps."""
-    fr, gpu, ora = run_free(orc, 1 << 20, E4M3, E4M3, 10)
-    excluded = int(fr.excluded.sum())
-    print("flips per check:", fr.report, "excluded groups:", excluded, "of", fr.ng)
-    assert excluded <= 0.05 * fr.ng
-
-
-@pytest.mark.parametrize("n", [1, 5, 127, 128, 129, 4095, 4096, 4097, 3 * 4096 + 77, 70000])
-def test_ragged_sizes_e5m2(orc, n):
-    fr, gpu, ora = run_free(orc, n, E4M3, E5M2, 3, tensor=n % 97)
-    h = gpu.host()
-    ng = -(-n // 128)
-    assert not h["mq"][n:].any() and not h["vq"][n:].any()   # padding codes written 0
-
-
-def test_e5m2_m_and_v(orc):
-    run_free(orc, 20000, E5M2, E5M2, 3, tensor=5)
+        assert np.array_equal(h["weight"], bf16_rne_bits(h["master"]))
+        cd1, sd1 = fr.check_state("step %d m" % t, fm, h["mq"], h["ms"], h["mk"], ora.mq, ora.ms, ora.mk)
+        cd2, sd2 = fr.check_state("step %d v" % t, fv, h["vq"], h["vs"], h["vk"], ora.vq, ora.vs, ora.vk)
+        fr.after_step(cd1 | cd2, sd1 | sd2)
+    print("free-running report (tag, flips among compared, groups compared, groups with "
+          "code diffs, groups with k/scale diffs):")
+    for r in fr.report:
+        print("  ", r)
+    print("groups whose master left the comparison: %d of %d" % (int(fr.flipped.sum()), fr.ng))
 
 
 def test_weight_out_optional_and_deterministic():
     n = 50000
     master = synth.master(0, 7, 0, n)
-    m0, v0 = synth.m_warm(0, 7, 0, n), synth.v_warm(0, 7, 0, n)
-    a = GpuSide(master, m0, v0, E4M3, E5M2, with_weight=True)
-    b = GpuSide(master, m0, v0, E4M3, E5M2, with_weight=False)
+    st = gen_state(n, 7, 1, E4M3, E5M2)
+    a = GpuSide(master, E4M3, E5M2, with_weight=True).set_state(st)
+    b = GpuSide(master, E4M3, E5M2, with_weight=False).set_state(st)
     for t in (1, 2):
         g = synth.grad_bits(0, 7, t, 0, n)
         a.step(g, t)
@@ -140,12 +219,12 @@ def test_resume_from_copied_state_is_bit_identical():
     """Checkpoint/resume: the state is the caller's buffers plus the step count."""
     n = 30000
     master = synth.master(0, 9, 0, n)
-    m0, v0 = synth.m_warm(0, 9, 0, n), synth.v_warm(0, 9, 0, n)
-    a = GpuSide(master, m0, v0, E4M3, E4M3)
+    st = gen_state(n, 9, 1, E4M3, E4M3)
+    a = GpuSide(master, E4M3, E4M3).set_state(st)
     for t in (1, 2):
         a.step(synth.grad_bits(0, 9, t, 0, n), t)
     saved = {k: getattr(a, k).clone() for k in ("master", "mq", "ms", "mk", "vq", "vs", "vk")}
-    b = GpuSide(master, m0, v0, E4M3, E4M3)
+    b = GpuSide(master, E4M3, E4M3)
     for k, v in saved.items():
         getattr(b, k).copy_(v)
     g3 = synth.grad_bits(0, 9, 3, 0, n)
@@ -162,8 +241,8 @@ def test_degenerate_groups_exact(orc):
     n = 128 * 6
     master = synth.master(0, 11, 0, n)
     zeros = np.zeros(n, np.float32)
-    gpu = GpuSide(master, zeros, zeros, E4M3, E4M3)
-    ora = OracleSide(orc, master, zeros, zeros, E4M3, E4M3)
+    gpu = GpuSide(master, E4M3, E4M3).warm_start(zeros, zeros)
+    ora = OracleSide(orc, master, E4M3, E4M3).warm_start(zeros, zeros)
     g = np.zeros(n, dtype=np.float32)
     g[128:256] = 0.25 * np.where(np.arange(128) % 3 == 0, -1, 1)   # one magnitude
     g[256:384] = 2.0 ** -10

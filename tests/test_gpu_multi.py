@@ -7,8 +7,8 @@ import torch
 import fp8_optimizer_state_b200 as coat
 import synth
 from synth import params as P
-from tests.parity import FreeRun
-from tests.test_gpu_adamw import GpuSide, OracleSide
+from tests.parity import check_master, check_state_all
+from tests.test_gpu_adamw import GpuSide, OracleSide, gen_state
 
 pytestmark = pytest.mark.gpu
 H = P.HYPER
@@ -24,7 +24,8 @@ def make_sides(sizes, fm, fv):
     sides = []
     for i, n in enumerate(sizes):
         master = synth.master(1, i, 0, n)
-        sides.append(GpuSide(master, synth.m_warm(1, i, 0, n), synth.v_warm(1, i, 0, n), fm, fv))
+        sides.append(GpuSide(master, fm, fv).warm_start(synth.m_warm(1, i, 0, n),
+                                                        synth.v_warm(1, i, 0, n)))
     return sides
 
 
@@ -57,31 +58,26 @@ def test_multi_equals_single_calls(fm, fv):
 
 
 def test_multi_vs_oracle(orc):
-    sizes = [5000, 129, 70001]
-    sides = make_sides(sizes, 0, 1)
-    oras = []
+    """One multi-tensor launch from identical generated states matches the oracle."""
+    sizes = [5000, 129, 70001, 4096 * 3]
+    sides, oras = [], []
     for i, n in enumerate(sizes):
-        oras.append(OracleSide(orc, synth.master(1, i, 0, n), synth.m_warm(1, i, 0, n),
-                               synth.v_warm(1, i, 0, n), 0, 1))
-    frs = [FreeRun(n) for n in sizes]
-    for fr, s, o in zip(frs, sides, oras):
-        h = s.host()
-        fl = fr.check_state("warm m", h["mq"], h["ms"], h["mk"], o.mq, o.ms, o.mk)
-        fl |= fr.check_state("warm v", h["vq"], h["vs"], h["vk"], o.vq, o.vs, o.vk)
-        fr.exclude(fl)
+        master = synth.master(1, i, 0, n)
+        st = gen_state(n, i, 4, 0, 1, seed=1)
+        sides.append(GpuSide(master, 0, 1).set_state(st))
+        oras.append(OracleSide(orc, master, 0, 1).set_state(st))
     plan = plan_of(sides, 0, 1)
-    for t in (1, 2):
-        upds = []
-        for i, (s, o) in enumerate(zip(sides, oras)):
-            g = synth.grad_bits(1, i, t, 0, sizes[i])
-            s.grad.copy_(torch.from_numpy(g.view(np.int16)))
-            upds.append(o.step(g, t))
-        coat.coat_adamw_step_multi(plan, lr=H["lr"], beta1=H["beta1"], beta2=H["beta2"],
-                                   eps=H["eps"], wd=H["wd"], step=t)
-        for fr, s, o, u in zip(frs, sides, oras, upds):
-            h = s.host()
-            fr.check_master("master", h["master"], o.master, u)
-            fl = fr.check_state("m", h["mq"], h["ms"], h["mk"], o.mq, o.ms, o.mk)
-            fl |= fr.check_state("v", h["vq"], h["vs"], h["vk"], o.vq, o.vs, o.vk)
-            fr.exclude(fl)
+    upds = []
+    for i, (s, o) in enumerate(zip(sides, oras)):
+        g = synth.grad_bits(1, i, 4, 0, sizes[i])
+        s.grad.copy_(torch.from_numpy(g.view(np.int16)))
+        upds.append(o.step(g, 4))
+    coat.coat_adamw_step_multi(plan, lr=H["lr"], beta1=H["beta1"], beta2=H["beta2"],
+                               eps=H["eps"], wd=H["wd"], step=4)
+    coat.coat_check_device_error()
+    for n, s, o, u in zip(sizes, sides, oras, upds):
+        h = s.host()
+        check_master("master", h["master"], o.master, u)
+        check_state_all("m", n, 0, h["mq"], h["ms"], h["mk"], o.mq, o.ms, o.mk)
+        check_state_all("v", n, 1, h["vq"], h["vs"], h["vk"], o.vq, o.vs, o.vk)
     plan.destroy()
