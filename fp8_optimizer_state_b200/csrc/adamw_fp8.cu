@@ -9,14 +9,16 @@
 // the new group max/min, and requantise.
 //
 // Design (HBM-bound: 16.25 algorithmic bytes per parameter, no tensor cores):
-//  * persistent CTAs, 2 per SM; tiles of 32 groups (4096 elements);
+//  * persistent CTAs, 2 per SM, 8 warps each (so that every SM sub-partition
+//    holds 4 warps and a thread may use 128 registers); tiles of 28 groups
+//    (3584 elements);
 //  * one producer thread streams whole tiles (master, grad, both code arrays,
-//    the four metadata arrays: 33,280 B) into a 3-stage shared-memory ring
+//    the four metadata arrays: 29,120 B) into a 3-stage shared-memory ring
 //    with 1-D cp.async.bulk copies completing on an mbarrier, so that bytes in
 //    flight do not depend on registers.  It keeps the current tensor's
 //    descriptor in registers, prefetches the next tile's tensor index, and
 //    writes the descriptor into the stage header for the consumers;
-//  * 8 consumer warps; each warp owns 4 groups of a tile, 8 lanes per group,
+//  * 7 consumer warps; each warp owns 4 groups of a tile, 8 lanes per group,
 //    16 elements per lane in 4 chunks of 4 contiguous elements (chunk order
 //    rotated per group to keep shared-memory reads conflict-free); group
 //    max / min-nonzero by 3 xor-shuffles inside the 8 lanes;
@@ -38,30 +40,34 @@
 namespace coat {
 namespace {
 
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = 7;
 constexpr int kGroupsPerWarp = 4;
-constexpr int kTileGroups = kConsumerWarps * kGroupsPerWarp;  // 32
-constexpr int kTileElems = kTileGroups * kGroup;               // 4096
+constexpr int kTileGroups = kConsumerWarps * kGroupsPerWarp;  // 28
+constexpr int kTileElems = kTileGroups * kGroup;               // 3584
 constexpr int kStages = 3;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;             // 288
+constexpr int kThreads = (kConsumerWarps + 1) * 32;             // 256
 constexpr int kCtasPerSm = 2;
 
-// Stage layout (bytes): every array starts on a 128-byte boundary.
+// Stage layout (bytes): the element arrays start on 128-byte boundaries, the
+// metadata arrays (112 B each) on 16-byte boundaries; stages are padded to a
+// multiple of 128 bytes.
 constexpr uint32_t kOffMaster = 0;
-constexpr uint32_t kOffGrad = kOffMaster + kTileElems * 4;   // 16384
-constexpr uint32_t kOffMq = kOffGrad + kTileElems * 2;       // 24576
-constexpr uint32_t kOffVq = kOffMq + kTileElems;             // 28672
-constexpr uint32_t kOffMs = kOffVq + kTileElems;             // 32768
+constexpr uint32_t kOffGrad = kOffMaster + kTileElems * 4;   // 14336
+constexpr uint32_t kOffMq = kOffGrad + kTileElems * 2;       // 21504
+constexpr uint32_t kOffVq = kOffMq + kTileElems;             // 25088
+constexpr uint32_t kOffMs = kOffVq + kTileElems;             // 28672
 constexpr uint32_t kOffMk = kOffMs + kTileGroups * 4;
 constexpr uint32_t kOffVs = kOffMk + kTileGroups * 4;
 constexpr uint32_t kOffVk = kOffVs + kTileGroups * 4;
-constexpr uint32_t kStageBytes = kOffVk + kTileGroups * 4;   // 33280
+constexpr uint32_t kTxBytes = kOffVk + kTileGroups * 4;      // 29120 copied per tile
+constexpr uint32_t kStageBytes = ((kTxBytes + 127) / 128) * 128;
+static_assert(kTileElems % 16 == 0 && (kTileGroups * 4) % 16 == 0, "bulk copies need 16-byte sizes");
 
 struct TileHeader {
   TensorArgs t;     // descriptor of the tile's tensor
   int64_t g0;       // first group of the tile within its tensor
   int32_t ngroups;  // groups of this tile that exist
-  int32_t full;     // 1: all 4096 elements valid and staged in shared memory
+  int32_t full;     // 1: all 3584 elements valid and staged in shared memory
 };
 
 struct Smem {
@@ -343,7 +349,7 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
 }
 
 template <int FM, int FV, class Map>
-__global__ void __maxnreg__(112)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     adamw_fp8_kernel(const Map map, const StepHyper h, unsigned* err) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>(smem_raw);
@@ -407,7 +413,7 @@ __global__ void __maxnreg__(112)
       hd.full = full ? 1 : 0;
       if (full) {
         uint8_t* st = stages + size_t(s) * kStageBytes;
-        mbar_arrive_expect_tx(&S.full_bar[s], kStageBytes);
+        mbar_arrive_expect_tx(&S.full_bar[s], kTxBytes);
         bulk_g2s(st + kOffMaster, ct.master + e0, kTileElems * 4, &S.full_bar[s]);
         bulk_g2s(st + kOffGrad, ct.grad + e0, kTileElems * 2, &S.full_bar[s]);
         bulk_g2s(st + kOffMq, ct.mq + e0, kTileElems, &S.full_bar[s]);

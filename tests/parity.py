@@ -24,8 +24,10 @@ Comparison modes:
     s_r) differs in any bit no longer has the same inputs at the next step;
     its k, s_r and codes are then not compared (a difference of one FP32 ulp
     in k is amplified by the cancellation in min|m'| into a k difference far
-    above 1e-5), and once its codes differ its master leaves the comparison
-    too.  Counts are reported.
+    above 1e-5).  Once its codes differ, or its k or s_r differ by more than
+    2e-6 relative, its dequantised moments differ by more than the master
+    tolerance can absorb and its master leaves the comparison too.  Counts are
+    reported.
 """
 from __future__ import annotations
 
@@ -130,13 +132,16 @@ class FreeRun:
         code_diff = (gq2 != oq2).any(axis=1)
         meta_diff = (np.asarray(gk)[:ng] != np.asarray(ok_)[:ng]) | \
                     (np.asarray(gs)[:ng] != np.asarray(os_)[:ng])
-        self.report.append((tag, nd, int(sel.sum()), int(code_diff.sum()), int(meta_diff.sum())))
-        return code_diff, code_diff | meta_diff
+        big = code_diff | (rel_err(np.asarray(gk)[:ng], np.asarray(ok_)[:ng]) > 2e-6) | \
+            (rel_err(np.asarray(gs)[:ng], np.asarray(os_)[:ng]) > 2e-6)
+        self.report.append((tag, nd, int(sel.sum()), int(code_diff.sum()), int(meta_diff.sum()),
+                            int(big.sum())))
+        return big, code_diff | meta_diff
 
     def check_master(self, tag, gm, om, upd_abs):
         self.upd_sum += upd_abs
         check_master(tag, gm, om, self.upd_sum, mask=self.element_mask())
 
-    def after_step(self, code_diff, state_diff):
-        self.flipped |= code_diff
+    def after_step(self, diverged, state_diff):
+        self.flipped |= diverged
         self.same &= ~state_diff

@@ -194,7 +194,7 @@ def test_free_running_10_steps(orc):
         cd2, sd2 = fr.check_state("step %d v" % t, fv, h["vq"], h["vs"], h["vk"], ora.vq, ora.vs, ora.vk)
         fr.after_step(cd1 | cd2, sd1 | sd2)
     print("free-running report (tag, flips among compared, groups compared, groups with "
-          "code diffs, groups with k/scale diffs):")
+          "code diffs, groups with k/scale diffs, groups diverged beyond 2e-6):")
     for r in fr.report:
         print("  ", r)
     print("groups whose master left the comparison: %d of %d" % (int(fr.flipped.sum()), fr.ng))
