@@ -200,9 +200,9 @@ __device__ __forceinline__ double exp2_table(double t, const double* exp2_16) {
 // cancellation between beta1*m and (1-beta1)*g, so its FP32 value carries the
 // FP32 dequantisation error amplified by |beta1 m| / |m'| (often 100x-1000x),
 // and k depends on it through ln(max/min).  The kernel keeps the two smallest
-// candidates (their positions packed into the low bits of the comparison keys,
-// at a cost of 2^-18 relative in the ordering) and recomputes both in double
-// precision: dequantisation, then m' = beta1 m + (1 - beta1) g.
+// candidates (their positions packed into the low 8 bits of the comparison
+// keys, at a cost of 2^-16 relative in the ordering) and recomputes them in
+// double precision: dequantisation, then m' = beta1 m + (1 - beta1) g.
 __device__ __forceinline__ float recompute_m_double(const LaneIn& in, int idx,
                                                     const StepHyper& h, const double* tabd_m,
                                                     const double* exp2_16) {
@@ -222,10 +222,11 @@ __device__ __forceinline__ float recompute_m_double(const LaneIn& in, int idx,
   return __double2float_rn(fabs(m1));
 }
 
-// Comparison key of |x|: FP32 bits without the sign, minus one (so that zero
-// becomes the largest key), low 4 bits replaced by the element index.
+// Comparison key of |x|: the FP32 bits shifted left by one (dropping the sign)
+// minus two, so that zero becomes the largest key and the order of nonzero
+// magnitudes is kept; the low 5 bits are replaced by the element index.
 __device__ __forceinline__ uint32_t min_key(float x, int idx) {
-  return (((__float_as_uint(x) & 0x7FFFFFFFu) - 1u) & 0xFFFFFFF0u) | static_cast<uint32_t>(idx);
+  return ((__float_as_uint(x) * 2u - 2u) & 0xFFFFFFE0u) | static_cast<uint32_t>(idx);
 }
 
 // The per-lane body: everything after the loads.  FULL: every element of the
@@ -260,9 +261,8 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
       float mn = __fmaf_rn(h.omb1, g, bm);
       float vn = __fmaf_rn(h.omb2 * g, g, bv);
       const float p = f4get(in.p[j], i);
-      const float denom = __fmaf_rn(sqrt_approx(vn), h.rsbc2, h.eps);
-      const float upd = (h.step_size * mn) * rcp_approx(denom);
-      pn[i] = p + __fmaf_rn(-p, h.lrwd, -upd);
+      const float upd = mn * rcp_approx(__fmaf_rn(sqrt_approx(vn), h.dsq, h.deps));
+      pn[i] = p + __fmaf_rn(-p, h.lrwd, h.zero_lr ? 0.f : -upd);
       if (!FULL) {
         const bool valid = active && (e + i < t.n);
         mn = valid ? mn : 0.f;
@@ -295,8 +295,8 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
   // group statistics over the 8 lanes of this group.  The m keys carry the
   // position (lane l, element index) of the two smallest |m'| in their low 7
   // bits; merging two sorted pairs keeps the two smallest of the union.
-  minm1 = (minm1 & ~0x70u) | (static_cast<uint32_t>(l) << 4);
-  minm2 = (minm2 & ~0x70u) | (static_cast<uint32_t>(l) << 4);
+  minm1 = (minm1 & ~0xE0u) | (static_cast<uint32_t>(l) << 5);
+  minm2 = (minm2 & ~0xE0u) | (static_cast<uint32_t>(l) << 5);
 #pragma unroll
   for (int off = 1; off < 8; off <<= 1) {
     maxm = fmaxf(maxm, __shfl_xor_sync(0xFFFFFFFFu, maxm, off));
@@ -307,16 +307,21 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
     minm2 = min(max(minm1, o1), min(minm2, o2));
     minm1 = min(minm1, o1);
   }
-  // min |m'| exact as FP32: the lanes owning the two candidates recompute them
+  // min |m'| exact as FP32: the lane owning the smallest candidate recomputes
+  // it; the runner-up is recomputed too when its FP32 key is within about
+  // 2^-7 relative of the smallest (a near-tie that the FP32 values, off by up
+  // to |beta1 m| / |m'| times their dequantisation error, may misorder)
+  const bool any_m = minm1 < 0xFFFFFF00u;
+  const bool tie = minm2 < 0xFFFFFF00u && (minm2 >> 8) - (minm1 >> 8) < (1u << 9);
   float mum = __int_as_float(0x7F800000);
-  if (minm1 < 0xFFFFFF80u && static_cast<int>((minm1 >> 4) & 7u) == l)
+  if (any_m && static_cast<int>((minm1 >> 5) & 7u) == l)
     mum = recompute_m_double(in, static_cast<int>(minm1 & 15u), h, S.tabd_m, S.exp2_16);
-  if (minm2 < 0xFFFFFF80u && static_cast<int>((minm2 >> 4) & 7u) == l)
+  if (tie && static_cast<int>((minm2 >> 5) & 7u) == l)
     mum = fminf(mum, recompute_m_double(in, static_cast<int>(minm2 & 15u), h, S.tabd_m,
                                         S.exp2_16));
 #pragma unroll
   for (int off = 1; off < 8; off <<= 1) mum = fminf(mum, __shfl_xor_sync(0xFFFFFFFFu, mum, off));
-  if (!(minm1 < 0xFFFFFF80u)) mum = 0.f;   // no nonzero element
+  if (!any_m) mum = 0.f;   // no nonzero element
   const float muv = __uint_as_float(minv + 1u);
   float km, srm, invMm, kv, srv, invMv;
   group_params<FM>(maxm, mum, true, km, srm, invMm);

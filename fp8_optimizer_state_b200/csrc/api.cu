@@ -109,10 +109,11 @@ coat::StepHyper make_hyper(float lr, float beta1, float beta2, float eps, float 
   h.beta2 = beta2;
   h.omb1 = static_cast<float>(1.0 - b1);
   h.omb2 = static_cast<float>(1.0 - b2);
-  h.step_size = static_cast<float>(static_cast<double>(lr) / bc1);
-  h.rsbc2 = static_cast<float>(1.0 / std::sqrt(bc2));
-  h.eps = eps;
-  h.lrwd = static_cast<float>(static_cast<double>(lr) * static_cast<double>(wd));
+  const double dlr = lr;
+  h.zero_lr = lr == 0.f ? 1 : 0;
+  h.dsq = h.zero_lr ? 1.f : static_cast<float>(bc1 / (dlr * std::sqrt(bc2)));
+  h.deps = h.zero_lr ? 1.f : static_cast<float>(static_cast<double>(eps) * bc1 / dlr);
+  h.lrwd = static_cast<float>(dlr * static_cast<double>(wd));
   return h;
 }
 

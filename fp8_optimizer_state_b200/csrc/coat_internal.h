@@ -22,15 +22,16 @@ struct TensorArgs {
   int64_t tile_begin;  // first tile of this tensor in a multi-tensor launch
 };
 
-// Hyperparameters as the kernel uses them (bias corrections folded on the host
-// in double): m' = beta1 m + omb1 g, v' = beta2 v + omb2 g^2,
-// p <- p - p lrwd - step_size m' / (sqrt(v') rsbc2 + eps).
+// Hyperparameters as the kernel uses them (bias corrections and the step size
+// folded on the host in double): m' = beta1 m + omb1 g, v' = beta2 v + omb2 g^2,
+// p <- p - p lrwd - m' / (sqrt(v') dsq + deps), which is
+// p - (lr / (1-beta1^t)) m' / (sqrt(v') / sqrt(1-beta2^t) + eps).
 struct StepHyper {
   float beta1, beta2, omb1, omb2;
-  float step_size;  // lr / (1 - beta1^t)
-  float rsbc2;      // 1 / sqrt(1 - beta2^t)
-  float eps;
+  float dsq;        // (1 - beta1^t) / (lr sqrt(1 - beta2^t))
+  float deps;       // eps (1 - beta1^t) / lr
   float lrwd;       // lr * wd
+  int zero_lr;      // lr == 0: the adaptive term is 0
 };
 
 int sm_count(int dev);
