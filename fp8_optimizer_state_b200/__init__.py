@@ -38,7 +38,10 @@ EXPORTS = [
     ("coat_multi_plan_destroy", _i32, [_vp]),
     ("coat_multi_plan_info", _i32, [_vp, ctypes.POINTER(_i64), ctypes.POINTER(_i32)]),
     ("coat_check_device_error", _i32, [_vp]),
+    ("coat_adamw_step_multi_noalloc", _i32, [_vp, _i32, _i32, _f32, _f32, _f32, _f32, _f32, _i64,
+                                             _i32, _i32, _vp]),
 ]
+NOALLOC_MAX_TENSORS = 1024
 
 
 class CoatError(RuntimeError):
@@ -191,6 +194,18 @@ def coat_adamw_step_multi(plan, *, lr, beta1, beta2, eps, wd, step, stream=None)
 
 def coat_multi_plan_destroy(plan):
     plan.destroy()
+
+
+def coat_adamw_step_multi_noalloc(descs, *, lr, beta1, beta2, eps, wd, step, fmt_m=COAT_E4M3,
+                                  fmt_v=COAT_E4M3, group=GROUP, stream=None):
+    """The multi-tensor step without any allocation (descs: list of TensorDesc,
+    at most NOALLOC_MAX_TENSORS).  Reports through the status code only."""
+    arr = (TensorDesc * len(descs))(*descs)
+    st = lib().coat_adamw_step_multi_noalloc(ctypes.cast(arr, ctypes.c_void_p), len(descs), group,
+                                             lr, beta1, beta2, eps, wd, step, fmt_m, fmt_v,
+                                             _s(stream))
+    if st != 0:
+        raise CoatError(st, "coat_adamw_step_multi_noalloc rejected the call")
 
 
 def coat_check_device_error(stream=None):

@@ -101,6 +101,28 @@ struct MultiTensor {
   __device__ __forceinline__ TensorArgs get(int32_t i) const { return descs[i]; }
 };
 
+// Multi-tensor launch without a per-tile map: the tile's tensor is found by
+// binary search over the tensors' first tiles (tile_begin[0..num], ascending;
+// empty tensors share the next tensor's first tile and are skipped because the
+// search returns the last tensor whose first tile is <= the tile).
+struct MultiTensorSearch {
+  static constexpr bool kSingle = false;
+  const TensorArgs* descs;
+  const int64_t* tile_begin;
+  int32_t num;
+  int64_t total_tiles;
+  __device__ __forceinline__ int64_t tiles() const { return total_tiles; }
+  __device__ __forceinline__ int32_t tensor_of(int64_t tile) const {
+    int32_t lo = 0, hi = num - 1;
+    while (lo < hi) {
+      const int32_t mid = (lo + hi + 1) >> 1;
+      if (tile_begin[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  }
+  __device__ __forceinline__ TensorArgs get(int32_t i) const { return descs[i]; }
+};
+
 // The 16 elements a lane owns, as loaded.
 struct LaneIn {
   float4 p[4];
@@ -508,6 +530,17 @@ cudaError_t launch_adamw_multi(const TensorArgs* d_descs, const int32_t* d_tile_
                                int64_t total_tiles, int fm, int fv, const StepHyper& h,
                                unsigned* err, cudaStream_t stream) {
   MultiTensor map{d_descs, d_tile_tensor, total_tiles};
+  return dispatch(fm, fv, map, total_tiles, h, err, stream);
+}
+
+}  // namespace coat
+
+namespace coat {
+
+cudaError_t launch_adamw_multi_search(const TensorArgs* d_descs, const int64_t* d_tile_begin,
+                                      int num, int64_t total_tiles, int fm, int fv,
+                                      const StepHyper& h, unsigned* err, cudaStream_t stream) {
+  MultiTensorSearch map{d_descs, d_tile_begin, num, total_tiles};
   return dispatch(fm, fv, map, total_tiles, h, err, stream);
 }
 

@@ -67,7 +67,7 @@ int sm_count(int dev) {
 
 // Device address of the error word on the current device (looked up once per
 // device with that device current).
-static cudaError_t device_error_ptr(unsigned** out) {
+cudaError_t device_error_ptr(unsigned** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -372,3 +372,116 @@ coat_status coat_check_device_error(cudaStream_t stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// coat_adamw_step_multi_noalloc: the multi-tensor step for callers that cannot
+// allocate device memory.  Its descriptor table lives in a fixed file-scope
+// device array instead of a plan's cudaMalloc'd table.
+// ---------------------------------------------------------------------------
+namespace {
+
+struct NoAllocScratch {
+  coat::TensorArgs descs[COAT_NOALLOC_MAX_TENSORS];
+  int64_t tile_begin[COAT_NOALLOC_MAX_TENSORS + 1];
+};
+
+// Every GPU that loads the library holds this array until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[sizeof(NoAllocScratch)];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64];
+
+// Device address of the scratch array on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device, with that device current, and cached.
+cudaError_t noalloc_scratch_ptr(NoAllocScratch** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = static_cast<NoAllocScratch*>(g_noalloc_ptr[dev]);
+  return cudaSuccess;
+}
+
+bool noalloc_desc_ok(const coat_tensor_desc& d, coat_status* st) {
+  if (d.n < 0) { *st = COAT_ERR_INVALID_ARG; return false; }
+  if (d.n == 0) return true;
+  const void* req[] = {d.master, d.grad, d.m_q, d.m_scale, d.m_k, d.v_q, d.v_scale, d.v_k};
+  for (const void* p : req) {
+    if (!p) { *st = COAT_ERR_INVALID_ARG; return false; }
+    if (!aligned(p, 16)) { *st = COAT_ERR_MISALIGNED; return false; }
+  }
+  if (d.weight_bf16_out && !aligned(d.weight_bf16_out, 16)) { *st = COAT_ERR_MISALIGNED; return false; }
+  return true;
+}
+
+}  // namespace
+
+extern "C" coat_status coat_adamw_step_multi_noalloc(const coat_tensor_desc* host_descs, int num,
+                                                     int group, float lr, float beta1,
+                                                     float beta2, float eps, float wd,
+                                                     int64_t step, coat_fmt fmt_m, coat_fmt fmt_v,
+                                                     cudaStream_t stream) {
+  if (!host_descs || num < 1) return COAT_ERR_INVALID_ARG;
+  if (group < 1 || !valid_fmt(fmt_m) || !valid_fmt(fmt_v)) return COAT_ERR_INVALID_ARG;
+  if (group != 128 || num > COAT_NOALLOC_MAX_TENSORS) return COAT_ERR_UNSUPPORTED;
+  if (!std::isfinite(lr) || lr < 0.f || !(beta1 >= 0.f && beta1 < 1.f) ||
+      !(beta2 >= 0.f && beta2 < 1.f) || !std::isfinite(eps) || !(eps > 0.f) ||
+      !std::isfinite(wd) || wd < 0.f || step < 1)
+    return COAT_ERR_INVALID_ARG;
+  coat_status st = COAT_OK;
+  for (int i = 0; i < num; ++i)
+    if (!noalloc_desc_ok(host_descs[i], &st)) return st;
+
+  NoAllocScratch* scratch = nullptr;
+  unsigned* err = nullptr;
+  if (noalloc_scratch_ptr(&scratch) != cudaSuccess || coat::device_error_ptr(&err) != cudaSuccess)
+    return COAT_ERR_CUDA;
+
+  // Stage the descriptor table through a small stack buffer, one async copy per
+  // chunk on the caller's stream (a copy from pageable memory returns once the
+  // source has been read, so the buffer can be reused at once).
+  constexpr int kChunk = 32;
+  coat::TensorArgs buf[kChunk];
+  int64_t begins[kChunk];
+  int64_t tiles = 0;
+  const int64_t tg = coat::step_tile_groups();
+  for (int c0 = 0; c0 < num; c0 += kChunk) {
+    const int cn = num - c0 < kChunk ? num - c0 : kChunk;
+    for (int j = 0; j < cn; ++j) {
+      const coat_tensor_desc& d = host_descs[c0 + j];
+      coat::TensorArgs& t = buf[j];
+      t.master = d.master;
+      t.wout = d.weight_bf16_out;
+      t.grad = d.grad;
+      t.mq = d.m_q;
+      t.ms = d.m_scale;
+      t.mk = d.m_k;
+      t.vq = d.v_q;
+      t.vs = d.v_scale;
+      t.vk = d.v_k;
+      t.n = d.n;
+      t.tiles = ((d.n + 127) / 128 + tg - 1) / tg;
+      t.tile_begin = tiles;
+      begins[j] = tiles;
+      tiles += t.tiles;
+    }
+    if (cudaMemcpyAsync(scratch->descs + c0, buf, sizeof(coat::TensorArgs) * cn,
+                        cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+        cudaMemcpyAsync(scratch->tile_begin + c0, begins, sizeof(int64_t) * cn,
+                        cudaMemcpyHostToDevice, stream) != cudaSuccess)
+      return COAT_ERR_CUDA;
+  }
+  if (tiles == 0) return COAT_OK;
+  const cudaError_t e = coat::launch_adamw_multi_search(
+      scratch->descs, scratch->tile_begin, num, tiles, fmt_m, fmt_v,
+      make_hyper(lr, beta1, beta2, eps, wd, step), err, stream);
+  return e == cudaSuccess ? COAT_OK : COAT_ERR_CUDA;
+}

@@ -35,6 +35,7 @@ struct StepHyper {
 };
 
 int sm_count(int dev);
+cudaError_t device_error_ptr(unsigned** out);
 int64_t step_tile_groups();
 
 cudaError_t launch_adamw_single(const TensorArgs& t, int fm, int fv, const StepHyper& h,
@@ -42,6 +43,10 @@ cudaError_t launch_adamw_single(const TensorArgs& t, int fm, int fv, const StepH
 cudaError_t launch_adamw_multi(const TensorArgs* d_descs, const int32_t* d_tile_tensor,
                                int64_t total_tiles, int fm, int fv, const StepHyper& h,
                                unsigned* err, cudaStream_t stream);
+
+cudaError_t launch_adamw_multi_search(const TensorArgs* d_descs, const int64_t* d_tile_begin,
+                                      int num, int64_t total_tiles, int fm, int fv,
+                                      const StepHyper& h, unsigned* err, cudaStream_t stream);
 
 cudaError_t launch_fp8_encode(const float* y, int64_t n, int fmt, uint8_t* q, cudaStream_t s);
 cudaError_t launch_fp8_decode(const uint8_t* q, int64_t n, int fmt, float* out, cudaStream_t s);

@@ -180,6 +180,44 @@ coat_status coat_multi_plan_info(coat_multi_plan_t plan, int64_t *total_elements
                                  int *num_tensors);
 
 /* ---------------------------------------------------------------------------
+ * No-allocation variant of the multi-tensor step.  The COAT pages have no
+ * counterpart: this is a deployment convenience of this library.
+ *
+ * Some callers cannot call cudaMalloc: code that runs inside a framework whose
+ * caching allocator must own all device memory (a raw allocation would bypass
+ * its accounting and may fail under its reservations), or code that must not
+ * allocate once set up (a cudaMalloc can synchronise the device and stall a
+ * latency-sensitive loop).  coat_adamw_step_multi_noalloc applies the same
+ * step as coat_multi_plan_create + coat_adamw_step_multi (identical results),
+ * but keeps the tensor table in a fixed array inside the library's device
+ * image instead of a cudaMalloc'd plan table.  It allocates nothing: no
+ * cudaMalloc/cudaFree, no allocating library routine, no heap use.
+ *
+ *   - host_descs: num descriptors in host memory (read during the call; the
+ *     caller may free them on return).  Each obeys the coat_adamw_step rules.
+ *   - num: 1 .. COAT_NOALLOC_MAX_TENSORS.  A larger num returns
+ *     COAT_ERR_UNSUPPORTED (as does group != 128); other bad arguments return
+ *     COAT_ERR_INVALID_ARG or COAT_ERR_MISALIGNED, before anything is enqueued.
+ *     This call reports through its return code only: it does not record a
+ *     message, so coat_last_error() keeps describing an earlier failure.
+ *   - The fixed array holds COAT_NOALLOC_MAX_TENSORS descriptors plus their
+ *     first-tile indices (about 106 KB); every GPU that loads the library keeps
+ *     it until the process exits.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and configures the kernel; make that first call
+ *     before any stream capture.
+ *   - Each call copies the table into the array on `stream`, then launches on
+ *     `stream`.  All calls share the one array and it keeps the last call's
+ *     contents: calls that may overlap on the GPU (different streams without
+ *     ordering between them) race on it and must not be issued.
+ * ------------------------------------------------------------------------- */
+#define COAT_NOALLOC_MAX_TENSORS 1024
+coat_status coat_adamw_step_multi_noalloc(const coat_tensor_desc *host_descs, int num, int group,
+                                          float lr, float beta1, float beta2, float eps,
+                                          float wd, int64_t step, coat_fmt fmt_m, coat_fmt fmt_v,
+                                          cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Device error word.  Kernels that wait on a shared-memory barrier give up
  * after a bounded time (about one second), set a flag and return;
  * coat_check_device_error synchronises `stream`, reads and clears the flag,
