@@ -356,15 +356,14 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
     uint32_t cmw[4], cvw[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float xm = m1[4 * j + i], xv = v1[4 * j + i];
-      cmw[i] = enc_signed<FM>(xm, expand_value<FM>(xm, invMm, km));
-      cvw[i] = enc_mag<FV>(expand_value<FV>(xv, invMv, kv));
+      cmw[i] = enc_mag<FM>(expand_value<FM>(m1[4 * j + i], invMm, km));
+      cvw[i] = enc_mag<FV>(expand_value<FV>(v1[4 * j + i], invMv, kv));
     }
     if (FULL || active) {
       *reinterpret_cast<uint32_t*>(t.mq + e) =
-          __byte_perm(__byte_perm(cmw[0], cmw[1], 0x0040), __byte_perm(cmw[2], cmw[3], 0x0040), 0x5410);
-      *reinterpret_cast<uint32_t*>(t.vq + e) =
-          __byte_perm(__byte_perm(cvw[0], cvw[1], 0x0040), __byte_perm(cvw[2], cvw[3], 0x0040), 0x5410);
+          merge_signs4(pack4(cmw[0], cmw[1], cmw[2], cmw[3]), m1[4 * j], m1[4 * j + 1],
+                       m1[4 * j + 2], m1[4 * j + 3]);
+      *reinterpret_cast<uint32_t*>(t.vq + e) = pack4(cvw[0], cvw[1], cvw[2], cvw[3]);
     }
   }
   if ((FULL || active) && l == 0) {

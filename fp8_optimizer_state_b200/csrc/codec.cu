@@ -65,8 +65,7 @@ __device__ __forceinline__ void load4(const void* base, int64_t idx, int valid, 
 
 __device__ __forceinline__ void store_codes4(uint8_t* q, uint32_t c[4], int valid) {
   if (valid >= 4) {
-    *reinterpret_cast<uint32_t*>(q) =
-        __byte_perm(__byte_perm(c[0], c[1], 0x0040), __byte_perm(c[2], c[3], 0x0040), 0x5410);
+    *reinterpret_cast<uint32_t*>(q) = pack4(c[0], c[1], c[2], c[3]);
   } else {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
