@@ -225,7 +225,7 @@ __device__ __forceinline__ double exp2_table(double t, const double* exp2_16) {
 // candidates (their positions packed into the low 8 bits of the comparison
 // keys, at a cost of 2^-16 relative in the ordering) and recomputes them in
 // double precision: dequantisation, then m' = beta1 m + (1 - beta1) g.
-__device__ __forceinline__ float recompute_m_double(const LaneIn& in, int idx,
+__device__ __forceinline__ float recompute_m_double(const LaneIn& in, int idx, double invk,
                                                     const StepHyper& h, const double* tabd_m,
                                                     const double* exp2_16) {
   const int j = idx >> 2, i = idx & 3;
@@ -234,9 +234,6 @@ __device__ __forceinline__ float recompute_m_double(const LaneIn& in, int idx,
   const uint32_t c = (mw >> (8 * i)) & 0xFFu;
   const uint32_t gw = (i < 2) ? gw2.x : gw2.y;
   const float g = (i & 1) ? bf16hi(gw) : bf16lo(gw);
-  const double k = static_cast<double>(in.mk);
-  const double r0 = static_cast<double>(rcp_approx(in.mk));
-  const double invk = r0 * fma(-k, r0, 2.0);   // one Newton step: ~1e-14 relative
   double x = exp2_table(tabd_m[c] * invk, exp2_16) * static_cast<double>(in.ms);
   if (c & 0x80u) x = -x;
   const double b1 = static_cast<double>(h.beta1);
@@ -261,6 +258,10 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
   // dequantisation constants of this group (stored k and root scale)
   const float invk_m = rcp_approx(in.mk), sb_m = in.ms * h.beta1;
   const float invk_v = rcp_approx(in.vk), sb_v = in.vs * h.beta2;
+  // 1/k of the m state in double for the min recompute (one Newton step from
+  // the FP32 reciprocal: ~1e-14 relative)
+  const double kd = static_cast<double>(in.mk), r0 = static_cast<double>(invk_m);
+  const double invk_md = r0 * fma(-kd, r0, 2.0);
 
   float m1[16], v1[16];
   float maxm = 0.f, maxv = 0.f;
@@ -333,16 +334,23 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
   // it; the runner-up is recomputed too when its FP32 key is within about
   // 2^-7 relative of the smallest (a near-tie that the FP32 values, off by up
   // to |beta1 m| / |m'| times their dequantisation error, may misorder)
+  // Every lane recomputes the element at the smallest key's index (only the
+  // owner lane's registers hold that element; the others compute a value that
+  // is discarded), so the common case runs converged; the owner's value is then
+  // broadcast to its 8-lane group.
   const bool any_m = minm1 < 0xFFFFFF00u;
   const bool tie = minm2 < 0xFFFFFF00u && (minm2 >> 8) - (minm1 >> 8) < (1u << 9);
-  float mum = __int_as_float(0x7F800000);
-  if (any_m && static_cast<int>((minm1 >> 5) & 7u) == l)
-    mum = recompute_m_double(in, static_cast<int>(minm1 & 15u), h, S.tabd_m, S.exp2_16);
-  if (tie && static_cast<int>((minm2 >> 5) & 7u) == l)
-    mum = fminf(mum, recompute_m_double(in, static_cast<int>(minm2 & 15u), h, S.tabd_m,
-                                        S.exp2_16));
+  float mum = recompute_m_double(in, static_cast<int>(minm1 & 15u), invk_md, h, S.tabd_m,
+                                 S.exp2_16);
+  mum = __shfl_sync(0xFFFFFFFFu, mum, (slot << 3) | static_cast<int>((minm1 >> 5) & 7u));
+  if (__any_sync(0xFFFFFFFFu, tie)) {
+    float m2 = __int_as_float(0x7F800000);
+    if (tie && static_cast<int>((minm2 >> 5) & 7u) == l)
+      m2 = recompute_m_double(in, static_cast<int>(minm2 & 15u), invk_md, h, S.tabd_m, S.exp2_16);
 #pragma unroll
-  for (int off = 1; off < 8; off <<= 1) mum = fminf(mum, __shfl_xor_sync(0xFFFFFFFFu, mum, off));
+    for (int off = 1; off < 8; off <<= 1) m2 = fminf(m2, __shfl_xor_sync(0xFFFFFFFFu, m2, off));
+    mum = fminf(mum, m2);
+  }
   if (!any_m) mum = 0.f;   // no nonzero element
   const float muv = __uint_as_float(minv + 1u);
   float km, srm, invMm, kv, srv, invMv;
@@ -356,8 +364,8 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
     uint32_t cmw[4], cvw[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      cmw[i] = enc_mag<FM>(expand_value<FM>(m1[4 * j + i], invMm, km));
-      cvw[i] = enc_mag<FV>(expand_value<FV>(v1[4 * j + i], invMv, kv));
+      cmw[i] = enc_mag_bounded<FM>(expand_value<FM>(m1[4 * j + i], invMm, km));
+      cvw[i] = enc_mag_bounded<FV>(expand_value<FV>(v1[4 * j + i], invMv, kv));
     }
     if (FULL || active) {
       *reinterpret_cast<uint32_t*>(t.mq + e) =
