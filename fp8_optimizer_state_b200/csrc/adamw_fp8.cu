@@ -9,16 +9,17 @@
 // the new group max/min, and requantise.
 //
 // Design (HBM-bound: 16.25 algorithmic bytes per parameter, no tensor cores):
-//  * persistent CTAs, 2 per SM, 8 warps each (so that every SM sub-partition
-//    holds 4 warps and a thread may use 128 registers); tiles of 28 groups
-//    (3584 elements);
+//  * one persistent CTA per SM, 16 warps (4 per SM sub-partition, so a thread
+//    may use 128 registers); tiles of 60 groups (7680 elements); every CTA owns
+//    a contiguous range of tiles;
 //  * one producer thread streams whole tiles (master, grad, both code arrays,
-//    the four metadata arrays: 29,120 B) into a 3-stage shared-memory ring
-//    with 1-D cp.async.bulk copies completing on an mbarrier, so that bytes in
-//    flight do not depend on registers.  It keeps the current tensor's
-//    descriptor in registers, prefetches the next tile's tensor index, and
-//    writes the descriptor into the stage header for the consumers;
-//  * 7 consumer warps; each warp owns 4 groups of a tile, 8 lanes per group,
+//    the four metadata arrays: 62,400 B) into a 3-stage shared-memory ring
+//    with 1-D cp.async.bulk copies completing on an mbarrier (30 KB per copy
+//    of the master array), so that bytes in flight do not depend on
+//    registers.  It walks the tensor list forward with its range, keeps the
+//    current tensor's descriptor in registers and writes the tile's array
+//    pointers into the stage header;
+//  * 15 consumer warps; each warp owns 4 groups of a tile, 8 lanes per group,
 //    16 elements per lane in 4 chunks of 4 contiguous elements (chunk order
 //    rotated per group to keep shared-memory reads conflict-free); group
 //    max / min-nonzero by 3 xor-shuffles inside the 8 lanes;
@@ -30,7 +31,8 @@
 //    consumers load from global memory with bounds checks, padding elements
 //    count as zero and their codes are written 0;
 //  * every mbarrier wait is bounded (about a second); on timeout the kernel
-//    sets a device error bit and returns.
+//    sets a device error bit and returns (the producer first waits, bounded,
+//    for the copies it still has in flight).
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -40,34 +42,53 @@
 namespace coat {
 namespace {
 
-constexpr int kConsumerWarps = 7;
+constexpr int kConsumerWarps = 15;
 constexpr int kGroupsPerWarp = 4;
-constexpr int kTileGroups = kConsumerWarps * kGroupsPerWarp;  // 28
-constexpr int kTileElems = kTileGroups * kGroup;               // 3584
+constexpr int kTileGroups = kConsumerWarps * kGroupsPerWarp;  // 60
+constexpr int kTileElems = kTileGroups * kGroup;               // 7680
 constexpr int kStages = 3;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;             // 256
-constexpr int kCtasPerSm = 2;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;             // 512
+constexpr int kCtasPerSm = 1;
 
 // Stage layout (bytes): the element arrays start on 128-byte boundaries, the
-// metadata arrays (112 B each) on 16-byte boundaries; stages are padded to a
+// metadata arrays (240 B each) on 16-byte boundaries; stages are padded to a
 // multiple of 128 bytes.
 constexpr uint32_t kOffMaster = 0;
-constexpr uint32_t kOffGrad = kOffMaster + kTileElems * 4;   // 14336
-constexpr uint32_t kOffMq = kOffGrad + kTileElems * 2;       // 21504
-constexpr uint32_t kOffVq = kOffMq + kTileElems;             // 25088
-constexpr uint32_t kOffMs = kOffVq + kTileElems;             // 28672
+constexpr uint32_t kOffGrad = kOffMaster + kTileElems * 4;   // 30720
+constexpr uint32_t kOffMq = kOffGrad + kTileElems * 2;       // 46080
+constexpr uint32_t kOffVq = kOffMq + kTileElems;             // 53760
+constexpr uint32_t kOffMs = kOffVq + kTileElems;             // 61440
 constexpr uint32_t kOffMk = kOffMs + kTileGroups * 4;
 constexpr uint32_t kOffVs = kOffMk + kTileGroups * 4;
 constexpr uint32_t kOffVk = kOffVs + kTileGroups * 4;
-constexpr uint32_t kTxBytes = kOffVk + kTileGroups * 4;      // 29120 copied per tile
+constexpr uint32_t kTxBytes = kOffVk + kTileGroups * 4;      // 62400 copied per tile
 constexpr uint32_t kStageBytes = ((kTxBytes + 127) / 128) * 128;
 static_assert(kTileElems % 16 == 0 && (kTileGroups * 4) % 16 == 0, "bulk copies need 16-byte sizes");
 
-struct TileHeader {
-  TensorArgs t;     // descriptor of the tile's tensor
-  int64_t g0;       // first group of the tile within its tensor
-  int32_t ngroups;  // groups of this tile that exist
-  int32_t full;     // 1: all 3584 elements valid and staged in shared memory
+// What the lanes need of a tile: its tensor's arrays offset to the tile's
+// first element (and first group, for the per-group arrays), so that a lane
+// addresses everything with its own tile-invariant 32-bit offsets.
+struct __align__(16) TileHeader {
+  float* master;
+  uint16_t* wout;  // null: no bf16 copy
+  uint8_t* mq;
+  uint8_t* vq;
+  float* ms;
+  float* mk;
+  float* vs;
+  float* vk;
+  const uint16_t* grad;
+  int32_t nvalid;   // elements of the tile that exist (kTileElems: full tile, staged)
+  int32_t ngroups;  // groups of the tile that exist
+};
+
+constexpr int64_t kNoTile = 0x7FFFFFFFFFFFFFFFLL;
+
+// The producer's current tensor: its descriptor and where the next one starts.
+struct Feed {
+  TensorArgs d;
+  int64_t next_begin;  // first tile of the next tensor (kNoTile: none)
+  int32_t ti;          // index of the current tensor
 };
 
 struct Smem {
@@ -81,46 +102,38 @@ struct Smem {
 };
 constexpr size_t kSmemHead = ((sizeof(Smem) + 127) / 128) * 128;
 constexpr size_t kSmemBytes = kSmemHead + size_t(kStages) * kStageBytes;
+static_assert(kSmemBytes * kCtasPerSm <= 227 * 1024, "shared memory per SM");
 
-// Tile -> tensor lookup.  Single-tensor launches use one descriptor passed by
-// value; multi-tensor launches use the plan's device tables.
+// Tile -> tensor.  Tensor i owns tiles [tile_begin_i, tile_begin_i + tiles_i),
+// in ascending order; an empty tensor shares the next tensor's first tile.
+// Single-tensor launches pass one descriptor by value.
 struct SingleTensor {
-  static constexpr bool kSingle = true;
   TensorArgs t;
   __device__ __forceinline__ int64_t tiles() const { return t.tiles; }
-  __device__ __forceinline__ int32_t tensor_of(int64_t) const { return 0; }
+  __device__ __forceinline__ int32_t find(int64_t) const { return 0; }
   __device__ __forceinline__ TensorArgs get(int32_t) const { return t; }
+  __device__ __forceinline__ int64_t begin_of(int32_t) const { return kNoTile; }  // no successor
 };
+// Multi-tensor launches read a device table of descriptors; the producer finds
+// the tensor of its first tile by binary search (the last tensor whose first
+// tile is <= the tile, which skips empty tensors) and then walks forward.
 struct MultiTensor {
-  static constexpr bool kSingle = false;
   const TensorArgs* descs;
-  const int32_t* tile_tensor;
-  int64_t total_tiles;
-  __device__ __forceinline__ int64_t tiles() const { return total_tiles; }
-  __device__ __forceinline__ int32_t tensor_of(int64_t tile) const { return __ldg(tile_tensor + tile); }
-  __device__ __forceinline__ TensorArgs get(int32_t i) const { return descs[i]; }
-};
-
-// Multi-tensor launch without a per-tile map: the tile's tensor is found by
-// binary search over the tensors' first tiles (tile_begin[0..num], ascending;
-// empty tensors share the next tensor's first tile and are skipped because the
-// search returns the last tensor whose first tile is <= the tile).
-struct MultiTensorSearch {
-  static constexpr bool kSingle = false;
-  const TensorArgs* descs;
-  const int64_t* tile_begin;
   int32_t num;
   int64_t total_tiles;
   __device__ __forceinline__ int64_t tiles() const { return total_tiles; }
-  __device__ __forceinline__ int32_t tensor_of(int64_t tile) const {
+  __device__ __forceinline__ int32_t find(int64_t tile) const {
     int32_t lo = 0, hi = num - 1;
     while (lo < hi) {
       const int32_t mid = (lo + hi + 1) >> 1;
-      if (tile_begin[mid] <= tile) lo = mid; else hi = mid - 1;
+      if (descs[mid].tile_begin <= tile) lo = mid; else hi = mid - 1;
     }
     return lo;
   }
   __device__ __forceinline__ TensorArgs get(int32_t i) const { return descs[i]; }
+  __device__ __forceinline__ int64_t begin_of(int32_t i) const {
+    return i < num ? descs[i].tile_begin : kNoTile;
+  }
 };
 
 // The 16 elements a lane owns, as loaded.
@@ -133,19 +146,17 @@ struct LaneIn {
 
 __device__ __forceinline__ int chunk_of(int j, int slot) { return (j + slot) & 3; }
 
-__device__ __forceinline__ void load_from_stage(const uint8_t* st, int lg, int slot, int l,
+__device__ __forceinline__ void load_from_stage(const uint8_t* st, const int (&off)[4], int lg,
                                                 LaneIn& in) {
-  const float* sm = reinterpret_cast<const float*>(st + kOffMaster) + lg * kGroup;
-  const uint16_t* sg = reinterpret_cast<const uint16_t*>(st + kOffGrad) + lg * kGroup;
-  const uint8_t* smq = st + kOffMq + lg * kGroup;
-  const uint8_t* svq = st + kOffVq + lg * kGroup;
+  const float* sm = reinterpret_cast<const float*>(st + kOffMaster);
+  const uint16_t* sg = reinterpret_cast<const uint16_t*>(st + kOffGrad);
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const int e = 32 * chunk_of(j, slot) + 4 * l;
+    const int e = off[j];
     in.p[j] = *reinterpret_cast<const float4*>(sm + e);
     in.g[j] = *reinterpret_cast<const uint2*>(sg + e);
-    in.mq[j] = *reinterpret_cast<const uint32_t*>(smq + e);
-    in.vq[j] = *reinterpret_cast<const uint32_t*>(svq + e);
+    in.mq[j] = *reinterpret_cast<const uint32_t*>(st + kOffMq + e);
+    in.vq[j] = *reinterpret_cast<const uint32_t*>(st + kOffVq + e);
   }
   in.ms = reinterpret_cast<const float*>(st + kOffMs)[lg];
   in.mk = reinterpret_cast<const float*>(st + kOffMk)[lg];
@@ -154,45 +165,45 @@ __device__ __forceinline__ void load_from_stage(const uint8_t* st, int lg, int s
 }
 
 // Direct loads for a tile that is not entirely valid.  Elements at or beyond
-// n read as zero; codes of a group that exists are always readable (the code
-// arrays hold whole groups).
-__device__ __forceinline__ void load_direct(const TensorArgs& t, int64_t gi, bool active, int slot,
-                                            int l, LaneIn& in) {
-  const int64_t base = gi * kGroup;
+// the tile's valid count read as zero; codes of a group that exists are always
+// readable (the code arrays hold whole groups).  off[j]: the lane's element
+// offsets within the tile; lg: its group within the tile.
+__device__ __forceinline__ void load_direct(const TileHeader& hd, const int (&off)[4], int lg,
+                                            bool active, LaneIn& in) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const int64_t e = base + 32 * chunk_of(j, slot) + 4 * l;
+    const int e = off[j];
     float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
     uint2 g = make_uint2(0u, 0u);
     uint32_t mq = 0u, vq = 0u;
     if (active) {
-      if (e + 4 <= t.n) {
-        p = *reinterpret_cast<const float4*>(t.master + e);
-        g = *reinterpret_cast<const uint2*>(t.grad + e);
+      if (e + 4 <= hd.nvalid) {
+        p = *reinterpret_cast<const float4*>(hd.master + e);
+        g = *reinterpret_cast<const uint2*>(hd.grad + e);
       } else {
         float pv[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t gv[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          if (e + i < t.n) {
-            pv[i] = t.master[e + i];
-            gv[i] = t.grad[e + i];
+          if (e + i < hd.nvalid) {
+            pv[i] = hd.master[e + i];
+            gv[i] = hd.grad[e + i];
           }
         p = make_float4(pv[0], pv[1], pv[2], pv[3]);
         g = make_uint2(gv[0] | (gv[1] << 16), gv[2] | (gv[3] << 16));
       }
-      mq = *reinterpret_cast<const uint32_t*>(t.mq + e);
-      vq = *reinterpret_cast<const uint32_t*>(t.vq + e);
+      mq = *reinterpret_cast<const uint32_t*>(hd.mq + e);
+      vq = *reinterpret_cast<const uint32_t*>(hd.vq + e);
     }
     in.p[j] = p;
     in.g[j] = g;
     in.mq[j] = mq;
     in.vq[j] = vq;
   }
-  in.ms = active ? t.ms[gi] : 1.f;
-  in.mk = active ? t.mk[gi] : 1.f;
-  in.vs = active ? t.vs[gi] : 1.f;
-  in.vk = active ? t.vk[gi] : 1.f;
+  in.ms = active ? hd.ms[lg] : 1.f;
+  in.mk = active ? hd.mk[lg] : 1.f;
+  in.vs = active ? hd.vs[lg] : 1.f;
+  in.vk = active ? hd.vk[lg] : 1.f;
 }
 
 __device__ __forceinline__ float f4get(const float4& v, int i) {
@@ -251,10 +262,9 @@ __device__ __forceinline__ uint32_t min_key(float x, int idx) {
 // The per-lane body: everything after the loads.  FULL: every element of the
 // tile is valid (no bounds logic).
 template <int FM, int FV, bool FULL>
-__device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, int64_t gi,
-                                        bool active, int slot, int l, const StepHyper& h,
+__device__ __forceinline__ void process(const LaneIn& in, const TileHeader& t, const int (&off)[4],
+                                        int lg, bool active, int slot, int l, const StepHyper& h,
                                         const Smem& S) {
-  const int64_t base = gi * kGroup;
   // dequantisation constants of this group (stored k and root scale)
   const float invk_m = rcp_approx(in.mk), sb_m = in.ms * h.beta1;
   const float invk_v = rcp_approx(in.vk), sb_v = in.vs * h.beta2;
@@ -269,7 +279,7 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
 
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const int64_t e = base + 32 * chunk_of(j, slot) + 4 * l;
+    const int e = off[j];
     float pn[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -285,9 +295,9 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
       float vn = __fmaf_rn(h.omb2 * g, g, bv);
       const float p = f4get(in.p[j], i);
       const float upd = mn * rcp_approx(__fmaf_rn(sqrt_approx(vn), h.dsq, h.deps));
-      pn[i] = p + __fmaf_rn(-p, h.lrwd, h.zero_lr ? 0.f : -upd);
+      pn[i] = p + __fmaf_rn(-p, h.lrwd, -upd);
       if (!FULL) {
-        const bool valid = active && (e + i < t.n);
+        const bool valid = active && (e + i < t.nvalid);
         mn = valid ? mn : 0.f;
         vn = valid ? vn : 0.f;
       }
@@ -295,12 +305,18 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
       v1[4 * j + i] = vn;
       maxm = fmaxf(maxm, fabsf(mn));
       maxv = fmaxf(maxv, vn);
-      const uint32_t key = min_key(mn, 4 * j + i);
-      minm2 = min(minm2, max(minm1, key));
-      minm1 = min(minm1, key);
       minv = min(minv, __float_as_uint(vn) - 1u);
     }
-    if (FULL || (active && e + 4 <= t.n)) {
+    // two smallest m keys: merge the sorted pairs of elements (0,1), (2,3)
+#pragma unroll
+    for (int i = 0; i < 4; i += 2) {
+      const uint32_t ka = min_key(m1[4 * j + i], 4 * j + i);
+      const uint32_t kb = min_key(m1[4 * j + i + 1], 4 * j + i + 1);
+      const uint32_t lo = min(ka, kb), hi = max(ka, kb);
+      minm2 = min(max(minm1, lo), min(minm2, hi));
+      minm1 = min(minm1, lo);
+    }
+    if (FULL || (active && e + 4 <= t.nvalid)) {
       *reinterpret_cast<float4*>(t.master + e) = make_float4(pn[0], pn[1], pn[2], pn[3]);
       if (t.wout)
         *reinterpret_cast<uint2*>(t.wout + e) =
@@ -308,7 +324,7 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
     } else if (active) {
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        if (e + i < t.n) {
+        if (e + i < t.nvalid) {
           t.master[e + i] = pn[i];
           if (t.wout) t.wout[e + i] = static_cast<uint16_t>(pack_bf16x2(pn[i], 0.f));
         }
@@ -353,14 +369,23 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
   }
   if (!any_m) mum = 0.f;   // no nonzero element
   const float muv = __uint_as_float(minv + 1u);
-  float km, srm, invMm, kv, srv, invMv;
-  group_params<FM>(maxm, mum, true, km, srm, invMm);
-  group_params<FV>(maxv, muv, true, kv, srv, invMv);
+  // lanes 0-3 of the group derive the m parameters, lanes 4-7 the v ones;
+  // then every lane takes k and 1/M of both moments from lanes 0 and 4
+  const bool vlane = l >= 4;
+  float kx, srx, invMx;
+  group_params_rt(vlane ? maxv : maxm, vlane ? muv : mum, true,
+                  vlane ? F8<FV>::LOG2MAX_HI : F8<FM>::LOG2MAX_HI,
+                  vlane ? F8<FV>::LOG2MAX_LO : F8<FM>::LOG2MAX_LO, kx, srx, invMx);
+  const int lane_m = slot << 3, lane_v = lane_m + 4;
+  const float km = __shfl_sync(0xFFFFFFFFu, kx, lane_m);
+  const float invMm = __shfl_sync(0xFFFFFFFFu, invMx, lane_m);
+  const float kv = __shfl_sync(0xFFFFFFFFu, kx, lane_v);
+  const float invMv = __shfl_sync(0xFFFFFFFFu, invMx, lane_v);
 
   // expand + encode, store codes (whole group, padding included) and metadata
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const int64_t e = base + 32 * chunk_of(j, slot) + 4 * l;
+    const int e = off[j];
     uint32_t cmw[4], cvw[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -374,11 +399,63 @@ __device__ __forceinline__ void process(const LaneIn& in, const TensorArgs& t, i
       *reinterpret_cast<uint32_t*>(t.vq + e) = pack4(cvw[0], cvw[1], cvw[2], cvw[3]);
     }
   }
-  if ((FULL || active) && l == 0) {
-    t.ms[gi] = srm;
-    t.mk[gi] = km;
-    t.vs[gi] = srv;
-    t.vk[gi] = kv;
+  if ((FULL || active) && (l & 3) == 0) {
+    (vlane ? t.vs : t.ms)[lg] = srx;
+    (vlane ? t.vk : t.mk)[lg] = kx;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// The producer thread stages the CTA's tiles.
+// ---------------------------------------------------------------------------
+template <class Map>
+__device__ __forceinline__ void feed_start(const Map& map, Feed& f, int64_t tile) {
+  const int32_t ti = map.find(tile);
+  f.ti = ti;
+  f.d = map.get(ti);
+  f.next_begin = map.begin_of(ti + 1);
+}
+
+// Stage `tile` into `st` (header into `hd`), completing on `bar`: a fully
+// valid tile is copied (kTxBytes of transaction), any other tile only arrives
+// and is read from global memory by the lanes.
+template <class Map>
+__device__ __forceinline__ void feed_issue(const Map& map, Feed& f, int64_t tile, uint8_t* st,
+                                           TileHeader& hd, uint64_t* bar) {
+  while (tile >= f.next_begin) {
+    const int32_t ti = ++f.ti;
+    f.d = map.get(ti);
+    f.next_begin = map.begin_of(ti + 1);
+  }
+  const TensorArgs& ct = f.d;
+  const int64_t g0 = (tile - ct.tile_begin) * kTileGroups;
+  const int64_t groups = (ct.n + kGroup - 1) / kGroup;
+  const int64_t ng = (groups - g0) < kTileGroups ? (groups - g0) : int64_t(kTileGroups);
+  const int64_t e0 = g0 * kGroup;
+  const bool full = (e0 + kTileElems <= ct.n);
+  hd.master = ct.master + e0;
+  hd.wout = ct.wout ? ct.wout + e0 : nullptr;
+  hd.mq = ct.mq + e0;
+  hd.vq = ct.vq + e0;
+  hd.ms = ct.ms + g0;
+  hd.mk = ct.mk + g0;
+  hd.vs = ct.vs + g0;
+  hd.vk = ct.vk + g0;
+  hd.grad = ct.grad + e0;
+  hd.nvalid = full ? kTileElems : static_cast<int32_t>(ct.n - e0);
+  hd.ngroups = static_cast<int32_t>(ng);
+  if (full) {
+    mbar_arrive_expect_tx(bar, kTxBytes);
+    bulk_g2s(st + kOffMaster, ct.master + e0, kTileElems * 4, bar);
+    bulk_g2s(st + kOffGrad, ct.grad + e0, kTileElems * 2, bar);
+    bulk_g2s(st + kOffMq, ct.mq + e0, kTileElems, bar);
+    bulk_g2s(st + kOffVq, ct.vq + e0, kTileElems, bar);
+    bulk_g2s(st + kOffMs, ct.ms + g0, kTileGroups * 4, bar);
+    bulk_g2s(st + kOffMk, ct.mk + g0, kTileGroups * 4, bar);
+    bulk_g2s(st + kOffVs, ct.vs + g0, kTileGroups * 4, bar);
+    bulk_g2s(st + kOffVk, ct.vk + g0, kTileGroups * 4, bar);
+  } else {
+    mbar_arrive(bar);
   }
 }
 
@@ -404,22 +481,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // this CTA's contiguous share of the tiles
   const int64_t ntiles = map.tiles();
+  const int64_t t0 = int64_t(blockIdx.x) * ntiles / gridDim.x;
+  const int64_t t1 = int64_t(blockIdx.x + 1) * ntiles / gridDim.x;
 
   if (warp == kConsumerWarps) {
     // ---------------- producer ----------------
-    if (lane != 0) return;
-    int32_t cur = -1;
-    TensorArgs ct{};
-    int32_t next_ti = blockIdx.x < ntiles ? map.tensor_of(blockIdx.x) : 0;
+    if (lane != 0 || t0 >= t1) return;
+    Feed f;
+    feed_start(map, f, t0);
     int64_t it = 0;
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
-      const int32_t ti = next_ti;
-      if (tile + gridDim.x < ntiles) next_ti = map.tensor_of(tile + gridDim.x);  // prefetch
-      if (ti != cur) {
-        ct = map.get(ti);
-        cur = ti;
-      }
+    for (int64_t tile = t0; tile < t1; ++tile, ++it) {
       const int s = static_cast<int>(it % kStages);
       const uint32_t use = static_cast<uint32_t>(it / kStages);
       if (use > 0 && !mbar_wait(&S.empty_bar[s], (use - 1) & 1u, kWaitBudgetCycles)) {
@@ -435,30 +508,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         }
         return;
       }
-      const int64_t g0 = (tile - ct.tile_begin) * kTileGroups;
-      const int64_t groups = (ct.n + kGroup - 1) / kGroup;
-      const int64_t ng = (groups - g0) < kTileGroups ? (groups - g0) : int64_t(kTileGroups);
-      const int64_t e0 = g0 * kGroup;
-      const bool full = (e0 + kTileElems <= ct.n);
-      TileHeader& hd = S.hdr[s];
-      if (!Map::kSingle) hd.t = ct;
-      hd.g0 = g0;
-      hd.ngroups = static_cast<int32_t>(ng);
-      hd.full = full ? 1 : 0;
-      if (full) {
-        uint8_t* st = stages + size_t(s) * kStageBytes;
-        mbar_arrive_expect_tx(&S.full_bar[s], kTxBytes);
-        bulk_g2s(st + kOffMaster, ct.master + e0, kTileElems * 4, &S.full_bar[s]);
-        bulk_g2s(st + kOffGrad, ct.grad + e0, kTileElems * 2, &S.full_bar[s]);
-        bulk_g2s(st + kOffMq, ct.mq + e0, kTileElems, &S.full_bar[s]);
-        bulk_g2s(st + kOffVq, ct.vq + e0, kTileElems, &S.full_bar[s]);
-        bulk_g2s(st + kOffMs, ct.ms + g0, kTileGroups * 4, &S.full_bar[s]);
-        bulk_g2s(st + kOffMk, ct.mk + g0, kTileGroups * 4, &S.full_bar[s]);
-        bulk_g2s(st + kOffVs, ct.vs + g0, kTileGroups * 4, &S.full_bar[s]);
-        bulk_g2s(st + kOffVk, ct.vk + g0, kTileGroups * 4, &S.full_bar[s]);
-      } else {
-        mbar_arrive(&S.full_bar[s]);
-      }
+      feed_issue(map, f, tile, stages + size_t(s) * kStageBytes, S.hdr[s], &S.full_bar[s]);
     }
     return;
   }
@@ -466,30 +516,34 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   // ---------------- consumers ----------------
   const int slot = lane >> 3, l = lane & 7;
   const int lg = warp * kGroupsPerWarp + slot;  // group within the tile
+  // the lane's elements: 4 chunks of 4, chunk j at 32 chunk_of(j, slot) + 4 l
+  // within its group
+  int off[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) off[j] = lg * kGroup + 32 * chunk_of(j, slot) + 4 * l;
   int64_t it = 0;
-  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+  for (int64_t tile = t0; tile < t1; ++tile, ++it) {
     const int s = static_cast<int>(it % kStages);
     const uint32_t use = static_cast<uint32_t>(it / kStages);
-    if (!mbar_wait(&S.full_bar[s], use & 1u, kWaitBudgetCycles)) {
-      atomicOr(err, kErrTimeoutConsumer);
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(&S.full_bar[s], use & 1u, kWaitBudgetCycles))) {
+      if (lane == 0) atomicOr(err, kErrTimeoutConsumer);
       return;
     }
-    const TileHeader& hd = S.hdr[s];
-    const TensorArgs t = Map::kSingle ? map.get(0) : hd.t;
-    const int64_t gi = hd.g0 + lg;
-    const bool full = hd.full != 0;
-    const bool active = lg < hd.ngroups;
+    // the header is copied to registers before the stage is released
+    const TileHeader t = S.hdr[s];
+    const bool full = t.nvalid == kTileElems;
+    const bool active = lg < t.ngroups;
     LaneIn in;
     if (full)
-      load_from_stage(stages + size_t(s) * kStageBytes, lg, slot, l, in);
+      load_from_stage(stages + size_t(s) * kStageBytes, off, lg, in);
     else
-      load_direct(t, gi, active, slot, l, in);
+      load_direct(t, off, lg, active, in);
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.empty_bar[s]);
     if (full)
-      process<FM, FV, true>(in, t, gi, true, slot, l, h, S);
+      process<FM, FV, true>(in, t, off, lg, true, slot, l, h, S);
     else
-      process<FM, FV, false>(in, t, gi, active, slot, l, h, S);
+      process<FM, FV, false>(in, t, off, lg, active, slot, l, h, S);
   }
 }
 
@@ -533,21 +587,9 @@ cudaError_t launch_adamw_single(const TensorArgs& t, int fm, int fv, const StepH
   return dispatch(fm, fv, map, t.tiles, h, err, stream);
 }
 
-cudaError_t launch_adamw_multi(const TensorArgs* d_descs, const int32_t* d_tile_tensor,
-                               int64_t total_tiles, int fm, int fv, const StepHyper& h,
-                               unsigned* err, cudaStream_t stream) {
-  MultiTensor map{d_descs, d_tile_tensor, total_tiles};
-  return dispatch(fm, fv, map, total_tiles, h, err, stream);
-}
-
-}  // namespace coat
-
-namespace coat {
-
-cudaError_t launch_adamw_multi_search(const TensorArgs* d_descs, const int64_t* d_tile_begin,
-                                      int num, int64_t total_tiles, int fm, int fv,
-                                      const StepHyper& h, unsigned* err, cudaStream_t stream) {
-  MultiTensorSearch map{d_descs, d_tile_begin, num, total_tiles};
+cudaError_t launch_adamw_multi(const TensorArgs* d_descs, int num, int64_t total_tiles, int fm,
+                               int fv, const StepHyper& h, unsigned* err, cudaStream_t stream) {
+  MultiTensor map{d_descs, num, total_tiles};
   return dispatch(fm, fv, map, total_tiles, h, err, stream);
 }
 

@@ -2,6 +2,7 @@
 // any CUDA call, so a bad call launches nothing and touches nothing), error
 // reporting, multi-tensor plans, and kernel launches on the caller's stream.
 #include <cmath>
+#include <limits>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -110,9 +111,17 @@ coat::StepHyper make_hyper(float lr, float beta1, float beta2, float eps, float 
   h.omb1 = static_cast<float>(1.0 - b1);
   h.omb2 = static_cast<float>(1.0 - b2);
   const double dlr = lr;
-  h.zero_lr = lr == 0.f ? 1 : 0;
-  h.dsq = h.zero_lr ? 1.f : static_cast<float>(bc1 / (dlr * std::sqrt(bc2)));
-  h.deps = h.zero_lr ? 1.f : static_cast<float>(static_cast<double>(eps) * bc1 / dlr);
+  const float dsq = static_cast<float>(bc1 / (dlr * std::sqrt(bc2)));
+  const float deps = static_cast<float>(static_cast<double>(eps) * bc1 / dlr);
+  if (lr == 0.f || !std::isfinite(dsq) || !std::isfinite(deps)) {
+    // No adaptive term (lr = 0, or lr so small that lr / (1 - beta1^t) is below
+    // FP32 range): 1 / (sqrt(v') 0 + inf) = 0 makes the kernel's update zero.
+    h.dsq = 0.f;
+    h.deps = std::numeric_limits<float>::infinity();
+  } else {
+    h.dsq = dsq;
+    h.deps = deps;
+  }
   h.lrwd = static_cast<float>(dlr * static_cast<double>(wd));
   return h;
 }
@@ -260,8 +269,7 @@ coat_status coat_adamw_step(float* master, uint16_t* weight_bf16_out, const uint
 }  // extern "C"
 
 struct coat_multi_plan {
-  coat::TensorArgs* d_descs = nullptr;  // one allocation: descriptors, then tile->tensor map
-  int32_t* d_tile_tensor = nullptr;
+  coat::TensorArgs* d_descs = nullptr;  // device copy of the descriptors (tile_begin ascending)
   int64_t total_tiles = 0;
   int64_t total_elements = 0;
   int num = 0;
@@ -290,18 +298,13 @@ coat_status coat_multi_plan_create(const coat_tensor_desc* host_descs, int num, 
     tiles += descs[i].tiles;
     elems += host_descs[i].n;
   }
-  if (tiles >= (int64_t(1) << 31)) return fail(COAT_ERR_UNSUPPORTED, "%s: too many tiles", fn);
-  std::vector<int32_t> map(static_cast<size_t>(tiles > 0 ? tiles : 1));
-  for (int i = 0; i < num; ++i)
-    for (int64_t t = 0; t < descs[i].tiles; ++t) map[descs[i].tile_begin + t] = i;
 
   coat_multi_plan* p = new (std::nothrow) coat_multi_plan;
   if (!p) return fail(COAT_ERR_NOMEM, "%s: host allocation failed", fn);
-  const size_t desc_bytes = ((sizeof(coat::TensorArgs) * num + 255) / 256) * 256;
-  const size_t map_bytes = sizeof(int32_t) * map.size();
+  const size_t desc_bytes = sizeof(coat::TensorArgs) * num;
   void* mem = nullptr;
   cudaError_t e = cudaGetDevice(&p->device);
-  if (e == cudaSuccess) e = cudaMalloc(&mem, desc_bytes + map_bytes);
+  if (e == cudaSuccess) e = cudaMalloc(&mem, desc_bytes);
   if (e != cudaSuccess) {
     delete p;
     cudaGetLastError();
@@ -309,12 +312,8 @@ coat_status coat_multi_plan_create(const coat_tensor_desc* host_descs, int num, 
                                           : cuda_fail(e, fn);
   }
   p->d_descs = static_cast<coat::TensorArgs*>(mem);
-  p->d_tile_tensor = reinterpret_cast<int32_t*>(static_cast<char*>(mem) + desc_bytes);
-  e = cudaMemcpyAsync(p->d_descs, descs.data(), sizeof(coat::TensorArgs) * num,
-                      cudaMemcpyHostToDevice, stream);
-  if (e == cudaSuccess)
-    e = cudaMemcpyAsync(p->d_tile_tensor, map.data(), map_bytes, cudaMemcpyHostToDevice, stream);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);  // host vectors die on return
+  e = cudaMemcpyAsync(p->d_descs, descs.data(), desc_bytes, cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);  // the host vector dies on return
   if (e != cudaSuccess) {
     cudaFree(mem);
     delete p;
@@ -338,7 +337,7 @@ coat_status coat_adamw_step_multi(coat_multi_plan_t plan, float lr, float beta1,
   unsigned* err = nullptr;
   cudaError_t e = coat::device_error_ptr(&err);
   if (e != cudaSuccess) return cuda_fail(e, "coat_adamw_step_multi");
-  e = coat::launch_adamw_multi(plan->d_descs, plan->d_tile_tensor, plan->total_tiles, plan->fmt_m,
+  e = coat::launch_adamw_multi(plan->d_descs, plan->num, plan->total_tiles, plan->fmt_m,
                                plan->fmt_v, make_hyper(lr, beta1, beta2, eps, wd, step), err, stream);
   return e == cudaSuccess ? COAT_OK : cuda_fail(e, "coat_adamw_step_multi");
 }
@@ -382,7 +381,6 @@ namespace {
 
 struct NoAllocScratch {
   coat::TensorArgs descs[COAT_NOALLOC_MAX_TENSORS];
-  int64_t tile_begin[COAT_NOALLOC_MAX_TENSORS + 1];
 };
 
 // Every GPU that loads the library holds this array until the process exits.
@@ -450,7 +448,6 @@ extern "C" coat_status coat_adamw_step_multi_noalloc(const coat_tensor_desc* hos
   // source has been read, so the buffer can be reused at once).
   constexpr int kChunk = 32;
   coat::TensorArgs buf[kChunk];
-  int64_t begins[kChunk];
   int64_t tiles = 0;
   const int64_t tg = coat::step_tile_groups();
   for (int c0 = 0; c0 < num; c0 += kChunk) {
@@ -470,18 +467,15 @@ extern "C" coat_status coat_adamw_step_multi_noalloc(const coat_tensor_desc* hos
       t.n = d.n;
       t.tiles = ((d.n + 127) / 128 + tg - 1) / tg;
       t.tile_begin = tiles;
-      begins[j] = tiles;
       tiles += t.tiles;
     }
     if (cudaMemcpyAsync(scratch->descs + c0, buf, sizeof(coat::TensorArgs) * cn,
-                        cudaMemcpyHostToDevice, stream) != cudaSuccess ||
-        cudaMemcpyAsync(scratch->tile_begin + c0, begins, sizeof(int64_t) * cn,
                         cudaMemcpyHostToDevice, stream) != cudaSuccess)
       return COAT_ERR_CUDA;
   }
   if (tiles == 0) return COAT_OK;
-  const cudaError_t e = coat::launch_adamw_multi_search(
-      scratch->descs, scratch->tile_begin, num, tiles, fmt_m, fmt_v,
-      make_hyper(lr, beta1, beta2, eps, wd, step), err, stream);
+  const cudaError_t e =
+      coat::launch_adamw_multi(scratch->descs, num, tiles, fmt_m, fmt_v,
+                               make_hyper(lr, beta1, beta2, eps, wd, step), err, stream);
   return e == cudaSuccess ? COAT_OK : COAT_ERR_CUDA;
 }

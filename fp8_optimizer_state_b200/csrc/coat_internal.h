@@ -28,10 +28,9 @@ struct TensorArgs {
 // p - (lr / (1-beta1^t)) m' / (sqrt(v') / sqrt(1-beta2^t) + eps).
 struct StepHyper {
   float beta1, beta2, omb1, omb2;
-  float dsq;        // (1 - beta1^t) / (lr sqrt(1 - beta2^t))
-  float deps;       // eps (1 - beta1^t) / lr
+  float dsq;        // (1 - beta1^t) / (lr sqrt(1 - beta2^t)); 0 when lr = 0
+  float deps;       // eps (1 - beta1^t) / lr; +inf when lr = 0
   float lrwd;       // lr * wd
-  int zero_lr;      // lr == 0: the adaptive term is 0
 };
 
 int sm_count(int dev);
@@ -40,13 +39,10 @@ int64_t step_tile_groups();
 
 cudaError_t launch_adamw_single(const TensorArgs& t, int fm, int fv, const StepHyper& h,
                                 unsigned* err, cudaStream_t stream);
-cudaError_t launch_adamw_multi(const TensorArgs* d_descs, const int32_t* d_tile_tensor,
-                               int64_t total_tiles, int fm, int fv, const StepHyper& h,
-                               unsigned* err, cudaStream_t stream);
-
-cudaError_t launch_adamw_multi_search(const TensorArgs* d_descs, const int64_t* d_tile_begin,
-                                      int num, int64_t total_tiles, int fm, int fv,
-                                      const StepHyper& h, unsigned* err, cudaStream_t stream);
+// d_descs: num descriptors in device memory, tile_begin ascending (an empty
+// tensor shares the next tensor's first tile); total_tiles: sum of tiles.
+cudaError_t launch_adamw_multi(const TensorArgs* d_descs, int num, int64_t total_tiles, int fm,
+                               int fv, const StepHyper& h, unsigned* err, cudaStream_t stream);
 
 cudaError_t launch_fp8_encode(const float* y, int64_t n, int fmt, uint8_t* q, cudaStream_t s);
 cudaError_t launch_fp8_decode(const uint8_t* q, int64_t n, int fmt, float* out, cudaStream_t s);

@@ -200,9 +200,9 @@ coat_status coat_multi_plan_info(coat_multi_plan_t plan, int64_t *total_elements
  *     COAT_ERR_INVALID_ARG or COAT_ERR_MISALIGNED, before anything is enqueued.
  *     This call reports through its return code only: it does not record a
  *     message, so coat_last_error() keeps describing an earlier failure.
- *   - The fixed array holds COAT_NOALLOC_MAX_TENSORS descriptors plus their
- *     first-tile indices (about 106 KB); every GPU that loads the library keeps
- *     it until the process exits.
+ *   - The fixed array holds COAT_NOALLOC_MAX_TENSORS kernel descriptors
+ *     (96 KB); every GPU that loads the library keeps it until the process
+ *     exits.
  *   - The first call on a device looks up the array's device address (with
  *     that device current) and configures the kernel; make that first call
  *     before any stream capture.

@@ -4,8 +4,9 @@ handed out as FP32 values for the caller to quantise with its own codec.
 
 Layout: one allocation per stream (master f32, grad bf16, weight bf16, m codes,
 v codes, and four per-group metadata arrays).  Tensor i starts at element
-offset off[i], a multiple of 128, so every tensor pointer is 16-byte aligned and
-its groups start at group offset off[i] / 128.
+offset off[i], a multiple of 512, so its groups start at group offset
+off[i] / 128, a multiple of 4, and every pointer of the tensor (element and
+per-group arrays alike) is 16-byte aligned.
 """
 from __future__ import annotations
 
@@ -20,7 +21,7 @@ class DeviceParamSet:
         self.names = [s[0] for s in shapes]
         self.sizes = [int(s[1]) for s in shapes]
         self.seed = seed
-        padded = [-(-n // 128) * 128 for n in self.sizes]
+        padded = [-(-n // 512) * 512 for n in self.sizes]
         self.off = np.concatenate([[0], np.cumsum(padded)]).astype(np.int64)
         total = int(self.off[-1])
         self.total_elements = sum(self.sizes)
