@@ -38,9 +38,10 @@ UNIT = "Gparams/s"
 HBM_FALLBACK_GBS = 6650.0
 KERNEL_SOURCES = ["fp8_optimizer_state_b200/csrc/adamw_fp8.cu",
                   "fp8_optimizer_state_b200/csrc/coat_device.cuh"]
-# DRAM bytes per launch of the step kernel from an ncu capture (see profiles/),
-# valid only for the kernel sources with this hash.
-TRAFFIC = {"sources_sha256": None, "bytes_per_param": None}
+# DRAM bytes (read + write) per parameter of the step kernel from an ncu
+# capture on a 268,435,456-parameter tensor (profiles/), scaled to a launch by
+# its parameter count; valid only for the kernel sources with this hash.
+TRAFFIC = {"sources_sha256": "fe808d2e5e9fdb4d", "bytes_per_param": 16.053}
 
 
 def kernel_hash():
