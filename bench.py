@@ -221,22 +221,12 @@ def barrier(ws, device):
 # ----------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------
-def run_ours(args, cfg, ws, rank, local):
+def make_workload(shapes, cfg, seed, coat):
+    """Device-resident parameter set with warm-started states (each moment's FP32
+    warm-start values quantised by the library's codec) and its multi-tensor plan."""
     import torch
-    import fp8_optimizer_state_b200 as coat
-    from synth.params import HYPER as H
     from synth.workload import DeviceParamSet
-
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if ws > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    coat.lib()
-
-    shapes = cfg["shapes"]()
-    ps = DeviceParamSet(shapes, seed=rank)
+    ps = DeviceParamSet(shapes, seed=seed)
     ps.fill_master()
     ps.fill_grad(1)
     tmp = None
@@ -258,6 +248,39 @@ def run_ours(args, cfg, ws, rank, local):
                                     v["vq"], v["vs"], v["vk"]))
     plan = coat.coat_multi_plan_create(descs, cfg["fmt_m"], cfg["fmt_v"])
     torch.cuda.synchronize()
+    return ps, plan
+
+
+def time_plan(plan, steps, warmup, H, coat, first_step=1):
+    """Mean device time (ms) per step of `steps` steps after `warmup` untimed ones."""
+    import torch
+    for t in range(warmup):
+        coat.coat_adamw_step_multi(plan, step=first_step + t, **H)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for t in range(steps):
+        coat.coat_adamw_step_multi(plan, step=first_step + warmup + t, **H)
+    b.record()
+    torch.cuda.synchronize()
+    coat.coat_check_device_error()
+    return a.elapsed_time(b) / steps
+
+
+def run_ours(args, cfg, ws, rank, local):
+    import torch
+    import fp8_optimizer_state_b200 as coat
+    from synth.params import HYPER as H
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    coat.lib()
+
+    ps, plan = make_workload(cfg["shapes"](), cfg, rank, coat)
 
     stream = torch.cuda.current_stream()
     step_no = [0]
@@ -304,6 +327,7 @@ def run_ours(args, cfg, ws, rank, local):
     elapsed_ms = max_over_ranks(elapsed_ms, ws, dev)
     kernel_ms = max_over_ranks(statistics.mean(launch_ms), ws, dev)
     n_params = ps.total_elements
+    n_tensors = len(ps)
     value = ws * n_params * args.steps / (elapsed_ms * 1e-3) / 1e9
 
     # roofline of the step kernel
@@ -330,6 +354,22 @@ def run_ours(args, cfg, ws, rank, local):
         e2e = run_e2e(args, cfg, ps, ws, dev, H, coat)
 
     plan.destroy()
+    # many-tensor launch overhead: the same parameter count as one flat tensor
+    vs_flat = None
+    if n_tensors > 1 and args.compare_flat:
+        n_total = ps.total_elements
+        del ps
+        torch.cuda.empty_cache()
+        fps, fplan = make_workload([("flat", n_total)], cfg, rank, coat)
+        flat_ms = max_over_ranks(time_plan(fplan, args.steps, args.warmup, H, coat), ws, dev)
+        fplan.destroy()
+        del fps
+        torch.cuda.empty_cache()
+        flat_value = ws * n_total / (flat_ms * 1e-3) / 1e9
+        vs_flat = {"flat_value": round(flat_value, 3), "unit": UNIT,
+                   "flat_ms_per_step": round(flat_ms, 4), "ratio": round(value / flat_value, 4),
+                   "how": "the same parameter count as one flat tensor, same formats and "
+                          "hyperparameters, device events around the same number of steps"}
     result = None
     if rank == 0:
         cpu = None
@@ -346,7 +386,7 @@ def run_ours(args, cfg, ws, rank, local):
             "ms_per_step": round(elapsed_ms / args.steps, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": cfg["workload"], "params_per_gpu": n_params,
-                       "tensors": len(ps), "group": 128,
+                       "tensors": n_tensors, "group": 128,
                        "fmt_m": "E4M3" if cfg["fmt_m"] == 0 else "E5M2",
                        "fmt_v": "E4M3" if cfg["fmt_v"] == 0 else "E5M2",
                        "hyper": H, "l2": "no flush: %.1f GB of inputs per step >> 126 MB L2"
@@ -356,6 +396,8 @@ def run_ours(args, cfg, ws, rank, local):
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps, "clocks": clocks,
         }
+        if vs_flat is not None:
+            result["vs_flat_tensor"] = vs_flat
     if ws > 1:
         import torch.distributed as dist
         dist.barrier(device_ids=[local])
@@ -420,6 +462,179 @@ def run_e2e(args, cfg, ps, ws, dev, H, coat):
             "gpu_launches_per_step": sum(1 for v in views if v["n"] > 0)}
 
 
+# ----------------------------------------------------------------------------
+# the mixed-granularity codec workload: activations bf16 [8192 x 4096] with 1x128
+# per-token groups and weights bf16 [4096 x 11008] with 128x128 blocks, to E4M3,
+# expansion off and on, then the dequantisation round trip to bf16
+# ----------------------------------------------------------------------------
+CODEC_METRIC = "GB/s of the FP8 group codec (quantize + dequantize); HBM GB/s as % of B200 roofline"
+CODEC_ACT = (8192, 4096)
+CODEC_W = (4096, 11008)
+
+
+def codec_bytes(rows, cols, gr, gc):
+    """Algorithmic bytes of one quantize (bf16 in, codes + scale + k out) or one
+    dequantize (codes + scale + k in, bf16 out): 3 B per element + 8 B per group."""
+    groups = -(-rows // gr) * -(-cols // gc)
+    return 3 * rows * cols + 8 * groups
+
+
+def run_codec(args, ws, rank, local):
+    import torch
+    import fp8_optimizer_state_b200 as coat
+    import synth
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    coat.lib()
+    E4M3 = 0
+    shapes = {"act": (CODEC_ACT, 1, 128), "w": (CODEC_W, 128, 128)}
+    bufs = {}
+    for name, ((r, c), gr, gc) in shapes.items():
+        x = torch.empty(r, c, dtype=torch.bfloat16, device=dev)
+        (synth.device_activations if name == "act" else synth.device_weight)(
+            x.view(torch.int16).view(-1), rank, 0)
+        nbr, nbc = -(-r // gr), -(-c // gc)
+        bufs[name] = dict(x=x, q=torch.empty(r, c, dtype=torch.uint8, device=dev),
+                          s=torch.empty(nbr, nbc, dtype=torch.float32, device=dev),
+                          k=torch.empty(nbr, nbc, dtype=torch.float32, device=dev),
+                          out=torch.empty(r, c, dtype=torch.bfloat16, device=dev), gr=gr, gc=gc)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
+
+    # the launches of one step, in order: (label, bytes, callable)
+    def launches():
+        out = []
+        for expand in (False, True):
+            for name in ("act", "w"):
+                b = bufs[name]
+                out.append(("quantize %s %dx%d expand=%s" % (name, b["gr"], b["gc"], expand),
+                            codec_bytes(*b["x"].shape, b["gr"], b["gc"]),
+                            (lambda b=b, e=expand: coat.coat_group_quantize(
+                                b["x"], b["gr"], b["gc"], e, E4M3, b["q"], b["s"], b["k"]))))
+        for name in ("act", "w"):
+            b = bufs[name]
+            out.append(("dequantize %s %dx%d" % (name, b["gr"], b["gc"]),
+                        codec_bytes(*b["x"].shape, b["gr"], b["gc"]),
+                        (lambda b=b: coat.coat_group_dequantize(b["q"], b["s"], b["k"], b["gr"],
+                                                                b["gc"], E4M3, b["out"]))))
+        return out
+
+    L = launches()
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        for _, _, f in L:
+            flush.fill_(1)
+            f()
+    torch.cuda.synchronize()
+    coat.coat_check_device_error()
+    props = torch.cuda.get_device_properties(dev)
+    bus = "%08x:%02x:%02x.0" % (int(getattr(props, "pci_domain_id", 0)),
+                                int(getattr(props, "pci_bus_id", 0)),
+                                int(getattr(props, "pci_device_id", 0)))
+    sampler = ClockSampler(bus)
+    sampler.start()
+    time.sleep(0.3)
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in L] for _ in range(args.steps)]
+    barrier(ws, dev)
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    for i in range(args.steps):
+        for j, (_, _, f) in enumerate(L):
+            flush.fill_(1)   # L2 flush between timed launches (not timed)
+            ev[i][j][0].record(stream)
+            f()
+            ev[i][j][1].record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    barrier(ws, dev)
+    time.sleep(0.2)
+    sampler.stop()
+    coat.coat_check_device_error()
+    per = [statistics.mean(ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(args.steps))
+           for j in range(len(L))]
+    per = [max_over_ranks(x, ws, dev) for x in per]
+    step_ms = sum(per)
+    step_bytes = sum(b for _, b, _ in L)
+    value = ws * step_bytes / (step_ms * 1e-3) / 1e9
+    peaks = measured_peaks()
+    peak = peaks["hbm_gbs"] if peaks and peaks.get("hbm_gbs") else HBM_FALLBACK_GBS
+    kern = [{"launch": lab, "ms": round(t, 4), "algorithmic_bytes": b,
+             "GB/s": round(b / (t * 1e-3) / 1e9, 1), "frac": round(b / (t * 1e-3) / 1e9 / peak, 4)}
+            for (lab, b, _), t in zip(L, per)]
+    top = max(range(len(L)), key=lambda j: per[j])
+    roofline = {"bound": "hbm", "achieved": kern[top]["GB/s"], "peak": peak, "unit": "GB/s",
+                "frac": kern[top]["frac"], "traffic": None, "kernel": kern[top]["launch"],
+                "peak_source": "measured" if peaks else "fallback"}
+    clocks = sampler.summary(wall0, wall1)
+
+    e2e = None
+    if not args.no_e2e:
+        # public API with host buffers: H2D of the bf16 activations from pinned
+        # memory, quantize (1x128, expansion on), D2H of codes, scales and k
+        b = bufs["act"]
+        hx = torch.empty(b["x"].shape, dtype=torch.bfloat16, pin_memory=True)
+        hq = torch.empty(b["q"].shape, dtype=torch.uint8, pin_memory=True)
+        hs = torch.empty(b["s"].shape, dtype=torch.float32, pin_memory=True)
+        hk = torch.empty(b["k"].shape, dtype=torch.float32, pin_memory=True)
+        hx.copy_(b["x"])
+        torch.cuda.synchronize()
+        steps = max(1, min(args.steps, args.e2e_steps))
+        barrier(ws, dev)
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            b["x"].copy_(hx, non_blocking=True)
+            coat.coat_group_quantize(b["x"], 1, 128, True, E4M3, b["q"], b["s"], b["k"])
+            hq.copy_(b["q"], non_blocking=True)
+            hs.copy_(b["s"], non_blocking=True)
+            hk.copy_(b["k"], non_blocking=True)
+        torch.cuda.synchronize()
+        el = max_over_ranks(time.perf_counter() - t0, ws, dev)
+        nb = codec_bytes(*b["x"].shape, 1, 128)
+        e2e = {"value": round(ws * nb * steps / el / 1e9, 3), "unit": "GB/s",
+               "h2d_bytes_per_step": hx.numel() * 2,
+               "d2h_bytes_per_step": hq.numel() + 4 * (hs.numel() + hk.numel()), "steps": steps,
+               "how": "activations only: H2D bf16 from pinned memory, coat_group_quantize 1x128 "
+                      "with expansion, D2H codes + scale + k; host wall clock"}
+    result = None
+    if rank == 0:
+        cpu = None
+        if ws == 1 and not args.no_cpu_baseline:
+            import oracle as orc
+            rows = 4096
+            x = synth.bf16_bits_to_f32(synth.activations_bits(rank, 0, 0, rows * CODEC_ACT[1]))
+            x = x.reshape(rows, CODEC_ACT[1]).astype(np.float64)
+            t0 = time.perf_counter()
+            orc.group_quantize(x, 1, 128, True, E4M3)
+            el = time.perf_counter() - t0
+            cpu = {"value": round(codec_bytes(rows, CODEC_ACT[1], 1, 128) / el / 1e9, 6),
+                   "unit": "GB/s", "cores": 1, "kind": "oracle",
+                   "sample": "first %d token rows of the activations, 1x128 groups with "
+                             "expansion, one host thread (%.2f s)" % (rows, el)}
+        result = {
+            "metric": CODEC_METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": "mixed-granularity codec: activations bf16 8192x4096 (N(0,1), "
+                                   "0.1% x100 outliers) in 1x128 groups and weights bf16 "
+                                   "4096x11008 in 128x128 blocks, to E4M3, expansion off and on, "
+                                   "dequantize round trip to bf16",
+                       "l2": "flushed (256 MB write) before every timed launch",
+                       "parallelism": "single GPU" if ws == 1 else "replicas%d" % ws},
+            "launches": kern, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": len(L) * args.steps, "clocks": clocks}
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return result
+
+
 def run_reference(args, cfg, ws, rank):
     """The CPU oracle on a bounded sample per step (one host thread)."""
     if rank != 0:
@@ -449,16 +664,27 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default="llama2-7b", choices=sorted(CONFIGS))
+    ap.add_argument("--config", default="llama2-7b", choices=sorted(CONFIGS) + ["act-codec"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--compare-flat", action="store_true",
+                    help="also time one flat tensor of the same parameter count")
     ap.add_argument("--cpu-sample", type=int, default=16 << 20)
     ap.add_argument("--ref-sample", type=int, default=2 << 20)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     ws, rank, local = dist_env()
+    if args.config == "act-codec":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the codec workload has no "
+                              "reference arm; the oracle CPU baseline is in the ours line"}))
+            return
+        res = run_codec(args, ws, rank, local)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
     cfg = CONFIGS[args.config]
     if args.impl == "reference":
         res = run_reference(args, cfg, ws, rank)

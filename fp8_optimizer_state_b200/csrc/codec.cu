@@ -6,9 +6,10 @@
 // "FP8量化训练实战指南", section "分块级缩放：精度优化的进阶方案" (1x128 tiles for
 // activations and gradients, 128x128 blocks for weights, one scale per tile).
 //
-// All kernels are HBM-bound streaming kernels: 16-byte (or 8/4-byte)
-// coalesced loads and stores, no shared-memory staging except the 256-entry
-// log2 decode table, grids sized in multiples of the SM count.
+// All kernels are HBM-bound streaming kernels: 16-byte coalesced loads and
+// stores, persistent grids sized to the resident CTAs of every SM, and the
+// next work item loaded into registers while the current one is computed; no
+// shared-memory staging except the 256-entry log2 decode table.
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -38,48 +39,108 @@ __global__ void fp8_decode_kernel(const uint8_t* __restrict__ q, int64_t n, floa
 }
 
 // ---------------------------------------------------------------------------
-// loading 4 contiguous elements of a row as float
+// 16 contiguous elements of a row, as loaded (bf16 pairs or fp32), so that the
+// next work item can be fetched into registers while the current one is
+// computed.  Row starts are 16-byte aligned (checked by the API), so a chunk
+// that starts at a multiple of 16 columns is 16-byte aligned too.
 // ---------------------------------------------------------------------------
+template <int DT> struct Raw16;
+template <> struct Raw16<0> { float4 a, b, c, d; };   // fp32
+template <> struct Raw16<1> { uint4 a, b; };          // bf16 pairs
+
 template <int DT>
-__device__ __forceinline__ void load4(const void* base, int64_t idx, int valid, float v[4]) {
-  if (DT == 0) {
-    const float* p = static_cast<const float*>(base) + idx;
-    if (valid >= 4) {
-      const float4 t = *reinterpret_cast<const float4*>(p);
-      v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+__device__ __forceinline__ void load16(const void* row, int64_t c, int valid, Raw16<DT>& r) {
+  if constexpr (DT == 0) {
+    const float* p = static_cast<const float*>(row) + c;
+    if (valid >= 16) {
+      r.a = __ldg(reinterpret_cast<const float4*>(p));
+      r.b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+      r.c = __ldg(reinterpret_cast<const float4*>(p) + 2);
+      r.d = __ldg(reinterpret_cast<const float4*>(p) + 3);
     } else {
+      float t[16];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) v[i] = i < valid ? p[i] : 0.f;
+      for (int i = 0; i < 16; ++i) t[i] = i < valid ? p[i] : 0.f;
+      r.a = make_float4(t[0], t[1], t[2], t[3]);
+      r.b = make_float4(t[4], t[5], t[6], t[7]);
+      r.c = make_float4(t[8], t[9], t[10], t[11]);
+      r.d = make_float4(t[12], t[13], t[14], t[15]);
     }
   } else {
-    const uint16_t* p = static_cast<const uint16_t*>(base) + idx;
-    if (valid >= 4) {
-      const uint2 t = *reinterpret_cast<const uint2*>(p);
-      v[0] = bf16lo(t.x); v[1] = bf16hi(t.x); v[2] = bf16lo(t.y); v[3] = bf16hi(t.y);
+    const uint16_t* p = static_cast<const uint16_t*>(row) + c;
+    if (valid >= 16) {
+      r.a = __ldg(reinterpret_cast<const uint4*>(p));
+      r.b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
     } else {
+      uint32_t t[16];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) v[i] = i < valid ? __uint_as_float(uint32_t(p[i]) << 16) : 0.f;
+      for (int i = 0; i < 16; ++i) t[i] = i < valid ? uint32_t(p[i]) : 0u;
+      r.a = make_uint4(t[0] | (t[1] << 16), t[2] | (t[3] << 16), t[4] | (t[5] << 16),
+                       t[6] | (t[7] << 16));
+      r.b = make_uint4(t[8] | (t[9] << 16), t[10] | (t[11] << 16), t[12] | (t[13] << 16),
+                       t[14] | (t[15] << 16));
     }
   }
 }
 
-__device__ __forceinline__ void store_codes4(uint8_t* q, uint32_t c[4], int valid) {
-  if (valid >= 4) {
-    *reinterpret_cast<uint32_t*>(q) = pack4(c[0], c[1], c[2], c[3]);
+template <int DT>
+__device__ __forceinline__ void unpack16(const Raw16<DT>& r, float v[16]) {
+  if constexpr (DT == 0) {
+    const float4 q[4] = {r.a, r.b, r.c, r.d};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[4 * j] = q[j].x; v[4 * j + 1] = q[j].y; v[4 * j + 2] = q[j].z; v[4 * j + 3] = q[j].w;
+    }
+  } else {
+    const uint32_t w[8] = {r.a.x, r.a.y, r.a.z, r.a.w, r.b.x, r.b.y, r.b.z, r.b.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      v[2 * j] = bf16lo(w[j]);
+      v[2 * j + 1] = bf16hi(w[j]);
+    }
+  }
+}
+
+// 16 codes to a row (one 16-byte store when the chunk is whole).
+__device__ __forceinline__ void store16(uint8_t* q, const uint32_t c[16], int valid) {
+  if (valid >= 16) {
+    *reinterpret_cast<uint4*>(q) = make_uint4(pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]),
+                                              pack4(c[8], c[9], c[10], c[11]),
+                                              pack4(c[12], c[13], c[14], c[15]));
   } else {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 16; ++i)
       if (i < valid) q[i] = static_cast<uint8_t>(c[i]);
   }
 }
 
-__device__ __forceinline__ int clamp_valid(int64_t left) {
-  return left <= 0 ? 0 : (left >= 4 ? 4 : static_cast<int>(left));
+__device__ __forceinline__ int clamp_valid(int64_t left, int width) {
+  return left <= 0 ? 0 : (left >= width ? width : static_cast<int>(left));
+}
+
+// Per-group max |x| and min nonzero |x| of 16 values, as (M, key) with
+// key = bits(|x|) - 1 (zero becomes the largest key).
+__device__ __forceinline__ void stats16(const float v[16], float& M, uint32_t& mink) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    M = fmaxf(M, fabsf(v[i]));
+    mink = min(mink, (__float_as_uint(v[i]) & 0x7FFFFFFFu) - 1u);
+  }
+}
+
+template <int FMT>
+__device__ __forceinline__ void encode16(const float v[16], float M, float invM, float k,
+                                         uint32_t c[16]) {
+  const GroupDiv d = group_div(M);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) c[i] = enc_signed<FMT>(v[i], codec_value<FMT>(v[i], M, d, invM, k));
 }
 
 // ---------------------------------------------------------------------------
-// 1 x 128 groups: 8 lanes per group, 16 elements per lane (4 chunks of 4),
-// 4 groups per warp; group max / min-nonzero by 3 xor-shuffles.
+// 1 x 128 groups: 8 lanes per group, 16 contiguous elements per lane, 4 groups
+// (one quad) per warp and work item.  Items (row, quad) are walked row-major
+// with a fixed stride per warp, advanced without divisions; the next item's
+// elements are loaded before the current one is computed.
 // ---------------------------------------------------------------------------
 template <int FMT, int DT>
 __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__ x, int64_t rows,
@@ -88,28 +149,38 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
                                                         float* __restrict__ scale,
                                                         float* __restrict__ kk) {
   const int lane = threadIdx.x & 31, slot = lane >> 3, l = lane & 7;
-  const int64_t nbc = (cols + kGroup - 1) / kGroup;
-  const int64_t ngroups = rows * nbc;
-  const int64_t warp0 = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5;
-  const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t w = warp0; w * 4 < ngroups; w += nwarps) {
-    const int64_t gidx = w * 4 + slot;
-    const bool active = gidx < ngroups;
-    const int64_t r = active ? gidx / nbc : 0, gc = active ? gidx % nbc : 0;
+  const int64_t nbc = (cols + kGroup - 1) / kGroup;   // groups per row
+  const int64_t nq = (nbc + 3) / 4;                    // quads per row
+  const int64_t w0 = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5;
+  const int64_t nw = (int64_t(gridDim.x) * blockDim.x) >> 5;
+  const int64_t dr = nw / nq, dq = nw % nq;            // stride in (rows, quads)
+  int64_t r = w0 / nq, gq = w0 % nq;
+  const size_t esz = DT == 0 ? 4 : 2;
+  auto where = [&](int64_t rr, int64_t qq, int64_t& c, int& valid) {
+    const int64_t g = qq * 4 + slot;
+    c = g * kGroup + 16 * l;
+    valid = (rr < rows && g < nbc) ? clamp_valid(cols - c, 16) : 0;
+  };
+  int64_t c;
+  int valid;
+  Raw16<DT> cur;
+  where(r, gq, c, valid);
+  if (r < rows) load16<DT>(static_cast<const char*>(x) + r * ldx * esz, c, valid, cur);
+  while (r < rows) {
+    // next item
+    int64_t rn = r + dr, qn = gq + dq;
+    if (qn >= nq) { qn -= nq; ++rn; }
+    int64_t cn;
+    int validn;
+    where(rn, qn, cn, validn);
+    Raw16<DT> nxt;
+    if (rn < rows) load16<DT>(static_cast<const char*>(x) + rn * ldx * esz, cn, validn, nxt);
+
     float v[16];
+    unpack16<DT>(cur, v);
     float M = 0.f;
     uint32_t mink = 0xFFFFFFFFu;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t c0 = gc * kGroup + 32 * j + 4 * l;
-      const int valid = active ? clamp_valid(cols - c0) : 0;
-      load4<DT>(x, r * ldx + c0, valid, &v[4 * j]);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        M = fmaxf(M, fabsf(v[4 * j + i]));
-        mink = min(mink, (__float_as_uint(v[4 * j + i]) & 0x7FFFFFFFu) - 1u);
-      }
-    }
+    stats16(v, M, mink);
 #pragma unroll
     for (int off = 1; off < 8; off <<= 1) {
       M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, off));
@@ -117,54 +188,122 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
     }
     float k, sr, invM;
     group_params<FMT>(M, __uint_as_float(mink + 1u), expand != 0, k, sr, invM);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t c0 = gc * kGroup + 32 * j + 4 * l;
-      const int valid = active ? clamp_valid(cols - c0) : 0;
-      uint32_t c[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        c[i] = enc_signed<FMT>(v[4 * j + i], codec_value<FMT>(v[4 * j + i], M, invM, k));
-      if (valid > 0) store_codes4(q + r * ldq + c0, c, valid);
+    uint32_t cd[16];
+    encode16<FMT>(v, M, invM, k, cd);
+    if (valid > 0) store16(q + r * ldq + c, cd, valid);
+    const int64_t g = gq * 4 + slot;
+    if (l == 0 && g < nbc) {
+      scale[r * nbc + g] = sr;
+      kk[r * nbc + g] = k;
     }
-    if (active && l == 0) {
-      scale[gidx] = sr;
-      kk[gidx] = k;
-    }
+    r = rn;
+    gq = qn;
+    c = cn;
+    valid = validn;
+    cur = nxt;
   }
 }
 
 // ---------------------------------------------------------------------------
-// 128 x 128 blocks: one 256-thread CTA per block; warp w takes rows
-// 16w..16w+15 of the block, lane takes 4 columns; two-level reduction
-// (shuffles, then shared memory across the 8 warps).
+// 128 x 128 blocks: one 256-thread CTA per block at a time; warp w takes rows
+// 16w..16w+15, each load instruction covers two rows (half-warp per row, 8
+// contiguous columns per lane); max / min by shuffles, then across the 8
+// warps through shared memory.  bf16 input: the next block is loaded into a
+// second register buffer before the current one is computed.
 // ---------------------------------------------------------------------------
+template <int DT> struct Block8;   // the 64 elements a thread holds, as loaded
+template <> struct Block8<0> { float4 a[8], b[8]; };
+template <> struct Block8<1> { uint4 a[8]; };
+
+template <int DT>
+__device__ __forceinline__ void load_block(const void* x, int64_t rows, int64_t cols, int64_t ldx,
+                                           int64_t br, int64_t bc, int warp, int lane,
+                                           Block8<DT>& B) {
+  const int64_t c = bc * 128 + 8 * (lane & 15);
+  const int cv = clamp_valid(cols - c, 8);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t r = br * 128 + warp * 16 + 2 * i + (lane >> 4);
+    const int valid = r < rows ? cv : 0;
+    if constexpr (DT == 0) {
+      const float* p = static_cast<const float*>(x) + r * ldx + c;
+      float4 u = make_float4(0.f, 0.f, 0.f, 0.f), w = u;
+      if (valid >= 8) {
+        u = __ldg(reinterpret_cast<const float4*>(p));
+        w = __ldg(reinterpret_cast<const float4*>(p) + 1);
+      } else if (valid > 0) {
+        float t[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) t[e] = e < valid ? p[e] : 0.f;
+        u = make_float4(t[0], t[1], t[2], t[3]);
+        w = make_float4(t[4], t[5], t[6], t[7]);
+      }
+      B.a[i] = u;
+      B.b[i] = w;
+    } else {
+      const uint16_t* p = static_cast<const uint16_t*>(x) + r * ldx + c;
+      uint4 u = make_uint4(0u, 0u, 0u, 0u);
+      if (valid >= 8) {
+        u = __ldg(reinterpret_cast<const uint4*>(p));
+      } else if (valid > 0) {
+        uint32_t t[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) t[e] = e < valid ? uint32_t(p[e]) : 0u;
+        u = make_uint4(t[0] | (t[1] << 16), t[2] | (t[3] << 16), t[4] | (t[5] << 16),
+                       t[6] | (t[7] << 16));
+      }
+      B.a[i] = u;
+    }
+  }
+}
+
+template <int DT>
+__device__ __forceinline__ void block_row(const Block8<DT>& B, int i, float v[8]) {
+  if constexpr (DT == 0) {
+    v[0] = B.a[i].x; v[1] = B.a[i].y; v[2] = B.a[i].z; v[3] = B.a[i].w;
+    v[4] = B.b[i].x; v[5] = B.b[i].y; v[6] = B.b[i].z; v[7] = B.b[i].w;
+  } else {
+    const uint4 u = B.a[i];
+    v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+    v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
+  }
+}
+
 template <int FMT, int DT>
 __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict__ x, int64_t rows,
                                                           int64_t cols, int64_t ldx, int expand,
                                                           uint8_t* __restrict__ q, int64_t ldq,
                                                           float* __restrict__ scale,
                                                           float* __restrict__ kk) {
-  __shared__ float sM[8];
-  __shared__ uint32_t sK[8];
+  __shared__ float sM[2][8];
+  __shared__ uint32_t sK[2][8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t nbc = (cols + 127) / 128, nbr = (rows + 127) / 128;
-  for (int64_t b = blockIdx.x; b < nbr * nbc; b += gridDim.x) {
-    const int64_t br = b / nbc, bc = b % nbc;
-    const int64_t c0 = bc * 128 + 4 * lane;
-    const int cvalid = clamp_valid(cols - c0);
-    float v[64];
+  const int64_t nb = nbr * nbc;
+  int64_t b = blockIdx.x;
+  if (b >= nb) return;
+  const int64_t dbr = gridDim.x / nbc, dbc = gridDim.x % nbc;
+  int64_t br = b / nbc, bc = b % nbc;
+  Block8<DT> cur;
+  load_block<DT>(x, rows, cols, ldx, br, bc, warp, lane, cur);
+  int par = 0;
+  while (b < nb) {
+    const int64_t bn = b + gridDim.x;
+    int64_t brn = br + dbr, bcn = bc + dbc;
+    if (bcn >= nbc) { bcn -= nbc; ++brn; }
+    Block8<DT> nxt;
+    if (DT == 1 && bn < nb) load_block<DT>(x, rows, cols, ldx, brn, bcn, warp, lane, nxt);
+
     float M = 0.f;
     uint32_t mink = 0xFFFFFFFFu;
 #pragma unroll
-    for (int rr = 0; rr < 16; ++rr) {
-      const int64_t r = br * 128 + warp * 16 + rr;
-      const int valid = r < rows ? cvalid : 0;
-      load4<DT>(x, r * ldx + c0, valid, &v[4 * rr]);
+    for (int i = 0; i < 8; ++i) {
+      float v[8];
+      block_row<DT>(cur, i, v);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        M = fmaxf(M, fabsf(v[4 * rr + i]));
-        mink = min(mink, (__float_as_uint(v[4 * rr + i]) & 0x7FFFFFFFu) - 1u);
+      for (int e = 0; e < 8; ++e) {
+        M = fmaxf(M, fabsf(v[e]));
+        mink = min(mink, (__float_as_uint(v[e]) & 0x7FFFFFFFu) - 1u);
       }
     }
 #pragma unroll
@@ -172,85 +311,151 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
       M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, off));
       mink = min(mink, __shfl_xor_sync(0xFFFFFFFFu, mink, off));
     }
-    __syncthreads();  // previous block's readers are done with sM / sK
+    // double-buffered partials: one barrier per block
     if (lane == 0) {
-      sM[warp] = M;
-      sK[warp] = mink;
+      sM[par][warp] = M;
+      sK[par][warp] = mink;
     }
     __syncthreads();
-    M = sM[0];
-    mink = sK[0];
+    M = sM[par][0];
+    mink = sK[par][0];
 #pragma unroll
     for (int w = 1; w < 8; ++w) {
-      M = fmaxf(M, sM[w]);
-      mink = min(mink, sK[w]);
+      M = fmaxf(M, sM[par][w]);
+      mink = min(mink, sK[par][w]);
     }
+    par ^= 1;
     float k, sr, invM;
     group_params<FMT>(M, __uint_as_float(mink + 1u), expand != 0, k, sr, invM);
+    const GroupDiv d = group_div(M);
+    const int64_t c = bc * 128 + 8 * (lane & 15);
+    const int cv = clamp_valid(cols - c, 8);
 #pragma unroll
-    for (int rr = 0; rr < 16; ++rr) {
-      const int64_t r = br * 128 + warp * 16 + rr;
-      const int valid = r < rows ? cvalid : 0;
-      uint32_t c[4];
+    for (int i = 0; i < 8; ++i) {
+      const int64_t r = br * 128 + warp * 16 + 2 * i + (lane >> 4);
+      float v[8];
+      block_row<DT>(cur, i, v);
+      uint32_t cd[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        c[i] = enc_signed<FMT>(v[4 * rr + i], codec_value<FMT>(v[4 * rr + i], M, invM, k));
-      if (valid > 0) store_codes4(q + r * ldq + c0, c, valid);
+      for (int e = 0; e < 8; ++e) cd[e] = enc_signed<FMT>(v[e], codec_value<FMT>(v[e], M, d, invM, k));
+      const int valid = r < rows ? cv : 0;
+      uint8_t* qp = q + r * ldq + c;
+      if (valid >= 8) {
+        *reinterpret_cast<uint2*>(qp) = make_uint2(pack4(cd[0], cd[1], cd[2], cd[3]),
+                                                   pack4(cd[4], cd[5], cd[6], cd[7]));
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (e < valid) qp[e] = static_cast<uint8_t>(cd[e]);
+      }
     }
     if (threadIdx.x == 0) {
       scale[b] = sr;
       kk[b] = k;
     }
+    b = bn;
+    br = brn;
+    bc = bcn;
+    if (DT == 1) {
+      cur = nxt;
+    } else if (b < nb) {
+      load_block<DT>(x, rows, cols, ldx, br, bc, warp, lane, cur);
+    }
   }
 }
 
 // ---------------------------------------------------------------------------
-// dequantise: one thread per 4 contiguous codes of a row (one group each).
+// dequantise: one thread per 16 contiguous codes of a row (all in one group,
+// since groups are 128 columns wide and start at multiples of 128); chunks
+// are walked row-major with a fixed stride per thread, and the next chunk's
+// codes and group metadata are loaded before the current chunk is computed.
+// GR: rows per group (1 or 128).
 // ---------------------------------------------------------------------------
-template <int FMT, int OT>
+template <int FMT, int OT, int GR>
 __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict__ q, int64_t ldq,
                                                       const float* __restrict__ scale,
                                                       const float* __restrict__ kk, int64_t rows,
-                                                      int64_t cols, int gr, int gc,
-                                                      void* __restrict__ out, int64_t ldo) {
+                                                      int64_t cols, void* __restrict__ out,
+                                                      int64_t ldo) {
   __shared__ float tab[256];
   fill_log2_table<FMT>(tab);
   __syncthreads();
-  const int64_t cpr = (cols + 3) / 4;  // chunks per row
-  const int64_t nbc = (cols + gc - 1) / gc;
-  for (int64_t t = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; t < rows * cpr;
-       t += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t r = t / cpr, c0 = (t % cpr) * 4;
-    const int valid = clamp_valid(cols - c0);
-    const int64_t g = (r / gr) * nbc + c0 / gc;
-    const float invk = rcp_approx(kk[g]), s = scale[g];
-    uint32_t w = 0;
-    const uint8_t* qp = q + r * ldq + c0;
-    if (valid >= 4) {
-      w = *reinterpret_cast<const uint32_t*>(qp);
+  const int64_t cpr = (cols + 15) / 16;  // chunks per row
+  const int64_t nbc = (cols + 127) / 128;
+  const int64_t t0 = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+  const int64_t nt = int64_t(gridDim.x) * blockDim.x;
+  const int64_t dr = nt / cpr, dc = nt % cpr;
+  int64_t r = t0 / cpr, cc = t0 % cpr;
+  auto fetch = [&](int64_t rr, int64_t ch, uint4& w, float& s, float& kv, int& valid) {
+    const int64_t c0 = ch * 16;
+    valid = clamp_valid(cols - c0, 16);
+    const uint8_t* qp = q + rr * ldq + c0;
+    if (valid >= 16) {
+      w = __ldg(reinterpret_cast<const uint4*>(qp));
     } else {
-      for (int i = 0; i < valid; ++i) w |= uint32_t(qp[i]) << (8 * i);
-    }
-    float x[4];
+      uint32_t t[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t c = (w >> (8 * i)) & 0xFFu;
-      const float a = ex2_approx(tab[c] * invk) * s;
-      x[i] = __uint_as_float(__float_as_uint(a) ^ ((c & 0x80u) << 24));
+      for (int i = 0; i < 16; ++i)
+        if (i < valid) t[i >> 2] |= uint32_t(qp[i]) << (8 * (i & 3));
+      w = make_uint4(t[0], t[1], t[2], t[3]);
     }
+    const int64_t g = (GR == 1 ? rr : rr / GR) * nbc + (ch >> 3);
+    s = __ldg(scale + g);
+    kv = __ldg(kk + g);
+  };
+  uint4 w;
+  float s, kv;
+  int valid;
+  if (r < rows) fetch(r, cc, w, s, kv, valid);
+  while (r < rows) {
+    int64_t rn = r + dr, cn = cc + dc;
+    if (cn >= cpr) { cn -= cpr; ++rn; }
+    uint4 wn;
+    float sn, kn;
+    int validn;
+    if (rn < rows) fetch(rn, cn, wn, sn, kn, validn);
+
+    const float invk = rcp_approx(kv);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    float xv[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t c = (ws[i >> 2] >> (8 * (i & 3))) & 0xFFu;
+      const float a = ex2_approx(tab[c] * invk) * s;
+      xv[i] = __uint_as_float(__float_as_uint(a) ^ ((c & 0x80u) << 24));
+    }
+    const int64_t c0 = cc * 16;
     if (OT == 0) {
       float* o = static_cast<float*>(out) + r * ldo + c0;
-      if (valid >= 4)
-        *reinterpret_cast<float4*>(o) = make_float4(x[0], x[1], x[2], x[3]);
-      else
-        for (int i = 0; i < valid; ++i) o[i] = x[i];
+      if (valid >= 16) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          reinterpret_cast<float4*>(o)[j] = make_float4(xv[4 * j], xv[4 * j + 1], xv[4 * j + 2], xv[4 * j + 3]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (i < valid) o[i] = xv[i];
+      }
     } else {
       uint16_t* o = static_cast<uint16_t*>(out) + r * ldo + c0;
-      if (valid >= 4)
-        *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]));
-      else
-        for (int i = 0; i < valid; ++i) o[i] = static_cast<uint16_t>(pack_bf16x2(x[i], 0.f));
+      if (valid >= 16) {
+        uint32_t p[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) p[j] = pack_bf16x2(xv[2 * j], xv[2 * j + 1]);
+        reinterpret_cast<uint4*>(o)[0] = make_uint4(p[0], p[1], p[2], p[3]);
+        reinterpret_cast<uint4*>(o)[1] = make_uint4(p[4], p[5], p[6], p[7]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (i < valid) o[i] = static_cast<uint16_t>(pack_bf16x2(xv[i], 0.f));
+      }
     }
+    r = rn;
+    cc = cn;
+    w = wn;
+    s = sn;
+    kv = kn;
+    valid = validn;
   }
 }
 
@@ -289,12 +494,13 @@ static void quant_dispatch(const void* x, int64_t rows, int64_t cols, int64_t ld
                            int expand, uint8_t* q, int64_t ldq, float* scale, float* k,
                            int dev, cudaStream_t s) {
   if (gr == 1) {
-    const int64_t groups = rows * ((cols + 127) / 128);
-    const unsigned g = grid_for((groups + 3) / 4, 8, dev, 8);   // 8 warps per block
+    const int64_t quads = rows * (((cols + 127) / 128 + 3) / 4);
+    // 64 registers per thread: 4 resident 256-thread CTAs per SM, persistent
+    const unsigned g = grid_for(quads, 8, dev, 4);
     quant_row_kernel<FMT, DT><<<g, 256, 0, s>>>(x, rows, cols, ldx, expand, q, ldq, scale, k);
   } else {
     const int64_t blocks = ((rows + 127) / 128) * ((cols + 127) / 128);
-    const unsigned g = grid_for(blocks, 1, dev, 4);
+    const unsigned g = grid_for(blocks, 1, dev, 2);   // ~120 registers: 2 CTAs per SM
     quant_block_kernel<FMT, DT><<<g, 256, 0, s>>>(x, rows, cols, ldx, expand, q, ldq, scale, k);
   }
 }
@@ -315,19 +521,30 @@ cudaError_t launch_group_quantize(const void* x, int xt, int64_t rows, int64_t c
   return cudaGetLastError();
 }
 
+template <int FMT, int OT>
+static void dequant_dispatch(const uint8_t* q, int64_t ldq, const float* scale, const float* k,
+                             int64_t rows, int64_t cols, int gr, void* out, int64_t ldo, unsigned g,
+                             cudaStream_t s) {
+  if (gr == 1)
+    dequant_kernel<FMT, OT, 1><<<g, 256, 0, s>>>(q, ldq, scale, k, rows, cols, out, ldo);
+  else
+    dequant_kernel<FMT, OT, 128><<<g, 256, 0, s>>>(q, ldq, scale, k, rows, cols, out, ldo);
+}
+
 cudaError_t launch_group_dequantize(const uint8_t* q, int64_t ldq, const float* scale,
                                     const float* k, int64_t rows, int64_t cols, int gr, int gc,
                                     int fmt, void* out, int ot, int64_t ldo, cudaStream_t s) {
   if (rows == 0 || cols == 0) return cudaSuccess;
+  if (gc != 128 || (gr != 1 && gr != 128)) return cudaErrorInvalidValue;
   int dev = 0;
   cudaGetDevice(&dev);
-  const unsigned g = grid_for(rows * ((cols + 3) / 4), 256, dev, 8);
+  const unsigned g = grid_for(rows * ((cols + 15) / 16), 256, dev, 4);   // persistent
   if (fmt == kE4M3) {
-    if (ot == 0) dequant_kernel<kE4M3, 0><<<g, 256, 0, s>>>(q, ldq, scale, k, rows, cols, gr, gc, out, ldo);
-    else dequant_kernel<kE4M3, 1><<<g, 256, 0, s>>>(q, ldq, scale, k, rows, cols, gr, gc, out, ldo);
+    if (ot == 0) dequant_dispatch<kE4M3, 0>(q, ldq, scale, k, rows, cols, gr, out, ldo, g, s);
+    else dequant_dispatch<kE4M3, 1>(q, ldq, scale, k, rows, cols, gr, out, ldo, g, s);
   } else {
-    if (ot == 0) dequant_kernel<kE5M2, 0><<<g, 256, 0, s>>>(q, ldq, scale, k, rows, cols, gr, gc, out, ldo);
-    else dequant_kernel<kE5M2, 1><<<g, 256, 0, s>>>(q, ldq, scale, k, rows, cols, gr, gc, out, ldo);
+    if (ot == 0) dequant_dispatch<kE5M2, 0>(q, ldq, scale, k, rows, cols, gr, out, ldo, g, s);
+    else dequant_dispatch<kE5M2, 1>(q, ldq, scale, k, rows, cols, gr, out, ldo, g, s);
   }
   return cudaGetLastError();
 }

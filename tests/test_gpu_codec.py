@@ -52,6 +52,25 @@ def test_encoder_matches_hardware_cast_in_range(fmt):
 
 
 @pytest.mark.parametrize("fmt", [E4M3, E5M2])
+def test_encoder_exhaustive_up_to_format_max(fmt):
+    """Every non-negative FP32 value up to FMT_MAX (1 + 2^-16) -- the range the
+    step's expanded values take -- encodes as the hardware's round-to-nearest-
+    even conversion does (about 1.1e9 values per format, in chunks)."""
+    top = 448.0 if fmt == E4M3 else 57344.0
+    last = int(np.float32(top * (1 + 2.0 ** -16)).view(np.uint32))
+    chunk = 1 << 27
+    q = torch.empty(chunk, dtype=torch.uint8, device="cuda")
+    for a in range(0, last + 1, chunk):
+        n = min(chunk, last + 1 - a)
+        y = torch.arange(a, a + n, dtype=torch.int64, device="cuda").to(torch.int32).view(torch.float32)
+        coat.coat_fp8_encode(y, fmt, q[:n])
+        ref = y.to(TORCH_DT[fmt]).view(torch.uint8)
+        bad = (q[:n] != ref).nonzero()
+        assert bad.numel() == 0, "y bits %#x: got %#x, want %#x" % (
+            a + int(bad[0]), int(q[int(bad[0])]), int(ref[int(bad[0])]))
+
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2])
 def test_decoder_all_codes(orc, fmt):
     q = torch.arange(256, dtype=torch.int32).to(torch.uint8).cuda()
     out = torch.empty(256, dtype=torch.float32, device="cuda")
