@@ -212,6 +212,12 @@ def max_over_ranks(x, ws, device):
     return float(t.item())
 
 
+def throughput_gparams(ws, n_params, steps, elapsed_ms):
+    """Whole-job throughput: every rank steps its own n_params parameters
+    (replicas, weak scaling), timed as the slowest rank."""
+    return ws * n_params * steps / (elapsed_ms * 1e-3) / 1e9
+
+
 def barrier(ws, device):
     if ws > 1:
         import torch.distributed as dist
@@ -328,7 +334,7 @@ def run_ours(args, cfg, ws, rank, local):
     kernel_ms = max_over_ranks(statistics.mean(launch_ms), ws, dev)
     n_params = ps.total_elements
     n_tensors = len(ps)
-    value = ws * n_params * args.steps / (elapsed_ms * 1e-3) / 1e9
+    value = throughput_gparams(ws, n_params, args.steps, elapsed_ms)
 
     # roofline of the step kernel
     peaks = measured_peaks()
