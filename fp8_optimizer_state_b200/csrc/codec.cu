@@ -11,6 +11,8 @@
 // next work item loaded into registers while the current one is computed; no
 // shared-memory staging except the 256-entry log2 decode table.
 #include <cstdint>
+#include <mutex>
+#include <unordered_map>
 #include <cuda_runtime.h>
 
 #include "coat_device.cuh"
@@ -101,16 +103,14 @@ __device__ __forceinline__ void unpack16(const Raw16<DT>& r, float v[16]) {
   }
 }
 
-// 16 codes to a row (one 16-byte store when the chunk is whole).
-__device__ __forceinline__ void store16(uint8_t* q, const uint32_t c[16], int valid) {
+// 16 codes (four packed words) to a row: one 16-byte store when the chunk is whole.
+__device__ __forceinline__ void store16(uint8_t* q, const uint32_t (&w)[4], int valid) {
   if (valid >= 16) {
-    *reinterpret_cast<uint4*>(q) = make_uint4(pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]),
-                                              pack4(c[8], c[9], c[10], c[11]),
-                                              pack4(c[12], c[13], c[14], c[15]));
+    *reinterpret_cast<uint4*>(q) = make_uint4(w[0], w[1], w[2], w[3]);
   } else {
 #pragma unroll
     for (int i = 0; i < 16; ++i)
-      if (i < valid) q[i] = static_cast<uint8_t>(c[i]);
+      if (i < valid) q[i] = static_cast<uint8_t>(w[i >> 2] >> (8 * (i & 3)));
   }
 }
 
@@ -118,22 +118,27 @@ __device__ __forceinline__ int clamp_valid(int64_t left, int width) {
   return left <= 0 ? 0 : (left >= width ? width : static_cast<int>(left));
 }
 
-// Per-group max |x| and min nonzero |x| of 16 values, as (M, key) with
-// key = bits(|x|) - 1 (zero becomes the largest key).
-__device__ __forceinline__ void stats16(const float v[16], float& M, uint32_t& mink) {
+// Max and min-nonzero of |x| over N values, on the FP32 bit patterns of |x|
+// (which order like the values): maxb = max bits(|x|) (above 0x7F800000 only
+// if a NaN is present, equal to it for an Inf), mink = min(bits(|x|) - 1), so
+// that zero becomes the largest key.
+template <int N>
+__device__ __forceinline__ void stats_bits(const float (&v)[N], uint32_t& maxb, uint32_t& mink) {
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    M = fmaxf(M, fabsf(v[i]));
-    mink = min(mink, (__float_as_uint(v[i]) & 0x7FFFFFFFu) - 1u);
+  for (int i = 0; i < N; ++i) {
+    const uint32_t a = __float_as_uint(v[i]) & 0x7FFFFFFFu;
+    maxb = max(maxb, a);
+    mink = min(mink, a - 1u);
   }
 }
 
-template <int FMT>
-__device__ __forceinline__ void encode16(const float v[16], float M, float invM, float k,
-                                         uint32_t c[16]) {
-  const GroupDiv d = group_div(M);
+// Max |x| ignoring NaN (the rare groups that hold an Inf or a NaN).
+template <int N>
+__device__ __forceinline__ float max_abs_nonnan(const float (&v)[N]) {
+  float M = 0.f;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) c[i] = enc_signed<FMT>(v[i], codec_value<FMT>(v[i], M, d, invM, k));
+  for (int i = 0; i < N; ++i) M = fmaxf(M, fabsf(v[i]));
+  return M;
 }
 
 // ---------------------------------------------------------------------------
@@ -178,19 +183,32 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
 
     float v[16];
     unpack16<DT>(cur, v);
-    float M = 0.f;
-    uint32_t mink = 0xFFFFFFFFu;
-    stats16(v, M, mink);
+    uint32_t maxb = 0u, mink = 0xFFFFFFFFu;
+    stats_bits(v, maxb, mink);
 #pragma unroll
     for (int off = 1; off < 8; off <<= 1) {
-      M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, off));
+      maxb = max(maxb, __shfl_xor_sync(0xFFFFFFFFu, maxb, off));
       mink = min(mink, __shfl_xor_sync(0xFFFFFFFFu, mink, off));
+    }
+    const bool special = maxb >= 0x7F800000u;   // an Inf or a NaN in the group
+    float M = __uint_as_float(maxb);
+    if (__any_sync(0xFFFFFFFFu, special)) {
+      float Mn = max_abs_nonnan(v);
+#pragma unroll
+      for (int off = 1; off < 8; off <<= 1) Mn = fmaxf(Mn, __shfl_xor_sync(0xFFFFFFFFu, Mn, off));
+      if (special) M = Mn;
     }
     float k, sr, invM;
     group_params<FMT>(M, __uint_as_float(mink + 1u), expand != 0, k, sr, invM);
-    uint32_t cd[16];
-    encode16<FMT>(v, M, invM, k, cd);
-    if (valid > 0) store16(q + r * ldq + c, cd, valid);
+    const bool use_div = k == 1.0f;
+    GroupDiv d{};
+    if (use_div) d = codec_div<FMT>(M);
+    uint32_t cw[4];
+    if (!special)
+      encode_words<FMT, 16, true>(v, use_div, d, invM, k, cw);
+    else
+      encode_words<FMT, 16, false>(v, use_div, d, invM, k, cw);
+    if (valid > 0) store16(q + r * ldq + c, cw, valid);
     const int64_t g = gq * 4 + slot;
     if (l == 0 && g < nbc) {
       scale[r * nbc + g] = sr;
@@ -275,7 +293,7 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
                                                           uint8_t* __restrict__ q, int64_t ldq,
                                                           float* __restrict__ scale,
                                                           float* __restrict__ kk) {
-  __shared__ float sM[2][8];
+  __shared__ uint32_t sM[2][8];
   __shared__ uint32_t sK[2][8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t nbc = (cols + 127) / 128, nbr = (rows + 127) / 128;
@@ -294,40 +312,57 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
     Block8<DT> nxt;
     if (DT == 1 && bn < nb) load_block<DT>(x, rows, cols, ldx, brn, bcn, warp, lane, nxt);
 
-    float M = 0.f;
-    uint32_t mink = 0xFFFFFFFFu;
+    uint32_t maxb = 0u, mink = 0xFFFFFFFFu;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       float v[8];
       block_row<DT>(cur, i, v);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        M = fmaxf(M, fabsf(v[e]));
-        mink = min(mink, (__float_as_uint(v[e]) & 0x7FFFFFFFu) - 1u);
-      }
+      stats_bits(v, maxb, mink);
     }
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-      M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, off));
+      maxb = max(maxb, __shfl_xor_sync(0xFFFFFFFFu, maxb, off));
       mink = min(mink, __shfl_xor_sync(0xFFFFFFFFu, mink, off));
     }
     // double-buffered partials: one barrier per block
     if (lane == 0) {
-      sM[par][warp] = M;
+      sM[par][warp] = maxb;
       sK[par][warp] = mink;
     }
     __syncthreads();
-    M = sM[par][0];
+    maxb = sM[par][0];
     mink = sK[par][0];
 #pragma unroll
     for (int w = 1; w < 8; ++w) {
-      M = fmaxf(M, sM[par][w]);
+      maxb = max(maxb, sM[par][w]);
       mink = min(mink, sK[par][w]);
+    }
+    const bool special = maxb >= 0x7F800000u;   // an Inf or a NaN in the block (CTA-uniform)
+    float M = __uint_as_float(maxb);
+    if (special) {
+      // max |x| ignoring NaN, through the other half of the partials buffer
+      float Mn = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float v[8];
+        block_row<DT>(cur, i, v);
+        Mn = fmaxf(Mn, max_abs_nonnan(v));
+      }
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) Mn = fmaxf(Mn, __shfl_xor_sync(0xFFFFFFFFu, Mn, off));
+      if (lane == 0) sM[par ^ 1][warp] = __float_as_uint(Mn);
+      __syncthreads();
+      M = __uint_as_float(sM[par ^ 1][0]);
+#pragma unroll
+      for (int w = 1; w < 8; ++w) M = fmaxf(M, __uint_as_float(sM[par ^ 1][w]));
+      __syncthreads();   // the partials buffer is free again before the next block writes it
     }
     par ^= 1;
     float k, sr, invM;
     group_params<FMT>(M, __uint_as_float(mink + 1u), expand != 0, k, sr, invM);
-    const GroupDiv d = group_div(M);
+    const bool use_div = k == 1.0f;
+    GroupDiv d{};
+    if (use_div) d = codec_div<FMT>(M);
     const int64_t c = bc * 128 + 8 * (lane & 15);
     const int cv = clamp_valid(cols - c, 8);
 #pragma unroll
@@ -335,18 +370,19 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
       const int64_t r = br * 128 + warp * 16 + 2 * i + (lane >> 4);
       float v[8];
       block_row<DT>(cur, i, v);
-      uint32_t cd[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) cd[e] = enc_signed<FMT>(v[e], codec_value<FMT>(v[e], M, d, invM, k));
+      uint32_t cw[2];
+      if (!special)
+        encode_words<FMT, 8, true>(v, use_div, d, invM, k, cw);
+      else
+        encode_words<FMT, 8, false>(v, use_div, d, invM, k, cw);
       const int valid = r < rows ? cv : 0;
       uint8_t* qp = q + r * ldq + c;
       if (valid >= 8) {
-        *reinterpret_cast<uint2*>(qp) = make_uint2(pack4(cd[0], cd[1], cd[2], cd[3]),
-                                                   pack4(cd[4], cd[5], cd[6], cd[7]));
+        *reinterpret_cast<uint2*>(qp) = make_uint2(cw[0], cw[1]);
       } else {
 #pragma unroll
         for (int e = 0; e < 8; ++e)
-          if (e < valid) qp[e] = static_cast<uint8_t>(cd[e]);
+          if (e < valid) qp[e] = static_cast<uint8_t>(cw[e >> 2] >> (8 * (e & 3)));
       }
     }
     if (threadIdx.x == 0) {
@@ -377,9 +413,15 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
                                                       const float* __restrict__ kk, int64_t rows,
                                                       int64_t cols, void* __restrict__ out,
                                                       int64_t ldo) {
-  __shared__ float tab[256];
-  fill_log2_table<FMT>(tab);
+  // log2|value(code)|, replicated once per lane (entry c of lane j at 32 c + j)
+  // so that the per-element lookups of a warp never share a bank
+  __shared__ float tab1[256];
+  __shared__ float tab[256 * 32];
+  fill_log2_table<FMT>(tab1);
   __syncthreads();
+  for (int e = threadIdx.x; e < 256 * 32; e += blockDim.x) tab[e] = tab1[e >> 5];
+  __syncthreads();
+  const float* tabl = tab + (threadIdx.x & 31);
   const int64_t cpr = (cols + 15) / 16;  // chunks per row
   const int64_t nbc = (cols + 127) / 128;
   const int64_t t0 = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
@@ -420,9 +462,10 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
     float xv[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const uint32_t c = (ws[i >> 2] >> (8 * (i & 3))) & 0xFFu;
-      const float a = ex2_approx(tab[c] * invk) * s;
-      xv[i] = __uint_as_float(__float_as_uint(a) ^ ((c & 0x80u) << 24));
+      const uint32_t wd = ws[i >> 2];
+      const uint32_t c = __byte_perm(wd, 0u, 0x4440u + (i & 3));
+      const float a = ex2_approx(tabl[c << 5] * invk) * s;
+      xv[i] = __uint_as_float(__float_as_uint(a) ^ ((wd << (24 - 8 * (i & 3))) & 0x80000000u));
     }
     const int64_t c0 = cc * 16;
     if (OT == 0) {
@@ -467,6 +510,23 @@ unsigned grid_for(int64_t work_items, int per_block, int dev, int max_blocks_per
   return static_cast<unsigned>(b);
 }
 
+// CTAs of `kernel` (256 threads, static shared memory only) resident per SM,
+// from the occupancy calculator, cached per kernel (all B200s give the same).
+std::mutex g_occ_mu;
+std::unordered_map<const void*, int> g_occ;
+int resident_ctas(const void* kernel) {
+  std::lock_guard<std::mutex> lk(g_occ_mu);
+  auto it = g_occ.find(kernel);
+  if (it != g_occ.end()) return it->second;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, 256, 0) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    n = 1;
+  }
+  g_occ.emplace(kernel, n);
+  return n;
+}
+
 }  // namespace
 
 cudaError_t launch_fp8_encode(const float* y, int64_t n, int fmt, uint8_t* q, cudaStream_t s) {
@@ -495,13 +555,14 @@ static void quant_dispatch(const void* x, int64_t rows, int64_t cols, int64_t ld
                            int dev, cudaStream_t s) {
   if (gr == 1) {
     const int64_t quads = rows * (((cols + 127) / 128 + 3) / 4);
-    // 64 registers per thread: 4 resident 256-thread CTAs per SM, persistent
-    const unsigned g = grid_for(quads, 8, dev, 4);
-    quant_row_kernel<FMT, DT><<<g, 256, 0, s>>>(x, rows, cols, ldx, expand, q, ldq, scale, k);
+    auto kern = quant_row_kernel<FMT, DT>;
+    const unsigned g = grid_for(quads, 8, dev, resident_ctas(reinterpret_cast<const void*>(kern)));
+    kern<<<g, 256, 0, s>>>(x, rows, cols, ldx, expand, q, ldq, scale, k);
   } else {
     const int64_t blocks = ((rows + 127) / 128) * ((cols + 127) / 128);
-    const unsigned g = grid_for(blocks, 1, dev, 2);   // ~120 registers: 2 CTAs per SM
-    quant_block_kernel<FMT, DT><<<g, 256, 0, s>>>(x, rows, cols, ldx, expand, q, ldq, scale, k);
+    auto kern = quant_block_kernel<FMT, DT>;
+    const unsigned g = grid_for(blocks, 1, dev, resident_ctas(reinterpret_cast<const void*>(kern)));
+    kern<<<g, 256, 0, s>>>(x, rows, cols, ldx, expand, q, ldq, scale, k);
   }
 }
 
@@ -523,12 +584,12 @@ cudaError_t launch_group_quantize(const void* x, int xt, int64_t rows, int64_t c
 
 template <int FMT, int OT>
 static void dequant_dispatch(const uint8_t* q, int64_t ldq, const float* scale, const float* k,
-                             int64_t rows, int64_t cols, int gr, void* out, int64_t ldo, unsigned g,
+                             int64_t rows, int64_t cols, int gr, void* out, int64_t ldo, int dev,
                              cudaStream_t s) {
-  if (gr == 1)
-    dequant_kernel<FMT, OT, 1><<<g, 256, 0, s>>>(q, ldq, scale, k, rows, cols, out, ldo);
-  else
-    dequant_kernel<FMT, OT, 128><<<g, 256, 0, s>>>(q, ldq, scale, k, rows, cols, out, ldo);
+  auto kern = gr == 1 ? dequant_kernel<FMT, OT, 1> : dequant_kernel<FMT, OT, 128>;
+  const unsigned g = grid_for(rows * ((cols + 15) / 16), 256, dev,
+                              resident_ctas(reinterpret_cast<const void*>(kern)));
+  kern<<<g, 256, 0, s>>>(q, ldq, scale, k, rows, cols, out, ldo);
 }
 
 cudaError_t launch_group_dequantize(const uint8_t* q, int64_t ldq, const float* scale,
@@ -538,13 +599,12 @@ cudaError_t launch_group_dequantize(const uint8_t* q, int64_t ldq, const float* 
   if (gc != 128 || (gr != 1 && gr != 128)) return cudaErrorInvalidValue;
   int dev = 0;
   cudaGetDevice(&dev);
-  const unsigned g = grid_for(rows * ((cols + 15) / 16), 256, dev, 4);   // persistent
   if (fmt == kE4M3) {
-    if (ot == 0) dequant_dispatch<kE4M3, 0>(q, ldq, scale, k, rows, cols, gr, out, ldo, g, s);
-    else dequant_dispatch<kE4M3, 1>(q, ldq, scale, k, rows, cols, gr, out, ldo, g, s);
+    if (ot == 0) dequant_dispatch<kE4M3, 0>(q, ldq, scale, k, rows, cols, gr, out, ldo, dev, s);
+    else dequant_dispatch<kE4M3, 1>(q, ldq, scale, k, rows, cols, gr, out, ldo, dev, s);
   } else {
-    if (ot == 0) dequant_dispatch<kE5M2, 0>(q, ldq, scale, k, rows, cols, gr, out, ldo, g, s);
-    else dequant_dispatch<kE5M2, 1>(q, ldq, scale, k, rows, cols, gr, out, ldo, g, s);
+    if (ot == 0) dequant_dispatch<kE5M2, 0>(q, ldq, scale, k, rows, cols, gr, out, ldo, dev, s);
+    else dequant_dispatch<kE5M2, 1>(q, ldq, scale, k, rows, cols, gr, out, ldo, dev, s);
   }
   return cudaGetLastError();
 }

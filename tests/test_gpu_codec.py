@@ -122,6 +122,60 @@ def test_group_quantize_vs_oracle(orc, gr, gc, rows, cols, fmt, expand, dtype):
 
 @pytest.mark.parametrize("gr", [1, 128])
 @pytest.mark.parametrize("fmt", [E4M3, E5M2])
+@pytest.mark.parametrize("expand", [False, True])
+def test_group_quantize_special_values(orc, gr, fmt, expand):
+    """Groups holding NaN or +-Inf follow the oracle: the maximum ignores NaN, a
+    NaN element encodes as a NaN code, an Inf maximum gives k = 1 and an
+    infinite scale with every finite element at code 0, and a group whose only
+    values are NaN is all zeros with k = 1, scale 1.  Ordinary groups beside
+    them are unaffected."""
+    rows, cols = (4, 512) if gr == 1 else (256, 256)
+    bits = synth.activations_bits(3, 7, 0, rows * cols).reshape(rows, cols)
+    x = synth.bf16_bits_to_f32(bits).copy()
+    nan, inf = np.float32(np.nan), np.float32(np.inf)
+    if gr == 1:
+        x[0, 5] = nan                  # group (0, 0): one NaN
+        x[1, 130] = inf                # group (1, 1): +Inf
+        x[2, 260], x[2, 300] = -inf, nan   # group (2, 2): -Inf and NaN
+        x[3, 384:512] = nan            # group (3, 3): all NaN
+    else:
+        x[3, 5] = nan                  # block (0, 0)
+        x[130, 7] = inf                # block (1, 0)
+        x[20, 200], x[90, 129] = -inf, nan   # block (0, 1)
+        x[128:, 128:] = nan            # block (1, 1): all NaN
+    xb = torch.from_numpy(x).to(torch.bfloat16).cuda()
+    nbr, nbc = -(-rows // gr), cols // 128
+    q = torch.zeros((rows, cols), dtype=torch.uint8, device="cuda")
+    s = torch.zeros((nbr, nbc), dtype=torch.float32, device="cuda")
+    k = torch.zeros((nbr, nbc), dtype=torch.float32, device="cuda")
+    coat.coat_group_quantize(xb, gr, 128, expand, fmt, q, s, k)
+    oq, os_, ok_ = orc.group_quantize(xb.float().cpu().numpy().astype(np.float64), gr, 128,
+                                      expand, fmt)
+    gq, gs, gk = q.cpu().numpy(), s.cpu().numpy(), k.cpu().numpy()
+    # exact groups: an Inf maximum, or NaN only (k = 1 and a scale of Inf or 1)
+    exact = np.zeros((nbr, nbc), dtype=bool)
+    xs = xb.float().cpu().numpy()
+    for bi in range(nbr):
+        for bj in range(nbc):
+            blk = xs[bi * gr:(bi + 1) * gr, bj * 128:(bj + 1) * 128]
+            exact[bi, bj] = np.isinf(blk).any() or np.isnan(blk).all()
+    assert exact.sum() == 3
+    assert np.array_equal(gk[exact], ok_[exact]) and np.array_equal(gs[exact], os_[exact])
+    assert np.all(rel_err(gk[~exact], ok_[~exact]) <= K_RTOL)
+    assert np.all(rel_err(gs[~exact], os_[~exact]) <= scale_rtol(ok_[~exact], fmt))
+    el_exact = np.repeat(np.repeat(exact, gr, axis=0), 128, axis=1)[:rows]
+    nan_code = (oq & 0x7F) == 0x7F
+    assert nan_code.sum() >= 3
+    assert np.all((gq[nan_code] & 0x7F) == 0x7F)              # NaN codes (sign may differ)
+    same = el_exact & ~nan_code
+    assert np.array_equal(gq[same], oq[same])
+    rest = ~el_exact & ~nan_code
+    diff, maxd = compare_codes(gq[rest], oq[rest])
+    assert maxd <= 1 and diff.sum() <= max(1, FLIP_FRACTION * diff.size)
+
+
+@pytest.mark.parametrize("gr", [1, 128])
+@pytest.mark.parametrize("fmt", [E4M3, E5M2])
 def test_group_dequantize_vs_oracle(orc, gr, fmt):
     rows, cols = 256, 640
     rng = np.random.default_rng(30 + gr + fmt)
