@@ -216,8 +216,11 @@ coat_status coat_group_quantize(const void* x, coat_dtype xt, int64_t rows, int6
   if (rows > 1 && ((ld_x * int64_t(dtype_size(xt))) % 16 != 0 || ld_q % 16 != 0))
     return fail(COAT_ERR_MISALIGNED, "%s: row strides must be multiples of 16 bytes", fn);
   if (!aligned(scale, 4) || !aligned(k, 4)) return fail(COAT_ERR_MISALIGNED, "%s: scale/k not 4-byte aligned", fn);
-  cudaError_t e = coat::launch_group_quantize(x, xt, rows, cols, ld_x, group_rows, expand, fmt, q,
-                                              ld_q, scale, k, stream);
+  unsigned* err = nullptr;
+  cudaError_t e = coat::device_error_ptr(&err);
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  e = coat::launch_group_quantize(x, xt, rows, cols, ld_x, group_rows, expand, fmt, q, ld_q, scale,
+                                  k, err, stream);
   return e == cudaSuccess ? COAT_OK : cuda_fail(e, fn);
 }
 

@@ -48,7 +48,7 @@ cudaError_t launch_fp8_encode(const float* y, int64_t n, int fmt, uint8_t* q, cu
 cudaError_t launch_fp8_decode(const uint8_t* q, int64_t n, int fmt, float* out, cudaStream_t s);
 cudaError_t launch_group_quantize(const void* x, int xt, int64_t rows, int64_t cols, int64_t ldx,
                                   int gr, int expand, int fmt, uint8_t* q, int64_t ldq,
-                                  float* scale, float* k, cudaStream_t s);
+                                  float* scale, float* k, unsigned* err, cudaStream_t s);
 cudaError_t launch_group_dequantize(const uint8_t* q, int64_t ldq, const float* scale,
                                     const float* k, int64_t rows, int64_t cols, int gr, int gc,
                                     int fmt, void* out, int ot, int64_t ldo, cudaStream_t s);

@@ -118,17 +118,18 @@ __device__ __forceinline__ int clamp_valid(int64_t left, int width) {
   return left <= 0 ? 0 : (left >= width ? width : static_cast<int>(left));
 }
 
-// Max and min-nonzero of |x| over N values, on the FP32 bit patterns of |x|
-// (which order like the values): maxb = max bits(|x|) (above 0x7F800000 only
-// if a NaN is present, equal to it for an Inf), mink = min(bits(|x|) - 1), so
-// that zero becomes the largest key.
+// Max and min-nonzero of |x| over N values, on twice the FP32 bit patterns
+// (a = bits(x) * 2 drops the sign, one multiply-add off the integer ALU, and
+// orders like |x|): maxb = max a = 2 bits(max|x|) (at least 0xFF000000 iff an
+// Inf or NaN is present), mink = min(a - 2), so that zero becomes the largest
+// key and min nonzero |x| has bits (mink + 2) / 2.
 template <int N>
 __device__ __forceinline__ void stats_bits(const float (&v)[N], uint32_t& maxb, uint32_t& mink) {
 #pragma unroll
   for (int i = 0; i < N; ++i) {
-    const uint32_t a = __float_as_uint(v[i]) & 0x7FFFFFFFu;
+    const uint32_t a = __float_as_uint(v[i]) * 2u;
     maxb = max(maxb, a);
-    mink = min(mink, a - 1u);
+    mink = min(mink, a - 2u);
   }
 }
 
@@ -190,8 +191,8 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
       maxb = max(maxb, __shfl_xor_sync(0xFFFFFFFFu, maxb, off));
       mink = min(mink, __shfl_xor_sync(0xFFFFFFFFu, mink, off));
     }
-    const bool special = maxb >= 0x7F800000u;   // an Inf or a NaN in the group
-    float M = __uint_as_float(maxb);
+    const bool special = maxb >= 0xFF000000u;   // an Inf or a NaN in the group
+    float M = __uint_as_float(maxb >> 1);
     if (__any_sync(0xFFFFFFFFu, special)) {
       float Mn = max_abs_nonnan(v);
 #pragma unroll
@@ -199,7 +200,7 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
       if (special) M = Mn;
     }
     float k, sr, invM;
-    group_params<FMT>(M, __uint_as_float(mink + 1u), expand != 0, k, sr, invM);
+    group_params<FMT>(M, __uint_as_float((mink + 2u) >> 1), expand != 0, k, sr, invM);
     const bool use_div = k == 1.0f;
     GroupDiv d{};
     if (use_div) d = codec_div<FMT>(M);
@@ -337,8 +338,8 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
       maxb = max(maxb, sM[par][w]);
       mink = min(mink, sK[par][w]);
     }
-    const bool special = maxb >= 0x7F800000u;   // an Inf or a NaN in the block (CTA-uniform)
-    float M = __uint_as_float(maxb);
+    const bool special = maxb >= 0xFF000000u;   // an Inf or a NaN in the block (CTA-uniform)
+    float M = __uint_as_float(maxb >> 1);
     if (special) {
       // max |x| ignoring NaN, through the other half of the partials buffer
       float Mn = 0.f;
@@ -359,7 +360,7 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
     }
     par ^= 1;
     float k, sr, invM;
-    group_params<FMT>(M, __uint_as_float(mink + 1u), expand != 0, k, sr, invM);
+    group_params<FMT>(M, __uint_as_float((mink + 2u) >> 1), expand != 0, k, sr, invM);
     const bool use_div = k == 1.0f;
     GroupDiv d{};
     if (use_div) d = codec_div<FMT>(M);
@@ -407,21 +408,111 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
 // codes and group metadata are loaded before the current chunk is computed.
 // GR: rows per group (1 or 128).
 // ---------------------------------------------------------------------------
+// 16 values of one group from their codes: x = sign(q) s 2^(log2|q| / k), with
+// tabl = this lane's copy of the log2 table (entry c at tabl[32 c]).
+__device__ __forceinline__ void dequant16(const uint4& w, const float* tabl, float invk, float s,
+                                          float (&xv)[16]) {
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t wd = ws[i >> 2];
+    const uint32_t c = __byte_perm(wd, 0u, 0x4440u + (i & 3));
+    const float a = ex2_approx(tabl[c << 5] * invk) * s;
+    xv[i] = __uint_as_float(__float_as_uint(a) ^ ((wd << (24 - 8 * (i & 3))) & 0x80000000u));
+  }
+}
+
+template <int OT>
+__device__ __forceinline__ void store_out16(void* o, const float (&xv)[16]) {
+  if (OT == 0) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      reinterpret_cast<float4*>(o)[j] = make_float4(xv[4 * j], xv[4 * j + 1], xv[4 * j + 2], xv[4 * j + 3]);
+  } else {
+    uint32_t p[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) p[j] = pack_bf16x2(xv[2 * j], xv[2 * j + 1]);
+    reinterpret_cast<uint4*>(o)[0] = make_uint4(p[0], p[1], p[2], p[3]);
+    reinterpret_cast<uint4*>(o)[1] = make_uint4(p[4], p[5], p[6], p[7]);
+  }
+}
+
+// log2 table replicated once per lane (entry c of lane j at 32 c + j), so that
+// the per-element lookups of a warp never share a bank; called by the whole CTA.
+template <int FMT>
+__device__ __forceinline__ const float* lane_log2_table(float* tab1, float* tab) {
+  fill_log2_table<FMT>(tab1);
+  __syncthreads();
+  for (int e = threadIdx.x; e < 256 * 32; e += blockDim.x) tab[e] = tab1[e >> 5];
+  __syncthreads();
+  return tab + (threadIdx.x & 31);
+}
+
+// Rows whose width is a multiple of 16: every chunk is whole, and the code,
+// output and metadata positions advance with the stride by pointer increments.
+template <int FMT, int OT, int GR>
+__global__ void __launch_bounds__(256) dequant_full_kernel(const uint8_t* __restrict__ q,
+                                                           int64_t ldq,
+                                                           const float* __restrict__ scale,
+                                                           const float* __restrict__ kk,
+                                                           int64_t rows, int64_t cols,
+                                                           void* __restrict__ out, int64_t ldo) {
+  __shared__ float tab1[256];
+  __shared__ float tab[256 * 32];
+  const float* tabl = lane_log2_table<FMT>(tab1, tab);
+  constexpr int64_t kOsz = OT == 0 ? 4 : 2;
+  const int64_t cpr = cols / 16;  // chunks per row
+  const int64_t nbc = (cols + 127) / 128;
+  const int64_t t0 = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
+  const int64_t nt = int64_t(gridDim.x) * blockDim.x;
+  const int64_t dr = nt / cpr, dc = nt % cpr;
+  int64_t r = t0 / cpr, cc = t0 % cpr;
+  if (r >= rows) return;
+  // byte steps of the code and output pointers: without / with a row carry
+  const int64_t qs = dr * ldq + 16 * dc, qsc = qs + ldq - 16 * cpr;
+  const int64_t os = (dr * ldo + 16 * dc) * kOsz, osc = os + (ldo - 16 * cpr) * kOsz;
+  const uint8_t* qp = q + r * ldq + 16 * cc;
+  char* op = static_cast<char*>(out) + (r * ldo + 16 * cc) * kOsz;
+  auto group = [&](int64_t rr, int64_t ch) { return (GR == 1 ? rr : rr / GR) * nbc + (ch >> 3); };
+  uint4 w = __ldg(reinterpret_cast<const uint4*>(qp));
+  int64_t g = group(r, cc);
+  float s = __ldg(scale + g), kv = __ldg(kk + g);
+  while (true) {
+    int64_t rn = r + dr, cn = cc + dc;
+    const bool carry = cn >= cpr;
+    if (carry) { cn -= cpr; ++rn; }
+    const uint8_t* qpn = qp + (carry ? qsc : qs);
+    uint4 wn;
+    float sn, kn;
+    if (rn < rows) {
+      wn = __ldg(reinterpret_cast<const uint4*>(qpn));
+      const int64_t gn = group(rn, cn);
+      sn = __ldg(scale + gn);
+      kn = __ldg(kk + gn);
+    }
+    float xv[16];
+    dequant16(w, tabl, rcp_approx(kv), s, xv);
+    store_out16<OT>(op, xv);
+    if (rn >= rows) break;
+    op += carry ? osc : os;
+    qp = qpn;
+    r = rn;
+    cc = cn;
+    w = wn;
+    s = sn;
+    kv = kn;
+  }
+}
+
 template <int FMT, int OT, int GR>
 __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict__ q, int64_t ldq,
                                                       const float* __restrict__ scale,
                                                       const float* __restrict__ kk, int64_t rows,
                                                       int64_t cols, void* __restrict__ out,
                                                       int64_t ldo) {
-  // log2|value(code)|, replicated once per lane (entry c of lane j at 32 c + j)
-  // so that the per-element lookups of a warp never share a bank
   __shared__ float tab1[256];
   __shared__ float tab[256 * 32];
-  fill_log2_table<FMT>(tab1);
-  __syncthreads();
-  for (int e = threadIdx.x; e < 256 * 32; e += blockDim.x) tab[e] = tab1[e >> 5];
-  __syncthreads();
-  const float* tabl = tab + (threadIdx.x & 31);
+  const float* tabl = lane_log2_table<FMT>(tab1, tab);
   const int64_t cpr = (cols + 15) / 16;  // chunks per row
   const int64_t nbc = (cols + 127) / 128;
   const int64_t t0 = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
@@ -457,16 +548,8 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
     int validn;
     if (rn < rows) fetch(rn, cn, wn, sn, kn, validn);
 
-    const float invk = rcp_approx(kv);
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
     float xv[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const uint32_t wd = ws[i >> 2];
-      const uint32_t c = __byte_perm(wd, 0u, 0x4440u + (i & 3));
-      const float a = ex2_approx(tabl[c << 5] * invk) * s;
-      xv[i] = __uint_as_float(__float_as_uint(a) ^ ((wd << (24 - 8 * (i & 3))) & 0x80000000u));
-    }
+    dequant16(w, tabl, rcp_approx(kv), s, xv);
     const int64_t c0 = cc * 16;
     if (OT == 0) {
       float* o = static_cast<float*>(out) + r * ldo + c0;
@@ -510,16 +593,17 @@ unsigned grid_for(int64_t work_items, int per_block, int dev, int max_blocks_per
   return static_cast<unsigned>(b);
 }
 
-// CTAs of `kernel` (256 threads, static shared memory only) resident per SM,
+// CTAs of `kernel` (256 threads, plus dyn_smem bytes of dynamic shared memory) resident per SM,
 // from the occupancy calculator, cached per kernel (all B200s give the same).
 std::mutex g_occ_mu;
 std::unordered_map<const void*, int> g_occ;
-int resident_ctas(const void* kernel) {
+int resident_ctas(const void* kernel, size_t dyn_smem = 0) {
   std::lock_guard<std::mutex> lk(g_occ_mu);
   auto it = g_occ.find(kernel);
   if (it != g_occ.end()) return it->second;
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, 256, 0) != cudaSuccess || n < 1) {
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, 256, dyn_smem) != cudaSuccess ||
+      n < 1) {
     cudaGetLastError();
     n = 1;
   }
@@ -550,13 +634,14 @@ cudaError_t launch_fp8_decode(const uint8_t* q, int64_t n, int fmt, float* out, 
 }
 
 template <int FMT, int DT>
-static void quant_dispatch(const void* x, int64_t rows, int64_t cols, int64_t ldx, int gr,
-                           int expand, uint8_t* q, int64_t ldq, float* scale, float* k,
-                           int dev, cudaStream_t s) {
+static cudaError_t quant_dispatch(const void* x, int64_t rows, int64_t cols, int64_t ldx, int gr,
+                                  int expand, uint8_t* q, int64_t ldq, float* scale, float* k,
+                                  unsigned* err, int dev, cudaStream_t s) {
   if (gr == 1) {
     const int64_t quads = rows * (((cols + 127) / 128 + 3) / 4);
     auto kern = quant_row_kernel<FMT, DT>;
-    const unsigned g = grid_for(quads, 8, dev, resident_ctas(reinterpret_cast<const void*>(kern)));
+    const unsigned g =
+        grid_for(quads, 8, dev, resident_ctas(reinterpret_cast<const void*>(kern)));
     kern<<<g, 256, 0, s>>>(x, rows, cols, ldx, expand, q, ldq, scale, k);
   } else {
     const int64_t blocks = ((rows + 127) / 128) * ((cols + 127) / 128);
@@ -564,21 +649,24 @@ static void quant_dispatch(const void* x, int64_t rows, int64_t cols, int64_t ld
     const unsigned g = grid_for(blocks, 1, dev, resident_ctas(reinterpret_cast<const void*>(kern)));
     kern<<<g, 256, 0, s>>>(x, rows, cols, ldx, expand, q, ldq, scale, k);
   }
+  return cudaSuccess;
 }
 
 cudaError_t launch_group_quantize(const void* x, int xt, int64_t rows, int64_t cols, int64_t ldx,
                                   int gr, int expand, int fmt, uint8_t* q, int64_t ldq,
-                                  float* scale, float* k, cudaStream_t s) {
+                                  float* scale, float* k, unsigned* err, cudaStream_t s) {
   if (rows == 0 || cols == 0) return cudaSuccess;
   int dev = 0;
   cudaGetDevice(&dev);
+  cudaError_t e;
   if (fmt == kE4M3) {
-    if (xt == 0) quant_dispatch<kE4M3, 0>(x, rows, cols, ldx, gr, expand, q, ldq, scale, k, dev, s);
-    else quant_dispatch<kE4M3, 1>(x, rows, cols, ldx, gr, expand, q, ldq, scale, k, dev, s);
+    e = xt == 0 ? quant_dispatch<kE4M3, 0>(x, rows, cols, ldx, gr, expand, q, ldq, scale, k, err, dev, s)
+                : quant_dispatch<kE4M3, 1>(x, rows, cols, ldx, gr, expand, q, ldq, scale, k, err, dev, s);
   } else {
-    if (xt == 0) quant_dispatch<kE5M2, 0>(x, rows, cols, ldx, gr, expand, q, ldq, scale, k, dev, s);
-    else quant_dispatch<kE5M2, 1>(x, rows, cols, ldx, gr, expand, q, ldq, scale, k, dev, s);
+    e = xt == 0 ? quant_dispatch<kE5M2, 0>(x, rows, cols, ldx, gr, expand, q, ldq, scale, k, err, dev, s)
+                : quant_dispatch<kE5M2, 1>(x, rows, cols, ldx, gr, expand, q, ldq, scale, k, err, dev, s);
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -586,7 +674,9 @@ template <int FMT, int OT>
 static void dequant_dispatch(const uint8_t* q, int64_t ldq, const float* scale, const float* k,
                              int64_t rows, int64_t cols, int gr, void* out, int64_t ldo, int dev,
                              cudaStream_t s) {
-  auto kern = gr == 1 ? dequant_kernel<FMT, OT, 1> : dequant_kernel<FMT, OT, 128>;
+  auto kern = cols % 16 == 0
+                  ? (gr == 1 ? dequant_full_kernel<FMT, OT, 1> : dequant_full_kernel<FMT, OT, 128>)
+                  : (gr == 1 ? dequant_kernel<FMT, OT, 1> : dequant_kernel<FMT, OT, 128>);
   const unsigned g = grid_for(rows * ((cols + 15) / 16), 256, dev,
                               resident_ctas(reinterpret_cast<const void*>(kern)));
   kern<<<g, 256, 0, s>>>(q, ldq, scale, k, rows, cols, out, ldo);
