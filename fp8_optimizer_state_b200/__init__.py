@@ -40,6 +40,7 @@ EXPORTS = [
     ("coat_check_device_error", _i32, [_vp]),
     ("coat_adamw_step_multi_noalloc", _i32, [_vp, _i32, _i32, _f32, _f32, _f32, _f32, _f32, _i64,
                                              _i32, _i32, _vp]),
+    ("coat_selftest_wait_timeout", _i32, [_i64, _vp]),
 ]
 NOALLOC_MAX_TENSORS = 1024
 
@@ -210,3 +211,9 @@ def coat_adamw_step_multi_noalloc(descs, *, lr, beta1, beta2, eps, wd, step, fmt
 
 def coat_check_device_error(stream=None):
     _check(lib().coat_check_device_error(_s(stream)))
+
+
+def coat_selftest_wait_timeout(budget_cycles, stream=None):
+    """Enqueue one warp whose bounded wait on a barrier nothing arrives on runs
+    out; see include/coat.h."""
+    _check(lib().coat_selftest_wait_timeout(int(budget_cycles), _s(stream)))

@@ -593,4 +593,24 @@ cudaError_t launch_adamw_multi(const TensorArgs* d_descs, int num, int64_t total
   return dispatch(fm, fv, map, total_tiles, h, err, stream);
 }
 
+namespace {
+// One warp waits, with the given bound, on an mbarrier that nothing arrives on.
+__global__ void wait_timeout_selftest_kernel(long long budget, unsigned* err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bar, 0u, budget)) && threadIdx.x == 0)
+    atomicOr(err, kErrTimeoutConsumer);
+}
+}  // namespace
+
+cudaError_t launch_wait_timeout_selftest(long long budget_cycles, unsigned* err,
+                                         cudaStream_t stream) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(budget_cycles, err);
+  return cudaGetLastError();
+}
+
 }  // namespace coat

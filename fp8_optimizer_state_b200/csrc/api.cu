@@ -359,6 +359,18 @@ coat_status coat_multi_plan_info(coat_multi_plan_t plan, int64_t* total_elements
   return COAT_OK;
 }
 
+coat_status coat_selftest_wait_timeout(int64_t budget_cycles, cudaStream_t stream) {
+  const char* fn = "coat_selftest_wait_timeout";
+  constexpr int64_t kMaxBudget = 2000000000;   // the kernels' own bound, about one second
+  if (budget_cycles < 1000 || budget_cycles > kMaxBudget)
+    return fail(COAT_ERR_INVALID_ARG, "%s: budget_cycles must be in [1000, %lld]", fn,
+                static_cast<long long>(kMaxBudget));
+  unsigned* err = nullptr;
+  cudaError_t e = coat::device_error_ptr(&err);
+  if (e == cudaSuccess) e = coat::launch_wait_timeout_selftest(budget_cycles, err, stream);
+  return e == cudaSuccess ? COAT_OK : cuda_fail(e, fn);
+}
+
 coat_status coat_check_device_error(cudaStream_t stream) {
   cudaError_t e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) return cuda_fail(e, "coat_check_device_error");

@@ -44,6 +44,10 @@ cudaError_t launch_adamw_single(const TensorArgs& t, int fm, int fv, const StepH
 cudaError_t launch_adamw_multi(const TensorArgs* d_descs, int num, int64_t total_tiles, int fm,
                                int fv, const StepHyper& h, unsigned* err, cudaStream_t stream);
 
+// One warp waits (bounded by budget_cycles) on a barrier nothing arrives on.
+cudaError_t launch_wait_timeout_selftest(long long budget_cycles, unsigned* err,
+                                         cudaStream_t stream);
+
 cudaError_t launch_fp8_encode(const float* y, int64_t n, int fmt, uint8_t* q, cudaStream_t s);
 cudaError_t launch_fp8_decode(const uint8_t* q, int64_t n, int fmt, float* out, cudaStream_t s);
 cudaError_t launch_group_quantize(const void* x, int xt, int64_t rows, int64_t cols, int64_t ldx,

@@ -226,6 +226,16 @@ coat_status coat_adamw_step_multi_noalloc(const coat_tensor_desc *host_descs, in
  * ------------------------------------------------------------------------- */
 coat_status coat_check_device_error(cudaStream_t stream);
 
+/* Self-test of the bounded waits (the COAT pages have no counterpart; this
+ * exists to test the failure path without a GPU fault).  Enqueues on `stream`
+ * one warp that waits, for at most budget_cycles SM clock cycles (1000 ..
+ * 2e9), on a shared-memory barrier that nothing ever arrives on; the warp gives
+ * up, sets the device error word and exits.  A following
+ * coat_check_device_error(stream) returns COAT_ERR_TIMEOUT and clears the
+ * word; the context stays usable.  Returns COAT_ERR_INVALID_ARG for a budget
+ * out of range, COAT_ERR_CUDA if the launch fails. */
+coat_status coat_selftest_wait_timeout(int64_t budget_cycles, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -80,6 +80,13 @@ def test_step_validation():
     assert "aligned" in coat.coat_last_error() or coat.coat_last_error() != ""
 
 
+def test_selftest_budget_validation():
+    L = coat.lib()
+    assert L.coat_selftest_wait_timeout(999, None) == INVALID
+    assert L.coat_selftest_wait_timeout(2000000001, None) == INVALID
+    assert "budget_cycles" in coat.coat_last_error()
+
+
 def test_codec_validation():
     L = coat.lib()
     q = lambda **k: L.coat_group_quantize(k.get("x", A), k.get("xt", 1), k.get("rows", 8),

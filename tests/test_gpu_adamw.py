@@ -258,6 +258,20 @@ def test_degenerate_groups_exact(orc):
         assert np.allclose(h["master"], ora.master, rtol=1e-6, atol=1e-10)
 
 
+def test_bounded_wait_gives_up_and_context_stays_usable(orc):
+    """A wait on a barrier that nothing arrives on runs out (short budget), the
+    device error word reports it once, and the next step still matches the
+    oracle: the failure is reported on the host without a GPU fault."""
+    coat.coat_check_device_error()                       # start clean
+    coat.coat_selftest_wait_timeout(2_000_000)           # ~1 ms of SM clock
+    with pytest.raises(coat.CoatError) as ei:
+        coat.coat_check_device_error()
+    assert ei.value.status == 5 and "bounded wait" in str(ei.value)   # COAT_ERR_TIMEOUT
+    coat.coat_check_device_error()                       # read once, then cleared
+    one_step_identical(orc, 4096 + 33, E4M3, E5M2, 1, tensor=11)
+    coat.coat_check_device_error()
+
+
 def test_zero_length_and_device_error_clear():
     e = torch.empty(0, device="cuda")
     coat.coat_adamw_step(e, None, e, e, e, e, e, e, e, lr=1e-3, beta1=0.9, beta2=0.95, eps=1e-8,
