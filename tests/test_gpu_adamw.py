@@ -272,6 +272,34 @@ def test_bounded_wait_gives_up_and_context_stays_usable(orc):
     coat.coat_check_device_error()
 
 
+@pytest.mark.parametrize("lr", [0.0, 1e-40])
+def test_no_adaptive_term_when_lr_is_zero_or_vanishing(orc, lr):
+    """lr = 0 (or so small that lr / (1 - beta1^t) leaves FP32 range) leaves the
+    master unchanged up to the decay p lr wd (zero here, or below FP32
+    resolution), while the moments still update and requantise as the oracle
+    does."""
+    n, t = 3 * 4096 + 77, 3
+    master = synth.master(0, 21, 0, n)
+    st = gen_state(n, 21, t, E4M3, E5M2)
+    gpu = GpuSide(master, E4M3, E5M2).set_state(st)
+    ora = OracleSide(orc, master, E4M3, E5M2).set_state(st)
+    g = synth.grad_bits(0, 21, t, 0, n)
+    gpu.grad.copy_(torch.from_numpy(g.view(np.int16)))
+    hp = dict(H, lr=lr)
+    coat.coat_adamw_step(gpu.master, gpu.weight, gpu.grad, gpu.mq, gpu.ms, gpu.mk, gpu.vq, gpu.vs,
+                         gpu.vk, lr=hp["lr"], beta1=hp["beta1"], beta2=hp["beta2"], eps=hp["eps"],
+                         wd=hp["wd"], step=t, fmt_m=E4M3, fmt_v=E5M2)
+    ora.orc.adamw_step(ora.master, ora.weight, g, ora.mq, ora.ms, ora.mk, ora.vq, ora.vs, ora.vk,
+                       lr=hp["lr"], beta1=hp["beta1"], beta2=hp["beta2"], eps=hp["eps"],
+                       wd=hp["wd"], step=t, fmt_m=E4M3, fmt_v=E5M2)
+    h = gpu.host()
+    assert np.array_equal(h["master"], master)          # no update at FP32 resolution
+    assert np.all(np.abs(ora.master.astype(np.float64) - master) <= 1e-30)
+    check_state_all("m", n, E4M3, h["mq"], h["ms"], h["mk"], ora.mq, ora.ms, ora.mk)
+    check_state_all("v", n, E5M2, h["vq"], h["vs"], h["vk"], ora.vq, ora.vs, ora.vk)
+    coat.coat_check_device_error()
+
+
 def test_zero_length_and_device_error_clear():
     e = torch.empty(0, device="cuda")
     coat.coat_adamw_step(e, None, e, e, e, e, e, e, e, lr=1e-3, beta1=0.9, beta2=0.95, eps=1e-8,
