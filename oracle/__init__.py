@@ -20,6 +20,7 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 
 E4M3 = 0
 E5M2 = 1
+E5M2_FULL = 2   # E5M2 codes, expansion to E5M2's own span
 
 _lib = None
 
@@ -54,7 +55,7 @@ def lib():
         L.orc_fmt_max.restype = ctypes.c_double
         L.orc_fmt_max.argtypes = [ctypes.c_int]
         L.orc_target_range.restype = ctypes.c_double
-        L.orc_target_range.argtypes = []
+        L.orc_target_range.argtypes = [ctypes.c_int]
         L.orc_float_to_bf16.restype = ctypes.c_uint16
         L.orc_float_to_bf16.argtypes = [ctypes.c_float]
         L.orc_group_params.restype = ctypes.c_double
@@ -126,8 +127,9 @@ def fmt_max(fmt: int) -> float:
     return lib().orc_fmt_max(fmt)
 
 
-def target_range() -> float:
-    return lib().orc_target_range()
+def target_range(fmt: int = 0) -> float:
+    """448 / 2^-9 for E4M3 and E5M2; 57344 / 2^-16 for E5M2_FULL."""
+    return lib().orc_target_range(fmt)
 
 
 def float_to_bf16_bits(x) -> np.ndarray:

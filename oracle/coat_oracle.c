@@ -46,6 +46,9 @@
 
 #define ORC_E4M3 0
 #define ORC_E5M2 1
+/* E5M2 codes whose expansion targets E5M2's own span (57344 / 2^-16) instead
+ * of E4M3's; as a number format it is E5M2. */
+#define ORC_E5M2_FULL 2
 
 /* ------------------------------------------------------------------ */
 /* FP8 formats, straight from the bit definitions ([P4] 格式选择).     */
@@ -87,8 +90,8 @@ static unsigned orc_max_code(int fmt) { return fmt == ORC_E4M3 ? 0x7Eu : 0x7Bu; 
 double orc_fmt_max(int fmt) { return orc_fp8_decode(fmt, orc_max_code(fmt)); }
 
 /* Positive finite values by code, filled on first use from orc_fp8_decode. */
-static double g_table[2][128];
-static int g_table_ready[2];
+static double g_table[3][128];
+static int g_table_ready[3];
 
 static const double *orc_table(int fmt)
 {
@@ -170,9 +173,14 @@ uint16_t orc_float_to_bf16(float f)
 /* ------------------------------------------------------------------ */
 
 /* The span the expansion aims for: E4M3's largest over smallest positive
- * value, 448 / 2^-9 ([P1] FP8优化器状态: 0.00195 ... 448, about 200000). */
-double orc_target_range(void)
+ * value, 448 / 2^-9 ([P1] FP8优化器状态: 0.00195 ... 448, about 200000), for
+ * E4M3 and E5M2 alike; for ORC_E5M2_FULL, E5M2's own largest over smallest
+ * positive value, 57344 / 2^-16 (the reading under which [P1] 解决方案：动态范围扩展's
+ * "E4M3 and E5M2 almost the same after expansion" for v holds). */
+double orc_target_range(int fmt)
 {
+    if (fmt == ORC_E5M2_FULL)
+        return orc_fp8_decode(ORC_E5M2, 0x7B) / orc_fp8_decode(ORC_E5M2, 0x01);
     return orc_fp8_decode(ORC_E4M3, 0x7E) / orc_fp8_decode(ORC_E4M3, 0x01);
 }
 
@@ -203,7 +211,7 @@ double orc_group_params(const double *x, int64_t cnt, int expand, int fmt,
     else if (M == mu)
         k = 16.0;
     else {
-        k = log(orc_target_range()) / log(M / mu);
+        k = log(orc_target_range(fmt)) / log(M / mu);
         if (k < 1.0)
             k = 1.0;
         if (k > 16.0)

@@ -19,9 +19,10 @@ import numpy as np
 import pytest
 import torch
 
-E4M3, E5M2 = 0, 1
+E4M3, E5M2, E5M2_FULL = 0, 1, 2
 R = 448.0 / 2.0 ** -9
-FMAX = {E4M3: 448.0, E5M2: 57344.0}
+R5 = 57344.0 / 2.0 ** -16   # E5M2's own span (the full-span reading)
+FMAX = {E4M3: 448.0, E5M2: 57344.0, E5M2_FULL: 57344.0}
 TORCH_DT = {E4M3: torch.float8_e4m3fn, E5M2: torch.float8_e5m2}
 
 
@@ -43,25 +44,29 @@ def loguniform_group(rng, n, ratio, sign=True):
 # ---------------------------------------------------------------------------
 # T3: the defining invariant of the expansion
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+@pytest.mark.parametrize("fmt", [E4M3, E5M2, E5M2_FULL])
 def test_expanded_span_equals_target(orc, fmt):
     rng = np.random.default_rng(10)
-    for ratio in [R ** (1 / 16) * 1.01, 3.0, 10.0, 100.0, 1000.0, 1e4, R * 0.999]:
+    Rf = R5 if fmt == E5M2_FULL else R
+    for ratio in [Rf ** (1 / 16) * 1.01, 3.0, 10.0, 100.0, 1000.0, 1e4, R * 0.999]:
+        if ratio < Rf ** (1 / 16):
+            continue                      # k would clamp at 16 (checked separately)
         x = loguniform_group(rng, 128, ratio) * 3e-4
         M, k, s = orc.group_params(x, True, fmt)
         a = np.abs(x)
         mu = a[a > 0].min()
         assert M == a.max()
-        expect_k = math.log(R) / math.log(M / mu)
+        expect_k = math.log(Rf) / math.log(M / mu)
         assert abs(k - expect_k) <= 1e-6 * expect_k
-        # expanded max / expanded min == R (k rounded to FP32: ~1e-6 relative)
-        assert abs((M / mu) ** k / R - 1) < 2e-6
+        # expanded max / expanded min == the target span (k rounded to FP32: ~1e-6 relative)
+        assert abs((M / mu) ** k / Rf - 1) < 2e-6 * max(1.0, k / 8)
         codes, k2, s2 = orc.quantize_group(x, True, fmt)
         assert (k2, s2) == (k, s)
         i_max, i_min = int(np.argmax(a)), int(np.argmin(np.where(a > 0, a, np.inf)))
         assert codes[i_max] & 0x7F == (0x7E if fmt == E4M3 else 0x7B)
-        # min maps to FMT_MAX/R: 2^-9 (E4M3 code 0x01) or 0.25 (E5M2 code 0x34)
-        assert codes[i_min] & 0x7F == (0x01 if fmt == E4M3 else 0x34)
+        # min maps to FMT_MAX/R: 2^-9 (E4M3 code 0x01), 0.25 (E5M2 code 0x34), or
+        # E5M2's own smallest value 2^-16 (code 0x01) with the full-span target
+        assert codes[i_min] & 0x7F == {E4M3: 0x01, E5M2: 0x34, E5M2_FULL: 0x01}[fmt]
         # the root scale brings the max code back to M
         assert abs(s * FMAX[fmt] ** (1 / k) / M - 1) < 2e-7
 
@@ -208,6 +213,24 @@ def _mse(orc, groups, fmt, expand):
         xr = np.array([orc.dequant_value(fmt, c, s, k) for c in q])
         err += float(np.mean((xr - x) ** 2))
     return err / len(groups)
+
+
+def test_e5m2_matches_e4m3_for_v_only_with_its_own_span(orc):
+    """Same section: after expansion E4M3 and E5M2 are almost the same for the
+    second moment.  With the literal target 448 / 2^-9 E5M2's error stays
+    several times E4M3's; expanding to E5M2's own span 57344 / 2^-16 brings it
+    to within a few percent of E4M3's."""
+    rng = np.random.default_rng(15)
+    v_groups = [loguniform_group(rng, 128, 10.0, sign=False) * 1e-6 for _ in range(60)]
+    e4 = _mse(orc, v_groups, E4M3, True)
+    e5 = _mse(orc, v_groups, E5M2, True)
+    e5f = _mse(orc, v_groups, E5M2_FULL, True)
+    assert e5 > 2.0 * e4
+    assert abs(e5f / e4 - 1.0) < 0.25
+    # and the full-span k is larger: the group is stretched over more binades
+    k4 = orc.group_params(v_groups[0], True, E4M3)[1]
+    k5f = orc.group_params(v_groups[0], True, E5M2_FULL)[1]
+    assert abs(k5f / k4 - math.log(R5) / math.log(R)) < 1e-6
 
 
 def test_expansion_reduces_error_on_pages_ratios(orc):

@@ -61,6 +61,8 @@ def test_e4m3_printed_constants(orc, pages):
     # "about 200000": within the page's one-significant-digit precision
     assert abs(rng - pages["e4m3_dynamic_range_approx"]) / pages["e4m3_dynamic_range_approx"] < 0.2
     assert orc.target_range() == rng
+    assert orc.target_range(1) == rng                       # E5M2: the same literal span
+    assert orc.target_range(2) == 57344.0 * 2.0 ** 16          # E5M2's own span
     # the group ratios the page reports are far below that range
     assert pages["first_moment_group_max_min_ratio_typical"] < rng
     assert pages["second_moment_group_max_min_ratio_typical"] < rng
