@@ -393,8 +393,8 @@ def run_ours(args, cfg, ws, rank, local):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": cfg["workload"], "params_per_gpu": n_params,
                        "tensors": n_tensors, "group": 128,
-                       "fmt_m": "E4M3" if cfg["fmt_m"] == 0 else "E5M2",
-                       "fmt_v": "E4M3" if cfg["fmt_v"] == 0 else "E5M2",
+                       "fmt_m": FMT_NAMES[cfg["fmt_m"]],
+                       "fmt_v": FMT_NAMES[cfg["fmt_v"]],
                        "hyper": H, "l2": "no flush: %.1f GB of inputs per step >> 126 MB L2"
                                          % (alg / 1e9),
                        "parallelism": "replicas%d (independent parameter groups, no collective)" % ws
@@ -473,6 +473,7 @@ def run_e2e(args, cfg, ps, ws, dev, H, coat):
 # per-token groups and weights bf16 [4096 x 11008] with 128x128 blocks, to E4M3,
 # expansion off and on, then the dequantisation round trip to bf16
 # ----------------------------------------------------------------------------
+FMT_NAMES = {0: "E4M3", 1: "E5M2", 2: "E5M2 (expanded to its own span)"}
 CODEC_METRIC = "GB/s of the FP8 group codec (quantize + dequantize); HBM GB/s as % of B200 roofline"
 CODEC_ACT = (8192, 4096)
 CODEC_COPIES = 3
@@ -690,6 +691,8 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fmt-v", type=int, choices=[0, 1, 2], default=None,
+                    help="override the workload's v format (2: E5M2 expanded to its own span)")
     ap.add_argument("--compare-flat", action="store_true",
                     help="also time one flat tensor of the same parameter count")
     ap.add_argument("--cpu-sample", type=int, default=16 << 20)
@@ -707,7 +710,10 @@ def main(argv=None):
         if res is not None:
             print(json.dumps(res), flush=True)
         return
-    cfg = CONFIGS[args.config]
+    cfg = dict(CONFIGS[args.config])
+    if args.fmt_v is not None and args.fmt_v != cfg["fmt_v"]:
+        cfg["fmt_v"] = args.fmt_v
+        cfg["workload"] = cfg["workload"].split(", E4M3")[0] + ", E4M3 m + %s v" % FMT_NAMES[args.fmt_v]
     if args.impl == "reference":
         res = run_reference(args, cfg, ws, rank)
     else:

@@ -14,7 +14,7 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libcoat.so")
 
-COAT_E4M3, COAT_E5M2 = 0, 1
+COAT_E4M3, COAT_E5M2, COAT_E5M2_FULL = 0, 1, 2
 COAT_F32, COAT_BF16 = 0, 1
 GROUP = 128
 STATUS = {0: "COAT_OK", 1: "COAT_ERR_INVALID_ARG", 2: "COAT_ERR_MISALIGNED",

@@ -375,7 +375,8 @@ __device__ __forceinline__ void process(const LaneIn& in, const TileHeader& t, c
   float kx, srx, invMx;
   group_params_rt(vlane ? maxv : maxm, vlane ? muv : mum, true,
                   vlane ? F8<FV>::LOG2MAX_HI : F8<FM>::LOG2MAX_HI,
-                  vlane ? F8<FV>::LOG2MAX_LO : F8<FM>::LOG2MAX_LO, kx, srx, invMx);
+                  vlane ? F8<FV>::LOG2MAX_LO : F8<FM>::LOG2MAX_LO,
+                  vlane ? F8<FV>::LOG2_TARGET : F8<FM>::LOG2_TARGET, kx, srx, invMx);
   const int lane_m = slot << 3, lane_v = lane_m + 4;
   const float km = __shfl_sync(0xFFFFFFFFu, kx, lane_m);
   const float invMm = __shfl_sync(0xFFFFFFFFu, invMx, lane_m);
@@ -571,10 +572,19 @@ cudaError_t launch_step(const Map& map, int64_t ntiles, const StepHyper& h, unsi
 template <class Map>
 cudaError_t dispatch(int fm, int fv, const Map& map, int64_t ntiles, const StepHyper& h,
                      unsigned* err, cudaStream_t stream) {
-  if (fm == kE4M3 && fv == kE4M3) return launch_step<kE4M3, kE4M3>(map, ntiles, h, err, stream);
-  if (fm == kE4M3 && fv == kE5M2) return launch_step<kE4M3, kE5M2>(map, ntiles, h, err, stream);
-  if (fm == kE5M2 && fv == kE4M3) return launch_step<kE5M2, kE4M3>(map, ntiles, h, err, stream);
-  return launch_step<kE5M2, kE5M2>(map, ntiles, h, err, stream);
+  switch (fm * 3 + fv) {
+    case kE4M3 * 3 + kE4M3: return launch_step<kE4M3, kE4M3>(map, ntiles, h, err, stream);
+    case kE4M3 * 3 + kE5M2: return launch_step<kE4M3, kE5M2>(map, ntiles, h, err, stream);
+    case kE4M3 * 3 + kE5M2Full: return launch_step<kE4M3, kE5M2Full>(map, ntiles, h, err, stream);
+    case kE5M2 * 3 + kE4M3: return launch_step<kE5M2, kE4M3>(map, ntiles, h, err, stream);
+    case kE5M2 * 3 + kE5M2: return launch_step<kE5M2, kE5M2>(map, ntiles, h, err, stream);
+    case kE5M2 * 3 + kE5M2Full: return launch_step<kE5M2, kE5M2Full>(map, ntiles, h, err, stream);
+    case kE5M2Full * 3 + kE4M3: return launch_step<kE5M2Full, kE4M3>(map, ntiles, h, err, stream);
+    case kE5M2Full * 3 + kE5M2: return launch_step<kE5M2Full, kE5M2>(map, ntiles, h, err, stream);
+    case kE5M2Full * 3 + kE5M2Full:
+      return launch_step<kE5M2Full, kE5M2Full>(map, ntiles, h, err, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace

@@ -34,7 +34,7 @@ coat_status cuda_fail(cudaError_t e, const char* where) {
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
-bool valid_fmt(int f) { return f == COAT_E4M3 || f == COAT_E5M2; }
+bool valid_fmt(int f) { return f == COAT_E4M3 || f == COAT_E5M2 || f == COAT_E5M2_FULL; }
 bool valid_dtype(int d) { return d == COAT_F32 || d == COAT_BF16; }
 size_t dtype_size(int d) { return d == COAT_F32 ? 4 : 2; }
 

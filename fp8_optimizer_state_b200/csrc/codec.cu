@@ -619,7 +619,7 @@ cudaError_t launch_fp8_encode(const float* y, int64_t n, int fmt, uint8_t* q, cu
   cudaGetDevice(&dev);
   const unsigned g = grid_for(n, 256, dev, 16);
   if (fmt == kE4M3) fp8_encode_kernel<kE4M3><<<g, 256, 0, s>>>(y, n, q);
-  else fp8_encode_kernel<kE5M2><<<g, 256, 0, s>>>(y, n, q);
+  else fp8_encode_kernel<kE5M2><<<g, 256, 0, s>>>(y, n, q);   // E5M2 and E5M2 full span
   return cudaGetLastError();
 }
 
@@ -629,7 +629,7 @@ cudaError_t launch_fp8_decode(const uint8_t* q, int64_t n, int fmt, float* out, 
   cudaGetDevice(&dev);
   const unsigned g = grid_for(n, 256, dev, 16);
   if (fmt == kE4M3) fp8_decode_kernel<kE4M3><<<g, 256, 0, s>>>(q, n, out);
-  else fp8_decode_kernel<kE5M2><<<g, 256, 0, s>>>(q, n, out);
+  else fp8_decode_kernel<kE5M2><<<g, 256, 0, s>>>(q, n, out);   // E5M2 and E5M2 full span
   return cudaGetLastError();
 }
 
@@ -662,9 +662,13 @@ cudaError_t launch_group_quantize(const void* x, int xt, int64_t rows, int64_t c
   if (fmt == kE4M3) {
     e = xt == 0 ? quant_dispatch<kE4M3, 0>(x, rows, cols, ldx, gr, expand, q, ldq, scale, k, err, dev, s)
                 : quant_dispatch<kE4M3, 1>(x, rows, cols, ldx, gr, expand, q, ldq, scale, k, err, dev, s);
-  } else {
+  } else if (fmt == kE5M2) {
     e = xt == 0 ? quant_dispatch<kE5M2, 0>(x, rows, cols, ldx, gr, expand, q, ldq, scale, k, err, dev, s)
                 : quant_dispatch<kE5M2, 1>(x, rows, cols, ldx, gr, expand, q, ldq, scale, k, err, dev, s);
+  } else {
+    e = xt == 0
+            ? quant_dispatch<kE5M2Full, 0>(x, rows, cols, ldx, gr, expand, q, ldq, scale, k, err, dev, s)
+            : quant_dispatch<kE5M2Full, 1>(x, rows, cols, ldx, gr, expand, q, ldq, scale, k, err, dev, s);
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -692,7 +696,7 @@ cudaError_t launch_group_dequantize(const uint8_t* q, int64_t ldq, const float* 
   if (fmt == kE4M3) {
     if (ot == 0) dequant_dispatch<kE4M3, 0>(q, ldq, scale, k, rows, cols, gr, out, ldo, dev, s);
     else dequant_dispatch<kE4M3, 1>(q, ldq, scale, k, rows, cols, gr, out, ldo, dev, s);
-  } else {
+  } else {   // E5M2 and E5M2 full span: the same codes
     if (ot == 0) dequant_dispatch<kE5M2, 0>(q, ldq, scale, k, rows, cols, gr, out, ldo, dev, s);
     else dequant_dispatch<kE5M2, 1>(q, ldq, scale, k, rows, cols, gr, out, ldo, dev, s);
   }

@@ -49,7 +49,13 @@
 extern "C" {
 #endif
 
-typedef enum { COAT_E4M3 = 0, COAT_E5M2 = 1 } coat_fmt;
+/* COAT_E5M2_FULL stores E5M2 codes like COAT_E5M2, but the dynamic-range
+ * expansion stretches a group to E5M2's own span (57344 / 2^-16, log2 31.8)
+ * instead of E4M3's 448 / 2^-9: k = clamp(ln(57344 / 2^-16) / ln(M / mu), 1, 16).
+ * With it E5M2 moments match E4M3's error after expansion, as [P1]
+ * 解决方案：动态范围扩展 reports for the second moment.  For the element codec
+ * (coat_fp8_encode/decode) and for dequantisation it is identical to E5M2. */
+typedef enum { COAT_E4M3 = 0, COAT_E5M2 = 1, COAT_E5M2_FULL = 2 } coat_fmt;
 typedef enum { COAT_F32 = 0, COAT_BF16 = 1 } coat_dtype;
 
 typedef enum {

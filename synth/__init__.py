@@ -177,7 +177,7 @@ def weight_bits(seed, tensor, start, count):
 # [0.02, 0.06) (largest |m| ~ s_g); k_v in [4, 8) (span ~5..22), s_v = s_g^2 *
 # [0.1, 0.3).  `step` selects an independent draw per step.
 # ----------------------------------------------------------------------------
-CODE_RANGE = {0: (0x01, 0x7E), 1: (0x34, 0x7B)}
+CODE_RANGE = {0: (0x01, 0x7E), 1: (0x34, 0x7B), 2: (0x01, 0x7B)}   # E5M2 full span: 2^-16..57344
 
 
 def _unit24(u):

@@ -150,7 +150,8 @@ int synth_weight(uint16_t* out, int64_t count, uint32_t seed, uint32_t tensor, i
 
 int synth_state_codes(uint8_t* out, int64_t count, uint32_t seed, uint32_t tensor, uint32_t step,
                       int64_t start, int fmt, int is_signed, cudaStream_t s) {
-  const uint32_t lo = fmt == 0 ? 0x01u : 0x34u, hi = fmt == 0 ? 0x7Eu : 0x7Bu;
+  // E4M3 0x01-0x7E; E5M2 0x34-0x7B (the literal span); E5M2 full span 0x01-0x7B
+  const uint32_t lo = fmt == 1 ? 0x34u : 0x01u, hi = fmt == 0 ? 0x7Eu : 0x7Bu;
   return launch(count, s, [=] __device__(int64_t t) {
     const Words u = draw(seed, is_signed ? MCODE : VCODE, start + t, tensor, step);
     uint32_t c = lo + u.w0 % (hi - lo + 1u);

@@ -38,7 +38,7 @@ import numpy as np
 K_RTOL = 1e-5
 FLIP_FRACTION = 1e-4
 MASTER_RTOL = 1e-6
-FMT_MAX = {0: 448.0, 1: 57344.0}
+FMT_MAX = {0: 448.0, 1: 57344.0, 2: 57344.0}   # E4M3, E5M2, E5M2 full span
 
 
 def scale_rtol(k, fmt):

@@ -62,7 +62,7 @@ def test_step_validation():
     assert step(n=-1) == INVALID
     assert step(group=0) == INVALID
     assert step(group=64) == UNSUPPORTED
-    assert step(fm=2) == INVALID and step(fv=-1) == INVALID
+    assert step(fm=3) == INVALID and step(fv=-1) == INVALID
     assert step(lr=-1.0) == INVALID and step(lr=float("nan")) == INVALID
     assert step(b1=1.0) == INVALID and step(b2=-0.1) == INVALID
     assert step(eps=0.0) == INVALID and step(wd=-0.5) == INVALID

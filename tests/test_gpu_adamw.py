@@ -17,7 +17,7 @@ from tests.parity import FreeRun, bf16_rne_bits, check_master, check_state_all
 
 pytestmark = pytest.mark.gpu
 H = P.HYPER
-E4M3, E5M2 = 0, 1
+E4M3, E5M2, E5M2_FULL = 0, 1, 2
 
 
 def to_dev(a, dtype=None):
@@ -140,7 +140,8 @@ def test_one_step_identical_inputs_tiny(orc, t):
     print("t=%d code flips m %d v %d of %d" % (t, flips[0], flips[1], 1 << 20))
 
 
-@pytest.mark.parametrize("fm,fv", [(E4M3, E5M2), (E5M2, E5M2), (E5M2, E4M3)])
+@pytest.mark.parametrize("fm,fv", [(E4M3, E5M2), (E5M2, E5M2), (E5M2, E4M3), (E4M3, E5M2_FULL),
+                                   (E5M2_FULL, E5M2_FULL)])
 def test_one_step_identical_inputs_formats(orc, fm, fv):
     one_step_identical(orc, 300000, fm, fv, 3, tensor=fm * 2 + fv)
 

@@ -9,7 +9,7 @@ import synth
 from tests.parity import compare_codes, rel_err, scale_rtol, K_RTOL, FLIP_FRACTION
 
 pytestmark = pytest.mark.gpu
-E4M3, E5M2 = 0, 1
+E4M3, E5M2, E5M2_FULL = 0, 1, 2
 TORCH_DT = {E4M3: torch.float8_e4m3fn, E5M2: torch.float8_e5m2}
 
 
@@ -92,7 +92,7 @@ CASES = [(1, 128, 200, 1000), (1, 128, 64, 4096), (128, 128, 300, 260), (128, 12
 
 
 @pytest.mark.parametrize("gr,gc,rows,cols", CASES)
-@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+@pytest.mark.parametrize("fmt", [E4M3, E5M2, E5M2_FULL])
 @pytest.mark.parametrize("expand", [False, True])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_group_quantize_vs_oracle(orc, gr, gc, rows, cols, fmt, expand, dtype):
@@ -121,7 +121,7 @@ def test_group_quantize_vs_oracle(orc, gr, gc, rows, cols, fmt, expand, dtype):
 
 
 @pytest.mark.parametrize("gr", [1, 128])
-@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+@pytest.mark.parametrize("fmt", [E4M3, E5M2, E5M2_FULL])
 @pytest.mark.parametrize("expand", [False, True])
 def test_group_quantize_special_values(orc, gr, fmt, expand):
     """Groups holding NaN or +-Inf follow the oracle: the maximum ignores NaN, a
@@ -175,7 +175,7 @@ def test_group_quantize_special_values(orc, gr, fmt, expand):
 
 
 @pytest.mark.parametrize("gr", [1, 128])
-@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+@pytest.mark.parametrize("fmt", [E4M3, E5M2, E5M2_FULL])
 def test_group_dequantize_vs_oracle(orc, gr, fmt):
     rows, cols = 256, 640
     rng = np.random.default_rng(30 + gr + fmt)

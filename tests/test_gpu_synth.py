@@ -24,3 +24,11 @@ def test_device_matches_host(start, count):
     assert np.array_equal(b.cpu().numpy().view(np.uint16), synth.activations_bits(0, 4, start, count))
     synth.device_weight(b, 0, 4, start)
     assert np.array_equal(b.cpu().numpy().view(np.uint16), synth.weight_bits(0, 4, start, count))
+
+
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+def test_state_codes_device_matches_host(fmt):
+    out = torch.empty(5000, dtype=torch.uint8, device="cuda")
+    for signed in (False, True):
+        synth.device_state_codes(out, 0, 3, 2, fmt, signed, 777)
+        assert np.array_equal(out.cpu().numpy(), synth.state_codes(0, 3, 2, 777, 5000, fmt, signed))
