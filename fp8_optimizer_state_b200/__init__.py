@@ -36,6 +36,7 @@ EXPORTS = [
     ("coat_multi_plan_create", _i32, [_vp, _i32, _i32, _i32, _i32, _vp, ctypes.POINTER(_vp)]),
     ("coat_adamw_step_multi", _i32, [_vp, _f32, _f32, _f32, _f32, _f32, _i64, _vp]),
     ("coat_multi_plan_destroy", _i32, [_vp]),
+    ("coat_multi_plan_set_wd_scale", _i32, [_vp, _vp, _vp]),
     ("coat_multi_plan_info", _i32, [_vp, ctypes.POINTER(_i64), ctypes.POINTER(_i32)]),
     ("coat_check_device_error", _i32, [_vp]),
     ("coat_adamw_step_multi_noalloc", _i32, [_vp, _i32, _i32, _f32, _f32, _f32, _f32, _f32, _i64,
@@ -167,6 +168,12 @@ class coat_multi_plan:
         c = ctypes.c_int()
         _check(lib().coat_multi_plan_info(self.handle, ctypes.byref(n), ctypes.byref(c)))
         return n.value, c.value
+
+    def set_wd_scale(self, scales, stream=None):
+        """Per-tensor weight decay multipliers (coat_multi_plan_set_wd_scale)."""
+        arr = (ctypes.c_float * len(scales))(*[float(x) for x in scales])
+        _check(lib().coat_multi_plan_set_wd_scale(self.handle, ctypes.cast(arr, ctypes.c_void_p),
+                                                  _s(stream)))
 
     def destroy(self):
         if self.handle:

@@ -80,6 +80,7 @@ struct __align__(16) TileHeader {
   const uint16_t* grad;
   int32_t nvalid;   // elements of the tile that exist (kTileElems: full tile, staged)
   int32_t ngroups;  // groups of the tile that exist
+  float lrwd;       // lr * wd of the tile's tensor (lr * wd * wd_scale)
 };
 
 constexpr int64_t kNoTile = 0x7FFFFFFFFFFFFFFFLL;
@@ -295,7 +296,7 @@ __device__ __forceinline__ void process(const LaneIn& in, const TileHeader& t, c
       float vn = __fmaf_rn(h.omb2 * g, g, bv);
       const float p = f4get(in.p[j], i);
       const float upd = mn * rcp_approx(__fmaf_rn(sqrt_approx(vn), h.dsq, h.deps));
-      pn[i] = p + __fmaf_rn(-p, h.lrwd, -upd);
+      pn[i] = p + __fmaf_rn(-p, t.lrwd, -upd);
       if (!FULL) {
         const bool valid = active && (e + i < t.nvalid);
         mn = valid ? mn : 0.f;
@@ -422,7 +423,7 @@ __device__ __forceinline__ void feed_start(const Map& map, Feed& f, int64_t tile
 // and is read from global memory by the lanes.
 template <class Map>
 __device__ __forceinline__ void feed_issue(const Map& map, Feed& f, int64_t tile, uint8_t* st,
-                                           TileHeader& hd, uint64_t* bar) {
+                                           TileHeader& hd, uint64_t* bar, float lrwd) {
   while (tile >= f.next_begin) {
     const int32_t ti = ++f.ti;
     f.d = map.get(ti);
@@ -445,6 +446,7 @@ __device__ __forceinline__ void feed_issue(const Map& map, Feed& f, int64_t tile
   hd.grad = ct.grad + e0;
   hd.nvalid = full ? kTileElems : static_cast<int32_t>(ct.n - e0);
   hd.ngroups = static_cast<int32_t>(ng);
+  hd.lrwd = lrwd * ct.wd_scale;
   if (full) {
     mbar_arrive_expect_tx(bar, kTxBytes);
     bulk_g2s(st + kOffMaster, ct.master + e0, kTileElems * 4, bar);
@@ -509,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         }
         return;
       }
-      feed_issue(map, f, tile, stages + size_t(s) * kStageBytes, S.hdr[s], &S.full_bar[s]);
+      feed_issue(map, f, tile, stages + size_t(s) * kStageBytes, S.hdr[s], &S.full_bar[s], h.lrwd);
     }
     return;
   }

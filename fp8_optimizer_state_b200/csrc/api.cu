@@ -157,6 +157,7 @@ coat::TensorArgs to_args(const coat_tensor_desc& d, int64_t tile_begin) {
   const int64_t tg = coat::step_tile_groups();
   t.tiles = (groups + tg - 1) / tg;
   t.tile_begin = tile_begin;
+  t.wd_scale = 1.0f;
   return t;
 }
 
@@ -345,6 +346,22 @@ coat_status coat_adamw_step_multi(coat_multi_plan_t plan, float lr, float beta1,
   return e == cudaSuccess ? COAT_OK : cuda_fail(e, "coat_adamw_step_multi");
 }
 
+coat_status coat_multi_plan_set_wd_scale(coat_multi_plan_t plan, const float* host_wd_scale,
+                                        cudaStream_t stream) {
+  const char* fn = "coat_multi_plan_set_wd_scale";
+  if (!plan) return fail(COAT_ERR_INVALID_ARG, "%s: plan is NULL", fn);
+  if (!host_wd_scale) return fail(COAT_ERR_INVALID_ARG, "%s: host_wd_scale is NULL", fn);
+  for (int i = 0; i < plan->num; ++i)
+    if (!std::isfinite(host_wd_scale[i]) || host_wd_scale[i] < 0.f)
+      return fail(COAT_ERR_INVALID_ARG, "%s: wd_scale[%d] must be finite and >= 0", fn, i);
+  // one strided copy into the wd_scale field of every device descriptor
+  cudaError_t e = cudaMemcpy2DAsync(&plan->d_descs[0].wd_scale, sizeof(coat::TensorArgs),
+                                    host_wd_scale, sizeof(float), sizeof(float), plan->num,
+                                    cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);   // the host array may go on return
+  return e == cudaSuccess ? COAT_OK : cuda_fail(e, fn);
+}
+
 coat_status coat_multi_plan_destroy(coat_multi_plan_t plan) {
   if (!plan) return COAT_OK;
   cudaError_t e = cudaFree(plan->d_descs);
@@ -482,6 +499,7 @@ extern "C" coat_status coat_adamw_step_multi_noalloc(const coat_tensor_desc* hos
       t.n = d.n;
       t.tiles = ((d.n + 127) / 128 + tg - 1) / tg;
       t.tile_begin = tiles;
+      t.wd_scale = 1.0f;
       tiles += t.tiles;
     }
     if (cudaMemcpyAsync(scratch->descs + c0, buf, sizeof(coat::TensorArgs) * cn,

@@ -20,6 +20,7 @@ struct TensorArgs {
   int64_t n;
   int64_t tiles;       // ceil(ceil(n/128) / groups-per-tile)
   int64_t tile_begin;  // first tile of this tensor in a multi-tensor launch
+  float wd_scale;      // this tensor's weight decay is wd * wd_scale (1 by default)
 };
 
 // Hyperparameters as the kernel uses them (bias corrections and the step size

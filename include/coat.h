@@ -181,6 +181,14 @@ coat_status coat_multi_plan_create(const coat_tensor_desc *host_descs, int num, 
 coat_status coat_adamw_step_multi(coat_multi_plan_t plan, float lr, float beta1, float beta2,
                                   float eps, float wd, int64_t step, cudaStream_t stream);
 coat_status coat_multi_plan_destroy(coat_multi_plan_t plan);
+/* Per-tensor weight decay of a plan: tensor i decays with wd * host_wd_scale[i]
+ * (e.g. 0 for normalisation weights, the usual exclusion from decoupled
+ * weight decay); every scale is 1 when the plan is created.  host_wd_scale
+ * holds one finite value >= 0 per tensor of the plan, read during the call
+ * (the call synchronises `stream` after its copy).  COAT_ERR_INVALID_ARG for a
+ * NULL argument or a negative or non-finite scale. */
+coat_status coat_multi_plan_set_wd_scale(coat_multi_plan_t plan, const float *host_wd_scale,
+                                        cudaStream_t stream);
 /* Number of elements and tensors covered by a plan. */
 coat_status coat_multi_plan_info(coat_multi_plan_t plan, int64_t *total_elements,
                                  int *num_tensors);

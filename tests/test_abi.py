@@ -80,6 +80,13 @@ def test_step_validation():
     assert "aligned" in coat.coat_last_error() or coat.coat_last_error() != ""
 
 
+def test_wd_scale_validation():
+    L = coat.lib()
+    one = (ctypes.c_float * 1)(1.0)
+    assert L.coat_multi_plan_set_wd_scale(None, ctypes.cast(one, ctypes.c_void_p), None) == INVALID
+    assert "plan is NULL" in coat.coat_last_error()
+
+
 def test_selftest_budget_validation():
     L = coat.lib()
     assert L.coat_selftest_wait_timeout(999, None) == INVALID

@@ -81,3 +81,56 @@ def test_multi_vs_oracle(orc):
         check_state_all("m", n, 0, h["mq"], h["ms"], h["mk"], o.mq, o.ms, o.mk)
         check_state_all("v", n, 1, h["vq"], h["vs"], h["vk"], o.vq, o.vs, o.vk)
     plan.destroy()
+
+
+def test_per_tensor_weight_decay():
+    """wd_scale 1 / 0 per tensor gives exactly the bits of single calls with wd
+    and with wd = 0 (e.g. normalisation weights excluded from decay); a scale of
+    0.5 matches the oracle with half the decay."""
+    sizes = [4096 + 3, 700, 128 * 40, 333]
+    scales = [1.0, 0.0, 1.0, 0.0]
+    a = make_sides(sizes, 0, 1)
+    b = make_sides(sizes, 0, 1)
+    plan = plan_of(b, 0, 1)
+    plan.set_wd_scale(scales)
+    for t in (1, 2):
+        for i, (sa, sb) in enumerate(zip(a, b)):
+            g = synth.grad_bits(1, i, t, 0, sizes[i])
+            sb.grad.copy_(torch.from_numpy(g.view(np.int16)))
+            sa.grad.copy_(torch.from_numpy(g.view(np.int16)))
+            coat.coat_adamw_step(sa.master, sa.weight, sa.grad, sa.mq, sa.ms, sa.mk, sa.vq, sa.vs,
+                                 sa.vk, lr=H["lr"], beta1=H["beta1"], beta2=H["beta2"],
+                                 eps=H["eps"], wd=H["wd"] * scales[i], step=t, fmt_m=0, fmt_v=1)
+        coat.coat_adamw_step_multi(plan, lr=H["lr"], beta1=H["beta1"], beta2=H["beta2"],
+                                   eps=H["eps"], wd=H["wd"], step=t)
+    coat.coat_check_device_error()
+    for sa, sb in zip(a, b):
+        ha, hb = sa.host(), sb.host()
+        for key in ("master", "weight", "mq", "ms", "mk", "vq", "vs", "vk"):
+            assert np.array_equal(ha[key], hb[key]), key
+    plan.destroy()
+
+
+def test_half_weight_decay_vs_oracle(orc):
+    n = 70001
+    master = synth.master(1, 9, 0, n)
+    st = gen_state(n, 9, 3, 0, 1, seed=1)
+    side = GpuSide(master, 0, 1).set_state(st)
+    ora = OracleSide(orc, master, 0, 1).set_state(st)
+    plan = plan_of([side], 0, 1)
+    plan.set_wd_scale([0.5])
+    g = synth.grad_bits(1, 9, 3, 0, n)
+    side.grad.copy_(torch.from_numpy(g.view(np.int16)))
+    upd = orc.adamw_step(ora.master, ora.weight, g, ora.mq, ora.ms, ora.mk, ora.vq, ora.vs,
+                         ora.vk, lr=H["lr"], beta1=H["beta1"], beta2=H["beta2"], eps=H["eps"],
+                         wd=H["wd"] * 0.5, step=3, fmt_m=0, fmt_v=1, want_update=True)
+    coat.coat_adamw_step_multi(plan, lr=H["lr"], beta1=H["beta1"], beta2=H["beta2"],
+                               eps=H["eps"], wd=H["wd"], step=3)
+    coat.coat_check_device_error()
+    h = side.host()
+    check_master("master", h["master"], ora.master, upd)
+    check_state_all("m", n, 0, h["mq"], h["ms"], h["mk"], ora.mq, ora.ms, ora.mk)
+    check_state_all("v", n, 1, h["vq"], h["vs"], h["vk"], ora.vq, ora.vs, ora.vk)
+    with pytest.raises(coat.CoatError):
+        plan.set_wd_scale([-1.0])
+    plan.destroy()
