@@ -84,6 +84,13 @@ def lib():
                                      ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_float,
                                      ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_int64,
                                      ctypes.c_int, ctypes.c_int, _P(ctypes.c_double)]
+        L.orc_adamw_step_scaled.restype = ctypes.c_int
+        L.orc_adamw_step_scaled.argtypes = L.orc_adamw_step.argtypes[:-1] + [
+            ctypes.c_double, _P(ctypes.c_double)]
+        L.orc_grad_sumsq.restype = ctypes.c_double
+        L.orc_grad_sumsq.argtypes = [_P(ctypes.c_uint16), ctypes.c_int64, _P(ctypes.c_int)]
+        L.orc_clip_coef.restype = ctypes.c_float
+        L.orc_clip_coef.argtypes = [ctypes.c_double, ctypes.c_float]
         L.orc_adamw_step_unquantized.restype = ctypes.c_int
         L.orc_adamw_step_unquantized.argtypes = [_P(ctypes.c_double)] * 4 + [
             ctypes.c_int64, ctypes.c_double, ctypes.c_double, ctypes.c_double, ctypes.c_double,
@@ -203,7 +210,7 @@ def group_dequantize(q, scale, k, group_rows: int, group_cols: int, fmt: int) ->
 # ----------------------------------------------------------------------------
 
 def adamw_step(master, weight_out, grad_bits, m_q, m_scale, m_k, v_q, v_scale, v_k, *, group=128,
-               lr, beta1, beta2, eps, wd, step, fmt_m, fmt_v, want_update=False):
+               lr, beta1, beta2, eps, wd, step, fmt_m, fmt_v, want_update=False, gscale=1.0):
     """In-place oracle step on numpy arrays (master f32, weight_out u16 or None,
     grad_bits u16, codes u8 padded to whole groups, scale/k f32 per group).
     Returns the per-element |adaptive update| (float64) if want_update."""
@@ -217,14 +224,28 @@ def adamw_step(master, weight_out, grad_bits, m_q, m_scale, m_k, v_q, v_scale, v
     ng = -(-n // group)
     assert m_q.size >= ng * group and v_q.size >= ng * group and m_k.size >= ng
     upd = np.zeros(n, dtype=np.float64) if want_update else None
-    rc = lib().orc_adamw_step(_ptr(master, ctypes.c_float), _ptr(weight_out, ctypes.c_uint16),
-                              _ptr(grad_bits, ctypes.c_uint16), _ptr(m_q, ctypes.c_uint8),
-                              _ptr(m_scale, ctypes.c_float), _ptr(m_k, ctypes.c_float),
-                              _ptr(v_q, ctypes.c_uint8), _ptr(v_scale, ctypes.c_float),
-                              _ptr(v_k, ctypes.c_float), n, group, lr, beta1, beta2, eps, wd,
-                              step, fmt_m, fmt_v, _ptr(upd, ctypes.c_double))
+    rc = lib().orc_adamw_step_scaled(_ptr(master, ctypes.c_float),
+                                     _ptr(weight_out, ctypes.c_uint16),
+                                     _ptr(grad_bits, ctypes.c_uint16), _ptr(m_q, ctypes.c_uint8),
+                                     _ptr(m_scale, ctypes.c_float), _ptr(m_k, ctypes.c_float),
+                                     _ptr(v_q, ctypes.c_uint8), _ptr(v_scale, ctypes.c_float),
+                                     _ptr(v_k, ctypes.c_float), n, group, lr, beta1, beta2, eps,
+                                     wd, step, fmt_m, fmt_v, float(gscale),
+                                     _ptr(upd, ctypes.c_double))
     assert rc == 0
     return upd
+
+
+def grad_sumsq(grad_bits):
+    """(sum of squares in double, any non-finite) of bf16 gradient bits."""
+    g = np.ascontiguousarray(grad_bits, dtype=np.uint16)
+    flag = ctypes.c_int(0)
+    s = lib().orc_grad_sumsq(_ptr(g, ctypes.c_uint16), g.size, ctypes.byref(flag))
+    return s, bool(flag.value)
+
+
+def clip_coef(sumsq: float, max_norm: float) -> float:
+    return lib().orc_clip_coef(sumsq, max_norm)
 
 
 def adamw_step_unquantized(p, m, v, g, *, lr, beta1, beta2, eps, wd, step):

@@ -326,11 +326,30 @@ int orc_group_dequantize(const uint8_t *q, int64_t ldq, const float *scale,
  * the update before any cancellation between the old moment and the new
  * gradient.  Tests use it to size the master-weight tolerance (it is not part
  * of the method's result).  Returns 0, or -1 on bad arguments. */
+int orc_adamw_step_scaled(float *master, uint16_t *weight_out, const uint16_t *grad,
+                          uint8_t *m_q, float *m_scale, float *m_k, uint8_t *v_q,
+                          float *v_scale, float *v_k, int64_t n, int group, float lr,
+                          float beta1, float beta2, float eps, float wd, int64_t step,
+                          int fmt_m, int fmt_v, double gscale, double *upd_out);
+
 int orc_adamw_step(float *master, uint16_t *weight_out, const uint16_t *grad,
                    uint8_t *m_q, float *m_scale, float *m_k, uint8_t *v_q,
                    float *v_scale, float *v_k, int64_t n, int group, float lr,
                    float beta1, float beta2, float eps, float wd, int64_t step,
                    int fmt_m, int fmt_v, double *upd_out)
+{
+    return orc_adamw_step_scaled(master, weight_out, grad, m_q, m_scale, m_k, v_q, v_scale, v_k,
+                                 n, group, lr, beta1, beta2, eps, wd, step, fmt_m, fmt_v, 1.0,
+                                 upd_out);
+}
+
+/* The step on the clipped gradient gscale * g (gradient-norm clipping, see
+ * orc_clip_coef; gscale = 1 is the plain step). */
+int orc_adamw_step_scaled(float *master, uint16_t *weight_out, const uint16_t *grad,
+                          uint8_t *m_q, float *m_scale, float *m_k, uint8_t *v_q,
+                          float *v_scale, float *v_k, int64_t n, int group, float lr,
+                          float beta1, float beta2, float eps, float wd, int64_t step,
+                          int fmt_m, int fmt_v, double gscale, double *upd_out)
 {
     if (n < 0 || group < 1 || step < 1)
         return -1;
@@ -352,7 +371,7 @@ int orc_adamw_step(float *master, uint16_t *weight_out, const uint16_t *grad,
             int64_t i = base + j;
             double m = orc_dequant_value(fmt_m, m_q[i], m_scale[g], m_k[g]);
             double v = orc_dequant_value(fmt_v, v_q[i], v_scale[g], v_k[g]);
-            double gi = orc_bf16_to_double(grad[i]);
+            double gi = gscale * orc_bf16_to_double(grad[i]);
             double m1 = b1 * m + (1.0 - b1) * gi;
             double v1 = b2 * v + (1.0 - b2) * gi * gi;
             double p = (double)master[i];
@@ -383,6 +402,35 @@ int orc_adamw_step(float *master, uint16_t *weight_out, const uint16_t *grad,
 /* The same step with the moments kept unquantised in double: the plain
  * AdamW recurrence, used to pin the optimizer arithmetic against closed
  * forms and torch.optim.AdamW. */
+/* ------------------------------------------------------------------ */
+/* Global gradient-norm clipping and the non-finite check before the   */
+/* step (not on the pages; the usual training-loop pre-step, as        */
+/* torch.nn.utils.clip_grad_norm_ defines it).                          */
+/* ------------------------------------------------------------------ */
+
+/* Sum of squares of n bf16 gradient values, in double, in element order;
+ * *nonfinite is set to 1 if any value is infinite or NaN (left as is
+ * otherwise, so that calls over several tensors accumulate). */
+double orc_grad_sumsq(const uint16_t *grad, int64_t n, int *nonfinite)
+{
+    double s = 0.0;
+    for (int64_t i = 0; i < n; i++) {
+        double g = orc_bf16_to_double(grad[i]);
+        if (!isfinite(g))
+            *nonfinite = 1;
+        s += g * g;
+    }
+    return s;
+}
+
+/* Clip coefficient for a total sum of squares: min(1, max_norm / (norm +
+ * 1e-6)) with norm = sqrt(sumsq), rounded to FP32 (max_norm = +inf: 1). */
+float orc_clip_coef(double sumsq, float max_norm)
+{
+    double c = (double)max_norm / (sqrt(sumsq) + 1e-6);
+    return (float)(c < 1.0 ? c : 1.0);
+}
+
 int orc_adamw_step_unquantized(double *p, double *m, double *v, const double *g,
                                int64_t n, double lr, double beta1, double beta2,
                                double eps, double wd, int64_t step)

@@ -157,3 +157,56 @@ def test_quantized_close_to_unquantized(orc):
     # FP8 moment error (~6% per element at most) moves p by a fraction of lr/bc1 per step
     assert np.max(np.abs(master - p)) < 3 * 0.2 * lr / (1 - b1)
     assert np.median(np.abs(master - p)) < 0.05 * lr / (1 - b1)
+
+
+# ---------------------------------------------------------------------------
+# Gradient-norm clipping and the non-finite check before the step
+# ---------------------------------------------------------------------------
+def _bf16(vals):
+    return torch.tensor(vals, dtype=torch.float32).to(torch.bfloat16).view(torch.int16) \
+        .numpy().view(np.uint16)
+
+
+def test_grad_sumsq_closed_forms(orc):
+    assert orc.grad_sumsq(_bf16([3.0, 4.0])) == (25.0, False)          # a 3-4-5 triangle
+    assert orc.grad_sumsq(_bf16([0.5] * 1000)) == (250.0, False)
+    assert orc.grad_sumsq(_bf16([-2.0 ** -10] * 64)) == (64 * 2.0 ** -20, False)
+    assert orc.grad_sumsq(np.zeros(0, np.uint16)) == (0.0, False)
+    for bad in (float("inf"), float("-inf"), float("nan")):
+        assert orc.grad_sumsq(_bf16([1.0, bad, 2.0]))[1] is True
+
+
+def test_clip_coef_closed_forms(orc):
+    # norm 5: max_norm / (norm + 1e-6), rounded to FP32, when below 1
+    assert orc.clip_coef(25.0, 1.0) == np.float32(1.0 / (5.0 + 1e-6))
+    assert orc.clip_coef(25.0, 2.5) == np.float32(2.5 / (5.0 + 1e-6))
+    assert orc.clip_coef(25.0, 10.0) == 1.0          # already below the limit
+    assert orc.clip_coef(0.0, 1.0) == 1.0            # zero gradient
+    assert orc.clip_coef(25.0, float("inf")) == 1.0  # no limit
+
+
+def test_scaled_step_is_the_step_on_the_scaled_gradient(orc):
+    """gscale = 0.5 gives exactly the state of the plain step on bf16 gradients
+    halved exactly (every value here is far from the bf16 subnormal range)."""
+    n = 128 * 5 + 17
+    rng = np.random.default_rng(3)
+    g = rng.normal(0, 1e-3, n).astype(np.float32)
+    g[np.abs(g) < 1e-6] = 1e-6
+    gb = _bf16(g)
+    gh = _bf16(torch.from_numpy(gb.view(np.int16)).view(torch.bfloat16).float().numpy() * 0.5)
+    m0 = np.random.default_rng(4).normal(0, 0.02, n).astype(np.float32)
+    res = []
+    for bits, gs in ((gb, 0.5), (gh, 1.0)):
+        master = m0.copy()
+        ng = -(-n // 128)
+        st = [np.zeros(ng * 128, np.uint8), np.ones(ng, np.float32), np.ones(ng, np.float32),
+              np.zeros(ng * 128, np.uint8), np.ones(ng, np.float32), np.ones(ng, np.float32)]
+        for t in (1, 2):
+            orc.adamw_step(master, None, bits, st[0], st[1], st[2], st[3], st[4], st[5], lr=1e-3,
+                           beta1=0.9, beta2=0.95, eps=1e-8, wd=0.1, step=t, fmt_m=E4M3,
+                           fmt_v=E4M3, gscale=gs)
+        res.append((master, st))
+    (ma, sa), (mb, sb) = res
+    assert np.array_equal(ma, mb)
+    for x, y in zip(sa, sb):
+        assert np.array_equal(x, y)
