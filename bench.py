@@ -41,7 +41,7 @@ KERNEL_SOURCES = ["fp8_optimizer_state_b200/csrc/adamw_fp8.cu",
 # DRAM bytes (read + write) per parameter of the step kernel from an ncu
 # capture on a 268,435,456-parameter tensor (profiles/), scaled to a launch by
 # its parameter count; valid only for the kernel sources with this hash.
-TRAFFIC = {"sources_sha256": "0ffe9dec43489a26", "bytes_per_param": 16.049}
+TRAFFIC = {"sources_sha256": "740c50438e52b1f9", "bytes_per_param": 16.053}
 
 
 def kernel_hash():
@@ -290,11 +290,21 @@ def run_ours(args, cfg, ws, rank, local):
 
     stream = torch.cuda.current_stream()
     step_no = [0]
+    clip_buf = coat.new_grad_clip(dev) if args.clip is not None else None
 
-    def one_step():
+    def one_step(mid=None):
+        # with --clip: the gradient-norm pass, then the step on coef * g
         step_no[0] += 1
-        coat.coat_adamw_step_multi(plan, lr=H["lr"], beta1=H["beta1"], beta2=H["beta2"],
-                                   eps=H["eps"], wd=H["wd"], step=step_no[0])
+        if clip_buf is not None:
+            plan.grad_norm(args.clip, clip_buf)
+            if mid is not None:
+                mid.record(stream)
+            coat.coat_adamw_step_multi_clipped(plan, clip_buf, lr=H["lr"], beta1=H["beta1"],
+                                               beta2=H["beta2"], eps=H["eps"], wd=H["wd"],
+                                               step=step_no[0])
+        else:
+            coat.coat_adamw_step_multi(plan, lr=H["lr"], beta1=H["beta1"], beta2=H["beta2"],
+                                       eps=H["eps"], wd=H["wd"], step=step_no[0])
 
     for _ in range(args.warmup):
         one_step()
@@ -308,7 +318,7 @@ def run_ours(args, cfg, ws, rank, local):
     sampler = ClockSampler(bus)
     sampler.start()
     time.sleep(0.3)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3))
           for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
@@ -318,7 +328,7 @@ def run_ours(args, cfg, ws, rank, local):
     t_start.record(stream)
     for i in range(args.steps):
         ev[i][0].record(stream)
-        one_step()
+        one_step(ev[i][2])
         ev[i][1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
@@ -329,7 +339,12 @@ def run_ours(args, cfg, ws, rank, local):
     coat.coat_check_device_error()
 
     elapsed_ms = t_start.elapsed_time(t_end)
-    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    if clip_buf is not None:
+        # the step kernel alone: from the event after the norm pass
+        launch_ms = [m.elapsed_time(b) for a, b, m in ev]
+        norm_ms = max_over_ranks(statistics.mean([a.elapsed_time(m) for a, b, m in ev]), ws, dev)
+    else:
+        launch_ms = [a.elapsed_time(b) for a, b, m in ev]
     elapsed_ms = max_over_ranks(elapsed_ms, ws, dev)
     kernel_ms = max_over_ranks(statistics.mean(launch_ms), ws, dev)
     n_params = ps.total_elements
@@ -351,12 +366,23 @@ def run_ours(args, cfg, ws, rank, local):
                 "bytes_per_param": round(alg / n_params, 4), "kernel_ms": round(kernel_ms, 4),
                 "frac_of_nominal_8TBs": round(achieved / 8000.0, 4)}
     clocks = sampler.summary(wall0, wall1)
+    clip = None
+    if clip_buf is not None:
+        rec = coat.read_grad_clip(clip_buf)
+        norm_bytes = 2 * n_params
+        norm_gbs = norm_bytes / (norm_ms * 1e-3) / 1e9
+        clip = {"max_norm": args.clip, "norm": float(rec.norm), "coef": float(rec.coef),
+                "found_inf": int(rec.found_inf), "norm_kernel_ms": round(norm_ms, 4),
+                "norm_algorithmic_bytes": norm_bytes, "norm_achieved_GBs": round(norm_gbs, 1),
+                "norm_frac": round(norm_gbs / peak, 4),
+                "how": "per step: gradient-norm pass (reads every bf16 gradient once) then the "
+                       "step on coef * g; roofline above is the step kernel alone"}
 
     # end to end through the public API with host buffers: per step, H2D of the
     # bf16 gradients from pinned memory, the step (per tensor, overlapped with the
     # copies on separate streams), D2H of the bf16 weight copy
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and clip_buf is None:
         e2e = run_e2e(args, cfg, ps, ws, dev, H, coat)
 
     plan.destroy()
@@ -400,8 +426,10 @@ def run_ours(args, cfg, ws, rank, local):
                        "parallelism": "replicas%d (independent parameter groups, no collective)" % ws
                        if ws > 1 else "single GPU"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": args.steps, "clocks": clocks,
+            "gpu_launches": args.steps * (2 if clip_buf is not None else 1), "clocks": clocks,
         }
+        if clip is not None:
+            result["clip"] = clip
         if vs_flat is not None:
             result["vs_flat_tensor"] = vs_flat
     if ws > 1:
@@ -695,6 +723,8 @@ def main(argv=None):
                     help="override the workload's v format (2: E5M2 expanded to its own span)")
     ap.add_argument("--compare-flat", action="store_true",
                     help="also time one flat tensor of the same parameter count")
+    ap.add_argument("--clip", type=float, default=None, metavar="MAX_NORM",
+                    help="time the clipped step: gradient-norm pass + step on coef * g")
     ap.add_argument("--cpu-sample", type=int, default=16 << 20)
     ap.add_argument("--ref-sample", type=int, default=2 << 20)
     args = ap.parse_args(argv)

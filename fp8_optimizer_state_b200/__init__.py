@@ -42,6 +42,8 @@ EXPORTS = [
     ("coat_adamw_step_multi_noalloc", _i32, [_vp, _i32, _i32, _f32, _f32, _f32, _f32, _f32, _i64,
                                              _i32, _i32, _vp]),
     ("coat_selftest_wait_timeout", _i32, [_i64, _vp]),
+    ("coat_multi_plan_grad_norm", _i32, [_vp, _f32, _vp, _vp]),
+    ("coat_adamw_step_multi_clipped", _i32, [_vp, _f32, _f32, _f32, _f32, _f32, _i64, _vp, _vp]),
 ]
 NOALLOC_MAX_TENSORS = 1024
 
@@ -50,6 +52,33 @@ class CoatError(RuntimeError):
     def __init__(self, status, message):
         super().__init__("%s: %s" % (STATUS.get(status, status), message))
         self.status = status
+
+
+class GradClip(ctypes.Structure):
+    """coat_grad_clip (24 bytes; lives in device memory)"""
+    _fields_ = [("sumsq", ctypes.c_double), ("norm", _f32), ("coef", _f32),
+                ("found_inf", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+def new_grad_clip(device=None):
+    """A zeroed device buffer holding one coat_grad_clip (a uint8 CUDA tensor)."""
+    import torch
+    return torch.zeros(ctypes.sizeof(GradClip), dtype=torch.uint8,
+                       device=device if device is not None else "cuda")
+
+
+def read_grad_clip(buf):
+    """Copy a coat_grad_clip device buffer to the host (synchronises)."""
+    raw = bytes(buf.cpu().numpy().tobytes())
+    return GradClip.from_buffer_copy(raw)
+
+
+def write_grad_clip(buf, coef, found_inf=0, sumsq=0.0, norm=0.0):
+    """Fill a coat_grad_clip device buffer from host values."""
+    import torch
+    rec = GradClip(float(sumsq), float(norm), float(coef), int(found_inf), 0)
+    host = torch.frombuffer(bytearray(bytes(rec)), dtype=torch.uint8)
+    buf.copy_(host)
 
 
 class TensorDesc(ctypes.Structure):
@@ -175,6 +204,10 @@ class coat_multi_plan:
         _check(lib().coat_multi_plan_set_wd_scale(self.handle, ctypes.cast(arr, ctypes.c_void_p),
                                                   _s(stream)))
 
+    def grad_norm(self, max_norm, clip_buf, stream=None):
+        """coat_multi_plan_grad_norm into clip_buf (see new_grad_clip)."""
+        coat_multi_plan_grad_norm(self, max_norm, clip_buf, stream)
+
     def destroy(self):
         if self.handle:
             _check(lib().coat_multi_plan_destroy(self.handle))
@@ -198,6 +231,20 @@ def coat_multi_plan_create(descs, fmt_m=COAT_E4M3, fmt_v=COAT_E4M3, group=GROUP,
 
 def coat_adamw_step_multi(plan, *, lr, beta1, beta2, eps, wd, step, stream=None):
     _check(lib().coat_adamw_step_multi(plan.handle, lr, beta1, beta2, eps, wd, step, _s(stream)))
+
+
+def coat_multi_plan_grad_norm(plan, max_norm, clip_buf, stream=None):
+    if clip_buf.numel() * clip_buf.element_size() < ctypes.sizeof(GradClip):
+        raise ValueError("clip_buf must hold %d bytes" % ctypes.sizeof(GradClip))
+    _check(lib().coat_multi_plan_grad_norm(plan.handle, max_norm, _p(clip_buf), _s(stream)))
+
+
+def coat_adamw_step_multi_clipped(plan, clip_buf, *, lr, beta1, beta2, eps, wd, step,
+                                  stream=None):
+    if clip_buf.numel() * clip_buf.element_size() < ctypes.sizeof(GradClip):
+        raise ValueError("clip_buf must hold %d bytes" % ctypes.sizeof(GradClip))
+    _check(lib().coat_adamw_step_multi_clipped(plan.handle, lr, beta1, beta2, eps, wd, step,
+                                               _p(clip_buf), _s(stream)))
 
 
 def coat_multi_plan_destroy(plan):

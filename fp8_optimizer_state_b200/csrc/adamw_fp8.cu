@@ -236,9 +236,11 @@ __device__ __forceinline__ double exp2_table(double t, const double* exp2_16) {
 // and k depends on it through ln(max/min).  The kernel keeps the two smallest
 // candidates (their positions packed into the low 8 bits of the comparison
 // keys, at a cost of 2^-16 relative in the ordering) and recomputes them in
-// double precision: dequantisation, then m' = beta1 m + (1 - beta1) g.
+// double precision: dequantisation, then m' = beta1 m + (1 - beta1) gs g, gs
+// the gradient-clipping coefficient (1 without clipping).
 __device__ __forceinline__ float recompute_m_double(const LaneIn& in, int idx, double invk,
-                                                    const StepHyper& h, const double* tabd_m,
+                                                    const StepHyper& h, float gs,
+                                                    const double* tabd_m,
                                                     const double* exp2_16) {
   const int j = idx >> 2, i = idx & 3;
   const uint32_t mw = j == 0 ? in.mq[0] : j == 1 ? in.mq[1] : j == 2 ? in.mq[2] : in.mq[3];
@@ -249,7 +251,7 @@ __device__ __forceinline__ float recompute_m_double(const LaneIn& in, int idx, d
   double x = exp2_table(tabd_m[c] * invk, exp2_16) * static_cast<double>(in.ms);
   if (c & 0x80u) x = -x;
   const double b1 = static_cast<double>(h.beta1);
-  const double m1 = fma(b1, x, (1.0 - b1) * static_cast<double>(g));
+  const double m1 = fma(b1, x, (1.0 - b1) * (static_cast<double>(gs) * static_cast<double>(g)));
   return __double2float_rn(fabs(m1));
 }
 
@@ -261,11 +263,13 @@ __device__ __forceinline__ uint32_t min_key(float x, int idx) {
 }
 
 // The per-lane body: everything after the loads.  FULL: every element of the
-// tile is valid (no bounds logic).
+// tile is valid (no bounds logic).  The gradient enters scaled by gs (the
+// clipping coefficient, 1 without clipping), folded into the moment weights:
+// omb1 = (1 - beta1) gs and omb2 = (1 - beta2) gs^2.
 template <int FM, int FV, bool FULL>
 __device__ __forceinline__ void process(const LaneIn& in, const TileHeader& t, const int (&off)[4],
                                         int lg, bool active, int slot, int l, const StepHyper& h,
-                                        const Smem& S) {
+                                        float omb1, float omb2, float gs, const Smem& S) {
   // dequantisation constants of this group (stored k and root scale)
   const float invk_m = rcp_approx(in.mk), sb_m = in.ms * h.beta1;
   const float invk_v = rcp_approx(in.vk), sb_v = in.vs * h.beta2;
@@ -292,8 +296,8 @@ __device__ __forceinline__ void process(const LaneIn& in, const TileHeader& t, c
       float bm = ex2_approx(S.tab_m[cm] * invk_m) * sb_m;
       bm = __uint_as_float(__float_as_uint(bm) ^ ((in.mq[j] << (24 - 8 * i)) & 0x80000000u));
       const float bv = ex2_approx(S.tab_v[cv] * invk_v) * sb_v;
-      float mn = __fmaf_rn(h.omb1, g, bm);
-      float vn = __fmaf_rn(h.omb2 * g, g, bv);
+      float mn = __fmaf_rn(omb1, g, bm);
+      float vn = __fmaf_rn(omb2 * g, g, bv);
       const float p = f4get(in.p[j], i);
       const float upd = mn * rcp_approx(__fmaf_rn(sqrt_approx(vn), h.dsq, h.deps));
       pn[i] = p + __fmaf_rn(-p, t.lrwd, -upd);
@@ -357,13 +361,14 @@ __device__ __forceinline__ void process(const LaneIn& in, const TileHeader& t, c
   // broadcast to its 8-lane group.
   const bool any_m = minm1 < 0xFFFFFF00u;
   const bool tie = minm2 < 0xFFFFFF00u && (minm2 >> 8) - (minm1 >> 8) < (1u << 9);
-  float mum = recompute_m_double(in, static_cast<int>(minm1 & 15u), invk_md, h, S.tabd_m,
+  float mum = recompute_m_double(in, static_cast<int>(minm1 & 15u), invk_md, h, gs, S.tabd_m,
                                  S.exp2_16);
   mum = __shfl_sync(0xFFFFFFFFu, mum, (slot << 3) | static_cast<int>((minm1 >> 5) & 7u));
   if (__any_sync(0xFFFFFFFFu, tie)) {
     float m2 = __int_as_float(0x7F800000);
     if (tie && static_cast<int>((minm2 >> 5) & 7u) == l)
-      m2 = recompute_m_double(in, static_cast<int>(minm2 & 15u), invk_md, h, S.tabd_m, S.exp2_16);
+      m2 = recompute_m_double(in, static_cast<int>(minm2 & 15u), invk_md, h, gs, S.tabd_m,
+                              S.exp2_16);
 #pragma unroll
     for (int off = 1; off < 8; off <<= 1) m2 = fminf(m2, __shfl_xor_sync(0xFFFFFFFFu, m2, off));
     mum = fminf(mum, m2);
@@ -464,7 +469,14 @@ __device__ __forceinline__ void feed_issue(const Map& map, Feed& f, int64_t tile
 
 template <int FM, int FV, class Map>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
-    adamw_fp8_kernel(const Map map, const StepHyper h, unsigned* err) {
+    adamw_fp8_kernel(const Map map, const StepHyper h, const ClipRecord* clip, unsigned* err) {
+  // Gradient clipping: a record with found_inf set skips the step (nothing is
+  // read or written); otherwise the gradient is scaled by its coefficient.
+  float gs = 1.f;
+  if (clip != nullptr) {
+    if (clip->found_inf) return;
+    gs = clip->coef;
+  }
   extern __shared__ __align__(128) uint8_t smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>(smem_raw);
   uint8_t* stages = smem_raw + kSmemHead;
@@ -519,6 +531,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   // ---------------- consumers ----------------
   const int slot = lane >> 3, l = lane & 7;
   const int lg = warp * kGroupsPerWarp + slot;  // group within the tile
+  const float omb1 = h.omb1 * gs, omb2 = h.omb2 * gs * gs;
   // the lane's elements: 4 chunks of 4, chunk j at 32 chunk_of(j, slot) + 4 l
   // within its group
   int off[4];
@@ -544,15 +557,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.empty_bar[s]);
     if (full)
-      process<FM, FV, true>(in, t, off, lg, true, slot, l, h, S);
+      process<FM, FV, true>(in, t, off, lg, true, slot, l, h, omb1, omb2, gs, S);
     else
-      process<FM, FV, false>(in, t, off, lg, active, slot, l, h, S);
+      process<FM, FV, false>(in, t, off, lg, active, slot, l, h, omb1, omb2, gs, S);
   }
 }
 
 template <int FM, int FV, class Map>
-cudaError_t launch_step(const Map& map, int64_t ntiles, const StepHyper& h, unsigned* err,
-                        cudaStream_t stream) {
+cudaError_t launch_step(const Map& map, int64_t ntiles, const StepHyper& h,
+                        const ClipRecord* clip, unsigned* err, cudaStream_t stream) {
   static bool configured[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -567,24 +580,26 @@ cudaError_t launch_step(const Map& map, int64_t ntiles, const StepHyper& h, unsi
   const int64_t want = int64_t(sm_count(dev)) * kCtasPerSm;
   const int64_t grid = ntiles < want ? ntiles : want;
   if (grid <= 0) return cudaSuccess;
-  kern<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(map, h, err);
+  kern<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(map, h, clip, err);
   return cudaGetLastError();
 }
 
 template <class Map>
 cudaError_t dispatch(int fm, int fv, const Map& map, int64_t ntiles, const StepHyper& h,
-                     unsigned* err, cudaStream_t stream) {
+                     const ClipRecord* clip, unsigned* err, cudaStream_t stream) {
   switch (fm * 3 + fv) {
-    case kE4M3 * 3 + kE4M3: return launch_step<kE4M3, kE4M3>(map, ntiles, h, err, stream);
-    case kE4M3 * 3 + kE5M2: return launch_step<kE4M3, kE5M2>(map, ntiles, h, err, stream);
-    case kE4M3 * 3 + kE5M2Full: return launch_step<kE4M3, kE5M2Full>(map, ntiles, h, err, stream);
-    case kE5M2 * 3 + kE4M3: return launch_step<kE5M2, kE4M3>(map, ntiles, h, err, stream);
-    case kE5M2 * 3 + kE5M2: return launch_step<kE5M2, kE5M2>(map, ntiles, h, err, stream);
-    case kE5M2 * 3 + kE5M2Full: return launch_step<kE5M2, kE5M2Full>(map, ntiles, h, err, stream);
-    case kE5M2Full * 3 + kE4M3: return launch_step<kE5M2Full, kE4M3>(map, ntiles, h, err, stream);
-    case kE5M2Full * 3 + kE5M2: return launch_step<kE5M2Full, kE5M2>(map, ntiles, h, err, stream);
-    case kE5M2Full * 3 + kE5M2Full:
-      return launch_step<kE5M2Full, kE5M2Full>(map, ntiles, h, err, stream);
+#define COAT_STEP_CASE(A, B) \
+  case A * 3 + B: return launch_step<A, B>(map, ntiles, h, clip, err, stream);
+    COAT_STEP_CASE(kE4M3, kE4M3)
+    COAT_STEP_CASE(kE4M3, kE5M2)
+    COAT_STEP_CASE(kE4M3, kE5M2Full)
+    COAT_STEP_CASE(kE5M2, kE4M3)
+    COAT_STEP_CASE(kE5M2, kE5M2)
+    COAT_STEP_CASE(kE5M2, kE5M2Full)
+    COAT_STEP_CASE(kE5M2Full, kE4M3)
+    COAT_STEP_CASE(kE5M2Full, kE5M2)
+    COAT_STEP_CASE(kE5M2Full, kE5M2Full)
+#undef COAT_STEP_CASE
     default: return cudaErrorInvalidValue;
   }
 }
@@ -596,13 +611,170 @@ int64_t step_tile_groups() { return kTileGroups; }
 cudaError_t launch_adamw_single(const TensorArgs& t, int fm, int fv, const StepHyper& h,
                                 unsigned* err, cudaStream_t stream) {
   SingleTensor map{t};
-  return dispatch(fm, fv, map, t.tiles, h, err, stream);
+  return dispatch(fm, fv, map, t.tiles, h, nullptr, err, stream);
 }
 
 cudaError_t launch_adamw_multi(const TensorArgs* d_descs, int num, int64_t total_tiles, int fm,
-                               int fv, const StepHyper& h, unsigned* err, cudaStream_t stream) {
+                               int fv, const StepHyper& h, const ClipRecord* clip, unsigned* err,
+                               cudaStream_t stream) {
   MultiTensor map{d_descs, num, total_tiles};
-  return dispatch(fm, fv, map, total_tiles, h, err, stream);
+  return dispatch(fm, fv, map, total_tiles, h, clip, err, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Gradient-norm pass before a clipped step (global-norm clipping as
+// torch.nn.utils.clip_grad_norm_ defines it, with the non-finite check of a
+// loss-scaled training loop): sum of g^2 over every gradient of the plan.
+//
+// HBM-bound (2 bytes per element read, nothing else): kNormCtasPerSm CTAs per
+// SM, each over a contiguous range of the step's tiles, so that every CTA
+// streams whole runs of each tensor's gradient with 16-byte loads.  A thread
+// squares the 8 bf16 values of a load in FP32 -- each square is exact there,
+// the 8-term sum rounds a few times at 2^-24 relative -- and adds the sum to a
+// double accumulator; if that FP32 sum overflowed (an element of magnitude
+// 2^64 or more) or met an Inf/NaN, the 8 values are redone in double, where no
+// sum of bf16 squares can overflow, so the total is non-finite exactly when an
+// element is.  CTA sums go to per-CTA slots; the last CTA to finish (ticket
+// counter) adds the slots in index order, so the result depends only on the
+// grid, which is fixed per device.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kNormThreads = 256;
+constexpr int kNormCtasPerSm = 4;
+constexpr int kNormUnroll = 4;
+
+__device__ __forceinline__ double sumsq8(const uint4 w) {
+  const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float lo = __uint_as_float(a[k] << 16), hi = __uint_as_float(a[k] & 0xFFFF0000u);
+    s0 = __fmaf_rn(lo, lo, s0);
+    s1 = __fmaf_rn(hi, hi, s1);
+  }
+  const float s = s0 + s1;
+  if (s <= 3.40282347e38f) return static_cast<double>(s);
+  double d = 0.0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const double lo = __uint_as_float(a[k] << 16), hi = __uint_as_float(a[k] & 0xFFFF0000u);
+    d = fma(lo, lo, d);
+    d = fma(hi, hi, d);
+  }
+  return d;
+}
+
+// Sum of g^2 over cnt elements from g (16-byte aligned) by the CTA's threads.
+__device__ __forceinline__ double sumsq_run(const uint16_t* g, int64_t cnt) {
+  const uint4* v = reinterpret_cast<const uint4*>(g);
+  const int64_t nv = cnt >> 3;
+  constexpr int T = kNormThreads;
+  double acc = 0.0;
+  int64_t i = threadIdx.x;
+  for (; i + (kNormUnroll - 1) * T < nv; i += kNormUnroll * T) {
+    uint4 w[kNormUnroll];
+#pragma unroll
+    for (int u = 0; u < kNormUnroll; ++u) w[u] = __ldcs(v + i + u * T);
+#pragma unroll
+    for (int u = 0; u < kNormUnroll; ++u) acc += sumsq8(w[u]);
+  }
+  for (; i < nv; i += T) acc += sumsq8(__ldcs(v + i));
+  const int64_t rem = cnt & 7;
+  if (threadIdx.x < rem) {
+    const double x = __uint_as_float(static_cast<uint32_t>(g[nv * 8 + threadIdx.x]) << 16);
+    acc = fma(x, x, acc);
+  }
+  return acc;
+}
+
+// Sum over the CTA in a fixed order; the result is valid in thread 0.
+__device__ __forceinline__ double cta_sum(double x, double* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o);
+  const int warp = threadIdx.x >> 5;
+  __syncthreads();  // red may still be read from an earlier call
+  if ((threadIdx.x & 31) == 0) red[warp] = x;
+  __syncthreads();
+  double t = 0.0;
+  if (threadIdx.x == 0)
+    for (int w = 0; w < kNormThreads / 32; ++w) t += red[w];
+  return t;
+}
+
+__global__ void __launch_bounds__(kNormThreads, kNormCtasPerSm)
+    grad_sumsq_kernel(const MultiTensor map, double* partials, unsigned* ticket, float max_norm,
+                      ClipRecord* out) {
+  __shared__ double red[kNormThreads / 32];
+  __shared__ bool last;
+  const int64_t ntiles = map.tiles();
+  const int64_t t0 = int64_t(blockIdx.x) * ntiles / gridDim.x;
+  const int64_t t1 = int64_t(blockIdx.x + 1) * ntiles / gridDim.x;
+  double acc = 0.0;
+  if (t0 < t1) {
+    // walk the tensors that own tiles [t0, t1): each contributes one run of
+    // its gradient (tile boundaries are 7680 elements apart, so every run
+    // starts 16-byte aligned)
+    int32_t ti = map.find(t0);
+    int64_t tile = t0;
+    while (tile < t1 && ti < map.num) {
+      const TensorArgs& d = map.descs[ti];
+      const int64_t tb = d.tile_begin, te = tb + d.tiles;
+      if (tile < te) {
+        const int64_t tend = te < t1 ? te : t1;
+        const int64_t ea = (tile - tb) * kTileElems;
+        const int64_t eb_tiles = (tend - tb) * kTileElems;
+        const int64_t eb = eb_tiles < d.n ? eb_tiles : d.n;
+        acc += sumsq_run(d.grad + ea, eb - ea);
+        tile = tend;
+      }
+      ++ti;
+    }
+  }
+  const double cta = cta_sum(acc, red);
+  if (threadIdx.x == 0) {
+    partials[blockIdx.x] = cta;
+    __threadfence();
+    last = atomicAdd(ticket, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!last) return;
+  // the last CTA: every other CTA's slot is written and visible
+  __threadfence();
+  double a = 0.0;
+  for (int i = threadIdx.x; i < static_cast<int>(gridDim.x); i += kNormThreads)
+    a += __ldcg(partials + i);
+  const double total = cta_sum(a, red);
+  if (threadIdx.x == 0) {
+    const double c = static_cast<double>(max_norm) / (sqrt(total) + 1e-6);
+    ClipRecord r;
+    r.sumsq = total;
+    r.norm = static_cast<float>(sqrt(total));
+    r.coef = static_cast<float>(c < 1.0 ? c : 1.0);
+    r.found_inf = isfinite(total) ? 0 : 1;
+    r.reserved = 0;
+    *out = r;
+    *ticket = 0u;  // ready for the next launch on this plan
+  }
+}
+
+}  // namespace
+
+int grad_sumsq_slots(int dev) { return sm_count(dev) * kNormCtasPerSm; }
+
+cudaError_t launch_grad_sumsq(const TensorArgs* d_descs, int num, int64_t total_tiles,
+                              double* partials, unsigned* ticket, float max_norm, ClipRecord* out,
+                              cudaStream_t stream) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const int64_t slots = grad_sumsq_slots(dev);
+  int64_t grid = total_tiles < slots ? total_tiles : slots;
+  if (grid < 1) grid = 1;  // an empty plan still writes its record
+  MultiTensor map{d_descs, num, total_tiles};
+  grad_sumsq_kernel<<<static_cast<unsigned>(grid), kNormThreads, 0, stream>>>(map, partials, ticket,
+                                                                             max_norm, out);
+  return cudaGetLastError();
 }
 
 namespace {

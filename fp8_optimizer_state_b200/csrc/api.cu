@@ -2,6 +2,7 @@
 // any CUDA call, so a bad call launches nothing and touches nothing), error
 // reporting, multi-tensor plans, and kernel launches on the caller's stream.
 #include <cmath>
+#include <cstddef>
 #include <limits>
 #include <cstdarg>
 #include <cstdio>
@@ -274,6 +275,8 @@ coat_status coat_adamw_step(float* master, uint16_t* weight_bf16_out, const uint
 
 struct coat_multi_plan {
   coat::TensorArgs* d_descs = nullptr;  // device copy of the descriptors (tile_begin ascending)
+  double* d_partials = nullptr;         // gradient-norm pass: one slot per CTA
+  unsigned* d_ticket = nullptr;         // gradient-norm pass: CTAs finished (0 between calls)
   int64_t total_tiles = 0;
   int64_t total_elements = 0;
   int num = 0;
@@ -305,10 +308,15 @@ coat_status coat_multi_plan_create(const coat_tensor_desc* host_descs, int num, 
 
   coat_multi_plan* p = new (std::nothrow) coat_multi_plan;
   if (!p) return fail(COAT_ERR_NOMEM, "%s: host allocation failed", fn);
+  // one allocation: descriptor table | gradient-norm slots | ticket
   const size_t desc_bytes = sizeof(coat::TensorArgs) * num;
+  const size_t off_partials = (desc_bytes + 255) / 256 * 256;
   void* mem = nullptr;
   cudaError_t e = cudaGetDevice(&p->device);
-  if (e == cudaSuccess) e = cudaMalloc(&mem, desc_bytes);
+  const size_t slot_bytes =
+      e == cudaSuccess ? sizeof(double) * static_cast<size_t>(coat::grad_sumsq_slots(p->device)) : 0;
+  const size_t off_ticket = off_partials + (slot_bytes + 255) / 256 * 256;
+  if (e == cudaSuccess) e = cudaMalloc(&mem, off_ticket + 256);
   if (e != cudaSuccess) {
     delete p;
     cudaGetLastError();
@@ -316,7 +324,10 @@ coat_status coat_multi_plan_create(const coat_tensor_desc* host_descs, int num, 
                                           : cuda_fail(e, fn);
   }
   p->d_descs = static_cast<coat::TensorArgs*>(mem);
+  p->d_partials = reinterpret_cast<double*>(static_cast<char*>(mem) + off_partials);
+  p->d_ticket = reinterpret_cast<unsigned*>(static_cast<char*>(mem) + off_ticket);
   e = cudaMemcpyAsync(p->d_descs, descs.data(), desc_bytes, cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(p->d_ticket, 0, sizeof(unsigned), stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(stream);  // the host vector dies on return
   if (e != cudaSuccess) {
     cudaFree(mem);
@@ -342,8 +353,48 @@ coat_status coat_adamw_step_multi(coat_multi_plan_t plan, float lr, float beta1,
   cudaError_t e = coat::device_error_ptr(&err);
   if (e != cudaSuccess) return cuda_fail(e, "coat_adamw_step_multi");
   e = coat::launch_adamw_multi(plan->d_descs, plan->num, plan->total_tiles, plan->fmt_m,
-                               plan->fmt_v, make_hyper(lr, beta1, beta2, eps, wd, step), err, stream);
+                               plan->fmt_v, make_hyper(lr, beta1, beta2, eps, wd, step), nullptr,
+                               err, stream);
   return e == cudaSuccess ? COAT_OK : cuda_fail(e, "coat_adamw_step_multi");
+}
+
+static_assert(sizeof(coat_grad_clip) == sizeof(coat::ClipRecord) &&
+                  offsetof(coat_grad_clip, sumsq) == offsetof(coat::ClipRecord, sumsq) &&
+                  offsetof(coat_grad_clip, norm) == offsetof(coat::ClipRecord, norm) &&
+                  offsetof(coat_grad_clip, coef) == offsetof(coat::ClipRecord, coef) &&
+                  offsetof(coat_grad_clip, found_inf) == offsetof(coat::ClipRecord, found_inf),
+              "coat_grad_clip and ClipRecord must share one layout");
+
+coat_status coat_multi_plan_grad_norm(coat_multi_plan_t plan, float max_norm,
+                                      coat_grad_clip* d_clip, cudaStream_t stream) {
+  const char* fn = "coat_multi_plan_grad_norm";
+  if (!plan) return fail(COAT_ERR_INVALID_ARG, "%s: plan is NULL", fn);
+  if (!d_clip) return fail(COAT_ERR_INVALID_ARG, "%s: d_clip is NULL", fn);
+  if (!aligned(d_clip, 8)) return fail(COAT_ERR_MISALIGNED, "%s: d_clip is not 8-byte aligned", fn);
+  if (!(max_norm > 0.f)) return fail(COAT_ERR_INVALID_ARG, "%s: max_norm must be > 0", fn);
+  cudaError_t e = coat::launch_grad_sumsq(plan->d_descs, plan->num, plan->total_tiles,
+                                          plan->d_partials, plan->d_ticket, max_norm,
+                                          reinterpret_cast<coat::ClipRecord*>(d_clip), stream);
+  return e == cudaSuccess ? COAT_OK : cuda_fail(e, fn);
+}
+
+coat_status coat_adamw_step_multi_clipped(coat_multi_plan_t plan, float lr, float beta1,
+                                          float beta2, float eps, float wd, int64_t step,
+                                          const coat_grad_clip* d_clip, cudaStream_t stream) {
+  const char* fn = "coat_adamw_step_multi_clipped";
+  if (!plan) return fail(COAT_ERR_INVALID_ARG, "%s: plan is NULL", fn);
+  if (!d_clip) return fail(COAT_ERR_INVALID_ARG, "%s: d_clip is NULL", fn);
+  if (!aligned(d_clip, 8)) return fail(COAT_ERR_MISALIGNED, "%s: d_clip is not 8-byte aligned", fn);
+  coat_status st = check_hyper(lr, beta1, beta2, eps, wd, step);
+  if (st != COAT_OK) return st;
+  if (plan->total_tiles == 0) return COAT_OK;
+  unsigned* err = nullptr;
+  cudaError_t e = coat::device_error_ptr(&err);
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  e = coat::launch_adamw_multi(plan->d_descs, plan->num, plan->total_tiles, plan->fmt_m,
+                               plan->fmt_v, make_hyper(lr, beta1, beta2, eps, wd, step),
+                               reinterpret_cast<const coat::ClipRecord*>(d_clip), err, stream);
+  return e == cudaSuccess ? COAT_OK : cuda_fail(e, fn);
 }
 
 coat_status coat_multi_plan_set_wd_scale(coat_multi_plan_t plan, const float* host_wd_scale,
@@ -509,6 +560,6 @@ extern "C" coat_status coat_adamw_step_multi_noalloc(const coat_tensor_desc* hos
   if (tiles == 0) return COAT_OK;
   const cudaError_t e =
       coat::launch_adamw_multi(scratch->descs, num, tiles, fmt_m, fmt_v,
-                               make_hyper(lr, beta1, beta2, eps, wd, step), err, stream);
+                               make_hyper(lr, beta1, beta2, eps, wd, step), nullptr, err, stream);
   return e == cudaSuccess ? COAT_OK : COAT_ERR_CUDA;
 }

@@ -34,6 +34,17 @@ struct StepHyper {
   float lrwd;       // lr * wd
 };
 
+// Result of the gradient-norm pass over a plan's gradients; the same layout as
+// coat_grad_clip in coat.h.
+struct ClipRecord {
+  double sumsq;       // sum of g^2 over every gradient element (non-finite: an Inf/NaN seen)
+  float norm;         // sqrt(sumsq) rounded to FP32
+  float coef;         // min(1, max_norm / (sqrt(sumsq) + 1e-6)) in double, rounded to FP32
+  int32_t found_inf;  // 1 when sumsq is not finite
+  int32_t reserved;
+};
+static_assert(sizeof(ClipRecord) == 24, "ClipRecord layout");
+
 int sm_count(int dev);
 cudaError_t device_error_ptr(unsigned** out);
 int64_t step_tile_groups();
@@ -42,8 +53,21 @@ cudaError_t launch_adamw_single(const TensorArgs& t, int fm, int fv, const StepH
                                 unsigned* err, cudaStream_t stream);
 // d_descs: num descriptors in device memory, tile_begin ascending (an empty
 // tensor shares the next tensor's first tile); total_tiles: sum of tiles.
+// clip: null, or a record written by launch_grad_sumsq: the step uses
+// coef * g as the gradient, and does nothing at all when found_inf is set.
 cudaError_t launch_adamw_multi(const TensorArgs* d_descs, int num, int64_t total_tiles, int fm,
-                               int fv, const StepHyper& h, unsigned* err, cudaStream_t stream);
+                               int fv, const StepHyper& h, const ClipRecord* clip, unsigned* err,
+                               cudaStream_t stream);
+
+// Slots of per-CTA partial sums the gradient-norm pass needs on device dev.
+int grad_sumsq_slots(int dev);
+// Sum of squares of every gradient element of the descriptors into *out (with
+// norm, clip coefficient for max_norm and the non-finite flag).  partials:
+// grad_sumsq_slots() doubles; ticket: one unsigned that is 0 before the launch
+// (the launch leaves it 0).  Deterministic for a given device.
+cudaError_t launch_grad_sumsq(const TensorArgs* d_descs, int num, int64_t total_tiles,
+                              double* partials, unsigned* ticket, float max_norm, ClipRecord* out,
+                              cudaStream_t stream);
 
 // One warp waits (bounded by budget_cycles) on a barrier nothing arrives on.
 cudaError_t launch_wait_timeout_selftest(long long budget_cycles, unsigned* err,

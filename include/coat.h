@@ -153,8 +153,8 @@ coat_status coat_adamw_step(float *master, uint16_t *weight_bf16_out, const uint
  *
  * coat_multi_plan_create copies `num` host descriptors (each obeying the
  * coat_adamw_step rules for its own n) into a device table owned by the plan
- * (one cudaMalloc; COAT_ERR_NOMEM on failure); the copy is enqueued on
- * `stream`.  The plan refers to the caller's buffers, which must stay valid
+ * (one cudaMalloc, which also holds the gradient-norm scratch below;
+ * COAT_ERR_NOMEM on failure); the copy is enqueued on `stream`.  The plan refers to the caller's buffers, which must stay valid
  * while the plan is used.  Tensors with n == 0 are allowed.  num >= 1.
  * coat_adamw_step_multi applies one step to all tensors on `stream`.
  * coat_multi_plan_destroy frees the table (after synchronising the device);
@@ -192,6 +192,51 @@ coat_status coat_multi_plan_set_wd_scale(coat_multi_plan_t plan, const float *ho
 /* Number of elements and tensors covered by a plan. */
 coat_status coat_multi_plan_info(coat_multi_plan_t plan, int64_t *total_elements,
                                  int *num_tensors);
+
+/* ---------------------------------------------------------------------------
+ * Global gradient-norm clipping and the non-finite check before the step.
+ * The COAT pages do not describe this step; it is the pre-step of an ordinary
+ * training loop (torch.nn.utils.clip_grad_norm_ over all parameters, and the
+ * found-Inf check of a loss-scaled loop that skips the step on overflow),
+ * kept on the device so that no value has to travel to the host between the
+ * backward pass and the optimizer step.
+ *
+ * coat_multi_plan_grad_norm reads every gradient of the plan once and writes
+ * one coat_grad_clip record to `d_clip` (device memory, 8-byte aligned, owned
+ * by the caller) on `stream`:
+ *   - sumsq: the sum of g^2 over all gradient elements, accumulated in double
+ *     (squares exact; partial sums of 8 squares rounded in FP32, so sumsq is
+ *     within about 3e-7 relative of the exact sum); +Inf or NaN when any
+ *     element is Inf or NaN;
+ *   - norm: sqrt(sumsq) rounded to FP32;
+ *   - coef: min(1, max_norm / (sqrt(sumsq) + 1e-6)), evaluated in double and
+ *     rounded to FP32 (1 for max_norm = +Inf);
+ *   - found_inf: 1 when sumsq is not finite, else 0; reserved: 0.
+ * max_norm > 0 (+Inf allowed: the norm without clipping).  The result is
+ * deterministic on a given device.  The plan holds the pass's scratch (one
+ * slot per CTA and a counter), so calls on one plan must be ordered on one
+ * stream, as steps are.
+ *
+ * coat_adamw_step_multi_clipped is coat_adamw_step_multi with every gradient
+ * element g replaced by coef * g, coef read from `d_clip` on the device when
+ * the step runs; when found_inf is nonzero the step changes nothing (master,
+ * bf16 copy, codes and metadata keep their bytes).  With coef = 1 it gives
+ * the same bytes as coat_adamw_step_multi.  d_clip: as written by
+ * coat_multi_plan_grad_norm, or by the caller in the same layout.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+    double sumsq;
+    float norm;
+    float coef;
+    int32_t found_inf;
+    int32_t reserved;
+} coat_grad_clip; /* 24 bytes */
+
+coat_status coat_multi_plan_grad_norm(coat_multi_plan_t plan, float max_norm,
+                                      coat_grad_clip *d_clip, cudaStream_t stream);
+coat_status coat_adamw_step_multi_clipped(coat_multi_plan_t plan, float lr, float beta1,
+                                          float beta2, float eps, float wd, int64_t step,
+                                          const coat_grad_clip *d_clip, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
  * No-allocation variant of the multi-tensor step.  The COAT pages have no

@@ -87,6 +87,32 @@ def test_wd_scale_validation():
     assert "plan is NULL" in coat.coat_last_error()
 
 
+def test_grad_clip_validation():
+    """Argument checks of the clipping entry points run before the plan or the
+    record is touched (a host buffer stands in for the plan handle)."""
+    L = coat.lib()
+    fake = ctypes.create_string_buffer(256)
+    plan = ctypes.cast(fake, ctypes.c_void_p)
+    rec = ctypes.addressof(fake) + 64
+    assert L.coat_multi_plan_grad_norm(None, 1.0, rec, None) == INVALID
+    assert "plan is NULL" in coat.coat_last_error()
+    assert L.coat_multi_plan_grad_norm(plan, 1.0, None, None) == INVALID
+    assert "d_clip is NULL" in coat.coat_last_error()
+    assert L.coat_multi_plan_grad_norm(plan, 1.0, rec + 4, None) == MISALIGNED
+    for bad in (0.0, -1.0, float("nan")):
+        assert L.coat_multi_plan_grad_norm(plan, bad, rec, None) == INVALID
+        assert "max_norm" in coat.coat_last_error()
+    step = lambda **k: L.coat_adamw_step_multi_clipped(
+        k.get("plan", plan), k.get("lr", 1e-3), 0.9, 0.95, 1e-8, 0.0, k.get("step", 1),
+        k.get("rec", rec), None)
+    assert step(plan=None) == INVALID
+    assert step(rec=None) == INVALID and "d_clip is NULL" in coat.coat_last_error()
+    assert step(rec=rec + 4) == MISALIGNED
+    assert step(lr=-1.0) == INVALID
+    assert step(step=0) == INVALID
+    assert ctypes.sizeof(coat.GradClip) == 24
+
+
 def test_selftest_budget_validation():
     L = coat.lib()
     assert L.coat_selftest_wait_timeout(999, None) == INVALID
