@@ -95,6 +95,18 @@ def lib():
         L.orc_adamw_step_unquantized.argtypes = [_P(ctypes.c_double)] * 4 + [
             ctypes.c_int64, ctypes.c_double, ctypes.c_double, ctypes.c_double, ctypes.c_double,
             ctypes.c_double, ctypes.c_int64]
+        L.orc_swiglu.restype = ctypes.c_double
+        L.orc_swiglu.argtypes = [ctypes.c_double, ctypes.c_double]
+        L.orc_swiglu_grad.restype = None
+        L.orc_swiglu_grad.argtypes = [ctypes.c_double] * 3 + [_P(ctypes.c_double)] * 2
+        _u8, _f, _i = _P(ctypes.c_uint8), _P(ctypes.c_float), ctypes.c_int64
+        L.orc_swiglu_fp8_forward.restype = ctypes.c_int
+        L.orc_swiglu_fp8_forward.argtypes = [_u8, _i, _f, _f, _i, _u8, _i, _f, _f, _i, _i, _i,
+                                             ctypes.c_int, ctypes.c_int, _u8, _i, _f, _f, _i]
+        L.orc_swiglu_fp8_backward.restype = ctypes.c_int
+        L.orc_swiglu_fp8_backward.argtypes = [_P(ctypes.c_uint16), _i, _u8, _i, _f, _f, _i, _u8,
+                                              _i, _f, _f, _i, _i, _i, ctypes.c_int,
+                                              _P(ctypes.c_uint16), _i, _P(ctypes.c_uint16), _i]
         _lib = L
     return _lib
 
@@ -256,3 +268,66 @@ def adamw_step_unquantized(p, m, v, g, *, lr, beta1, beta2, eps, wd, step):
                                           _ptr(v, ctypes.c_double), _ptr(g, ctypes.c_double),
                                           p.size, lr, beta1, beta2, eps, wd, step)
     assert rc == 0
+
+
+# ----------------------------------------------------------------------------
+# FP8 precision flow through the SwiGLU activation (silu(gate) * up)
+# ----------------------------------------------------------------------------
+
+def swiglu(g: float, u: float) -> float:
+    return lib().orc_swiglu(float(g), float(u))
+
+
+def swiglu_grad(g: float, u: float, dh: float):
+    """(d/dgate, d/dup) of dh * silu(g) * u."""
+    a, b = ctypes.c_double(), ctypes.c_double()
+    lib().orc_swiglu_grad(float(g), float(u), float(dh), ctypes.byref(a), ctypes.byref(b))
+    return a.value, b.value
+
+
+def _act(t):
+    q, s, k = (np.ascontiguousarray(t[0], dtype=np.uint8), np.ascontiguousarray(t[1], np.float32),
+               np.ascontiguousarray(t[2], np.float32))
+    assert q.ndim == 2 and s.shape == k.shape and s.shape[0] == q.shape[0]
+    assert s.shape[1] == -(-q.shape[1] // 128)
+    return q, s, k
+
+
+def swiglu_fp8_forward(gate, up, fmt: int, expand: bool):
+    """gate, up: (codes u8 [rows, cols], scale f32 [rows, ngroups], k f32 [rows, ngroups]).
+    Returns the output in the same form, quantised per 1x128 group."""
+    gq, gs, gk = _act(gate)
+    uq, us, uk = _act(up)
+    assert gq.shape == uq.shape
+    rows, cols = gq.shape
+    ng = gs.shape[1]
+    oq = np.zeros((rows, cols), np.uint8)
+    os_ = np.zeros((rows, ng), np.float32)
+    ok = np.zeros((rows, ng), np.float32)
+    u8, f = ctypes.c_uint8, ctypes.c_float
+    rc = lib().orc_swiglu_fp8_forward(_ptr(gq, u8), cols, _ptr(gs, f), _ptr(gk, f), ng,
+                                      _ptr(uq, u8), cols, _ptr(us, f), _ptr(uk, f), ng, rows, cols,
+                                      fmt, int(bool(expand)), _ptr(oq, u8), cols, _ptr(os_, f),
+                                      _ptr(ok, f), ng)
+    assert rc == 0
+    return oq, os_, ok
+
+
+def swiglu_fp8_backward(dh_bits, gate, up, fmt: int):
+    """dh_bits: bf16 bits u16 [rows, cols]; gate / up as for the forward.
+    Returns (dgate, dup) as bf16 bits."""
+    gq, gs, gk = _act(gate)
+    uq, us, uk = _act(up)
+    dh = np.ascontiguousarray(dh_bits, dtype=np.uint16)
+    assert dh.shape == gq.shape == uq.shape
+    rows, cols = gq.shape
+    ng = gs.shape[1]
+    dg = np.zeros((rows, cols), np.uint16)
+    du = np.zeros((rows, cols), np.uint16)
+    u8, f, u16 = ctypes.c_uint8, ctypes.c_float, ctypes.c_uint16
+    rc = lib().orc_swiglu_fp8_backward(_ptr(dh, u16), cols, _ptr(gq, u8), cols, _ptr(gs, f),
+                                       _ptr(gk, f), ng, _ptr(uq, u8), cols, _ptr(us, f),
+                                       _ptr(uk, f), ng, rows, cols, fmt, _ptr(dg, u16), cols,
+                                       _ptr(du, u16), cols)
+    assert rc == 0
+    return dg, du

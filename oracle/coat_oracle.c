@@ -447,3 +447,94 @@ int orc_adamw_step_unquantized(double *p, double *m, double *v, const double *g,
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* FP8 precision flow through a non-linear layer ([P1] sections        */
+/* "FP8激活" and "解决方案：混合粒度FP8精度流"): the layer's inputs and  */
+/* output are FP8 tensors in 1x128 per-token groups, and the FP8 inputs */
+/* are what the backward pass reads (nothing is requantised for it).   */
+/* The layer is Llama's gated activation h = silu(gate) * up (SwiGLU),  */
+/* silu(g) = g sigmoid(g) = g / (1 + e^-g).                            */
+/* Readings: the activation value h is rounded to FP32 before it is     */
+/* quantised (the kernel's precision decides the codes); the incoming   */
+/* gradient and the outgoing input gradients are bf16, the gradients    */
+/* rounded double -> FP32 -> bf16 (RNE both times).                     */
+/* ------------------------------------------------------------------ */
+
+static double orc_sigmoid(double g) { return 1.0 / (1.0 + exp(-g)); }
+
+/* silu(g) * u */
+double orc_swiglu(double g, double u)
+{
+    return g * orc_sigmoid(g) * u;
+}
+
+/* Partial derivatives of dh * silu(g) u:
+ *   d/du = dh silu(g),
+ *   d/dg = dh u (sigmoid(g) + g sigmoid(g)(1 - sigmoid(g))). */
+void orc_swiglu_grad(double g, double u, double dh, double *dg, double *du)
+{
+    double s = orc_sigmoid(g);
+    *du = dh * g * s;
+    *dg = dh * u * s * (1.0 + g * (1.0 - s));
+}
+
+/* Forward over a rows x cols FP8 layer.  gate / up / out: codes with row
+ * stride ld*_q bytes; per-group scale and k with row stride ld*_s floats
+ * (groups of 128 along a row, the last one partial when cols % 128 != 0).
+ * The output is quantised per 1x128 group with or without expansion.
+ * Returns 0, or -1 on bad arguments. */
+int orc_swiglu_fp8_forward(const uint8_t *gq, int64_t ldgq, const float *gs, const float *gk,
+                           int64_t ldgs, const uint8_t *uq, int64_t lduq, const float *us,
+                           const float *uk, int64_t ldus, int64_t rows, int64_t cols, int fmt,
+                           int expand, uint8_t *oq, int64_t ldoq, float *os, float *ok,
+                           int64_t ldos)
+{
+    if (rows < 0 || cols < 0 || ldgq < cols || lduq < cols || ldoq < cols)
+        return -1;
+    int64_t ng = (cols + 127) / 128;
+    if (ldgs < ng || ldus < ng || ldos < ng)
+        return -1;
+    double h[128];
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t j = 0; j < ng; j++) {
+            int64_t c0 = j * 128, cnt = cols - c0 < 128 ? cols - c0 : 128;
+            for (int64_t i = 0; i < cnt; i++) {
+                double g = orc_dequant_value(fmt, gq[r * ldgq + c0 + i], gs[r * ldgs + j],
+                                             gk[r * ldgs + j]);
+                double u = orc_dequant_value(fmt, uq[r * lduq + c0 + i], us[r * ldus + j],
+                                             uk[r * ldus + j]);
+                h[i] = (double)(float)orc_swiglu(g, u);
+            }
+            orc_quantize_group(h, cnt, expand, fmt, oq + r * ldoq + c0, &ok[r * ldos + j],
+                               &os[r * ldos + j]);
+        }
+    return 0;
+}
+
+/* Backward: dh (bf16 bits, row stride lddh elements) and the forward's FP8
+ * inputs give dgate and dup (bf16 bits, row strides lddg / lddu). */
+int orc_swiglu_fp8_backward(const uint16_t *dh, int64_t lddh, const uint8_t *gq, int64_t ldgq,
+                            const float *gs, const float *gk, int64_t ldgs, const uint8_t *uq,
+                            int64_t lduq, const float *us, const float *uk, int64_t ldus,
+                            int64_t rows, int64_t cols, int fmt, uint16_t *dg, int64_t lddg,
+                            uint16_t *du, int64_t lddu)
+{
+    if (rows < 0 || cols < 0 || lddh < cols || ldgq < cols || lduq < cols || lddg < cols ||
+        lddu < cols)
+        return -1;
+    int64_t ng = (cols + 127) / 128;
+    if (ldgs < ng || ldus < ng)
+        return -1;
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t c = 0; c < cols; c++) {
+            int64_t j = c / 128;
+            double g = orc_dequant_value(fmt, gq[r * ldgq + c], gs[r * ldgs + j], gk[r * ldgs + j]);
+            double u = orc_dequant_value(fmt, uq[r * lduq + c], us[r * ldus + j], uk[r * ldus + j]);
+            double a, b;
+            orc_swiglu_grad(g, u, orc_bf16_to_double(dh[r * lddh + c]), &a, &b);
+            dg[r * lddg + c] = orc_float_to_bf16((float)a);
+            du[r * lddu + c] = orc_float_to_bf16((float)b);
+        }
+    return 0;
+}
