@@ -456,12 +456,18 @@ int orc_adamw_step_unquantized(double *p, double *m, double *v, const double *g,
 /* The layer is Llama's gated activation h = silu(gate) * up (SwiGLU),  */
 /* silu(g) = g sigmoid(g) = g / (1 + e^-g).                            */
 /* Readings: the activation value h is rounded to FP32 before it is     */
-/* quantised (the kernel's precision decides the codes); the incoming   */
-/* gradient and the outgoing input gradients are bf16, the gradients    */
-/* rounded double -> FP32 -> bf16 (RNE both times).                     */
+/* quantised (the kernel's precision decides the codes); a sigmoid      */
+/* below FP32's normal range (2^-126, i.e. g < -87.3) counts as 0, as   */
+/* in FP32 arithmetic that flushes subnormals; the incoming gradient    */
+/* and the outgoing input gradients are bf16, the gradients rounded     */
+/* double -> FP32 -> bf16 (RNE both times).                             */
 /* ------------------------------------------------------------------ */
 
-static double orc_sigmoid(double g) { return 1.0 / (1.0 + exp(-g)); }
+static double orc_sigmoid(double g)
+{
+    double s = 1.0 / (1.0 + exp(-g));
+    return s < 0x1p-126 ? 0.0 : s;
+}
 
 /* silu(g) * u */
 double orc_swiglu(double g, double u)

@@ -37,6 +37,9 @@ def test_swiglu_closed_forms(orc):
     # e^-64 is below half an ulp of 1: sigmoid(64) is exactly 1 in double
     assert orc.swiglu(64.0, 5.0) == 320.0
     assert math.isclose(orc.swiglu(-64.0, 1.0), -64.0 * math.exp(-64.0), rel_tol=1e-12)
+    # a sigmoid below FP32's normal range (2^-126) counts as 0
+    assert orc.swiglu(-87.0, 1.0) != 0.0 and orc.swiglu(-88.0, 1.0) == 0.0
+    assert orc.swiglu_grad(-88.0, 2.0, 1.0) == (0.0, 0.0)
 
 
 def test_swiglu_grad_closed_forms(orc):
