@@ -686,6 +686,164 @@ def run_codec(args, ws, rank, local):
     return result
 
 
+SWIGLU_METRIC = ("GB/s of the FP8 SwiGLU layer (forward + backward, FP8 1x128 in/out); "
+                 "HBM GB/s as % of B200 roofline")
+SWIGLU_SHAPE = (8192, 11008)   # tokens x Llama-2-7B MLP width
+
+
+def swiglu_bytes(rows, cols):
+    """Algorithmic bytes: forward = two codes in, one out (3 B per element) + 24 B
+    of scale / k per group; backward = dh in, two codes in, two bf16 out
+    (8 B per element) + 16 B per group."""
+    groups = rows * -(-cols // 128)
+    return 3 * rows * cols + 24 * groups, 8 * rows * cols + 16 * groups
+
+
+def run_swiglu(args, ws, rank, local):
+    import torch
+    import fp8_optimizer_state_b200 as coat
+    import synth
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    coat.lib()
+    E4M3 = 0
+    T, F = SWIGLU_SHAPE
+    ng = F // 128
+    # the fused up/gate projection output [T, 2F] as bf16 activations, quantised
+    # to E4M3 1x128 (no expansion) by the library's codec: gate = [:, :F], up = [:, F:]
+    x = torch.empty(T, 2 * F, dtype=torch.bfloat16, device=dev)
+    synth.device_activations(x.view(torch.int16).view(-1), rank, 0)
+    xq = torch.empty(T, 2 * F, dtype=torch.uint8, device=dev)
+    xs = torch.empty(T, 2 * ng, dtype=torch.float32, device=dev)
+    xk = torch.empty(T, 2 * ng, dtype=torch.float32, device=dev)
+    coat.coat_group_quantize(x, 1, 128, False, E4M3, xq, xs, xk)
+    del x
+    gate = (xq[:, :F], xs[:, :ng], xk[:, :ng])
+    up = (xq[:, F:], xs[:, ng:], xk[:, ng:])
+    out = (torch.empty(T, F, dtype=torch.uint8, device=dev),
+           torch.empty(T, ng, dtype=torch.float32, device=dev),
+           torch.empty(T, ng, dtype=torch.float32, device=dev))
+    dh = torch.empty(T, F, dtype=torch.int16, device=dev)
+    synth.device_grad(dh.view(-1), rank, 9, 1)
+    grads = torch.empty(T, 2 * F, dtype=torch.int16, device=dev)
+    fwd = lambda: coat.coat_swiglu_fp8_forward(gate, up, E4M3, False, out)
+    bwd = lambda: coat.coat_swiglu_fp8_backward(dh, gate, up, E4M3, grads[:, :F], grads[:, F:])
+    for _ in range(args.warmup):
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    props = torch.cuda.get_device_properties(dev)
+    bus = "%08x:%02x:%02x.0" % (int(getattr(props, "pci_domain_id", 0)),
+                                int(getattr(props, "pci_bus_id", 0)),
+                                int(getattr(props, "pci_device_id", 0)))
+    sampler = ClockSampler(bus)
+    sampler.start()
+    time.sleep(0.3)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    barrier(ws, dev)
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        fwd()
+        ev[i][1].record(stream)
+        bwd()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    barrier(ws, dev)
+    time.sleep(0.2)
+    sampler.stop()
+    f_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in ev), ws, dev)
+    b_ms = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in ev), ws, dev)
+    fb, bb = swiglu_bytes(T, F)
+    step_ms = f_ms + b_ms
+    value = ws * (fb + bb) / (step_ms * 1e-3) / 1e9
+    peaks = measured_peaks()
+    peak = peaks["hbm_gbs"] if peaks and peaks.get("hbm_gbs") else HBM_FALLBACK_GBS
+    kern = [{"launch": lab, "ms": round(t, 4), "algorithmic_bytes": b,
+             "GB/s": round(b / (t * 1e-3) / 1e9, 1), "frac": round(b / (t * 1e-3) / 1e9 / peak, 4)}
+            for lab, t, b in (("forward", f_ms, fb), ("backward", b_ms, bb))]
+    top = 0 if f_ms >= b_ms else 1
+    roofline = {"bound": "hbm", "achieved": kern[top]["GB/s"], "peak": peak, "unit": "GB/s",
+                "frac": kern[top]["frac"], "traffic": None, "kernel": kern[top]["launch"],
+                "peak_source": "measured" if peaks else "fallback"}
+    clocks = sampler.summary(wall0, wall1)
+
+    e2e = None
+    if not args.no_e2e:
+        # public API with host buffers: H2D of the FP8 gate/up (codes, scale, k)
+        # and of dh from pinned memory, forward + backward, D2H of the FP8
+        # output and of both bf16 input gradients
+        hin = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (xq, xs, xk, dh)]
+        hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (*out, grads)]
+        for h, t in zip(hin, (xq, xs, xk, dh)):
+            h.copy_(t)
+        torch.cuda.synchronize()
+        steps = max(1, min(args.steps, args.e2e_steps))
+        barrier(ws, dev)
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            for h, t in zip(hin, (xq, xs, xk, dh)):
+                t.copy_(h, non_blocking=True)
+            fwd()
+            bwd()
+            for h, t in zip(hout, (*out, grads)):
+                h.copy_(t, non_blocking=True)
+        torch.cuda.synchronize()
+        el = max_over_ranks(time.perf_counter() - t0, ws, dev)
+        e2e = {"value": round(ws * (fb + bb) * steps / el / 1e9, 3), "unit": "GB/s",
+               "h2d_bytes_per_step": sum(h.numel() * h.element_size() for h in hin),
+               "d2h_bytes_per_step": sum(h.numel() * h.element_size() for h in hout),
+               "steps": steps,
+               "how": "H2D of the FP8 inputs and dh from pinned memory, forward + backward, D2H "
+                      "of the FP8 output and both bf16 gradients; host wall clock"}
+    coat.coat_check_device_error()
+    result = None
+    if rank == 0:
+        cpu = None
+        if ws == 1 and not args.no_cpu_baseline:
+            import oracle as orc
+            rows = 16
+            hq, hs, hk = xq[:rows].cpu().numpy(), xs[:rows].cpu().numpy(), xk[:rows].cpu().numpy()
+            g_ = (hq[:, :F].copy(), hs[:, :ng].copy(), hk[:, :ng].copy())
+            u_ = (hq[:, F:].copy(), hs[:, ng:].copy(), hk[:, ng:].copy())
+            d_ = dh[:rows].cpu().numpy().view(np.uint16)
+            t0 = time.perf_counter()
+            orc.swiglu_fp8_forward(g_, u_, E4M3, False)
+            orc.swiglu_fp8_backward(d_, g_, u_, E4M3)
+            el = time.perf_counter() - t0
+            sb = sum(swiglu_bytes(rows, F))
+            cpu = {"value": round(sb / el / 1e9, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                   "sample": "first %d token rows, forward + backward, one host thread (%.2f s)"
+                             % (rows, el)}
+        result = {
+            "metric": SWIGLU_METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": "FP8 SwiGLU layer, %d tokens x %d (Llama-2-7B MLP width): gate "
+                                   "and up as the halves of one E4M3 1x128 [T, 2F] tensor "
+                                   "(N(0,1) activations with 0.1%% x100 outliers), E4M3 1x128 "
+                                   "output without expansion, bf16 gradients" % (T, F),
+                       "l2": "no flush: %.0f MB forward + %.0f MB backward per step >> 126 MB L2"
+                             % (fb / 1e6, bb / 1e6),
+                       "parallelism": "single GPU" if ws == 1 else "replicas%d" % ws},
+            "launches": kern, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": 2 * args.steps, "clocks": clocks}
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return result
+
+
 def run_reference(args, cfg, ws, rank):
     """The CPU oracle on a bounded sample per step (one host thread)."""
     if rank != 0:
@@ -715,7 +873,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default="llama2-7b", choices=sorted(CONFIGS) + ["act-codec"])
+    ap.add_argument("--config", default="llama2-7b",
+                    choices=sorted(CONFIGS) + ["act-codec", "swiglu-fp8"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -731,12 +890,13 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     ws, rank, local = dist_env()
-    if args.config == "act-codec":
+    if args.config in ("act-codec", "swiglu-fp8"):
         if args.impl == "reference":
-            print(json.dumps({"impl": "reference", "unavailable": "the codec workload has no "
+            print(json.dumps({"impl": "reference", "unavailable": "this workload has no "
                               "reference arm; the oracle CPU baseline is in the ours line"}))
             return
-        res = run_codec(args, ws, rank, local)
+        run = run_codec if args.config == "act-codec" else run_swiglu
+        res = run(args, ws, rank, local)
         if res is not None:
             print(json.dumps(res), flush=True)
         return

@@ -44,6 +44,9 @@ EXPORTS = [
     ("coat_selftest_wait_timeout", _i32, [_i64, _vp]),
     ("coat_multi_plan_grad_norm", _i32, [_vp, _f32, _vp, _vp]),
     ("coat_adamw_step_multi_clipped", _i32, [_vp, _f32, _f32, _f32, _f32, _f32, _i64, _vp, _vp]),
+    ("coat_swiglu_fp8_forward", _i32, [_vp, _vp, _i64, _i64, _i32, _i32, _vp, _vp]),
+    ("coat_swiglu_fp8_backward", _i32, [_vp, _i64, _vp, _vp, _i64, _i64, _i32, _vp, _i64, _vp,
+                                        _i64, _vp]),
 ]
 NOALLOC_MAX_TENSORS = 1024
 
@@ -79,6 +82,43 @@ def write_grad_clip(buf, coef, found_inf=0, sumsq=0.0, norm=0.0):
     rec = GradClip(float(sumsq), float(norm), float(coef), int(found_inf), 0)
     host = torch.frombuffer(bytearray(bytes(rec)), dtype=torch.uint8)
     buf.copy_(host)
+
+
+class Fp8Act(ctypes.Structure):
+    """coat_fp8_act"""
+    _fields_ = [("q", _vp), ("scale", _vp), ("k", _vp), ("ldq", _i64), ("lds", _i64)]
+
+
+def _act(t):
+    """(codes [rows, cols] uint8, scale [rows, groups] f32, k [rows, groups] f32) CUDA
+    tensors, unit stride along a row (views into a wider buffer are fine)."""
+    q, sc, k = t
+    if q.dim() != 2 or sc.dim() != 2 or k.dim() != 2 or sc.stride() != k.stride():
+        raise ValueError("expected 2-D codes, scale and k with matching strides")
+    if q.stride(1) != 1 or sc.stride(1) != 1:
+        raise ValueError("rows must be contiguous")
+    return Fp8Act(_p(q), _p(sc), _p(k), q.stride(0), sc.stride(0))
+
+
+def coat_swiglu_fp8_forward(gate, up, fmt, expand_out, out, stream=None):
+    """gate, up, out: (codes, scale, k) tensors in the 1x128 layout; out is written."""
+    g, u, o = _act(gate), _act(up), _act(out)
+    rows, cols = gate[0].shape
+    _check(lib().coat_swiglu_fp8_forward(ctypes.byref(g), ctypes.byref(u), rows, cols, fmt,
+                                         int(bool(expand_out)), ctypes.byref(o), _s(stream)))
+
+
+def coat_swiglu_fp8_backward(grad_out, gate, up, fmt, grad_gate, grad_up, stream=None):
+    """grad_out, grad_gate, grad_up: bf16 (or int16 bit) [rows, cols] CUDA tensors."""
+    g, u = _act(gate), _act(up)
+    rows, cols = gate[0].shape
+    for t in (grad_out, grad_gate, grad_up):
+        if t.dim() != 2 or t.stride(1) != 1 or t.element_size() != 2:
+            raise ValueError("expected 2-D bf16 tensors with contiguous rows")
+    _check(lib().coat_swiglu_fp8_backward(_p(grad_out), grad_out.stride(0), ctypes.byref(g),
+                                          ctypes.byref(u), rows, cols, fmt, _p(grad_gate),
+                                          grad_gate.stride(0), _p(grad_up), grad_up.stride(0),
+                                          _s(stream)))
 
 
 class TensorDesc(ctypes.Structure):

@@ -19,7 +19,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libcoat.so")
-SOURCES = ["api.cu", "adamw_fp8.cu", "codec.cu"]
+SOURCES = ["api.cu", "adamw_fp8.cu", "codec.cu", "fp8_flow.cu"]
 HEADERS = ["coat_device.cuh", "coat_internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",

@@ -248,6 +248,76 @@ coat_status coat_group_dequantize(const uint8_t* q, int64_t ld_q, const float* s
   return e == cudaSuccess ? COAT_OK : cuda_fail(e, fn);
 }
 
+static coat_status check_act(const char* fn, const char* name, const coat_fp8_act* a, int64_t rows,
+                             int64_t cols) {
+  if (!a) return fail(COAT_ERR_INVALID_ARG, "%s: %s is NULL", fn, name);
+  const int64_t ng = (cols + 127) / 128;
+  if (a->ldq < cols || a->lds < ng)
+    return fail(COAT_ERR_INVALID_ARG, "%s: %s strides too small (ldq >= cols, lds >= groups)", fn, name);
+  if (rows == 0 || cols == 0) return COAT_OK;
+  if (!a->q || !a->scale || !a->k) return fail(COAT_ERR_INVALID_ARG, "%s: %s has a NULL array", fn, name);
+  if (!aligned(a->q, 16) || (rows > 1 && a->ldq % 16 != 0))
+    return fail(COAT_ERR_MISALIGNED, "%s: %s codes need 16-byte alignment and row stride", fn, name);
+  if (!aligned(a->scale, 4) || !aligned(a->k, 4))
+    return fail(COAT_ERR_MISALIGNED, "%s: %s scale/k not 4-byte aligned", fn, name);
+  return COAT_OK;
+}
+
+static coat_status check_bf16(const char* fn, const char* name, const void* p, int64_t ld,
+                              int64_t rows, int64_t cols) {
+  if (ld < cols) return fail(COAT_ERR_INVALID_ARG, "%s: %s leading dimension < cols", fn, name);
+  if (rows == 0 || cols == 0) return COAT_OK;
+  if (!p) return fail(COAT_ERR_INVALID_ARG, "%s: %s is NULL", fn, name);
+  if (!aligned(p, 16) || (rows > 1 && (ld * 2) % 16 != 0))
+    return fail(COAT_ERR_MISALIGNED, "%s: %s needs 16-byte alignment and row stride", fn, name);
+  return COAT_OK;
+}
+
+static coat::ActArgs act_args(const coat_fp8_act* a) {
+  return coat::ActArgs{a->q, a->scale, a->k, a->ldq, a->lds};
+}
+
+coat_status coat_swiglu_fp8_forward(const coat_fp8_act* gate, const coat_fp8_act* up, int64_t rows,
+                                    int64_t cols, coat_fmt fmt, int expand_out,
+                                    const coat_fp8_act* out, cudaStream_t stream) {
+  const char* fn = "coat_swiglu_fp8_forward";
+  if (rows < 0 || cols < 0) return fail(COAT_ERR_INVALID_ARG, "%s: negative shape", fn);
+  if (!valid_fmt(fmt)) return fail(COAT_ERR_INVALID_ARG, "%s: bad fmt %d", fn, int(fmt));
+  if (expand_out != 0 && expand_out != 1)
+    return fail(COAT_ERR_INVALID_ARG, "%s: expand_out must be 0 or 1", fn);
+  if (cols % 16 != 0) return fail(COAT_ERR_UNSUPPORTED, "%s: cols must be a multiple of 16", fn);
+  coat_status st = check_act(fn, "gate", gate, rows, cols);
+  if (st == COAT_OK) st = check_act(fn, "up", up, rows, cols);
+  if (st == COAT_OK) st = check_act(fn, "out", out, rows, cols);
+  if (st != COAT_OK) return st;
+  if (rows == 0 || cols == 0) return COAT_OK;
+  cudaError_t e = coat::launch_swiglu_fp8_forward(act_args(gate), act_args(up), rows, cols, fmt,
+                                                  expand_out, act_args(out), stream);
+  return e == cudaSuccess ? COAT_OK : cuda_fail(e, fn);
+}
+
+coat_status coat_swiglu_fp8_backward(const uint16_t* grad_out, int64_t ld_grad_out,
+                                     const coat_fp8_act* gate, const coat_fp8_act* up,
+                                     int64_t rows, int64_t cols, coat_fmt fmt,
+                                     uint16_t* grad_gate, int64_t ld_grad_gate, uint16_t* grad_up,
+                                     int64_t ld_grad_up, cudaStream_t stream) {
+  const char* fn = "coat_swiglu_fp8_backward";
+  if (rows < 0 || cols < 0) return fail(COAT_ERR_INVALID_ARG, "%s: negative shape", fn);
+  if (!valid_fmt(fmt)) return fail(COAT_ERR_INVALID_ARG, "%s: bad fmt %d", fn, int(fmt));
+  if (cols % 16 != 0) return fail(COAT_ERR_UNSUPPORTED, "%s: cols must be a multiple of 16", fn);
+  coat_status st = check_act(fn, "gate", gate, rows, cols);
+  if (st == COAT_OK) st = check_act(fn, "up", up, rows, cols);
+  if (st == COAT_OK) st = check_bf16(fn, "grad_out", grad_out, ld_grad_out, rows, cols);
+  if (st == COAT_OK) st = check_bf16(fn, "grad_gate", grad_gate, ld_grad_gate, rows, cols);
+  if (st == COAT_OK) st = check_bf16(fn, "grad_up", grad_up, ld_grad_up, rows, cols);
+  if (st != COAT_OK) return st;
+  if (rows == 0 || cols == 0) return COAT_OK;
+  cudaError_t e = coat::launch_swiglu_fp8_backward(grad_out, ld_grad_out, act_args(gate),
+                                                   act_args(up), rows, cols, fmt, grad_gate,
+                                                   ld_grad_gate, grad_up, ld_grad_up, stream);
+  return e == cudaSuccess ? COAT_OK : cuda_fail(e, fn);
+}
+
 coat_status coat_adamw_step(float* master, uint16_t* weight_bf16_out, const uint16_t* grad,
                             uint8_t* m_q, float* m_scale, float* m_k, uint8_t* v_q, float* v_scale,
                             float* v_k, int64_t n, int group, float lr, float beta1, float beta2,

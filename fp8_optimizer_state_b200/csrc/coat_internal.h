@@ -46,6 +46,12 @@ struct ClipRecord {
 static_assert(sizeof(ClipRecord) == 24, "ClipRecord layout");
 
 int sm_count(int dev);
+// Grid of at most sm_count(dev) * max_blocks_per_sm CTAs for work_items items
+// of per_block each (at least 1).
+unsigned grid_for(int64_t work_items, int per_block, int dev, int max_blocks_per_sm);
+// CTAs of a 256-thread kernel (plus dyn_smem bytes of dynamic shared memory)
+// resident per SM, from the occupancy calculator, cached per kernel.
+int resident_ctas(const void* kernel, size_t dyn_smem = 0);
 cudaError_t device_error_ptr(unsigned** out);
 int64_t step_tile_groups();
 
@@ -81,5 +87,26 @@ cudaError_t launch_group_quantize(const void* x, int xt, int64_t rows, int64_t c
 cudaError_t launch_group_dequantize(const uint8_t* q, int64_t ldq, const float* scale,
                                     const float* k, int64_t rows, int64_t cols, int gr, int gc,
                                     int fmt, void* out, int ot, int64_t ldo, cudaStream_t s);
+
+// One FP8 activation tensor in 1x128 per-token groups (device pointers):
+// codes rows x cols with row stride ldq bytes; root scale and k per group,
+// rows x ceil(cols/128) with row stride lds floats.
+struct ActArgs {
+  uint8_t* q;
+  float* scale;
+  float* k;
+  int64_t ldq;
+  int64_t lds;
+};
+
+// h = silu(gate) * up, quantised per 1x128 group (cols % 16 == 0).
+cudaError_t launch_swiglu_fp8_forward(const ActArgs& gate, const ActArgs& up, int64_t rows,
+                                      int64_t cols, int fmt, int expand, const ActArgs& out,
+                                      cudaStream_t s);
+// dgate, dup (bf16) from dh (bf16) and the forward's FP8 inputs (cols % 16 == 0).
+cudaError_t launch_swiglu_fp8_backward(const uint16_t* dh, int64_t lddh, const ActArgs& gate,
+                                       const ActArgs& up, int64_t rows, int64_t cols, int fmt,
+                                       uint16_t* dg, int64_t lddg, uint16_t* du, int64_t lddu,
+                                       cudaStream_t s);
 
 }  // namespace coat

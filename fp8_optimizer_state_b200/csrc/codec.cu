@@ -103,44 +103,6 @@ __device__ __forceinline__ void unpack16(const Raw16<DT>& r, float v[16]) {
   }
 }
 
-// 16 codes (four packed words) to a row: one 16-byte store when the chunk is whole.
-__device__ __forceinline__ void store16(uint8_t* q, const uint32_t (&w)[4], int valid) {
-  if (valid >= 16) {
-    *reinterpret_cast<uint4*>(q) = make_uint4(w[0], w[1], w[2], w[3]);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-      if (i < valid) q[i] = static_cast<uint8_t>(w[i >> 2] >> (8 * (i & 3)));
-  }
-}
-
-__device__ __forceinline__ int clamp_valid(int64_t left, int width) {
-  return left <= 0 ? 0 : (left >= width ? width : static_cast<int>(left));
-}
-
-// Max and min-nonzero of |x| over N values, on twice the FP32 bit patterns
-// (a = bits(x) * 2 drops the sign, one multiply-add off the integer ALU, and
-// orders like |x|): maxb = max a = 2 bits(max|x|) (at least 0xFF000000 iff an
-// Inf or NaN is present), mink = min(a - 2), so that zero becomes the largest
-// key and min nonzero |x| has bits (mink + 2) / 2.
-template <int N>
-__device__ __forceinline__ void stats_bits(const float (&v)[N], uint32_t& maxb, uint32_t& mink) {
-#pragma unroll
-  for (int i = 0; i < N; ++i) {
-    const uint32_t a = __float_as_uint(v[i]) * 2u;
-    maxb = max(maxb, a);
-    mink = min(mink, a - 2u);
-  }
-}
-
-// Max |x| ignoring NaN (the rare groups that hold an Inf or a NaN).
-template <int N>
-__device__ __forceinline__ float max_abs_nonnan(const float (&v)[N]) {
-  float M = 0.f;
-#pragma unroll
-  for (int i = 0; i < N; ++i) M = fmaxf(M, fabsf(v[i]));
-  return M;
-}
 
 // ---------------------------------------------------------------------------
 // 1 x 128 groups: 8 lanes per group, 16 contiguous elements per lane, 4 groups
@@ -585,6 +547,8 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
   }
 }
 
+}  // namespace
+
 unsigned grid_for(int64_t work_items, int per_block, int dev, int max_blocks_per_sm) {
   int64_t b = (work_items + per_block - 1) / per_block;
   const int64_t cap = int64_t(sm_count(dev)) * max_blocks_per_sm;
@@ -595,9 +559,12 @@ unsigned grid_for(int64_t work_items, int per_block, int dev, int max_blocks_per
 
 // CTAs of `kernel` (256 threads, plus dyn_smem bytes of dynamic shared memory) resident per SM,
 // from the occupancy calculator, cached per kernel (all B200s give the same).
+namespace {
 std::mutex g_occ_mu;
 std::unordered_map<const void*, int> g_occ;
-int resident_ctas(const void* kernel, size_t dyn_smem = 0) {
+}  // namespace
+
+int resident_ctas(const void* kernel, size_t dyn_smem) {
   std::lock_guard<std::mutex> lk(g_occ_mu);
   auto it = g_occ.find(kernel);
   if (it != g_occ.end()) return it->second;
@@ -611,7 +578,6 @@ int resident_ctas(const void* kernel, size_t dyn_smem = 0) {
   return n;
 }
 
-}  // namespace
 
 cudaError_t launch_fp8_encode(const float* y, int64_t n, int fmt, uint8_t* q, cudaStream_t s) {
   if (n == 0) return cudaSuccess;

@@ -277,6 +277,53 @@ coat_status coat_adamw_step_multi_noalloc(const coat_tensor_desc *host_descs, in
                                           cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * FP8 precision flow through a non-linear layer ([P1] FP8激活 and
+ * 解决方案：混合粒度FP8精度流): the layer's input and output are FP8 tensors
+ * in 1x128 per-token groups, and the backward pass reads the FP8 input as the
+ * forward received it (nothing is re-quantised to save it).  The layer is
+ * Llama's gated activation h = silu(gate) * up, silu(g) = g / (1 + e^-g).
+ *
+ * coat_fp8_act describes one rows x cols FP8 tensor in the codec's 1x128
+ * layout (coat_group_quantize with group 1x128): codes q (row stride ldq
+ * bytes), and per group a root scale and k (rows x ceil(cols/128), row stride
+ * lds floats); a value is sign(q) scale |q|^(1/k), k = 1 without expansion.
+ * gate and up may be two halves of one [rows x 2F] buffer (strides 2F and
+ * 2F/128, up starting F codes / F/128 groups in, F a multiple of 128).
+ *
+ * coat_swiglu_fp8_forward: h = silu(gate) up computed in FP32, then quantised
+ * per 1x128 group into `out` exactly as coat_group_quantize does (expand_out
+ * 0: k = 1; 1: expansion).  A sigmoid below 2^-126 is 0 (FP32 with subnormals
+ * flushed).  `out` must not overlap the inputs.
+ * coat_swiglu_fp8_backward: grad_out (bf16, row stride ld elements) and the
+ * forward's gate / up give
+ *   grad_up   = grad_out silu(g),
+ *   grad_gate = grad_out u sigmoid(g) (1 + g (1 - sigmoid(g))),
+ * computed in FP32 and rounded to bf16 (nearest even).
+ * Requirements: rows, cols >= 0 (0 is a no-op); cols a multiple of 16
+ * (COAT_ERR_UNSUPPORTED otherwise; the last group may be partial); every code
+ * and bf16 array 16-byte aligned with row strides that are multiples of 16
+ * bytes (ldq >= cols; bf16 strides >= cols); scale / k 4-byte aligned with
+ * lds >= ceil(cols/128); fmt the format of all three tensors.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+    uint8_t *q;
+    float *scale;
+    float *k;
+    int64_t ldq;
+    int64_t lds;
+} coat_fp8_act;
+
+coat_status coat_swiglu_fp8_forward(const coat_fp8_act *gate, const coat_fp8_act *up,
+                                    int64_t rows, int64_t cols, coat_fmt fmt, int expand_out,
+                                    const coat_fp8_act *out, cudaStream_t stream);
+coat_status coat_swiglu_fp8_backward(const uint16_t *grad_out, int64_t ld_grad_out,
+                                     const coat_fp8_act *gate, const coat_fp8_act *up,
+                                     int64_t rows, int64_t cols, coat_fmt fmt,
+                                     uint16_t *grad_gate, int64_t ld_grad_gate,
+                                     uint16_t *grad_up, int64_t ld_grad_up,
+                                     cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Device error word.  Kernels that wait on a shared-memory barrier give up
  * after a bounded time (about one second), set a flag and return;
  * coat_check_device_error synchronises `stream`, reads and clears the flag,

@@ -113,6 +113,38 @@ def test_grad_clip_validation():
     assert ctypes.sizeof(coat.GradClip) == 24
 
 
+def test_swiglu_validation():
+    """Argument checks of the FP8 SwiGLU entry points (fake, never dereferenced
+    device addresses)."""
+    L = coat.lib()
+    ok = lambda **k: coat.Fp8Act(k.get("q", A), k.get("s", A), k.get("k", A), k.get("ldq", 256),
+                                 k.get("lds", 2))
+    fwd = lambda g=None, u=None, o=None, rows=4, cols=256, fmt=0, ex=0: L.coat_swiglu_fp8_forward(
+        ctypes.byref(g or ok()), ctypes.byref(u or ok()), rows, cols, fmt, ex,
+        ctypes.byref(o or ok()), None)
+    assert fwd(rows=-1) == INVALID
+    assert fwd(cols=250) == UNSUPPORTED and "multiple of 16" in coat.coat_last_error()
+    assert fwd(fmt=3) == INVALID
+    assert fwd(ex=2) == INVALID
+    assert fwd(g=ok(q=None)) == INVALID and "gate" in coat.coat_last_error()
+    assert fwd(u=ok(q=A + 8)) == MISALIGNED and "up" in coat.coat_last_error()
+    assert fwd(o=ok(ldq=264)) == MISALIGNED and "out" in coat.coat_last_error()
+    assert fwd(o=ok(s=A + 2)) == MISALIGNED
+    assert fwd(g=ok(lds=1)) == INVALID and "strides" in coat.coat_last_error()
+    assert fwd(g=ok(ldq=128)) == INVALID
+    assert L.coat_swiglu_fp8_forward(None, ctypes.byref(ok()), 4, 256, 0, 0, ctypes.byref(ok()),
+                                     None) == INVALID
+    assert fwd(rows=0) == OK and fwd(cols=0) == OK
+    bwd = lambda d=A, ldd=256, dg=A, ldg=256, du=A, ldu=256, cols=256: \
+        L.coat_swiglu_fp8_backward(d, ldd, ctypes.byref(ok()), ctypes.byref(ok()), 4, cols, 0,
+                                   dg, ldg, du, ldu, None)
+    assert bwd(d=None) == INVALID and "grad_out" in coat.coat_last_error()
+    assert bwd(dg=A + 2) == MISALIGNED and "grad_gate" in coat.coat_last_error()
+    assert bwd(ldu=260) == MISALIGNED and "grad_up" in coat.coat_last_error()
+    assert bwd(ldd=100) == INVALID
+    assert bwd(cols=40) == UNSUPPORTED
+
+
 def test_selftest_budget_validation():
     L = coat.lib()
     assert L.coat_selftest_wait_timeout(999, None) == INVALID
