@@ -286,6 +286,7 @@ coat_status coat_swiglu_fp8_forward(const coat_fp8_act* gate, const coat_fp8_act
   if (expand_out != 0 && expand_out != 1)
     return fail(COAT_ERR_INVALID_ARG, "%s: expand_out must be 0 or 1", fn);
   if (cols % 16 != 0) return fail(COAT_ERR_UNSUPPORTED, "%s: cols must be a multiple of 16", fn);
+  if (cols > (int64_t(1) << 30)) return fail(COAT_ERR_UNSUPPORTED, "%s: cols above 2^30", fn);
   coat_status st = check_act(fn, "gate", gate, rows, cols);
   if (st == COAT_OK) st = check_act(fn, "up", up, rows, cols);
   if (st == COAT_OK) st = check_act(fn, "out", out, rows, cols);

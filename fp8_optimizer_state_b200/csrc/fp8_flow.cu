@@ -17,13 +17,14 @@
 //    16 contiguous columns per lane, 4 groups per warp and work item, the
 //    next item's codes and metadata loaded before the current one is
 //    computed; group statistics by 3 xor-shuffles; the quantiser arithmetic
-//    is the codec's (correctly rounded division when k = 1, the expansion
-//    otherwise, software RNE encoder, the NaN/Inf slow path);
+//    is the codec's (the expansion, the software RNE encoder, the NaN/Inf
+//    slow path), with k = 1 groups scaled by one multiply;
 //  * backward (8.06 B per element: dh in, two codes in, two bf16 out, group
 //    metadata): one thread per 16 contiguous columns, no cross-lane work.
 // Dequantisation of a k = 1 group (no expansion, the usual activation case)
-// converts code pairs exactly to f16 with the hardware FP8 conversion and
-// multiplies by the scale; other groups use a 256-entry log2 table and ex2.
+// converts code pairs exactly to f16 with the hardware FP8 conversion (and
+// the forward folds both scales into one product per group); other groups
+// use a 256-entry log2 table and ex2.
 // The sigmoid is 1 / (1 + 2^(-g log2 e)) with the approximate ex2 and
 // reciprocal (relative error a few 2^-23); results below FP32's normal range
 // flush to 0.
@@ -84,21 +85,76 @@ __device__ __forceinline__ void decode16(const uint4& w, float s, float k, const
   }
 }
 
+// max(a, b) that returns NaN when either is NaN.
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
 // sigmoid(g) = 1 / (1 + e^-g); 0 once the result is below 2^-126 (the
 // reciprocal flushes), 1 for large g.
 __device__ __forceinline__ float sigmoid(float g) {
   return rcp_approx(1.0f + ex2_approx(g * -1.4426950408889634f));
 }
 
-// One lane's forward work item: 16 gate and 16 up codes and their groups' metadata.
+// |q|^(1/k) with the code's sign for the 16 codes of one lane (the group's
+// scale is applied by the caller).  plain: every group of the warp has k = 1,
+// so the values are the FP8 values themselves, converted exactly.
+template <int FMT>
+__device__ __forceinline__ void decode16_raw(const uint4& w, float k, bool plain,
+                                             const float* tab, float (&f)[16]) {
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+  if (plain) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 a = f16x2_to_float2(fp8x2_to_f16x2<FMT>(ws[j]));
+      const float2 b = f16x2_to_float2(fp8x2_to_f16x2<FMT>(ws[j] >> 16));
+      f[4 * j] = a.x;
+      f[4 * j + 1] = a.y;
+      f[4 * j + 2] = b.x;
+      f[4 * j + 3] = b.y;
+    }
+  } else if (k == 1.0f) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      f[i] = dec_value<FMT>(__byte_perm(ws[i >> 2], 0u, 0x4440u + (i & 3)));
+  } else {
+    const float invk = rcp_approx(k);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t wd = ws[i >> 2];
+      const uint32_t c = __byte_perm(wd, 0u, 0x4440u + (i & 3));
+      const float a = ex2_approx(tab[c] * invk);
+      f[i] = __uint_as_float(__float_as_uint(a) ^ ((wd << (24 - 8 * (i & 3))) & 0x80000000u));
+    }
+  }
+}
+
+// One lane's forward work item: 16 gate and 16 up codes, their groups'
+// metadata, and the item's row and the lane's first column.
 struct FwdItem {
   uint4 gw, uw;
   float gs, gk, us, uk;
+  int64_t r;
+  int32_t c;
+  bool valid;   // the lane's 16 columns exist
 };
 
-template <int FMT>
+// h = silu(g) u with g = f_g s_g, u = f_u s_u, as ((f_g f_u) sigmoid(g)) (s_g s_u):
+// f_g f_u is exact for k = 1 inputs (two FP8 significands), so h takes two
+// roundings besides the sigmoid's.  The output codes: k = 1 groups encode
+// FMT_MAX |h| / M as |h| (FMT_MAX / M) (a few ulps from the correctly rounded
+// quotient, which only decides codes at exact ties of the real-number result;
+// at most FMT_MAX (1 + 2^-21), inside the bounded encoder's range) with root
+// scale M / FMT_MAX; expanded groups use the codec's expansion.  EXPAND:
+// output expansion on.
+// Work: the rows x ceil(groups/4) items (4 groups of a row, 8 lanes each) in
+// row-major order, a contiguous range per warp (columns advanced by 512 with
+// a row carry); the next item is loaded before the current one is computed.
+template <int FMT, bool EXPAND>
 __global__ void __launch_bounds__(256) swiglu_fwd_kernel(const ActArgs gate, const ActArgs up,
-                                                         int64_t rows, int64_t cols, int expand,
+                                                         int64_t rows, int64_t cols,
                                                          const ActArgs out) {
   __shared__ float tab[256];
   fill_log2_table<FMT>(tab);
@@ -106,80 +162,125 @@ __global__ void __launch_bounds__(256) swiglu_fwd_kernel(const ActArgs gate, con
   const int lane = threadIdx.x & 31, slot = lane >> 3, l = lane & 7;
   const int64_t nbc = (cols + kGroup - 1) / kGroup;   // groups per row
   const int64_t nq = (nbc + 3) / 4;                    // quads per row
-  const int64_t w0 = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5;
+  const int64_t nitems = rows * nq;
+  const int64_t wid = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5;
   const int64_t nw = (int64_t(gridDim.x) * blockDim.x) >> 5;
-  const int64_t dr = nw / nq, dq = nw % nq;            // stride in (rows, quads)
-  int64_t r = w0 / nq, gq = w0 % nq;
-  // cols is a multiple of 16, so a lane's 16 columns are all valid or all absent
-  auto fetch = [&](int64_t rr, int64_t qq, FwdItem& it, bool& valid) {
-    const int64_t g = qq * 4 + slot;
-    const int64_t c = g * kGroup + 16 * l;
-    valid = rr < rows && g < nbc && c < cols;
-    if (valid) {
-      it.gw = __ldg(reinterpret_cast<const uint4*>(gate.q + rr * gate.ldq + c));
-      it.uw = __ldg(reinterpret_cast<const uint4*>(up.q + rr * up.ldq + c));
-      it.gs = __ldg(gate.scale + rr * gate.lds + g);
-      it.gk = __ldg(gate.k + rr * gate.lds + g);
-      it.us = __ldg(up.scale + rr * up.lds + g);
-      it.uk = __ldg(up.k + rr * up.lds + g);
+  const int64_t i0 = wid * nitems / nw, i1 = (wid + 1) * nitems / nw;
+  if (i0 >= i1) return;
+  const int lc = slot * kGroup + 16 * l;   // the lane's column within an item
+  int64_t cr = i0 / nq;                     // row and lane column of the next item to load
+  int32_t cc = static_cast<int32_t>((i0 - cr * nq) * 4 * kGroup) + lc;
+  const int32_t rowspan = static_cast<int32_t>(nq * 4 * kGroup);
+  auto load = [&](FwdItem& it) {
+    it.r = cr;
+    it.c = cc;
+    it.valid = cc < cols;
+    const int32_t g = cc >> 7;
+    if (it.valid) {
+      it.gw = __ldg(reinterpret_cast<const uint4*>(gate.q + cr * gate.ldq + cc));
+      it.uw = __ldg(reinterpret_cast<const uint4*>(up.q + cr * up.ldq + cc));
+      it.gs = __ldg(gate.scale + cr * gate.lds + g);
+      it.gk = __ldg(gate.k + cr * gate.lds + g);
+      it.us = __ldg(up.scale + cr * up.lds + g);
+      it.uk = __ldg(up.k + cr * up.lds + g);
     } else {
       it.gw = it.uw = make_uint4(0u, 0u, 0u, 0u);
       it.gs = it.gk = it.us = it.uk = 1.0f;
     }
+    cc += 4 * kGroup;
+    if (cc >= rowspan) { cc -= rowspan; ++cr; }
   };
   FwdItem cur;
-  bool valid = false;
-  if (r < rows) fetch(r, gq, cur, valid);
-  while (r < rows) {
-    int64_t rn = r + dr, qn = gq + dq;
-    if (qn >= nq) { qn -= nq; ++rn; }
+  load(cur);
+  for (int64_t item = i0; item < i1; ++item) {
     FwdItem nxt;
-    bool validn = false;
-    if (rn < rows) fetch(rn, qn, nxt, validn);
+    if (item + 1 < i1) load(nxt);
 
-    float g[16], u[16], h[16];
-    decode16<FMT>(cur.gw, cur.gs, cur.gk, tab, g);
-    decode16<FMT>(cur.uw, cur.us, cur.uk, tab, u);
+    const bool plain = __all_sync(0xFFFFFFFFu, cur.gk == 1.0f && cur.uk == 1.0f);
+    float fg[16], fu[16], h[16];
+    decode16_raw<FMT>(cur.gw, cur.gk, plain, tab, fg);
+    decode16_raw<FMT>(cur.uw, cur.uk, plain, tab, fu);
+    const float ct = cur.gs * -1.4426950408889634f;   // -log2(e) s_g
+    const float S = cur.gs * cur.us;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) h[i] = (g[i] * sigmoid(g[i])) * u[i];
+    for (int i = 0; i < 16; ++i) {
+      const float sg = rcp_approx(1.0f + ex2_approx(fg[i] * ct));
+      h[i] = ((fg[i] * fu[i]) * sg) * S;
+    }
 
-    uint32_t maxb = 0u, mink = 0xFFFFFFFFu;
-    stats_bits(h, maxb, mink);
+    // group max |h| (NaN-propagating, so that one test finds NaN and Inf) and,
+    // with expansion, min nonzero |h| on twice the bit patterns (zero becomes
+    // the largest key)
+    float mx = 0.0f;
+    uint32_t mink = 0xFFFFFFFFu;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      mx = fmax_nan(mx, fabsf(h[i]));
+      if (EXPAND) mink = min(mink, __float_as_uint(h[i]) * 2u - 2u);
+    }
 #pragma unroll
     for (int off = 1; off < 8; off <<= 1) {
-      maxb = max(maxb, __shfl_xor_sync(0xFFFFFFFFu, maxb, off));
-      mink = min(mink, __shfl_xor_sync(0xFFFFFFFFu, mink, off));
+      mx = fmax_nan(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+      if (EXPAND) mink = min(mink, __shfl_xor_sync(0xFFFFFFFFu, mink, off));
     }
-    const bool special = maxb >= 0xFF000000u;   // an Inf or a NaN in the group
-    float M = __uint_as_float(maxb >> 1);
-    if (__any_sync(0xFFFFFFFFu, special)) {
+    // slow path: an Inf or a NaN in the group, a scale product that overflowed,
+    // or a maximum so small that 1/M would leave FP32 (below 2^-64)
+    const bool special = !(mx <= 3.40282347e38f) || !(S <= 3.40282347e38f) ||
+                         (mx > 0.0f && mx < 5.421010862427522e-20f);
+    uint32_t cw[4];
+    float k, sr;
+    if (!__any_sync(0xFFFFFFFFu, special)) {
+      const float M = mx;
+      float invM;
+      if (EXPAND) {
+        group_params<FMT>(M, __uint_as_float((mink + 2u) >> 1), true, k, sr, invM);
+      } else {
+        k = 1.0f;
+        sr = M > 0.0f ? M * (1.0f / F8<FMT>::MAXV) : 1.0f;
+        invM = M > 0.0f ? rcp_approx(M) : 0.0f;   // an all-zero group encodes to zeros
+      }
+      uint32_t mag[16];
+      if (k == 1.0f) {
+        const float c = F8<FMT>::MAXV * invM;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) mag[i] = enc_mag_bounded<FMT>(fabsf(h[i]) * c);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) mag[i] = enc_mag_bounded<FMT>(expand_value<FMT>(h[i], invM, k));
+      }
+#pragma unroll
+      for (int w = 0; w < 4; ++w)
+        cw[w] = merge_signs4(pack4(mag[4 * w], mag[4 * w + 1], mag[4 * w + 2], mag[4 * w + 3]),
+                             h[4 * w], h[4 * w + 1], h[4 * w + 2], h[4 * w + 3]);
+    } else {
+      // the codec's slow path: the maximum ignores NaN, IEEE division for k = 1
       float Mn = max_abs_nonnan(h);
 #pragma unroll
       for (int off = 1; off < 8; off <<= 1) Mn = fmaxf(Mn, __shfl_xor_sync(0xFFFFFFFFu, Mn, off));
-      if (special) M = Mn;
+      uint32_t mk2 = 0xFFFFFFFFu;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) mk2 = min(mk2, __float_as_uint(h[i]) * 2u - 2u);
+#pragma unroll
+      for (int off = 1; off < 8; off <<= 1) mk2 = min(mk2, __shfl_xor_sync(0xFFFFFFFFu, mk2, off));
+      const float M = special ? Mn : mx;
+      float invM;
+      group_params<FMT>(M, __uint_as_float((mk2 + 2u) >> 1), EXPAND, k, sr, invM);
+      const bool use_div = k == 1.0f;
+      GroupDiv d{};
+      if (use_div) d = codec_div<FMT>(M);
+      if (special)
+        encode_words<FMT, 16, false>(h, use_div, d, invM, k, cw);
+      else
+        encode_words<FMT, 16, true>(h, use_div, d, invM, k, cw);
     }
-    float k, sr, invM;
-    group_params<FMT>(M, __uint_as_float((mink + 2u) >> 1), expand != 0, k, sr, invM);
-    const bool use_div = k == 1.0f;
-    GroupDiv d{};
-    if (use_div) d = codec_div<FMT>(M);
-    uint32_t cw[4];
-    if (!special)
-      encode_words<FMT, 16, true>(h, use_div, d, invM, k, cw);
-    else
-      encode_words<FMT, 16, false>(h, use_div, d, invM, k, cw);
-    const int64_t grp = gq * 4 + slot;
-    if (valid)
-      *reinterpret_cast<uint4*>(out.q + r * out.ldq + grp * kGroup + 16 * l) =
-          make_uint4(cw[0], cw[1], cw[2], cw[3]);
-    if (l == 0 && grp < nbc) {
-      out.scale[r * out.lds + grp] = sr;
-      out.k[r * out.lds + grp] = k;
+    if (cur.valid) {
+      *reinterpret_cast<uint4*>(out.q + cur.r * out.ldq + cur.c) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      if (l == 0) {
+        out.scale[cur.r * out.lds + (cur.c >> 7)] = sr;
+        out.k[cur.r * out.lds + (cur.c >> 7)] = k;
+      }
     }
-    r = rn;
-    gq = qn;
     cur = nxt;
-    valid = validn;
   }
 }
 
@@ -262,10 +363,10 @@ __global__ void __launch_bounds__(256) swiglu_bwd_kernel(const uint16_t* __restr
 template <int FMT>
 void fwd_launch(const ActArgs& gate, const ActArgs& up, int64_t rows, int64_t cols, int expand,
                 const ActArgs& out, int dev, cudaStream_t s) {
-  auto kern = swiglu_fwd_kernel<FMT>;
+  auto kern = expand ? swiglu_fwd_kernel<FMT, true> : swiglu_fwd_kernel<FMT, false>;
   const int64_t quads = rows * (((cols + 127) / 128 + 3) / 4);
   const unsigned g = grid_for(quads, 8, dev, resident_ctas(reinterpret_cast<const void*>(kern)));
-  kern<<<g, 256, 0, s>>>(gate, up, rows, cols, expand, out);
+  kern<<<g, 256, 0, s>>>(gate, up, rows, cols, out);
 }
 
 template <int FMT>

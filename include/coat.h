@@ -299,8 +299,9 @@ coat_status coat_adamw_step_multi_noalloc(const coat_tensor_desc *host_descs, in
  *   grad_up   = grad_out silu(g),
  *   grad_gate = grad_out u sigmoid(g) (1 + g (1 - sigmoid(g))),
  * computed in FP32 and rounded to bf16 (nearest even).
- * Requirements: rows, cols >= 0 (0 is a no-op); cols a multiple of 16
- * (COAT_ERR_UNSUPPORTED otherwise; the last group may be partial); every code
+ * Requirements: rows, cols >= 0 (0 is a no-op); cols a multiple of 16, and
+ * at most 2^30 for the forward (COAT_ERR_UNSUPPORTED otherwise; the last group
+ * may be partial); every code
  * and bf16 array 16-byte aligned with row strides that are multiples of 16
  * bytes (ldq >= cols; bf16 strides >= cols); scale / k 4-byte aligned with
  * lds >= ceil(cols/128); fmt the format of all three tensors.

@@ -33,11 +33,13 @@ ULP_FRACTION = 2e-3     # device sigmoid / product error (~1e-6 rel) against the
 
 
 def make_inputs(orc, rows, cols, fmt, expand_in, seed):
+    """expand_in: one flag for both inputs, or a (gate, up) pair."""
+    flags = expand_in if isinstance(expand_in, tuple) else (expand_in, expand_in)
     acts = []
     for t in (0, 1):
         bits = synth.activations_bits(seed, t, 0, rows * cols).reshape(rows, cols)
         x = synth.bf16_bits_to_f32(bits).astype(np.float64)
-        acts.append(orc.group_quantize(x, 1, 128, expand_in, fmt))
+        acts.append(orc.group_quantize(x, 1, 128, flags[t], fmt))
     return acts
 
 
@@ -140,6 +142,7 @@ def forward_case(orc, rows, cols, fmt, expand_in, expand_out, seed=1):
     (64, 1024, E4M3, False, False),       # the usual case: no expansion anywhere
     (33, 11008, E4M3, False, False),      # a Llama-2-7B MLP width (86 groups), ragged quads
     (40, 1024, E4M3, True, True),         # expanded inputs (table decode) and output
+    (24, 1024, E4M3, (False, True), False),   # k = 1 gate beside expanded up in one warp
     (17, 304, E5M2, False, False),        # E5M2; a partial last group of 48
     (9, 304, E5M2_FULL, False, True),
     (5, 16, E4M3, False, True),           # one partial group per row
@@ -223,6 +226,7 @@ def backward_case(orc, rows, cols, fmt, expand_in, seed=2):
     (64, 1024, E4M3, False),
     (33, 11008, E4M3, False),
     (40, 1024, E4M3, True),
+    (24, 1024, E4M3, (False, True)),
     (17, 304, E5M2, False),
     (3, 16, E4M3, False),
 ])
