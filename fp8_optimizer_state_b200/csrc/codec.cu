@@ -106,64 +106,98 @@ __device__ __forceinline__ void unpack16(const Raw16<DT>& r, float v[16]) {
 
 // ---------------------------------------------------------------------------
 // 1 x 128 groups: 8 lanes per group, 16 contiguous elements per lane, 4 groups
-// (one quad) per warp and work item.  Items (row, quad) are walked row-major
-// with a fixed stride per warp, advanced without divisions; the next item's
-// elements are loaded before the current one is computed.
+// (one quad) per warp and work item.  The rows x quads items are taken in
+// row-major order, a contiguous range per warp, with the lane's column
+// advanced by 512 and a row carry; the next item's elements are loaded before
+// the current one is computed.  EXPAND (a template parameter): without
+// expansion the group statistics are one NaN-propagating max per element (one
+// test then finds NaN and Inf); with it, max and min-nonzero on the bit
+// patterns.
 // ---------------------------------------------------------------------------
-template <int FMT, int DT>
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+template <int DT>
+struct RowItem {
+  Raw16<DT> raw;
+  int64_t r, c;   // row and the lane's first column
+  int valid;      // elements of the lane's 16 that exist
+};
+
+template <int FMT, int DT, bool EXPAND>
 __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__ x, int64_t rows,
-                                                        int64_t cols, int64_t ldx, int expand,
+                                                        int64_t cols, int64_t ldx,
                                                         uint8_t* __restrict__ q, int64_t ldq,
                                                         float* __restrict__ scale,
                                                         float* __restrict__ kk) {
   const int lane = threadIdx.x & 31, slot = lane >> 3, l = lane & 7;
   const int64_t nbc = (cols + kGroup - 1) / kGroup;   // groups per row
   const int64_t nq = (nbc + 3) / 4;                    // quads per row
-  const int64_t w0 = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5;
+  const int64_t nitems = rows * nq;
+  const int64_t wid = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5;
   const int64_t nw = (int64_t(gridDim.x) * blockDim.x) >> 5;
-  const int64_t dr = nw / nq, dq = nw % nq;            // stride in (rows, quads)
-  int64_t r = w0 / nq, gq = w0 % nq;
+  const int64_t i0 = wid * nitems / nw, i1 = (wid + 1) * nitems / nw;
+  if (i0 >= i1) return;
   const size_t esz = DT == 0 ? 4 : 2;
-  auto where = [&](int64_t rr, int64_t qq, int64_t& c, int& valid) {
-    const int64_t g = qq * 4 + slot;
-    c = g * kGroup + 16 * l;
-    valid = (rr < rows && g < nbc) ? clamp_valid(cols - c, 16) : 0;
+  const int64_t rowspan = nq * 4 * kGroup;
+  int64_t cr = i0 / nq;                                  // the next item to load
+  int64_t cc = (i0 - cr * nq) * 4 * kGroup + slot * kGroup + 16 * l;
+  auto load = [&](RowItem<DT>& it) {
+    it.r = cr;
+    it.c = cc;
+    it.valid = clamp_valid(cols - cc, 16);
+    load16<DT>(static_cast<const char*>(x) + cr * ldx * esz, cc, it.valid, it.raw);
+    cc += 4 * kGroup;
+    if (cc >= rowspan) { cc -= rowspan; ++cr; }
   };
-  int64_t c;
-  int valid;
-  Raw16<DT> cur;
-  where(r, gq, c, valid);
-  if (r < rows) load16<DT>(static_cast<const char*>(x) + r * ldx * esz, c, valid, cur);
-  while (r < rows) {
-    // next item
-    int64_t rn = r + dr, qn = gq + dq;
-    if (qn >= nq) { qn -= nq; ++rn; }
-    int64_t cn;
-    int validn;
-    where(rn, qn, cn, validn);
-    Raw16<DT> nxt;
-    if (rn < rows) load16<DT>(static_cast<const char*>(x) + rn * ldx * esz, cn, validn, nxt);
+  RowItem<DT> cur;
+  load(cur);
+  for (int64_t item = i0; item < i1; ++item) {
+    RowItem<DT> nxt;
+    if (item + 1 < i1) load(nxt);
 
     float v[16];
-    unpack16<DT>(cur, v);
-    uint32_t maxb = 0u, mink = 0xFFFFFFFFu;
-    stats_bits(v, maxb, mink);
+    unpack16<DT>(cur.raw, v);
+    float M, mu = 0.0f;
+    bool special;
+    if (EXPAND) {
+      uint32_t maxb = 0u, mink = 0xFFFFFFFFu;
+      stats_bits(v, maxb, mink);
 #pragma unroll
-    for (int off = 1; off < 8; off <<= 1) {
-      maxb = max(maxb, __shfl_xor_sync(0xFFFFFFFFu, maxb, off));
-      mink = min(mink, __shfl_xor_sync(0xFFFFFFFFu, mink, off));
+      for (int off = 1; off < 8; off <<= 1) {
+        maxb = max(maxb, __shfl_xor_sync(0xFFFFFFFFu, maxb, off));
+        mink = min(mink, __shfl_xor_sync(0xFFFFFFFFu, mink, off));
+      }
+      special = maxb >= 0xFF000000u;   // an Inf or a NaN in the group
+      M = __uint_as_float(maxb >> 1);
+      mu = __uint_as_float((mink + 2u) >> 1);
+    } else {
+      float mx = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) mx = fmax_nan(mx, fabsf(v[i]));
+#pragma unroll
+      for (int off = 1; off < 8; off <<= 1) mx = fmax_nan(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+      special = !(mx <= 3.40282347e38f);   // NaN or Inf
+      M = mx;
     }
-    const bool special = maxb >= 0xFF000000u;   // an Inf or a NaN in the group
-    float M = __uint_as_float(maxb >> 1);
     if (__any_sync(0xFFFFFFFFu, special)) {
       float Mn = max_abs_nonnan(v);
 #pragma unroll
       for (int off = 1; off < 8; off <<= 1) Mn = fmaxf(Mn, __shfl_xor_sync(0xFFFFFFFFu, Mn, off));
       if (special) M = Mn;
     }
-    float k, sr, invM;
-    group_params<FMT>(M, __uint_as_float((mink + 2u) >> 1), expand != 0, k, sr, invM);
-    const bool use_div = k == 1.0f;
+    float k, sr, invM = 0.0f;
+    if (EXPAND) {
+      group_params<FMT>(M, mu, true, k, sr, invM);
+    } else {
+      // k = 1: the root scale is M / FMT_MAX, correctly rounded (1 for an all-zero group)
+      k = 1.0f;
+      sr = M > 0.0f ? __fdiv_rn(M, F8<FMT>::MAXV) : 1.0f;
+    }
+    const bool use_div = !EXPAND || k == 1.0f;
     GroupDiv d{};
     if (use_div) d = codec_div<FMT>(M);
     uint32_t cw[4];
@@ -171,16 +205,13 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
       encode_words<FMT, 16, true>(v, use_div, d, invM, k, cw);
     else
       encode_words<FMT, 16, false>(v, use_div, d, invM, k, cw);
-    if (valid > 0) store16(q + r * ldq + c, cw, valid);
-    const int64_t g = gq * 4 + slot;
-    if (l == 0 && g < nbc) {
-      scale[r * nbc + g] = sr;
-      kk[r * nbc + g] = k;
+    if (cur.valid > 0) store16(q + cur.r * ldq + cur.c, cw, cur.valid);
+    // lane 0 of a group holds its first column, so it exists exactly when the group does
+    if (l == 0 && cur.valid > 0) {
+      const int64_t g = cur.r * nbc + (cur.c >> 7);
+      scale[g] = sr;
+      kk[g] = k;
     }
-    r = rn;
-    gq = qn;
-    c = cn;
-    valid = validn;
     cur = nxt;
   }
 }
@@ -250,9 +281,9 @@ __device__ __forceinline__ void block_row(const Block8<DT>& B, int i, float v[8]
   }
 }
 
-template <int FMT, int DT>
+template <int FMT, int DT, bool EXPAND>
 __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict__ x, int64_t rows,
-                                                          int64_t cols, int64_t ldx, int expand,
+                                                          int64_t cols, int64_t ldx,
                                                           uint8_t* __restrict__ q, int64_t ldq,
                                                           float* __restrict__ scale,
                                                           float* __restrict__ kk) {
@@ -275,17 +306,48 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
     Block8<DT> nxt;
     if (DT == 1 && bn < nb) load_block<DT>(x, rows, cols, ldx, brn, bcn, warp, lane, nxt);
 
+    // with expansion: max and min-nonzero on twice the bit patterns; without:
+    // the bit pattern of a NaN-propagating max |x| (non-negative floats and
+    // the NaN it returns order like their bit patterns)
     uint32_t maxb = 0u, mink = 0xFFFFFFFFu;
+    if constexpr (EXPAND) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float v[8];
-      block_row<DT>(cur, i, v);
-      stats_bits(v, maxb, mink);
-    }
+      for (int i = 0; i < 8; ++i) {
+        float v[8];
+        block_row<DT>(cur, i, v);
+        stats_bits(v, maxb, mink);
+      }
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      maxb = max(maxb, __shfl_xor_sync(0xFFFFFFFFu, maxb, off));
-      mink = min(mink, __shfl_xor_sync(0xFFFFFFFFu, mink, off));
+      for (int off = 1; off < 32; off <<= 1) {
+        maxb = max(maxb, __shfl_xor_sync(0xFFFFFFFFu, maxb, off));
+        mink = min(mink, __shfl_xor_sync(0xFFFFFFFFu, mink, off));
+      }
+    } else if constexpr (DT == 1) {
+      // bf16: |x| bit patterns compared two at a time (16-bit lanes); NaN
+      // patterns are above Inf's, so the test below still finds both
+      uint32_t m2 = 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint4 u = cur.a[i];
+        m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(u.x & 0x7FFF7FFFu, u.y & 0x7FFF7FFFu),
+                                   __vmaxu2(u.z & 0x7FFF7FFFu, u.w & 0x7FFF7FFFu)));
+      }
+      uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+      maxb = m >= 0x7F80u ? 0x7FFFFFFFu : (m << 16);
+    } else {
+      float mx = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float v[8];
+        block_row<DT>(cur, i, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx = fmax_nan(mx, fabsf(v[e]));
+      }
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) mx = fmax_nan(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+      maxb = __float_as_uint(mx);
     }
     // double-buffered partials: one barrier per block
     if (lane == 0) {
@@ -300,8 +362,9 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
       maxb = max(maxb, sM[par][w]);
       mink = min(mink, sK[par][w]);
     }
-    const bool special = maxb >= 0xFF000000u;   // an Inf or a NaN in the block (CTA-uniform)
-    float M = __uint_as_float(maxb >> 1);
+    // an Inf or a NaN in the block (CTA-uniform)
+    const bool special = EXPAND ? maxb >= 0xFF000000u : maxb >= 0x7F800000u;
+    float M = __uint_as_float(EXPAND ? maxb >> 1 : maxb);
     if (special) {
       // max |x| ignoring NaN, through the other half of the partials buffer
       float Mn = 0.f;
@@ -321,9 +384,15 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
       __syncthreads();   // the partials buffer is free again before the next block writes it
     }
     par ^= 1;
-    float k, sr, invM;
-    group_params<FMT>(M, __uint_as_float((mink + 2u) >> 1), expand != 0, k, sr, invM);
-    const bool use_div = k == 1.0f;
+    float k, sr, invM = 0.0f;
+    if (EXPAND) {
+      group_params<FMT>(M, __uint_as_float((mink + 2u) >> 1), true, k, sr, invM);
+    } else {
+      // k = 1: the root scale is M / FMT_MAX, correctly rounded (1 for an all-zero block)
+      k = 1.0f;
+      sr = M > 0.0f ? __fdiv_rn(M, F8<FMT>::MAXV) : 1.0f;
+    }
+    const bool use_div = !EXPAND || k == 1.0f;
     GroupDiv d{};
     if (use_div) d = codec_div<FMT>(M);
     const int64_t c = bc * 128 + 8 * (lane & 15);
@@ -605,15 +674,15 @@ static cudaError_t quant_dispatch(const void* x, int64_t rows, int64_t cols, int
                                   unsigned* err, int dev, cudaStream_t s) {
   if (gr == 1) {
     const int64_t quads = rows * (((cols + 127) / 128 + 3) / 4);
-    auto kern = quant_row_kernel<FMT, DT>;
+    auto kern = expand ? quant_row_kernel<FMT, DT, true> : quant_row_kernel<FMT, DT, false>;
     const unsigned g =
         grid_for(quads, 8, dev, resident_ctas(reinterpret_cast<const void*>(kern)));
-    kern<<<g, 256, 0, s>>>(x, rows, cols, ldx, expand, q, ldq, scale, k);
+    kern<<<g, 256, 0, s>>>(x, rows, cols, ldx, q, ldq, scale, k);
   } else {
     const int64_t blocks = ((rows + 127) / 128) * ((cols + 127) / 128);
-    auto kern = quant_block_kernel<FMT, DT>;
+    auto kern = expand ? quant_block_kernel<FMT, DT, true> : quant_block_kernel<FMT, DT, false>;
     const unsigned g = grid_for(blocks, 1, dev, resident_ctas(reinterpret_cast<const void*>(kern)));
-    kern<<<g, 256, 0, s>>>(x, rows, cols, ldx, expand, q, ldq, scale, k);
+    kern<<<g, 256, 0, s>>>(x, rows, cols, ldx, q, ldq, scale, k);
   }
   return cudaSuccess;
 }

@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(256) swiglu_fwd_kernel(const ActArgs gate, con
         group_params<FMT>(M, __uint_as_float((mink + 2u) >> 1), true, k, sr, invM);
       } else {
         k = 1.0f;
-        sr = M > 0.0f ? M * (1.0f / F8<FMT>::MAXV) : 1.0f;
+        sr = M > 0.0f ? __fdiv_rn(M, F8<FMT>::MAXV) : 1.0f;   // M / FMT_MAX, correctly rounded
         invM = M > 0.0f ? rcp_approx(M) : 0.0f;   // an all-zero group encodes to zeros
       }
       uint32_t mag[16];

@@ -118,6 +118,11 @@ def test_group_quantize_vs_oracle(orc, gr, gc, rows, cols, fmt, expand, dtype):
     torch.cuda.synchronize()
     _check_quant(q.cpu().numpy()[:, :cols], s.cpu().numpy(), k.cpu().numpy(), oq, os_, ok_, fmt)
     assert not q.cpu().numpy()[:, cols:].any()     # nothing written past cols
+    if not expand:
+        # k = 1: the root scale is M / FMT_MAX correctly rounded on both sides
+        # (the oracle's double product rounds to the same FP32 value except in
+        # double-rounding cases, about one in 2^29)
+        assert np.array_equal(s.cpu().numpy(), os_)
 
 
 @pytest.mark.parametrize("gr", [1, 128])
