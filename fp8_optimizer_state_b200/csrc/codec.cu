@@ -479,8 +479,29 @@ __device__ __forceinline__ const float* lane_log2_table(float* tab1, float* tab)
   return tab + (threadIdx.x & 31);
 }
 
+// 16 values of one group with k = 1: the codes converted exactly (FP8 -> f16 ->
+// f32 in hardware) times the scale, one rounding.
+template <int FMT>
+__device__ __forceinline__ void dequant16_k1(const uint4& w, float s, float (&xv)[16]) {
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 a = f16x2_to_float2(fp8x2_to_f16x2<FMT>(ws[j]));
+    const float2 b = f16x2_to_float2(fp8x2_to_f16x2<FMT>(ws[j] >> 16));
+    xv[4 * j] = a.x * s;
+    xv[4 * j + 1] = a.y * s;
+    xv[4 * j + 2] = b.x * s;
+    xv[4 * j + 3] = b.y * s;
+  }
+}
+
 // Rows whose width is a multiple of 16: every chunk is whole, and the code,
 // output and metadata positions advance with the stride by pointer increments.
+// A thread loads kBatch chunks (its next kBatch positions of the stride walk)
+// before it computes any of them, so that each thread keeps kBatch 16-byte
+// loads in flight.
+constexpr int kBatch = 4;
+
 template <int FMT, int OT, int GR>
 __global__ void __launch_bounds__(256) dequant_full_kernel(const uint8_t* __restrict__ q,
                                                            int64_t ldq,
@@ -498,40 +519,44 @@ __global__ void __launch_bounds__(256) dequant_full_kernel(const uint8_t* __rest
   const int64_t nt = int64_t(gridDim.x) * blockDim.x;
   const int64_t dr = nt / cpr, dc = nt % cpr;
   int64_t r = t0 / cpr, cc = t0 % cpr;
-  if (r >= rows) return;
   // byte steps of the code and output pointers: without / with a row carry
   const int64_t qs = dr * ldq + 16 * dc, qsc = qs + ldq - 16 * cpr;
   const int64_t os = (dr * ldo + 16 * dc) * kOsz, osc = os + (ldo - 16 * cpr) * kOsz;
   const uint8_t* qp = q + r * ldq + 16 * cc;
   char* op = static_cast<char*>(out) + (r * ldo + 16 * cc) * kOsz;
-  auto group = [&](int64_t rr, int64_t ch) { return (GR == 1 ? rr : rr / GR) * nbc + (ch >> 3); };
-  uint4 w = __ldg(reinterpret_cast<const uint4*>(qp));
-  int64_t g = group(r, cc);
-  float s = __ldg(scale + g), kv = __ldg(kk + g);
-  while (true) {
-    int64_t rn = r + dr, cn = cc + dc;
-    const bool carry = cn >= cpr;
-    if (carry) { cn -= cpr; ++rn; }
-    const uint8_t* qpn = qp + (carry ? qsc : qs);
-    uint4 wn;
-    float sn, kn;
-    if (rn < rows) {
-      wn = __ldg(reinterpret_cast<const uint4*>(qpn));
-      const int64_t gn = group(rn, cn);
-      sn = __ldg(scale + gn);
-      kn = __ldg(kk + gn);
+  while (r < rows) {
+    uint4 w[kBatch];
+    float s[kBatch], kv[kBatch];
+    char* o[kBatch];
+    bool ok[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      ok[j] = r < rows;
+      if (ok[j]) {
+        w[j] = __ldg(reinterpret_cast<const uint4*>(qp));
+        const int64_t g = (GR == 1 ? r : r / GR) * nbc + (cc >> 3);
+        s[j] = __ldg(scale + g);
+        kv[j] = __ldg(kk + g);
+        o[j] = op;
+        int64_t cn = cc + dc;
+        const bool carry = cn >= cpr;
+        if (carry) cn -= cpr;
+        r += dr + (carry ? 1 : 0);
+        cc = cn;
+        qp += carry ? qsc : qs;
+        op += carry ? osc : os;
+      }
     }
-    float xv[16];
-    dequant16(w, tabl, rcp_approx(kv), s, xv);
-    store_out16<OT>(op, xv);
-    if (rn >= rows) break;
-    op += carry ? osc : os;
-    qp = qpn;
-    r = rn;
-    cc = cn;
-    w = wn;
-    s = sn;
-    kv = kn;
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      if (!ok[j]) break;
+      float xv[16];
+      if (kv[j] == 1.0f)
+        dequant16_k1<FMT>(w[j], s[j], xv);
+      else
+        dequant16(w[j], tabl, rcp_approx(kv[j]), s[j], xv);
+      store_out16<OT>(o[j], xv);
+    }
   }
 }
 

@@ -37,27 +37,6 @@
 namespace coat {
 namespace {
 
-// Two FP8 codes (low byte first) to two f16 values packed in a word: exact.
-template <int FMT>
-__device__ __forceinline__ uint32_t fp8x2_to_f16x2(uint32_t pair) {
-  uint32_t h;
-  const uint16_t p = static_cast<uint16_t>(pair);
-  if (FMT == kE4M3)
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(p));
-  else
-    asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h) : "h"(p));
-  return h;
-}
-
-__device__ __forceinline__ float2 f16x2_to_float2(uint32_t h) {
-  float a, b;
-  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
-      "cvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
-      : "=f"(a), "=f"(b)
-      : "r"(h));
-  return make_float2(a, b);
-}
-
 // The 16 values x = sign(q) s |q|^(1/k) of one lane's codes (all in one group).
 template <int FMT>
 __device__ __forceinline__ void decode16(const uint4& w, float s, float k, const float* tab,
