@@ -605,7 +605,10 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
     if (rn < rows) fetch(rn, cn, wn, sn, kn, validn);
 
     float xv[16];
-    dequant16(w, tabl, rcp_approx(kv), s, xv);
+    if (kv == 1.0f)
+      dequant16_k1<FMT>(w, s, xv);
+    else
+      dequant16(w, tabl, rcp_approx(kv), s, xv);
     const int64_t c0 = cc * 16;
     if (OT == 0) {
       float* o = static_cast<float*>(out) + r * ldo + c0;

@@ -181,27 +181,36 @@ def test_group_quantize_special_values(orc, gr, fmt, expand):
 
 @pytest.mark.parametrize("gr", [1, 128])
 @pytest.mark.parametrize("fmt", [E4M3, E5M2, E5M2_FULL])
-def test_group_dequantize_vs_oracle(orc, gr, fmt):
-    rows, cols = 256, 640
+@pytest.mark.parametrize("rows,cols", [(256, 640), (100, 650)])
+def test_group_dequantize_vs_oracle(orc, gr, fmt, rows, cols):
+    """cols = 650: rows that are not a multiple of 16 wide (the ragged kernel),
+    strided buffers, a partial 128x128 block."""
     rng = np.random.default_rng(30 + gr + fmt)
     top = 0x7E if fmt == E4M3 else 0x7B
     q = rng.integers(0, top + 1, (rows, cols)).astype(np.uint8) | \
         rng.choice([0, 0x80], (rows, cols)).astype(np.uint8)
     nbr, nbc = -(-rows // gr), -(-cols // 128)
     k = rng.uniform(1.0, 16.0, (nbr, nbc)).astype(np.float32)
-    k[0, 0] = 1.0
+    k[:, ::2] = 1.0                  # k = 1 groups beside expanded ones (the exact decode)
     s = np.exp(rng.uniform(-25, 0, (nbr, nbc))).astype(np.float32)
     ref = orc.group_dequantize(q, s, k, gr, 128, fmt)
-    out = torch.empty((rows, cols), dtype=torch.float32, device="cuda")
-    coat.coat_group_dequantize(torch.from_numpy(q).cuda(), torch.from_numpy(s).cuda(),
-                               torch.from_numpy(k).cuda(), gr, 128, fmt, out)
+    ld = -(-cols // 16) * 16           # row strides that are multiples of 16 bytes
+    qd = torch.zeros((rows, ld), dtype=torch.uint8, device="cuda")
+    qd[:, :cols] = torch.from_numpy(q).cuda()
+    qd = qd[:, :cols]
+    out = torch.zeros((rows, ld), dtype=torch.float32, device="cuda")[:, :cols]
+    coat.coat_group_dequantize(qd, torch.from_numpy(s).cuda(), torch.from_numpy(k).cuda(), gr,
+                               128, fmt, out)
     got = out.cpu().numpy().astype(np.float64)
     # x = s * 2^(log2|q| / k): FP32 exponent arithmetic and MUFU ex2 give a few
     # 1e-7 relative (the argument reaches |log2 q| <= 16 at k = 1)
     assert np.all(np.sign(got) == np.sign(ref))
     assert rel_err(got[ref != 0], ref[ref != 0]).max() < 2e-6
-    outb = torch.empty((rows, cols), dtype=torch.bfloat16, device="cuda")
-    coat.coat_group_dequantize(torch.from_numpy(q).cuda(), torch.from_numpy(s).cuda(),
-                               torch.from_numpy(k).cuda(), gr, 128, fmt, outb)
+    # k = 1: s * value(q) with one rounding, equal to the oracle's exact product rounded
+    k1 = np.repeat(np.repeat(k == 1.0, gr, axis=0), 128, axis=1)[:rows, :cols]
+    assert np.array_equal(got[k1], ref[k1].astype(np.float32).astype(np.float64))
+    outb = torch.zeros((rows, ld), dtype=torch.bfloat16, device="cuda")[:, :cols]
+    coat.coat_group_dequantize(qd, torch.from_numpy(s).cuda(), torch.from_numpy(k).cuda(), gr,
+                               128, fmt, outb)
     gb = outb.float().cpu().numpy()
     assert np.array_equal(gb, torch.from_numpy(got.astype(np.float32)).bfloat16().float().numpy())
