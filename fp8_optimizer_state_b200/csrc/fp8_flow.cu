@@ -12,14 +12,14 @@
 //   dup = dh silu(g),  dgate = dh u sigmoid(g) (1 + g (1 - sigmoid(g))).
 //
 // Both kernels stream HBM (no tensor cores: nothing here is a contraction):
-//  * forward (3.06 algorithmic bytes per element: two codes in, one code out,
+//  * forward (3.19 algorithmic bytes per element: two codes in, one code out,
 //    24 B of group metadata per 128 elements): 8 lanes per 128-column group,
 //    16 contiguous columns per lane, 4 groups per warp and work item, the
 //    next item's codes and metadata loaded before the current one is
 //    computed; group statistics by 3 xor-shuffles; the quantiser arithmetic
 //    is the codec's (the expansion, the software RNE encoder, the NaN/Inf
 //    slow path), with k = 1 groups scaled by one multiply;
-//  * backward (8.06 B per element: dh in, two codes in, two bf16 out, group
+//  * backward (8.13 B per element: dh in, two codes in, two bf16 out, group
 //    metadata): one thread per 16 contiguous columns, no cross-lane work.
 // Dequantisation of a k = 1 group (no expansion, the usual activation case)
 // converts code pairs exactly to f16 with the hardware FP8 conversion (and
