@@ -107,6 +107,15 @@ def lib():
         L.orc_swiglu_fp8_backward.argtypes = [_P(ctypes.c_uint16), _i, _u8, _i, _f, _f, _i, _u8,
                                               _i, _f, _f, _i, _i, _i, ctypes.c_int,
                                               _P(ctypes.c_uint16), _i, _P(ctypes.c_uint16), _i]
+        L.orc_rmsnorm_fp8_forward.restype = ctypes.c_int
+        L.orc_rmsnorm_fp8_forward.argtypes = [_u8, _i, _f, _f, _i, _P(ctypes.c_uint16), _i, _i,
+                                              ctypes.c_double, ctypes.c_int, ctypes.c_int, _u8, _i,
+                                              _f, _f, _i, _P(ctypes.c_double)]
+        L.orc_rmsnorm_fp8_backward.restype = ctypes.c_int
+        L.orc_rmsnorm_fp8_backward.argtypes = [_P(ctypes.c_uint16), _i, _u8, _i, _f, _f, _i,
+                                               _P(ctypes.c_uint16), _i, _i, ctypes.c_double,
+                                               ctypes.c_int, _P(ctypes.c_uint16), _i,
+                                               _P(ctypes.c_double)]
         _lib = L
     return _lib
 
@@ -331,3 +340,46 @@ def swiglu_fp8_backward(dh_bits, gate, up, fmt: int):
                                        _ptr(du, u16), cols)
     assert rc == 0
     return dg, du
+
+
+# ----------------------------------------------------------------------------
+# FP8 precision flow through RMSNorm (x / sqrt(mean(x^2) + eps) * w)
+# ----------------------------------------------------------------------------
+
+def rmsnorm_fp8_forward(x, w_bits, eps, fmt: int, expand: bool, want_rstd=False):
+    """x: (codes u8 [rows, d], scale f32 [rows, groups], k f32 [rows, groups]);
+    w_bits: bf16 bits u16 [d].  Returns the output (codes, scale, k) [and rstd]."""
+    xq, xs, xk = _act(x)
+    w = np.ascontiguousarray(w_bits, dtype=np.uint16)
+    rows, d = xq.shape
+    assert w.size == d
+    ng = xs.shape[1]
+    oq = np.zeros((rows, d), np.uint8)
+    os_ = np.zeros((rows, ng), np.float32)
+    ok = np.zeros((rows, ng), np.float32)
+    rstd = np.zeros(rows, np.float64)
+    u8, f = ctypes.c_uint8, ctypes.c_float
+    rc = lib().orc_rmsnorm_fp8_forward(_ptr(xq, u8), d, _ptr(xs, f), _ptr(xk, f), ng,
+                                       _ptr(w, ctypes.c_uint16), rows, d, float(eps), fmt,
+                                       int(bool(expand)), _ptr(oq, u8), d, _ptr(os_, f),
+                                       _ptr(ok, f), ng, _ptr(rstd, ctypes.c_double))
+    assert rc == 0
+    return ((oq, os_, ok), rstd) if want_rstd else (oq, os_, ok)
+
+
+def rmsnorm_fp8_backward(dy_bits, x, w_bits, eps, fmt: int):
+    """Returns (dx as bf16 bits u16 [rows, d], dw float64 [d])."""
+    xq, xs, xk = _act(x)
+    w = np.ascontiguousarray(w_bits, dtype=np.uint16)
+    dy = np.ascontiguousarray(dy_bits, dtype=np.uint16)
+    rows, d = xq.shape
+    assert dy.shape == (rows, d) and w.size == d
+    ng = xs.shape[1]
+    dx = np.zeros((rows, d), np.uint16)
+    dw = np.zeros(d, np.float64)
+    u8, f, u16 = ctypes.c_uint8, ctypes.c_float, ctypes.c_uint16
+    rc = lib().orc_rmsnorm_fp8_backward(_ptr(dy, u16), d, _ptr(xq, u8), d, _ptr(xs, f),
+                                        _ptr(xk, f), ng, _ptr(w, u16), rows, d, float(eps), fmt,
+                                        _ptr(dx, u16), d, _ptr(dw, ctypes.c_double))
+    assert rc == 0
+    return dx, dw

@@ -544,3 +544,106 @@ int orc_swiglu_fp8_backward(const uint16_t *dh, int64_t lddh, const uint8_t *gq,
         }
     return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* The second non-linear layer of the FP8 precision flow: Llama's      */
+/* RMSNorm, y = x / sqrt(mean(x^2) + eps) * w, per row of d features,   */
+/* with FP8 1x128 input and output and a bf16 weight; the backward      */
+/* reads the saved FP8 input and a bf16 output gradient.                */
+/* Readings: y is rounded to FP32 before it is quantised (the kernel's  */
+/* precision decides the codes); dx is rounded double -> FP32 -> bf16;  */
+/* dw (summed over rows) is returned in double and compared with a      */
+/* tolerance, its summation order being the kernel's own.              */
+/* ------------------------------------------------------------------ */
+
+/* 1 / sqrt(mean(x^2) + eps) of one row of d values. */
+static double orc_rstd(const double *x, int64_t d, double eps)
+{
+    double s = 0.0;
+    for (int64_t i = 0; i < d; i++)
+        s += x[i] * x[i];
+    return 1.0 / sqrt(s / (double)d + eps);
+}
+
+static void orc_dequant_row(const uint8_t *q, const float *s, const float *k, int64_t d, int fmt,
+                            double *x)
+{
+    for (int64_t i = 0; i < d; i++)
+        x[i] = orc_dequant_value(fmt, q[i], s[i / 128], k[i / 128]);
+}
+
+/* Forward over rows x d: x codes (row stride ldxq bytes) with per-group
+ * scale / k (row stride ldxs floats); w: d bf16 values; the output quantised
+ * per 1x128 group into oq / os / ok.  rstd_out (may be NULL) receives each
+ * row's 1 / sqrt(mean(x^2) + eps).  Returns 0, or -1 on bad arguments. */
+int orc_rmsnorm_fp8_forward(const uint8_t *xq, int64_t ldxq, const float *xs, const float *xk,
+                            int64_t ldxs, const uint16_t *w, int64_t rows, int64_t d, double eps,
+                            int fmt, int expand, uint8_t *oq, int64_t ldoq, float *os, float *ok,
+                            int64_t ldos, double *rstd_out)
+{
+    if (rows < 0 || d < 0 || ldxq < d || ldoq < d || !(eps > 0.0))
+        return -1;
+    int64_t ng = (d + 127) / 128;
+    if (ldxs < ng || ldos < ng)
+        return -1;
+    double *x = (double *)malloc(sizeof(double) * (size_t)(d > 0 ? d : 1));
+    double *y = (double *)malloc(sizeof(double) * (size_t)(d > 0 ? d : 1));
+    if (!x || !y) {
+        free(x);
+        free(y);
+        return -1;
+    }
+    for (int64_t r = 0; r < rows; r++) {
+        orc_dequant_row(xq + r * ldxq, xs + r * ldxs, xk + r * ldxs, d, fmt, x);
+        double rs = orc_rstd(x, d, eps);
+        if (rstd_out)
+            rstd_out[r] = rs;
+        for (int64_t i = 0; i < d; i++)
+            y[i] = (double)(float)(x[i] * rs * orc_bf16_to_double(w[i]));
+        for (int64_t j = 0; j < ng; j++) {
+            int64_t c0 = j * 128, cnt = d - c0 < 128 ? d - c0 : 128;
+            orc_quantize_group(y + c0, cnt, expand, fmt, oq + r * ldoq + c0, &ok[r * ldos + j],
+                               &os[r * ldos + j]);
+        }
+    }
+    free(x);
+    free(y);
+    return 0;
+}
+
+/* Backward: with xh = x rstd and g = dy w,
+ *   dx = rstd (g - xh mean(g xh)),   dw = sum over rows of dy xh.
+ * dy: bf16 (row stride lddy); dx: bf16 (row stride lddx); dw: d doubles. */
+int orc_rmsnorm_fp8_backward(const uint16_t *dy, int64_t lddy, const uint8_t *xq, int64_t ldxq,
+                             const float *xs, const float *xk, int64_t ldxs, const uint16_t *w,
+                             int64_t rows, int64_t d, double eps, int fmt, uint16_t *dx,
+                             int64_t lddx, double *dw)
+{
+    if (rows < 0 || d < 0 || lddy < d || ldxq < d || lddx < d || !(eps > 0.0))
+        return -1;
+    int64_t ng = (d + 127) / 128;
+    if (ldxs < ng)
+        return -1;
+    double *x = (double *)malloc(sizeof(double) * (size_t)(d > 0 ? d : 1));
+    if (!x)
+        return -1;
+    for (int64_t i = 0; i < d; i++)
+        dw[i] = 0.0;
+    for (int64_t r = 0; r < rows; r++) {
+        orc_dequant_row(xq + r * ldxq, xs + r * ldxs, xk + r * ldxs, d, fmt, x);
+        double rs = orc_rstd(x, d, eps);
+        double dot = 0.0;   /* sum of g xh */
+        for (int64_t i = 0; i < d; i++)
+            dot += orc_bf16_to_double(dy[r * lddy + i]) * orc_bf16_to_double(w[i]) * x[i] * rs;
+        double mean = dot / (double)d;
+        for (int64_t i = 0; i < d; i++) {
+            double dyi = orc_bf16_to_double(dy[r * lddy + i]);
+            double xh = x[i] * rs;
+            double g = dyi * orc_bf16_to_double(w[i]);
+            dx[r * lddx + i] = orc_float_to_bf16((float)(rs * (g - xh * mean)));
+            dw[i] += dyi * xh;
+        }
+    }
+    free(x);
+    return 0;
+}
