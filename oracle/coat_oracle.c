@@ -550,10 +550,13 @@ int orc_swiglu_fp8_backward(const uint16_t *dh, int64_t lddh, const uint8_t *gq,
 /* RMSNorm, y = x / sqrt(mean(x^2) + eps) * w, per row of d features,   */
 /* with FP8 1x128 input and output and a bf16 weight; the backward      */
 /* reads the saved FP8 input and a bf16 output gradient.                */
-/* Readings: y is rounded to FP32 before it is quantised (the kernel's  */
-/* precision decides the codes); dx is rounded double -> FP32 -> bf16;  */
-/* dw (summed over rows) is returned in double and compared with a      */
-/* tolerance, its summation order being the kernel's own.              */
+/* Readings: y is quantised from its double value (no FP32 rounding of  */
+/* y itself: within a group y_i / y_max = x_i w_i / (x_max w_max), and  */
+/* for k = 1 inputs that ratio is one of exact FP8 x bf16 products, so  */
+/* the code is decided on the exact real number, ties to even, as the   */
+/* kernel does); dx is rounded double -> FP32 -> bf16; dw (summed over  */
+/* rows) is returned in double and compared with a tolerance, its       */
+/* summation order being the kernel's own.                              */
 /* ------------------------------------------------------------------ */
 
 /* 1 / sqrt(mean(x^2) + eps) of one row of d values. */
@@ -599,7 +602,7 @@ int orc_rmsnorm_fp8_forward(const uint8_t *xq, int64_t ldxq, const float *xs, co
         if (rstd_out)
             rstd_out[r] = rs;
         for (int64_t i = 0; i < d; i++)
-            y[i] = (double)(float)(x[i] * rs * orc_bf16_to_double(w[i]));
+            y[i] = x[i] * rs * orc_bf16_to_double(w[i]);
         for (int64_t j = 0; j < ng; j++) {
             int64_t c0 = j * 128, cnt = d - c0 < 128 ? d - c0 : 128;
             orc_quantize_group(y + c0, cnt, expand, fmt, oq + r * ldoq + c0, &ok[r * ldos + j],
