@@ -47,6 +47,10 @@ EXPORTS = [
     ("coat_swiglu_fp8_forward", _i32, [_vp, _vp, _i64, _i64, _i32, _i32, _vp, _vp]),
     ("coat_swiglu_fp8_backward", _i32, [_vp, _i64, _vp, _vp, _i64, _i64, _i32, _vp, _i64, _vp,
                                         _i64, _vp]),
+    ("coat_rmsnorm_fp8_forward", _i32, [_vp, _vp, _i64, _i64, _f32, _i32, _i32, _vp, _vp]),
+    ("coat_rmsnorm_fp8_workspace_size", _i32, [_i64, ctypes.POINTER(ctypes.c_size_t)]),
+    ("coat_rmsnorm_fp8_backward", _i32, [_vp, _i64, _vp, _vp, _i64, _i64, _f32, _i32, _vp, _i64,
+                                         _vp, _vp, ctypes.c_size_t, _vp]),
 ]
 NOALLOC_MAX_TENSORS = 1024
 
@@ -119,6 +123,34 @@ def coat_swiglu_fp8_backward(grad_out, gate, up, fmt, grad_gate, grad_up, stream
                                           ctypes.byref(u), rows, cols, fmt, _p(grad_gate),
                                           grad_gate.stride(0), _p(grad_up), grad_up.stride(0),
                                           _s(stream)))
+
+
+def coat_rmsnorm_fp8_forward(x, w, eps, fmt, expand_out, out, stream=None):
+    """x, out: (codes, scale, k) tensors in the 1x128 layout; w: bf16 [d] CUDA tensor."""
+    xa, oa = _act(x), _act(out)
+    rows, d = x[0].shape
+    _check(lib().coat_rmsnorm_fp8_forward(ctypes.byref(xa), _p(w), rows, d, eps, fmt,
+                                          int(bool(expand_out)), ctypes.byref(oa), _s(stream)))
+
+
+def coat_rmsnorm_fp8_workspace_size(d):
+    n = ctypes.c_size_t()
+    _check(lib().coat_rmsnorm_fp8_workspace_size(d, ctypes.byref(n)))
+    return n.value
+
+
+def coat_rmsnorm_fp8_backward(dy, x, w, eps, fmt, dx, dw, workspace, stream=None):
+    """dy, dx: bf16 [rows, d]; dw: float32 [d]; workspace: a CUDA buffer of at
+    least coat_rmsnorm_fp8_workspace_size(d) bytes."""
+    xa = _act(x)
+    rows, d = x[0].shape
+    for t in (dy, dx):
+        if t.dim() != 2 or t.stride(1) != 1 or t.element_size() != 2:
+            raise ValueError("expected 2-D bf16 tensors with contiguous rows")
+    _check(lib().coat_rmsnorm_fp8_backward(_p(dy), dy.stride(0), ctypes.byref(xa), _p(w), rows, d,
+                                           eps, fmt, _p(dx), dx.stride(0), _p(dw), _p(workspace),
+                                           workspace.numel() * workspace.element_size(),
+                                           _s(stream)))
 
 
 class TensorDesc(ctypes.Structure):

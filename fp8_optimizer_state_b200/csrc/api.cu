@@ -319,6 +319,80 @@ coat_status coat_swiglu_fp8_backward(const uint16_t* grad_out, int64_t ld_grad_o
   return e == cudaSuccess ? COAT_OK : cuda_fail(e, fn);
 }
 
+static coat_status check_rms_shape(const char* fn, int64_t rows, int64_t d, float eps,
+                                   coat_fmt fmt, const uint16_t* w) {
+  if (rows < 0 || d < 0) return fail(COAT_ERR_INVALID_ARG, "%s: negative shape", fn);
+  if (!valid_fmt(fmt)) return fail(COAT_ERR_INVALID_ARG, "%s: bad fmt %d", fn, int(fmt));
+  if (!std::isfinite(eps) || !(eps > 0.f)) return fail(COAT_ERR_INVALID_ARG, "%s: eps must be finite and > 0", fn);
+  if (d % 128 != 0 || d > coat::rmsnorm_max_d())
+    return fail(COAT_ERR_UNSUPPORTED, "%s: d must be a multiple of 128, at most %lld", fn,
+                static_cast<long long>(coat::rmsnorm_max_d()));
+  if (d > 0 && !w) return fail(COAT_ERR_INVALID_ARG, "%s: w is NULL", fn);
+  if (d > 0 && !aligned(w, 16)) return fail(COAT_ERR_MISALIGNED, "%s: w is not 16-byte aligned", fn);
+  return COAT_OK;
+}
+
+coat_status coat_rmsnorm_fp8_forward(const coat_fp8_act* x, const uint16_t* w, int64_t rows,
+                                     int64_t d, float eps, coat_fmt fmt, int expand_out,
+                                     const coat_fp8_act* out, cudaStream_t stream) {
+  const char* fn = "coat_rmsnorm_fp8_forward";
+  coat_status st = check_rms_shape(fn, rows, d, eps, fmt, w);
+  if (st != COAT_OK) return st;
+  if (expand_out != 0 && expand_out != 1)
+    return fail(COAT_ERR_INVALID_ARG, "%s: expand_out must be 0 or 1", fn);
+  st = check_act(fn, "x", x, rows, d);
+  if (st == COAT_OK) st = check_act(fn, "out", out, rows, d);
+  if (st != COAT_OK) return st;
+  if (rows == 0 || d == 0) return COAT_OK;
+  cudaError_t e = coat::launch_rmsnorm_fp8_forward(act_args(x), w, rows, d, eps, fmt, expand_out,
+                                                   act_args(out), stream);
+  return e == cudaSuccess ? COAT_OK : cuda_fail(e, fn);
+}
+
+coat_status coat_rmsnorm_fp8_workspace_size(int64_t d, size_t* bytes) {
+  const char* fn = "coat_rmsnorm_fp8_workspace_size";
+  if (!bytes) return fail(COAT_ERR_INVALID_ARG, "%s: bytes is NULL", fn);
+  *bytes = 0;
+  if (d < 0) return fail(COAT_ERR_INVALID_ARG, "%s: negative d", fn);
+  if (d % 128 != 0 || d > coat::rmsnorm_max_d())
+    return fail(COAT_ERR_UNSUPPORTED, "%s: d must be a multiple of 128, at most %lld", fn,
+                static_cast<long long>(coat::rmsnorm_max_d()));
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  *bytes = coat::rmsnorm_workspace_bytes(dev, d);
+  return COAT_OK;
+}
+
+coat_status coat_rmsnorm_fp8_backward(const uint16_t* dy, int64_t ld_dy, const coat_fp8_act* x,
+                                      const uint16_t* w, int64_t rows, int64_t d, float eps,
+                                      coat_fmt fmt, uint16_t* dx, int64_t ld_dx, float* dw,
+                                      void* workspace, size_t workspace_bytes,
+                                      cudaStream_t stream) {
+  const char* fn = "coat_rmsnorm_fp8_backward";
+  coat_status st = check_rms_shape(fn, rows, d, eps, fmt, w);
+  if (st != COAT_OK) return st;
+  st = check_act(fn, "x", x, rows, d);
+  if (st == COAT_OK) st = check_bf16(fn, "dy", dy, ld_dy, rows, d);
+  if (st == COAT_OK) st = check_bf16(fn, "dx", dx, ld_dx, rows, d);
+  if (st != COAT_OK) return st;
+  if (d == 0) return COAT_OK;
+  if (!dw) return fail(COAT_ERR_INVALID_ARG, "%s: dw is NULL", fn);
+  if (!aligned(dw, 4)) return fail(COAT_ERR_MISALIGNED, "%s: dw is not 4-byte aligned", fn);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  const size_t need = coat::rmsnorm_workspace_bytes(dev, d);
+  if (rows > 0) {
+    if (!workspace || workspace_bytes < need)
+      return fail(COAT_ERR_INVALID_ARG, "%s: workspace needs %zu bytes", fn, need);
+    if (!aligned(workspace, 16)) return fail(COAT_ERR_MISALIGNED, "%s: workspace is not 16-byte aligned", fn);
+  }
+  e = coat::launch_rmsnorm_fp8_backward(dy, ld_dy, act_args(x), w, rows, d, eps, fmt, dx, ld_dx,
+                                        dw, static_cast<float*>(workspace), stream);
+  return e == cudaSuccess ? COAT_OK : cuda_fail(e, fn);
+}
+
 coat_status coat_adamw_step(float* master, uint16_t* weight_bf16_out, const uint16_t* grad,
                             uint8_t* m_q, float* m_scale, float* m_k, uint8_t* v_q, float* v_scale,
                             float* v_k, int64_t n, int group, float lr, float beta1, float beta2,

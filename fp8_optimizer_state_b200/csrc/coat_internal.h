@@ -109,4 +109,19 @@ cudaError_t launch_swiglu_fp8_backward(const uint16_t* dh, int64_t lddh, const A
                                        uint16_t* dg, int64_t lddg, uint16_t* du, int64_t lddu,
                                        cudaStream_t s);
 
+// RMSNorm y = x / sqrt(mean(x^2) + eps) * w per row (d a multiple of 128, at
+// most rmsnorm_max_d()), FP8 1x128 in and out, bf16 w.
+int64_t rmsnorm_max_d();
+// Bytes of the backward's per-CTA dw partials for rows of d features.
+size_t rmsnorm_workspace_bytes(int dev, int64_t d);
+cudaError_t launch_rmsnorm_fp8_forward(const ActArgs& x, const uint16_t* w, int64_t rows, int64_t d,
+                                       float eps, int fmt, int expand, const ActArgs& out,
+                                       cudaStream_t s);
+// dx (bf16) and dw (FP32, summed over rows in a fixed order) from dy (bf16)
+// and the forward's FP8 input; partial: rmsnorm_workspace_bytes() of scratch.
+cudaError_t launch_rmsnorm_fp8_backward(const uint16_t* dy, int64_t lddy, const ActArgs& x,
+                                        const uint16_t* w, int64_t rows, int64_t d, float eps,
+                                        int fmt, uint16_t* dx, int64_t lddx, float* dw,
+                                        float* partial, cudaStream_t s);
+
 }  // namespace coat

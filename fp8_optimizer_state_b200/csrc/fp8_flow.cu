@@ -110,6 +110,81 @@ __device__ __forceinline__ void decode16_raw(const uint4& w, float k, bool plain
   }
 }
 
+// Quantise the 16 values a lane holds of an 8-lane 1x128 group, as the 1x128
+// codec does (called by all 32 lanes of a warp: 4 groups).  Group max |h| by a
+// NaN-propagating max (one test then finds NaN and Inf) and, with expansion,
+// min nonzero |h| on twice the bit patterns (zero becomes the largest key).
+// k = 1 groups encode FMT_MAX |h| / M as |h| (FMT_MAX / M) (a few ulps from the
+// correctly rounded quotient, which decides a code only at an exact tie of
+// the real-number result; at most FMT_MAX (1 + 2^-21), inside the bounded
+// encoder's range) with root scale M / FMT_MAX correctly rounded; expanded
+// groups use the codec's expansion.  The slow path (the codec's NaN rules and
+// IEEE division) takes groups with a NaN or an Inf, a maximum below 2^-64
+// (1/M would leave FP32), or force_slow (the same for the 8 lanes of a group).
+template <int FMT, bool EXPAND>
+__device__ __forceinline__ void quantize_lane16(const float (&h)[16], bool force_slow,
+                                                uint32_t (&cw)[4], float& k, float& sr) {
+  float mx = 0.0f;
+  uint32_t mink = 0xFFFFFFFFu;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    mx = fmax_nan(mx, fabsf(h[i]));
+    if (EXPAND) mink = min(mink, __float_as_uint(h[i]) * 2u - 2u);
+  }
+#pragma unroll
+  for (int off = 1; off < 8; off <<= 1) {
+    mx = fmax_nan(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+    if (EXPAND) mink = min(mink, __shfl_xor_sync(0xFFFFFFFFu, mink, off));
+  }
+  const bool special = !(mx <= 3.40282347e38f) || force_slow ||
+                       (mx > 0.0f && mx < 5.421010862427522e-20f);
+  if (!__any_sync(0xFFFFFFFFu, special)) {
+    const float M = mx;
+    float invM;
+    if (EXPAND) {
+      group_params<FMT>(M, __uint_as_float((mink + 2u) >> 1), true, k, sr, invM);
+    } else {
+      k = 1.0f;
+      sr = M > 0.0f ? __fdiv_rn(M, F8<FMT>::MAXV) : 1.0f;   // M / FMT_MAX, correctly rounded
+      invM = M > 0.0f ? rcp_approx(M) : 0.0f;   // an all-zero group encodes to zeros
+    }
+    uint32_t mag[16];
+    if (k == 1.0f) {
+      const float c = F8<FMT>::MAXV * invM;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) mag[i] = enc_mag_bounded<FMT>(fabsf(h[i]) * c);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) mag[i] = enc_mag_bounded<FMT>(expand_value<FMT>(h[i], invM, k));
+    }
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+      cw[w] = merge_signs4(pack4(mag[4 * w], mag[4 * w + 1], mag[4 * w + 2], mag[4 * w + 3]),
+                           h[4 * w], h[4 * w + 1], h[4 * w + 2], h[4 * w + 3]);
+  } else {
+    // the codec's slow path: the maximum ignores NaN, IEEE division for k = 1
+    float Mn = max_abs_nonnan(h);
+#pragma unroll
+    for (int off = 1; off < 8; off <<= 1) Mn = fmaxf(Mn, __shfl_xor_sync(0xFFFFFFFFu, Mn, off));
+    uint32_t mk2 = 0xFFFFFFFFu;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) mk2 = min(mk2, __float_as_uint(h[i]) * 2u - 2u);
+#pragma unroll
+    for (int off = 1; off < 8; off <<= 1) mk2 = min(mk2, __shfl_xor_sync(0xFFFFFFFFu, mk2, off));
+    const float M = special ? Mn : mx;
+    float invM;
+    group_params<FMT>(M, __uint_as_float((mk2 + 2u) >> 1), EXPAND, k, sr, invM);
+    if (!EXPAND) sr = M > 0.0f ? __fdiv_rn(M, F8<FMT>::MAXV) : 1.0f;
+    const bool use_div = k == 1.0f;
+    GroupDiv d{};
+    if (use_div) d = codec_div<FMT>(M);
+    if (special)
+      encode_words<FMT, 16, false>(h, use_div, d, invM, k, cw);
+    else
+      encode_words<FMT, 16, true>(h, use_div, d, invM, k, cw);
+  }
+}
+
 // One lane's forward work item: 16 gate and 16 up codes, their groups'
 // metadata, and the item's row and the lane's first column.
 struct FwdItem {
@@ -122,12 +197,8 @@ struct FwdItem {
 
 // h = silu(g) u with g = f_g s_g, u = f_u s_u, as ((f_g f_u) sigmoid(g)) (s_g s_u):
 // f_g f_u is exact for k = 1 inputs (two FP8 significands), so h takes two
-// roundings besides the sigmoid's.  The output codes: k = 1 groups encode
-// FMT_MAX |h| / M as |h| (FMT_MAX / M) (a few ulps from the correctly rounded
-// quotient, which only decides codes at exact ties of the real-number result;
-// at most FMT_MAX (1 + 2^-21), inside the bounded encoder's range) with root
-// scale M / FMT_MAX; expanded groups use the codec's expansion.  EXPAND:
-// output expansion on.
+// roundings besides the sigmoid's; h is then quantised by quantize_lane16.
+// EXPAND: output expansion on.
 // Work: the rows x ceil(groups/4) items (4 groups of a row, 8 lanes each) in
 // row-major order, a contiguous range per warp (columns advanced by 512 with
 // a row carry); the next item is loaded before the current one is computed.
@@ -187,71 +258,10 @@ __global__ void __launch_bounds__(256) swiglu_fwd_kernel(const ActArgs gate, con
       h[i] = ((fg[i] * fu[i]) * sg) * S;
     }
 
-    // group max |h| (NaN-propagating, so that one test finds NaN and Inf) and,
-    // with expansion, min nonzero |h| on twice the bit patterns (zero becomes
-    // the largest key)
-    float mx = 0.0f;
-    uint32_t mink = 0xFFFFFFFFu;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      mx = fmax_nan(mx, fabsf(h[i]));
-      if (EXPAND) mink = min(mink, __float_as_uint(h[i]) * 2u - 2u);
-    }
-#pragma unroll
-    for (int off = 1; off < 8; off <<= 1) {
-      mx = fmax_nan(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
-      if (EXPAND) mink = min(mink, __shfl_xor_sync(0xFFFFFFFFu, mink, off));
-    }
-    // slow path: an Inf or a NaN in the group, a scale product that overflowed,
-    // or a maximum so small that 1/M would leave FP32 (below 2^-64)
-    const bool special = !(mx <= 3.40282347e38f) || !(S <= 3.40282347e38f) ||
-                         (mx > 0.0f && mx < 5.421010862427522e-20f);
+    // slow path also when the scale product overflowed
     uint32_t cw[4];
     float k, sr;
-    if (!__any_sync(0xFFFFFFFFu, special)) {
-      const float M = mx;
-      float invM;
-      if (EXPAND) {
-        group_params<FMT>(M, __uint_as_float((mink + 2u) >> 1), true, k, sr, invM);
-      } else {
-        k = 1.0f;
-        sr = M > 0.0f ? __fdiv_rn(M, F8<FMT>::MAXV) : 1.0f;   // M / FMT_MAX, correctly rounded
-        invM = M > 0.0f ? rcp_approx(M) : 0.0f;   // an all-zero group encodes to zeros
-      }
-      uint32_t mag[16];
-      if (k == 1.0f) {
-        const float c = F8<FMT>::MAXV * invM;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) mag[i] = enc_mag_bounded<FMT>(fabsf(h[i]) * c);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) mag[i] = enc_mag_bounded<FMT>(expand_value<FMT>(h[i], invM, k));
-      }
-#pragma unroll
-      for (int w = 0; w < 4; ++w)
-        cw[w] = merge_signs4(pack4(mag[4 * w], mag[4 * w + 1], mag[4 * w + 2], mag[4 * w + 3]),
-                             h[4 * w], h[4 * w + 1], h[4 * w + 2], h[4 * w + 3]);
-    } else {
-      // the codec's slow path: the maximum ignores NaN, IEEE division for k = 1
-      float Mn = max_abs_nonnan(h);
-#pragma unroll
-      for (int off = 1; off < 8; off <<= 1) Mn = fmaxf(Mn, __shfl_xor_sync(0xFFFFFFFFu, Mn, off));
-      uint32_t mk2 = 0xFFFFFFFFu;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) mk2 = min(mk2, __float_as_uint(h[i]) * 2u - 2u);
-#pragma unroll
-      for (int off = 1; off < 8; off <<= 1) mk2 = min(mk2, __shfl_xor_sync(0xFFFFFFFFu, mk2, off));
-      const float M = special ? Mn : mx;
-      float invM;
-      group_params<FMT>(M, __uint_as_float((mk2 + 2u) >> 1), EXPAND, k, sr, invM);
-      const bool use_div = k == 1.0f;
-      GroupDiv d{};
-      if (use_div) d = codec_div<FMT>(M);
-      if (special)
-        encode_words<FMT, 16, false>(h, use_div, d, invM, k, cw);
-      else
-        encode_words<FMT, 16, true>(h, use_div, d, invM, k, cw);
-    }
+    quantize_lane16<FMT, EXPAND>(h, !(S <= 3.40282347e38f), cw, k, sr);
     if (cur.valid) {
       *reinterpret_cast<uint4*>(out.q + cur.r * out.ldq + cur.c) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
       if (l == 0) {
@@ -339,6 +349,259 @@ __global__ void __launch_bounds__(256) swiglu_bwd_kernel(const uint16_t* __restr
   }
 }
 
+// ---------------------------------------------------------------------------
+// RMSNorm, the other non-linear layer of a Llama block:
+// y = x / sqrt(mean(x^2) + eps) * w per row of d features (d a multiple of
+// 128, at most kNormThreads * 16 * CPT), FP8 1x128 input and output, bf16 w.
+// One 256-thread CTA per row at a time (a persistent loop over rows); thread t
+// holds the 16-column chunks t, t + 256, ... (CPT of them), so that 8
+// consecutive threads hold one 128-column group and w stays in registers
+// across rows.  Row sums go through warp shuffles and shared memory.
+// ---------------------------------------------------------------------------
+constexpr int kNormThreads = 256;
+
+// Sum of v over the CTA, returned to every thread (red: kNormThreads/32 floats
+// per value, reused only after the barrier that ends this call's reads).
+template <int NV>
+__device__ __forceinline__ void cta_sum_all(float (&v)[NV], float (*red)[kNormThreads / 32]) {
+#pragma unroll
+  for (int n = 0; n < NV; ++n)
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v[n] += __shfl_xor_sync(0xFFFFFFFFu, v[n], off);
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0)
+#pragma unroll
+    for (int n = 0; n < NV; ++n) red[n][warp] = v[n];
+  __syncthreads();
+#pragma unroll
+  for (int n = 0; n < NV; ++n) {
+    float t = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kNormThreads / 32; ++w) t += red[n][w];
+    v[n] = t;
+  }
+  __syncthreads();
+}
+
+// 16 bf16 values to floats.
+__device__ __forceinline__ void bf16x16(const uint4& a, const uint4& b, float (&f)[16]) {
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    f[2 * j] = bf16lo(w[j]);
+    f[2 * j + 1] = bf16hi(w[j]);
+  }
+}
+
+// Quantise y = p C (C > 0, one value per group) from a lane's 16 values p of
+// an 8-lane 1x128 group.  Without expansion the codes are decided on the
+// ratio |p_i| / max|p| = |y_i| / max|y| (C cancels), as one correctly rounded
+// division: for k = 1 inputs p_i = (FP8 value) x (bf16 weight) is exact, so an
+// exact tie of the real-number result stays a tie and is broken to even, as
+// the oracle does; the root scale is max|y| / FMT_MAX.  With expansion, and
+// for groups with a NaN/Inf or an unusable C, the values y go through
+// quantize_lane16.
+template <int FMT, bool EXPAND>
+__device__ __forceinline__ void quantize_scaled16(const float (&p)[16], float C, uint32_t (&cw)[4],
+                                                  float& k, float& sr) {
+  float y[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) y[i] = p[i] * C;
+  if (EXPAND) {
+    quantize_lane16<FMT, true>(y, false, cw, k, sr);
+    return;
+  }
+  float mp = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) mp = fmax_nan(mp, fabsf(p[i]));
+#pragma unroll
+  for (int off = 1; off < 8; off <<= 1) mp = fmax_nan(mp, __shfl_xor_sync(0xFFFFFFFFu, mp, off));
+  const float My = mp * C;
+  const bool special = !(mp <= 3.40282347e38f) || !(My <= 3.40282347e38f) || !(C > 0.0f);
+  if (__any_sync(0xFFFFFFFFu, special)) {
+    quantize_lane16<FMT, false>(y, special, cw, k, sr);
+    return;
+  }
+  k = 1.0f;
+  sr = My > 0.0f ? __fdiv_rn(My, F8<FMT>::MAXV) : 1.0f;
+  const GroupDiv dv = codec_div<FMT>(mp);
+  encode_words<FMT, 16, true>(p, true, dv, 0.0f, 1.0f, cw);
+}
+
+template <int FMT, bool EXPAND, int CPT>
+__global__ void __launch_bounds__(kNormThreads) rmsnorm_fwd_kernel(const ActArgs x,
+                                                                   const uint16_t* __restrict__ w,
+                                                                   int64_t rows, int64_t d,
+                                                                   float eps, const ActArgs out) {
+  __shared__ float tab[256];
+  __shared__ float red[1][kNormThreads / 32];
+  fill_log2_table<FMT>(tab);
+  __syncthreads();
+  const float inv_d = 1.0f / static_cast<float>(d);
+  float wv[CPT][16];
+  bool ok[CPT];
+#pragma unroll
+  for (int j = 0; j < CPT; ++j) {
+    const int64_t c = (threadIdx.x + int64_t(j) * kNormThreads) * 16;
+    ok[j] = c < d;
+    if (ok[j]) {
+      const uint4* wp = reinterpret_cast<const uint4*>(w + c);
+      bf16x16(__ldg(wp), __ldg(wp + 1), wv[j]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) wv[j][i] = 0.0f;
+    }
+  }
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    float pv[CPT][16], sv[CPT];
+    float ss[1] = {0.0f};
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+      const int64_t c = (threadIdx.x + int64_t(j) * kNormThreads) * 16;
+      uint4 q = make_uint4(0u, 0u, 0u, 0u);
+      float s = 1.0f, k = 1.0f;
+      if (ok[j]) {
+        q = __ldg(reinterpret_cast<const uint4*>(x.q + r * x.ldq + c));
+        s = __ldg(x.scale + r * x.lds + (c >> 7));
+        k = __ldg(x.k + r * x.lds + (c >> 7));
+      }
+      const bool plain = __all_sync(0xFFFFFFFFu, k == 1.0f);
+      float f[16];
+      decode16_raw<FMT>(q, k, plain, tab, f);
+      float sf = 0.0f;   // sum of f^2 (x = f s)
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        sf = __fmaf_rn(f[i], f[i], sf);
+        pv[j][i] = f[i] * wv[j][i];   // exact for k = 1: an FP8 value times a bf16 value
+      }
+      ss[0] = __fmaf_rn(sf, s * s, ss[0]);
+      sv[j] = s;
+    }
+    cta_sum_all(ss, red);
+    const float rstd = 1.0f / sqrtf(__fmaf_rn(ss[0], inv_d, eps));
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+      uint32_t cw[4];
+      float k, sr;
+      quantize_scaled16<FMT, EXPAND>(pv[j], sv[j] * rstd, cw, k, sr);
+      if (ok[j]) {
+        const int64_t c = (threadIdx.x + int64_t(j) * kNormThreads) * 16;
+        *reinterpret_cast<uint4*>(out.q + r * out.ldq + c) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        if ((threadIdx.x & 7) == 0) {
+          out.scale[r * out.lds + (c >> 7)] = sr;
+          out.k[r * out.lds + (c >> 7)] = k;
+        }
+      }
+    }
+  }
+}
+
+// Backward: with xh = x rstd and g = dy w,
+//   dx = rstd (g - xh mean(g xh)) = rstd g - (rstd^2 mean) x,
+// and each CTA sums dy xh over its rows into its own row of `partial`
+// (partial[blockIdx.x][0..d)); rmsnorm_dw_kernel adds the rows in index order.
+template <int FMT, int CPT>
+__global__ void __launch_bounds__(kNormThreads) rmsnorm_bwd_kernel(
+    const uint16_t* __restrict__ dy, int64_t lddy, const ActArgs x,
+    const uint16_t* __restrict__ w, int64_t rows, int64_t d, float eps,
+    uint16_t* __restrict__ dx, int64_t lddx, float* __restrict__ partial) {
+  __shared__ float tab[256];
+  __shared__ float red[2][kNormThreads / 32];
+  fill_log2_table<FMT>(tab);
+  __syncthreads();
+  const float inv_d = 1.0f / static_cast<float>(d);
+  float wv[CPT][16], acc[CPT][16];
+  bool ok[CPT];
+#pragma unroll
+  for (int j = 0; j < CPT; ++j) {
+    const int64_t c = (threadIdx.x + int64_t(j) * kNormThreads) * 16;
+    ok[j] = c < d;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc[j][i] = 0.0f;
+    if (ok[j]) {
+      const uint4* wp = reinterpret_cast<const uint4*>(w + c);
+      bf16x16(__ldg(wp), __ldg(wp + 1), wv[j]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) wv[j][i] = 0.0f;
+    }
+  }
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    float xv[CPT][16], dv[CPT][16];
+    float sums[2] = {0.0f, 0.0f};   // sum x^2, sum g x
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+      const int64_t c = (threadIdx.x + int64_t(j) * kNormThreads) * 16;
+      uint4 q = make_uint4(0u, 0u, 0u, 0u), d0 = q, d1 = q;
+      float s = 1.0f, k = 1.0f;
+      if (ok[j]) {
+        q = __ldcs(reinterpret_cast<const uint4*>(x.q + r * x.ldq + c));
+        s = __ldg(x.scale + r * x.lds + (c >> 7));
+        k = __ldg(x.k + r * x.lds + (c >> 7));
+        const uint4* dp = reinterpret_cast<const uint4*>(dy + r * lddy + c);
+        d0 = __ldcs(dp);
+        d1 = __ldcs(dp + 1);
+      }
+      const bool plain = __all_sync(0xFFFFFFFFu, k == 1.0f);
+      float f[16];
+      decode16_raw<FMT>(q, k, plain, tab, f);
+      bf16x16(d0, d1, dv[j]);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        xv[j][i] = f[i] * s;
+        sums[0] = __fmaf_rn(xv[j][i], xv[j][i], sums[0]);
+        sums[1] = __fmaf_rn(dv[j][i] * wv[j][i], xv[j][i], sums[1]);
+      }
+    }
+    cta_sum_all(sums, red);
+    const float rstd = 1.0f / sqrtf(__fmaf_rn(sums[0], inv_d, eps));
+    // rstd^2 mean(g xh) = rstd^3 sum(g x) / d
+    const float cx = rstd * rstd * rstd * sums[1] * inv_d;
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+      uint32_t o[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        float a[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int i = 2 * e + h;
+          const float g = dv[j][i] * wv[j][i];
+          a[h] = __fmaf_rn(rstd, g, -cx * xv[j][i]);
+          acc[j][i] = __fmaf_rn(dv[j][i], xv[j][i] * rstd, acc[j][i]);
+        }
+        o[e] = pack_bf16x2(a[0], a[1]);
+      }
+      if (ok[j]) {
+        const int64_t c = (threadIdx.x + int64_t(j) * kNormThreads) * 16;
+        uint4* op = reinterpret_cast<uint4*>(dx + r * lddx + c);
+        op[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        op[1] = make_uint4(o[4], o[5], o[6], o[7]);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < CPT; ++j) {
+    if (!ok[j]) continue;
+    const int64_t c = (threadIdx.x + int64_t(j) * kNormThreads) * 16;
+    float4* pp = reinterpret_cast<float4*>(partial + blockIdx.x * d + c);
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+      pp[v] = make_float4(acc[j][4 * v], acc[j][4 * v + 1], acc[j][4 * v + 2], acc[j][4 * v + 3]);
+  }
+}
+
+// dw[c] = sum over the nparts rows of partial[., c], in row order, in double.
+__global__ void __launch_bounds__(kNormThreads) rmsnorm_dw_kernel(const float* __restrict__ partial,
+                                                                  int nparts, int64_t d,
+                                                                  float* __restrict__ dw) {
+  const int64_t c = blockIdx.x * int64_t(kNormThreads) + threadIdx.x;
+  if (c >= d) return;
+  double t = 0.0;
+  for (int p = 0; p < nparts; ++p) t += static_cast<double>(__ldg(partial + p * d + c));
+  dw[c] = static_cast<float>(t);
+}
+
 template <int FMT>
 void fwd_launch(const ActArgs& gate, const ActArgs& up, int64_t rows, int64_t cols, int expand,
                 const ActArgs& out, int dev, cudaStream_t s) {
@@ -358,7 +621,79 @@ void bwd_launch(const uint16_t* dh, int64_t lddh, const ActArgs& gate, const Act
   kern<<<g, 256, 0, s>>>(dh, lddh, gate, up, rows, cols, dg, lddg, du, lddu);
 }
 
+constexpr int kNormMaxCtasPerSm = 8;
+
+template <int FMT, bool EXPAND, int CPT>
+cudaError_t rms_fwd_launch(const ActArgs& x, const uint16_t* w, int64_t rows, int64_t d, float eps,
+                           const ActArgs& out, int dev, cudaStream_t s) {
+  auto kern = rmsnorm_fwd_kernel<FMT, EXPAND, CPT>;
+  const int per_sm = resident_ctas(reinterpret_cast<const void*>(kern));
+  const unsigned g = grid_for(rows, 1, dev, per_sm < kNormMaxCtasPerSm ? per_sm : kNormMaxCtasPerSm);
+  kern<<<g, kNormThreads, 0, s>>>(x, w, rows, d, eps, out);
+  return cudaGetLastError();
+}
+
+template <int FMT, int CPT>
+cudaError_t rms_bwd_launch(const uint16_t* dy, int64_t lddy, const ActArgs& x, const uint16_t* w,
+                           int64_t rows, int64_t d, float eps, uint16_t* dx, int64_t lddx,
+                           float* dw, float* partial, int dev, cudaStream_t s) {
+  auto kern = rmsnorm_bwd_kernel<FMT, CPT>;
+  const int per_sm = resident_ctas(reinterpret_cast<const void*>(kern));
+  const unsigned g = grid_for(rows, 1, dev, per_sm < kNormMaxCtasPerSm ? per_sm : kNormMaxCtasPerSm);
+  kern<<<g, kNormThreads, 0, s>>>(dy, lddy, x, w, rows, d, eps, dx, lddx, partial);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  rmsnorm_dw_kernel<<<static_cast<unsigned>((d + kNormThreads - 1) / kNormThreads), kNormThreads,
+                      0, s>>>(partial, static_cast<int>(g), d, dw);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+size_t rmsnorm_workspace_bytes(int dev, int64_t d) {
+  return sizeof(float) * size_t(sm_count(dev)) * kNormMaxCtasPerSm * size_t(d);
+}
+
+int64_t rmsnorm_max_d() { return int64_t(kNormThreads) * 16 * 2; }
+
+cudaError_t launch_rmsnorm_fp8_forward(const ActArgs& x, const uint16_t* w, int64_t rows, int64_t d,
+                                       float eps, int fmt, int expand, const ActArgs& out,
+                                       cudaStream_t s) {
+  if (rows == 0 || d == 0) return cudaSuccess;
+  if (d % kGroup != 0 || d > rmsnorm_max_d()) return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool two = d > int64_t(kNormThreads) * 16;
+#define COAT_RMS_FWD(F)                                                                        \
+  return two ? (expand ? rms_fwd_launch<F, true, 2>(x, w, rows, d, eps, out, dev, s)          \
+                       : rms_fwd_launch<F, false, 2>(x, w, rows, d, eps, out, dev, s))        \
+             : (expand ? rms_fwd_launch<F, true, 1>(x, w, rows, d, eps, out, dev, s)          \
+                       : rms_fwd_launch<F, false, 1>(x, w, rows, d, eps, out, dev, s));
+  if (fmt == kE4M3) { COAT_RMS_FWD(kE4M3) }
+  if (fmt == kE5M2) { COAT_RMS_FWD(kE5M2) }
+  COAT_RMS_FWD(kE5M2Full)
+#undef COAT_RMS_FWD
+}
+
+cudaError_t launch_rmsnorm_fp8_backward(const uint16_t* dy, int64_t lddy, const ActArgs& x,
+                                        const uint16_t* w, int64_t rows, int64_t d, float eps,
+                                        int fmt, uint16_t* dx, int64_t lddx, float* dw,
+                                        float* partial, cudaStream_t s) {
+  if (d == 0) return cudaSuccess;
+  if (d % kGroup != 0 || d > rmsnorm_max_d()) return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (rows == 0) return cudaMemsetAsync(dw, 0, sizeof(float) * size_t(d), s);
+  const bool two = d > int64_t(kNormThreads) * 16;
+  // decoding is the same for both E5M2 variants
+  if (fmt == kE4M3)
+    return two ? rms_bwd_launch<kE4M3, 2>(dy, lddy, x, w, rows, d, eps, dx, lddx, dw, partial, dev, s)
+               : rms_bwd_launch<kE4M3, 1>(dy, lddy, x, w, rows, d, eps, dx, lddx, dw, partial, dev, s);
+  return two ? rms_bwd_launch<kE5M2, 2>(dy, lddy, x, w, rows, d, eps, dx, lddx, dw, partial, dev, s)
+             : rms_bwd_launch<kE5M2, 1>(dy, lddy, x, w, rows, d, eps, dx, lddx, dw, partial, dev, s);
+}
 
 cudaError_t launch_swiglu_fp8_forward(const ActArgs& gate, const ActArgs& up, int64_t rows,
                                       int64_t cols, int fmt, int expand, const ActArgs& out,

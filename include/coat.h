@@ -325,6 +325,38 @@ coat_status coat_swiglu_fp8_backward(const uint16_t *grad_out, int64_t ld_grad_o
                                      cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * The FP8 precision flow through RMSNorm, the other non-linear layer of a
+ * Llama block ([P1] FP8激活 / 混合粒度FP8精度流):
+ *   y = x / sqrt(mean(x^2) + eps) * w   per row of d features,
+ * x and y FP8 tensors in the 1x128 layout (coat_fp8_act), w a bf16 vector of d.
+ *
+ * coat_rmsnorm_fp8_forward: y computed in FP32 (the row's mean of squares
+ * summed in FP32) and quantised per 1x128 group exactly as coat_group_quantize
+ * does (expand_out 0 or 1).  `out` must not overlap x.
+ * coat_rmsnorm_fp8_backward: from dy (bf16, row stride ld_dy) and the
+ * forward's FP8 x, with xh = x rstd and g = dy w,
+ *   dx = rstd (g - xh mean(g xh))         (bf16, row stride ld_dx),
+ *   dw = sum over rows of dy xh            (d floats, summed per CTA in FP32
+ *                                           and over CTAs in index order in
+ *                                           double: deterministic on a device).
+ * The backward needs `workspace` (device memory, 16-byte aligned, owned by the
+ * caller) of at least coat_rmsnorm_fp8_workspace_size(d) bytes; calls that
+ * share a workspace must be ordered on one stream.  rows == 0 writes dw = 0.
+ * Requirements: d a multiple of 128 and at most 8192 (COAT_ERR_UNSUPPORTED
+ * otherwise); eps finite and > 0; w 16-byte aligned; code and bf16 arrays as
+ * for the SwiGLU calls; dw 4-byte aligned.
+ * ------------------------------------------------------------------------- */
+coat_status coat_rmsnorm_fp8_forward(const coat_fp8_act *x, const uint16_t *w, int64_t rows,
+                                     int64_t d, float eps, coat_fmt fmt, int expand_out,
+                                     const coat_fp8_act *out, cudaStream_t stream);
+coat_status coat_rmsnorm_fp8_workspace_size(int64_t d, size_t *bytes);
+coat_status coat_rmsnorm_fp8_backward(const uint16_t *dy, int64_t ld_dy, const coat_fp8_act *x,
+                                      const uint16_t *w, int64_t rows, int64_t d, float eps,
+                                      coat_fmt fmt, uint16_t *dx, int64_t ld_dx, float *dw,
+                                      void *workspace, size_t workspace_bytes,
+                                      cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Device error word.  Kernels that wait on a shared-memory barrier give up
  * after a bounded time (about one second), set a flag and return;
  * coat_check_device_error synchronises `stream`, reads and clears the flag,

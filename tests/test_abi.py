@@ -145,6 +145,29 @@ def test_swiglu_validation():
     assert bwd(cols=40) == UNSUPPORTED
 
 
+def test_rmsnorm_validation():
+    L = coat.lib()
+    act = lambda **k: coat.Fp8Act(k.get("q", A), k.get("s", A), k.get("k", A), k.get("ldq", 4096),
+                                  k.get("lds", 32))
+    fwd = lambda x=None, o=None, w=A, rows=4, d=4096, eps=1e-6, fmt=0, ex=0: \
+        L.coat_rmsnorm_fp8_forward(ctypes.byref(x or act()), w, rows, d, eps, fmt, ex,
+                                   ctypes.byref(o or act()), None)
+    assert fwd(d=4000) == UNSUPPORTED and "multiple of 128" in coat.coat_last_error()
+    assert fwd(d=8192 + 128, x=act(ldq=8320, lds=65), o=act(ldq=8320, lds=65)) == UNSUPPORTED
+    assert fwd(eps=0.0) == INVALID and fwd(eps=float("nan")) == INVALID
+    assert fwd(w=None) == INVALID and fwd(w=A + 2) == MISALIGNED
+    assert fwd(fmt=5) == INVALID and fwd(ex=3) == INVALID and fwd(rows=-1) == INVALID
+    assert fwd(x=act(q=A + 4)) == MISALIGNED and fwd(o=act(lds=8)) == INVALID
+    assert fwd(rows=0) == OK
+    n = ctypes.c_size_t(7)
+    assert L.coat_rmsnorm_fp8_workspace_size(4000, ctypes.byref(n)) == UNSUPPORTED and n.value == 0
+    assert L.coat_rmsnorm_fp8_workspace_size(4096, None) == INVALID
+    bwd = lambda dy=A, dx=A, dw=A, ws=A, wsb=1 << 30, rows=4: L.coat_rmsnorm_fp8_backward(
+        dy, 4096, ctypes.byref(act()), A, rows, 4096, 1e-6, 0, dx, 4096, dw, ws, wsb, None)
+    assert bwd(dy=None) == INVALID and "dy" in coat.coat_last_error()
+    assert bwd(dx=A + 2) == MISALIGNED and bwd(dw=None) == INVALID and bwd(dw=A + 2) == MISALIGNED
+
+
 def test_selftest_budget_validation():
     L = coat.lib()
     assert L.coat_selftest_wait_timeout(999, None) == INVALID
