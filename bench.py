@@ -844,6 +844,175 @@ def run_swiglu(args, ws, rank, local):
     return result
 
 
+RMSNORM_METRIC = ("GB/s of the FP8 RMSNorm layer (forward + backward, FP8 1x128 in/out); "
+                  "HBM GB/s as % of B200 roofline")
+RMSNORM_SHAPE = (8192, 4096)   # tokens x Llama-2-7B hidden size
+RMSNORM_EPS = 1e-6
+
+
+def rmsnorm_bytes(rows, d):
+    """Algorithmic bytes: forward = codes in and out (2 B per element) + 16 B of
+    scale / k per group + the bf16 weight; backward = dy in, codes in, dx out
+    (5 B per element) + 8 B per group + the weight and the FP32 dw."""
+    groups = rows * -(-d // 128)
+    return 2 * rows * d + 16 * groups + 2 * d, 5 * rows * d + 8 * groups + 6 * d
+
+
+def run_rmsnorm(args, ws, rank, local):
+    import torch
+    import fp8_optimizer_state_b200 as coat
+    import synth
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    coat.lib()
+    E4M3 = 0
+    T, d = RMSNORM_SHAPE
+    ng = d // 128
+    w = torch.empty(d, dtype=torch.bfloat16, device=dev)
+    synth.device_weight(w.view(torch.int16), rank, 1)
+    w = (w.float() * 5.0 + 1.0).to(torch.bfloat16)      # a norm weight near 1
+    dw = torch.empty(d, dtype=torch.float32, device=dev)
+    wsp = torch.empty(coat.coat_rmsnorm_fp8_workspace_size(d), dtype=torch.uint8, device=dev)
+    # CODEC_COPIES copies of the per-token tensors; step s runs the forward on
+    # copy s and the backward on copy s + 1, so that neither finds its input in L2
+    cps = []
+    for cp in range(CODEC_COPIES):
+        x = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+        synth.device_activations(x.view(torch.int16).view(-1), rank, cp)
+        xa = (torch.empty(T, d, dtype=torch.uint8, device=dev),
+              torch.empty(T, ng, dtype=torch.float32, device=dev),
+              torch.empty(T, ng, dtype=torch.float32, device=dev))
+        coat.coat_group_quantize(x, 1, 128, False, E4M3, *xa)
+        del x
+        dy = torch.empty(T, d, dtype=torch.int16, device=dev)
+        synth.device_grad(dy.view(-1), rank, 9 + cp, 1)
+        cps.append(dict(xa=xa, dy=dy, dx=torch.empty(T, d, dtype=torch.int16, device=dev),
+                        out=(torch.empty(T, d, dtype=torch.uint8, device=dev),
+                             torch.empty(T, ng, dtype=torch.float32, device=dev),
+                             torch.empty(T, ng, dtype=torch.float32, device=dev))))
+    xa, dy, dx, out = cps[0]["xa"], cps[0]["dy"], cps[0]["dx"], cps[0]["out"]
+    fwd = lambda c=cps[0]: coat.coat_rmsnorm_fp8_forward(c["xa"], w, RMSNORM_EPS, E4M3, False,
+                                                         c["out"])
+    bwd = lambda c=cps[0]: coat.coat_rmsnorm_fp8_backward(c["dy"], c["xa"], w, RMSNORM_EPS,
+                                                          E4M3, c["dx"], dw, wsp)
+    nc = len(cps)
+    for i in range(args.warmup):
+        fwd(cps[i % nc])
+        bwd(cps[(i + 1) % nc])
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    props = torch.cuda.get_device_properties(dev)
+    bus = "%08x:%02x:%02x.0" % (int(getattr(props, "pci_domain_id", 0)),
+                                int(getattr(props, "pci_bus_id", 0)),
+                                int(getattr(props, "pci_device_id", 0)))
+    sampler = ClockSampler(bus)
+    sampler.start()
+    time.sleep(0.3)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    barrier(ws, dev)
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        fwd(cps[i % nc])
+        ev[i][1].record(stream)
+        bwd(cps[(i + 1) % nc])
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    barrier(ws, dev)
+    time.sleep(0.2)
+    sampler.stop()
+    f_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in ev), ws, dev)
+    b_ms = max_over_ranks(statistics.mean(e[1].elapsed_time(e[2]) for e in ev), ws, dev)
+    fb, bb = rmsnorm_bytes(T, d)
+    step_ms = f_ms + b_ms
+    value = ws * (fb + bb) / (step_ms * 1e-3) / 1e9
+    peaks = measured_peaks()
+    peak = peaks["hbm_gbs"] if peaks and peaks.get("hbm_gbs") else HBM_FALLBACK_GBS
+    kern = [{"launch": lab, "ms": round(t, 4), "algorithmic_bytes": b,
+             "GB/s": round(b / (t * 1e-3) / 1e9, 1), "frac": round(b / (t * 1e-3) / 1e9 / peak, 4)}
+            for lab, t, b in (("forward", f_ms, fb), ("backward (+ dw reduction)", b_ms, bb))]
+    top = 0 if f_ms >= b_ms else 1
+    roofline = {"bound": "hbm", "achieved": kern[top]["GB/s"], "peak": peak, "unit": "GB/s",
+                "frac": kern[top]["frac"], "traffic": None, "kernel": kern[top]["launch"],
+                "peak_source": "measured" if peaks else "fallback"}
+    clocks = sampler.summary(wall0, wall1)
+
+    e2e = None
+    if not args.no_e2e:
+        # H2D of the FP8 x (codes, scale, k) and dy from pinned memory, forward +
+        # backward, D2H of the FP8 output, dx and dw
+        ins = (*xa, dy)
+        outs = (*out, dx, dw)
+        hin = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in ins]
+        hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+        for h, t in zip(hin, ins):
+            h.copy_(t)
+        torch.cuda.synchronize()
+        steps = max(1, min(args.steps, args.e2e_steps))
+        barrier(ws, dev)
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            for h, t in zip(hin, ins):
+                t.copy_(h, non_blocking=True)
+            fwd()
+            bwd()
+            for h, t in zip(hout, outs):
+                h.copy_(t, non_blocking=True)
+        torch.cuda.synchronize()
+        el = max_over_ranks(time.perf_counter() - t0, ws, dev)
+        e2e = {"value": round(ws * (fb + bb) * steps / el / 1e9, 3), "unit": "GB/s",
+               "h2d_bytes_per_step": sum(h.numel() * h.element_size() for h in hin),
+               "d2h_bytes_per_step": sum(h.numel() * h.element_size() for h in hout),
+               "steps": steps,
+               "how": "H2D of the FP8 x and dy from pinned memory, forward + backward, D2H of "
+                      "the FP8 output, dx and dw; host wall clock"}
+    coat.coat_check_device_error()
+    result = None
+    if rank == 0:
+        cpu = None
+        if ws == 1 and not args.no_cpu_baseline:
+            import oracle as orc
+            rows = 32
+            h = tuple(t[:rows].cpu().numpy() for t in xa)
+            wb = w.view(torch.int16).cpu().numpy().view(np.uint16)
+            dyb = dy[:rows].cpu().numpy().view(np.uint16)
+            t0 = time.perf_counter()
+            orc.rmsnorm_fp8_forward(h, wb, RMSNORM_EPS, E4M3, False)
+            orc.rmsnorm_fp8_backward(dyb, h, wb, RMSNORM_EPS, E4M3)
+            el = time.perf_counter() - t0
+            sb = sum(rmsnorm_bytes(rows, d))
+            cpu = {"value": round(sb / el / 1e9, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                   "sample": "first %d token rows, forward + backward, one host thread (%.2f s)"
+                             % (rows, el)}
+        result = {
+            "metric": RMSNORM_METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": "FP8 RMSNorm layer, %d tokens x %d (Llama-2-7B hidden size): "
+                                   "x E4M3 1x128 (N(0,1) activations with 0.1%% x100 outliers), "
+                                   "bf16 weight near 1, E4M3 1x128 output without expansion, "
+                                   "bf16 dy / dx, FP32 dw" % (T, d),
+                       "l2": "inputs not in L2: %d copies of the per-token tensors, the forward "
+                             "of step s on copy s, the backward on copy s+1 (%.0f MB forward + "
+                             "%.0f MB backward per step)" % (CODEC_COPIES, fb / 1e6, bb / 1e6),
+                       "parallelism": "single GPU" if ws == 1 else "replicas%d" % ws},
+            "launches": kern, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": 3 * args.steps, "clocks": clocks}
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return result
+
+
 def run_reference(args, cfg, ws, rank):
     """The CPU oracle on a bounded sample per step (one host thread)."""
     if rank != 0:
@@ -874,7 +1043,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="llama2-7b",
-                    choices=sorted(CONFIGS) + ["act-codec", "swiglu-fp8"])
+                    choices=sorted(CONFIGS) + ["act-codec", "swiglu-fp8", "rmsnorm-fp8"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -890,12 +1059,13 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     ws, rank, local = dist_env()
-    if args.config in ("act-codec", "swiglu-fp8"):
+    if args.config in ("act-codec", "swiglu-fp8", "rmsnorm-fp8"):
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable": "this workload has no "
                               "reference arm; the oracle CPU baseline is in the ours line"}))
             return
-        run = run_codec if args.config == "act-codec" else run_swiglu
+        run = {"act-codec": run_codec, "swiglu-fp8": run_swiglu,
+               "rmsnorm-fp8": run_rmsnorm}[args.config]
         res = run(args, ws, rank, local)
         if res is not None:
             print(json.dumps(res), flush=True)

@@ -404,10 +404,10 @@ __device__ __forceinline__ void bf16x16(const uint4& a, const uint4& b, float (&
 template <int FMT, bool EXPAND>
 __device__ __forceinline__ void quantize_scaled16(const float (&p)[16], float C, uint32_t (&cw)[4],
                                                   float& k, float& sr) {
-  float y[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) y[i] = p[i] * C;
   if (EXPAND) {
+    float y[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) y[i] = p[i] * C;
     quantize_lane16<FMT, true>(y, false, cw, k, sr);
     return;
   }
@@ -419,6 +419,9 @@ __device__ __forceinline__ void quantize_scaled16(const float (&p)[16], float C,
   const float My = mp * C;
   const bool special = !(mp <= 3.40282347e38f) || !(My <= 3.40282347e38f) || !(C > 0.0f);
   if (__any_sync(0xFFFFFFFFu, special)) {
+    float y[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) y[i] = p[i] * C;
     quantize_lane16<FMT, false>(y, special, cw, k, sr);
     return;
   }
@@ -452,19 +455,32 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_fwd_kernel(const ActArgs
       for (int i = 0; i < 16; ++i) wv[j][i] = 0.0f;
     }
   }
+  // the next row's codes and metadata are loaded before this row's reduction
+  struct In { uint4 q; float s, k; };
+  auto load = [&](int64_t r, In (&in)[CPT]) {
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+      const int64_t c = (threadIdx.x + int64_t(j) * kNormThreads) * 16;
+      in[j].q = make_uint4(0u, 0u, 0u, 0u);
+      in[j].s = in[j].k = 1.0f;
+      if (ok[j]) {
+        in[j].q = __ldcs(reinterpret_cast<const uint4*>(x.q + r * x.ldq + c));
+        in[j].s = __ldg(x.scale + r * x.lds + (c >> 7));
+        in[j].k = __ldg(x.k + r * x.lds + (c >> 7));
+      }
+    }
+  };
+  In cur[CPT];
+  if (blockIdx.x < rows) load(blockIdx.x, cur);
   for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    In nxt[CPT];
+    if (r + gridDim.x < rows) load(r + gridDim.x, nxt);
     float pv[CPT][16], sv[CPT];
     float ss[1] = {0.0f};
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
-      const int64_t c = (threadIdx.x + int64_t(j) * kNormThreads) * 16;
-      uint4 q = make_uint4(0u, 0u, 0u, 0u);
-      float s = 1.0f, k = 1.0f;
-      if (ok[j]) {
-        q = __ldg(reinterpret_cast<const uint4*>(x.q + r * x.ldq + c));
-        s = __ldg(x.scale + r * x.lds + (c >> 7));
-        k = __ldg(x.k + r * x.lds + (c >> 7));
-      }
+      const uint4 q = cur[j].q;
+      const float s = cur[j].s, k = cur[j].k;
       const bool plain = __all_sync(0xFFFFFFFFu, k == 1.0f);
       float f[16];
       decode16_raw<FMT>(q, k, plain, tab, f);
@@ -493,6 +509,8 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_fwd_kernel(const ActArgs
         }
       }
     }
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) cur[j] = nxt[j];
   }
 }
 
@@ -526,39 +544,55 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_bwd_kernel(
       for (int i = 0; i < 16; ++i) wv[j][i] = 0.0f;
     }
   }
-  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-    float xv[CPT][16], dv[CPT][16];
-    float sums[2] = {0.0f, 0.0f};   // sum x^2, sum g x
+  // the next row's codes, scales and dy are loaded before this row's reduction
+  struct In { uint4 q, d0, d1; float s, k; };
+  auto load = [&](int64_t r, In (&in)[CPT]) {
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
       const int64_t c = (threadIdx.x + int64_t(j) * kNormThreads) * 16;
-      uint4 q = make_uint4(0u, 0u, 0u, 0u), d0 = q, d1 = q;
-      float s = 1.0f, k = 1.0f;
+      in[j].q = in[j].d0 = in[j].d1 = make_uint4(0u, 0u, 0u, 0u);
+      in[j].s = in[j].k = 1.0f;
       if (ok[j]) {
-        q = __ldcs(reinterpret_cast<const uint4*>(x.q + r * x.ldq + c));
-        s = __ldg(x.scale + r * x.lds + (c >> 7));
-        k = __ldg(x.k + r * x.lds + (c >> 7));
+        in[j].q = __ldcs(reinterpret_cast<const uint4*>(x.q + r * x.ldq + c));
+        in[j].s = __ldg(x.scale + r * x.lds + (c >> 7));
+        in[j].k = __ldg(x.k + r * x.lds + (c >> 7));
         const uint4* dp = reinterpret_cast<const uint4*>(dy + r * lddy + c);
-        d0 = __ldcs(dp);
-        d1 = __ldcs(dp + 1);
+        in[j].d0 = __ldcs(dp);
+        in[j].d1 = __ldcs(dp + 1);
       }
-      const bool plain = __all_sync(0xFFFFFFFFu, k == 1.0f);
-      float f[16];
-      decode16_raw<FMT>(q, k, plain, tab, f);
-      bf16x16(d0, d1, dv[j]);
+    }
+  };
+  In cur[CPT];
+  if (blockIdx.x < rows) load(blockIdx.x, cur);
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    In nxt[CPT];
+    if (r + gridDim.x < rows) load(r + gridDim.x, nxt);
+    // pass 1: the row sums; the decoded values are not kept across the barrier
+    float sums[2] = {0.0f, 0.0f};   // sum x^2, sum g x
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) {
+      const bool plain = __all_sync(0xFFFFFFFFu, cur[j].k == 1.0f);
+      float f[16], dv[16];
+      decode16_raw<FMT>(cur[j].q, cur[j].k, plain, tab, f);
+      bf16x16(cur[j].d0, cur[j].d1, dv);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        xv[j][i] = f[i] * s;
-        sums[0] = __fmaf_rn(xv[j][i], xv[j][i], sums[0]);
-        sums[1] = __fmaf_rn(dv[j][i] * wv[j][i], xv[j][i], sums[1]);
+        const float xv = f[i] * cur[j].s;
+        sums[0] = __fmaf_rn(xv, xv, sums[0]);
+        sums[1] = __fmaf_rn(dv[i] * wv[j][i], xv, sums[1]);
       }
     }
     cta_sum_all(sums, red);
     const float rstd = 1.0f / sqrtf(__fmaf_rn(sums[0], inv_d, eps));
     // rstd^2 mean(g xh) = rstd^3 sum(g x) / d
     const float cx = rstd * rstd * rstd * sums[1] * inv_d;
+    // pass 2: dx and the dw sums, decoding again
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
+      const bool plain = __all_sync(0xFFFFFFFFu, cur[j].k == 1.0f);
+      float f[16], dv[16];
+      decode16_raw<FMT>(cur[j].q, cur[j].k, plain, tab, f);
+      bf16x16(cur[j].d0, cur[j].d1, dv);
       uint32_t o[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -566,9 +600,10 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_bwd_kernel(
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int i = 2 * e + h;
-          const float g = dv[j][i] * wv[j][i];
-          a[h] = __fmaf_rn(rstd, g, -cx * xv[j][i]);
-          acc[j][i] = __fmaf_rn(dv[j][i], xv[j][i] * rstd, acc[j][i]);
+          const float xv = f[i] * cur[j].s;
+          const float g = dv[i] * wv[j][i];
+          a[h] = __fmaf_rn(rstd, g, -cx * xv);
+          acc[j][i] = __fmaf_rn(dv[i], xv * rstd, acc[j][i]);
         }
         o[e] = pack_bf16x2(a[0], a[1]);
       }
@@ -579,6 +614,8 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_bwd_kernel(
         op[1] = make_uint4(o[4], o[5], o[6], o[7]);
       }
     }
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) cur[j] = nxt[j];
   }
 #pragma unroll
   for (int j = 0; j < CPT; ++j) {
@@ -591,15 +628,42 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_bwd_kernel(
   }
 }
 
-// dw[c] = sum over the nparts rows of partial[., c], in row order, in double.
-__global__ void __launch_bounds__(kNormThreads) rmsnorm_dw_kernel(const float* __restrict__ partial,
-                                                                  int nparts, int64_t d,
-                                                                  float* __restrict__ dw) {
-  const int64_t c = blockIdx.x * int64_t(kNormThreads) + threadIdx.x;
-  if (c >= d) return;
+// dw[c] = sum over the nparts rows of partial[., c] in double, in a fixed
+// order: a 1024-thread CTA takes 32 columns; warp w adds rows w, w + 32, ...
+// (coalesced 128-byte reads, four loads in flight), then warp 0 adds the 32
+// warp sums.
+constexpr int kDwCols = 32;
+constexpr int kDwThreads = 1024;
+__global__ void __launch_bounds__(kDwThreads) rmsnorm_dw_kernel(const float* __restrict__ partial,
+                                                                int nparts, int64_t d,
+                                                                float* __restrict__ dw) {
+  constexpr int kWarps = kDwThreads / 32;
+  __shared__ double red[kWarps][kDwCols];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t c = blockIdx.x * int64_t(kDwCols) + lane;
   double t = 0.0;
-  for (int p = 0; p < nparts; ++p) t += static_cast<double>(__ldg(partial + p * d + c));
-  dw[c] = static_cast<float>(t);
+  if (c < d) {
+    int p = warp;
+    for (; p + 3 * kWarps < nparts; p += 4 * kWarps) {
+      const float a0 = __ldg(partial + int64_t(p) * d + c);
+      const float a1 = __ldg(partial + int64_t(p + kWarps) * d + c);
+      const float a2 = __ldg(partial + int64_t(p + 2 * kWarps) * d + c);
+      const float a3 = __ldg(partial + int64_t(p + 3 * kWarps) * d + c);
+      t += static_cast<double>(a0);
+      t += static_cast<double>(a1);
+      t += static_cast<double>(a2);
+      t += static_cast<double>(a3);
+    }
+    for (; p < nparts; p += kWarps) t += static_cast<double>(__ldg(partial + int64_t(p) * d + c));
+  }
+  red[warp][lane] = t;
+  __syncthreads();
+  if (warp == 0 && c < d) {
+    double s = 0.0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) s += red[w][lane];
+    dw[c] = static_cast<float>(s);
+  }
 }
 
 template <int FMT>
@@ -643,8 +707,8 @@ cudaError_t rms_bwd_launch(const uint16_t* dy, int64_t lddy, const ActArgs& x, c
   kern<<<g, kNormThreads, 0, s>>>(dy, lddy, x, w, rows, d, eps, dx, lddx, partial);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  rmsnorm_dw_kernel<<<static_cast<unsigned>((d + kNormThreads - 1) / kNormThreads), kNormThreads,
-                      0, s>>>(partial, static_cast<int>(g), d, dw);
+  rmsnorm_dw_kernel<<<static_cast<unsigned>((d + kDwCols - 1) / kDwCols), kDwThreads, 0, s>>>(
+      partial, static_cast<int>(g), d, dw);
   return cudaGetLastError();
 }
 
