@@ -16,8 +16,8 @@ from tests.parity import bf16_rne_bits, check_master, check_state_all
 pytestmark = pytest.mark.gpu
 
 
-def _build(fm, fv, step):
-    cfg = CONFIGS["llama2-7b"]
+def _build(fm, fv, step, config="llama2-7b"):
+    cfg = CONFIGS[config]
     ps = DeviceParamSet(cfg["shapes"](), seed=0)
     ps.fill_master()
     ps.fill_grad(step)
@@ -159,6 +159,36 @@ def test_llama2_7b_grad_norm_and_clipped_step_full_size(orc):
         coat.coat_check_device_error()
         post = [_grab(ps, i, gi) for i, gi in samples]
         _check_samples(orc, samples, post, step, fm, fv, gscale=coef)
+        plan.destroy()
+    finally:
+        del ps
+        torch.cuda.empty_cache()
+
+
+def test_llama2_13b_full_size_sampled(orc):
+    """The 13B-shaped list (363 tensors, 1.30e10 parameters, E4M3 m and v; about
+    132 GB resident) in one multi-tensor launch, sampled groups against the
+    oracle and the per-element properties."""
+    cfg = CONFIGS["llama2-13b"]
+    fm, fv = cfg["fmt_m"], cfg["fmt_v"]
+    step = 1
+    ps = _build(fm, fv, step, "llama2-13b")
+    try:
+        plan = coat.coat_multi_plan_create([_desc(ps, i) for i in range(len(ps))], fm, fv)
+        assert plan.info() == (13015864320, 363)
+        samples = _samples(ps, 53)
+        torch.cuda.synchronize()
+        coat.coat_adamw_step_multi(plan, step=step,
+                                   **{k: H[k] for k in ("lr", "beta1", "beta2", "eps", "wd")})
+        coat.coat_check_device_error()
+        post = [_grab(ps, i, gi) for i, gi in samples]
+        _check_samples(orc, samples, post, step, fm, fv)
+        for k in (ps.mk, ps.vk):
+            assert bool(((k >= 1) & (k <= 16)).all())
+        for s_ in (ps.ms, ps.vs):
+            assert bool((torch.isfinite(s_) & (s_ > 0)).all())
+        for i in range(len(ps)):      # per tensor: a whole-array temporary would not fit
+            assert bool(torch.isfinite(ps.views(i)["master"]).all()), i
         plan.destroy()
     finally:
         del ps
