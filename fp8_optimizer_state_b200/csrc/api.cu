@@ -171,7 +171,7 @@ extern "C" {
 
 const char* coat_last_error(void) { return g_last_error.c_str(); }
 
-int coat_version(void) { return 10000; }
+int coat_version(void) { return 10300; }   // 1.3: clipping pre-step, FP8 SwiGLU and RMSNorm layers
 
 coat_status coat_fp8_encode(const float* y, int64_t n, coat_fmt fmt, uint8_t* q, cudaStream_t stream) {
   if (n < 0) return fail(COAT_ERR_INVALID_ARG, "coat_fp8_encode: n < 0");
