@@ -185,6 +185,57 @@ __device__ __forceinline__ void quantize_lane16(const float (&h)[16], bool force
   }
 }
 
+// Quantise y = p C (C > 0, one value per group) from a lane's 16 values p of
+// an 8-lane 1x128 group.  Without expansion the codes are decided on the
+// ratio |p_i| / max|p| = |y_i| / max|y| (C cancels, so y itself is never
+// rounded); the root scale is max|y| / FMT_MAX.  EXACT: the ratio as one
+// correctly rounded division (for exact p an exact tie of the real-number
+// result stays a tie and is broken to even, as the oracle does); otherwise
+// one multiply by FMT_MAX / max|p| (a few ulps; for p that are not exact
+// anyway).  With expansion, and for groups with a NaN/Inf, a maximum below
+// 2^-64 or an unusable C, the values y go through quantize_lane16.
+template <int FMT, bool EXPAND, bool EXACT>
+__device__ __forceinline__ void quantize_scaled16(const float (&p)[16], float C, uint32_t (&cw)[4],
+                                                  float& k, float& sr) {
+  if (EXPAND) {
+    float y[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) y[i] = p[i] * C;
+    quantize_lane16<FMT, true>(y, false, cw, k, sr);
+    return;
+  }
+  float mp = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) mp = fmax_nan(mp, fabsf(p[i]));
+#pragma unroll
+  for (int off = 1; off < 8; off <<= 1) mp = fmax_nan(mp, __shfl_xor_sync(0xFFFFFFFFu, mp, off));
+  const float My = mp * C;
+  const bool special = !(mp <= 3.40282347e38f) || !(My <= 3.40282347e38f) || !(C > 0.0f) ||
+                       (mp > 0.0f && mp < 5.421010862427522e-20f);
+  if (__any_sync(0xFFFFFFFFu, special)) {
+    float y[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) y[i] = p[i] * C;
+    quantize_lane16<FMT, false>(y, special, cw, k, sr);
+    return;
+  }
+  k = 1.0f;
+  sr = My > 0.0f ? __fdiv_rn(My, F8<FMT>::MAXV) : 1.0f;
+  if (EXACT) {
+    const GroupDiv dv = codec_div<FMT>(mp);
+    encode_words<FMT, 16, true>(p, true, dv, 0.0f, 1.0f, cw);
+  } else {
+    const float c = mp > 0.0f ? F8<FMT>::MAXV * rcp_approx(mp) : 0.0f;
+    uint32_t mag[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) mag[i] = enc_mag_bounded<FMT>(fabsf(p[i]) * c);
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+      cw[w] = merge_signs4(pack4(mag[4 * w], mag[4 * w + 1], mag[4 * w + 2], mag[4 * w + 3]),
+                           p[4 * w], p[4 * w + 1], p[4 * w + 2], p[4 * w + 3]);
+  }
+}
+
 // One lane's forward work item: 16 gate and 16 up codes, their groups'
 // metadata, and the item's row and the lane's first column.
 struct FwdItem {
@@ -196,8 +247,9 @@ struct FwdItem {
 };
 
 // h = silu(g) u with g = f_g s_g, u = f_u s_u, as ((f_g f_u) sigmoid(g)) (s_g s_u):
-// f_g f_u is exact for k = 1 inputs (two FP8 significands), so h takes two
-// roundings besides the sigmoid's; h is then quantised by quantize_lane16.
+// f_g f_u is exact for k = 1 inputs (two FP8 significands); h / (s_g s_u) takes
+// one rounding besides the sigmoid's and is quantised with the group's scale
+// product by quantize_scaled16 (the product cancels from the codes).
 // EXPAND: output expansion on.
 // Work: the rows x ceil(groups/4) items (4 groups of a row, 8 lanes each) in
 // row-major order, a contiguous range per warp (columns advanced by 512 with
@@ -255,13 +307,12 @@ __global__ void __launch_bounds__(256) swiglu_fwd_kernel(const ActArgs gate, con
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const float sg = rcp_approx(1.0f + ex2_approx(fg[i] * ct));
-      h[i] = ((fg[i] * fu[i]) * sg) * S;
+      h[i] = (fg[i] * fu[i]) * sg;   // h / (s_g s_u)
     }
 
-    // slow path also when the scale product overflowed
     uint32_t cw[4];
     float k, sr;
-    quantize_lane16<FMT, EXPAND>(h, !(S <= 3.40282347e38f), cw, k, sr);
+    quantize_scaled16<FMT, EXPAND, false>(h, S, cw, k, sr);
     if (cur.valid) {
       *reinterpret_cast<uint4*>(out.q + cur.r * out.ldq + cur.c) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
       if (l == 0) {
@@ -393,44 +444,6 @@ __device__ __forceinline__ void bf16x16(const uint4& a, const uint4& b, float (&
   }
 }
 
-// Quantise y = p C (C > 0, one value per group) from a lane's 16 values p of
-// an 8-lane 1x128 group.  Without expansion the codes are decided on the
-// ratio |p_i| / max|p| = |y_i| / max|y| (C cancels), as one correctly rounded
-// division: for k = 1 inputs p_i = (FP8 value) x (bf16 weight) is exact, so an
-// exact tie of the real-number result stays a tie and is broken to even, as
-// the oracle does; the root scale is max|y| / FMT_MAX.  With expansion, and
-// for groups with a NaN/Inf or an unusable C, the values y go through
-// quantize_lane16.
-template <int FMT, bool EXPAND>
-__device__ __forceinline__ void quantize_scaled16(const float (&p)[16], float C, uint32_t (&cw)[4],
-                                                  float& k, float& sr) {
-  if (EXPAND) {
-    float y[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) y[i] = p[i] * C;
-    quantize_lane16<FMT, true>(y, false, cw, k, sr);
-    return;
-  }
-  float mp = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) mp = fmax_nan(mp, fabsf(p[i]));
-#pragma unroll
-  for (int off = 1; off < 8; off <<= 1) mp = fmax_nan(mp, __shfl_xor_sync(0xFFFFFFFFu, mp, off));
-  const float My = mp * C;
-  const bool special = !(mp <= 3.40282347e38f) || !(My <= 3.40282347e38f) || !(C > 0.0f);
-  if (__any_sync(0xFFFFFFFFu, special)) {
-    float y[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) y[i] = p[i] * C;
-    quantize_lane16<FMT, false>(y, special, cw, k, sr);
-    return;
-  }
-  k = 1.0f;
-  sr = My > 0.0f ? __fdiv_rn(My, F8<FMT>::MAXV) : 1.0f;
-  const GroupDiv dv = codec_div<FMT>(mp);
-  encode_words<FMT, 16, true>(p, true, dv, 0.0f, 1.0f, cw);
-}
-
 template <int FMT, bool EXPAND, int CPT>
 __global__ void __launch_bounds__(kNormThreads) rmsnorm_fwd_kernel(const ActArgs x,
                                                                    const uint16_t* __restrict__ w,
@@ -499,7 +512,7 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_fwd_kernel(const ActArgs
     for (int j = 0; j < CPT; ++j) {
       uint32_t cw[4];
       float k, sr;
-      quantize_scaled16<FMT, EXPAND>(pv[j], sv[j] * rstd, cw, k, sr);
+      quantize_scaled16<FMT, EXPAND, true>(pv[j], sv[j] * rstd, cw, k, sr);
       if (ok[j]) {
         const int64_t c = (threadIdx.x + int64_t(j) * kNormThreads) * 16;
         *reinterpret_cast<uint4*>(out.q + r * out.ldq + c) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
