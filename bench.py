@@ -74,6 +74,15 @@ def algorithmic_bytes(sizes, with_weight=True):
 # ----------------------------------------------------------------------------
 # clocks during the timed region
 # ----------------------------------------------------------------------------
+def pci_bus_id(dev):
+    """The device's PCI bus id as nvidia-smi prints it (for the clock sampler)."""
+    import torch
+    props = torch.cuda.get_device_properties(dev)
+    return "%08x:%02x:%02x.0" % (int(getattr(props, "pci_domain_id", 0)),
+                                 int(getattr(props, "pci_bus_id", 0)),
+                                 int(getattr(props, "pci_device_id", 0)))
+
+
 class ClockSampler:
     FIELDS = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -311,11 +320,7 @@ def run_ours(args, cfg, ws, rank, local):
     torch.cuda.synchronize()
     coat.coat_check_device_error()
 
-    props = torch.cuda.get_device_properties(dev)
-    bus = "%08x:%02x:%02x.0" % (int(getattr(props, "pci_domain_id", 0)),
-                                int(getattr(props, "pci_bus_id", 0)),
-                                int(getattr(props, "pci_device_id", 0)))
-    sampler = ClockSampler(bus)
+    sampler = ClockSampler(pci_bus_id(dev))
     sampler.start()
     time.sleep(0.3)
     ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3))
@@ -581,11 +586,7 @@ def run_codec(args, ws, rank, local):
             n_launch += 1
     torch.cuda.synchronize()
     coat.coat_check_device_error()
-    props = torch.cuda.get_device_properties(dev)
-    bus = "%08x:%02x:%02x.0" % (int(getattr(props, "pci_domain_id", 0)),
-                                int(getattr(props, "pci_bus_id", 0)),
-                                int(getattr(props, "pci_device_id", 0)))
-    sampler = ClockSampler(bus)
+    sampler = ClockSampler(pci_bus_id(dev))
     sampler.start()
     time.sleep(0.3)
     ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -738,11 +739,7 @@ def run_swiglu(args, ws, rank, local):
         bwd()
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
-    props = torch.cuda.get_device_properties(dev)
-    bus = "%08x:%02x:%02x.0" % (int(getattr(props, "pci_domain_id", 0)),
-                                int(getattr(props, "pci_bus_id", 0)),
-                                int(getattr(props, "pci_device_id", 0)))
-    sampler = ClockSampler(bus)
+    sampler = ClockSampler(pci_bus_id(dev))
     sampler.start()
     time.sleep(0.3)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
@@ -906,11 +903,7 @@ def run_rmsnorm(args, ws, rank, local):
         bwd(cps[(i + 1) % nc])
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
-    props = torch.cuda.get_device_properties(dev)
-    bus = "%08x:%02x:%02x.0" % (int(getattr(props, "pci_domain_id", 0)),
-                                int(getattr(props, "pci_bus_id", 0)),
-                                int(getattr(props, "pci_device_id", 0)))
-    sampler = ClockSampler(bus)
+    sampler = ClockSampler(pci_bus_id(dev))
     sampler.start()
     time.sleep(0.3)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
