@@ -233,3 +233,46 @@ def test_norm_then_clipped_step_vs_oracle_chain(orc):
         check_state_all("m", n, 0, h["mq"], h["ms"], h["mk"], o.mq, o.ms, o.mk)
         check_state_all("v", n, 1, h["vq"], h["vs"], h["vk"], o.vq, o.vs, o.vk)
     plan.destroy()
+
+
+def test_clipped_step_replays_from_a_cuda_graph():
+    """Norm pass and clipped step enqueue no host round trip, so one training
+    step's pair of launches can be captured once and replayed; two replays give
+    the bytes of two eager steps."""
+    sizes = [5000, 70001, 129, 7680 * 2]
+    a = make_sides(sizes, 0, 1)
+    b = make_sides(sizes, 0, 1)
+    pa, pb = plan_of(a, 0, 1), plan_of(b, 0, 1)
+    grads = grads_of(sizes, 1)
+    load_grads(a, grads)
+    load_grads(b, grads)
+    ra, rb = coat.new_grad_clip(), coat.new_grad_clip()
+    # eager: two steps on side a (the first call of each entry point also
+    # configures its kernels, which a capture must not be the first to do)
+    for t in (1, 2):
+        pa.grad_norm(0.5, ra)
+        coat.coat_adamw_step_multi_clipped(pa, ra, step=t, **HK)
+    torch.cuda.synchronize()
+    # captured: the same step number both times (the step count is a launch argument)
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        pb.grad_norm(0.5, rb)
+        coat.coat_adamw_step_multi_clipped(pb, rb, step=1, **HK)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        pb.grad_norm(0.5, rb)
+        coat.coat_adamw_step_multi_clipped(pb, rb, step=2, **HK)
+    g.replay()
+    torch.cuda.synchronize()
+    coat.coat_check_device_error()
+    for sa, sb in zip(a, b):
+        ha, hb = sa.host(), sb.host()
+        for key in ("master", "weight", "mq", "ms", "mk", "vq", "vs", "vk"):
+            assert np.array_equal(ha[key], hb[key]), key
+    assert torch.equal(ra, rb)
+    del g
+    pa.destroy()
+    pb.destroy()
