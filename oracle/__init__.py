@@ -1,4 +1,6 @@
-"""CPU oracle for the COAT FP8-optimizer-state AdamW step (test infrastructure).
+"""CPU oracle for the COAT FP8-optimizer-state AdamW step, its FP8 codec, the
+gradient-clipping pre-step and the FP8 SwiGLU and RMSNorm layers (test
+infrastructure).
 
 Plain double-precision C (``coat_oracle.c``) behind a small ctypes loader.
 Only the test-suite, ``__graft_entry__.smoke()`` and the benchmark's CPU
