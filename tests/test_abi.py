@@ -168,6 +168,26 @@ def test_rmsnorm_validation():
     assert bwd(dx=A + 2) == MISALIGNED and bwd(dw=None) == INVALID and bwd(dw=A + 2) == MISALIGNED
 
 
+def test_header_compiles_as_c99(tmp_path):
+    """include/coat.h is a C header: a C99 translation unit that includes it and
+    takes the address of every entry point compiles."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    cuda_inc = "/usr/local/cuda/include"
+    if gcc is None or not os.path.exists(os.path.join(cuda_inc, "cuda_runtime_api.h")):
+        pytest.skip("gcc or the CUDA headers are not available")
+    names = declared_functions()
+    src = tmp_path / "use_coat.c"
+    src.write_text('#include "coat.h"\n' + "typedef void (*entry)(void);\n" +
+                   "entry entry_points[] = {\n" + ",\n".join("  (entry)%s" % n for n in names) +
+                   "\n};\nint main(void) { return entry_points[0] == 0; }\n")
+    p = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-fsyntax-only",
+                        "-I", os.path.join(ROOT, "include"), "-isystem", cuda_inc, str(src)],
+                       capture_output=True, text=True)
+    assert p.returncode == 0, p.stderr
+
+
 def test_selftest_budget_validation():
     L = coat.lib()
     assert L.coat_selftest_wait_timeout(999, None) == INVALID

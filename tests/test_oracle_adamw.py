@@ -176,6 +176,18 @@ def test_grad_sumsq_closed_forms(orc):
         assert orc.grad_sumsq(_bf16([1.0, bad, 2.0]))[1] is True
 
 
+def test_grad_sumsq_matches_numpy_on_random_bf16(orc):
+    """The sum of squares of 100,000 bf16 values against numpy's float64 dot
+    product (a library routine; squares of bf16 values are exact in double)."""
+    rng = np.random.default_rng(11)
+    x = (rng.standard_normal(100000) * np.exp(rng.uniform(-20, 20, 100000))).astype(np.float32)
+    bits = (x.view(np.uint32) >> 16).astype(np.uint16)       # truncation: any bf16 will do
+    vals = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    s, bad = orc.grad_sumsq(bits)
+    assert not bad
+    assert abs(s - float(np.dot(vals, vals))) <= 1e-12 * s
+
+
 def test_clip_coef_closed_forms(orc):
     # norm 5: max_norm / (norm + 1e-6), rounded to FP32, when below 1
     assert orc.clip_coef(25.0, 1.0) == np.float32(1.0 / (5.0 + 1e-6))
