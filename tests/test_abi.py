@@ -241,3 +241,29 @@ def test_binding_raises_without_fallback():
     with pytest.raises(coat.CoatError) as ei:
         coat._check(step(group=64))
     assert ei.value.status == UNSUPPORTED
+
+
+def test_binding_refuses_host_tensors():
+    """The binding passes device pointers only: CPU tensors raise before any
+    call into the library (there is no CPU path)."""
+    import torch
+    q = torch.zeros((2, 128), dtype=torch.uint8)
+    s = torch.ones((2, 1))
+    act = (q, s, s)
+    with pytest.raises(ValueError):
+        coat.coat_swiglu_fp8_forward(act, act, 0, False, act)
+    with pytest.raises(ValueError):
+        coat.coat_rmsnorm_fp8_forward(act, torch.ones(128, dtype=torch.bfloat16), 1e-6, 0, False,
+                                      act)
+    with pytest.raises(ValueError):
+        coat.coat_group_quantize(torch.zeros((2, 128), dtype=torch.bfloat16), 1, 128, False, 0,
+                                 q, s, s)
+
+
+def test_binding_shape_checks():
+    import torch
+    q = torch.zeros((2, 128), dtype=torch.uint8)
+    with pytest.raises(ValueError):
+        coat._act((q, torch.ones(2), torch.ones(2)))              # 1-D scale
+    with pytest.raises(ValueError):
+        coat._act((q.t(), torch.ones((128, 1)), torch.ones((128, 1))))   # rows not contiguous
