@@ -51,6 +51,8 @@ EXPORTS = [
     ("coat_rmsnorm_fp8_workspace_size", _i32, [_i64, ctypes.POINTER(ctypes.c_size_t)]),
     ("coat_rmsnorm_fp8_backward", _i32, [_vp, _i64, _vp, _vp, _i64, _i64, _f32, _i32, _vp, _i64,
                                          _vp, _vp, ctypes.c_size_t, _vp]),
+    ("coat_zero1_layout", _i32, [_vp, _i32, _i32, _i32, _i32, _vp, _i32, ctypes.POINTER(_i32),
+                                 ctypes.POINTER(_i64), ctypes.POINTER(_i64), _vp]),
 ]
 NOALLOC_MAX_TENSORS = 1024
 
@@ -333,6 +335,29 @@ def coat_adamw_step_multi_noalloc(descs, *, lr, beta1, beta2, eps, wd, step, fmt
                                              _s(stream))
     if st != 0:
         raise CoatError(st, "coat_adamw_step_multi_noalloc rejected the call")
+
+
+class ShardPiece(ctypes.Structure):
+    """coat_shard_piece"""
+    _fields_ = [("tensor", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("elem_begin", _i64), ("n_elems", _i64), ("shard_begin", _i64)]
+
+
+def coat_zero1_layout(sizes, world_size, rank, group=GROUP):
+    """ZeRO-1 partition of tensors of `sizes` elements (host-only; no GPU).
+    Returns (pieces, shard_elems, flat_elems, flat_offsets): pieces is this
+    rank's list of (tensor, elem_begin, n_elems, shard_begin) tuples."""
+    n = len(sizes)
+    arr = (_i64 * n)(*[int(x) for x in sizes])
+    offs = (_i64 * n)()
+    pieces = (ShardPiece * n)()
+    cnt, shard, flat = ctypes.c_int(), _i64(), _i64()
+    _check(lib().coat_zero1_layout(ctypes.cast(arr, _vp), n, group, world_size, rank,
+                                   ctypes.cast(pieces, _vp), n, ctypes.byref(cnt),
+                                   ctypes.byref(shard), ctypes.byref(flat),
+                                   ctypes.cast(offs, _vp)))
+    out = [(p.tensor, p.elem_begin, p.n_elems, p.shard_begin) for p in pieces[:cnt.value]]
+    return out, shard.value, flat.value, list(offs)
 
 
 def coat_check_device_error(stream=None):

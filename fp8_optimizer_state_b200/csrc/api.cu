@@ -1,6 +1,7 @@
 // api.cu -- the C ABI declared in include/coat.h: argument validation (before
 // any CUDA call, so a bad call launches nothing and touches nothing), error
 // reporting, multi-tensor plans, and kernel launches on the caller's stream.
+#include <algorithm>
 #include <cmath>
 #include <cstddef>
 #include <limits>
@@ -171,7 +172,7 @@ extern "C" {
 
 const char* coat_last_error(void) { return g_last_error.c_str(); }
 
-int coat_version(void) { return 10300; }   // 1.3: clipping pre-step, FP8 SwiGLU and RMSNorm layers
+int coat_version(void) { return 10400; }   // 1.4: ZeRO-1 layout; 1.3: clipping pre-step, FP8 layers
 
 coat_status coat_fp8_encode(const float* y, int64_t n, coat_fmt fmt, uint8_t* q, cudaStream_t stream) {
   if (n < 0) return fail(COAT_ERR_INVALID_ARG, "coat_fp8_encode: n < 0");
@@ -569,6 +570,60 @@ coat_status coat_multi_plan_info(coat_multi_plan_t plan, int64_t* total_elements
   if (!plan) return fail(COAT_ERR_INVALID_ARG, "coat_multi_plan_info: plan is NULL");
   if (total_elements) *total_elements = plan->total_elements;
   if (num_tensors) *num_tensors = plan->num;
+  return COAT_OK;
+}
+
+coat_status coat_zero1_layout(const int64_t* sizes, int num_tensors, int group, int world_size,
+                              int rank, coat_shard_piece* pieces, int max_pieces,
+                              int* num_pieces, int64_t* shard_elems, int64_t* flat_elems,
+                              int64_t* flat_offsets) {
+  const char* fn = "coat_zero1_layout";
+  if (!sizes || !num_pieces || !shard_elems || !flat_elems)
+    return fail(COAT_ERR_INVALID_ARG, "%s: NULL argument", fn);
+  if (num_tensors < 1) return fail(COAT_ERR_INVALID_ARG, "%s: num_tensors must be >= 1", fn);
+  if (group != 128) return fail(COAT_ERR_UNSUPPORTED, "%s: group %d not supported (128)", fn, group);
+  if (world_size < 1 || rank < 0 || rank >= world_size)
+    return fail(COAT_ERR_INVALID_ARG, "%s: need world_size >= 1 and 0 <= rank < world_size", fn);
+  if (max_pieces < 0 || (max_pieces > 0 && !pieces))
+    return fail(COAT_ERR_INVALID_ARG, "%s: pieces is NULL or max_pieces < 0", fn);
+  // Blocks of 4 groups: a piece's first group then has its four per-group
+  // floats on a 16-byte boundary, as the step's descriptors require.
+  const int64_t blk = 4 * static_cast<int64_t>(group);
+  constexpr int64_t kMaxBlocks = std::numeric_limits<int64_t>::max() / 512 / 2;
+  int64_t total_blocks = 0;
+  for (int i = 0; i < num_tensors; ++i) {
+    if (sizes[i] < 0) return fail(COAT_ERR_INVALID_ARG, "%s: sizes[%d] < 0", fn, i);
+    if (sizes[i] > kMaxBlocks * blk) return fail(COAT_ERR_INVALID_ARG, "%s: too many elements", fn);
+    total_blocks += (sizes[i] + blk - 1) / blk;
+    if (total_blocks > kMaxBlocks) return fail(COAT_ERR_INVALID_ARG, "%s: too many elements", fn);
+  }
+  const int64_t shard = (total_blocks + world_size - 1) / world_size * blk;
+  const int64_t lo_e = shard * rank, hi_e = shard * (rank + 1);
+  // Pieces: the intersection of [lo_e, hi_e) with each tensor's flat range.
+  int count = 0;
+  int64_t off = 0;
+  for (int i = 0; i < num_tensors; ++i) {
+    if (flat_offsets) flat_offsets[i] = off;
+    const int64_t lo = std::max(off, lo_e), hi = std::min(off + sizes[i], hi_e);
+    if (lo < hi) {
+      if (count < max_pieces) {
+        coat_shard_piece& pc = pieces[count];
+        pc.tensor = i;
+        pc.reserved = 0;
+        pc.elem_begin = lo - off;
+        pc.n_elems = hi - lo;
+        pc.shard_begin = lo - lo_e;
+      }
+      ++count;
+    }
+    off += (sizes[i] + blk - 1) / blk * blk;
+  }
+  *num_pieces = count;
+  *shard_elems = shard;
+  *flat_elems = shard * world_size;
+  if (count > max_pieces)
+    return fail(COAT_ERR_INVALID_ARG, "%s: %d pieces needed, max_pieces is %d", fn, count,
+                max_pieces);
   return COAT_OK;
 }
 

@@ -31,7 +31,7 @@ def test_library_exports_every_declared_symbol():
     L = coat.lib()
     for name in declared_functions():
         assert hasattr(L, name), name
-    assert coat.coat_version() == 10300
+    assert coat.coat_version() == 10400
 
 
 def test_nm_exports_match():
