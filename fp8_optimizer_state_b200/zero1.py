@@ -116,6 +116,39 @@ class Zero1AdamW:
         if self._plan is not None:
             self._plan.set_wd_scale(self._wd_scale)
 
+    _STATE = ("master", "m_q", "m_scale", "m_k", "v_q", "v_scale", "v_k")
+
+    def state_dict(self):
+        """This rank's optimizer state (CPU copies): the shard's master
+        weights and FP8 moments, with the layout they belong to."""
+        out = {k: getattr(self, k).detach().cpu().clone() for k in self._STATE}
+        out.update(sizes=list(self.sizes), world_size=self.world, rank=self.rank,
+                   fmt_m=self.fmt_m, fmt_v=self.fmt_v)
+        return out
+
+    def load_state_dict(self, state):
+        """Restore this rank's state saved by state_dict() under the same
+        sizes, world size, rank and formats, then rebuild the bf16 weights:
+        each piece's bf16 copy is RNE(master), as the step writes it, and the
+        weights are all-gathered (a collective: every rank calls this)."""
+        want = dict(sizes=self.sizes, world_size=self.world, rank=self.rank, fmt_m=self.fmt_m,
+                    fmt_v=self.fmt_v)
+        got = {k: state[k] for k in want}
+        if got != want:
+            raise ValueError("state was saved under another layout: %r, expected %r"
+                             % (got, want))
+        for k in self._STATE:
+            dst = getattr(self, k)
+            src = state[k]
+            if src.dtype != dst.dtype or src.shape != dst.shape:
+                raise ValueError("state %s has %s %s, expected %s %s"
+                                 % (k, src.dtype, tuple(src.shape), dst.dtype, tuple(dst.shape)))
+            dst.copy_(src)
+        for piece in self.pieces:
+            v = self.piece_views(piece)
+            v["weight"].copy_(v["master"].to(torch.bfloat16))
+        self.all_gather_weights()
+
     # -- the step ---------------------------------------------------------
     def reduce_scatter_grads(self):
         dist.reduce_scatter_tensor(self.grad_shard, self.flat_grad, op=dist.ReduceOp.SUM,

@@ -228,6 +228,60 @@ def _rank_main(rank, world, port, fmt_m, fmt_v):
         dist.destroy_process_group()
 
 
+def _resume_main(rank, world, port, out_dir):
+    """Two steps, a checkpoint, a fresh object restored from it: its third
+    step gives the same bytes as the original's third step."""
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import oracle as orc
+    import synth
+    from fp8_optimizer_state_b200.zero1 import Zero1AdamW
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        def run_step(z, step):
+            for i, n in enumerate(SIZES):
+                bits = synth.grad_bits(30 + rank, i, step, 0, n)
+                z.grad(i).copy_(torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16))
+            z.reduce_scatter_grads()
+            _oracle_local_step(z, orc, step, 0, 1)
+            z.all_gather_weights()
+
+        a = Zero1AdamW(SIZES, device="cpu", fmt_m=0, fmt_v=1)
+        a.set_wd_scale(WD_SCALE)
+        a.load_weights([torch.from_numpy(synth.master(8, i, 0, n).copy())
+                        for i, n in enumerate(SIZES)])
+        run_step(a, 1)
+        run_step(a, 2)
+        path = os.path.join(out_dir, "rank%d.pt" % rank)
+        torch.save(a.state_dict(), path)
+        b = Zero1AdamW(SIZES, device="cpu", fmt_m=0, fmt_v=1)
+        b.set_wd_scale(WD_SCALE)
+        b.load_state_dict(torch.load(path))
+        assert torch.equal(b.flat_weight.view(torch.int16), a.flat_weight.view(torch.int16))
+        run_step(a, 3)
+        run_step(b, 3)
+        for k in Zero1AdamW._STATE + ("flat_weight",):
+            x, y = getattr(a, k), getattr(b, k)
+            assert torch.equal(x.view(torch.uint8), y.view(torch.uint8)), k
+        # a state saved under another layout is refused
+        bad = dict(a.state_dict(), world_size=world + 1)
+        with pytest.raises(ValueError, match="another layout"):
+            b.load_state_dict(bad)
+        bad = dict(a.state_dict(), m_q=a.m_q[:-1].clone())
+        with pytest.raises(ValueError, match="m_q"):
+            b.load_state_dict(bad)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_checkpoint_resume_is_bit_identical(tmp_path):
+    mp.start_processes(_resume_main, args=(2, _free_port(), str(tmp_path)), nprocs=2, join=True,
+                       start_method="spawn")
+
+
 @pytest.mark.parametrize("world,fmt_m,fmt_v", [(2, 0, 0), (3, 0, 1)])
 def test_sharded_step_equals_the_unsharded_oracle_step(world, fmt_m, fmt_v):
     mp.start_processes(_rank_main, args=(world, _free_port(), fmt_m, fmt_v), nprocs=world,
