@@ -37,10 +37,14 @@ class Zero1AdamW:
                    the caller before step(); the padding stays zero.
       flat_weight  flat_elems bf16: tensor i's bf16 weights are weight(i),
                    complete on every rank after step().
-      master, m_q, v_q, grad_shard, weight_shard: shard_elems each (FP32, u8,
-                   u8, bf16, bf16); m_scale, m_k, v_scale, v_k: one float per
-                   group of the shard.  Moments start at zero (codes 0, scale
-                   1, k 1).
+      grad_shard, weight_shard: this rank's slices of the flat buffers
+                   (shard_elems each, starting at rank * shard_elems).
+      master, m_q, v_q: shard_elems each (FP32, u8, u8); m_scale, m_k,
+                   v_scale, v_k: one float per group of the shard.  Moments
+                   start at zero (codes 0, scale 1, k 1).
+    Per rank: 4 bytes per parameter for the two flat bf16 buffers, and
+    6.125 / world_size for the sharded state (master 4, codes 2, scale and k
+    16 per group of 128).
     The process group's collectives must support bf16 reduce-scatter and
     all-gather (NCCL; gloo on the CPU)."""
 
@@ -58,8 +62,12 @@ class Zero1AdamW:
         f32 = dict(dtype=torch.float32, device=dev)
         self.flat_grad = torch.zeros(self.flat_elems, **bf16)
         self.flat_weight = torch.zeros(self.flat_elems, **bf16)
-        self.grad_shard = torch.zeros(e, **bf16)
-        self.weight_shard = torch.zeros(e, **bf16)
+        # The rank's shards are its slices of the flat buffers: the
+        # reduce-scatter and the all-gather then run in place (NCCL's in-place
+        # forms), and no second copy of either is held.
+        lo = self.rank * e
+        self.grad_shard = self.flat_grad[lo:lo + e]
+        self.weight_shard = self.flat_weight[lo:lo + e]
         self.master = torch.zeros(e, **f32)
         self.m_q = torch.zeros(e, dtype=torch.uint8, device=dev)
         self.v_q = torch.zeros(e, dtype=torch.uint8, device=dev)

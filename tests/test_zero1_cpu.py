@@ -176,6 +176,10 @@ def _rank_main(rank, world, port, fmt_m, fmt_v):
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         z = Zero1AdamW(SIZES, device="cpu", fmt_m=fmt_m, fmt_v=fmt_v)
+        # the shards are the rank's slices of the flat buffers (in-place collectives)
+        lo = 2 * rank * z.shard_elems
+        assert z.grad_shard.data_ptr() == z.flat_grad.data_ptr() + lo
+        assert z.weight_shard.data_ptr() == z.flat_weight.data_ptr() + lo
         z.set_wd_scale(WD_SCALE)
         masters = [torch.from_numpy(synth.master(7, i, 0, n).copy()) for i, n in enumerate(SIZES)]
         z.load_weights(masters)
