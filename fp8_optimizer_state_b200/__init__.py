@@ -51,6 +51,7 @@ EXPORTS = [
     ("coat_rmsnorm_fp8_workspace_size", _i32, [_i64, ctypes.POINTER(ctypes.c_size_t)]),
     ("coat_rmsnorm_fp8_backward", _i32, [_vp, _i64, _vp, _vp, _i64, _i64, _f32, _i32, _vp, _i64,
                                          _vp, _vp, ctypes.c_size_t, _vp]),
+    ("coat_grad_clip_finalize", _i32, [_vp, _f32, _vp]),
     ("coat_zero1_layout", _i32, [_vp, _i32, _i32, _i32, _i32, _vp, _i32, ctypes.POINTER(_i32),
                                  ctypes.POINTER(_i64), ctypes.POINTER(_i64), _vp]),
 ]
@@ -319,6 +320,14 @@ def coat_adamw_step_multi_clipped(plan, clip_buf, *, lr, beta1, beta2, eps, wd, 
         raise ValueError("clip_buf must hold %d bytes" % ctypes.sizeof(GradClip))
     _check(lib().coat_adamw_step_multi_clipped(plan.handle, lr, beta1, beta2, eps, wd, step,
                                                _p(clip_buf), _s(stream)))
+
+
+def coat_grad_clip_finalize(clip_buf, max_norm, stream=None):
+    """Recompute norm, coef and found_inf of a clip record from its sumsq
+    (after the ranks' sums have been added into it)."""
+    if clip_buf.numel() * clip_buf.element_size() < ctypes.sizeof(GradClip):
+        raise ValueError("clip_buf must hold %d bytes" % ctypes.sizeof(GradClip))
+    _check(lib().coat_grad_clip_finalize(_p(clip_buf), max_norm, _s(stream)))
 
 
 def coat_multi_plan_destroy(plan):

@@ -419,6 +419,23 @@ coat_status coat_adamw_step(float* master, uint16_t* weight_bf16_out, const uint
 
 }  // extern "C"
 
+namespace {
+
+// Norm, coefficient and found-Inf of a clip record from its sum of squares:
+// the arithmetic of the gradient-norm pass's last CTA (double sqrt and
+// division, both correctly rounded, then FP32), so that a record finalised
+// here equals one the pass writes for the same sum.
+__global__ void clip_finalize_kernel(coat::ClipRecord* rec, float max_norm) {
+  const double total = rec->sumsq;
+  const double c = static_cast<double>(max_norm) / (sqrt(total) + 1e-6);
+  rec->norm = static_cast<float>(sqrt(total));
+  rec->coef = static_cast<float>(c < 1.0 ? c : 1.0);
+  rec->found_inf = isfinite(total) ? 0 : 1;
+  rec->reserved = 0;
+}
+
+}  // namespace
+
 struct coat_multi_plan {
   coat::TensorArgs* d_descs = nullptr;  // device copy of the descriptors (tile_begin ascending)
   double* d_partials = nullptr;         // gradient-norm pass: one slot per CTA
@@ -521,6 +538,17 @@ coat_status coat_multi_plan_grad_norm(coat_multi_plan_t plan, float max_norm,
   cudaError_t e = coat::launch_grad_sumsq(plan->d_descs, plan->num, plan->total_tiles,
                                           plan->d_partials, plan->d_ticket, max_norm,
                                           reinterpret_cast<coat::ClipRecord*>(d_clip), stream);
+  return e == cudaSuccess ? COAT_OK : cuda_fail(e, fn);
+}
+
+coat_status coat_grad_clip_finalize(coat_grad_clip* d_clip, float max_norm,
+                                    cudaStream_t stream) {
+  const char* fn = "coat_grad_clip_finalize";
+  if (!d_clip) return fail(COAT_ERR_INVALID_ARG, "%s: d_clip is NULL", fn);
+  if (!aligned(d_clip, 8)) return fail(COAT_ERR_MISALIGNED, "%s: d_clip is not 8-byte aligned", fn);
+  if (!(max_norm > 0.f)) return fail(COAT_ERR_INVALID_ARG, "%s: max_norm must be > 0", fn);
+  clip_finalize_kernel<<<1, 1, 0, stream>>>(reinterpret_cast<coat::ClipRecord*>(d_clip), max_norm);
+  cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? COAT_OK : cuda_fail(e, fn);
 }
 

@@ -25,8 +25,9 @@ from __future__ import annotations
 import torch
 import torch.distributed as dist
 
-from . import (COAT_E4M3, GROUP, coat_adamw_step_multi, coat_multi_plan_create,
-               coat_zero1_layout, make_desc)
+from . import (COAT_E4M3, GROUP, coat_adamw_step_multi, coat_adamw_step_multi_clipped,
+               coat_grad_clip_finalize, coat_multi_plan_create, coat_zero1_layout, make_desc,
+               new_grad_clip)
 
 
 class Zero1AdamW:
@@ -74,6 +75,10 @@ class Zero1AdamW:
         self.m_scale, self.m_k, self.v_scale, self.v_k = (torch.ones(ng, **f32) for _ in range(4))
         self._plan = None
         self._wd_scale = None
+        # clip record (24 bytes): its first double, the sum of squares, is
+        # all-reduced over the ranks
+        self.clip = new_grad_clip(dev)
+        self.clip_sumsq = self.clip[:8].view(torch.float64)
 
     # -- views ------------------------------------------------------------
     def grad(self, i):
@@ -162,10 +167,7 @@ class Zero1AdamW:
         dist.reduce_scatter_tensor(self.grad_shard, self.flat_grad, op=dist.ReduceOp.SUM,
                                    group=self.pg)
 
-    def local_step(self, *, lr, beta1, beta2, eps, wd, step, stream=None):
-        """The FP8 AdamW step over this rank's pieces (one kernel launch)."""
-        if not self.pieces:
-            return
+    def _get_plan(self, stream=None):
         if self._plan is None:
             descs = []
             for piece in self.pieces:
@@ -175,17 +177,53 @@ class Zero1AdamW:
             self._plan = coat_multi_plan_create(descs, self.fmt_m, self.fmt_v, stream=stream)
             if self._wd_scale is not None:
                 self._plan.set_wd_scale(self._wd_scale, stream=stream)
-        coat_adamw_step_multi(self._plan, lr=lr, beta1=beta1, beta2=beta2, eps=eps, wd=wd,
-                              step=step, stream=stream)
+        return self._plan
+
+    def local_grad_sumsq(self):
+        """This rank's sum of squared summed gradients into the clip record
+        (the gradient-norm pass over the rank's pieces; 0 without pieces)."""
+        if self.pieces:
+            self._get_plan().grad_norm(float("inf"), self.clip)
+        else:
+            self.clip.zero_()
+
+    def allreduce_grad_sumsq(self):
+        dist.all_reduce(self.clip_sumsq, op=dist.ReduceOp.SUM, group=self.pg)
+
+    def finalize_clip(self, max_norm):
+        """Norm, coefficient and found-Inf from the global sum of squares."""
+        coat_grad_clip_finalize(self.clip, max_norm)
+
+    def local_step(self, *, lr, beta1, beta2, eps, wd, step, clipped=False, stream=None):
+        """The FP8 AdamW step over this rank's pieces (one kernel launch);
+        clipped: scale the gradients by the clip record's coefficient, or
+        skip the step when it found an Inf or NaN."""
+        if not self.pieces:
+            return
+        plan = self._get_plan(stream)
+        if clipped:
+            coat_adamw_step_multi_clipped(plan, self.clip, lr=lr, beta1=beta1, beta2=beta2,
+                                          eps=eps, wd=wd, step=step, stream=stream)
+        else:
+            coat_adamw_step_multi(plan, lr=lr, beta1=beta1, beta2=beta2, eps=eps, wd=wd,
+                                  step=step, stream=stream)
 
     def all_gather_weights(self):
         dist.all_gather_into_tensor(self.flat_weight, self.weight_shard, group=self.pg)
 
-    def step(self, *, lr, beta1, beta2, eps, wd, step):
+    def step(self, *, lr, beta1, beta2, eps, wd, step, max_norm=None):
         """Reduce-scatter the gradients, step this rank's share, all-gather
-        the bf16 weights."""
+        the bf16 weights.  With max_norm, the summed gradients are clipped to
+        that global 2-norm first (the norm over all ranks' shards: each rank's
+        sum of squares, all-reduced, then the coefficient on the device), and
+        an Inf or NaN anywhere skips the step on every rank."""
         self.reduce_scatter_grads()
-        self.local_step(lr=lr, beta1=beta1, beta2=beta2, eps=eps, wd=wd, step=step)
+        if max_norm is not None:
+            self.local_grad_sumsq()
+            self.allreduce_grad_sumsq()
+            self.finalize_clip(max_norm)
+        self.local_step(lr=lr, beta1=beta1, beta2=beta2, eps=eps, wd=wd, step=step,
+                        clipped=max_norm is not None)
         self.all_gather_weights()
 
     def close(self):

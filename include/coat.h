@@ -238,6 +238,17 @@ coat_status coat_multi_plan_grad_norm(coat_multi_plan_t plan, float max_norm,
 coat_status coat_adamw_step_multi_clipped(coat_multi_plan_t plan, float lr, float beta1,
                                           float beta2, float eps, float wd, int64_t step,
                                           const coat_grad_clip *d_clip, cudaStream_t stream);
+/* Clipping over data-parallel ranks, each holding part of the gradients (a
+ * ZeRO-1 shard, see coat_zero1_layout): each rank runs
+ * coat_multi_plan_grad_norm on its own plan (max_norm = +Inf), the callers
+ * sum the records' sumsq fields over the ranks (an all-reduce of that one
+ * double), and coat_grad_clip_finalize then rewrites norm, coef, found_inf and
+ * reserved of the record at d_clip from its sumsq and max_norm, with the same
+ * arithmetic as coat_multi_plan_grad_norm (so one rank gives that call's
+ * record bit for bit).  One thread on `stream`; d_clip 8-byte aligned device
+ * memory; max_norm > 0 (+Inf allowed); COAT_ERR_INVALID_ARG /
+ * COAT_ERR_MISALIGNED otherwise, before anything is enqueued. */
+coat_status coat_grad_clip_finalize(coat_grad_clip *d_clip, float max_norm, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
  * No-allocation variant of the multi-tensor step.  The COAT pages have no

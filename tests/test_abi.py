@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import fp8_optimizer_state_b200 as coat
 
@@ -111,6 +112,15 @@ def test_grad_clip_validation():
     assert step(lr=-1.0) == INVALID
     assert step(step=0) == INVALID
     assert ctypes.sizeof(coat.GradClip) == 24
+    # the finalisation after an all-reduce of the ranks' sums of squares
+    assert L.coat_grad_clip_finalize(None, 1.0, None) == INVALID
+    assert "d_clip is NULL" in coat.coat_last_error()
+    assert L.coat_grad_clip_finalize(rec + 4, 1.0, None) == MISALIGNED
+    for bad in (0.0, -1.0, float("nan")):
+        assert L.coat_grad_clip_finalize(rec, bad, None) == INVALID
+        assert "max_norm" in coat.coat_last_error()
+    with pytest.raises(ValueError):
+        coat.coat_grad_clip_finalize(torch.zeros(16, dtype=torch.uint8), 1.0)
 
 
 def test_swiglu_validation():

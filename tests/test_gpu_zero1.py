@@ -1,7 +1,8 @@
 """ZeRO-1 on one GPU: world size 1 over NCCL runs the product path end to end
 (reduce-scatter of the flat gradients, the multi-tensor FP8 step over the
-shard's pieces, all-gather of the bf16 weights), which must give the bits of
-the plain multi-tensor step on the same tensors.  More ranks need more GPUs;
+shard's pieces, all-gather of the bf16 weights; with clipping, the norm pass,
+an all-reduce of the sum of squares and coat_grad_clip_finalize), which must
+give the bits of the plain multi-tensor step on the same tensors.  More ranks need more GPUs;
 their partition and collectives are covered by two and three gloo ranks on
 the CPU, with the oracle's step in the kernel's place."""
 import datetime
@@ -40,7 +41,11 @@ def _plain_side(master):
                 v_scale=torch.ones(ng, **dev), v_k=torch.ones(ng, **dev))
 
 
-def test_world_size_one_equals_the_multi_tensor_step():
+@pytest.mark.parametrize("max_norm", [None, 1e-3])
+def test_world_size_one_equals_the_multi_tensor_step(max_norm):
+    """max_norm: the clipped step over ranks (norm pass on the shard, an
+    all-reduce of the sum of squares, coat_grad_clip_finalize) against the
+    plain plan's norm pass and clipped step; the clip records must match too."""
     from fp8_optimizer_state_b200.zero1 import Zero1AdamW
     sizes = [300, 128, 1000, 5, 0, 2125, 4096 * 3 + 7]
     wd_scale = [1.0, 0.0, 1.0, 0.5, 1.0, 1.0, 0.0]
@@ -60,14 +65,22 @@ def test_world_size_one_equals_the_multi_tensor_step():
                             s["m_k"], s["v_q"], s["v_scale"], s["v_k"]) for s in sides],
             coat.COAT_E4M3, coat.COAT_E5M2)
         plan.set_wd_scale(wd_scale)
+        rec = coat.new_grad_clip()
         hp = dict(lr=H["lr"], beta1=H["beta1"], beta2=H["beta2"], eps=H["eps"], wd=H["wd"])
         for t in (1, 2, 3):
             for i, n in enumerate(sizes):
                 g = torch.from_numpy(synth.grad_bits(3, i, t, 0, n).view(np.int16)).cuda()
                 z.grad(i).view(torch.int16).copy_(g)
                 sides[i]["grad"].copy_(g)
-            z.step(step=t, **hp)
-            coat.coat_adamw_step_multi(plan, step=t, **hp)
+            z.step(step=t, max_norm=max_norm, **hp)
+            if max_norm is None:
+                coat.coat_adamw_step_multi(plan, step=t, **hp)
+            else:
+                plan.grad_norm(max_norm, rec)
+                coat.coat_adamw_step_multi_clipped(plan, rec, step=t, **hp)
+                a, b = coat.read_grad_clip(z.clip), coat.read_grad_clip(rec)
+                assert bytes(a) == bytes(b), (t, a.sumsq, b.sumsq, a.coef, b.coef)
+                assert 0.0 < b.coef < 1.0 and b.found_inf == 0
         coat.coat_check_device_error()
         torch.cuda.synchronize()
         for i, n in enumerate(sizes):

@@ -129,12 +129,12 @@ def _np(t):
     return t.numpy()
 
 
-def _oracle_local_step(z, orc, step, fmt_m, fmt_v):
+def _oracle_local_step(z, orc, step, fmt_m, fmt_v, gscale=1.0):
     for piece in z.pieces:
         v = {k: _np(x) for k, x in z.piece_views(piece).items()}
         orc.adamw_step(v["master"], v["weight"], v["grad"], v["m_q"], v["m_scale"], v["m_k"],
                        v["v_q"], v["v_scale"], v["v_k"], step=step, fmt_m=fmt_m, fmt_v=fmt_v,
-                       **dict(HP, wd=HP["wd"] * WD_SCALE[piece[0]]))
+                       gscale=gscale, **dict(HP, wd=HP["wd"] * WD_SCALE[piece[0]]))
 
 
 def _plan_status(descs):
@@ -165,71 +165,142 @@ def _check_descriptors(z):
     assert _plan_status([_host_desc(views[0], shift_scale=1)]) == 2
 
 
-def _rank_main(rank, world, port, fmt_m, fmt_v):
+def _setup(rank, world, port, fmt_m, fmt_v, seed):
+    """Process group, a Zero1AdamW on the CPU with loaded weights, and the
+    unsharded reference state (whole tensors, zero moments)."""
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
-    import oracle as orc
     import synth
     from fp8_optimizer_state_b200.zero1 import Zero1AdamW
 
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
+    z = Zero1AdamW(SIZES, device="cpu", fmt_m=fmt_m, fmt_v=fmt_v)
+    z.set_wd_scale(WD_SCALE)
+    masters = [torch.from_numpy(synth.master(seed, i, 0, n).copy()) for i, n in enumerate(SIZES)]
+    z.load_weights(masters)
+    ref = []
+    for i, n in enumerate(SIZES):
+        ng = _groups(n)
+        ref.append(dict(master=masters[i].numpy().copy(), weight=np.zeros(n, np.uint16),
+                        m_q=np.zeros(ng * G, np.uint8), v_q=np.zeros(ng * G, np.uint8),
+                        m_scale=np.ones(ng, np.float32), m_k=np.ones(ng, np.float32),
+                        v_scale=np.ones(ng, np.float32), v_k=np.ones(ng, np.float32)))
+    return z, ref
+
+
+def _write_grads(z, rank, seed, step, inf_at=None):
+    import synth
+    for i, n in enumerate(SIZES):
+        bits = synth.grad_bits(seed + rank, i, step, 0, n)
+        if inf_at is not None and inf_at[0] == i:
+            bits[inf_at[1]] = 0x7F80                      # +Inf in bf16
+        z.grad(i).copy_(torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16))
+
+
+def _summed_grads(z):
+    """The summed gradients as the reduce-scatter produced them, per tensor."""
+    import torch.distributed as dist
+    full = torch.zeros(z.flat_elems, dtype=torch.bfloat16)
+    dist.all_gather_into_tensor(full, z.grad_shard)
+    return [_np(full)[o:o + n].copy() for o, n in zip(z.flat_offsets, SIZES)]
+
+
+def _reference_step(orc, ref, grads, step, fmt_m, fmt_v, gscale=1.0):
+    for i, r in enumerate(ref):
+        orc.adamw_step(r["master"], r["weight"], grads[i], r["m_q"], r["m_scale"], r["m_k"],
+                       r["v_q"], r["v_scale"], r["v_k"], step=step, fmt_m=fmt_m, fmt_v=fmt_v,
+                       gscale=gscale, **dict(HP, wd=HP["wd"] * WD_SCALE[i]))
+
+
+def _compare(z, ref, tag):
+    for i, n in enumerate(SIZES):
+        assert np.array_equal(_np(z.weight(i)), ref[i]["weight"]), (tag, i)
+    for piece in z.pieces:
+        t, b, n, _ = piece
+        v = z.piece_views(piece)
+        r = ref[t]
+        g0, ng = b // G, _groups(n)
+        assert np.array_equal(_np(v["master"]).view(np.uint32),
+                              r["master"][b:b + n].view(np.uint32)), (tag, t)
+        for key in ("m_q", "v_q"):
+            assert np.array_equal(_np(v[key])[:n], r[key][b:b + n]), (tag, t, key)
+        for key in ("m_scale", "m_k", "v_scale", "v_k"):
+            assert np.array_equal(_np(v[key]), r[key][g0:g0 + ng]), (tag, t, key)
+    # padding in the flat buffers is never written
+    pad = np.ones(z.flat_elems, bool)
+    for i, n in enumerate(SIZES):
+        pad[z.flat_offsets[i]:z.flat_offsets[i] + n] = False
+    assert pad.any() and not _np(z.flat_weight)[pad].any()
+
+
+def _rank_main(rank, world, port, fmt_m, fmt_v):
+    import torch.distributed as dist
+    import oracle as orc
     try:
-        z = Zero1AdamW(SIZES, device="cpu", fmt_m=fmt_m, fmt_v=fmt_v)
+        z, ref = _setup(rank, world, port, fmt_m, fmt_v, 7)
         # the shards are the rank's slices of the flat buffers (in-place collectives)
         lo = 2 * rank * z.shard_elems
         assert z.grad_shard.data_ptr() == z.flat_grad.data_ptr() + lo
         assert z.weight_shard.data_ptr() == z.flat_weight.data_ptr() + lo
-        z.set_wd_scale(WD_SCALE)
-        masters = [torch.from_numpy(synth.master(7, i, 0, n).copy()) for i, n in enumerate(SIZES)]
-        z.load_weights(masters)
         _check_descriptors(z)
-        # the unsharded reference: whole tensors, zero moments
-        ref = []
-        for i, n in enumerate(SIZES):
-            ng = _groups(n)
-            ref.append(dict(master=masters[i].numpy().copy(), weight=np.zeros(n, np.uint16),
-                            m_q=np.zeros(ng * G, np.uint8), v_q=np.zeros(ng * G, np.uint8),
-                            m_scale=np.ones(ng, np.float32), m_k=np.ones(ng, np.float32),
-                            v_scale=np.ones(ng, np.float32), v_k=np.ones(ng, np.float32)))
-        full_grad = torch.zeros(z.flat_elems, dtype=torch.bfloat16)
         for step in (1, 2, 3):
-            for i, n in enumerate(SIZES):
-                bits = synth.grad_bits(20 + rank, i, step, 0, n)
-                z.grad(i).copy_(torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16))
+            _write_grads(z, rank, 20, step)
             z.reduce_scatter_grads()
             _oracle_local_step(z, orc, step, fmt_m, fmt_v)
             z.all_gather_weights()
-            # the summed gradients as the reduce-scatter produced them
-            dist.all_gather_into_tensor(full_grad, z.grad_shard)
-            for i, n in enumerate(SIZES):
-                o = z.flat_offsets[i]
-                g = _np(full_grad)[o:o + n].copy()
-                r = ref[i]
-                orc.adamw_step(r["master"], r["weight"], g, r["m_q"], r["m_scale"], r["m_k"],
-                               r["v_q"], r["v_scale"], r["v_k"], step=step, fmt_m=fmt_m,
-                               fmt_v=fmt_v, **dict(HP, wd=HP["wd"] * WD_SCALE[i]))
-            for i, n in enumerate(SIZES):
-                assert np.array_equal(_np(z.weight(i)), ref[i]["weight"]), (rank, step, i)
-            for piece in z.pieces:
-                t, b, n, _ = piece
-                v = z.piece_views(piece)
-                r = ref[t]
-                g0, ng = b // G, _groups(n)
-                assert np.array_equal(_np(v["master"]).view(np.uint32),
-                                      r["master"][b:b + n].view(np.uint32)), (rank, step, t)
-                for key in ("m_q", "v_q"):
-                    assert np.array_equal(_np(v[key])[:n], r[key][b:b + n]), (rank, step, t, key)
-                for key in ("m_scale", "m_k", "v_scale", "v_k"):
-                    assert np.array_equal(_np(v[key]), r[key][g0:g0 + ng]), (rank, step, t, key)
-        # padding in the flat buffers and shards is never written
-        pad = np.ones(z.flat_elems, bool)
-        for i, n in enumerate(SIZES):
-            pad[z.flat_offsets[i]:z.flat_offsets[i] + n] = False
-        assert pad.any() and not _np(z.flat_weight)[pad].any()
+            _reference_step(orc, ref, _summed_grads(z), step, fmt_m, fmt_v)
+            _compare(z, ref, (rank, step))
         dist.barrier()
     finally:
         dist.destroy_process_group()
+
+
+MAX_NORM = 0.05
+
+
+def _clip_main(rank, world, port):
+    """Clipping over ranks: each rank's sum of squares over its pieces (the
+    oracle's, in the norm pass's place), summed by Zero1AdamW's all-reduce;
+    the coefficient from that sum must be the one of the whole summed
+    gradient, and the clipped states the unsharded clipped step's.  Step 2
+    has an Inf in one rank's gradient of a tensor another rank owns: every
+    rank must then skip the step."""
+    import math
+    import torch.distributed as dist
+    import oracle as orc
+    try:
+        z, ref = _setup(rank, world, port, 0, 1, 9)
+        coefs = []
+        for step in (1, 2, 3):
+            _write_grads(z, rank, 40, step, inf_at=(5, 1900) if step == 2 and rank == 0 else None)
+            z.reduce_scatter_grads()
+            local = sum(orc.grad_sumsq(_np(z.piece_views(p)["grad"]))[0] for p in z.pieces)
+            z.clip_sumsq.fill_(local)
+            z.allreduce_grad_sumsq()
+            total = float(z.clip_sumsq.item())
+            grads = _summed_grads(z)
+            whole, bad = orc.grad_sumsq(np.concatenate(grads))
+            assert bad == (not math.isfinite(total)) == (step == 2)
+            if not bad:
+                assert abs(total - whole) <= 1e-13 * whole
+                coef = orc.clip_coef(total, MAX_NORM)
+                assert coef == orc.clip_coef(whole, MAX_NORM)
+                coefs.append(coef)
+                _oracle_local_step(z, orc, step, 0, 1, gscale=coef)
+                _reference_step(orc, ref, grads, step, 0, 1, gscale=coef)
+            z.all_gather_weights()
+            _compare(z, ref, (rank, step))
+        assert all(c < 1.0 for c in coefs)               # the clip was active
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_clipping_over_ranks_equals_the_unsharded_clipped_step(world):
+    mp.start_processes(_clip_main, args=(world, _free_port()), nprocs=world, join=True,
+                       start_method="spawn")
 
 
 def _resume_main(rank, world, port, out_dir):
