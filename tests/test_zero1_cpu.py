@@ -200,10 +200,7 @@ def _write_grads(z, rank, seed, step, inf_at=None):
 
 def _summed_grads(z):
     """The summed gradients as the reduce-scatter produced them, per tensor."""
-    import torch.distributed as dist
-    full = torch.zeros(z.flat_elems, dtype=torch.bfloat16)
-    dist.all_gather_into_tensor(full, z.grad_shard)
-    return [_np(full)[o:o + n].copy() for o, n in zip(z.flat_offsets, SIZES)]
+    return _summed_grads_of(z, SIZES)
 
 
 def _reference_step(orc, ref, grads, step, fmt_m, fmt_v, gscale=1.0):
@@ -300,6 +297,70 @@ def _clip_main(rank, world, port):
 @pytest.mark.parametrize("world", [2, 3])
 def test_clipping_over_ranks_equals_the_unsharded_clipped_step(world):
     mp.start_processes(_clip_main, args=(world, _free_port()), nprocs=world, join=True,
+                       start_method="spawn")
+
+
+def _empty_ranks_main(rank, world, port):
+    """More ranks than blocks: two blocks over three ranks, so rank 2 owns no
+    group (no pieces, no plan) yet takes every collective step; the clipped
+    result is the unsharded clipped step's on every rank."""
+    import torch.distributed as dist
+    import oracle as orc
+    import synth
+    from fp8_optimizer_state_b200.zero1 import Zero1AdamW
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        sizes = [100, 0, 300]
+        z = Zero1AdamW(sizes, device="cpu")
+        assert (len(z.pieces) > 0) == (rank < 2)
+        master = [torch.from_numpy(synth.master(11, i, 0, n).copy()) for i, n in enumerate(sizes)]
+        z.load_weights(master)
+        ref = [dict(master=m.numpy().copy(), weight=np.zeros(m.numel(), np.uint16),
+                    q=[np.zeros(_groups(m.numel()) * G, np.uint8) for _ in range(2)],
+                    s=[np.ones(_groups(m.numel()), np.float32) for _ in range(4)])
+               for m in master]
+        for step in (1, 2):
+            grads = []
+            for i, n in enumerate(sizes):
+                bits = synth.grad_bits(50 + rank, i, step, 0, n)
+                z.grad(i).copy_(torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16))
+            z.reduce_scatter_grads()
+            grads = _summed_grads_of(z, sizes)
+            local = sum(orc.grad_sumsq(_np(z.piece_views(p)["grad"]))[0] for p in z.pieces)
+            if not z.pieces:
+                z.clip.zero_()
+            z.clip_sumsq.fill_(local)
+            z.allreduce_grad_sumsq()
+            total = float(z.clip_sumsq.item())
+            coef = orc.clip_coef(total, MAX_NORM)
+            assert coef == orc.clip_coef(orc.grad_sumsq(np.concatenate(grads))[0], MAX_NORM)
+            for piece in z.pieces:
+                v = {k: _np(x) for k, x in z.piece_views(piece).items()}
+                orc.adamw_step(v["master"], v["weight"], v["grad"], v["m_q"], v["m_scale"],
+                               v["m_k"], v["v_q"], v["v_scale"], v["v_k"], step=step, fmt_m=0,
+                               fmt_v=0, gscale=coef, **HP)
+            z.all_gather_weights()
+            for i, r in enumerate(ref):
+                orc.adamw_step(r["master"], r["weight"], grads[i], r["q"][0], r["s"][0],
+                               r["s"][1], r["q"][1], r["s"][2], r["s"][3], step=step, fmt_m=0,
+                               fmt_v=0, gscale=coef, **HP)
+                assert np.array_equal(_np(z.weight(i)), r["weight"]), (rank, step, i)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def _summed_grads_of(z, sizes):
+    import torch.distributed as dist
+    full = torch.zeros(z.flat_elems, dtype=torch.bfloat16)
+    dist.all_gather_into_tensor(full, z.grad_shard)
+    return [_np(full)[o:o + n].copy() for o, n in zip(z.flat_offsets, sizes)]
+
+
+def test_ranks_without_groups_take_every_collective_step():
+    mp.start_processes(_empty_ranks_main, args=(3, _free_port()), nprocs=3, join=True,
                        start_method="spawn")
 
 
