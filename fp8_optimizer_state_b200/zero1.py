@@ -1,11 +1,12 @@
 """ZeRO-1 data parallelism around the FP8-state AdamW step.
 
-COAT's per-GPU memory figures ("FP8训练新范式：减少40%显存占用，训练速度提高1.4倍",
-section 训练加速1.43倍，显存降低1.54倍) are for data-parallel training, where
-the optimizer states are what each GPU may keep for a share of the parameters
-only.  Here each of world_size ranks keeps the FP32 master weights and the
-FP8 moments (codes, root scales, k) of 1/world_size of all parameter groups,
-as coat_zero1_layout partitions them, and every rank keeps the whole bf16
+COAT's memory figures ("FP8训练新范式：减少40%显存占用，训练速度提高1.4倍",
+section 训练加速1.43倍，显存降低1.54倍) are per GPU of a four-GPU training run;
+the page does not say how the run is parallelised.  Under data parallelism
+the optimizer states need only be kept once across the GPUs: here each of
+world_size ranks keeps the FP32 master weights and the FP8 moments (codes,
+root scales, k) of 1/world_size of all parameter groups, as
+coat_zero1_layout partitions them, and every rank keeps the whole bf16
 weight copy and a whole gradient buffer.  One step:
 
   1. a reduce-scatter (sum over ranks) of the flat bf16 gradient buffer, so

@@ -370,11 +370,11 @@ coat_status coat_rmsnorm_fp8_backward(const uint16_t *dy, int64_t ld_dy, const c
 
 /* ---------------------------------------------------------------------------
  * ZeRO-1 partition of a tensor list over data-parallel ranks.  [P1]
- * 训练加速1.43倍，显存降低1.54倍 reports per-GPU memory of data-parallel
- * training with FP8 optimizer states; keeping each rank's states for a
- * 1/world_size share of the parameters is this library's layout for that
- * setting (each group's states live on exactly one rank).  Host-only: this
- * call makes no CUDA call and works on a host without a GPU.
+ * 训练加速1.43倍，显存降低1.54倍 reports per-GPU memory of a four-GPU run with
+ * FP8 optimizer states (its parallelism unstated); keeping each rank's states
+ * for a 1/world_size share of the parameters is this library's layout for
+ * data parallelism (each group's states live on exactly one rank).
+ * Host-only: this call makes no CUDA call and works on a host without a GPU.
  *
  * Flat layout, in blocks of 4 groups (B = 4 * group = 512 elements, so that
  * every piece's per-group scale and k arrays start on a 16-byte boundary, as
