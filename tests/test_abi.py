@@ -198,6 +198,44 @@ def test_header_compiles_as_c99(tmp_path):
     assert p.returncode == 0, p.stderr
 
 
+def test_struct_layouts_match_the_binding(tmp_path):
+    """Every struct of include/coat.h has the size and field offsets of the
+    binding's ctypes mirror (a C program built against the header prints
+    them)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    cuda_inc = "/usr/local/cuda/include"
+    if gcc is None or not os.path.exists(os.path.join(cuda_inc, "cuda_runtime_api.h")):
+        pytest.skip("gcc or the CUDA headers are not available")
+    mirrors = {"coat_tensor_desc": coat.TensorDesc, "coat_grad_clip": coat.GradClip,
+               "coat_fp8_act": coat.Fp8Act, "coat_shard_piece": coat.ShardPiece}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "coat.h"',
+             'int main(void) {']
+    for cname, py in mirrors.items():
+        lines.append('  printf("%s size %%zu\\n", sizeof(%s));' % (cname, cname))
+        for field, _ in py._fields_:
+            lines.append('  printf("%s %s %%zu\\n", offsetof(%s, %s));'
+                         % (cname, field, cname, field))
+    lines += ['  return 0;', '}']
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    p = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        "-isystem", cuda_inc, str(src), "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert p.returncode == 0, p.stderr
+    got = {}
+    for line in subprocess.run([str(exe)], capture_output=True, text=True,
+                               check=True).stdout.splitlines():
+        cname, field, value = line.split()
+        got[(cname, field)] = int(value)
+    for cname, py in mirrors.items():
+        assert got[(cname, "size")] == ctypes.sizeof(py), cname
+        for field, _ in py._fields_:
+            assert got[(cname, field)] == getattr(py, field).offset, (cname, field)
+
+
 def test_selftest_budget_validation():
     L = coat.lib()
     assert L.coat_selftest_wait_timeout(999, None) == INVALID
