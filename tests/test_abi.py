@@ -28,6 +28,20 @@ def test_header_and_binding_agree():
     assert sorted(n for n, _, _ in coat.EXPORTS) == names
 
 
+def test_binding_argument_counts_match_the_header():
+    """Each declaration's parameter count equals the number of argtypes the
+    binding gives ctypes (a missing or extra argument would shift every
+    later one)."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    decls = dict(re.findall(r"\b(coat_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", src))
+    exports = {n: args for n, _, args in coat.EXPORTS}
+    assert set(decls) == set(exports)
+    for name, params in decls.items():
+        params = params.strip()
+        count = 0 if params in ("", "void") else params.count(",") + 1
+        assert count == len(exports[name]), name
+
+
 def test_library_exports_every_declared_symbol():
     L = coat.lib()
     for name in declared_functions():
