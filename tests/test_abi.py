@@ -42,6 +42,34 @@ def test_binding_argument_counts_match_the_header():
         assert count == len(exports[name]), name
 
 
+def _ctype_of(param):
+    """The ctypes type a C parameter declaration must be passed as."""
+    param = " ".join(param.split())
+    if "*" in param or param.split()[0] in ("cudaStream_t", "coat_multi_plan_t"):
+        return "pointer"
+    base = param.replace("const ", "").split()[0]
+    return {"int64_t": ctypes.c_int64, "int": ctypes.c_int, "coat_fmt": ctypes.c_int,
+            "coat_dtype": ctypes.c_int, "float": ctypes.c_float,
+            "size_t": ctypes.c_size_t}[base]
+
+
+def test_binding_argument_types_match_the_header():
+    """Each argtype has the C parameter's width and kind: pointers (and the
+    stream and plan handles) as pointers, int64_t / int / enum / float /
+    size_t as those ctypes types."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    decls = dict(re.findall(r"\b(coat_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", src))
+    for name, res, args in coat.EXPORTS:
+        params = [p for p in decls[name].split(",") if p.strip() not in ("", "void")]
+        for i, (param, arg) in enumerate(zip(params, args)):
+            want = _ctype_of(param)
+            if want == "pointer":
+                assert arg is ctypes.c_void_p or hasattr(arg, "_type_") and \
+                    issubclass(arg, ctypes._Pointer), (name, i, param)
+            else:
+                assert arg is want, (name, i, param, arg)
+
+
 def test_library_exports_every_declared_symbol():
     L = coat.lib()
     for name in declared_functions():
