@@ -108,6 +108,9 @@ class Zero1AdamW:
     def load_weights(self, tensors):
         """Set the master weights of this rank's pieces and the whole bf16
         copy from full-precision `tensors` (one per size, any shape)."""
+        if len(tensors) != len(self.sizes):
+            raise ValueError("need one tensor per size (%d), got %d"
+                             % (len(self.sizes), len(tensors)))
         for i, t in enumerate(tensors):
             flat = t.detach().reshape(-1)
             if flat.numel() != self.sizes[i]:
@@ -116,10 +119,8 @@ class Zero1AdamW:
             self.weight(i).copy_(flat.to(torch.float32).to(torch.bfloat16))
         for piece in self.pieces:
             t, b, n, _ = piece
-            src = tensors[t].detach().reshape(-1)[b:b + n].to(torch.float32)
-            v = self.piece_views(piece)
-            v["master"].copy_(src)
-            v["weight"].copy_(src.to(torch.bfloat16))
+            self.piece_views(piece)["master"].copy_(
+                tensors[t].detach().reshape(-1)[b:b + n].to(torch.float32))
 
     def set_wd_scale(self, scales):
         """Per-tensor weight decay multipliers (one per size; e.g. 0 for

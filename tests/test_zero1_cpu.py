@@ -394,6 +394,8 @@ def _resume_main(rank, world, port, out_dir):
         torch.save(a.state_dict(), path)
         b = Zero1AdamW(SIZES, device="cpu", fmt_m=0, fmt_v=1)
         b.set_wd_scale(WD_SCALE)
+        with pytest.raises(ValueError, match="one tensor per size"):
+            b.load_weights([torch.zeros(3)])
         b.load_state_dict(torch.load(path))
         assert torch.equal(b.flat_weight.view(torch.int16), a.flat_weight.view(torch.int16))
         run_step(a, 3)
