@@ -172,7 +172,7 @@ extern "C" {
 
 const char* coat_last_error(void) { return g_last_error.c_str(); }
 
-int coat_version(void) { return 10400; }   // 1.4: ZeRO-1 layout; 1.3: clipping pre-step, FP8 layers
+int coat_version(void) { return 10400; }   // 1.4: ZeRO-1 layout and clipping across ranks; 1.3: clipping pre-step, FP8 layers
 
 coat_status coat_fp8_encode(const float* y, int64_t n, coat_fmt fmt, uint8_t* q, cudaStream_t stream) {
   if (n < 0) return fail(COAT_ERR_INVALID_ARG, "coat_fp8_encode: n < 0");
