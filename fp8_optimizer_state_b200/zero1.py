@@ -165,9 +165,13 @@ class Zero1AdamW:
         self.all_gather_weights()
 
     # -- the step ---------------------------------------------------------
-    def reduce_scatter_grads(self):
-        dist.reduce_scatter_tensor(self.grad_shard, self.flat_grad, op=dist.ReduceOp.SUM,
-                                   group=self.pg)
+    def reduce_scatter_grads(self, async_op=False):
+        """Sum the ranks' flat gradients into this rank's shard (in place).
+        async_op: return the collective's work handle instead of waiting, so
+        that the caller can overlap it (wait() before the norm pass or step)."""
+        return dist.reduce_scatter_tensor(self.grad_shard, self.flat_grad,
+                                          op=dist.ReduceOp.SUM, group=self.pg,
+                                          async_op=async_op)
 
     def _get_plan(self, stream=None):
         if self._plan is None:
@@ -210,8 +214,12 @@ class Zero1AdamW:
             coat_adamw_step_multi(plan, lr=lr, beta1=beta1, beta2=beta2, eps=eps, wd=wd,
                                   step=step, stream=stream)
 
-    def all_gather_weights(self):
-        dist.all_gather_into_tensor(self.flat_weight, self.weight_shard, group=self.pg)
+    def all_gather_weights(self, async_op=False):
+        """Gather every rank's bf16 weight shard into the flat weights (in
+        place).  async_op: return the work handle, e.g. to overlap the gather
+        with work that does not read the weights; wait() before reading them."""
+        return dist.all_gather_into_tensor(self.flat_weight, self.weight_shard, group=self.pg,
+                                           async_op=async_op)
 
     def step(self, *, lr, beta1, beta2, eps, wd, step, max_norm=None):
         """Reduce-scatter the gradients, step this rank's share, all-gather

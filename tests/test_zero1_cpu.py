@@ -243,9 +243,15 @@ def _rank_main(rank, world, port, fmt_m, fmt_v):
         _check_descriptors(z)
         for step in (1, 2, 3):
             _write_grads(z, rank, 20, step)
-            z.reduce_scatter_grads()
+            if step == 2:            # the asynchronous forms, waited on
+                z.reduce_scatter_grads(async_op=True).wait()
+            else:
+                assert z.reduce_scatter_grads() is None
             _oracle_local_step(z, orc, step, fmt_m, fmt_v)
-            z.all_gather_weights()
+            if step == 2:
+                z.all_gather_weights(async_op=True).wait()
+            else:
+                z.all_gather_weights()
             _reference_step(orc, ref, _summed_grads(z), step, fmt_m, fmt_v)
             _compare(z, ref, (rank, step))
         dist.barrier()
