@@ -270,13 +270,17 @@ template <int FM, int FV, bool FULL>
 __device__ __forceinline__ void process(const LaneIn& in, const TileHeader& t, const int (&off)[4],
                                         int lg, bool active, int slot, int l, const StepHyper& h,
                                         float omb1, float omb2, float gs, const Smem& S) {
-  // dequantisation constants of this group (stored k and root scale)
-  const float invk_m = rcp_approx(in.mk), sb_m = in.ms * h.beta1;
-  const float invk_v = rcp_approx(in.vk), sb_v = in.vs * h.beta2;
+  // dequantisation constants of this group (stored k and root scale), as
+  // (m, v) pairs for the packed FP32 operations
+  const float invk_m = rcp_approx(in.mk);
+  const float2 invk = make_float2(invk_m, rcp_approx(in.vk));
+  const float2 sb = mul2(make_float2(in.ms, in.vs), make_float2(h.beta1, h.beta2));
   // 1/k of the m state in double for the min recompute (one Newton step from
   // the FP32 reciprocal: ~1e-14 relative)
   const double kd = static_cast<double>(in.mk), r0 = static_cast<double>(invk_m);
   const double invk_md = r0 * fma(-kd, r0, 2.0);
+  const float2 dsq2 = make_float2(h.dsq, h.dsq), deps2 = make_float2(h.deps, h.deps);
+  const float2 lrwd2 = make_float2(t.lrwd, t.lrwd), omb2x2 = make_float2(omb2, omb2);
 
   float m1[16], v1[16];
   float maxm = 0.f, maxv = 0.f;
@@ -286,31 +290,49 @@ __device__ __forceinline__ void process(const LaneIn& in, const TileHeader& t, c
   for (int j = 0; j < 4; ++j) {
     const int e = off[j];
     float pn[4];
+    // element pairs (2u, 2u + 1): the two bf16 gradients of one word
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t gw = (i < 2) ? in.g[j].x : in.g[j].y;
-      const float g = (i & 1) ? bf16hi(gw) : bf16lo(gw);
-      const uint32_t cm = __byte_perm(in.mq[j], 0u, 0x4440u + i);
-      const uint32_t cv = __byte_perm(in.vq[j], 0u, 0x4440u + i);
-      // beta1 * m and beta2 * v, dequantised: s_r * beta * 2^(log2|q| / k)
-      float bm = ex2_approx(S.tab_m[cm] * invk_m) * sb_m;
-      bm = __uint_as_float(__float_as_uint(bm) ^ ((in.mq[j] << (24 - 8 * i)) & 0x80000000u));
-      const float bv = ex2_approx(S.tab_v[cv] * invk_v) * sb_v;
-      float mn = __fmaf_rn(omb1, g, bm);
-      float vn = __fmaf_rn(omb2 * g, g, bv);
-      const float p = f4get(in.p[j], i);
-      const float upd = mn * rcp_approx(__fmaf_rn(sqrt_approx(vn), h.dsq, h.deps));
-      pn[i] = p + __fmaf_rn(-p, t.lrwd, -upd);
-      if (!FULL) {
-        const bool valid = active && (e + i < t.nvalid);
-        mn = valid ? mn : 0.f;
-        vn = valid ? vn : 0.f;
+    for (int u = 0; u < 2; ++u) {
+      const uint32_t gw = u ? in.g[j].y : in.g[j].x;
+      const float2 g2 = make_float2(bf16lo(gw), bf16hi(gw));
+      const float2 og = mul2(g2, omb2x2);   // (1 - beta2) g, both elements
+      float2 mv[2];                         // (m', v') of each element
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        const int i = 2 * u + w;
+        const float g = w ? g2.y : g2.x;
+        const uint32_t cm = __byte_perm(in.mq[j], 0u, 0x4440u + i);
+        const uint32_t cv = __byte_perm(in.vq[j], 0u, 0x4440u + i);
+        // beta1 * m and beta2 * v, dequantised: s_r * beta * 2^(log2|q| / k)
+        const float2 tl = mul2(make_float2(S.tab_m[cm], S.tab_v[cv]), invk);
+        float2 b = mul2(make_float2(ex2_approx(tl.x), ex2_approx(tl.y)), sb);
+        b.x = __uint_as_float(__float_as_uint(b.x) ^ ((in.mq[j] << (24 - 8 * i)) & 0x80000000u));
+        // m' = beta1 m + (1 - beta1) g, v' = beta2 v + (1 - beta2) g^2
+        mv[w] = fma2(make_float2(omb1, w ? og.y : og.x), make_float2(g, g), b);
       }
-      m1[4 * j + i] = mn;
-      v1[4 * j + i] = vn;
-      maxm = fmaxf(maxm, fabsf(mn));
-      maxv = fmaxf(maxv, vn);
-      minv = min(minv, __float_as_uint(vn) - 1u);
+      // p - (p lr wd + m' / (sqrt(v') dsq + deps)) for both elements
+      const float2 den = fma2(make_float2(sqrt_approx(mv[0].y), sqrt_approx(mv[1].y)), dsq2, deps2);
+      const float2 upd = mul2(make_float2(mv[0].x, mv[1].x),
+                              make_float2(rcp_approx(den.x), rcp_approx(den.y)));
+      const float2 p = make_float2(f4get(in.p[j], 2 * u), f4get(in.p[j], 2 * u + 1));
+      const float2 pnew = sub2(p, fma2(p, lrwd2, upd));
+      pn[2 * u] = pnew.x;
+      pn[2 * u + 1] = pnew.y;
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        const int i = 2 * u + w;
+        float mn = mv[w].x, vn = mv[w].y;
+        if (!FULL) {
+          const bool valid = active && (e + i < t.nvalid);
+          mn = valid ? mn : 0.f;
+          vn = valid ? vn : 0.f;
+        }
+        m1[4 * j + i] = mn;
+        v1[4 * j + i] = vn;
+        maxm = fmaxf(maxm, fabsf(mn));
+        maxv = fmaxf(maxv, vn);
+        minv = min(minv, __float_as_uint(vn) - 1u);
+      }
     }
     // two smallest m keys: merge the sorted pairs of elements (0,1), (2,3)
 #pragma unroll
@@ -388,6 +410,8 @@ __device__ __forceinline__ void process(const LaneIn& in, const TileHeader& t, c
   const float invMm = __shfl_sync(0xFFFFFFFFu, invMx, lane_m);
   const float kv = __shfl_sync(0xFFFFFFFFu, kx, lane_v);
   const float invMv = __shfl_sync(0xFFFFFFFFu, invMx, lane_v);
+  const float2 invM2 = make_float2(invMm, invMv), k2 = make_float2(km, kv);
+  const float2 log2max2 = make_float2(F8<FM>::LOG2MAX_HI, F8<FV>::LOG2MAX_HI);
 
   // expand + encode, store codes (whole group, padding included) and metadata
 #pragma unroll
@@ -396,8 +420,12 @@ __device__ __forceinline__ void process(const LaneIn& in, const TileHeader& t, c
     uint32_t cmw[4], cvw[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      cmw[i] = enc_mag_bounded<FM>(expand_value<FM>(m1[4 * j + i], invMm, km));
-      cvw[i] = enc_mag_bounded<FV>(expand_value<FV>(v1[4 * j + i], invMv, kv));
+      // y = FMT_MAX (|x| / M)^k = 2^(k log2(|x| / M) + log2 FMT_MAX) for m' and v'
+      const float2 a = mul2(make_float2(m1[4 * j + i], v1[4 * j + i]), invM2);
+      const float2 ty = fma2(k2, make_float2(lg2_approx(fabsf(a.x)), lg2_approx(fabsf(a.y))), log2max2);
+      const uint2 c = enc_mag_bounded2<FM, FV>(ex2_approx(ty.x), ex2_approx(ty.y));
+      cmw[i] = c.x;
+      cvw[i] = c.y;
     }
     if (FULL || active) {
       *reinterpret_cast<uint32_t*>(t.mq + e) =
