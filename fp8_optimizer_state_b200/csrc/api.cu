@@ -693,9 +693,28 @@ namespace {
 struct NoAllocScratch {
   coat::TensorArgs descs[COAT_NOALLOC_MAX_TENSORS];
 };
+// The size include/coat.h states for the array (104 bytes per descriptor).
+static_assert(sizeof(coat::TensorArgs) == 104, "descriptor size stated in coat.h");
+static_assert(sizeof(NoAllocScratch) == 106496, "array size stated in coat.h");
 
 // Every GPU that loads the library holds this array until the process exits.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[sizeof(NoAllocScratch)];
+
+// Descriptors travel to the array as kernel parameters, a chunk per launch:
+// the launch copies its parameters when it is enqueued, so no host buffer has
+// to outlive the call and no pageable-memory copy (which may wait for earlier
+// work on the stream) is involved.  32 descriptors keep the parameters below
+// the classic 4 KB limit.
+constexpr int kNoAllocChunk = 32;
+struct NoAllocChunk {
+  coat::TensorArgs d[kNoAllocChunk];
+};
+static_assert(sizeof(NoAllocChunk) + 16 <= 4096, "kernel parameter space");
+
+__global__ void noalloc_stage_kernel(const NoAllocChunk chunk, int count, coat::TensorArgs* dst) {
+  const int i = threadIdx.x;
+  if (i < count) dst[i] = chunk.d[i];
+}
 
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[64];
@@ -754,36 +773,17 @@ extern "C" coat_status coat_adamw_step_multi_noalloc(const coat_tensor_desc* hos
   if (noalloc_scratch_ptr(&scratch) != cudaSuccess || coat::device_error_ptr(&err) != cudaSuccess)
     return COAT_ERR_CUDA;
 
-  // Stage the descriptor table through a small stack buffer, one async copy per
-  // chunk on the caller's stream (a copy from pageable memory returns once the
-  // source has been read, so the buffer can be reused at once).
-  constexpr int kChunk = 32;
-  coat::TensorArgs buf[kChunk];
+  // The table, chunk by chunk, each entry built exactly as a plan builds it.
+  NoAllocChunk chunk = {};
   int64_t tiles = 0;
-  const int64_t tg = coat::step_tile_groups();
-  for (int c0 = 0; c0 < num; c0 += kChunk) {
-    const int cn = num - c0 < kChunk ? num - c0 : kChunk;
+  for (int c0 = 0; c0 < num; c0 += kNoAllocChunk) {
+    const int cn = num - c0 < kNoAllocChunk ? num - c0 : kNoAllocChunk;
     for (int j = 0; j < cn; ++j) {
-      const coat_tensor_desc& d = host_descs[c0 + j];
-      coat::TensorArgs& t = buf[j];
-      t.master = d.master;
-      t.wout = d.weight_bf16_out;
-      t.grad = d.grad;
-      t.mq = d.m_q;
-      t.ms = d.m_scale;
-      t.mk = d.m_k;
-      t.vq = d.v_q;
-      t.vs = d.v_scale;
-      t.vk = d.v_k;
-      t.n = d.n;
-      t.tiles = ((d.n + 127) / 128 + tg - 1) / tg;
-      t.tile_begin = tiles;
-      t.wd_scale = 1.0f;
-      tiles += t.tiles;
+      chunk.d[j] = to_args(host_descs[c0 + j], tiles);
+      tiles += chunk.d[j].tiles;
     }
-    if (cudaMemcpyAsync(scratch->descs + c0, buf, sizeof(coat::TensorArgs) * cn,
-                        cudaMemcpyHostToDevice, stream) != cudaSuccess)
-      return COAT_ERR_CUDA;
+    noalloc_stage_kernel<<<1, kNoAllocChunk, 0, stream>>>(chunk, cn, scratch->descs + c0);
+    if (cudaGetLastError() != cudaSuccess) return COAT_ERR_CUDA;
   }
   if (tiles == 0) return COAT_OK;
   const cudaError_t e =

@@ -139,7 +139,7 @@ coat_status coat_group_dequantize(const uint8_t *q, int64_t ld_q, const float *s
  * m_scale, m_k, v_scale, v_k: ceil(n/128) floats each.
  * Alignment: every pointer 16-byte aligned (COAT_ERR_MISALIGNED otherwise).
  * Hyperparameters: lr >= 0, 0 <= beta1, beta2 < 1, eps > 0, wd >= 0, all finite;
- * step >= 1.  fmt_m, fmt_v: COAT_E4M3 or COAT_E5M2.
+ * step >= 1.  fmt_m, fmt_v: COAT_E4M3, COAT_E5M2 or COAT_E5M2_FULL.
  * ------------------------------------------------------------------------- */
 coat_status coat_adamw_step(float *master, uint16_t *weight_bf16_out, const uint16_t *grad,
                             uint8_t *m_q, float *m_scale, float *m_k, uint8_t *v_q,
@@ -264,23 +264,28 @@ coat_status coat_grad_clip_finalize(coat_grad_clip *d_clip, float max_norm, cuda
  * image instead of a cudaMalloc'd plan table.  It allocates nothing: no
  * cudaMalloc/cudaFree, no allocating library routine, no heap use.
  *
- *   - host_descs: num descriptors in host memory (read during the call; the
- *     caller may free them on return).  Each obeys the coat_adamw_step rules.
+ *   - host_descs: num descriptors in host memory, read before the call returns
+ *     (the caller may change or free them on return).  Each obeys the
+ *     coat_adamw_step rules.
  *   - num: 1 .. COAT_NOALLOC_MAX_TENSORS.  A larger num returns
  *     COAT_ERR_UNSUPPORTED (as does group != 128); other bad arguments return
  *     COAT_ERR_INVALID_ARG or COAT_ERR_MISALIGNED, before anything is enqueued.
  *     This call reports through its return code only: it does not record a
  *     message, so coat_last_error() keeps describing an earlier failure.
- *   - The fixed array holds COAT_NOALLOC_MAX_TENSORS kernel descriptors
- *     (96 KB); every GPU that loads the library keeps it until the process
- *     exits.
+ *   - The fixed array holds COAT_NOALLOC_MAX_TENSORS kernel descriptors of
+ *     104 bytes each (106,496 bytes); every GPU that loads the library keeps
+ *     it until the process exits.
  *   - The first call on a device looks up the array's device address (with
  *     that device current) and configures the kernel; make that first call
  *     before any stream capture.
- *   - Each call copies the table into the array on `stream`, then launches on
- *     `stream`.  All calls share the one array and it keeps the last call's
- *     contents: calls that may overlap on the GPU (different streams without
- *     ordering between them) race on it and must not be issued.
+ *   - Each call enqueues, on `stream`, small copy kernels that write the table
+ *     into the array (the descriptors travel as their kernel parameters, 32
+ *     per launch, so no host buffer is read after the call returns and no
+ *     copy from pageable memory makes the call wait for earlier work on
+ *     `stream`), then the step kernel.  All calls share the one array and it
+ *     keeps the last call's contents: calls that may overlap on the GPU
+ *     (different streams without ordering between them) race on it and must
+ *     not be issued.
  * ------------------------------------------------------------------------- */
 #define COAT_NOALLOC_MAX_TENSORS 1024
 coat_status coat_adamw_step_multi_noalloc(const coat_tensor_desc *host_descs, int num, int group,

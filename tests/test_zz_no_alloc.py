@@ -5,8 +5,9 @@ Its tensor table lives in a fixed array inside the library instead of a plan's
 cudaMalloc'd table.
 
 Checked here through the C ABI: two calls in a row give exactly the bits of the
-plan-based entry point on the same inputs, and a table larger than the fixed
-array is rejected.  This file is collected last on purpose; it needs nothing
+plan-based entry point on the same inputs, a table of the largest accepted size
+gives them too even when the caller overwrites its host table as soon as the
+call returns, and a table larger than the fixed array is rejected.  This file is collected last on purpose; it needs nothing
 from the other tests and passes on its own in a fresh process."""
 import ctypes
 
@@ -93,3 +94,33 @@ def test_noalloc_rejects_tables_beyond_the_fixed_array():
     before = t["master"].clone()
     torch.cuda.synchronize()
     assert torch.equal(t["master"], before)      # nothing was launched
+
+
+def test_noalloc_full_table_and_host_table_reused_at_once():
+    """A table of the largest size (COAT_NOALLOC_MAX_TENSORS tensors, staged in
+    chunks) matches the plan-based call, and the host table may be overwritten
+    as soon as the call returns: the call has read it by then."""
+    fm, fv = 0, 2
+    rng = np.random.default_rng(5)
+    sizes = [int(x) for x in rng.integers(1, 2500, coat.NOALLOC_MAX_TENSORS)]
+    sizes[17] = 0
+    a = make_set(sizes, fm, fv, seed=9)
+    b = make_set(sizes, fm, fv, seed=9)
+    plan = coat.coat_multi_plan_create(descs_of(a), fm, fv)
+    stream = torch.cuda.current_stream().cuda_stream
+    L = coat.lib()
+    for step in (1, 2):
+        set_grads(a, step, seed=9)
+        set_grads(b, step, seed=9)
+        arr = (coat.TensorDesc * len(sizes))(*descs_of(b))
+        coat.coat_adamw_step_multi(plan, step=step, **H)
+        st = L.coat_adamw_step_multi_noalloc(ctypes.cast(arr, ctypes.c_void_p), len(sizes), 128,
+                                             H["lr"], H["beta1"], H["beta2"], H["eps"], H["wd"],
+                                             step, fm, fv, stream)
+        assert st == OK
+        ctypes.memset(arr, 0xFF, ctypes.sizeof(arr))   # the GPU may not have run the copies yet
+        coat.coat_check_device_error()
+        for da, db in zip(a, b):
+            for key in ("master", "weight", "mq", "ms", "mk", "vq", "vs", "vk"):
+                assert torch.equal(da[key], db[key]), (step, key)
+    plan.destroy()
