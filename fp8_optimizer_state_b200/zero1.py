@@ -20,6 +20,13 @@ B200s); the step is the library's kernel and no arithmetic of the step runs
 here.  Gradients are summed, not averaged: scale the loss by 1/world_size for
 their mean.  Groups never span ranks, so the result is the single-GPU step on
 the summed gradients, bit for bit.
+
+The sum itself is taken in bf16 by the collective, which may round after each
+of its world_size - 1 additions: an element of the summed gradient is within
+(world_size - 1) u (1 + world_size u) sum_r |g_r| of the exact sum (u = 2^-8,
+bf16's unit roundoff; each partial sum is at most sum_r |g_r|).  That is the
+only difference from a step on the exact sum of the ranks' gradients
+(tests/test_zero1_cpu.py checks the bound at 2, 4 and 8 ranks).
 """
 from __future__ import annotations
 

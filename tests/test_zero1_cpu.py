@@ -445,3 +445,53 @@ def test_local_step_refuses_host_tensors():
             z.local_step(step=1, **HP)
     finally:
         dist.destroy_process_group()
+
+
+BF16_U = 2.0 ** -8        # bf16 unit roundoff (8-bit significands, round to nearest)
+
+
+def _sum_bound_main(rank, world, port):
+    """The reduce-scatter sums the ranks' bf16 gradients in bf16 (a reduction
+    may round after every addition), so the summed gradient the step receives
+    differs from the exact sum.  Any order of world - 1 rounded additions keeps
+    |sum - exact| <= (world - 1) u (1 + world u) sum|g_r| (u = 2^-8: each
+    partial sum is at most sum|g_r|).  Each rank regenerates every rank's
+    gradients, sums its shard exactly in double, and checks the bound on every
+    element."""
+    import torch.distributed as dist
+    import synth
+    from fp8_optimizer_state_b200.zero1 import Zero1AdamW
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        sizes = [40000, 777, 131072]
+        z = Zero1AdamW(sizes, device="cpu")
+        worst = 0.0
+        for step in (1, 2):
+            for i, n in enumerate(sizes):
+                bits = synth.grad_bits(50 + rank, i, step, 0, n)
+                z.grad(i).copy_(torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16))
+            z.reduce_scatter_grads()
+            got = _np(z.grad_shard).copy()
+            for t, b, n, sb in z.pieces:
+                parts = [synth.bf16_bits_to_f32(synth.grad_bits(50 + r, t, step, b, n)).astype(np.float64)
+                         for r in range(world)]
+                exact = np.sum(parts, axis=0)
+                mag = np.sum(np.abs(parts), axis=0)
+                val = synth.bf16_bits_to_f32(got[sb:sb + n]).astype(np.float64)
+                bound = (world - 1) * BF16_U * (1 + world * BF16_U) * mag
+                err = np.abs(val - exact)
+                assert np.all(err <= bound), (rank, t, float((err - bound).max()))
+                nz = mag > 0
+                worst = max(worst, float((err[nz] / mag[nz]).max()))
+        print("world %d rank %d: worst |sum - exact| / sum|g| = %.3g (bound %.3g)"
+              % (world, rank, worst, (world - 1) * BF16_U * (1 + world * BF16_U)))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4, 8])
+def test_bf16_gradient_sum_is_within_its_rounding_bound(world):
+    mp.start_processes(_sum_bound_main, args=(world, _free_port()), nprocs=world, join=True,
+                       start_method="spawn")
