@@ -259,6 +259,35 @@ def adamw_step(master, weight_out, grad_bits, m_q, m_scale, m_k, v_q, v_scale, v
     return upd
 
 
+def adamw_step_threads(master, weight_out, grad_bits, m_q, m_scale, m_k, v_q, v_scale, v_k, *,
+                       threads, group=128, **hyper):
+    """adamw_step over `threads` host threads, for timing the oracle on every
+    core: the groups are split into contiguous, group-aligned slices and each
+    slice is one call of the same C step (ctypes releases the GIL for the
+    call).  Groups are independent, so the result is bit for bit that of one
+    call over all of them."""
+    import concurrent.futures as cf
+    n = master.size
+    ng = -(-n // group)
+    threads = max(1, min(int(threads), ng))
+    bounds = [ng * i // threads for i in range(threads + 1)]
+
+    def run(i):
+        g0, g1 = bounds[i], bounds[i + 1]
+        e0, e1 = g0 * group, min(n, g1 * group)
+        if e0 >= e1:
+            return
+        adamw_step(master[e0:e1], None if weight_out is None else weight_out[e0:e1],
+                   grad_bits[e0:e1], m_q[g0 * group:g1 * group], m_scale[g0:g1], m_k[g0:g1],
+                   v_q[g0 * group:g1 * group], v_scale[g0:g1], v_k[g0:g1], group=group, **hyper)
+
+    if threads == 1:
+        run(0)
+        return
+    with cf.ThreadPoolExecutor(threads) as ex:
+        list(ex.map(run, range(threads)))
+
+
 def grad_sumsq(grad_bits):
     """(sum of squares in double, any non-finite) of bf16 gradient bits."""
     g = np.ascontiguousarray(grad_bits, dtype=np.uint16)

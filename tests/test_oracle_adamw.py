@@ -222,3 +222,31 @@ def test_scaled_step_is_the_step_on_the_scaled_gradient(orc):
     assert np.array_equal(ma, mb)
     for x, y in zip(sa, sb):
         assert np.array_equal(x, y)
+
+
+def test_threaded_timing_form_is_bit_identical(orc):
+    """The all-cores timing helper (group-aligned slices, one C call each, on
+    host threads) gives exactly the bytes of one call over every group."""
+    import synth
+    n, fm, fv = 100_003, E4M3, E5M2
+    ng = -(-n // 128)
+    master = synth.master(0, 3, 0, n)
+    g = synth.grad_bits(0, 3, 2, 0, n)
+    mq = np.zeros(ng * 128, np.uint8)
+    vq = np.zeros(ng * 128, np.uint8)
+    mq[:n] = synth.state_codes(0, 3, 2, 0, n, fm, True)
+    vq[:n] = synth.state_codes(0, 3, 2, 0, n, fv, False)
+    km, sm, kv, sv = synth.state_groups(0, 3, 2, 0, ng)
+    hyper = dict(lr=1e-4, beta1=0.9, beta2=0.95, eps=1e-8, wd=0.1, step=2, fmt_m=fm, fmt_v=fv)
+    outs = []
+    for threads in (None, 7):
+        st = [a.copy() for a in (master, mq, sm, km, vq, sv, kv)]
+        w = np.zeros(n, np.uint16)
+        if threads is None:
+            orc.adamw_step(st[0], w, g, st[1], st[2], st[3], st[4], st[5], st[6], **hyper)
+        else:
+            orc.adamw_step_threads(st[0], w, g, st[1], st[2], st[3], st[4], st[5], st[6],
+                                   threads=threads, **hyper)
+        outs.append(st + [w])
+    for a, b in zip(*outs):
+        assert np.array_equal(a, b)
