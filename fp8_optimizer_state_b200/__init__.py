@@ -8,17 +8,21 @@ CPU fallback -- if libcoat.so is missing, every call raises.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libcoat.so")
+# the checked build (index checks in every kernel; see include/coat.h)
+LIB_CHECKED_PATH = os.path.join(HERE, "libcoat_debug.so")
 
 COAT_E4M3, COAT_E5M2, COAT_E5M2_FULL = 0, 1, 2
 COAT_F32, COAT_BF16 = 0, 1
 GROUP = 128
 STATUS = {0: "COAT_OK", 1: "COAT_ERR_INVALID_ARG", 2: "COAT_ERR_MISALIGNED",
-          3: "COAT_ERR_UNSUPPORTED", 4: "COAT_ERR_CUDA", 5: "COAT_ERR_TIMEOUT", 6: "COAT_ERR_NOMEM"}
+          3: "COAT_ERR_UNSUPPORTED", 4: "COAT_ERR_CUDA", 5: "COAT_ERR_TIMEOUT", 6: "COAT_ERR_NOMEM",
+          7: "COAT_ERR_DEVICE_CHECK"}
 
 # (name, restype, argtypes) of every exported entry point
 _vp, _i64, _i32, _f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
@@ -39,6 +43,8 @@ EXPORTS = [
     ("coat_multi_plan_set_wd_scale", _i32, [_vp, _vp, _vp]),
     ("coat_multi_plan_info", _i32, [_vp, ctypes.POINTER(_i64), ctypes.POINTER(_i32)]),
     ("coat_check_device_error", _i32, [_vp]),
+    ("coat_build_checked", _i32, []),
+    ("coat_set_exact_group_params", _i32, [_i32]),
     ("coat_adamw_step_multi_noalloc", _i32, [_vp, _i32, _i32, _f32, _f32, _f32, _f32, _f32, _i64,
                                              _i32, _i32, _vp]),
     ("coat_selftest_wait_timeout", _i32, [_i64, _vp]),
@@ -164,27 +170,48 @@ class TensorDesc(ctypes.Structure):
 
 
 _lib = None
+_loaded = {}
 
 
-def lib():
-    """Load libcoat.so (raises if it has not been built)."""
-    global _lib
-    if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError("libcoat.so is not built (%s); run "
-                               "`python -m fp8_optimizer_state_b200.build`" % LIB_PATH)
-        L = ctypes.CDLL(LIB_PATH)
+def _load(path):
+    if path not in _loaded:
+        if not os.path.exists(path):
+            raise RuntimeError("%s is not built; run `python -m fp8_optimizer_state_b200.build`"
+                               " (add --checked for the checked build)" % path)
+        L = ctypes.CDLL(path)
         for name, res, args in EXPORTS:
             f = getattr(L, name)
             f.restype = res
             f.argtypes = args
-        _lib = L
+        _loaded[path] = L
+    return _loaded[path]
+
+
+def lib():
+    """The loaded library: libcoat.so, or the checked build libcoat_debug.so
+    when the environment sets COAT_DEBUG=1 (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        _lib = _load(LIB_CHECKED_PATH if os.environ.get("COAT_DEBUG") == "1" else LIB_PATH)
     return _lib
 
 
-def _check(status):
+@contextlib.contextmanager
+def checked_library():
+    """Route every call of this module to the checked build inside the block
+    (a plan keeps the library that created it)."""
+    global _lib
+    prev = lib()
+    _lib = _load(LIB_CHECKED_PATH)
+    try:
+        yield _lib
+    finally:
+        _lib = prev
+
+
+def _check(status, L=None):
     if status != 0:
-        raise CoatError(status, lib().coat_last_error().decode())
+        raise CoatError(status, (L or lib()).coat_last_error().decode())
 
 
 def _p(t):
@@ -266,18 +293,21 @@ class coat_multi_plan:
     def __init__(self, handle, descs):
         self.handle = handle
         self._descs = descs
+        self._lib = lib()
 
     def info(self):
         n = ctypes.c_int64()
         c = ctypes.c_int()
-        _check(lib().coat_multi_plan_info(self.handle, ctypes.byref(n), ctypes.byref(c)))
+        _check(self._lib.coat_multi_plan_info(self.handle, ctypes.byref(n), ctypes.byref(c)),
+               self._lib)
         return n.value, c.value
 
     def set_wd_scale(self, scales, stream=None):
         """Per-tensor weight decay multipliers (coat_multi_plan_set_wd_scale)."""
         arr = (ctypes.c_float * len(scales))(*[float(x) for x in scales])
-        _check(lib().coat_multi_plan_set_wd_scale(self.handle, ctypes.cast(arr, ctypes.c_void_p),
-                                                  _s(stream)))
+        _check(self._lib.coat_multi_plan_set_wd_scale(self.handle,
+                                                      ctypes.cast(arr, ctypes.c_void_p), _s(stream)),
+               self._lib)
 
     def grad_norm(self, max_norm, clip_buf, stream=None):
         """coat_multi_plan_grad_norm into clip_buf (see new_grad_clip)."""
@@ -285,7 +315,7 @@ class coat_multi_plan:
 
     def destroy(self):
         if self.handle:
-            _check(lib().coat_multi_plan_destroy(self.handle))
+            _check(self._lib.coat_multi_plan_destroy(self.handle), self._lib)
             self.handle = None
 
     def __del__(self):
@@ -305,21 +335,23 @@ def coat_multi_plan_create(descs, fmt_m=COAT_E4M3, fmt_v=COAT_E4M3, group=GROUP,
 
 
 def coat_adamw_step_multi(plan, *, lr, beta1, beta2, eps, wd, step, stream=None):
-    _check(lib().coat_adamw_step_multi(plan.handle, lr, beta1, beta2, eps, wd, step, _s(stream)))
+    _check(plan._lib.coat_adamw_step_multi(plan.handle, lr, beta1, beta2, eps, wd, step,
+                                           _s(stream)), plan._lib)
 
 
 def coat_multi_plan_grad_norm(plan, max_norm, clip_buf, stream=None):
     if clip_buf.numel() * clip_buf.element_size() < ctypes.sizeof(GradClip):
         raise ValueError("clip_buf must hold %d bytes" % ctypes.sizeof(GradClip))
-    _check(lib().coat_multi_plan_grad_norm(plan.handle, max_norm, _p(clip_buf), _s(stream)))
+    _check(plan._lib.coat_multi_plan_grad_norm(plan.handle, max_norm, _p(clip_buf), _s(stream)),
+           plan._lib)
 
 
 def coat_adamw_step_multi_clipped(plan, clip_buf, *, lr, beta1, beta2, eps, wd, step,
                                   stream=None):
     if clip_buf.numel() * clip_buf.element_size() < ctypes.sizeof(GradClip):
         raise ValueError("clip_buf must hold %d bytes" % ctypes.sizeof(GradClip))
-    _check(lib().coat_adamw_step_multi_clipped(plan.handle, lr, beta1, beta2, eps, wd, step,
-                                               _p(clip_buf), _s(stream)))
+    _check(plan._lib.coat_adamw_step_multi_clipped(plan.handle, lr, beta1, beta2, eps, wd, step,
+                                                   _p(clip_buf), _s(stream)), plan._lib)
 
 
 def coat_grad_clip_finalize(clip_buf, max_norm, stream=None):
@@ -367,6 +399,21 @@ def coat_zero1_layout(sizes, world_size, rank, group=GROUP):
                                    ctypes.cast(offs, _vp)))
     out = [(p.tensor, p.elem_begin, p.n_elems, p.shard_begin) for p in pieces[:cnt.value]]
     return out, shard.value, flat.value, list(offs)
+
+
+def coat_set_exact_group_params(on):
+    """Group-parameter mode of the step (see include/coat.h); returns the previous one."""
+    return lib().coat_set_exact_group_params(int(bool(on)))
+
+
+@contextlib.contextmanager
+def exact_group_params(on=True):
+    """Run the block with the step's group-parameter mode set to `on`."""
+    prev = coat_set_exact_group_params(on)
+    try:
+        yield
+    finally:
+        coat_set_exact_group_params(prev)
 
 
 def coat_check_device_error(stream=None):

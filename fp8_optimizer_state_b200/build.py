@@ -1,6 +1,9 @@
-"""Build libcoat.so in-tree with nvcc for sm_100a (B200) only.
+"""Build libcoat.so in-tree with nvcc for sm_100a (B200) only, and its checked
+variant libcoat_debug.so (compiled with COAT_DEBUG: every kernel checks the
+indices it derives before each access, counts failures on the device and
+skips the access; see coat_check_device_error in include/coat.h).
 
-    python -m fp8_optimizer_state_b200.build [--force] [--verbose-ptxas]
+    python -m fp8_optimizer_state_b200.build [--force] [--verbose-ptxas] [--checked]
 
 The library links the CUDA runtime statically, so loading it needs no CUDA
 driver (a GPU-less host can load it and check its exports); the first CUDA
@@ -19,6 +22,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libcoat.so")
+LIB_CHECKED = os.path.join(HERE, "libcoat_debug.so")
 SOURCES = ["api.cu", "adamw_fp8.cu", "codec.cu", "fp8_flow.cu"]
 HEADERS = ["coat_device.cuh", "coat_internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -40,14 +44,15 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, ptxas_verbose: bool = False) -> str:
+def build(force: bool = False, ptxas_verbose: bool = False, checked: bool = False) -> str:
+    lib = LIB_CHECKED if checked else LIB
     deps = [os.path.join(CSRC, s) for s in SOURCES + HEADERS] + [os.path.join(INCLUDE, "coat.h"),
                                                                  __file__]
-    if not force and not _stale(LIB, deps):
-        return LIB
-    objdir = os.path.join(HERE, "_build")
+    if not force and not _stale(lib, deps):
+        return lib
+    objdir = os.path.join(HERE, "_build_checked" if checked else "_build")
     os.makedirs(objdir, exist_ok=True)
-    extra = ["-Xptxas", "-v"] if ptxas_verbose else []
+    extra = (["-Xptxas", "-v"] if ptxas_verbose else []) + (["-DCOAT_DEBUG"] if checked else [])
 
     def compile_one(src):
         obj = os.path.join(objdir, src.replace(".cu", ".o"))
@@ -61,14 +66,15 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
 
     with cf.ThreadPoolExecutor(len(SOURCES)) as ex:
         objs = list(ex.map(compile_one, SOURCES))
-    tmp = LIB + ".tmp%d" % os.getpid()
+    tmp = lib + ".tmp%d" % os.getpid()
     cmd = [nvcc()] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("link failed:\n%s\n%s" % (r.stdout, r.stderr))
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, ptxas_verbose="--verbose-ptxas" in sys.argv))
+    print(build(force="--force" in sys.argv, ptxas_verbose="--verbose-ptxas" in sys.argv,
+                checked="--checked" in sys.argv))

@@ -10,15 +10,17 @@
 //
 // Design (HBM-bound: 16.25 algorithmic bytes per parameter, no tensor cores):
 //  * one persistent CTA per SM, 16 warps (4 per SM sub-partition, so a thread
-//    may use 128 registers); tiles of 60 groups (7680 elements); every CTA owns
-//    a contiguous range of tiles;
+//    may use 128 registers); tiles of 60 groups (7680 elements); CTA b takes
+//    tiles b, b + grid, b + 2 grid, ...;
 //  * one producer thread streams whole tiles (master, grad, both code arrays,
 //    the four metadata arrays: 62,400 B) into a 3-stage shared-memory ring
 //    with 1-D cp.async.bulk copies completing on an mbarrier (30 KB per copy
 //    of the master array), so that bytes in flight do not depend on
-//    registers.  It walks the tensor list forward with its range, keeps the
-//    current tensor's descriptor in registers and writes the tile's array
-//    pointers into the stage header;
+//    registers; every byte is read once, so the copies carry an L2
+//    evict-first policy and the results are written with streaming stores.
+//    It walks the tensor list forward with its tiles, keeps the current
+//    tensor's descriptor in registers and writes the tile's array pointers
+//    into the stage header;
 //  * 15 consumer warps; each warp owns 4 groups of a tile, 8 lanes per group,
 //    16 elements per lane in 4 chunks of 4 contiguous elements (chunk order
 //    rotated per group to keep shared-memory reads conflict-free); group
@@ -92,14 +94,26 @@ struct Feed {
   int32_t ti;          // index of the current tensor
 };
 
+// log2(F) and 1/F for F = 1 + (j + 1/2)/128, the centre of the j-th of 128
+// equal bins of [1, 2) (log2_table below).
+struct LogEntry {
+  double log2f, inv;
+};
+
 struct Smem {
-  double tabd_m[256];  // log2|value(code)| of the m format, double (min recompute)
-  double exp2_16[16];  // 2^(j/16), double
-  float tab_m[256];    // log2|value(code)| of the m format
-  float tab_v[256];    // log2|value(code)| of the v format
+  double tabd_m[256];   // log2|value(code)| of the m format, double (group extremes)
+  double tabd_v[256];   // log2|value(code)| of the v format, double
+  LogEntry lgt[128];
+  double exp2_16[16];   // 2^(j/16), double
+  float tab_m[256];     // log2|value(code)| of the m format
+  float tab_v[256];     // log2|value(code)| of the v format
   uint64_t full_bar[kStages];
   uint64_t empty_bar[kStages];
   TileHeader hdr[kStages];
+  // each consumer lane's m codes, v codes and gradients of the current tile
+  // (64 bytes: 16 + 16 + 32), read back by the lanes that recompute a group's
+  // extreme elements
+  uint4 scratch[kConsumerWarps * 32 * 4];
 };
 constexpr size_t kSmemHead = ((sizeof(Smem) + 127) / 128) * 128;
 constexpr size_t kSmemBytes = kSmemHead + size_t(kStages) * kStageBytes;
@@ -114,6 +128,7 @@ struct SingleTensor {
   __device__ __forceinline__ int32_t find(int64_t) const { return 0; }
   __device__ __forceinline__ TensorArgs get(int32_t) const { return t; }
   __device__ __forceinline__ int64_t begin_of(int32_t) const { return kNoTile; }  // no successor
+  __device__ __forceinline__ int32_t advance(int32_t ti, int64_t) const { return ti; }
 };
 // Multi-tensor launches read a device table of descriptors; the producer finds
 // the tensor of its first tile by binary search (the last tensor whose first
@@ -134,6 +149,22 @@ struct MultiTensor {
   __device__ __forceinline__ TensorArgs get(int32_t i) const { return descs[i]; }
   __device__ __forceinline__ int64_t begin_of(int32_t i) const {
     return i < num ? descs[i].tile_begin : kNoTile;
+  }
+  // The tensor of `tile` (the last one whose first tile is <= tile), searching
+  // forward from tensor ti, which starts at or before it.  Eight first-tile
+  // indices are read per round with independent loads, so a jump across many
+  // small tensors costs one memory latency per eight of them.
+  __device__ __forceinline__ int32_t advance(int32_t ti, int64_t tile) const {
+    for (;;) {
+      int64_t b[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) b[k] = begin_of(ti + 1 + k);
+      int c = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) c += b[k] <= tile ? 1 : 0;
+      ti += c;
+      if (c < 8) return ti;
+    }
   }
 };
 
@@ -193,8 +224,10 @@ __device__ __forceinline__ void load_direct(const TileHeader& hd, const int (&of
         p = make_float4(pv[0], pv[1], pv[2], pv[3]);
         g = make_uint2(gv[0] | (gv[1] << 16), gv[2] | (gv[3] << 16));
       }
-      mq = *reinterpret_cast<const uint32_t*>(hd.mq + e);
-      vq = *reinterpret_cast<const uint32_t*>(hd.vq + e);
+      if (COAT_INDEX_OK(e + 4 <= hd.ngroups * kGroup)) {
+        mq = *reinterpret_cast<const uint32_t*>(hd.mq + e);
+        vq = *reinterpret_cast<const uint32_t*>(hd.vq + e);
+      }
     }
     in.p[j] = p;
     in.g[j] = g;
@@ -214,14 +247,16 @@ __device__ __forceinline__ float f4get(const float4& v, int i) {
 // 2^t in double for |t| < 1000, table-driven (P. T. P. Tang, "Table-driven
 // implementation of the exponential function", ACM TOMS 15(2), 1989):
 // t = (16n' + j)/16 + r with |r| <= 1/32, 2^t = 2^n' * 2^(j/16) * e^(r ln 2),
-// the last factor by its Taylor series to the z^5 term (|z| <= ln2/32, so the
-// truncation is below 2e-13 relative).
+// the last factor by its Taylor series to the z^7 term (|z| <= ln2/32, so the
+// truncation is below 2e-18 relative).
 __device__ __forceinline__ double exp2_table(double t, const double* exp2_16) {
   const double s = t * 16.0;
   const double n = rint(s);
   const double z = (s - n) * 0.043321698784996581;  // (s - n)/16 * ln 2
   const int ni = static_cast<int>(n);
-  double p = fma(z, 1.0 / 120.0, 1.0 / 24.0);
+  double p = fma(z, 1.0 / 5040.0, 1.0 / 720.0);
+  p = fma(p, z, 1.0 / 120.0);
+  p = fma(p, z, 1.0 / 24.0);
   p = fma(p, z, 1.0 / 6.0);
   p = fma(p, z, 0.5);
   p = fma(p, z, 1.0);
@@ -230,14 +265,42 @@ __device__ __forceinline__ double exp2_table(double t, const double* exp2_16) {
   return exp2_16[ni & 15] * p * scale;
 }
 
-// The element of a group with the smallest nonzero |m'| usually comes from
-// cancellation between beta1*m and (1-beta1)*g, so its FP32 value carries the
-// FP32 dequantisation error amplified by |beta1 m| / |m'| (often 100x-1000x),
-// and k depends on it through ln(max/min).  The kernel keeps the two smallest
-// candidates (their positions packed into the low 8 bits of the comparison
-// keys, at a cost of 2^-16 relative in the ordering) and recomputes them in
-// double precision: dequantisation, then m' = beta1 m + (1 - beta1) gs g, gs
-// the gradient-clipping coefficient (1 without clipping).
+// log2(x) in double for a finite normal x > 0, table-driven: x = 2^e f with f in
+// [1, 2), F the centre of f's bin of width 1/128 (f - F is exact), r = (f - F)/F
+// with |r| < 2^-8, log2 x = e + log2 F + ln(1 + r) log2(e), ln(1 + r) by its
+// series to the r^6 term (truncation below 1e-17).
+__device__ __forceinline__ double log2_table(double x, const LogEntry* lgt) {
+  const long long b = __double_as_longlong(x);
+  const int e = static_cast<int>(b >> 52) - 1023;
+  const int j = static_cast<int>((b >> 45) & 127);
+  const double f = __longlong_as_double((b & 0x000FFFFFFFFFFFFFLL) | 0x3FF0000000000000LL);
+  const double F = 1.0 + (static_cast<double>(j) + 0.5) * (1.0 / 128.0);
+  const LogEntry E = lgt[j];
+  const double r = (f - F) * E.inv;
+  double q = fma(r, -1.0 / 6.0, 0.2);
+  q = fma(q, r, -0.25);
+  q = fma(q, r, 1.0 / 3.0);
+  q = fma(q, r, -0.5);
+  q = fma(q, r, 1.0);
+  return fma(q * r, 1.4426950408889634, static_cast<double>(e) + E.log2f);
+}
+
+// 1/x in double for x in [2^-120, 2^120]: the FP32 reciprocal refined by two
+// Newton steps (within about an ulp of 1/x; no division).
+__device__ __forceinline__ double rcp_d(double x) {
+  double r = static_cast<double>(rcp_approx(__double2float_rn(x)));
+  r = r * fma(-x, r, 2.0);
+  return r * fma(-x, r, 2.0);
+}
+
+// The fast group parameters' minimum: the element of a group with the
+// smallest nonzero |m'| usually comes from cancellation between beta1 m and
+// (1 - beta1) g, so its FP32 value carries the FP32 dequantisation error
+// amplified by |beta1 m| / |m'| (often 100x-1000x), and k depends on it
+// through ln(max/min).  The kernel keeps the two smallest candidates (their
+// positions packed into the low bits of the comparison keys) and recomputes
+// them in double precision: dequantisation (zero for a zero code), then
+// m' = beta1 m + (1 - beta1) gs g, gs the gradient-clipping coefficient.
 __device__ __forceinline__ float recompute_m_double(const LaneIn& in, int idx, double invk,
                                                     const StepHyper& h, float gs,
                                                     const double* tabd_m,
@@ -248,43 +311,63 @@ __device__ __forceinline__ float recompute_m_double(const LaneIn& in, int idx, d
   const uint32_t c = (mw >> (8 * i)) & 0xFFu;
   const uint32_t gw = (i < 2) ? gw2.x : gw2.y;
   const float g = (i & 1) ? bf16hi(gw) : bf16lo(gw);
-  double x = exp2_table(tabd_m[c] * invk, exp2_16) * static_cast<double>(in.ms);
+  double x = (c & 0x7Fu) ? exp2_table(tabd_m[c] * invk, exp2_16) * static_cast<double>(in.ms) : 0.0;
   if (c & 0x80u) x = -x;
   const double b1 = static_cast<double>(h.beta1);
   const double m1 = fma(b1, x, (1.0 - b1) * (static_cast<double>(gs) * static_cast<double>(g)));
   return __double2float_rn(fabs(m1));
 }
-
-// Comparison key of |x|: the FP32 bits shifted left by one (dropping the sign)
-// minus two, so that zero becomes the largest key and the order of nonzero
-// magnitudes is kept; the low 5 bits are replaced by the element index.
 __device__ __forceinline__ uint32_t min_key(float x, int idx) {
   return ((__float_as_uint(x) * 2u - 2u) & 0xFFFFFFE0u) | static_cast<uint32_t>(idx);
+}
+
+// Comparison keys ordered like |x|, with the element index i (0..15) in the
+// low bits: for m' twice the FP32 bits (the sign drops out) with the low 5 bits
+// replaced by i, for v' (never negative) the FP32 bits with the low 4 bits
+// replaced by i.  A zero gives the key i, below every nonzero key.
+__device__ __forceinline__ uint32_t key_m(float x, int i) {
+  return ((__float_as_uint(x) << 1) & 0xFFFFFFE0u) | static_cast<uint32_t>(i);
+}
+__device__ __forceinline__ uint32_t key_v(float x, int i) {
+  return (__float_as_uint(x) & 0xFFFFFFF0u) | static_cast<uint32_t>(i);
 }
 
 // The per-lane body: everything after the loads.  FULL: every element of the
 // tile is valid (no bounds logic).  The gradient enters scaled by gs (the
 // clipping coefficient, 1 without clipping), folded into the moment weights:
 // omb1 = (1 - beta1) gs and omb2 = (1 - beta2) gs^2.
-template <int FM, int FV, bool FULL>
+template <int FM, int FV, bool EXACT, bool FULL>
 __device__ __forceinline__ void process(const LaneIn& in, const TileHeader& t, const int (&off)[4],
                                         int lg, bool active, int slot, int l, const StepHyper& h,
-                                        float omb1, float omb2, float gs, const Smem& S) {
+                                        float omb1, float omb2, float gs, const Smem& S,
+                                        uint4* scratch_lane, const uint8_t* scratch_warp) {
+  // this lane's codes and gradients, for the lanes that recompute the group's
+  // extreme elements (the previous tile's reads ended at the last shuffle)
+  if constexpr (EXACT) {
+    __syncwarp();
+    scratch_lane[0] = make_uint4(in.mq[0], in.mq[1], in.mq[2], in.mq[3]);
+    scratch_lane[1] = make_uint4(in.vq[0], in.vq[1], in.vq[2], in.vq[3]);
+    scratch_lane[2] = make_uint4(in.g[0].x, in.g[0].y, in.g[1].x, in.g[1].y);
+    scratch_lane[3] = make_uint4(in.g[2].x, in.g[2].y, in.g[3].x, in.g[3].y);
+  }
+
   // dequantisation constants of this group (stored k and root scale), as
   // (m, v) pairs for the packed FP32 operations
-  const float invk_m = rcp_approx(in.mk);
-  const float2 invk = make_float2(invk_m, rcp_approx(in.vk));
+  const float2 invk = make_float2(rcp_approx(in.mk), rcp_approx(in.vk));
   const float2 sb = mul2(make_float2(in.ms, in.vs), make_float2(h.beta1, h.beta2));
-  // 1/k of the m state in double for the min recompute (one Newton step from
-  // the FP32 reciprocal: ~1e-14 relative)
-  const double kd = static_cast<double>(in.mk), r0 = static_cast<double>(invk_m);
-  const double invk_md = r0 * fma(-kd, r0, 2.0);
   const float2 dsq2 = make_float2(h.dsq, h.dsq), deps2 = make_float2(h.deps, h.deps);
   const float2 lrwd2 = make_float2(t.lrwd, t.lrwd), omb2x2 = make_float2(omb2, omb2);
 
   float m1[16], v1[16];
+  // EXACT: keys (key_m, key_v) of the group's extremes: max |m'|, the two
+  // smallest nonzero |m'|, max v', smallest nonzero v' (for the minima the keys
+  // are shifted down by one index block, so that zeros wrap to the top).
+  // Otherwise: max |m'|, max v' and min nonzero v' in FP32, and the keys
+  // (min_key) of the two smallest nonzero |m'|.
+  uint32_t maxmk = 0u, maxvk = 0u, minvk = 0xFFFFFFFFu;
   float maxm = 0.f, maxv = 0.f;
-  uint32_t minm1 = 0xFFFFFFFFu, minm2 = 0xFFFFFFFFu, minv = 0xFFFFFFFFu;
+  uint32_t minv = 0xFFFFFFFFu;
+  uint32_t minm1 = 0xFFFFFFFFu, minm2 = 0xFFFFFFFFu;
 
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -329,25 +412,46 @@ __device__ __forceinline__ void process(const LaneIn& in, const TileHeader& t, c
         }
         m1[4 * j + i] = mn;
         v1[4 * j + i] = vn;
-        maxm = fmaxf(maxm, fabsf(mn));
-        maxv = fmaxf(maxv, vn);
-        minv = min(minv, __float_as_uint(vn) - 1u);
+        if constexpr (!EXACT) {
+          maxm = fmaxf(maxm, fabsf(mn));
+          maxv = fmaxf(maxv, vn);
+          minv = min(minv, __float_as_uint(vn) - 1u);
+        }
       }
     }
-    // two smallest m keys: merge the sorted pairs of elements (0,1), (2,3)
+    if constexpr (EXACT) {
+      // keys of the elements, in pairs (0,1), (2,3); the two smallest m keys
+      // merge the sorted pair into the running pair
+  #pragma unroll
+      for (int i = 0; i < 4; i += 2) {
+        const uint32_t ka = key_m(m1[4 * j + i], 4 * j + i);
+        const uint32_t kb = key_m(m1[4 * j + i + 1], 4 * j + i + 1);
+        maxmk = max(maxmk, max(ka, kb));
+        const uint32_t a = ka - 32u, b = kb - 32u;
+        const uint32_t lo = min(a, b), hi = max(a, b);
+        minm2 = min(max(minm1, lo), min(minm2, hi));
+        minm1 = min(minm1, lo);
+        const uint32_t va = key_v(v1[4 * j + i], 4 * j + i);
+        const uint32_t vb = key_v(v1[4 * j + i + 1], 4 * j + i + 1);
+        maxvk = max(maxvk, max(va, vb));
+        minvk = min(minvk, min(va - 16u, vb - 16u));
+      }
+    } else {
+      // two smallest m keys: merge the sorted pairs of elements (0,1), (2,3)
 #pragma unroll
-    for (int i = 0; i < 4; i += 2) {
-      const uint32_t ka = min_key(m1[4 * j + i], 4 * j + i);
-      const uint32_t kb = min_key(m1[4 * j + i + 1], 4 * j + i + 1);
-      const uint32_t lo = min(ka, kb), hi = max(ka, kb);
-      minm2 = min(max(minm1, lo), min(minm2, hi));
-      minm1 = min(minm1, lo);
+      for (int i = 0; i < 4; i += 2) {
+        const uint32_t ka = min_key(m1[4 * j + i], 4 * j + i);
+        const uint32_t kb = min_key(m1[4 * j + i + 1], 4 * j + i + 1);
+        const uint32_t lo = min(ka, kb), hi = max(ka, kb);
+        minm2 = min(max(minm1, lo), min(minm2, hi));
+        minm1 = min(minm1, lo);
+      }
     }
-    if (FULL || (active && e + 4 <= t.nvalid)) {
-      *reinterpret_cast<float4*>(t.master + e) = make_float4(pn[0], pn[1], pn[2], pn[3]);
+    if (FULL ? COAT_INDEX_OK(e + 4 <= t.nvalid) : (active && e + 4 <= t.nvalid)) {
+      __stcs(reinterpret_cast<float4*>(t.master + e), make_float4(pn[0], pn[1], pn[2], pn[3]));
       if (t.wout)
-        *reinterpret_cast<uint2*>(t.wout + e) =
-            make_uint2(pack_bf16x2(pn[0], pn[1]), pack_bf16x2(pn[2], pn[3]));
+        __stcs(reinterpret_cast<uint2*>(t.wout + e),
+               make_uint2(pack_bf16x2(pn[0], pn[1]), pack_bf16x2(pn[2], pn[3])));
     } else if (active) {
 #pragma unroll
       for (int i = 0; i < 4; ++i)
@@ -358,53 +462,133 @@ __device__ __forceinline__ void process(const LaneIn& in, const TileHeader& t, c
     }
   }
 
-  // group statistics over the 8 lanes of this group.  The m keys carry the
-  // position (lane l, element index) of the two smallest |m'| in their low 7
-  // bits; merging two sorted pairs keeps the two smallest of the union.
-  minm1 = (minm1 & ~0xE0u) | (static_cast<uint32_t>(l) << 5);
-  minm2 = (minm2 & ~0xE0u) | (static_cast<uint32_t>(l) << 5);
-#pragma unroll
-  for (int off = 1; off < 8; off <<= 1) {
-    maxm = fmaxf(maxm, __shfl_xor_sync(0xFFFFFFFFu, maxm, off));
-    maxv = fmaxf(maxv, __shfl_xor_sync(0xFFFFFFFFu, maxv, off));
-    minv = min(minv, __shfl_xor_sync(0xFFFFFFFFu, minv, off));
-    const uint32_t o1 = __shfl_xor_sync(0xFFFFFFFFu, minm1, off);
-    const uint32_t o2 = __shfl_xor_sync(0xFFFFFFFFu, minm2, off);
-    minm2 = min(max(minm1, o1), min(minm2, o2));
-    minm1 = min(minm1, o1);
-  }
-  // min |m'| exact as FP32: the lane owning the smallest candidate recomputes
-  // it; the runner-up is recomputed too when its FP32 key is within about
-  // 2^-7 relative of the smallest (a near-tie that the FP32 values, off by up
-  // to |beta1 m| / |m'| times their dequantisation error, may misorder)
-  // Every lane recomputes the element at the smallest key's index (only the
-  // owner lane's registers hold that element; the others compute a value that
-  // is discarded), so the common case runs converged; the owner's value is then
-  // broadcast to its 8-lane group.
-  const bool any_m = minm1 < 0xFFFFFF00u;
-  const bool tie = minm2 < 0xFFFFFF00u && (minm2 >> 8) - (minm1 >> 8) < (1u << 9);
-  float mum = recompute_m_double(in, static_cast<int>(minm1 & 15u), invk_md, h, gs, S.tabd_m,
-                                 S.exp2_16);
-  mum = __shfl_sync(0xFFFFFFFFu, mum, (slot << 3) | static_cast<int>((minm1 >> 5) & 7u));
-  if (__any_sync(0xFFFFFFFFu, tie)) {
-    float m2 = __int_as_float(0x7F800000);
-    if (tie && static_cast<int>((minm2 >> 5) & 7u) == l)
-      m2 = recompute_m_double(in, static_cast<int>(minm2 & 15u), invk_md, h, gs, S.tabd_m,
-                              S.exp2_16);
-#pragma unroll
-    for (int off = 1; off < 8; off <<= 1) m2 = fminf(m2, __shfl_xor_sync(0xFFFFFFFFu, m2, off));
-    mum = fminf(mum, m2);
-  }
-  if (!any_m) mum = 0.f;   // no nonzero element
-  const float muv = __uint_as_float(minv + 1u);
-  // lanes 0-3 of the group derive the m parameters, lanes 4-7 the v ones;
-  // then every lane takes k and 1/M of both moments from lanes 0 and 4
-  const bool vlane = l >= 4;
+  const bool vrole = l >= 4;   // lanes 4-7 of a group work on v, lanes 0-3 on m
   float kx, srx, invMx;
-  group_params_rt(vlane ? maxv : maxm, vlane ? muv : mum, true,
-                  vlane ? F8<FV>::LOG2MAX_HI : F8<FM>::LOG2MAX_HI,
-                  vlane ? F8<FV>::LOG2MAX_LO : F8<FM>::LOG2MAX_LO,
-                  vlane ? F8<FV>::LOG2_TARGET : F8<FM>::LOG2_TARGET, kx, srx, invMx);
+  if constexpr (EXACT) {
+    // Group extremes over the 8 lanes.  The keys take the lane in bits 5-7 (m)
+    // or 4-6 (v), so that each carries its element's position (ordering to
+    // 2^-16 relative); merging two sorted pairs keeps the two smallest.
+    const uint32_t lm = static_cast<uint32_t>(l) << 5, lv = static_cast<uint32_t>(l) << 4;
+    maxmk = (maxmk & ~0xE0u) | lm;
+    minm1 = (minm1 & ~0xE0u) | lm;
+    minm2 = (minm2 & ~0xE0u) | lm;
+    maxvk = (maxvk & ~0x70u) | lv;
+    minvk = (minvk & ~0x70u) | lv;
+  #pragma unroll
+    for (int off = 1; off < 8; off <<= 1) {
+      maxmk = max(maxmk, __shfl_xor_sync(0xFFFFFFFFu, maxmk, off));
+      maxvk = max(maxvk, __shfl_xor_sync(0xFFFFFFFFu, maxvk, off));
+      minvk = min(minvk, __shfl_xor_sync(0xFFFFFFFFu, minvk, off));
+      const uint32_t o1 = __shfl_xor_sync(0xFFFFFFFFu, minm1, off);
+      const uint32_t o2 = __shfl_xor_sync(0xFFFFFFFFu, minm2, off);
+      minm2 = min(max(minm1, o1), min(minm2, o2));
+      minm1 = min(minm1, o1);
+    }
+
+    // The group's k and root scale are computed in double from the extremes
+    // recomputed in double, as the definition has them, so that the FP32 k and
+    // s_r stored are the correctly rounded values of the exact ones (FP32 values
+    // of the extremes carry the dequantisation error, and the smallest |m'|
+    // usually comes from cancellation between beta1 m and (1 - beta1) g, which
+    // amplifies it by |beta1 m| / |m'|).  Each extreme is recomputed by one lane
+    // of the group, from the owner's codes and gradient in the scratch copy:
+    // lane 0 max |m'|, lanes 1 and 2 the two smallest |m'| (FP32 may misorder a
+    // near-tie), lane 4 max v', lane 5 the smallest v'; lanes 3, 6, 7 repeat a
+    // maximum.
+    const int role = l & 3;
+    const bool is_min = role == 1 || (!vrole && role == 2);
+    const uint32_t key = vrole ? (role == 1 ? minvk : maxvk)
+                               : (role == 1 ? minm1 : role == 2 ? minm2 : maxmk);
+    const bool found = is_min ? key < 0xFFFFFF00u : key >= 0x100u;
+    const int owner = static_cast<int>(vrole ? (key >> 4) & 7u : (key >> 5) & 7u);
+    const int idx = static_cast<int>(key & 15u);
+    const uint8_t* src = scratch_warp + (slot * 8 + owner) * 64;
+    const uint32_t code = src[(vrole ? 16 : 0) + idx];
+    const uint32_t gbits = *reinterpret_cast<const uint16_t*>(src + 32 + 2 * idx);
+    // val: |m'| or v' of the extreme in double; lval: its log2 (-inf for a zero
+    // maximum, +inf for a missing minimum)
+    double val, lval;
+    {
+      const double invkd = rcp_d(static_cast<double>(vrole ? in.vk : in.mk));
+      const double srd = static_cast<double>(vrole ? in.vs : in.ms);
+      const double beta = static_cast<double>(vrole ? h.beta2 : h.beta1);
+      const double* tabd = vrole ? S.tabd_v : S.tabd_m;
+      // x = sign(q) s_r |q|^(1/k) (zero for a zero code)
+      double x = (code & 0x7Fu) ? exp2_table(tabd[code] * invkd, S.exp2_16) * srd : 0.0;
+      if (!vrole && (code & 0x80u)) x = -x;
+      // m' = beta1 m + (1 - beta1) g, v' = beta2 v + ((1 - beta2) g) g, g the
+      // clipped gradient, each product and the sum rounded separately
+      const double gi = static_cast<double>(gs) * static_cast<double>(__uint_as_float(gbits << 16));
+      double term = __dmul_rn(1.0 - beta, gi);
+      if (vrole) term = __dmul_rn(term, gi);
+      const double r = fabs(__dadd_rn(__dmul_rn(beta, x), term));
+      const double inf = __longlong_as_double(0x7FF0000000000000LL);
+      val = found ? r : 0.0;
+      lval = found && r > 0.0 ? log2_table(r, S.lgt) : (is_min ? inf : -inf);
+    }
+    const int base = slot << 3;
+    const double M = __shfl_sync(0xFFFFFFFFu, val, base + (vrole ? 4 : 0));
+    const double lM = __shfl_sync(0xFFFFFFFFu, lval, base + (vrole ? 4 : 0));
+    const double lmu = fmin(__shfl_sync(0xFFFFFFFFu, lval, base + (vrole ? 5 : 1)),
+                            __shfl_sync(0xFFFFFFFFu, lval, base + (vrole ? 5 : 2)));
+    // lanes 0-3 derive the m parameters, lanes 4-7 the v ones:
+    // k = clamp(log2(R) / log2(M / mu), 1, 16) (16 when M == mu; 1, s_r = 1
+    // for an all-zero group), then s_r = M FMT_MAX^(-1/k) = 2^(log2 M -
+    // log2(FMT_MAX) / k) with the FP32 k.
+    const bool nonzero = M > 0.0;
+    const bool spread = nonzero && lmu < lM;
+    double kd = spread ? fmin(fmax((vrole ? F8<FV>::LOG2_TARGET_D : F8<FM>::LOG2_TARGET_D) *
+                                       rcp_d(lM - lmu), 1.0), 16.0)
+                       : 16.0;
+    if (!nonzero) kd = 1.0;
+    kx = __double2float_rn(kd);
+    const double ex = lM - (vrole ? F8<FV>::LOG2MAX_D : F8<FM>::LOG2MAX_D) *
+                               rcp_d(static_cast<double>(kx));
+    srx = nonzero ? __double2float_rn(exp2_table(ex, S.exp2_16)) : 1.0f;
+    invMx = nonzero ? rcp_approx(__double2float_rn(M)) : 0.0f;
+  } else {
+    minm1 = (minm1 & ~0xE0u) | (static_cast<uint32_t>(l) << 5);
+    minm2 = (minm2 & ~0xE0u) | (static_cast<uint32_t>(l) << 5);
+  #pragma unroll
+    for (int off = 1; off < 8; off <<= 1) {
+      maxm = fmaxf(maxm, __shfl_xor_sync(0xFFFFFFFFu, maxm, off));
+      maxv = fmaxf(maxv, __shfl_xor_sync(0xFFFFFFFFu, maxv, off));
+      minv = min(minv, __shfl_xor_sync(0xFFFFFFFFu, minv, off));
+      const uint32_t o1 = __shfl_xor_sync(0xFFFFFFFFu, minm1, off);
+      const uint32_t o2 = __shfl_xor_sync(0xFFFFFFFFu, minm2, off);
+      minm2 = min(max(minm1, o1), min(minm2, o2));
+      minm1 = min(minm1, o1);
+    }
+    const double kd0 = static_cast<double>(in.mk), r0 = static_cast<double>(rcp_approx(in.mk));
+    const double invk_md = r0 * fma(-kd0, r0, 2.0);
+    // min |m'| exact as FP32: the lane owning the smallest candidate recomputes
+    // it; the runner-up is recomputed too when its FP32 key is within about
+    // 2^-7 relative of the smallest (a near-tie that the FP32 values may
+    // misorder).  Every lane recomputes the element at the smallest key's index
+    // (only the owner's registers hold it; the others' values are discarded),
+    // so the common case runs converged.
+    const bool any_m = minm1 < 0xFFFFFF00u;
+    const bool tie = minm2 < 0xFFFFFF00u && (minm2 >> 8) - (minm1 >> 8) < (1u << 9);
+    float mum = recompute_m_double(in, static_cast<int>(minm1 & 15u), invk_md, h, gs, S.tabd_m,
+                                   S.exp2_16);
+    mum = __shfl_sync(0xFFFFFFFFu, mum, (slot << 3) | static_cast<int>((minm1 >> 5) & 7u));
+    if (__any_sync(0xFFFFFFFFu, tie)) {
+      float m2 = __int_as_float(0x7F800000);
+      if (tie && static_cast<int>((minm2 >> 5) & 7u) == l)
+        m2 = recompute_m_double(in, static_cast<int>(minm2 & 15u), invk_md, h, gs, S.tabd_m,
+                                S.exp2_16);
+  #pragma unroll
+      for (int off = 1; off < 8; off <<= 1) m2 = fminf(m2, __shfl_xor_sync(0xFFFFFFFFu, m2, off));
+      mum = fminf(mum, m2);
+    }
+    if (!any_m) mum = 0.f;
+    const float muv = __uint_as_float(minv + 1u);
+    // lanes 0-3 of the group derive the m parameters, lanes 4-7 the v ones
+    group_params_rt(vrole ? maxv : maxm, vrole ? muv : mum, true,
+                    vrole ? F8<FV>::LOG2MAX_HI : F8<FM>::LOG2MAX_HI,
+                    vrole ? F8<FV>::LOG2MAX_LO : F8<FM>::LOG2MAX_LO,
+                    vrole ? F8<FV>::LOG2_TARGET : F8<FM>::LOG2_TARGET, kx, srx, invMx);
+  }
   const int lane_m = slot << 3, lane_v = lane_m + 4;
   const float km = __shfl_sync(0xFFFFFFFFu, kx, lane_m);
   const float invMm = __shfl_sync(0xFFFFFFFFu, invMx, lane_m);
@@ -427,16 +611,16 @@ __device__ __forceinline__ void process(const LaneIn& in, const TileHeader& t, c
       cmw[i] = c.x;
       cvw[i] = c.y;
     }
-    if (FULL || active) {
-      *reinterpret_cast<uint32_t*>(t.mq + e) =
-          merge_signs4(pack4(cmw[0], cmw[1], cmw[2], cmw[3]), m1[4 * j], m1[4 * j + 1],
-                       m1[4 * j + 2], m1[4 * j + 3]);
-      *reinterpret_cast<uint32_t*>(t.vq + e) = pack4(cvw[0], cvw[1], cvw[2], cvw[3]);
+    if ((FULL || active) && COAT_INDEX_OK(e + 4 <= t.ngroups * kGroup)) {
+      __stcs(reinterpret_cast<unsigned int*>(t.mq + e),
+             merge_signs4(pack4(cmw[0], cmw[1], cmw[2], cmw[3]), m1[4 * j], m1[4 * j + 1],
+                          m1[4 * j + 2], m1[4 * j + 3]));
+      __stcs(reinterpret_cast<unsigned int*>(t.vq + e), pack4(cvw[0], cvw[1], cvw[2], cvw[3]));
     }
   }
-  if ((FULL || active) && (l & 3) == 0) {
-    (vlane ? t.vs : t.ms)[lg] = srx;
-    (vlane ? t.vk : t.mk)[lg] = kx;
+  if ((FULL || active) && (l & 3) == 0 && COAT_INDEX_OK(lg < t.ngroups)) {
+    (vrole ? t.vs : t.ms)[lg] = srx;
+    (vrole ? t.vk : t.mk)[lg] = kx;
   }
 }
 
@@ -451,23 +635,35 @@ __device__ __forceinline__ void feed_start(const Map& map, Feed& f, int64_t tile
   f.next_begin = map.begin_of(ti + 1);
 }
 
-// Stage `tile` into `st` (header into `hd`), completing on `bar`: a fully
-// valid tile is copied (kTxBytes of transaction), any other tile only arrives
-// and is read from global memory by the lanes.
+// Make f describe the tensor of `tile` (tiles only move forward).
 template <class Map>
-__device__ __forceinline__ void feed_issue(const Map& map, Feed& f, int64_t tile, uint8_t* st,
-                                           TileHeader& hd, uint64_t* bar, float lrwd) {
-  while (tile >= f.next_begin) {
-    const int32_t ti = ++f.ti;
+__device__ __forceinline__ void feed_locate(const Map& map, Feed& f, int64_t tile) {
+  if (tile >= f.next_begin) {
+    const int32_t ti = map.advance(f.ti, tile);
+    f.ti = ti;
     f.d = map.get(ti);
     f.next_begin = map.begin_of(ti + 1);
   }
+}
+
+// Stage `tile` (located in f) into `st` (header into `hd`), completing on
+// `bar`: a fully valid tile is copied (kTxBytes of transaction), any other tile
+// only arrives and is read from global memory by the lanes.
+__device__ __forceinline__ void feed_issue(const Feed& f, int64_t tile, uint8_t* st,
+                                           TileHeader& hd, uint64_t* bar, float lrwd,
+                                           uint64_t policy) {
   const TensorArgs& ct = f.d;
   const int64_t g0 = (tile - ct.tile_begin) * kTileGroups;
   const int64_t groups = (ct.n + kGroup - 1) / kGroup;
   const int64_t ng = (groups - g0) < kTileGroups ? (groups - g0) : int64_t(kTileGroups);
   const int64_t e0 = g0 * kGroup;
   const bool full = (e0 + kTileElems <= ct.n);
+  if (!COAT_INDEX_OK(tile >= ct.tile_begin && tile < ct.tile_begin + ct.tiles && e0 < ct.n)) {
+    hd.nvalid = 0;   // a tile outside its tensor: the lanes find no group and touch nothing
+    hd.ngroups = 0;
+    mbar_arrive(bar);
+    return;
+  }
   hd.master = ct.master + e0;
   hd.wout = ct.wout ? ct.wout + e0 : nullptr;
   hd.mq = ct.mq + e0;
@@ -482,20 +678,20 @@ __device__ __forceinline__ void feed_issue(const Map& map, Feed& f, int64_t tile
   hd.lrwd = lrwd * ct.wd_scale;
   if (full) {
     mbar_arrive_expect_tx(bar, kTxBytes);
-    bulk_g2s(st + kOffMaster, ct.master + e0, kTileElems * 4, bar);
-    bulk_g2s(st + kOffGrad, ct.grad + e0, kTileElems * 2, bar);
-    bulk_g2s(st + kOffMq, ct.mq + e0, kTileElems, bar);
-    bulk_g2s(st + kOffVq, ct.vq + e0, kTileElems, bar);
-    bulk_g2s(st + kOffMs, ct.ms + g0, kTileGroups * 4, bar);
-    bulk_g2s(st + kOffMk, ct.mk + g0, kTileGroups * 4, bar);
-    bulk_g2s(st + kOffVs, ct.vs + g0, kTileGroups * 4, bar);
-    bulk_g2s(st + kOffVk, ct.vk + g0, kTileGroups * 4, bar);
+    bulk_g2s_hint(st + kOffMaster, ct.master + e0, kTileElems * 4, bar, policy);
+    bulk_g2s_hint(st + kOffGrad, ct.grad + e0, kTileElems * 2, bar, policy);
+    bulk_g2s_hint(st + kOffMq, ct.mq + e0, kTileElems, bar, policy);
+    bulk_g2s_hint(st + kOffVq, ct.vq + e0, kTileElems, bar, policy);
+    bulk_g2s_hint(st + kOffMs, ct.ms + g0, kTileGroups * 4, bar, policy);
+    bulk_g2s_hint(st + kOffMk, ct.mk + g0, kTileGroups * 4, bar, policy);
+    bulk_g2s_hint(st + kOffVs, ct.vs + g0, kTileGroups * 4, bar, policy);
+    bulk_g2s_hint(st + kOffVk, ct.vk + g0, kTileGroups * 4, bar, policy);
   } else {
     mbar_arrive(bar);
   }
 }
 
-template <int FM, int FV, class Map>
+template <int FM, int FV, bool EXACT, class Map>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     adamw_fp8_kernel(const Map map, const StepHyper h, const ClipRecord* clip, unsigned* err) {
   // Gradient clipping: a record with found_inf set skips the step (nothing is
@@ -511,8 +707,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
   fill_log2_table<FM>(S.tab_m);
   fill_log2_table<FV>(S.tab_v);
-  for (int c = threadIdx.x; c < 256; c += blockDim.x)
+  for (int c = threadIdx.x; c < 256; c += blockDim.x) {
     S.tabd_m[c] = log2(static_cast<double>(fabsf(dec_value<FM>(c))));
+    if (EXACT) S.tabd_v[c] = log2(static_cast<double>(fabsf(dec_value<FV>(c))));
+  }
+  if (EXACT) {
+    for (int j = threadIdx.x; j < 128; j += blockDim.x) {
+      const double F = 1.0 + (static_cast<double>(j) + 0.5) * (1.0 / 128.0);
+      S.lgt[j].log2f = log2(F);
+      S.lgt[j].inv = 1.0 / F;
+    }
+  }
   if (threadIdx.x < 16) S.exp2_16[threadIdx.x] = exp2(static_cast<double>(threadIdx.x) / 16.0);
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -524,20 +729,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // this CTA's contiguous share of the tiles
+  // this CTA's tiles: blockIdx.x, blockIdx.x + gridDim.x, ... (at any moment the
+  // CTAs stream neighbouring regions of every array)
   const int64_t ntiles = map.tiles();
-  const int64_t t0 = int64_t(blockIdx.x) * ntiles / gridDim.x;
-  const int64_t t1 = int64_t(blockIdx.x + 1) * ntiles / gridDim.x;
+  const int64_t t0 = blockIdx.x, dt = gridDim.x;
 
   if (warp == kConsumerWarps) {
     // ---------------- producer ----------------
-    if (lane != 0 || t0 >= t1) return;
+    if (lane != 0 || t0 >= ntiles) return;
     Feed f;
     feed_start(map, f, t0);
+    const uint64_t policy = l2_evict_first_policy();
     int64_t it = 0;
-    for (int64_t tile = t0; tile < t1; ++tile, ++it) {
+    for (int64_t tile = t0; tile < ntiles; tile += dt, ++it) {
       const int s = static_cast<int>(it % kStages);
       const uint32_t use = static_cast<uint32_t>(it / kStages);
+      feed_locate(map, f, tile);   // before the wait: its loads overlap it
       if (use > 0 && !mbar_wait(&S.empty_bar[s], (use - 1) & 1u, kWaitBudgetCycles)) {
         atomicOr(err, kErrTimeoutProducer);
         // Drain copies still in flight into stages the consumers never freed.
@@ -551,7 +758,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         }
         return;
       }
-      feed_issue(map, f, tile, stages + size_t(s) * kStageBytes, S.hdr[s], &S.full_bar[s], h.lrwd);
+      feed_issue(f, tile, stages + size_t(s) * kStageBytes, S.hdr[s], &S.full_bar[s], h.lrwd,
+                 policy);
     }
     return;
   }
@@ -559,6 +767,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   // ---------------- consumers ----------------
   const int slot = lane >> 3, l = lane & 7;
   const int lg = warp * kGroupsPerWarp + slot;  // group within the tile
+  uint4* scratch_lane = S.scratch + (warp * 32 + lane) * 4;
+  const uint8_t* scratch_warp = reinterpret_cast<const uint8_t*>(S.scratch + warp * 32 * 4);
   const float omb1 = h.omb1 * gs, omb2 = h.omb2 * gs * gs;
   // the lane's elements: 4 chunks of 4, chunk j at 32 chunk_of(j, slot) + 4 l
   // within its group
@@ -566,7 +776,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #pragma unroll
   for (int j = 0; j < 4; ++j) off[j] = lg * kGroup + 32 * chunk_of(j, slot) + 4 * l;
   int64_t it = 0;
-  for (int64_t tile = t0; tile < t1; ++tile, ++it) {
+  for (int64_t tile = t0; tile < ntiles; tile += dt, ++it) {
     const int s = static_cast<int>(it % kStages);
     const uint32_t use = static_cast<uint32_t>(it / kStages);
     if (!__all_sync(0xFFFFFFFFu, mbar_wait(&S.full_bar[s], use & 1u, kWaitBudgetCycles))) {
@@ -585,20 +795,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.empty_bar[s]);
     if (full)
-      process<FM, FV, true>(in, t, off, lg, true, slot, l, h, omb1, omb2, gs, S);
+      process<FM, FV, EXACT, true>(in, t, off, lg, true, slot, l, h, omb1, omb2, gs, S, scratch_lane,
+                            scratch_warp);
     else
-      process<FM, FV, false>(in, t, off, lg, active, slot, l, h, omb1, omb2, gs, S);
+      process<FM, FV, EXACT, false>(in, t, off, lg, active, slot, l, h, omb1, omb2, gs, S, scratch_lane,
+                             scratch_warp);
   }
 }
 
-template <int FM, int FV, class Map>
+template <int FM, int FV, bool EXACT, class Map>
 cudaError_t launch_step(const Map& map, int64_t ntiles, const StepHyper& h,
                         const ClipRecord* clip, unsigned* err, cudaStream_t stream) {
   static bool configured[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  auto kern = adamw_fp8_kernel<FM, FV, Map>;
+  auto kern = adamw_fp8_kernel<FM, FV, EXACT, Map>;
   if (dev < 64 && !configured[dev]) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemBytes));
@@ -616,8 +828,10 @@ template <class Map>
 cudaError_t dispatch(int fm, int fv, const Map& map, int64_t ntiles, const StepHyper& h,
                      const ClipRecord* clip, unsigned* err, cudaStream_t stream) {
   switch (fm * 3 + fv) {
-#define COAT_STEP_CASE(A, B) \
-  case A * 3 + B: return launch_step<A, B>(map, ntiles, h, clip, err, stream);
+#define COAT_STEP_CASE(A, B)                                                  \
+  case A * 3 + B:                                                             \
+    return h.exact ? launch_step<A, B, true>(map, ntiles, h, clip, err, stream) \
+                   : launch_step<A, B, false>(map, ntiles, h, clip, err, stream);
     COAT_STEP_CASE(kE4M3, kE4M3)
     COAT_STEP_CASE(kE4M3, kE5M2)
     COAT_STEP_CASE(kE4M3, kE5M2Full)
@@ -635,6 +849,8 @@ cudaError_t dispatch(int fm, int fv, const Map& map, int64_t ntiles, const StepH
 }  // namespace
 
 int64_t step_tile_groups() { return kTileGroups; }
+
+COAT_INDEX_FAULT_READER(index_faults_step)
 
 cudaError_t launch_adamw_single(const TensorArgs& t, int fm, int fv, const StepHyper& h,
                                 unsigned* err, cudaStream_t stream) {
@@ -753,7 +969,7 @@ __global__ void __launch_bounds__(kNormThreads, kNormCtasPerSm)
         const int64_t ea = (tile - tb) * kTileElems;
         const int64_t eb_tiles = (tend - tb) * kTileElems;
         const int64_t eb = eb_tiles < d.n ? eb_tiles : d.n;
-        acc += sumsq_run(d.grad + ea, eb - ea);
+        if (COAT_INDEX_OK(ea >= 0 && ea <= eb && eb <= d.n)) acc += sumsq_run(d.grad + ea, eb - ea);
         tile = tend;
       }
       ++ti;

@@ -2,6 +2,7 @@
 // any CUDA call, so a bad call launches nothing and touches nothing), error
 // reporting, multi-tensor plans, and kernel launches on the caller's stream.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstddef>
 #include <limits>
@@ -103,6 +104,9 @@ coat_status check_hyper(float lr, float beta1, float beta2, float eps, float wd,
   return COAT_OK;
 }
 
+// The group-parameter mode of the step entry points (coat_set_exact_group_params).
+std::atomic<int> g_exact_group_params{0};
+
 coat::StepHyper make_hyper(float lr, float beta1, float beta2, float eps, float wd, int64_t step) {
   const double b1 = beta1, b2 = beta2;
   const double bc1 = 1.0 - std::pow(b1, static_cast<double>(step));
@@ -125,6 +129,7 @@ coat::StepHyper make_hyper(float lr, float beta1, float beta2, float eps, float 
     h.deps = deps;
   }
   h.lrwd = static_cast<float>(dlr * static_cast<double>(wd));
+  h.exact = g_exact_group_params.load(std::memory_order_relaxed);
   return h;
 }
 
@@ -673,12 +678,34 @@ coat_status coat_check_device_error(cudaStream_t stream) {
   unsigned v = 0;
   e = cudaMemcpyFromSymbol(&v, g_coat_device_error, sizeof(v));
   if (e != cudaSuccess) return cuda_fail(e, "coat_check_device_error");
+  // failed index checks of the checked build (each read clears its count)
+  unsigned fs = 0, fc = 0, ff = 0;
+  if (e == cudaSuccess) e = coat::index_faults_step(&fs);
+  if (e == cudaSuccess) e = coat::index_faults_codec(&fc);
+  if (e == cudaSuccess) e = coat::index_faults_flow(&ff);
+  if (e != cudaSuccess) return cuda_fail(e, "coat_check_device_error");
   if (v != 0) {
     const unsigned zero = 0;
     cudaMemcpyToSymbol(g_coat_device_error, &zero, sizeof(zero));
     return fail(COAT_ERR_TIMEOUT, "a kernel gave up a bounded wait (device error bits 0x%x)", v);
   }
+  if (fs + fc + ff != 0)
+    return fail(COAT_ERR_DEVICE_CHECK,
+                "checked build: %u device index checks failed (step %u, codec %u, layers %u)",
+                fs + fc + ff, fs, fc, ff);
   return COAT_OK;
+}
+
+int coat_set_exact_group_params(int on) {
+  return g_exact_group_params.exchange(on ? 1 : 0);
+}
+
+int coat_build_checked(void) {
+#ifdef COAT_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
 }
 
 }  // extern "C"

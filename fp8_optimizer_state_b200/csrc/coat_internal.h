@@ -32,6 +32,7 @@ struct StepHyper {
   float dsq;        // (1 - beta1^t) / (lr sqrt(1 - beta2^t)); 0 when lr = 0
   float deps;       // eps (1 - beta1^t) / lr; +inf when lr = 0
   float lrwd;       // lr * wd
+  int32_t exact;    // 1: exact group parameters (coat_set_exact_group_params)
 };
 
 // Result of the gradient-norm pass over a plan's gradients; the same layout as
@@ -44,6 +45,12 @@ struct ClipRecord {
   int32_t reserved;
 };
 static_assert(sizeof(ClipRecord) == 24, "ClipRecord layout");
+
+// Failed index checks counted by each kernel file since the last read (the
+// checked build; always 0 in the release build); each call clears its count.
+cudaError_t index_faults_step(unsigned* count);
+cudaError_t index_faults_codec(unsigned* count);
+cudaError_t index_faults_flow(unsigned* count);
 
 int sm_count(int dev);
 // Grid of at most sm_count(dev) * max_blocks_per_sm CTAs for work_items items

@@ -148,7 +148,7 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
   auto load = [&](RowItem<DT>& it) {
     it.r = cr;
     it.c = cc;
-    it.valid = clamp_valid(cols - cc, 16);
+    it.valid = COAT_INDEX_OK(cr < rows) ? clamp_valid(cols - cc, 16) : 0;
     load16<DT>(static_cast<const char*>(x) + cr * ldx * esz, cc, it.valid, it.raw);
     cc += 4 * kGroup;
     if (cc >= rowspan) { cc -= rowspan; ++cr; }
@@ -205,12 +205,15 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
       encode_words<FMT, 16, true>(v, use_div, d, invM, k, cw);
     else
       encode_words<FMT, 16, false>(v, use_div, d, invM, k, cw);
-    if (cur.valid > 0) store16(q + cur.r * ldq + cur.c, cw, cur.valid);
+    if (cur.valid > 0 && COAT_INDEX_OK(cur.r < rows && cur.c + cur.valid <= cols))
+      store16(q + cur.r * ldq + cur.c, cw, cur.valid);
     // lane 0 of a group holds its first column, so it exists exactly when the group does
     if (l == 0 && cur.valid > 0) {
       const int64_t g = cur.r * nbc + (cur.c >> 7);
-      scale[g] = sr;
-      kk[g] = k;
+      if (COAT_INDEX_OK(g < rows * nbc)) {
+        scale[g] = sr;
+        kk[g] = k;
+      }
     }
     cur = nxt;
   }
@@ -407,7 +410,7 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
         encode_words<FMT, 8, true>(v, use_div, d, invM, k, cw);
       else
         encode_words<FMT, 8, false>(v, use_div, d, invM, k, cw);
-      const int valid = r < rows ? cv : 0;
+      const int valid = r < rows && COAT_INDEX_OK(cv == 0 || c + cv <= cols) ? cv : 0;
       uint8_t* qp = q + r * ldq + c;
       if (valid >= 8) {
         *reinterpret_cast<uint2*>(qp) = make_uint2(cw[0], cw[1]);
@@ -417,7 +420,7 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
           if (e < valid) qp[e] = static_cast<uint8_t>(cw[e >> 2] >> (8 * (e & 3)));
       }
     }
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && COAT_INDEX_OK(b < nb)) {
       scale[b] = sr;
       kk[b] = k;
     }
@@ -531,7 +534,7 @@ __global__ void __launch_bounds__(256) dequant_full_kernel(const uint8_t* __rest
     bool ok[kBatch];
 #pragma unroll
     for (int j = 0; j < kBatch; ++j) {
-      ok[j] = r < rows;
+      ok[j] = r < rows && COAT_INDEX_OK(16 * cc + 16 <= cols);
       if (ok[j]) {
         w[j] = __ldg(reinterpret_cast<const uint4*>(qp));
         const int64_t g = (GR == 1 ? r : r / GR) * nbc + (cc >> 3);
@@ -577,7 +580,7 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
   int64_t r = t0 / cpr, cc = t0 % cpr;
   auto fetch = [&](int64_t rr, int64_t ch, uint4& w, float& s, float& kv, int& valid) {
     const int64_t c0 = ch * 16;
-    valid = clamp_valid(cols - c0, 16);
+    valid = COAT_INDEX_OK(rr < rows && c0 < cols) ? clamp_valid(cols - c0, 16) : 0;
     const uint8_t* qp = q + rr * ldq + c0;
     if (valid >= 16) {
       w = __ldg(reinterpret_cast<const uint4*>(qp));
@@ -589,8 +592,8 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
       w = make_uint4(t[0], t[1], t[2], t[3]);
     }
     const int64_t g = (GR == 1 ? rr : rr / GR) * nbc + (ch >> 3);
-    s = __ldg(scale + g);
-    kv = __ldg(kk + g);
+    s = valid > 0 ? __ldg(scale + g) : 0.f;
+    kv = valid > 0 ? __ldg(kk + g) : 1.f;
   };
   uint4 w;
   float s, kv;
@@ -645,6 +648,8 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
 }
 
 }  // namespace
+
+COAT_INDEX_FAULT_READER(index_faults_codec)
 
 unsigned grid_for(int64_t work_items, int per_block, int dev, int max_blocks_per_sm) {
   int64_t b = (work_items + per_block - 1) / per_block;

@@ -64,6 +64,37 @@ __device__ __forceinline__ void decode16(const uint4& w, float s, float k, const
   }
 }
 
+// FP8 codes of 16 signed values y with |y| <= FMT_MAX (1 + 2^-16), four per
+// word, by the hardware conversion (cvt.rn.satfinite, two values per
+// instruction: round to nearest even, saturating to +-FMT_MAX).  On that range
+// it gives the software encoder's codes (tests compare the two on every FP32
+// value up to FMT_MAX (1 + 2^-16)), except that it keeps the sign of a value
+// that rounds to zero: such codes are set back to 0x00, the library's only
+// zero code.
+template <int FMT>
+__device__ __forceinline__ void encode_hw16(const float (&y)[16], uint32_t (&cw)[4]) {
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    uint16_t lo, hi;
+    if (FMT == kE4M3) {
+      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(y[4 * w + 1]), "f"(y[4 * w]));
+      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(y[4 * w + 3]), "f"(y[4 * w + 2]));
+    } else {
+      asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(y[4 * w + 1]), "f"(y[4 * w]));
+      asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(y[4 * w + 3]), "f"(y[4 * w + 2]));
+    }
+    const uint32_t v = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+    const uint32_t mags = v & 0x7F7F7F7Fu;
+    // (mag + 0x7F) has bit 7 set iff mag != 0; adding to four bytes <= 0x7F never carries
+    cw[w] = mags | (v & (mags + 0x7F7F7F7Fu) & 0x80808080u);
+  }
+}
+
+// y with the sign of s (y >= 0).
+__device__ __forceinline__ float with_sign_of(float y, float s) {
+  return __uint_as_float(__float_as_uint(y) | (__float_as_uint(s) & 0x80000000u));
+}
+
 // max(a, b) that returns NaN when either is NaN.
 __device__ __forceinline__ float fmax_nan(float a, float b) {
   float r;
@@ -148,19 +179,16 @@ __device__ __forceinline__ void quantize_lane16(const float (&h)[16], bool force
       sr = M > 0.0f ? __fdiv_rn(M, F8<FMT>::MAXV) : 1.0f;   // M / FMT_MAX, correctly rounded
       invM = M > 0.0f ? rcp_approx(M) : 0.0f;   // an all-zero group encodes to zeros
     }
-    uint32_t mag[16];
+    float y[16];
     if (k == 1.0f) {
       const float c = F8<FMT>::MAXV * invM;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) mag[i] = enc_mag_bounded<FMT>(fabsf(h[i]) * c);
+      for (int i = 0; i < 16; ++i) y[i] = h[i] * c;
     } else {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) mag[i] = enc_mag_bounded<FMT>(expand_value<FMT>(h[i], invM, k));
+      for (int i = 0; i < 16; ++i) y[i] = with_sign_of(expand_value<FMT>(h[i], invM, k), h[i]);
     }
-#pragma unroll
-    for (int w = 0; w < 4; ++w)
-      cw[w] = merge_signs4(pack4(mag[4 * w], mag[4 * w + 1], mag[4 * w + 2], mag[4 * w + 3]),
-                           h[4 * w], h[4 * w + 1], h[4 * w + 2], h[4 * w + 3]);
+    encode_hw16<FMT>(y, cw);
   } else {
     // the codec's slow path: the maximum ignores NaN, IEEE division for k = 1
     float Mn = max_abs_nonnan(h);
@@ -221,19 +249,17 @@ __device__ __forceinline__ void quantize_scaled16(const float (&p)[16], float C,
   }
   k = 1.0f;
   sr = My > 0.0f ? __fdiv_rn(My, F8<FMT>::MAXV) : 1.0f;
+  float y[16];
   if (EXACT) {
     const GroupDiv dv = codec_div<FMT>(mp);
-    encode_words<FMT, 16, true>(p, true, dv, 0.0f, 1.0f, cw);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) y[i] = with_sign_of(div_exact(p[i], dv), p[i]);
   } else {
     const float c = mp > 0.0f ? F8<FMT>::MAXV * rcp_approx(mp) : 0.0f;
-    uint32_t mag[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) mag[i] = enc_mag_bounded<FMT>(fabsf(p[i]) * c);
-#pragma unroll
-    for (int w = 0; w < 4; ++w)
-      cw[w] = merge_signs4(pack4(mag[4 * w], mag[4 * w + 1], mag[4 * w + 2], mag[4 * w + 3]),
-                           p[4 * w], p[4 * w + 1], p[4 * w + 2], p[4 * w + 3]);
+    for (int i = 0; i < 16; ++i) y[i] = p[i] * c;
   }
+  encode_hw16<FMT>(y, cw);
 }
 
 // One lane's forward work item: 16 gate and 16 up codes, their groups'
@@ -276,7 +302,7 @@ __global__ void __launch_bounds__(256) swiglu_fwd_kernel(const ActArgs gate, con
   auto load = [&](FwdItem& it) {
     it.r = cr;
     it.c = cc;
-    it.valid = cc < cols;
+    it.valid = cc < cols && COAT_INDEX_OK(cr < rows && cc + 16 <= cols);
     const int32_t g = cc >> 7;
     if (it.valid) {
       it.gw = __ldg(reinterpret_cast<const uint4*>(gate.q + cr * gate.ldq + cc));
@@ -348,6 +374,10 @@ __global__ void __launch_bounds__(256) swiglu_bwd_kernel(const uint16_t* __restr
   int64_t r = t0 / cpr, cc = t0 % cpr;
   auto fetch = [&](int64_t rr, int64_t ch, BwdItem& it) {
     const int64_t c = ch * 16, g = ch >> 3;
+    if (!COAT_INDEX_OK(rr < rows && c + 16 <= cols)) {
+      it = BwdItem{};
+      return;
+    }
     const uint4* dp = reinterpret_cast<const uint4*>(dh + rr * lddh + c);
     it.d0 = __ldcs(dp);
     it.d1 = __ldcs(dp + 1);
@@ -388,12 +418,14 @@ __global__ void __launch_bounds__(256) swiglu_bwd_kernel(const uint16_t* __restr
       ou[j] = pack_bf16x2(b[0], b[1]);
     }
     const int64_t c = cc * 16;
-    uint4* gp = reinterpret_cast<uint4*>(dg + r * lddg + c);
-    uint4* up_ = reinterpret_cast<uint4*>(du + r * lddu + c);
-    gp[0] = make_uint4(og[0], og[1], og[2], og[3]);
-    gp[1] = make_uint4(og[4], og[5], og[6], og[7]);
-    up_[0] = make_uint4(ou[0], ou[1], ou[2], ou[3]);
-    up_[1] = make_uint4(ou[4], ou[5], ou[6], ou[7]);
+    if (COAT_INDEX_OK(c + 16 <= cols)) {
+      uint4* gp = reinterpret_cast<uint4*>(dg + r * lddg + c);
+      uint4* up_ = reinterpret_cast<uint4*>(du + r * lddu + c);
+      gp[0] = make_uint4(og[0], og[1], og[2], og[3]);
+      gp[1] = make_uint4(og[4], og[5], og[6], og[7]);
+      up_[0] = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+      up_[1] = make_uint4(ou[4], ou[5], ou[6], ou[7]);
+    }
     r = rn;
     cc = cn;
     cur = nxt;
@@ -513,8 +545,8 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_fwd_kernel(const ActArgs
       uint32_t cw[4];
       float k, sr;
       quantize_scaled16<FMT, EXPAND, true>(pv[j], sv[j] * rstd, cw, k, sr);
-      if (ok[j]) {
-        const int64_t c = (threadIdx.x + int64_t(j) * kNormThreads) * 16;
+      const int64_t c = (threadIdx.x + int64_t(j) * kNormThreads) * 16;
+      if (ok[j] && COAT_INDEX_OK(c + 16 <= d)) {
         *reinterpret_cast<uint4*>(out.q + r * out.ldq + c) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
         if ((threadIdx.x & 7) == 0) {
           out.scale[r * out.lds + (c >> 7)] = sr;
@@ -620,8 +652,8 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_bwd_kernel(
         }
         o[e] = pack_bf16x2(a[0], a[1]);
       }
-      if (ok[j]) {
-        const int64_t c = (threadIdx.x + int64_t(j) * kNormThreads) * 16;
+      const int64_t c = (threadIdx.x + int64_t(j) * kNormThreads) * 16;
+      if (ok[j] && COAT_INDEX_OK(c + 16 <= d)) {
         uint4* op = reinterpret_cast<uint4*>(dx + r * lddx + c);
         op[0] = make_uint4(o[0], o[1], o[2], o[3]);
         op[1] = make_uint4(o[4], o[5], o[6], o[7]);
@@ -632,8 +664,8 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_bwd_kernel(
   }
 #pragma unroll
   for (int j = 0; j < CPT; ++j) {
-    if (!ok[j]) continue;
     const int64_t c = (threadIdx.x + int64_t(j) * kNormThreads) * 16;
+    if (!ok[j] || !COAT_INDEX_OK(c + 16 <= d)) continue;
     float4* pp = reinterpret_cast<float4*>(partial + blockIdx.x * d + c);
 #pragma unroll
     for (int v = 0; v < 4; ++v)
@@ -726,6 +758,8 @@ cudaError_t rms_bwd_launch(const uint16_t* dy, int64_t lddy, const ActArgs& x, c
 }
 
 }  // namespace
+
+COAT_INDEX_FAULT_READER(index_faults_flow)
 
 size_t rmsnorm_workspace_bytes(int dev, int64_t d) {
   return sizeof(float) * size_t(sm_count(dev)) * kNormMaxCtasPerSm * size_t(d);

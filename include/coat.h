@@ -66,7 +66,9 @@ typedef enum {
     COAT_ERR_UNSUPPORTED = 3, /* a valid request this library does not implement (e.g. group != 128) */
     COAT_ERR_CUDA = 4,        /* the CUDA runtime reported an error at launch or copy */
     COAT_ERR_TIMEOUT = 5,     /* a kernel gave up a bounded wait; results are invalid */
-    COAT_ERR_NOMEM = 6        /* host or device allocation failed (plan creation only) */
+    COAT_ERR_NOMEM = 6,       /* host or device allocation failed (plan creation only) */
+    COAT_ERR_DEVICE_CHECK = 7 /* checked build only: a kernel's index check failed and the
+                                 access was skipped; results are invalid */
 } coat_status;
 
 /* Thread-local description of the last non-OK status returned on this thread. */
@@ -146,6 +148,30 @@ coat_status coat_adamw_step(float *master, uint16_t *weight_bf16_out, const uint
                             float *v_scale, float *v_k, int64_t n, int group, float lr,
                             float beta1, float beta2, float eps, float wd, int64_t step,
                             coat_fmt fmt_m, coat_fmt fmt_v, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Group-parameter mode of every AdamW step entry point (coat_adamw_step, the
+ * multi-tensor, clipped and no-allocation steps), process-wide; returns the
+ * previous mode.  The COAT pages give no precision for k and the scale; the
+ * definition computes them from the new moments' group maximum and nonzero
+ * minimum.
+ *
+ * on = 0 (the default): each group's extremes are the FP32 values of m' and
+ *   v' (the smallest |m'| recomputed in double, since it usually comes from
+ *   cancellation between beta1 m and (1 - beta1) g), and k and the root scale
+ *   are derived from them with FP32 approximations: within about 3e-7 (k) and
+ *   5e-6 (scale) of the exact values.
+ * on = 1: each group's extremes (max |m'|, the two smallest nonzero |m'|, max
+ *   v', the smallest nonzero v') are recomputed in double from the stored codes
+ *   and the gradient, and k and the root scale are computed in double and
+ *   rounded to FP32 once: the correctly rounded values of the definition
+ *   (except when an FP32 near-tie hides the true extreme).  Two runs that
+ *   start from the same state then keep bit-identical k, scales and codes
+ *   apart from rare code-rounding differences, so they stay in lockstep.  The
+ *   step is about 15% slower (a serial double-precision phase per group).
+ * Codes come from the same FP32 expansion and software encoder in both modes.
+ * ------------------------------------------------------------------------- */
+int coat_set_exact_group_params(int on);
 
 /* ---------------------------------------------------------------------------
  * Multi-tensor launcher over a ragged list of parameter tensors: one kernel
@@ -429,8 +455,20 @@ coat_status coat_zero1_layout(const int64_t *sizes, int num_tensors, int group, 
  * coat_check_device_error synchronises `stream`, reads and clears the flag,
  * and returns COAT_ERR_TIMEOUT if it was set (COAT_OK otherwise, or
  * COAT_ERR_CUDA if the synchronisation itself failed).
+ *
+ * Checked build (libcoat_debug.so, compiled with COAT_DEBUG; the library's
+ * stand-in for a memory checker): before each load or store whose index it
+ * derives, a kernel checks the index against the extents it was given (tile
+ * within its tensor, element below n, group below the group count, row and
+ * column within the shape); a failed check is counted on the device and the
+ * access is skipped, never trapped.  coat_check_device_error then also reads
+ * and clears the counts and returns COAT_ERR_DEVICE_CHECK if any check
+ * failed.  The release build (libcoat.so) compiles the checks away.
  * ------------------------------------------------------------------------- */
 coat_status coat_check_device_error(cudaStream_t stream);
+
+/* 1 in the checked build (libcoat_debug.so), 0 in the release build. */
+int coat_build_checked(void);
 
 /* Self-test of the bounded waits (the COAT pages have no counterpart; this
  * exists to test the failure path without a GPU fault).  Enqueues on `stream`

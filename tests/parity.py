@@ -19,15 +19,14 @@ Comparison modes:
   * identical inputs: both sides start a step from the same generated state
     (codes, k, s_r from the seeded generator) -- every tolerance applies to
     every element and group;
-  * free-running: each side quantises the FP32 warm start with its own codec
-    and then runs its own trajectory.  A group whose stored state (codes, k or
-    s_r) differs in any bit no longer has the same inputs at the next step;
-    its k, s_r and codes are then not compared (a difference of one FP32 ulp
-    in k is amplified by the cancellation in min|m'| into a k difference far
-    above 1e-5).  Once its codes differ, or its k or s_r differ by more than
-    2e-6 relative, its dequantised moments differ by more than the master
-    tolerance can absorb and its master leaves the comparison too.  Counts are
-    reported.
+  * free-running: both sides start from the same state and each then runs its
+    own trajectory.  Groups whose stored state is still bit-identical to the
+    oracle's get every identical-input check at the next step, their master
+    included (asserted).  A group that differs in any bit leaves that
+    comparison for good: its next step no longer has the oracle's inputs.  The
+    groups that stay within the per-step tolerances (codes identical, k within
+    1e-5, s_r within its tolerance) are counted too, and every element's master
+    deviation is recorded, unmasked, for the caller to bound.
 """
 from __future__ import annotations
 
@@ -105,6 +104,20 @@ def check_master(tag, gm, om, upd_abs_sum, mask=None):
         tag, int(bad.sum()), float(np.max(np.abs(gm - om) - tol)))
 
 
+def literal_master_fail(gm, om, t):
+    """Elements outside the literal master tolerance 1e-6 |p_oracle| + 1e-10 t
+    (the floor keeps p = 0 from needing an exact zero)."""
+    gm = np.asarray(gm, dtype=np.float64)
+    om = np.asarray(om, dtype=np.float64)
+    return np.abs(gm - om) > MASTER_RTOL * np.abs(om) + 1e-10 * t
+
+
+def literal_scale_fail(gs, os_):
+    """Groups whose root scale is outside the literal 1e-5 relative tolerance
+    (the bound the checks above widen by k's reach through the exponent)."""
+    return rel_err(gs, os_) > K_RTOL
+
+
 class FreeRun:
     """Bookkeeping of a free-running comparison (see the module docstring)."""
 
@@ -113,35 +126,63 @@ class FreeRun:
         self.group = group
         self.ng = -(-n // group)
         self.same = np.ones(self.ng, dtype=bool)      # stored state bit-identical so far
-        self.flipped = np.zeros(self.ng, dtype=bool)  # codes ever differed
+        self.live = np.ones(self.ng, dtype=bool)      # within the tolerances so far
         self.upd_sum = np.zeros(n, dtype=np.float64)
         self.report = []
+        self.master_dev = []                          # per step: all-element deviations
 
     def element_mask(self):
-        return np.repeat(~self.flipped, self.group)[: self.n]
+        return np.repeat(self.live, self.group)[: self.n]
 
     def check_state(self, tag, fmt, gq, gs, gk, oq, os_, ok_):
-        """Compare one moment's state on the groups that entered this step with
-        identical inputs; returns the groups whose stored state now differs."""
-        sel = self.same.copy()
-        nd, diff = check_state_all(tag, self.n, fmt, gq, gs, gk, oq, os_, ok_, groups=sel,
-                                   group=self.group)
+        """Compare one moment's new state.  Groups that entered the step with
+        bit-identical state get the identical-input checks (asserted); every
+        live group is tested against the tolerances.  Returns (groups leaving
+        the comparison, groups whose state now differs in any bit)."""
+        nd, _ = check_state_all(tag, self.n, fmt, gq, gs, gk, oq, os_, ok_, groups=self.same,
+                                group=self.group)
         ng = self.ng
         gq2 = np.asarray(gq)[: ng * self.group].reshape(ng, self.group)
         oq2 = np.asarray(oq)[: ng * self.group].reshape(ng, self.group)
+        gk_, ok2 = np.asarray(gk)[:ng], np.asarray(ok_)[:ng]
+        gs_, os2 = np.asarray(gs)[:ng], np.asarray(os_)[:ng]
         code_diff = (gq2 != oq2).any(axis=1)
-        meta_diff = (np.asarray(gk)[:ng] != np.asarray(ok_)[:ng]) | \
-                    (np.asarray(gs)[:ng] != np.asarray(os_)[:ng])
-        big = code_diff | (rel_err(np.asarray(gk)[:ng], np.asarray(ok_)[:ng]) > 2e-6) | \
-            (rel_err(np.asarray(gs)[:ng], np.asarray(os_)[:ng]) > 2e-6)
-        self.report.append((tag, nd, int(sel.sum()), int(code_diff.sum()), int(meta_diff.sum()),
-                            int(big.sum())))
-        return big, code_diff | meta_diff
+        code_far = np.abs(code_ordinal(gq2) - code_ordinal(oq2)).max(axis=1) > 1
+        differ = code_diff | (gk_ != ok2) | (gs_ != os2)
+        leave = code_diff | (rel_err(gk_, ok2) > K_RTOL) | (rel_err(gs_, os2) > scale_rtol(ok2, fmt))
+        live = self.live
+        self.report.append(dict(tag=tag, live=int(live.sum()), same=int(self.same.sum()),
+                                flips_same=int(nd), code_groups=int((code_diff & live).sum()),
+                                code_far=int((code_far & live).sum()),
+                                k_bits_differ=int(((gk_ != ok2) & live).sum()),
+                                s_bits_differ=int(((gs_ != os2) & live).sum()),
+                                s_literal_fail=int((literal_scale_fail(gs_, os2) & live).sum()),
+                                leave=int((leave & live).sum())))
+        return leave, differ
 
-    def check_master(self, tag, gm, om, upd_abs):
+    def check_master(self, tag, gm, om, upd_abs, t):
+        """Master of every element whose group entered the step with the
+        oracle's state bit for bit: within the tolerance (asserted).  For all
+        elements the deviation |dp| / (|p| + sum u^abs) is recorded (groups
+        that entered with a state differing from the oracle's no longer share
+        its inputs, so no per-step tolerance applies to them) and returned."""
         self.upd_sum += upd_abs
-        check_master(tag, gm, om, self.upd_sum, mask=self.element_mask())
+        same = np.repeat(self.same, self.group)[: self.n]
+        check_master(tag, gm, om, self.upd_sum, mask=same)
+        gm64 = np.asarray(gm, dtype=np.float64)
+        om64 = np.asarray(om, dtype=np.float64)
+        dev = np.abs(gm64 - om64) / (np.abs(om64) + self.upd_sum)
+        lit = literal_master_fail(gm, om, t)
+        live = self.element_mask()
+        self.master_dev.append(dict(step=t, same_elements=int(same.sum()),
+                                    live_elements=int(live.sum()),
+                                    literal_fail_same=int((lit & same).sum()),
+                                    literal_fail_all=int(lit.sum()),
+                                    q50=float(np.quantile(dev, 0.5)),
+                                    q99=float(np.quantile(dev, 0.99)),
+                                    q999=float(np.quantile(dev, 0.999)), max=float(dev.max())))
+        return dev
 
-    def after_step(self, diverged, state_diff):
-        self.flipped |= diverged
-        self.same &= ~state_diff
+    def after_step(self, leave, differ):
+        self.live &= ~leave
+        self.same &= ~differ
