@@ -13,8 +13,9 @@ Multi-GPU (torchrun): every rank updates its own full parameter list (the
 parameter groups are independent; there is no exchange step), so per-GPU work
 is fixed ("weak" scaling); time = max over ranks of device time.
 
---impl reference times the CPU oracle (plain double-precision C, one host
-thread) on a bounded sample of the same workload per step.
+--impl reference times the CPU oracle (plain double-precision C) on every host
+core, over a bounded sample of the workload's token embedding and first layer
+per step.
 """
 from __future__ import annotations
 
@@ -153,52 +154,108 @@ class ClockSampler:
 # ----------------------------------------------------------------------------
 # CPU oracle timing (the reference arm and the cpu_baseline key)
 # ----------------------------------------------------------------------------
-def oracle_sample_inputs(cfg, count, use_device):
-    """Inputs of the first `count` elements of the workload's first tensor (bits
-    from the seeded generator; on the device when one is in use, which is
-    bit-identical and much faster than the NumPy generator)."""
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# The oracle is timed on a bounded sample of the Llama-2-7B list's token
+# embedding and first layer (10 tensors; the step's cost per element does not
+# depend on the tensor), extrapolated to the whole list.
+SLICE_TENSORS = 10
+SLICE_NAME = "token embedding + layer 0 of the Llama-2-7B list"
+LLAMA2_7B_PARAMS = 6738415616
+
+
+def oracle_slice_inputs(per_tensor, fmt_m, fmt_v, use_device):
+    """Inputs of the first `per_tensor` elements (whole groups) of each tensor
+    of the slice, concatenated: master, gradient bits and a stored state (codes,
+    root scale, k) drawn by the seeded generator -- the same recipe as the
+    parity tests' identical-input states.  On the device when one is in use
+    (bit-identical and much faster than the NumPy generator), else NumPy on
+    host threads."""
     import synth
+    from synth.params import llama2_7b
+    shapes = llama2_7b()[:SLICE_TENSORS]
+    counts = [min(n, per_tensor) // 128 * 128 for _, n in shapes]
+
+    def one(i):
+        c = counts[i]
+        ng = c // 128
+        if use_device:
+            import torch
+            m = torch.empty(c, dtype=torch.float32, device="cuda")
+            g = torch.empty(c, dtype=torch.int16, device="cuda")
+            q = torch.empty(c, dtype=torch.uint8, device="cuda")
+            synth.device_master(m, 0, i)
+            synth.device_grad(g, 0, i, 1)
+            master, grad = m.cpu().numpy(), g.cpu().numpy().view(np.uint16)
+            synth.device_state_codes(q, 0, i, 1, fmt_m, True)
+            mq = q.cpu().numpy()
+            synth.device_state_codes(q, 0, i, 1, fmt_v, False)
+            vq = q.cpu().numpy()
+        else:
+            master = synth.master(0, i, 0, c)
+            grad = synth.grad_bits(0, i, 1, 0, c)
+            mq = synth.state_codes(0, i, 1, 0, c, fmt_m, True)
+            vq = synth.state_codes(0, i, 1, 0, c, fmt_v, False)
+        km, sm, kv, sv = synth.state_groups(0, i, 1, 0, ng)
+        return master, grad, mq, vq, sm, km, sv, kv
+
     if use_device:
-        import torch
-        m = torch.empty(count, dtype=torch.float32, device="cuda")
-        g = torch.empty(count, dtype=torch.int16, device="cuda")
-        synth.device_master(m, 0, 0)
-        master = m.cpu().numpy()
-        synth.device_m_warm(m, 0, 0)
-        m0 = m.cpu().numpy()
-        synth.device_v_warm(m, 0, 0)
-        v0 = m.cpu().numpy()
-        synth.device_grad(g, 0, 0, 1)
-        grad = g.cpu().numpy().view(np.uint16)
-        del m, g
+        parts = [one(i) for i in range(len(shapes))]
     else:
-        master = synth.master(0, 0, 0, count)
-        m0 = synth.m_warm(0, 0, 0, count)
-        v0 = synth.v_warm(0, 0, 0, count)
-        grad = synth.grad_bits(0, 0, 1, 0, count)
-    return master, m0, v0, grad
+        import concurrent.futures as cf
+        with cf.ThreadPoolExecutor(min(len(shapes), host_cores())) as ex:
+            parts = list(ex.map(one, range(len(shapes))))
+    cat = [np.ascontiguousarray(np.concatenate([p[j] for p in parts])) for j in range(8)]
+    return cat, counts
 
 
-def time_oracle(cfg, count, steps, use_device):
+def time_oracle(cfg, per_tensor, steps, threads, use_device, inputs=None):
+    """Per-step seconds of the oracle's step over the slice sample on `threads`
+    host threads (group-aligned slices, one C call each; bit for bit the
+    single-call result)."""
     import oracle as orc
     from synth.params import HYPER as H
-    master, m0, v0, grad = oracle_sample_inputs(cfg, count, use_device)
-    ng = -(-count // 128)
-    mq = np.zeros(ng * 128, np.uint8)
-    vq = np.zeros(ng * 128, np.uint8)
-    q, s, k = orc.group_quantize(m0.reshape(1, count), 1, 128, True, cfg["fmt_m"])
-    mq[:count], ms, mk = q.ravel(), s.ravel().copy(), k.ravel().copy()
-    q, s, k = orc.group_quantize(v0.reshape(1, count), 1, 128, True, cfg["fmt_v"])
-    vq[:count], vs, vk = q.ravel(), s.ravel().copy(), k.ravel().copy()
-    weight = np.zeros(count, np.uint16)
+    if inputs is None:
+        inputs, _ = oracle_slice_inputs(per_tensor, cfg["fmt_m"], cfg["fmt_v"], use_device)
+    master, grad, mq, vq, sm, km, sv, kv = (a.copy() for a in inputs)
+    weight = np.zeros(master.size, np.uint16)
     times = []
     for t in range(1, steps + 1):
         t0 = time.perf_counter()
-        orc.adamw_step(master, weight, grad, mq, ms, mk, vq, vs, vk, lr=H["lr"], beta1=H["beta1"],
-                       beta2=H["beta2"], eps=H["eps"], wd=H["wd"], step=t, fmt_m=cfg["fmt_m"],
-                       fmt_v=cfg["fmt_v"])
+        orc.adamw_step_threads(master, weight, grad, mq, sm, km, vq, sv, kv, threads=threads,
+                               lr=H["lr"], beta1=H["beta1"], beta2=H["beta2"], eps=H["eps"],
+                               wd=H["wd"], step=t, fmt_m=cfg["fmt_m"], fmt_v=cfg["fmt_v"])
         times.append(time.perf_counter() - t0)
     return times
+
+
+def cpu_baseline(cfg, per_tensor, use_device):
+    """The oracle on every host core over the slice sample (median of three
+    steps), next to one core on its first 2^21 elements, and the whole 7B
+    list's step time extrapolated from the all-cores rate."""
+    cores = host_cores()
+    inputs, counts = oracle_slice_inputs(per_tensor, cfg["fmt_m"], cfg["fmt_v"], use_device)
+    total = int(sum(counts))
+    t_all = statistics.median(time_oracle(cfg, per_tensor, 3, cores, use_device, inputs))
+    one = min(total, 1 << 21)
+    t_one = time_oracle(cfg, per_tensor, 1, 1, use_device, [a[:one] if a.size == total else
+                                                           a[:one // 128] for a in inputs])[0]
+    rate = total / t_all
+    return {"value": round(rate / 1e9, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": "first %d elements of each of the %d tensors of the %s (%d elements, "
+                      "stored states from the seeded generator), one step on %d host threads, "
+                      "median of 3 steps (%.2f s each)" % (per_tensor, len(counts), SLICE_NAME,
+                                                             total, cores, t_all),
+            "one_core": {"value": round(one / t_one / 1e9, 6), "unit": UNIT, "cores": 1,
+                         "sample": "first %d elements of the same sample, one step (%.2f s)"
+                                   % (one, t_one)},
+            "llama2_7b_step_s_extrapolated": round(LLAMA2_7B_PARAMS / rate, 1),
+            "nproc": cores}
 
 
 # ----------------------------------------------------------------------------
@@ -315,8 +372,11 @@ def run_ours(args, cfg, ws, rank, local):
             coat.coat_adamw_step_multi(plan, lr=H["lr"], beta1=H["beta1"], beta2=H["beta2"],
                                        eps=H["eps"], wd=H["wd"], step=step_no[0])
 
+    nvtx = torch.cuda.nvtx
+    nvtx.range_push("warm-up: %d steps" % args.warmup)
     for _ in range(args.warmup):
         one_step()
+    nvtx.range_pop()
     torch.cuda.synchronize()
     coat.coat_check_device_error()
 
@@ -330,12 +390,16 @@ def run_ours(args, cfg, ws, rank, local):
     barrier(ws, dev)
     torch.cuda.synchronize()
     wall0 = time.time()
+    nvtx.range_push("timed region: %d steps" % args.steps)
     t_start.record(stream)
     for i in range(args.steps):
+        nvtx.range_push("step %d" % i)
         ev[i][0].record(stream)
         one_step(ev[i][2])
         ev[i][1].record(stream)
+        nvtx.range_pop()
     t_end.record(stream)
+    nvtx.range_pop()
     torch.cuda.synchronize()
     wall1 = time.time()
     barrier(ws, dev)
@@ -391,12 +455,12 @@ def run_ours(args, cfg, ws, rank, local):
         e2e = run_e2e(args, cfg, ps, ws, dev, H, coat)
 
     plan.destroy()
+    n_total = ps.total_elements
+    del ps
+    torch.cuda.empty_cache()
     # many-tensor launch overhead: the same parameter count as one flat tensor
     vs_flat = None
     if n_tensors > 1 and args.compare_flat:
-        n_total = ps.total_elements
-        del ps
-        torch.cuda.empty_cache()
         fps, fplan = make_workload([("flat", n_total)], cfg, rank, coat)
         flat_ms = max_over_ranks(time_plan(fplan, args.steps, args.warmup, H, coat), ws, dev)
         fplan.destroy()
@@ -407,16 +471,14 @@ def run_ours(args, cfg, ws, rank, local):
                    "flat_ms_per_step": round(flat_ms, 4), "ratio": round(value / flat_value, 4),
                    "how": "the same parameter count as one flat tensor, same formats and "
                           "hyperparameters, device events around the same number of steps"}
+    extras = None
+    if ws == 1 and args.extras and args.config == "llama2-7b" and clip_buf is None:
+        extras = run_extras(args, coat, H, local)
     result = None
     if rank == 0:
         cpu = None
         if ws == 1 and not args.no_cpu_baseline:
-            count = args.cpu_sample
-            times = time_oracle(cfg, count, 1, use_device=True)
-            cpu = {"value": round(count / times[0] / 1e9, 6), "unit": UNIT, "cores": 1,
-                   "kind": "oracle",
-                   "sample": "first %d elements of tensor 0 of the workload, 1 step, one host "
-                             "thread (%.1f s)" % (count, times[0])}
+            cpu = cpu_baseline(cfg, args.cpu_sample, use_device=True)
         result = {
             "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup,
@@ -435,6 +497,8 @@ def run_ours(args, cfg, ws, rank, local):
         }
         if clip is not None:
             result["clip"] = clip
+        if extras is not None:
+            result["other_workloads"] = extras
         if vs_flat is not None:
             result["vs_flat_tensor"] = vs_flat
     if ws > 1:
@@ -442,6 +506,61 @@ def run_ours(args, cfg, ws, rank, local):
         dist.barrier(device_ids=[local])
         dist.destroy_process_group()
     return result
+
+
+def run_extras(args, coat, H, local):
+    """Figures of the other workloads in the same run (one GPU), so that they are
+    recorded next to the headline: the ragged 10,000-tensor list against one flat
+    tensor of the same size (multi-tensor overhead), the Llama-2-13B list, and
+    the mixed-granularity codec workload.  Each list: device events around
+    `steps` launches after 3 warm-up launches, inputs far larger than L2."""
+    import torch
+    from synth.params import CONFIGS
+    peaks = measured_peaks()
+    peak = peaks["hbm_gbs"] if peaks and peaks.get("hbm_gbs") else HBM_FALLBACK_GBS
+    steps = max(3, min(args.steps, 10))
+    out = {"how": "per workload: %d timed launches after 3 warm-up launches, CUDA events on the "
+                  "launching stream; frac = algorithmic bytes / kernel time / peak (%s %.1f GB/s)"
+                  % (steps, "measured" if peaks else "fallback", peak)}
+
+    def one_list(name, shapes):
+        cfg = dict(CONFIGS[name]) if name in CONFIGS else None
+        ps, plan = make_workload(shapes, cfg, 0, coat)
+        ms = time_plan(plan, steps, 3, H, coat)
+        n, sizes = ps.total_elements, list(ps.sizes)
+        plan.destroy()
+        del ps
+        torch.cuda.empty_cache()
+        alg = algorithmic_bytes(sizes, with_weight=True)
+        gbs = alg / (ms * 1e-3) / 1e9
+        return {"value": round(n / (ms * 1e-3) / 1e9, 3), "unit": UNIT, "ms_per_step": round(ms, 4),
+                "params": n, "tensors": len(sizes), "achieved_GBs": round(gbs, 1),
+                "frac": round(gbs / peak, 4)}, n
+
+    from synth.params import ragged, llama2_13b
+    r, n_r = one_list("ragged", ragged())
+    flat_cfg = dict(CONFIGS["ragged"])
+    fps, fplan = make_workload([("flat", n_r)], flat_cfg, 0, coat)
+    fms = time_plan(fplan, steps, 3, H, coat)
+    fplan.destroy()
+    del fps
+    torch.cuda.empty_cache()
+    r["workload"] = CONFIGS["ragged"]["workload"]
+    r["flat_value"] = round(n_r / (fms * 1e-3) / 1e9, 3)
+    r["ratio_to_flat"] = round(r["value"] / r["flat_value"], 4)
+    out["ragged"] = r
+    b, _ = one_list("llama2-13b", llama2_13b())
+    b["workload"] = CONFIGS["llama2-13b"]["workload"]
+    out["llama2_13b"] = b
+    cargs = argparse.Namespace(steps=steps, warmup=3, no_e2e=True, no_cpu_baseline=True,
+                               e2e_steps=1)
+    c = run_codec(cargs, 1, 0, local)
+    out["act_codec"] = {"value": c["value"], "unit": c["unit"], "ms_per_step": c["ms_per_step"],
+                        "workload": c["config"]["workload"],
+                        "launches": [{k: x[k] for k in ("launch", "ms", "GB/s", "frac")}
+                                     for x in c["launches"]]}
+    coat.coat_check_device_error()
+    return out
 
 
 def run_e2e(args, cfg, ps, ws, dev, H, coat):
@@ -1006,24 +1125,155 @@ def run_rmsnorm(args, ws, rank, local):
     return result
 
 
+ZERO1_METRIC = ("Gparams/s of the ZeRO-1 sharded FP8-state AdamW step (reduce-scatter + step + "
+                "all-gather); HBM GB/s as % of B200 roofline")
+
+
+def run_zero1(args, cfg, ws, rank, local):
+    """ZeRO-1 over the Llama-2-7B list on N ranks: per step an NCCL reduce-scatter
+    (sum) of the flat bf16 gradients, the FP8 step on the rank's 1/N of the
+    groups, an NCCL all-gather of the bf16 weights.  The list is fixed, so the
+    per-rank work shrinks with N ("strong" scaling).  Device events around each
+    phase on the launching stream; every figure is the max over ranks.  The
+    gradient buffer is not refilled between steps (the reduce-scatter sums in
+    place, so the shard's values grow by about N g per step, which changes no
+    timing)."""
+    import datetime
+    import socket
+    import torch
+    import torch.distributed as dist
+    import fp8_optimizer_state_b200 as coat
+    import synth
+    from fp8_optimizer_state_b200.zero1 import Zero1AdamW
+    from synth.params import HYPER as H
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws == 1 and "MASTER_PORT" not in os.environ:
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(sk.getsockname()[1]))
+    dist.init_process_group("nccl", rank=rank, world_size=ws,
+                            timeout=datetime.timedelta(seconds=120), device_id=dev)
+    coat.lib()
+    shapes = cfg["shapes"]()
+    sizes = [n for _, n in shapes]
+    z = Zero1AdamW(sizes, device=dev, fmt_m=cfg["fmt_m"], fmt_v=cfg["fmt_v"])
+    for i, n in enumerate(sizes):
+        synth.device_grad(z.grad(i), rank, i, 1)
+    tmp = None
+    for piece in z.pieces:
+        t, b, n, _ = piece
+        v = z.piece_views(piece)
+        synth.device_master(v["master"], 0, t, start=b)
+        for which, q, sc, kk, fmt in (("m", "m_q", "m_scale", "m_k", cfg["fmt_m"]),
+                                      ("v", "v_q", "v_scale", "v_k", cfg["fmt_v"])):
+            if tmp is None or tmp.numel() < n:
+                tmp = torch.empty(n, dtype=torch.float32, device=dev)
+            (synth.device_m_warm if which == "m" else synth.device_v_warm)(tmp[:n], 0, t, start=b)
+            coat.coat_group_quantize(tmp[:n].view(1, n), 1, 128, True, fmt, v[q].view(1, -1),
+                                     v[sc].view(1, -1), v[kk].view(1, -1))
+    del tmp
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    hp = dict(lr=H["lr"], beta1=H["beta1"], beta2=H["beta2"], eps=H["eps"], wd=H["wd"])
+    step_no = [0]
+
+    def one_step(ev=None):
+        step_no[0] += 1
+        if ev is not None:
+            ev[0].record(stream)
+        z.reduce_scatter_grads()
+        if ev is not None:
+            ev[1].record(stream)
+        z.local_step(step=step_no[0], **hp)
+        if ev is not None:
+            ev[2].record(stream)
+        z.all_gather_weights()
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    coat.coat_check_device_error()
+    sampler = ClockSampler(pci_bus_id(dev))
+    sampler.start()
+    time.sleep(0.3)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier(device_ids=[local])
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    t0.record(stream)
+    for i in range(args.steps):
+        one_step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    dist.barrier(device_ids=[local])
+    time.sleep(0.2)
+    sampler.stop()
+    coat.coat_check_device_error()
+    elapsed = max_over_ranks(t0.elapsed_time(t1), ws, dev)
+    phase = [max_over_ranks(statistics.mean(e[k].elapsed_time(e[k + 1]) for e in evs), ws, dev)
+             for k in range(3)]
+    n_params = sum(sizes)
+    shard_sizes = [n for _, _, n, _ in z.pieces]
+    alg = algorithmic_bytes(shard_sizes, with_weight=True)
+    alg_max = max_over_ranks(float(alg), ws, dev)
+    peaks = measured_peaks()
+    peak = peaks["hbm_gbs"] if peaks and peaks.get("hbm_gbs") else HBM_FALLBACK_GBS
+    step_gbs = alg_max / (phase[1] * 1e-3) / 1e9 if phase[1] > 0 else 0.0
+    mem = sum(x.numel() * x.element_size() for x in
+              (z.flat_grad, z.flat_weight, z.master, z.m_q, z.v_q, z.m_scale, z.m_k, z.v_scale, z.v_k))
+    clocks = sampler.summary(wall0, wall1)
+    z.close()
+    result = None
+    if rank == 0:
+        result = {
+            "metric": ZERO1_METRIC, "value": round(n_params * args.steps / (elapsed * 1e-3) / 1e9, 3),
+            "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(elapsed / args.steps, 4), "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": cfg["workload"] + ", ZeRO-1 over %d ranks" % ws,
+                       "params_total": n_params, "shard_elems": z.shard_elems,
+                       "parallelism": "zero1-dp%d (NCCL reduce-scatter + all-gather)" % ws,
+                       "l2": "no flush: every array is far larger than L2"},
+            "phases_ms": {"reduce_scatter": round(phase[0], 4), "step": round(phase[1], 4),
+                          "all_gather": round(phase[2], 4)},
+            "roofline": {"bound": "hbm", "achieved": round(step_gbs, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(step_gbs / peak, 4), "traffic": None,
+                         "kernel": "the step on the rank's shard",
+                         "peak_source": "measured" if peaks else "fallback"},
+            "bytes_per_rank": mem, "gpu_launches": args.steps, "clocks": clocks,
+            "cpu_baseline": None, "e2e": None}
+    dist.barrier(device_ids=[local])
+    dist.destroy_process_group()
+    return result
+
+
 def run_reference(args, cfg, ws, rank):
-    """The CPU oracle on a bounded sample per step (one host thread)."""
+    """The CPU oracle, every host core, on the bounded slice sample per step."""
     if rank != 0:
         return None
-    count = args.ref_sample
-    times = time_oracle(cfg, count, args.warmup + args.steps, use_device=False)
+    cores = host_cores()
+    inputs, counts = oracle_slice_inputs(args.ref_sample, cfg["fmt_m"], cfg["fmt_v"], False)
+    total = int(sum(counts))
+    times = time_oracle(cfg, args.ref_sample, args.warmup + args.steps, cores, False, inputs)
     timed = times[args.warmup:]
-    total = sum(timed)
-    value = count * len(timed) / total / 1e9
-    sample = ("first %d elements of tensor 0 of the workload per step (bits from the seeded "
-              "generator), oracle adamw_step, one host thread" % count)
+    el = sum(timed)
+    value = total * len(timed) / el / 1e9
+    sample = ("first %d elements of each of the %d tensors of the %s per step (%d elements; "
+              "stored states from the seeded generator), oracle adamw_step on %d host threads "
+              "(group-aligned slices)" % (args.ref_sample, len(counts), SLICE_NAME, total, cores))
     return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(1e3 * total / len(timed), 3), "higher_is_better": True,
+            "ms_per_step": round(1e3 * el / len(timed), 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": cfg["workload"], "sample_elements": count},
-            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
-                             "sample": sample},
+            "config": {"workload": cfg["workload"], "sample_elements": total},
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores,
+                             "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
@@ -1046,8 +1296,15 @@ def main(argv=None):
                     help="also time one flat tensor of the same parameter count")
     ap.add_argument("--clip", type=float, default=None, metavar="MAX_NORM",
                     help="time the clipped step: gradient-norm pass + step on coef * g")
-    ap.add_argument("--cpu-sample", type=int, default=16 << 20)
-    ap.add_argument("--ref-sample", type=int, default=2 << 20)
+    ap.add_argument("--zero1", action="store_true",
+                    help="time the ZeRO-1 sharded step (reduce-scatter, step, all-gather) over "
+                         "the ranks instead of one replica per rank")
+    ap.add_argument("--no-extras", dest="extras", action="store_false",
+                    help="skip the ragged, 13B and codec figures of the default run")
+    ap.add_argument("--cpu-sample", type=int, default=1 << 20,
+                    help="oracle baseline: elements per tensor of the 7B slice")
+    ap.add_argument("--ref-sample", type=int, default=1 << 19,
+                    help="reference arm: elements per tensor of the 7B slice per step")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -1069,6 +1326,8 @@ def main(argv=None):
         cfg["workload"] = cfg["workload"].split(", E4M3")[0] + ", E4M3 m + %s v" % FMT_NAMES[args.fmt_v]
     if args.impl == "reference":
         res = run_reference(args, cfg, ws, rank)
+    elif args.zero1:
+        res = run_zero1(args, cfg, ws, rank, local)
     else:
         res = run_ours(args, cfg, ws, rank, local)
     if res is not None:

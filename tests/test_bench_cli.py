@@ -38,4 +38,5 @@ def test_reference_arm_single_process_line():
     for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
                 "higher_is_better", "cpu_baseline", "e2e", "config"):
         assert key in rec, key
-    assert rec["n_gpus"] == 1 and rec["cpu_baseline"]["cores"] == 1
+    assert rec["n_gpus"] == 1 and rec["cpu_baseline"]["cores"] == len(os.sched_getaffinity(0))
+    assert rec["config"]["sample_elements"] == 8 * 4096 + 2 * 4096   # 10 tensors of the 7B slice

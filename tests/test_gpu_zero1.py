@@ -103,3 +103,21 @@ def test_world_size_one_equals_the_multi_tensor_step(max_norm):
         if plan is not None:
             plan.destroy()
         dist.destroy_process_group()
+
+
+def test_bench_zero1_mode_line():
+    """bench.py --zero1 (one NCCL rank here): the sharded step's JSON line with
+    its three phases."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    p = subprocess.run([sys.executable, "bench.py", "--zero1", "--config", "flat-256m", "--steps",
+                        "3", "--warmup", "3"], cwd=root, capture_output=True, text=True,
+                       timeout=600)
+    assert p.returncode == 0, p.stderr[-3000:]
+    rec = json.loads([l for l in p.stdout.splitlines() if l.startswith("{")][0])
+    assert rec["scaling"] == "strong" and rec["n_gpus"] == 1 and rec["value"] > 0
+    assert set(rec["phases_ms"]) == {"reduce_scatter", "step", "all_gather"}
+    assert 0 < rec["roofline"]["frac"] < 1.5
