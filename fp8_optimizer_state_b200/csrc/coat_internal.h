@@ -56,9 +56,10 @@ int sm_count(int dev);
 // Grid of at most sm_count(dev) * max_blocks_per_sm CTAs for work_items items
 // of per_block each (at least 1).
 unsigned grid_for(int64_t work_items, int per_block, int dev, int max_blocks_per_sm);
-// CTAs of a 256-thread kernel (plus dyn_smem bytes of dynamic shared memory)
-// resident per SM, from the occupancy calculator, cached per kernel.
-int resident_ctas(const void* kernel, size_t dyn_smem = 0);
+// CTAs of a kernel launched with `threads` threads (plus dyn_smem bytes of
+// dynamic shared memory) resident per SM, from the occupancy calculator,
+// cached per kernel.
+int resident_ctas(const void* kernel, size_t dyn_smem = 0, int threads = 256);
 cudaError_t device_error_ptr(unsigned** out);
 int64_t step_tile_groups();
 

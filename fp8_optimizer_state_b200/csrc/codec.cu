@@ -127,6 +127,76 @@ struct RowItem {
   int valid;      // elements of the lane's 16 that exist
 };
 
+// Codes of 8 bf16 values (the words of u) of a group without an Inf or a NaN,
+// with k = 1: the same codes as encode_words<FMT, 8, true> with use_div, with
+// the arithmetic on element pairs.  The magnitudes are the words with their
+// sign bits cleared; the correctly rounded quotients FMT_MAX |x| / M
+// (div_exact) and the encoder's fused adds run as packed FP32 pairs, and the
+// signs come from the words' top bits.
+template <int FMT>
+__device__ __forceinline__ void encode8_bf16_div(const uint4& u, const GroupDiv& d,
+                                                 uint32_t (&cw)[2]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  const float2 num2 = make_float2(d.num, d.num), y2 = make_float2(d.y, d.y);
+  const float2 nb2 = make_float2(-d.b, -d.b);
+  uint32_t mag[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t aw = w[j] & 0x7FFF7FFFu;
+    const float2 a = mul2(make_float2(bf16lo(aw), bf16hi(aw)), num2);
+    const float2 q0 = mul2(a, y2);
+    const float2 y = fma2(fma2(q0, nb2, a), y2, q0);
+    const uint2 c = enc_mag_bounded2<FMT, FMT>(y.x, y.y);
+    mag[2 * j] = c.x;
+    mag[2 * j + 1] = c.y;
+  }
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const uint32_t mags = pack4(mag[4 * t], mag[4 * t + 1], mag[4 * t + 2], mag[4 * t + 3]);
+    const uint32_t top = __byte_perm(w[2 * t], w[2 * t + 1], 0x7531u);
+    cw[t] = mags | (top & (mags + 0x7F7F7F7Fu) & 0x80808080u);
+  }
+}
+
+// bf16 input without expansion, when none of the warp's four groups holds an
+// Inf or a NaN (returns false otherwise, and the caller takes the general
+// path): the general path's codes and scales.  The group maximum is an
+// unsigned 16-bit max over the words with their sign bits cleared, whose
+// halves order like the magnitudes they encode (an Inf or a NaN pattern is
+// above every finite one).
+template <int FMT>
+__device__ __forceinline__ bool quant_bf16_plain(const RowItem<1>& it, int64_t rows, int64_t cols,
+                                                 int l, int64_t nbc, uint8_t* __restrict__ q,
+                                                 int64_t ldq, float* __restrict__ scale,
+                                                 float* __restrict__ kk) {
+  const uint4 u[2] = {it.raw.a, it.raw.b};
+  uint32_t mx2 = 0u;
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+    mx2 = __vmaxu2(mx2, __vmaxu2(__vmaxu2(u[h].x & 0x7FFF7FFFu, u[h].y & 0x7FFF7FFFu),
+                                 __vmaxu2(u[h].z & 0x7FFF7FFFu, u[h].w & 0x7FFF7FFFu)));
+  uint32_t mxb = max(mx2 & 0xFFFFu, mx2 >> 16);
+#pragma unroll
+  for (int off = 1; off < 8; off <<= 1) mxb = max(mxb, __shfl_xor_sync(0xFFFFFFFFu, mxb, off));
+  if (__any_sync(0xFFFFFFFFu, mxb >= 0x7F80u)) return false;
+  const float M = __uint_as_float(mxb << 16);
+  const GroupDiv d = codec_div<FMT>(M);
+  uint32_t lo[2], hi[2];
+  encode8_bf16_div<FMT>(u[0], d, lo);
+  encode8_bf16_div<FMT>(u[1], d, hi);
+  const uint32_t cw[4] = {lo[0], lo[1], hi[0], hi[1]};
+  if (it.valid > 0 && COAT_INDEX_OK(it.r < rows && it.c + it.valid <= cols))
+    store16(q + it.r * ldq + it.c, cw, it.valid);
+  if (l == 0 && it.valid > 0) {
+    const int64_t g = it.r * nbc + (it.c >> 7);
+    if (COAT_INDEX_OK(g < rows * nbc)) {
+      scale[g] = M > 0.0f ? div_fmax<FMT>(M) : 1.0f;
+      kk[g] = 1.0f;
+    }
+  }
+  return true;
+}
+
 template <int FMT, int DT, bool EXPAND>
 __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__ x, int64_t rows,
                                                         int64_t cols, int64_t ldx,
@@ -153,12 +223,10 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
     cc += 4 * kGroup;
     if (cc >= rowspan) { cc -= rowspan; ++cr; }
   };
-  RowItem<DT> cur;
-  load(cur);
-  for (int64_t item = i0; item < i1; ++item) {
-    RowItem<DT> nxt;
-    if (item + 1 < i1) load(nxt);
-
+  auto body = [&](const RowItem<DT>& cur) {
+    if constexpr (DT == 1 && !EXPAND) {
+      if (quant_bf16_plain<FMT>(cur, rows, cols, l, nbc, q, ldq, scale, kk)) return;
+    }
     float v[16];
     unpack16<DT>(cur.raw, v);
     float M, mu = 0.0f;
@@ -195,7 +263,7 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
     } else {
       // k = 1: the root scale is M / FMT_MAX, correctly rounded (1 for an all-zero group)
       k = 1.0f;
-      sr = M > 0.0f ? __fdiv_rn(M, F8<FMT>::MAXV) : 1.0f;
+      sr = M > 0.0f ? div_fmax<FMT>(M) : 1.0f;
     }
     const bool use_div = !EXPAND || k == 1.0f;
     GroupDiv d{};
@@ -215,6 +283,13 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
         kk[g] = k;
       }
     }
+  };
+  RowItem<DT> cur;
+  load(cur);
+  for (int64_t item = i0; item < i1; ++item) {
+    RowItem<DT> nxt;
+    if (item + 1 < i1) load(nxt);
+    body(cur);
     cur = nxt;
   }
 }
@@ -393,7 +468,7 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
     } else {
       // k = 1: the root scale is M / FMT_MAX, correctly rounded (1 for an all-zero block)
       k = 1.0f;
-      sr = M > 0.0f ? __fdiv_rn(M, F8<FMT>::MAXV) : 1.0f;
+      sr = M > 0.0f ? div_fmax<FMT>(M) : 1.0f;
     }
     const bool use_div = !EXPAND || k == 1.0f;
     GroupDiv d{};
@@ -403,13 +478,22 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int64_t r = br * 128 + warp * 16 + 2 * i + (lane >> 4);
-      float v[8];
-      block_row<DT>(cur, i, v);
       uint32_t cw[2];
-      if (!special)
-        encode_words<FMT, 8, true>(v, use_div, d, invM, k, cw);
-      else
-        encode_words<FMT, 8, false>(v, use_div, d, invM, k, cw);
+      bool packed = false;
+      if constexpr (DT == 1) {
+        if (!special && use_div) {
+          encode8_bf16_div<FMT>(cur.a[i], d, cw);
+          packed = true;
+        }
+      }
+      if (!packed) {
+        float v[8];
+        block_row<DT>(cur, i, v);
+        if (!special)
+          encode_words<FMT, 8, true>(v, use_div, d, invM, k, cw);
+        else
+          encode_words<FMT, 8, false>(v, use_div, d, invM, k, cw);
+      }
       const int valid = r < rows && COAT_INDEX_OK(cv == 0 || c + cv <= cols) ? cv : 0;
       uint8_t* qp = q + r * ldq + c;
       if (valid >= 8) {
@@ -666,12 +750,12 @@ std::mutex g_occ_mu;
 std::unordered_map<const void*, int> g_occ;
 }  // namespace
 
-int resident_ctas(const void* kernel, size_t dyn_smem) {
+int resident_ctas(const void* kernel, size_t dyn_smem, int threads) {
   std::lock_guard<std::mutex> lk(g_occ_mu);
   auto it = g_occ.find(kernel);
   if (it != g_occ.end()) return it->second;
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, 256, dyn_smem) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, dyn_smem) != cudaSuccess ||
       n < 1) {
     cudaGetLastError();
     n = 1;

@@ -176,14 +176,19 @@ __device__ __forceinline__ void quantize_lane16(const float (&h)[16], bool force
       group_params<FMT>(M, __uint_as_float((mink + 2u) >> 1), true, k, sr, invM);
     } else {
       k = 1.0f;
-      sr = M > 0.0f ? __fdiv_rn(M, F8<FMT>::MAXV) : 1.0f;   // M / FMT_MAX, correctly rounded
+      sr = M > 0.0f ? div_fmax<FMT>(M) : 1.0f;   // M / FMT_MAX, correctly rounded
       invM = M > 0.0f ? rcp_approx(M) : 0.0f;   // an all-zero group encodes to zeros
     }
     float y[16];
     if (k == 1.0f) {
       const float c = F8<FMT>::MAXV * invM;
+      const float2 c2 = make_float2(c, c);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) y[i] = h[i] * c;
+      for (int i = 0; i < 16; i += 2) {
+        const float2 q = mul2(make_float2(h[i], h[i + 1]), c2);
+        y[i] = q.x;
+        y[i + 1] = q.y;
+      }
     } else {
 #pragma unroll
       for (int i = 0; i < 16; ++i) y[i] = with_sign_of(expand_value<FMT>(h[i], invM, k), h[i]);
@@ -248,16 +253,32 @@ __device__ __forceinline__ void quantize_scaled16(const float (&p)[16], float C,
     return;
   }
   k = 1.0f;
-  sr = My > 0.0f ? __fdiv_rn(My, F8<FMT>::MAXV) : 1.0f;
+  sr = My > 0.0f ? div_fmax<FMT>(My) : 1.0f;
   float y[16];
   if (EXACT) {
+    // div_exact on the signed values, two at a time: every step rounds to
+    // nearest, which is symmetric in the sign, so each result is
+    // sign(p) RN(FMT_MAX |p| / max|p|)
     const GroupDiv dv = codec_div<FMT>(mp);
+    const float2 num2 = make_float2(dv.num, dv.num), y2 = make_float2(dv.y, dv.y);
+    const float2 nb2 = make_float2(-dv.b, -dv.b);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) y[i] = with_sign_of(div_exact(p[i], dv), p[i]);
+    for (int i = 0; i < 16; i += 2) {
+      const float2 a = mul2(make_float2(p[i], p[i + 1]), num2);
+      const float2 q0 = mul2(a, y2);
+      const float2 q = fma2(fma2(q0, nb2, a), y2, q0);
+      y[i] = q.x;
+      y[i + 1] = q.y;
+    }
   } else {
     const float c = mp > 0.0f ? F8<FMT>::MAXV * rcp_approx(mp) : 0.0f;
+    const float2 c2 = make_float2(c, c);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) y[i] = p[i] * c;
+    for (int i = 0; i < 16; i += 2) {
+      const float2 q = mul2(make_float2(p[i], p[i + 1]), c2);
+      y[i] = q.x;
+      y[i + 1] = q.y;
+    }
   }
   encode_hw16<FMT>(y, cw);
 }
@@ -318,22 +339,25 @@ __global__ void __launch_bounds__(256) swiglu_fwd_kernel(const ActArgs gate, con
     cc += 4 * kGroup;
     if (cc >= rowspan) { cc -= rowspan; ++cr; }
   };
-  FwdItem cur;
-  load(cur);
-  for (int64_t item = i0; item < i1; ++item) {
-    FwdItem nxt;
-    if (item + 1 < i1) load(nxt);
-
+  auto body = [&](const FwdItem& cur) {
     const bool plain = __all_sync(0xFFFFFFFFu, cur.gk == 1.0f && cur.uk == 1.0f);
     float fg[16], fu[16], h[16];
     decode16_raw<FMT>(cur.gw, cur.gk, plain, tab, fg);
     decode16_raw<FMT>(cur.uw, cur.uk, plain, tab, fu);
     const float ct = cur.gs * -1.4426950408889634f;   // -log2(e) s_g
     const float S = cur.gs * cur.us;
+    const float2 ct2 = make_float2(ct, ct), one2 = make_float2(1.0f, 1.0f);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float sg = rcp_approx(1.0f + ex2_approx(fg[i] * ct));
-      h[i] = (fg[i] * fu[i]) * sg;   // h / (s_g s_u)
+    for (int i = 0; i < 16; i += 2) {
+      // sigmoid(g) = 1 / (1 + 2^(-log2(e) g)) and h / (s_g s_u) = (f_g f_u) sigmoid(g),
+      // two elements per operation
+      const float2 f = make_float2(fg[i], fg[i + 1]);
+      const float2 e = mul2(f, ct2);
+      const float2 den = add2(make_float2(ex2_approx(e.x), ex2_approx(e.y)), one2);
+      const float2 hh = mul2(mul2(f, make_float2(fu[i], fu[i + 1])),
+                             make_float2(rcp_approx(den.x), rcp_approx(den.y)));
+      h[i] = hh.x;
+      h[i + 1] = hh.y;
     }
 
     uint32_t cw[4];
@@ -346,6 +370,13 @@ __global__ void __launch_bounds__(256) swiglu_fwd_kernel(const ActArgs gate, con
         out.k[cur.r * out.lds + (cur.c >> 7)] = k;
       }
     }
+  };
+  FwdItem cur;
+  load(cur);
+  for (int64_t item = i0; item < i1; ++item) {
+    FwdItem nxt;
+    if (item + 1 < i1) load(nxt);
+    body(cur);
     cur = nxt;
   }
 }
@@ -435,18 +466,19 @@ __global__ void __launch_bounds__(256) swiglu_bwd_kernel(const uint16_t* __restr
 // ---------------------------------------------------------------------------
 // RMSNorm, the other non-linear layer of a Llama block:
 // y = x / sqrt(mean(x^2) + eps) * w per row of d features (d a multiple of
-// 128, at most kNormThreads * 16 * CPT), FP8 1x128 input and output, bf16 w.
-// One 256-thread CTA per row at a time (a persistent loop over rows); thread t
-// holds the 16-column chunks t, t + 256, ... (CPT of them), so that 8
+// 128, at most 256 * 16 * 2), FP8 1x128 input and output, bf16 w.  One CTA of
+// NT threads (128 or 256) per row at a time (a persistent loop over rows);
+// thread t holds the 16-column chunks t, t + NT, ... (CPT of them), so that 8
 // consecutive threads hold one 128-column group and w stays in registers
-// across rows.  Row sums go through warp shuffles and shared memory.
+// across rows.  Row sums go through warp shuffles and shared memory.  The
+// backward uses 256-thread CTAs.
 // ---------------------------------------------------------------------------
 constexpr int kNormThreads = 256;
 
-// Sum of v over the CTA, returned to every thread (red: kNormThreads/32 floats
-// per value, reused only after the barrier that ends this call's reads).
-template <int NV>
-__device__ __forceinline__ void cta_sum_all(float (&v)[NV], float (*red)[kNormThreads / 32]) {
+// Sum of v over the NT threads of the CTA, returned to every thread (red: NT/32
+// floats per value, reused only after the barrier that ends this call's reads).
+template <int NV, int NT>
+__device__ __forceinline__ void cta_sum_all(float (&v)[NV], float (*red)[NT / 32]) {
 #pragma unroll
   for (int n = 0; n < NV; ++n)
 #pragma unroll
@@ -460,7 +492,7 @@ __device__ __forceinline__ void cta_sum_all(float (&v)[NV], float (*red)[kNormTh
   for (int n = 0; n < NV; ++n) {
     float t = 0.0f;
 #pragma unroll
-    for (int w = 0; w < kNormThreads / 32; ++w) t += red[n][w];
+    for (int w = 0; w < NT / 32; ++w) t += red[n][w];
     v[n] = t;
   }
   __syncthreads();
@@ -476,13 +508,13 @@ __device__ __forceinline__ void bf16x16(const uint4& a, const uint4& b, float (&
   }
 }
 
-template <int FMT, bool EXPAND, int CPT>
-__global__ void __launch_bounds__(kNormThreads) rmsnorm_fwd_kernel(const ActArgs x,
+template <int FMT, bool EXPAND, int CPT, int NT>
+__global__ void __launch_bounds__(NT, CPT == 2 ? 16 / (NT / 32) : 1) rmsnorm_fwd_kernel(const ActArgs x,
                                                                    const uint16_t* __restrict__ w,
                                                                    int64_t rows, int64_t d,
                                                                    float eps, const ActArgs out) {
   __shared__ float tab[256];
-  __shared__ float red[1][kNormThreads / 32];
+  __shared__ float red[1][NT / 32];
   fill_log2_table<FMT>(tab);
   __syncthreads();
   const float inv_d = 1.0f / static_cast<float>(d);
@@ -490,7 +522,7 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_fwd_kernel(const ActArgs
   bool ok[CPT];
 #pragma unroll
   for (int j = 0; j < CPT; ++j) {
-    const int64_t c = (threadIdx.x + int64_t(j) * kNormThreads) * 16;
+    const int64_t c = (threadIdx.x + int64_t(j) * NT) * 16;
     ok[j] = c < d;
     if (ok[j]) {
       const uint4* wp = reinterpret_cast<const uint4*>(w + c);
@@ -505,7 +537,7 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_fwd_kernel(const ActArgs
   auto load = [&](int64_t r, In (&in)[CPT]) {
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
-      const int64_t c = (threadIdx.x + int64_t(j) * kNormThreads) * 16;
+      const int64_t c = (threadIdx.x + int64_t(j) * NT) * 16;
       in[j].q = make_uint4(0u, 0u, 0u, 0u);
       in[j].s = in[j].k = 1.0f;
       if (ok[j]) {
@@ -515,11 +547,7 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_fwd_kernel(const ActArgs
       }
     }
   };
-  In cur[CPT];
-  if (blockIdx.x < rows) load(blockIdx.x, cur);
-  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-    In nxt[CPT];
-    if (r + gridDim.x < rows) load(r + gridDim.x, nxt);
+  auto body = [&](int64_t r, const In (&cur)[CPT]) {
     float pv[CPT][16], sv[CPT];
     float ss[1] = {0.0f};
 #pragma unroll
@@ -529,23 +557,29 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_fwd_kernel(const ActArgs
       const bool plain = __all_sync(0xFFFFFFFFu, k == 1.0f);
       float f[16];
       decode16_raw<FMT>(q, k, plain, tab, f);
-      float sf = 0.0f;   // sum of f^2 (x = f s)
+      // sum of f^2 (x = f s) in two interleaved partial sums; p = f w, exact for
+      // k = 1 (an FP8 value times a bf16 value); two elements per operation
+      float2 sf = make_float2(0.0f, 0.0f);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        sf = __fmaf_rn(f[i], f[i], sf);
-        pv[j][i] = f[i] * wv[j][i];   // exact for k = 1: an FP8 value times a bf16 value
+      for (int i = 0; i < 16; i += 2) {
+        const float2 f2 = make_float2(f[i], f[i + 1]);
+        sf = fma2(f2, f2, sf);
+        const float2 p2 = mul2(f2, make_float2(wv[j][i], wv[j][i + 1]));
+        pv[j][i] = p2.x;
+        pv[j][i + 1] = p2.y;
       }
-      ss[0] = __fmaf_rn(sf, s * s, ss[0]);
+      ss[0] = __fmaf_rn(sf.x + sf.y, s * s, ss[0]);
       sv[j] = s;
     }
-    cta_sum_all(ss, red);
-    const float rstd = 1.0f / sqrtf(__fmaf_rn(ss[0], inv_d, eps));
+    cta_sum_all<1, NT>(ss, red);
+    // rstd only scales the root scales (the codes depend on p / max|p| alone)
+    const float rstd = rsqrt_approx(__fmaf_rn(ss[0], inv_d, eps));
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
       uint32_t cw[4];
       float k, sr;
       quantize_scaled16<FMT, EXPAND, true>(pv[j], sv[j] * rstd, cw, k, sr);
-      const int64_t c = (threadIdx.x + int64_t(j) * kNormThreads) * 16;
+      const int64_t c = (threadIdx.x + int64_t(j) * NT) * 16;
       if (ok[j] && COAT_INDEX_OK(c + 16 <= d)) {
         *reinterpret_cast<uint4*>(out.q + r * out.ldq + c) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
         if ((threadIdx.x & 7) == 0) {
@@ -554,6 +588,13 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_fwd_kernel(const ActArgs
         }
       }
     }
+  };
+  In cur[CPT];
+  if (blockIdx.x < rows) load(blockIdx.x, cur);
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    In nxt[CPT];
+    if (r + gridDim.x < rows) load(r + gridDim.x, nxt);
+    body(r, cur);
 #pragma unroll
     for (int j = 0; j < CPT; ++j) cur[j] = nxt[j];
   }
@@ -627,7 +668,7 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_bwd_kernel(
         sums[1] = __fmaf_rn(dv[i] * wv[j][i], xv, sums[1]);
       }
     }
-    cta_sum_all(sums, red);
+    cta_sum_all<2, kNormThreads>(sums, red);
     const float rstd = 1.0f / sqrtf(__fmaf_rn(sums[0], inv_d, eps));
     // rstd^2 mean(g xh) = rstd^3 sum(g x) / d
     const float cx = rstd * rstd * rstd * sums[1] * inv_d;
@@ -732,14 +773,27 @@ void bwd_launch(const uint16_t* dh, int64_t lddh, const ActArgs& gate, const Act
 
 constexpr int kNormMaxCtasPerSm = 8;
 
-template <int FMT, bool EXPAND, int CPT>
+template <int FMT, bool EXPAND, int CPT, int NT>
 cudaError_t rms_fwd_launch(const ActArgs& x, const uint16_t* w, int64_t rows, int64_t d, float eps,
                            const ActArgs& out, int dev, cudaStream_t s) {
-  auto kern = rmsnorm_fwd_kernel<FMT, EXPAND, CPT>;
-  const int per_sm = resident_ctas(reinterpret_cast<const void*>(kern));
+  auto kern = rmsnorm_fwd_kernel<FMT, EXPAND, CPT, NT>;
+  const int per_sm = resident_ctas(reinterpret_cast<const void*>(kern), 0, NT);
   const unsigned g = grid_for(rows, 1, dev, per_sm < kNormMaxCtasPerSm ? per_sm : kNormMaxCtasPerSm);
-  kern<<<g, kNormThreads, 0, s>>>(x, w, rows, d, eps, out);
+  kern<<<g, NT, 0, s>>>(x, w, rows, d, eps, out);
   return cudaGetLastError();
+}
+
+// The forward's shape for rows of d features: 128-thread CTAs holding one or
+// two 16-column chunks per thread up to d = 4096 (so that a thread's per-row
+// work -- its part of the row sum, the group maxima and divisors -- covers as
+// many elements as the registers allow, and an SM keeps four rows in flight),
+// 256 threads with two chunks above.
+template <int FMT, bool EXPAND>
+cudaError_t rms_fwd_dispatch(const ActArgs& x, const uint16_t* w, int64_t rows, int64_t d,
+                             float eps, const ActArgs& out, int dev, cudaStream_t s) {
+  if (d <= 128 * 16) return rms_fwd_launch<FMT, EXPAND, 1, 128>(x, w, rows, d, eps, out, dev, s);
+  if (d <= 128 * 32) return rms_fwd_launch<FMT, EXPAND, 2, 128>(x, w, rows, d, eps, out, dev, s);
+  return rms_fwd_launch<FMT, EXPAND, 2, kNormThreads>(x, w, rows, d, eps, out, dev, s);
 }
 
 template <int FMT, int CPT>
@@ -775,12 +829,9 @@ cudaError_t launch_rmsnorm_fp8_forward(const ActArgs& x, const uint16_t* w, int6
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const bool two = d > int64_t(kNormThreads) * 16;
 #define COAT_RMS_FWD(F)                                                                        \
-  return two ? (expand ? rms_fwd_launch<F, true, 2>(x, w, rows, d, eps, out, dev, s)          \
-                       : rms_fwd_launch<F, false, 2>(x, w, rows, d, eps, out, dev, s))        \
-             : (expand ? rms_fwd_launch<F, true, 1>(x, w, rows, d, eps, out, dev, s)          \
-                       : rms_fwd_launch<F, false, 1>(x, w, rows, d, eps, out, dev, s));
+  return expand ? rms_fwd_dispatch<F, true>(x, w, rows, d, eps, out, dev, s)                   \
+                : rms_fwd_dispatch<F, false>(x, w, rows, d, eps, out, dev, s);
   if (fmt == kE4M3) { COAT_RMS_FWD(kE4M3) }
   if (fmt == kE5M2) { COAT_RMS_FWD(kE5M2) }
   COAT_RMS_FWD(kE5M2Full)

@@ -176,6 +176,7 @@ class FreeRun:
         live = self.element_mask()
         self.master_dev.append(dict(step=t, same_elements=int(same.sum()),
                                     live_elements=int(live.sum()),
+                                    live_fail=int((live & (dev > MASTER_RTOL)).sum()),
                                     literal_fail_same=int((lit & same).sum()),
                                     literal_fail_all=int(lit.sum()),
                                     q50=float(np.quantile(dev, 0.5)),
