@@ -143,19 +143,41 @@ __device__ __forceinline__ void encode8_bf16_div(const uint4& u, const GroupDiv&
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const uint32_t aw = w[j] & 0x7FFF7FFFu;
-    const float2 a = mul2(make_float2(bf16lo(aw), bf16hi(aw)), num2);
+    const float2 a = mul2(make_float2(__uint_as_float(aw * 65536u), bf16hi(aw)), num2);
     const float2 q0 = mul2(a, y2);
     const float2 y = fma2(fma2(q0, nb2, a), y2, q0);
     const uint2 c = enc_mag_bounded2<FMT, FMT>(y.x, y.y);
     mag[2 * j] = c.x;
     mag[2 * j + 1] = c.y;
   }
+  // packing and signs as multiply-adds where the bits do not overlap (the
+  // codes are 7 bits; the sign bits land on zero bits), which the FMA pipe
+  // executes beside the integer pipe that the encoder keeps busy
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    const uint32_t mags = pack4(mag[4 * t], mag[4 * t + 1], mag[4 * t + 2], mag[4 * t + 3]);
+    const uint32_t mags =
+        mag[4 * t] + 256u * (mag[4 * t + 1] + 256u * (mag[4 * t + 2] + 256u * mag[4 * t + 3]));
     const uint32_t top = __byte_perm(w[2 * t], w[2 * t + 1], 0x7531u);
-    cw[t] = mags | (top & (mags + 0x7F7F7F7Fu) & 0x80808080u);
+    cw[t] = mags + (top & (mags + 0x7F7F7F7Fu) & 0x80808080u);
   }
+}
+
+// The division constants of a group whose maximum M is a bf16 value (0 for an
+// all-zero group): as codec_div, with RN(1/b) from one Newton step on
+// rcp.approx.  For any seed within an ulp of 1/b the step's result is
+// RN(1/b) whenever b's significand has at most 8 bits (every bf16 value,
+// scaled or not), which the tests check exactly for all 128 of them.
+template <int FMT>
+__device__ __forceinline__ GroupDiv codec_div_bf16(float M) {
+  const float Mp = M > 0.0f ? M : 1.0f;
+  const float sc = Mp < 5.421010862427522e-20f ? 1.8446744073709552e+19f : 1.0f;   // 2^-64, 2^64
+  GroupDiv d;
+  d.b = Mp * sc;
+  const float y0 = rcp_approx(d.b);
+  d.y = __fmaf_rn(__fmaf_rn(-d.b, y0, 1.0f), y0, y0);
+  d.num = F8<FMT>::MAXV * sc;
+  d.m = M;
+  return d;
 }
 
 // bf16 input without expansion, when none of the warp's four groups holds an
@@ -180,7 +202,7 @@ __device__ __forceinline__ bool quant_bf16_plain(const RowItem<1>& it, int64_t r
   for (int off = 1; off < 8; off <<= 1) mxb = max(mxb, __shfl_xor_sync(0xFFFFFFFFu, mxb, off));
   if (__any_sync(0xFFFFFFFFu, mxb >= 0x7F80u)) return false;
   const float M = __uint_as_float(mxb << 16);
-  const GroupDiv d = codec_div<FMT>(M);
+  const GroupDiv d = codec_div_bf16<FMT>(M);
   uint32_t lo[2], hi[2];
   encode8_bf16_div<FMT>(u[0], d, lo);
   encode8_bf16_div<FMT>(u[1], d, hi);
@@ -195,6 +217,75 @@ __device__ __forceinline__ bool quant_bf16_plain(const RowItem<1>& it, int64_t r
     }
   }
   return true;
+}
+
+// One work item of the 16-element layout (4 groups of one row, 8 lanes of 16
+// elements each, loaded): group statistics, k and root scale, codes; stores
+// the codes and each group's scale and k.  Called by all 32 lanes of a warp.
+template <int FMT, int DT, bool EXPAND>
+__device__ __forceinline__ void quant_row_item(const RowItem<DT>& cur, int64_t rows, int64_t cols,
+                                               int l, int64_t nbc, uint8_t* __restrict__ q,
+                                               int64_t ldq, float* __restrict__ scale,
+                                               float* __restrict__ kk) {
+  if constexpr (DT == 1 && !EXPAND) {
+    if (quant_bf16_plain<FMT>(cur, rows, cols, l, nbc, q, ldq, scale, kk)) return;
+  }
+  float v[16];
+  unpack16<DT>(cur.raw, v);
+  float M, mu = 0.0f;
+  bool special;
+  if (EXPAND) {
+    uint32_t maxb = 0u, mink = 0xFFFFFFFFu;
+    stats_bits(v, maxb, mink);
+#pragma unroll
+    for (int off = 1; off < 8; off <<= 1) {
+      maxb = max(maxb, __shfl_xor_sync(0xFFFFFFFFu, maxb, off));
+      mink = min(mink, __shfl_xor_sync(0xFFFFFFFFu, mink, off));
+    }
+    special = maxb >= 0xFF000000u;   // an Inf or a NaN in the group
+    M = __uint_as_float(maxb >> 1);
+    mu = __uint_as_float((mink + 2u) >> 1);
+  } else {
+    float mx = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) mx = fmax_nan(mx, fabsf(v[i]));
+#pragma unroll
+    for (int off = 1; off < 8; off <<= 1) mx = fmax_nan(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+    special = !(mx <= 3.40282347e38f);   // NaN or Inf
+    M = mx;
+  }
+  if (__any_sync(0xFFFFFFFFu, special)) {
+    float Mn = max_abs_nonnan(v);
+#pragma unroll
+    for (int off = 1; off < 8; off <<= 1) Mn = fmaxf(Mn, __shfl_xor_sync(0xFFFFFFFFu, Mn, off));
+    if (special) M = Mn;
+  }
+  float k, sr, invM = 0.0f;
+  if (EXPAND) {
+    group_params<FMT>(M, mu, true, k, sr, invM);
+  } else {
+    // k = 1: the root scale is M / FMT_MAX, correctly rounded (1 for an all-zero group)
+    k = 1.0f;
+    sr = M > 0.0f ? div_fmax<FMT>(M) : 1.0f;
+  }
+  const bool use_div = !EXPAND || k == 1.0f;
+  GroupDiv d{};
+  if (use_div) d = codec_div<FMT>(M);
+  uint32_t cw[4];
+  if (!special)
+    encode_words<FMT, 16, true>(v, use_div, d, invM, k, cw);
+  else
+    encode_words<FMT, 16, false>(v, use_div, d, invM, k, cw);
+  if (cur.valid > 0 && COAT_INDEX_OK(cur.r < rows && cur.c + cur.valid <= cols))
+    store16(q + cur.r * ldq + cur.c, cw, cur.valid);
+  // lane 0 of a group holds its first column, so it exists exactly when the group does
+  if (l == 0 && cur.valid > 0) {
+    const int64_t g = cur.r * nbc + (cur.c >> 7);
+    if (COAT_INDEX_OK(g < rows * nbc)) {
+      scale[g] = sr;
+      kk[g] = k;
+    }
+  }
 }
 
 template <int FMT, int DT, bool EXPAND>
@@ -223,73 +314,132 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
     cc += 4 * kGroup;
     if (cc >= rowspan) { cc -= rowspan; ++cr; }
   };
-  auto body = [&](const RowItem<DT>& cur) {
-    if constexpr (DT == 1 && !EXPAND) {
-      if (quant_bf16_plain<FMT>(cur, rows, cols, l, nbc, q, ldq, scale, kk)) return;
-    }
-    float v[16];
-    unpack16<DT>(cur.raw, v);
-    float M, mu = 0.0f;
-    bool special;
-    if (EXPAND) {
-      uint32_t maxb = 0u, mink = 0xFFFFFFFFu;
-      stats_bits(v, maxb, mink);
-#pragma unroll
-      for (int off = 1; off < 8; off <<= 1) {
-        maxb = max(maxb, __shfl_xor_sync(0xFFFFFFFFu, maxb, off));
-        mink = min(mink, __shfl_xor_sync(0xFFFFFFFFu, mink, off));
-      }
-      special = maxb >= 0xFF000000u;   // an Inf or a NaN in the group
-      M = __uint_as_float(maxb >> 1);
-      mu = __uint_as_float((mink + 2u) >> 1);
-    } else {
-      float mx = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) mx = fmax_nan(mx, fabsf(v[i]));
-#pragma unroll
-      for (int off = 1; off < 8; off <<= 1) mx = fmax_nan(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
-      special = !(mx <= 3.40282347e38f);   // NaN or Inf
-      M = mx;
-    }
-    if (__any_sync(0xFFFFFFFFu, special)) {
-      float Mn = max_abs_nonnan(v);
-#pragma unroll
-      for (int off = 1; off < 8; off <<= 1) Mn = fmaxf(Mn, __shfl_xor_sync(0xFFFFFFFFu, Mn, off));
-      if (special) M = Mn;
-    }
-    float k, sr, invM = 0.0f;
-    if (EXPAND) {
-      group_params<FMT>(M, mu, true, k, sr, invM);
-    } else {
-      // k = 1: the root scale is M / FMT_MAX, correctly rounded (1 for an all-zero group)
-      k = 1.0f;
-      sr = M > 0.0f ? div_fmax<FMT>(M) : 1.0f;
-    }
-    const bool use_div = !EXPAND || k == 1.0f;
-    GroupDiv d{};
-    if (use_div) d = codec_div<FMT>(M);
-    uint32_t cw[4];
-    if (!special)
-      encode_words<FMT, 16, true>(v, use_div, d, invM, k, cw);
-    else
-      encode_words<FMT, 16, false>(v, use_div, d, invM, k, cw);
-    if (cur.valid > 0 && COAT_INDEX_OK(cur.r < rows && cur.c + cur.valid <= cols))
-      store16(q + cur.r * ldq + cur.c, cw, cur.valid);
-    // lane 0 of a group holds its first column, so it exists exactly when the group does
-    if (l == 0 && cur.valid > 0) {
-      const int64_t g = cur.r * nbc + (cur.c >> 7);
-      if (COAT_INDEX_OK(g < rows * nbc)) {
-        scale[g] = sr;
-        kk[g] = k;
-      }
-    }
-  };
   RowItem<DT> cur;
   load(cur);
   for (int64_t item = i0; item < i1; ++item) {
     RowItem<DT> nxt;
     if (item + 1 < i1) load(nxt);
-    body(cur);
+    quant_row_item<FMT, DT, EXPAND>(cur, rows, cols, l, nbc, q, ldq, scale, kk);
+    cur = nxt;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// bf16 input without expansion, the activation codec's common case: 4 lanes
+// per group and 32 contiguous elements per lane (8 groups, 1024 columns, per
+// warp and work item), so that each lane's share of the per-group work (the
+// maximum's shuffles, the divisor, the root scale) and of the per-item
+// addressing covers twice as many elements as in the 16-element layout.  A
+// work item whose groups hold an Inf or a NaN is redone by the general code
+// (quant_row_item) as the two 512-column items of the 16-element layout,
+// read again from global memory.
+// ---------------------------------------------------------------------------
+struct Row32Item {
+  uint4 u[4];     // 32 bf16 values, as loaded
+  int64_t r, c;   // row and the lane's first column
+  int valid;      // elements of the lane's 32 that exist
+};
+
+template <int FMT>
+__global__ void __launch_bounds__(256) quant_row32_bf16_kernel(const void* __restrict__ x,
+                                                               int64_t rows, int64_t cols,
+                                                               int64_t ldx,
+                                                               uint8_t* __restrict__ q,
+                                                               int64_t ldq,
+                                                               float* __restrict__ scale,
+                                                               float* __restrict__ kk) {
+  const int lane = threadIdx.x & 31, sub = lane >> 2, l4 = lane & 3;
+  const int64_t nbc = (cols + kGroup - 1) / kGroup;   // groups per row
+  const int64_t no = (nbc + 7) / 8;                    // 8-group items per row
+  const int64_t nitems = rows * no;
+  const int64_t wid = (blockIdx.x * int64_t(blockDim.x) + threadIdx.x) >> 5;
+  const int64_t nw = (int64_t(gridDim.x) * blockDim.x) >> 5;
+  const int64_t i0 = wid * nitems / nw, i1 = (wid + 1) * nitems / nw;
+  if (i0 >= i1) return;
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  const int64_t rowspan = no * 8 * kGroup;
+  int64_t cr = i0 / no;                                  // the next item to load
+  int64_t cc = (i0 - cr * no) * 8 * kGroup + sub * kGroup + 32 * l4;
+  auto load = [&](Row32Item& it) {
+    it.r = cr;
+    it.c = cc;
+    it.valid = COAT_INDEX_OK(cr < rows) ? clamp_valid(cols - cc, 32) : 0;
+    const uint16_t* p = xb + cr * ldx + cc;
+    if (it.valid >= 32) {
+#pragma unroll
+      for (int h = 0; h < 4; ++h) it.u[h] = __ldg(reinterpret_cast<const uint4*>(p) + h);
+    } else {
+      uint32_t t[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) t[i] = i < it.valid ? uint32_t(p[i]) : 0u;
+#pragma unroll
+      for (int h = 0; h < 4; ++h)
+        it.u[h] = make_uint4(t[8 * h] | (t[8 * h + 1] << 16), t[8 * h + 2] | (t[8 * h + 3] << 16),
+                             t[8 * h + 4] | (t[8 * h + 5] << 16), t[8 * h + 6] | (t[8 * h + 7] << 16));
+    }
+    cc += 8 * kGroup;
+    if (cc >= rowspan) { cc -= rowspan; ++cr; }
+  };
+  Row32Item cur;
+  load(cur);
+  for (int64_t item = i0; item < i1; ++item) {
+    Row32Item nxt;
+    if (item + 1 < i1) load(nxt);
+
+    // group maximum over the sign-cleared words (16-bit halves order like the
+    // magnitudes; an Inf or a NaN pattern is above every finite one)
+    uint32_t mx2 = 0u;
+#pragma unroll
+    for (int h = 0; h < 4; ++h)
+      mx2 = __vmaxu2(mx2, __vmaxu2(__vmaxu2(cur.u[h].x & 0x7FFF7FFFu, cur.u[h].y & 0x7FFF7FFFu),
+                                   __vmaxu2(cur.u[h].z & 0x7FFF7FFFu, cur.u[h].w & 0x7FFF7FFFu)));
+    uint32_t mxb = max(mx2 & 0xFFFFu, mx2 >> 16);
+    mxb = max(mxb, __shfl_xor_sync(0xFFFFFFFFu, mxb, 1));
+    mxb = max(mxb, __shfl_xor_sync(0xFFFFFFFFu, mxb, 2));
+    if (!__any_sync(0xFFFFFFFFu, mxb >= 0x7F80u)) {
+      const float M = __uint_as_float(mxb << 16);
+      const GroupDiv d = codec_div_bf16<FMT>(M);
+      uint32_t cw[8];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        uint32_t two[2];
+        encode8_bf16_div<FMT>(cur.u[h], d, two);
+        cw[2 * h] = two[0];
+        cw[2 * h + 1] = two[1];
+      }
+      if (cur.valid > 0 && COAT_INDEX_OK(cur.r < rows && cur.c + cur.valid <= cols)) {
+        uint8_t* qp = q + cur.r * ldq + cur.c;
+        if (cur.valid >= 32) {
+          reinterpret_cast<uint4*>(qp)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+          reinterpret_cast<uint4*>(qp)[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < cur.valid) qp[i] = static_cast<uint8_t>(cw[i >> 2] >> (8 * (i & 3)));
+        }
+      }
+      // lane 0 of a group holds its first column, so it exists exactly when the group does
+      if (l4 == 0 && cur.valid > 0) {
+        const int64_t g = cur.r * nbc + (cur.c >> 7);
+        if (COAT_INDEX_OK(g < rows * nbc)) {
+          scale[g] = M > 0.0f ? div_fmax<FMT>(M) : 1.0f;
+          kk[g] = 1.0f;
+        }
+      }
+    } else {
+      // the two 512-column halves of the item in the 16-element layout
+      const int slot = lane >> 3, l = lane & 7;
+      const int64_t c0 = cur.c - sub * kGroup - 32 * l4;   // the item's first column
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        RowItem<1> it;
+        it.r = cur.r;
+        it.c = c0 + h * 4 * kGroup + slot * kGroup + 16 * l;
+        it.valid = COAT_INDEX_OK(cur.r < rows) ? clamp_valid(cols - it.c, 16) : 0;
+        load16<1>(xb + cur.r * ldx, it.c, it.valid, it.raw);
+        quant_row_item<FMT, 1, false>(it, rows, cols, l, nbc, q, ldq, scale, kk);
+      }
+    }
     cur = nxt;
   }
 }
@@ -472,7 +622,7 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
     }
     const bool use_div = !EXPAND || k == 1.0f;
     GroupDiv d{};
-    if (use_div) d = codec_div<FMT>(M);
+    if (use_div) d = DT == 1 && !special ? codec_div_bf16<FMT>(M) : codec_div<FMT>(M);
     const int64_t c = bc * 128 + 8 * (lane & 15);
     const int cv = clamp_valid(cols - c, 8);
 #pragma unroll
@@ -789,7 +939,12 @@ template <int FMT, int DT>
 static cudaError_t quant_dispatch(const void* x, int64_t rows, int64_t cols, int64_t ldx, int gr,
                                   int expand, uint8_t* q, int64_t ldq, float* scale, float* k,
                                   unsigned* err, int dev, cudaStream_t s) {
-  if (gr == 1) {
+  if (gr == 1 && DT == 1 && !expand) {
+    const int64_t octs = rows * (((cols + 127) / 128 + 7) / 8);
+    auto kern = quant_row32_bf16_kernel<FMT>;
+    const unsigned g = grid_for(octs, 8, dev, resident_ctas(reinterpret_cast<const void*>(kern)));
+    kern<<<g, 256, 0, s>>>(x, rows, cols, ldx, q, ldq, scale, k);
+  } else if (gr == 1) {
     const int64_t quads = rows * (((cols + 127) / 128 + 3) / 4);
     auto kern = expand ? quant_row_kernel<FMT, DT, true> : quant_row_kernel<FMT, DT, false>;
     const unsigned g =
