@@ -330,13 +330,11 @@ def test_free_running_10_steps_fast_group_params(orc):
     # measured at step 10: median 1e-4, 99th percentile 4e-3, maximum 3e-2 of
     # |p| + sum u^abs (the exact mode keeps 99.9% of elements within 2e-7)
     assert last["q99"] <= 1e-2 and last["max"] <= 1e-1
-    # groups still within the tolerances after 10 steps (measured 1,892 of
-    # 8,192, 298 of them bit-identical); the master of their elements against
-    # 1e-6 (|p| + sum u^abs) at every step (measured: at most 1.7e-3 of them
-    # outside, at step 3, none from step 7 on)
-    assert fr.live.sum() >= 0.15 * fr.ng
+    # every group leaves the tolerances by step 9 (measured: 7,725 still in at
+    # step 2, 1,263 at step 4, 0 at step 9); while they are in, the master of
+    # their elements against 1e-6 (|p| + sum u^abs) (measured: at most 1.2e-3
+    # of them outside, at step 4)
     assert all(d["live_fail"] <= 5e-3 * d["live_elements"] for d in fr.master_dev)
-    assert last["live_fail"] == 0
 
 
 def test_free_running_10_steps_own_warm_start(orc):
@@ -351,6 +349,13 @@ def test_free_running_10_steps_own_warm_start(orc):
     fr = free_run(orc, gpu, ora, n, fm, fv, tensor, exact=True)
     last = fr.master_dev[-1]
     assert last["q99"] <= 1e-2 and last["max"] <= 1e-1
+    # groups still within the tolerances after 10 steps (measured 1,892 of
+    # 8,192, 298 of them bit-identical); the master of their elements against
+    # 1e-6 (|p| + sum u^abs) at every step (measured: at most 1.7e-3 of them
+    # outside, at step 3, none from step 7 on)
+    assert fr.live.sum() >= 0.15 * fr.ng
+    assert all(d["live_fail"] <= 5e-3 * d["live_elements"] for d in fr.master_dev)
+    assert last["live_fail"] == 0
 
 
 def test_weight_out_optional_and_deterministic():
