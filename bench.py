@@ -511,8 +511,9 @@ def run_ours(args, cfg, ws, rank, local):
 def run_extras(args, coat, H, local):
     """Figures of the other workloads in the same run (one GPU), so that they are
     recorded next to the headline: the ragged 10,000-tensor list against one flat
-    tensor of the same size (multi-tensor overhead), the Llama-2-13B list, and
-    the mixed-granularity codec workload.  Each list: device events around
+    tensor of the same size (multi-tensor overhead), that flat tensor with exact
+    group parameters, the Llama-2-13B list, and the mixed-granularity codec
+    workload.  Each list: device events around
     `steps` launches after 3 warm-up launches, inputs far larger than L2."""
     import torch
     from synth.params import CONFIGS
@@ -542,6 +543,10 @@ def run_extras(args, coat, H, local):
     flat_cfg = dict(CONFIGS["ragged"])
     fps, fplan = make_workload([("flat", n_r)], flat_cfg, 0, coat)
     fms = time_plan(fplan, steps, 3, H, coat)
+    # the same flat tensor with exact group parameters (k and the root scales
+    # recomputed in double from the codes)
+    with coat.exact_group_params(True):
+        ems = time_plan(fplan, steps, 3, H, coat)
     fplan.destroy()
     del fps
     torch.cuda.empty_cache()
@@ -549,6 +554,13 @@ def run_extras(args, coat, H, local):
     r["flat_value"] = round(n_r / (fms * 1e-3) / 1e9, 3)
     r["ratio_to_flat"] = round(r["value"] / r["flat_value"], 4)
     out["ragged"] = r
+    egbs = algorithmic_bytes([n_r], with_weight=True) / (ems * 1e-3) / 1e9
+    out["exact_group_params"] = {
+        "value": round(n_r / (ems * 1e-3) / 1e9, 3), "unit": UNIT, "ms_per_step": round(ems, 4),
+        "achieved_GBs": round(egbs, 1), "frac": round(egbs / peak, 4),
+        "ratio_to_default": round(fms / ems, 4),
+        "workload": "one flat tensor of %d params (E4M3 m + E5M2 v), exact group parameters "
+                    "(coat_set_exact_group_params(1))" % n_r}
     b, _ = one_list("llama2-13b", llama2_13b())
     b["workload"] = CONFIGS["llama2-13b"]["workload"]
     out["llama2_13b"] = b
