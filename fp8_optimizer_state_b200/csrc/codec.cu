@@ -162,6 +162,35 @@ __device__ __forceinline__ void encode8_bf16_div(const uint4& u, const GroupDiv&
   }
 }
 
+// Codes of 8 bf16 values (the words of u) of an expanded group without an Inf
+// or a NaN: the same codes as encode_words<FMT, 8, true> with expansion, with
+// y = 2^(k log2(|x| invM) + log2 FMT_MAX) evaluated by the same operations on
+// element pairs.
+template <int FMT>
+__device__ __forceinline__ void encode8_bf16_expand(const uint4& u, float invM, float k,
+                                                    uint32_t (&cw)[2]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  const float2 invM2 = make_float2(invM, invM), k2 = make_float2(k, k);
+  const float2 L2 = make_float2(F8<FMT>::LOG2MAX_HI, F8<FMT>::LOG2MAX_HI);
+  uint32_t mag[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t aw = w[j] & 0x7FFF7FFFu;
+    const float2 a = mul2(make_float2(__uint_as_float(aw * 65536u), bf16hi(aw)), invM2);
+    const float2 t = fma2(k2, make_float2(lg2_approx(a.x), lg2_approx(a.y)), L2);
+    const uint2 c = enc_mag_bounded2<FMT, FMT>(ex2_approx(t.x), ex2_approx(t.y));
+    mag[2 * j] = c.x;
+    mag[2 * j + 1] = c.y;
+  }
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const uint32_t mags =
+        mag[4 * t] + 256u * (mag[4 * t + 1] + 256u * (mag[4 * t + 2] + 256u * mag[4 * t + 3]));
+    const uint32_t top = __byte_perm(w[2 * t], w[2 * t + 1], 0x7531u);
+    cw[t] = mags + (top & (mags + 0x7F7F7F7Fu) & 0x80808080u);
+  }
+}
+
 // The division constants of a group whose maximum M is a bf16 value (0 for an
 // all-zero group): as codec_div, with RN(1/b) from one Newton step on
 // rcp.approx.  For any seed within an ulp of 1/b the step's result is
@@ -325,14 +354,17 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
 }
 
 // ---------------------------------------------------------------------------
-// bf16 input without expansion, the activation codec's common case: 4 lanes
-// per group and 32 contiguous elements per lane (8 groups, 1024 columns, per
-// warp and work item), so that each lane's share of the per-group work (the
-// maximum's shuffles, the divisor, the root scale) and of the per-item
-// addressing covers twice as many elements as in the 16-element layout.  A
-// work item whose groups hold an Inf or a NaN is redone by the general code
-// (quant_row_item) as the two 512-column items of the 16-element layout,
-// read again from global memory.
+// bf16 input, the activation codec's case: 4 lanes per group and 32
+// contiguous elements per lane (8 groups, 1024 columns, per warp and work
+// item), so that each lane's share of the per-group work (the extremes'
+// shuffles, k, the divisor, the root scale) and of the per-item addressing
+// covers twice as many elements as in the 16-element layout.  The extremes
+// come from the sign-cleared words, two elements per instruction: their 16-bit
+// halves order like the magnitudes (an Inf or a NaN pattern is above every
+// finite one), and subtracting one from each half first makes zeros the
+// largest for the minimum.  A work item whose groups hold an Inf or a NaN is
+// redone by the general code (quant_row_item) as the two 512-column items of
+// the 16-element layout, read again from global memory.
 // ---------------------------------------------------------------------------
 struct Row32Item {
   uint4 u[4];     // 32 bf16 values, as loaded
@@ -340,7 +372,7 @@ struct Row32Item {
   int valid;      // elements of the lane's 32 that exist
 };
 
-template <int FMT>
+template <int FMT, bool EXPAND>
 __global__ void __launch_bounds__(256) quant_row32_bf16_kernel(const void* __restrict__ x,
                                                                int64_t rows, int64_t cols,
                                                                int64_t ldx,
@@ -396,16 +428,45 @@ __global__ void __launch_bounds__(256) quant_row32_bf16_kernel(const void* __res
     uint32_t mxb = max(mx2 & 0xFFFFu, mx2 >> 16);
     mxb = max(mxb, __shfl_xor_sync(0xFFFFFFFFu, mxb, 1));
     mxb = max(mxb, __shfl_xor_sync(0xFFFFFFFFu, mxb, 2));
+    uint32_t mnb = 0xFFFFu;   // (min nonzero magnitude bits) - 1; 0xFFFF: all zero
+    if (EXPAND) {
+      uint32_t mn2 = 0xFFFFFFFFu;
+#pragma unroll
+      for (int h = 0; h < 4; ++h)
+        mn2 = __vminu2(mn2, __vminu2(__vminu2(__vsub2(cur.u[h].x & 0x7FFF7FFFu, 0x00010001u),
+                                              __vsub2(cur.u[h].y & 0x7FFF7FFFu, 0x00010001u)),
+                                     __vminu2(__vsub2(cur.u[h].z & 0x7FFF7FFFu, 0x00010001u),
+                                              __vsub2(cur.u[h].w & 0x7FFF7FFFu, 0x00010001u))));
+      mnb = min(mn2 & 0xFFFFu, mn2 >> 16);
+      mnb = min(mnb, __shfl_xor_sync(0xFFFFFFFFu, mnb, 1));
+      mnb = min(mnb, __shfl_xor_sync(0xFFFFFFFFu, mnb, 2));
+    }
     if (!__any_sync(0xFFFFFFFFu, mxb >= 0x7F80u)) {
       const float M = __uint_as_float(mxb << 16);
-      const GroupDiv d = codec_div_bf16<FMT>(M);
+      float k = 1.0f, sr, invM = 0.0f;
+      if (EXPAND) {
+        group_params<FMT>(M, __uint_as_float(((mnb + 1u) & 0xFFFFu) << 16), true, k, sr, invM);
+      } else {
+        sr = M > 0.0f ? div_fmax<FMT>(M) : 1.0f;
+      }
       uint32_t cw[8];
+      if (!EXPAND || k == 1.0f) {
+        const GroupDiv d = codec_div_bf16<FMT>(M);
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        uint32_t two[2];
-        encode8_bf16_div<FMT>(cur.u[h], d, two);
-        cw[2 * h] = two[0];
-        cw[2 * h + 1] = two[1];
+        for (int h = 0; h < 4; ++h) {
+          uint32_t two[2];
+          encode8_bf16_div<FMT>(cur.u[h], d, two);
+          cw[2 * h] = two[0];
+          cw[2 * h + 1] = two[1];
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          uint32_t two[2];
+          encode8_bf16_expand<FMT>(cur.u[h], invM, k, two);
+          cw[2 * h] = two[0];
+          cw[2 * h + 1] = two[1];
+        }
       }
       if (cur.valid > 0 && COAT_INDEX_OK(cur.r < rows && cur.c + cur.valid <= cols)) {
         uint8_t* qp = q + cur.r * ldq + cur.c;
@@ -422,8 +483,8 @@ __global__ void __launch_bounds__(256) quant_row32_bf16_kernel(const void* __res
       if (l4 == 0 && cur.valid > 0) {
         const int64_t g = cur.r * nbc + (cur.c >> 7);
         if (COAT_INDEX_OK(g < rows * nbc)) {
-          scale[g] = M > 0.0f ? div_fmax<FMT>(M) : 1.0f;
-          kk[g] = 1.0f;
+          scale[g] = sr;
+          kk[g] = k;
         }
       }
     } else {
@@ -437,7 +498,7 @@ __global__ void __launch_bounds__(256) quant_row32_bf16_kernel(const void* __res
         it.c = c0 + h * 4 * kGroup + slot * kGroup + 16 * l;
         it.valid = COAT_INDEX_OK(cur.r < rows) ? clamp_valid(cols - it.c, 16) : 0;
         load16<1>(xb + cur.r * ldx, it.c, it.valid, it.raw);
-        quant_row_item<FMT, 1, false>(it, rows, cols, l, nbc, q, ldq, scale, kk);
+        quant_row_item<FMT, 1, EXPAND>(it, rows, cols, l, nbc, q, ldq, scale, kk);
       }
     }
     cur = nxt;
@@ -939,9 +1000,9 @@ template <int FMT, int DT>
 static cudaError_t quant_dispatch(const void* x, int64_t rows, int64_t cols, int64_t ldx, int gr,
                                   int expand, uint8_t* q, int64_t ldq, float* scale, float* k,
                                   unsigned* err, int dev, cudaStream_t s) {
-  if (gr == 1 && DT == 1 && !expand) {
+  if (gr == 1 && DT == 1) {
     const int64_t octs = rows * (((cols + 127) / 128 + 7) / 8);
-    auto kern = quant_row32_bf16_kernel<FMT>;
+    auto kern = expand ? quant_row32_bf16_kernel<FMT, true> : quant_row32_bf16_kernel<FMT, false>;
     const unsigned g = grid_for(octs, 8, dev, resident_ctas(reinterpret_cast<const void*>(kern)));
     kern<<<g, 256, 0, s>>>(x, rows, cols, ldx, q, ldq, scale, k);
   } else if (gr == 1) {
