@@ -653,45 +653,55 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_bwd_kernel(
   for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
     In nxt[CPT];
     if (r + gridDim.x < rows) load(r + gridDim.x, nxt);
-    // pass 1: the row sums; the decoded values are not kept across the barrier
-    float sums[2] = {0.0f, 0.0f};   // sum x^2, sum g x
+    // pass 1: the row sums, element pairs in two interleaved partial sums each;
+    // the decoded values are not kept across the barrier
+    float sums[2];   // sum x^2, sum g x
+    {
+      float2 sxx = make_float2(0.0f, 0.0f), sgx = make_float2(0.0f, 0.0f);
 #pragma unroll
-    for (int j = 0; j < CPT; ++j) {
-      const bool plain = __all_sync(0xFFFFFFFFu, cur[j].k == 1.0f);
-      float f[16], dv[16];
-      decode16_raw<FMT>(cur[j].q, cur[j].k, plain, tab, f);
-      bf16x16(cur[j].d0, cur[j].d1, dv);
+      for (int j = 0; j < CPT; ++j) {
+        const bool plain = __all_sync(0xFFFFFFFFu, cur[j].k == 1.0f);
+        float f[16], dv[16];
+        decode16_raw<FMT>(cur[j].q, cur[j].k, plain, tab, f);
+        bf16x16(cur[j].d0, cur[j].d1, dv);
+        const float2 s2 = make_float2(cur[j].s, cur[j].s);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float xv = f[i] * cur[j].s;
-        sums[0] = __fmaf_rn(xv, xv, sums[0]);
-        sums[1] = __fmaf_rn(dv[i] * wv[j][i], xv, sums[1]);
+        for (int i = 0; i < 16; i += 2) {
+          const float2 xv = mul2(make_float2(f[i], f[i + 1]), s2);
+          const float2 g = mul2(make_float2(dv[i], dv[i + 1]), make_float2(wv[j][i], wv[j][i + 1]));
+          sxx = fma2(xv, xv, sxx);
+          sgx = fma2(g, xv, sgx);
+        }
       }
+      sums[0] = sxx.x + sxx.y;
+      sums[1] = sgx.x + sgx.y;
     }
     cta_sum_all<2, kNormThreads>(sums, red);
-    const float rstd = 1.0f / sqrtf(__fmaf_rn(sums[0], inv_d, eps));
+    const float rstd = rsqrt_approx(__fmaf_rn(sums[0], inv_d, eps));
     // rstd^2 mean(g xh) = rstd^3 sum(g x) / d
     const float cx = rstd * rstd * rstd * sums[1] * inv_d;
-    // pass 2: dx and the dw sums, decoding again
+    const float2 rstd2 = make_float2(rstd, rstd), ncx2 = make_float2(-cx, -cx);
+    // pass 2: dx and the dw sums, decoding again, element pairs
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
       const bool plain = __all_sync(0xFFFFFFFFu, cur[j].k == 1.0f);
       float f[16], dv[16];
       decode16_raw<FMT>(cur[j].q, cur[j].k, plain, tab, f);
       bf16x16(cur[j].d0, cur[j].d1, dv);
+      const float2 s2 = make_float2(cur[j].s, cur[j].s);
       uint32_t o[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        float a[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int i = 2 * e + h;
-          const float xv = f[i] * cur[j].s;
-          const float g = dv[i] * wv[j][i];
-          a[h] = __fmaf_rn(rstd, g, -cx * xv);
-          acc[j][i] = __fmaf_rn(dv[i], xv * rstd, acc[j][i]);
-        }
-        o[e] = pack_bf16x2(a[0], a[1]);
+        const int i = 2 * e;
+        const float2 dv2 = make_float2(dv[i], dv[i + 1]);
+        const float2 xv = mul2(make_float2(f[i], f[i + 1]), s2);
+        const float2 g = mul2(dv2, make_float2(wv[j][i], wv[j][i + 1]));
+        // dx = rstd g - cx x; dw += dy x rstd
+        const float2 a = fma2(rstd2, g, mul2(ncx2, xv));
+        const float2 ac = fma2(dv2, mul2(xv, rstd2), make_float2(acc[j][i], acc[j][i + 1]));
+        acc[j][i] = ac.x;
+        acc[j][i + 1] = ac.y;
+        o[e] = pack_bf16x2(a.x, a.y);
       }
       const int64_t c = (threadIdx.x + int64_t(j) * kNormThreads) * 16;
       if (ok[j] && COAT_INDEX_OK(c + 16 <= d)) {
