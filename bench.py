@@ -512,8 +512,8 @@ def run_extras(args, coat, H, local):
     """Figures of the other workloads in the same run (one GPU), so that they are
     recorded next to the headline: the ragged 10,000-tensor list against one flat
     tensor of the same size (multi-tensor overhead), that flat tensor with exact
-    group parameters, the Llama-2-13B list, and the mixed-granularity codec
-    workload.  Each list: device events around
+    group parameters, the Llama-2-13B list, the tiny one-tensor case (L2-resident)
+    and the mixed-granularity codec workload.  Each list: device events around
     `steps` launches after 3 warm-up launches, inputs far larger than L2."""
     import torch
     from synth.params import CONFIGS
@@ -564,6 +564,12 @@ def run_extras(args, coat, H, local):
     b, _ = one_list("llama2-13b", llama2_13b())
     b["workload"] = CONFIGS["llama2-13b"]["workload"]
     out["llama2_13b"] = b
+    from synth.params import tiny
+    t, _ = one_list("tiny", tiny())
+    t["workload"] = CONFIGS["tiny"]["workload"]
+    t["l2"] = ("17 MB of inputs: L2-resident across launches, so not a roofline point "
+               "(the fraction can exceed the HBM peak)")
+    out["tiny"] = t
     cargs = argparse.Namespace(steps=steps, warmup=3, no_e2e=True, no_cpu_baseline=True,
                                e2e_steps=1)
     c = run_codec(cargs, 1, 0, local)
