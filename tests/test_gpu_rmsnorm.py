@@ -53,6 +53,8 @@ def exact_y(orc, xa, w, fmt):
     (8, 8192, E5M2, False, True),          # the largest d
     (5, 128, E4M3, False, False),
     (3, 640, E5M2_FULL, False, True),
+    (33, 2048, E5M2, True, False),         # expanded input, one warp per row
+    (7, 640, E4M3, True, False),
 ])
 def test_forward_vs_oracle(orc, rows, d, fmt, expand_in, expand_out):
     xa, w = make_inputs(orc, rows, d, fmt, expand_in, 1)
@@ -64,6 +66,32 @@ def test_forward_vs_oracle(orc, rows, d, fmt, expand_in, expand_out):
     print("flips", flips)
     if not expand_in and not expand_out:
         assert flips == 0
+
+
+@pytest.mark.parametrize("d,fmt,code", [(256, E4M3, 0x7F), (4096, E5M2, 0x7C), (4096, E4M3, 0xFF),
+                                         (5120, E5M2, 0x7E)])
+def test_forward_special_values(orc, d, fmt, code):
+    """A NaN or an Inf code in a row makes the row's mean of squares NaN or
+    Inf, and every value of that row NaN or 0: its groups are all zero codes
+    with k = 1 and scale 1 (the codec's rule for groups without a finite
+    nonzero maximum), as the oracle gives; the other rows are unaffected."""
+    rows = 6
+    xa, w = make_inputs(orc, rows, d, fmt, False, 3)
+    xa = tuple(a.copy() for a in xa)
+    xa[0][1, 5] = code
+    xa[0][4, d - 1] = code
+    out = empty_act(rows, d)
+    coat.coat_rmsnorm_fp8_forward(to_dev(xa), w_dev(w), EPS, fmt, False, out)
+    qd, sd, kd = host(out)
+    qo, so, ko = orc.rmsnorm_fp8_forward(xa, w, EPS, fmt, False)
+    for r in (1, 4):
+        assert not qd[r].any() and not qo[r].any()
+        assert np.all(sd[r] == 1.0) and np.all(kd[r] == 1.0)
+        assert np.array_equal(sd[r], so[r]) and np.array_equal(kd[r], ko[r])
+    keep = np.array([0, 2, 3, 5])
+    flips = check_act("rmsnorm special", fmt, (qd[keep], sd[keep], kd[keep]),
+                      (qo[keep], so[keep], ko[keep]), exact_y(orc, tuple(a[keep] for a in xa), w, fmt))
+    assert flips == 0
 
 
 def backward_case(orc, rows, d, fmt, expand_in, seed=2):
