@@ -302,8 +302,7 @@ coat_status coat_grad_clip_finalize(coat_grad_clip *d_clip, float max_norm, cuda
  *     104 bytes each (106,496 bytes); every GPU that loads the library keeps
  *     it until the process exits.
  *   - The first call on a device looks up the array's device address (with
- *     that device current) and configures the kernel; make that first call
- *     before any stream capture.
+ *     that device current) and configures the kernel.
  *   - Each call enqueues, on `stream`, small copy kernels that write the table
  *     into the array (the descriptors travel as their kernel parameters, 32
  *     per launch, so no host buffer is read after the call returns and no
