@@ -179,7 +179,7 @@ def oracle_slice_inputs(per_tensor, fmt_m, fmt_v, use_device):
     import synth
     from synth.params import llama2_7b
     shapes = llama2_7b()[:SLICE_TENSORS]
-    counts = [min(n, per_tensor) // 128 * 128 for _, n in shapes]
+    counts = [(min(n, per_tensor) if per_tensor > 0 else n) // 128 * 128 for _, n in shapes]
 
     def one(i):
         c = counts[i]
@@ -235,22 +235,27 @@ def time_oracle(cfg, per_tensor, steps, threads, use_device, inputs=None):
 
 
 def cpu_baseline(cfg, per_tensor, use_device):
-    """The oracle on every host core over the slice sample (median of three
-    steps), next to one core on its first 2^21 elements, and the whole 7B
-    list's step time extrapolated from the all-cores rate."""
+    """The oracle on every host core over the slice (whole tensors when
+    per_tensor is 0: one step; else the first per_tensor elements of each:
+    median of three steps), next to one core on its first 2^21 elements, and
+    the whole 7B list's step time extrapolated from the all-cores rate."""
     cores = host_cores()
     inputs, counts = oracle_slice_inputs(per_tensor, cfg["fmt_m"], cfg["fmt_v"], use_device)
     total = int(sum(counts))
-    t_all = statistics.median(time_oracle(cfg, per_tensor, 3, cores, use_device, inputs))
+    steps = 1 if per_tensor <= 0 else 3
+    t_all = statistics.median(time_oracle(cfg, per_tensor, steps, cores, use_device, inputs))
     one = min(total, 1 << 21)
     t_one = time_oracle(cfg, per_tensor, 1, 1, use_device, [a[:one] if a.size == total else
                                                            a[:one // 128] for a in inputs])[0]
     rate = total / t_all
+    what = ("the whole %d tensors of the %s" % (len(counts), SLICE_NAME) if per_tensor <= 0 else
+            "first %d elements of each of the %d tensors of the %s" % (per_tensor, len(counts),
+                                                                       SLICE_NAME))
     return {"value": round(rate / 1e9, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": "first %d elements of each of the %d tensors of the %s (%d elements, "
-                      "stored states from the seeded generator), one step on %d host threads, "
-                      "median of 3 steps (%.2f s each)" % (per_tensor, len(counts), SLICE_NAME,
-                                                             total, cores, t_all),
+            "sample": "%s (%d elements, stored states from the seeded generator), on %d host "
+                      "threads, %s (%.2f s each)" % (what, total, cores,
+                                                    "one step" if steps == 1 else
+                                                    "median of 3 steps", t_all),
             "one_core": {"value": round(one / t_one / 1e9, 6), "unit": UNIT, "cores": 1,
                          "sample": "first %d elements of the same sample, one step (%.2f s)"
                                    % (one, t_one)},
@@ -1319,8 +1324,9 @@ def main(argv=None):
                          "the ranks instead of one replica per rank")
     ap.add_argument("--no-extras", dest="extras", action="store_false",
                     help="skip the ragged, 13B and codec figures of the default run")
-    ap.add_argument("--cpu-sample", type=int, default=1 << 20,
-                    help="oracle baseline: elements per tensor of the 7B slice")
+    ap.add_argument("--cpu-sample", type=int, default=0,
+                    help="oracle baseline: elements per tensor of the 7B slice (0: whole "
+                         "tensors, the slice's 333,455,360 parameters)")
     ap.add_argument("--ref-sample", type=int, default=1 << 19,
                     help="reference arm: elements per tensor of the 7B slice per step")
     args = ap.parse_args(argv)
