@@ -253,9 +253,9 @@ def cpu_baseline(cfg, per_tensor, use_device):
                                                                        SLICE_NAME))
     return {"value": round(rate / 1e9, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": "%s (%d elements, stored states from the seeded generator), on %d host "
-                      "threads, %s (%.2f s each)" % (what, total, cores,
-                                                    "one step" if steps == 1 else
-                                                    "median of 3 steps", t_all),
+                      "threads, %s (%.2f s)" % (what, total, cores,
+                                               "one step" if steps == 1 else
+                                               "median of 3 steps, each", t_all),
             "one_core": {"value": round(one / t_one / 1e9, 6), "unit": UNIT, "cores": 1,
                          "sample": "first %d elements of the same sample, one step (%.2f s)"
                                    % (one, t_one)},
