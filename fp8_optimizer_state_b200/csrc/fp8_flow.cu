@@ -288,8 +288,8 @@ __device__ __forceinline__ void quantize_scaled16(const float (&p)[16], float C,
 struct FwdItem {
   uint4 gw, uw;
   float gs, gk, us, uk;
-  int64_t r;
-  int32_t c;
+  int64_t oq;   // the lane's first output code: r ldq_out + c
+  int64_t om;   // its group's output scale and k: r lds_out + c / 128
   bool valid;   // the lane's 16 columns exist
 };
 
@@ -302,7 +302,7 @@ struct FwdItem {
 // row-major order, a contiguous range per warp (columns advanced by 512 with
 // a row carry); the next item is loaded before the current one is computed.
 template <int FMT, bool EXPAND>
-__global__ void __launch_bounds__(256) swiglu_fwd_kernel(const ActArgs gate, const ActArgs up,
+__global__ void __launch_bounds__(256, 3) swiglu_fwd_kernel(const ActArgs gate, const ActArgs up,
                                                          int64_t rows, int64_t cols,
                                                          const ActArgs out) {
   __shared__ float tab[256];
@@ -320,24 +320,37 @@ __global__ void __launch_bounds__(256) swiglu_fwd_kernel(const ActArgs gate, con
   int64_t cr = i0 / nq;                     // row and lane column of the next item to load
   int32_t cc = static_cast<int32_t>((i0 - cr * nq) * 4 * kGroup) + lc;
   const int32_t rowspan = static_cast<int32_t>(nq * 4 * kGroup);
+  // row offsets of the next item's row in each array, advanced by one row
+  // stride at a row carry (no per-item 64-bit multiplies)
+  int64_t rg = cr * gate.ldq, ru = cr * up.ldq, rmg = cr * gate.lds, rmu = cr * up.lds;
+  int64_t ro = cr * out.ldq, rmo = cr * out.lds;
   auto load = [&](FwdItem& it) {
-    it.r = cr;
-    it.c = cc;
+    it.oq = ro + cc;
     it.valid = cc < cols && COAT_INDEX_OK(cr < rows && cc + 16 <= cols);
     const int32_t g = cc >> 7;
+    it.om = rmo + g;
     if (it.valid) {
-      it.gw = __ldg(reinterpret_cast<const uint4*>(gate.q + cr * gate.ldq + cc));
-      it.uw = __ldg(reinterpret_cast<const uint4*>(up.q + cr * up.ldq + cc));
-      it.gs = __ldg(gate.scale + cr * gate.lds + g);
-      it.gk = __ldg(gate.k + cr * gate.lds + g);
-      it.us = __ldg(up.scale + cr * up.lds + g);
-      it.uk = __ldg(up.k + cr * up.lds + g);
+      it.gw = __ldg(reinterpret_cast<const uint4*>(gate.q + rg + cc));
+      it.uw = __ldg(reinterpret_cast<const uint4*>(up.q + ru + cc));
+      it.gs = __ldg(gate.scale + rmg + g);
+      it.gk = __ldg(gate.k + rmg + g);
+      it.us = __ldg(up.scale + rmu + g);
+      it.uk = __ldg(up.k + rmu + g);
     } else {
       it.gw = it.uw = make_uint4(0u, 0u, 0u, 0u);
       it.gs = it.gk = it.us = it.uk = 1.0f;
     }
     cc += 4 * kGroup;
-    if (cc >= rowspan) { cc -= rowspan; ++cr; }
+    if (cc >= rowspan) {
+      cc -= rowspan;
+      ++cr;
+      rg += gate.ldq;
+      ru += up.ldq;
+      rmg += gate.lds;
+      rmu += up.lds;
+      ro += out.ldq;
+      rmo += out.lds;
+    }
   };
   auto body = [&](const FwdItem& cur) {
     const bool plain = __all_sync(0xFFFFFFFFu, cur.gk == 1.0f && cur.uk == 1.0f);
@@ -364,10 +377,10 @@ __global__ void __launch_bounds__(256) swiglu_fwd_kernel(const ActArgs gate, con
     float k, sr;
     quantize_scaled16<FMT, EXPAND, false>(h, S, cw, k, sr);
     if (cur.valid) {
-      *reinterpret_cast<uint4*>(out.q + cur.r * out.ldq + cur.c) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      *reinterpret_cast<uint4*>(out.q + cur.oq) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
       if (l == 0) {
-        out.scale[cur.r * out.lds + (cur.c >> 7)] = sr;
-        out.k[cur.r * out.lds + (cur.c >> 7)] = k;
+        out.scale[cur.om] = sr;
+        out.k[cur.om] = k;
       }
     }
   };
