@@ -1000,17 +1000,20 @@ template <int FMT, int DT>
 static cudaError_t quant_dispatch(const void* x, int64_t rows, int64_t cols, int64_t ldx, int gr,
                                   int expand, uint8_t* q, int64_t ldq, float* scale, float* k,
                                   unsigned* err, int dev, cudaStream_t s) {
-  if (gr == 1 && DT == 1) {
-    const int64_t octs = rows * (((cols + 127) / 128 + 7) / 8);
-    auto kern = expand ? quant_row32_bf16_kernel<FMT, true> : quant_row32_bf16_kernel<FMT, false>;
-    const unsigned g = grid_for(octs, 8, dev, resident_ctas(reinterpret_cast<const void*>(kern)));
-    kern<<<g, 256, 0, s>>>(x, rows, cols, ldx, q, ldq, scale, k);
-  } else if (gr == 1) {
-    const int64_t quads = rows * (((cols + 127) / 128 + 3) / 4);
-    auto kern = expand ? quant_row_kernel<FMT, DT, true> : quant_row_kernel<FMT, DT, false>;
-    const unsigned g =
-        grid_for(quads, 8, dev, resident_ctas(reinterpret_cast<const void*>(kern)));
-    kern<<<g, 256, 0, s>>>(x, rows, cols, ldx, q, ldq, scale, k);
+  if (gr == 1) {
+    // bf16: 32 elements per lane; FP32: 16 (the general layout)
+    if constexpr (DT == 1) {
+      const int64_t octs = rows * (((cols + 127) / 128 + 7) / 8);
+      auto kern = expand ? quant_row32_bf16_kernel<FMT, true> : quant_row32_bf16_kernel<FMT, false>;
+      const unsigned g = grid_for(octs, 8, dev, resident_ctas(reinterpret_cast<const void*>(kern)));
+      kern<<<g, 256, 0, s>>>(x, rows, cols, ldx, q, ldq, scale, k);
+    } else {
+      const int64_t quads = rows * (((cols + 127) / 128 + 3) / 4);
+      auto kern = expand ? quant_row_kernel<FMT, DT, true> : quant_row_kernel<FMT, DT, false>;
+      const unsigned g =
+          grid_for(quads, 8, dev, resident_ctas(reinterpret_cast<const void*>(kern)));
+      kern<<<g, 256, 0, s>>>(x, rows, cols, ldx, q, ldq, scale, k);
+    }
   } else {
     const int64_t blocks = ((rows + 127) / 128) * ((cols + 127) / 128);
     auto kern = expand ? quant_block_kernel<FMT, DT, true> : quant_block_kernel<FMT, DT, false>;
