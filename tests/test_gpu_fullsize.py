@@ -52,9 +52,11 @@ def _grab(ps, i, gi):
                 mk=f(ps.mk, g, g + 1), vs=f(ps.vs, g, g + 1), vk=f(ps.vk, g, g + 1), cnt=cnt)
 
 
-def _check_samples(orc, samples, post, step, fm, fv, gscale=1.0):
+def _check_samples(orc, samples, post, step, fm, fv, gscale=1.0, same_out=None):
     """The oracle on each sampled group, its inputs regenerated on the host from
-    the same counters; returns the number of code flips."""
+    the same counters; returns the number of code flips.  same_out (a list):
+    receives, per sampled group and moment, whether k and the root scale equal
+    the oracle's bit for bit."""
     flips = 0
     for (i, gi), a in zip(samples, post):
         cnt, e0 = a["cnt"], gi * 128
@@ -73,6 +75,9 @@ def _check_samples(orc, samples, post, step, fm, fv, gscale=1.0):
                                  mq, sm, km)[0]
         flips += check_state_all("v %d/%d" % (i, gi), cnt, fv, a["vq"], a["vs"], a["vk"],
                                  vq, sv, kv)[0]
+        if same_out is not None:
+            same_out.append(bool(a["mk"][0] == km[0] and a["ms"][0] == sm[0]))
+            same_out.append(bool(a["vk"][0] == kv[0] and a["vs"][0] == sv[0]))
     n_el = 2 * 128 * len(samples)
     print("sampled groups %d, code flips %d of %d codes" % (len(samples), flips, n_el))
     assert flips <= max(2, 1e-4 * n_el)
@@ -105,6 +110,34 @@ def test_llama2_7b_full_size_sampled(orc):
             assert bool(((k >= 1) & (k <= 16)).all())
         for s_ in (ps.ms, ps.vs):
             assert bool((torch.isfinite(s_) & (s_ > 0)).all())
+        plan.destroy()
+    finally:
+        del ps
+        torch.cuda.empty_cache()
+
+
+def test_llama2_7b_full_size_sampled_exact_group_params(orc):
+    """The full-size launch with exact group parameters: besides the tolerances,
+    k and the root scale of the sampled groups are the oracle's bits (the
+    correctly rounded values of the definition), except where an FP32 near-tie
+    hides the true extreme."""
+    cfg = CONFIGS["llama2-7b"]
+    fm, fv = cfg["fmt_m"], cfg["fmt_v"]
+    step = 3
+    ps = _build(fm, fv, step)
+    try:
+        plan = coat.coat_multi_plan_create([_desc(ps, i) for i in range(len(ps))], fm, fv)
+        samples = _samples(ps, 51)
+        torch.cuda.synchronize()
+        with coat.exact_group_params(True):
+            coat.coat_adamw_step_multi(plan, step=step,
+                                       **{k: H[k] for k in ("lr", "beta1", "beta2", "eps", "wd")})
+        coat.coat_check_device_error()
+        post = [_grab(ps, i, gi) for i, gi in samples]
+        same = []
+        _check_samples(orc, samples, post, step, fm, fv, same_out=same)
+        print("k and scale bit-identical: %d of %d sampled group moments" % (sum(same), len(same)))
+        assert sum(same) >= 0.99 * len(same)
         plan.destroy()
     finally:
         del ps
