@@ -1327,7 +1327,7 @@ def main(argv=None):
     ap.add_argument("--cpu-sample", type=int, default=0,
                     help="oracle baseline: elements per tensor of the 7B slice (0: whole "
                          "tensors, the slice's 333,455,360 parameters)")
-    ap.add_argument("--ref-sample", type=int, default=1 << 19,
+    ap.add_argument("--ref-sample", type=int, default=1 << 21,
                     help="reference arm: elements per tensor of the 7B slice per step")
     args = ap.parse_args(argv)
     if args.warmup < 3:
