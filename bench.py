@@ -356,6 +356,8 @@ def run_ours(args, cfg, ws, rank, local):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     coat.lib()
+    if args.exact_group_params:
+        coat.coat_set_exact_group_params(True)
 
     ps, plan = make_workload(cfg["shapes"](), cfg, rank, coat)
 
@@ -431,7 +433,8 @@ def run_ours(args, cfg, ws, rank, local):
     alg = algorithmic_bytes(ps.sizes, with_weight=True)
     achieved = alg / (kernel_ms * 1e-3) / 1e9
     traffic = None
-    if TRAFFIC["sources_sha256"] == kernel_hash() and TRAFFIC["bytes_per_param"]:
+    if (TRAFFIC["sources_sha256"] == kernel_hash() and TRAFFIC["bytes_per_param"]
+            and not args.exact_group_params):   # the capture is of the fast-mode kernel
         traffic = TRAFFIC["bytes_per_param"] * n_params
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -495,6 +498,7 @@ def run_ours(args, cfg, ws, rank, local):
                        "fmt_v": FMT_NAMES[cfg["fmt_v"]],
                        "hyper": H, "l2": "no flush: %.1f GB of inputs per step >> 126 MB L2"
                                          % (alg / 1e9),
+                       "group_params": "exact" if args.exact_group_params else "fast",
                        "parallelism": "replicas%d (independent parameter groups, no collective)" % ws
                        if ws > 1 else "single GPU"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
@@ -1322,6 +1326,8 @@ def main(argv=None):
     ap.add_argument("--zero1", action="store_true",
                     help="time the ZeRO-1 sharded step (reduce-scatter, step, all-gather) over "
                          "the ranks instead of one replica per rank")
+    ap.add_argument("--exact-group-params", action="store_true",
+                    help="run the step with exact group parameters (coat_set_exact_group_params)")
     ap.add_argument("--no-extras", dest="extras", action="store_false",
                     help="skip the ragged, 13B and codec figures of the default run")
     ap.add_argument("--cpu-sample", type=int, default=0,
