@@ -191,27 +191,9 @@ __device__ __forceinline__ void encode8_bf16_expand(const uint4& u, float invM, 
   }
 }
 
-// The division constants of a group whose maximum M is a bf16 value (0 for an
-// all-zero group): as codec_div, with RN(1/b) from one Newton step on
-// rcp.approx.  For any seed within an ulp of 1/b the step's result is
-// RN(1/b) whenever b's significand has at most 8 bits (every bf16 value,
-// scaled or not), which the tests check exactly for all 128 of them.
-template <int FMT>
-__device__ __forceinline__ GroupDiv codec_div_bf16(float M) {
-  const float Mp = M > 0.0f ? M : 1.0f;
-  const float sc = Mp < 5.421010862427522e-20f ? 1.8446744073709552e+19f : 1.0f;   // 2^-64, 2^64
-  GroupDiv d;
-  d.b = Mp * sc;
-  const float y0 = rcp_approx(d.b);
-  d.y = __fmaf_rn(__fmaf_rn(-d.b, y0, 1.0f), y0, y0);
-  d.num = F8<FMT>::MAXV * sc;
-  d.m = M;
-  return d;
-}
-
 // bf16 input without expansion, when none of the warp's four groups holds an
-// Inf or a NaN (returns false otherwise, and the caller takes the general
-// path): the general path's codes and scales.  The group maximum is an
+// Inf, a NaN or a maximum above 2^100 (returns false otherwise, and the caller
+// takes the general path): the general path's codes and scales.  The group maximum is an
 // unsigned 16-bit max over the words with their sign bits cleared, whose
 // halves order like the magnitudes they encode (an Inf or a NaN pattern is
 // above every finite one).
@@ -229,9 +211,10 @@ __device__ __forceinline__ bool quant_bf16_plain(const RowItem<1>& it, int64_t r
   uint32_t mxb = max(mx2 & 0xFFFFu, mx2 >> 16);
 #pragma unroll
   for (int off = 1; off < 8; off <<= 1) mxb = max(mxb, __shfl_xor_sync(0xFFFFFFFFu, mxb, off));
-  if (__any_sync(0xFFFFFFFFu, mxb >= 0x7F80u)) return false;
+  // an Inf, a NaN or a maximum above 2^100 (0x7180): the general path
+  if (__any_sync(0xFFFFFFFFu, mxb > 0x7180u)) return false;
   const float M = __uint_as_float(mxb << 16);
-  const GroupDiv d = codec_div_bf16<FMT>(M);
+  const GroupDiv d = codec_div_short<FMT>(M);
   uint32_t lo[2], hi[2];
   encode8_bf16_div<FMT>(u[0], d, lo);
   encode8_bf16_div<FMT>(u[1], d, hi);
@@ -271,7 +254,9 @@ __device__ __forceinline__ void quant_row_item(const RowItem<DT>& cur, int64_t r
       maxb = max(maxb, __shfl_xor_sync(0xFFFFFFFFu, maxb, off));
       mink = min(mink, __shfl_xor_sync(0xFFFFFFFFu, mink, off));
     }
-    special = maxb >= 0xFF000000u;   // an Inf or a NaN in the group
+    // an Inf or a NaN in the group, or a finite maximum outside [2^-100, 2^100]
+    // (twice the bits)
+    special = maxb > 0xE3000000u || (maxb != 0u && maxb < 0x1B000000u);
     M = __uint_as_float(maxb >> 1);
     mu = __uint_as_float((mink + 2u) >> 1);
   } else {
@@ -280,22 +265,32 @@ __device__ __forceinline__ void quant_row_item(const RowItem<DT>& cur, int64_t r
     for (int i = 0; i < 16; ++i) mx = fmax_nan(mx, fabsf(v[i]));
 #pragma unroll
     for (int off = 1; off < 8; off <<= 1) mx = fmax_nan(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
-    special = !(mx <= 3.40282347e38f);   // NaN or Inf
+    // NaN, Inf, or a maximum above 2^100 (small maxima need nothing here)
+    special = !(mx <= 0x1p100f);
     M = mx;
   }
+  float M0 = M, sig = 1.0f;
   if (__any_sync(0xFFFFFFFFu, special)) {
     float Mn = max_abs_nonnan(v);
 #pragma unroll
     for (int off = 1; off < 8; off <<= 1) Mn = fmaxf(Mn, __shfl_xor_sync(0xFFFFFFFFu, Mn, off));
     if (special) M = Mn;
+    M0 = M;
+    // a maximum outside [2^-100, 2^100]: the group's values scaled into range
+    sig = range_sigma(M);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] *= sig;
+    M *= sig;
+    mu *= sig;
   }
   float k, sr, invM = 0.0f;
   if (EXPAND) {
     group_params<FMT>(M, mu, true, k, sr, invM);
+    if (sig != 1.0f) sr *= sig < 1.0f ? 0x1p100f : 0x1p-100f;
   } else {
     // k = 1: the root scale is M / FMT_MAX, correctly rounded (1 for an all-zero group)
     k = 1.0f;
-    sr = M > 0.0f ? div_fmax<FMT>(M) : 1.0f;
+    sr = M0 > 0.0f ? div_fmax<FMT>(M0) : 1.0f;
   }
   const bool use_div = !EXPAND || k == 1.0f;
   GroupDiv d{};
@@ -362,9 +357,10 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const void* __restrict__
 // come from the sign-cleared words, two elements per instruction: their 16-bit
 // halves order like the magnitudes (an Inf or a NaN pattern is above every
 // finite one), and subtracting one from each half first makes zeros the
-// largest for the minimum.  A work item whose groups hold an Inf or a NaN is
-// redone by the general code (quant_row_item) as the two 512-column items of
-// the 16-element layout, read again from global memory.
+// largest for the minimum.  A work item whose groups hold an Inf or a NaN, or
+// a maximum outside the range range_sigma() describes, is redone by the
+// general code (quant_row_item) as the two 512-column items of the 16-element
+// layout, read again from global memory.
 // ---------------------------------------------------------------------------
 struct Row32Item {
   uint4 u[4];     // 32 bf16 values, as loaded
@@ -441,7 +437,10 @@ __global__ void __launch_bounds__(256) quant_row32_bf16_kernel(const void* __res
       mnb = min(mnb, __shfl_xor_sync(0xFFFFFFFFu, mnb, 1));
       mnb = min(mnb, __shfl_xor_sync(0xFFFFFFFFu, mnb, 2));
     }
-    if (!__any_sync(0xFFFFFFFFu, mxb >= 0x7F80u)) {
+    // an Inf, a NaN or a maximum above 2^100 (bits 0x7180), or with
+    // expansion a nonzero maximum below 2^-100 (0x0D80): the general path
+    const bool slow = mxb > 0x7180u || (EXPAND && mxb != 0u && mxb < 0x0D80u);
+    if (!__any_sync(0xFFFFFFFFu, slow)) {
       const float M = __uint_as_float(mxb << 16);
       float k = 1.0f, sr, invM = 0.0f;
       if (EXPAND) {
@@ -451,7 +450,7 @@ __global__ void __launch_bounds__(256) quant_row32_bf16_kernel(const void* __res
       }
       uint32_t cw[8];
       if (!EXPAND || k == 1.0f) {
-        const GroupDiv d = codec_div_bf16<FMT>(M);
+        const GroupDiv d = codec_div_short<FMT>(M);
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
           uint32_t two[2];
@@ -651,9 +650,15 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
       maxb = max(maxb, sM[par][w]);
       mink = min(mink, sK[par][w]);
     }
-    // an Inf or a NaN in the block (CTA-uniform)
-    const bool special = EXPAND ? maxb >= 0xFF000000u : maxb >= 0x7F800000u;
+    // special (CTA-uniform): an Inf or a NaN in the block, or a finite maximum
+    // outside [2^-100, 2^100] (bits 0x71800000 and 0x0D800000, doubled with
+    // expansion; without expansion small maxima need nothing), whose values
+    // are scaled into range (range_sigma)
+    const bool special = EXPAND ? maxb > 0xE3000000u || (maxb != 0u && maxb < 0x1B000000u)
+                                : maxb > 0x71800000u;
     float M = __uint_as_float(EXPAND ? maxb >> 1 : maxb);
+    float mu = EXPAND ? __uint_as_float((mink + 2u) >> 1) : 0.0f;
+    float M0 = M, sig = 1.0f;
     if (special) {
       // max |x| ignoring NaN, through the other half of the partials buffer
       float Mn = 0.f;
@@ -671,19 +676,24 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
 #pragma unroll
       for (int w = 1; w < 8; ++w) M = fmaxf(M, __uint_as_float(sM[par ^ 1][w]));
       __syncthreads();   // the partials buffer is free again before the next block writes it
+      M0 = M;
+      sig = range_sigma(M);
+      M *= sig;
+      mu *= sig;
     }
     par ^= 1;
     float k, sr, invM = 0.0f;
     if (EXPAND) {
-      group_params<FMT>(M, __uint_as_float((mink + 2u) >> 1), true, k, sr, invM);
+      group_params<FMT>(M, mu, true, k, sr, invM);
+      if (special && sig != 1.0f) sr *= sig < 1.0f ? 0x1p100f : 0x1p-100f;
     } else {
       // k = 1: the root scale is M / FMT_MAX, correctly rounded (1 for an all-zero block)
       k = 1.0f;
-      sr = M > 0.0f ? div_fmax<FMT>(M) : 1.0f;
+      sr = M0 > 0.0f ? div_fmax<FMT>(M0) : 1.0f;
     }
     const bool use_div = !EXPAND || k == 1.0f;
     GroupDiv d{};
-    if (use_div) d = DT == 1 && !special ? codec_div_bf16<FMT>(M) : codec_div<FMT>(M);
+    if (use_div) d = DT == 1 && !special ? codec_div_short<FMT>(M) : codec_div<FMT>(M);
     const int64_t c = bc * 128 + 8 * (lane & 15);
     const int cv = clamp_valid(cols - c, 8);
 #pragma unroll
@@ -700,6 +710,10 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
       if (!packed) {
         float v[8];
         block_row<DT>(cur, i, v);
+        if (special) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] *= sig;
+        }
         if (!special)
           encode_words<FMT, 8, true>(v, use_div, d, invM, k, cw);
         else

@@ -150,8 +150,9 @@ __device__ __forceinline__ void decode16_raw(const uint4& w, float k, bool plain
 // the real-number result; at most FMT_MAX (1 + 2^-21), inside the bounded
 // encoder's range) with root scale M / FMT_MAX correctly rounded; expanded
 // groups use the codec's expansion.  The slow path (the codec's NaN rules and
-// IEEE division) takes groups with a NaN or an Inf, a maximum below 2^-64
-// (1/M would leave FP32), or force_slow (the same for the 8 lanes of a group).
+// IEEE division) takes groups with a NaN or an Inf, a maximum below 2^-64 or
+// above 2^100 (their values are scaled into range there, see range_sigma), or
+// force_slow (the same for the 8 lanes of a group).
 template <int FMT, bool EXPAND>
 __device__ __forceinline__ void quantize_lane16(const float (&h)[16], bool force_slow,
                                                 uint32_t (&cw)[4], float& k, float& sr) {
@@ -167,7 +168,7 @@ __device__ __forceinline__ void quantize_lane16(const float (&h)[16], bool force
     mx = fmax_nan(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
     if (EXPAND) mink = min(mink, __shfl_xor_sync(0xFFFFFFFFu, mink, off));
   }
-  const bool special = !(mx <= 3.40282347e38f) || force_slow ||
+  const bool special = !(mx <= 0x1p100f) || force_slow ||
                        (mx > 0.0f && mx < 5.421010862427522e-20f);
   if (!__any_sync(0xFFFFFFFFu, special)) {
     const float M = mx;
@@ -204,17 +205,23 @@ __device__ __forceinline__ void quantize_lane16(const float (&h)[16], bool force
     for (int i = 0; i < 16; ++i) mk2 = min(mk2, __float_as_uint(h[i]) * 2u - 2u);
 #pragma unroll
     for (int off = 1; off < 8; off <<= 1) mk2 = min(mk2, __shfl_xor_sync(0xFFFFFFFFu, mk2, off));
-    const float M = special ? Mn : mx;
+    const float M0 = special ? Mn : mx;
+    // a maximum outside [2^-100, 2^100]: the values scaled into range
+    const float sig = range_sigma(M0), M = M0 * sig;
+    float hs[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) hs[i] = h[i] * sig;
     float invM;
-    group_params<FMT>(M, __uint_as_float((mk2 + 2u) >> 1), EXPAND, k, sr, invM);
-    if (!EXPAND) sr = M > 0.0f ? __fdiv_rn(M, F8<FMT>::MAXV) : 1.0f;
+    group_params<FMT>(M, __uint_as_float((mk2 + 2u) >> 1) * sig, EXPAND, k, sr, invM);
+    if (sig != 1.0f) sr *= sig < 1.0f ? 0x1p100f : 0x1p-100f;
+    if (!EXPAND) sr = M0 > 0.0f ? __fdiv_rn(M0, F8<FMT>::MAXV) : 1.0f;
     const bool use_div = k == 1.0f;
     GroupDiv d{};
     if (use_div) d = codec_div<FMT>(M);
     if (special)
-      encode_words<FMT, 16, false>(h, use_div, d, invM, k, cw);
+      encode_words<FMT, 16, false>(hs, use_div, d, invM, k, cw);
     else
-      encode_words<FMT, 16, true>(h, use_div, d, invM, k, cw);
+      encode_words<FMT, 16, true>(hs, use_div, d, invM, k, cw);
   }
 }
 
@@ -225,11 +232,12 @@ __device__ __forceinline__ void quantize_lane16(const float (&h)[16], bool force
 // correctly rounded division (for exact p an exact tie of the real-number
 // result stays a tie and is broken to even, as the oracle does); otherwise
 // one multiply by FMT_MAX / max|p| (a few ulps; for p that are not exact
-// anyway).  With expansion, and for groups with a NaN/Inf, a maximum below
-// 2^-64 or an unusable C, the values y go through quantize_lane16.
+// anyway).  With expansion, and for groups with a NaN/Inf, a maximum |p|
+// below 2^-64 or above 2^100 or an unusable C, the values y go through
+// quantize_lane16.
 template <int FMT, bool EXPAND, bool EXACT>
 __device__ __forceinline__ void quantize_scaled16(const float (&p)[16], float C, uint32_t (&cw)[4],
-                                                  float& k, float& sr) {
+                                                  float& k, float& sr, bool short_sig = false) {
   if (EXPAND) {
     float y[16];
 #pragma unroll
@@ -243,7 +251,7 @@ __device__ __forceinline__ void quantize_scaled16(const float (&p)[16], float C,
 #pragma unroll
   for (int off = 1; off < 8; off <<= 1) mp = fmax_nan(mp, __shfl_xor_sync(0xFFFFFFFFu, mp, off));
   const float My = mp * C;
-  const bool special = !(mp <= 3.40282347e38f) || !(My <= 3.40282347e38f) || !(C > 0.0f) ||
+  const bool special = !(mp <= 0x1p100f) || !(My <= 3.40282347e38f) || !(C > 0.0f) ||
                        (mp > 0.0f && mp < 5.421010862427522e-20f);
   if (__any_sync(0xFFFFFFFFu, special)) {
     float y[16];
@@ -259,7 +267,11 @@ __device__ __forceinline__ void quantize_scaled16(const float (&p)[16], float C,
     // div_exact on the signed values, two at a time: every step rounds to
     // nearest, which is symmetric in the sign, so each result is
     // sign(p) RN(FMT_MAX |p| / max|p|)
-    const GroupDiv dv = codec_div<FMT>(mp);
+    GroupDiv dv;
+    if (short_sig)
+      dv = codec_div_short<FMT>(mp);   // exact for the short significands of k = 1 products
+    else
+      dv = codec_div<FMT>(mp);
     const float2 num2 = make_float2(dv.num, dv.num), y2 = make_float2(dv.y, dv.y);
     const float2 nb2 = make_float2(-dv.b, -dv.b);
 #pragma unroll
@@ -526,11 +538,14 @@ __global__ void __launch_bounds__(NT, CPT == 2 ? 16 / (NT / 32) : 1) rmsnorm_fwd
                                                                    const uint16_t* __restrict__ w,
                                                                    int64_t rows, int64_t d,
                                                                    float eps, const ActArgs out) {
+  constexpr int NW = NT / 32;
   __shared__ float tab[256];
-  __shared__ float red[1][NT / 32];
+  __shared__ float red[1][NW];
+  __shared__ double redd[NW];    // the row's warp partials in double, when its FP32 sum overflows
   fill_log2_table<FMT>(tab);
   __syncthreads();
   const float inv_d = 1.0f / static_cast<float>(d);
+  const int warp = threadIdx.x >> 5;
   float wv[CPT][16];
   bool ok[CPT];
 #pragma unroll
@@ -545,7 +560,7 @@ __global__ void __launch_bounds__(NT, CPT == 2 ? 16 / (NT / 32) : 1) rmsnorm_fwd
       for (int i = 0; i < 16; ++i) wv[j][i] = 0.0f;
     }
   }
-  // the next row's codes and metadata are loaded before this row's reduction
+  // the next row's codes and metadata are loaded before this row's work
   struct In { uint4 q; float s, k; };
   auto load = [&](int64_t r, In (&in)[CPT]) {
 #pragma unroll
@@ -561,17 +576,17 @@ __global__ void __launch_bounds__(NT, CPT == 2 ? 16 / (NT / 32) : 1) rmsnorm_fwd
     }
   };
   auto body = [&](int64_t r, const In (&cur)[CPT]) {
-    float pv[CPT][16], sv[CPT];
+    // p = f w (f the FP8 value, or |q|^(1/k) with its sign; x = f s): exact
+    // for k = 1 (an FP8 value times a bf16 value); the row's sum of x^2 as
+    // the sum over chunks of (sum of f^2) s^2
+    float pv[CPT][16], sfv[CPT];
+    bool plain[CPT];
     float ss[1] = {0.0f};
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
-      const uint4 q = cur[j].q;
-      const float s = cur[j].s, k = cur[j].k;
-      const bool plain = __all_sync(0xFFFFFFFFu, k == 1.0f);
+      plain[j] = __all_sync(0xFFFFFFFFu, cur[j].k == 1.0f);
       float f[16];
-      decode16_raw<FMT>(q, k, plain, tab, f);
-      // sum of f^2 (x = f s) in two interleaved partial sums; p = f w, exact for
-      // k = 1 (an FP8 value times a bf16 value); two elements per operation
+      decode16_raw<FMT>(cur[j].q, cur[j].k, plain[j], tab, f);
       float2 sf = make_float2(0.0f, 0.0f);
 #pragma unroll
       for (int i = 0; i < 16; i += 2) {
@@ -581,17 +596,43 @@ __global__ void __launch_bounds__(NT, CPT == 2 ? 16 / (NT / 32) : 1) rmsnorm_fwd
         pv[j][i] = p2.x;
         pv[j][i + 1] = p2.y;
       }
-      ss[0] = __fmaf_rn(sf.x + sf.y, s * s, ss[0]);
-      sv[j] = s;
+      sfv[j] = sf.x + sf.y;
+      ss[0] = __fmaf_rn(sfv[j], cur[j].s * cur[j].s, ss[0]);
     }
     cta_sum_all<1, NT>(ss, red);
-    // rstd only scales the root scales (the codes depend on p / max|p| alone)
-    const float rstd = rsqrt_approx(__fmaf_rn(ss[0], inv_d, eps));
+    float C[CPT];
+    if (ss[0] <= 3.40282347e38f) {
+      // rstd only scales the root scales (the codes depend on p / max|p| alone)
+      const float rstd = rsqrt_approx(__fmaf_rn(ss[0], inv_d, eps));
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) C[j] = cur[j].s * rstd;
+    } else {
+      // The FP32 sum is Inf or NaN (CTA-uniform).  Finite inputs whose x^2
+      // sum leaves FP32 are summed again in double, where no such sum
+      // overflows; the scale products s rstd are formed in double and rounded
+      // once.  A NaN or an Inf input keeps a non-finite sum.
+      double sd = 0.0;
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) {
+        const double sj = static_cast<double>(cur[j].s);
+        sd = fma(static_cast<double>(sfv[j]), sj * sj, sd);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sd += __shfl_xor_sync(0xFFFFFFFFu, sd, off);
+      if ((threadIdx.x & 31) == 0) redd[warp] = sd;
+      __syncthreads();
+      double td = 0.0;
+#pragma unroll
+      for (int v = 0; v < NW; ++v) td += redd[v];
+      const double rstd = 1.0 / sqrt(td / static_cast<double>(d) + static_cast<double>(eps));
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) C[j] = static_cast<float>(static_cast<double>(cur[j].s) * rstd);
+    }
 #pragma unroll
     for (int j = 0; j < CPT; ++j) {
       uint32_t cw[4];
       float k, sr;
-      quantize_scaled16<FMT, EXPAND, true>(pv[j], sv[j] * rstd, cw, k, sr);
+      quantize_scaled16<FMT, EXPAND, true>(pv[j], C[j], cw, k, sr, plain[j]);
       const int64_t c = (threadIdx.x + int64_t(j) * NT) * 16;
       if (ok[j] && COAT_INDEX_OK(c + 16 <= d)) {
         *reinterpret_cast<uint4*>(out.q + r * out.ldq + c) = make_uint4(cw[0], cw[1], cw[2], cw[3]);

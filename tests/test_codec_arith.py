@@ -5,7 +5,9 @@ restated in rational arithmetic on the CPU (no GPU, no library code).
   possibly scaled by 2^64) as one Newton step y1 = RN(y0 + y0 RN(1 - b y0))
   from the hardware's approximate reciprocal y0, which is within one ulp of
   1/b.  The step must give RN(1/b) for every such seed: checked for all 128
-  bf16 significands and both neighbours of 1/b.
+  bf16 significands and both neighbours of 1/b.  The RMSNorm forward does the
+  same for products of an FP8 value and a bf16 value: all 2048 significands
+  of at most 12 bits.
 * The root scale M / FMT_MAX is taken as q1 = RN(q0 + r y) with y = RN(1/FMT_MAX),
   q0 = RN(M y), r = RN(M - q0 FMT_MAX) (the division's correction step).  It
   must equal RN(M / FMT_MAX): checked for every bf16 significand and, for
@@ -67,6 +69,20 @@ def test_newton_reciprocal_is_correctly_rounded_for_bf16_significands(scale_exp)
         for seed in seeds_within_ulp(b):
             got = fma(fma(-b, seed, Fr(1)), seed, seed)
             if got != want:
+                bad.append((m, seed))
+    assert not bad
+
+
+def test_newton_reciprocal_is_correctly_rounded_for_12_bit_significands():
+    # the RMSNorm forward's group maximum max|f w| is a product of an FP8 value
+    # (at most 4 significant bits) and a bf16 weight (8 bits): at most 12 bits,
+    # every one of which is covered here
+    bad = []
+    for m in range(2048):
+        b = 1 + Fr(m, 2048)
+        want = rn32(1 / b)
+        for seed in seeds_within_ulp(b):
+            if fma(fma(-b, seed, Fr(1)), seed, seed) != want:
                 bad.append((m, seed))
     assert not bad
 

@@ -179,6 +179,56 @@ def test_group_quantize_special_values(orc, gr, fmt, expand):
     assert maxd <= 1 and diff.sum() <= max(1, FLIP_FRACTION * diff.size)
 
 
+# Exponents of the power of two each row (1x128) or each 128-row block
+# (128x128) is multiplied by: group maxima from 2^127.3 down to FP32
+# subnormals, across the points where FMT_MAX |x| overflows (2^112-2^119), the
+# approximate reciprocal flushes (2^126, 2^-126) and the 2^+-100 bounds of the
+# range the kernels scale groups into.
+EXTREME_EXPONENTS = [119, 116, 112, 105, 101, 100, 99, 0, -99, -100, -101, -110, -120, -126,
+                     -130, -135]
+
+
+@pytest.mark.parametrize("gr", [1, 128])
+@pytest.mark.parametrize("fmt", [E4M3, E5M2, E5M2_FULL])
+@pytest.mark.parametrize("expand", [False, True])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_group_quantize_extreme_magnitudes(orc, gr, fmt, expand, dtype):
+    """Groups of every magnitude FP32 holds follow the oracle (which divides in
+    double and never overflows): k, the root scale (within its tolerance or one
+    subnormal step, whichever is larger; bit-exact without expansion) and the
+    codes."""
+    ne = len(EXTREME_EXPONENTS)
+    cols = 512
+    rows = ne * gr
+    bits = synth.activations_bits(4, rows + cols, 0, rows * cols).reshape(rows, cols)
+    xv = synth.bf16_bits_to_f32(bits).astype(np.float64)
+    xv *= np.repeat(2.0 ** np.array(EXTREME_EXPONENTS, dtype=np.float64), gr)[:, None]
+    if dtype == "bf16":
+        xd = torch.from_numpy(xv.astype(np.float32)).to(torch.bfloat16).cuda()
+        xh = xd.float().cpu().numpy()
+    else:
+        xh = xv.astype(np.float32)
+        xd = torch.from_numpy(xh).cuda()
+    assert np.isfinite(xh).all()
+    nbr, nbc = rows // gr, cols // 128
+    q = torch.zeros((rows, cols), dtype=torch.uint8, device="cuda")
+    s = torch.zeros((nbr, nbc), dtype=torch.float32, device="cuda")
+    k = torch.zeros((nbr, nbc), dtype=torch.float32, device="cuda")
+    coat.coat_group_quantize(xd, gr, 128, expand, fmt, q, s, k)
+    oq, os_, ok_ = orc.group_quantize(xh.astype(np.float64), gr, 128, expand, fmt)
+    gq, gs, gk = q.cpu().numpy(), s.cpu().numpy(), k.cpu().numpy()
+    assert rel_err(gk, ok_).max() <= K_RTOL
+    # the scale tolerance, but never below one subnormal step (2^-149): a
+    # subnormal root scale keeps only the bits above it, on both sides
+    tol = np.maximum(scale_rtol(ok_, fmt) * np.abs(os_.astype(np.float64)), 2.0 ** -149)
+    assert np.all(np.abs(gs.astype(np.float64) - os_) <= tol)
+    if not expand:
+        assert np.array_equal(gs, os_)
+    diff, maxd = compare_codes(gq, oq)
+    assert maxd <= 1
+    assert diff.sum() <= max(1, FLIP_FRACTION * diff.size), int(diff.sum())
+
+
 @pytest.mark.parametrize("gr", [1, 128])
 @pytest.mark.parametrize("fmt", [E4M3, E5M2, E5M2_FULL])
 @pytest.mark.parametrize("rows,cols", [(256, 640), (100, 650)])

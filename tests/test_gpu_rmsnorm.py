@@ -94,6 +94,34 @@ def test_forward_special_values(orc, d, fmt, code):
     assert flips == 0
 
 
+@pytest.mark.parametrize("d,fmt,expand_out", [(4096, E4M3, False), (4096, E4M3, True),
+                                               (5120, E5M2, False)])
+def test_forward_extreme_scales(orc, d, fmt, expand_out):
+    """Input scales far from 1: rows whose sum of x^2 leaves FP32's range
+    (input scales 2^70 and 2^100 times the usual; the kernel sums such rows
+    again in double, where the oracle always sums), a row at 2^40 (still
+    inside FP32), a row of tiny scales, and a row whose groups mix 2^90 and 1.
+    k and scales within their tolerances, codes as in the plain case: without
+    expansion none differs."""
+    rows = 6
+    xa, w = make_inputs(orc, rows, d, fmt, False, 5)
+    q, s, k = (a.copy() for a in xa)
+    mult = np.ones(s.shape, np.float64)
+    mult[1] = 2.0 ** 40
+    mult[2] = 2.0 ** 70
+    mult[3] = 2.0 ** 100
+    mult[4] = 2.0 ** -60
+    mult[5, ::2] = 2.0 ** 90
+    xa = (q, (s.astype(np.float64) * mult).astype(np.float32), k)
+    assert np.isfinite(xa[1]).all()
+    out = empty_act(rows, d)
+    coat.coat_rmsnorm_fp8_forward(to_dev(xa), w_dev(w), EPS, fmt, expand_out, out)
+    want = orc.rmsnorm_fp8_forward(xa, w, EPS, fmt, expand_out)
+    flips = check_act("rmsnorm extreme scales", fmt, host(out), want, exact_y(orc, xa, w, fmt))
+    if not expand_out:
+        assert flips == 0
+
+
 def backward_case(orc, rows, d, fmt, expand_in, seed=2):
     xa, w = make_inputs(orc, rows, d, fmt, expand_in, seed)
     dy = synth.grad_bits(seed, 3, 1, 0, rows * d).reshape(rows, d)
