@@ -628,11 +628,7 @@ __global__ void __launch_bounds__(NT, CPT == 2 ? 16 / (NT / 32) : 1) rmsnorm_fwd
 #pragma unroll
       for (int j = 0; j < CPT; ++j) C[j] = static_cast<float>(static_cast<double>(cur[j].s) * rstd);
     }
-#pragma unroll
-    for (int j = 0; j < CPT; ++j) {
-      uint32_t cw[4];
-      float k, sr;
-      quantize_scaled16<FMT, EXPAND, true>(pv[j], C[j], cw, k, sr, plain[j]);
+    auto store = [&](int j, const uint32_t (&cw)[4], float sr, float k) {
       const int64_t c = (threadIdx.x + int64_t(j) * NT) * 16;
       if (ok[j] && COAT_INDEX_OK(c + 16 <= d)) {
         *reinterpret_cast<uint4*>(out.q + r * out.ldq + c) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
@@ -640,6 +636,73 @@ __global__ void __launch_bounds__(NT, CPT == 2 ? 16 / (NT / 32) : 1) rmsnorm_fwd
           out.scale[r * out.lds + (c >> 7)] = sr;
           out.k[r * out.lds + (c >> 7)] = k;
         }
+      }
+    };
+    // Without expansion, when no group of the warp's chunks needs the general
+    // path, the chunks are quantised in one block without branches, so that
+    // their dependency chains interleave: the group maxima and their shuffles,
+    // one vote over every range condition, the divisions by a Newton
+    // reciprocal (exact for the short significands of k = 1 products, within
+    // an ulp for expanded inputs, whose products are approximate anyway) and
+    // the root scales by the correction step without its range test.  Every
+    // other case takes quantize_scaled16 chunk by chunk.
+    bool fast = false;
+    float mp[CPT], My[CPT];
+    if constexpr (!EXPAND) {
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) {
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) m = fmax_nan(m, fabsf(pv[j][i]));
+        mp[j] = m;
+      }
+#pragma unroll
+      for (int off = 1; off < 8; off <<= 1)
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) mp[j] = fmax_nan(mp[j], __shfl_xor_sync(0xFFFFFFFFu, mp[j], off));
+      bool sp = false;
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) {
+        My[j] = mp[j] * C[j];
+        sp = sp || !(mp[j] <= 0x1p100f) || (mp[j] > 0.0f && mp[j] < 5.421010862427522e-20f) ||
+             !(My[j] <= 3.40282347e38f) || !(C[j] > 0.0f) ||
+             (My[j] > 0.0f && My[j] < 7.888609052210118e-31f);
+      }
+      fast = !__any_sync(0xFFFFFFFFu, sp);
+    }
+    if (fast) {
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) {
+        const GroupDiv dv = codec_div_short<FMT>(mp[j]);
+        const float2 num2 = make_float2(dv.num, dv.num), y2 = make_float2(dv.y, dv.y);
+        const float2 nb2 = make_float2(-dv.b, -dv.b);
+        float y[16];
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+          // sign(p) RN(FMT_MAX |p| / max|p|): every step rounds to nearest,
+          // which is symmetric in the sign
+          const float2 a = mul2(make_float2(pv[j][i], pv[j][i + 1]), num2);
+          const float2 q0 = mul2(a, y2);
+          const float2 q = fma2(fma2(q0, nb2, a), y2, q0);
+          y[i] = q.x;
+          y[i + 1] = q.y;
+        }
+        uint32_t cw[4];
+        encode_hw16<FMT>(y, cw);
+        // M / FMT_MAX correctly rounded (div_fmax's step; My is in its range)
+        const float q0 = My[j] * F8<FMT>::RCPMAX;
+        const float sr = My[j] > 0.0f
+                             ? __fmaf_rn(__fmaf_rn(-q0, F8<FMT>::MAXV, My[j]), F8<FMT>::RCPMAX, q0)
+                             : 1.0f;
+        store(j, cw, sr, 1.0f);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) {
+        uint32_t cw[4];
+        float k, sr;
+        quantize_scaled16<FMT, EXPAND, true>(pv[j], C[j], cw, k, sr, plain[j]);
+        store(j, cw, sr, k);
       }
     }
   };
