@@ -437,16 +437,18 @@ __global__ void __launch_bounds__(256) quant_row32_bf16_kernel(const void* __res
       mnb = min(mnb, __shfl_xor_sync(0xFFFFFFFFu, mnb, 1));
       mnb = min(mnb, __shfl_xor_sync(0xFFFFFFFFu, mnb, 2));
     }
-    // an Inf, a NaN or a maximum above 2^100 (bits 0x7180), or with
-    // expansion a nonzero maximum below 2^-100 (0x0D80): the general path
-    const bool slow = mxb > 0x7180u || (EXPAND && mxb != 0u && mxb < 0x0D80u);
+    // an Inf, a NaN, a maximum above 2^100 (bits 0x7180) or a nonzero one
+    // below 2^-100 (0x0D80): the general path (so that below, the root scale
+    // M / FMT_MAX takes div_fmax's correction step without its range test)
+    const bool slow = mxb > 0x7180u || (mxb != 0u && mxb < 0x0D80u);
     if (!__any_sync(0xFFFFFFFFu, slow)) {
       const float M = __uint_as_float(mxb << 16);
       float k = 1.0f, sr, invM = 0.0f;
       if (EXPAND) {
         group_params<FMT>(M, __uint_as_float(((mnb + 1u) & 0xFFFFu) << 16), true, k, sr, invM);
       } else {
-        sr = M > 0.0f ? div_fmax<FMT>(M) : 1.0f;
+        const float q0 = M * F8<FMT>::RCPMAX;
+        sr = M > 0.0f ? __fmaf_rn(__fmaf_rn(-q0, F8<FMT>::MAXV, M), F8<FMT>::RCPMAX, q0) : 1.0f;
       }
       uint32_t cw[8];
       if (!EXPAND || k == 1.0f) {
