@@ -168,7 +168,8 @@ coat_status coat_adamw_step(float *master, uint16_t *weight_bf16_out, const uint
  *   (except when an FP32 near-tie hides the true extreme).  Two runs that
  *   start from the same state then keep bit-identical k, scales and codes
  *   apart from rare code-rounding differences, so they stay in lockstep.  The
- *   step is about 25% slower (a serial double-precision phase per group).
+ *   step is 15-25% slower: the double-precision work of each group adds about
+ *   20% to the instructions per parameter.
  * Codes come from the same FP32 expansion and software encoder in both modes.
  * ------------------------------------------------------------------------- */
 int coat_set_exact_group_params(int on);
