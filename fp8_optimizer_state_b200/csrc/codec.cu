@@ -193,10 +193,10 @@ __device__ __forceinline__ void encode8_bf16_expand(const uint4& u, float invM, 
 
 // bf16 input without expansion, when none of the warp's four groups holds an
 // Inf, a NaN or a maximum above 2^100 (returns false otherwise, and the caller
-// takes the general path): the general path's codes and scales.  The group maximum is an
-// unsigned 16-bit max over the words with their sign bits cleared, whose
-// halves order like the magnitudes they encode (an Inf or a NaN pattern is
-// above every finite one).
+// takes the general path): the general path's codes and scales.  The group
+// maximum is an unsigned 16-bit max over the words with their sign bits
+// cleared, whose halves order like the magnitudes they encode (an Inf or a NaN
+// pattern is above every finite one).
 template <int FMT>
 __device__ __forceinline__ bool quant_bf16_plain(const RowItem<1>& it, int64_t rows, int64_t cols,
                                                  int l, int64_t nbc, uint8_t* __restrict__ q,
