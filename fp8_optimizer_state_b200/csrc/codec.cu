@@ -704,8 +704,12 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
       uint32_t cw[2];
       bool packed = false;
       if constexpr (DT == 1) {
-        if (!special && use_div) {
-          encode8_bf16_div<FMT>(cur.a[i], d, cw);
+        if (!special) {
+          // bf16 words on element pairs: the same codes as encode_words
+          if (use_div)
+            encode8_bf16_div<FMT>(cur.a[i], d, cw);
+          else
+            encode8_bf16_expand<FMT>(cur.a[i], invM, k, cw);
           packed = true;
         }
       }
