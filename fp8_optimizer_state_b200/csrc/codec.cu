@@ -698,33 +698,9 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
     if (use_div) d = DT == 1 && !special ? codec_div_short<FMT>(M) : codec_div<FMT>(M);
     const int64_t c = bc * 128 + 8 * (lane & 15);
     const int cv = clamp_valid(cols - c, 8);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    // the 8 codes of this lane's row i of the block
+    auto put = [&](int i, const uint32_t (&cw)[2]) {
       const int64_t r = br * 128 + warp * 16 + 2 * i + (lane >> 4);
-      uint32_t cw[2];
-      bool packed = false;
-      if constexpr (DT == 1) {
-        if (!special) {
-          // bf16 words on element pairs: the same codes as encode_words
-          if (use_div)
-            encode8_bf16_div<FMT>(cur.a[i], d, cw);
-          else
-            encode8_bf16_expand<FMT>(cur.a[i], invM, k, cw);
-          packed = true;
-        }
-      }
-      if (!packed) {
-        float v[8];
-        block_row<DT>(cur, i, v);
-        if (special) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) v[e] *= sig;
-        }
-        if (!special)
-          encode_words<FMT, 8, true>(v, use_div, d, invM, k, cw);
-        else
-          encode_words<FMT, 8, false>(v, use_div, d, invM, k, cw);
-      }
       const int valid = r < rows && COAT_INDEX_OK(cv == 0 || c + cv <= cols) ? cv : 0;
       uint8_t* qp = q + r * ldq + c;
       if (valid >= 8) {
@@ -733,6 +709,56 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const void* __restrict
 #pragma unroll
         for (int e = 0; e < 8; ++e)
           if (e < valid) qp[e] = static_cast<uint8_t>(cw[e >> 2] >> (8 * (e & 3)));
+      }
+    };
+    if constexpr (DT == 1) {
+      // bf16: one unrolled loop per fast path (the CTA-uniform branch is taken
+      // once per block), so that the loop's code stays small
+      if (!special && use_div) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          uint32_t cw[2];
+          encode8_bf16_div<FMT>(cur.a[i], d, cw);
+          put(i, cw);
+        }
+      } else if (!special) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          uint32_t cw[2];
+          encode8_bf16_expand<FMT>(cur.a[i], invM, k, cw);
+          put(i, cw);
+        }
+      } else {
+        // a block with special values or an out-of-range maximum: the general
+        // encoder, one row at a time, each row read again from global memory
+        // (a rolled loop cannot index the registers that hold the block)
+#pragma unroll 1
+        for (int i = 0; i < 8; ++i) {
+          const int64_t r = br * 128 + warp * 16 + 2 * i + (lane >> 4);
+          const int valid = r < rows ? cv : 0;
+          const uint16_t* xp = static_cast<const uint16_t*>(x) + r * ldx + c;
+          float v[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] = e < valid ? bf16lo(uint32_t(xp[e])) * sig : 0.0f;
+          uint32_t cw[2];
+          encode_words<FMT, 8, false>(v, use_div, d, invM, k, cw);
+          put(i, cw);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float v[8];
+        block_row<DT>(cur, i, v);
+        uint32_t cw[2];
+        if (special) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] *= sig;
+          encode_words<FMT, 8, false>(v, use_div, d, invM, k, cw);
+        } else {
+          encode_words<FMT, 8, true>(v, use_div, d, invM, k, cw);
+        }
+        put(i, cw);
       }
     }
     if (threadIdx.x == 0 && COAT_INDEX_OK(b < nb)) {
